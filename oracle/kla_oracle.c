@@ -1,0 +1,129 @@
+/*
+ * Oracle for Kaczmarz Linear Attention (KLA) -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, fp64, token-by-token evaluation of the recurrence.  Only the
+ * test-suite, the smoke check and the CPU-baseline leg of the benchmark may
+ * load this library; the product path never does.  It shares no code, header
+ * or constant with the CUDA library.
+ *
+ * What it computes (h = S^T stored [dk][dv] per head):
+ *
+ *   beta_t = eta_t / (||k_t||_2^2 + eps)
+ *       Kaczmarz Linear Attention (tomesphere summary of arXiv 2605.08587),
+ *       Abstract: the key-norm-normalised step size.
+ *   S_t = alpha_t * S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *   alpha_t = exp(g_t)
+ *       Gated DeltaNet recurrence ("Deep Dive into KDA", section 2.2), of which
+ *       KLA is the one-scalar modification (same Abstract).  The page prints
+ *       the erase factor on the left of S; with S mapping keys to values
+ *       (S is dv x dk) only the right-hand placement type-checks, and for a
+ *       scalar gate the two placements of alpha agree.
+ *   o_t = S_t q_t   (the updated state is read)
+ *
+ * In h-form, per token:  r = h^T k;  u = beta (v - alpha r);
+ *                        h = alpha h + k u^T;  o = h^T q.
+ * which is the line above transposed: S^T = alpha (I - beta k k^T) S_{t-1}^T
+ * + beta k v^T  and  alpha (I - beta k k^T) h + beta k v^T
+ *  = alpha h + k (beta v - alpha beta k^T h)^T.
+ *
+ * Layouts (row-major, contiguous):
+ *   q, k : [B][T][H][dk]     v, o : [B][T][H][dv]
+ *   g, eta, beta : [B][T][H]
+ *   h0, hT : [B][H][dk][dv]  (h0 may be NULL = zeros; hT may be NULL)
+ * Heads (b, h) are independent; OpenMP runs them in parallel.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* beta_t = eta_t / (||k_t||^2 + eps), one value per (b, t, h). */
+void kla_oracle_beta(const double *k, const double *eta, double eps,
+                     double *beta, int B, int T, int H, int dk)
+{
+    long n = (long)B * T * H;
+    for (long p = 0; p < n; ++p) {
+        const double *kp = k + p * dk;
+        double n2 = 0.0;
+        for (int i = 0; i < dk; ++i) n2 += kp[i] * kp[i];
+        beta[p] = eta[p] / (n2 + eps);
+    }
+}
+
+/* The gated delta rule with beta supplied per token (GDN form). */
+void kla_oracle_gated_delta(const double *q, const double *k, const double *v,
+                            const double *g, const double *beta,
+                            const double *h0, double *o, double *hT,
+                            int B, int T, int H, int dk, int dv)
+{
+    int nheads = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < nheads; ++bh) {
+        int b = bh / H, hh = bh % H;
+        double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+        double *r = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+        if (h0)
+            memcpy(S, h0 + (size_t)bh * dk * dv, sizeof(double) * (size_t)dk * dv);
+        else
+            memset(S, 0, sizeof(double) * (size_t)dk * dv);
+        for (int t = 0; t < T; ++t) {
+            size_t tok = ((size_t)b * T + t) * H + hh;
+            const double *kt = k + tok * dk;
+            const double *qt = q + tok * dk;
+            const double *vt = v + tok * dv;
+            double alpha = exp(g[tok]);
+            double bt = beta[tok];
+            /* r = h^T k  (= S_{t-1} k_t) */
+            for (int j = 0; j < dv; ++j) r[j] = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                const double *Si = S + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) r[j] += Si[j] * kt[i];
+            }
+            /* u = beta (v - alpha r) */
+            for (int j = 0; j < dv; ++j) u[j] = bt * (vt[j] - alpha * r[j]);
+            /* h = alpha h + k u^T */
+            for (int i = 0; i < dk; ++i) {
+                double *Si = S + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) Si[j] = alpha * Si[j] + kt[i] * u[j];
+            }
+            /* o = h^T q with the updated state */
+            double *ot = o + tok * dv;
+            for (int j = 0; j < dv; ++j) ot[j] = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                const double *Si = S + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) ot[j] += Si[j] * qt[i];
+            }
+        }
+        if (hT) memcpy(hT + (size_t)bh * dk * dv, S, sizeof(double) * (size_t)dk * dv);
+        free(S);
+        free(r);
+        free(u);
+    }
+}
+
+/* KLA forward: beta from the key norm, then the gated delta rule. */
+void kla_oracle_forward(const double *q, const double *k, const double *v,
+                        const double *g, const double *eta, double eps,
+                        const double *h0, double *o, double *hT,
+                        int B, int T, int H, int dk, int dv)
+{
+    size_t n = (size_t)B * T * H;
+    double *beta = (double *)malloc(sizeof(double) * (n ? n : 1));
+    kla_oracle_beta(k, eta, eps, beta, B, T, H, dk);
+    kla_oracle_gated_delta(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv);
+    free(beta);
+}
+
+/* Number of OpenMP threads a parallel region would use (for reporting). */
+int kla_oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
