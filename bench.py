@@ -1,0 +1,408 @@
+"""Benchmark of the KLA hot path on B200: prefill tokens/s (+ roofline) and
+decode tokens/s (+ HBM GB/s), one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill_4k]
+  python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N
+  python bench.py --impl reference     # the fp64 oracle on the host cores
+
+A step is one prefill of the workload (default: the 0.4B-scale layer,
+B=8 T=4096 H=8 d=128, bf16) through kla_chunk_fwd.  Each rank processes its
+own batch (independent sequences, no collective on the data path): weak
+scaling.  L2 is flushed (512 MiB written then read) before every timed step
+and each step is bracketed by CUDA events on the launching stream; the job
+time is the max over ranks.  The decode workload (B=64 H=16 d=128, 32K-token
+state, 1000 in-place steps, L2 flushed before each) is measured on every rank
+after the prefill and reported under "decode".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# --------------------------------------------------------------- workloads
+def prefill_work(w):
+    """Algorithmic flops and minimum HBM bytes of one prefill."""
+    C = 64
+    d = w.dk
+    es = 2 if w.dtype == "bf16" else 4
+    ntok = w.B * w.T * w.H  # head-tokens
+    # dense tensor work per head-token: 5 (C x C x d) + 3 (C x d x d) products
+    flops = ntok * (10 * C * d + 6 * d * d)
+    state = w.B * w.H * w.dk * w.dv * 4
+    byts = ntok * (2 * w.dk + 2 * w.dv) * es + ntok * 8 + state * (2 if w.kind == "stress" else 1)
+    return flops, byts
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampling during a timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        busy = sorted(sm)[len(sm) // 2:]  # upper half: samples under load
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class L2Flush:
+    """Writes then reads a buffer larger than L2 (126 MB on B200), so the next
+    kernel starts with a cold L2 and no dirty lines to write back."""
+
+    def __init__(self, dev, mib=512):
+        self.buf = torch.empty(mib * (1 << 20) // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1.0)
+        self.buf.sum()
+
+
+# ------------------------------------------------------------- our arm
+def run_ours(args, rank, world, dev):
+    from delta_rule_linear_kla_b200 import api, inputs
+
+    peaks, peak_src = load_peaks()
+    w = inputs.WORKLOADS[args.workload]
+    w = w.scaled(seed=w.seed + 100 * rank)
+    x = inputs.make_prefill(w)
+    xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    fn = api.chunk_fwd if args.path == "chunk" else api.recurrent_fwd
+    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=w.torch_dtype, device=dev)
+    hT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    flush = L2Flush(dev)
+
+    def step():
+        fn(xd["q"], xd["k"], xd["v"], xd["g"], xd["eta"], x["eps"], xd["h0"], o=o, hT=hT)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    api.check_device_error()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t0 = time.perf_counter()
+        for e0, e1 in evs:
+            flush()
+            e0.record(stream)
+            step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+    barrier(world)
+    api.check_device_error()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    ms_max = allreduce_max(ms, world, dev)
+
+    tokens_per_rank = w.B * w.T
+    value = tokens_per_rank * world / (ms_max / 1e3)
+    flops, byts = prefill_work(w)
+    achieved_gbs = byts / (ms / 1e3) / 1e9
+    achieved_tf = flops / (ms / 1e3) / 1e12
+    hbm_peak = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+
+    # end to end through the public API with host buffers (pinned)
+    e2e = measure_e2e(args, w, x, fn, dev, stream, world)
+
+    res = {
+        "metric": "prefill tokens/s (0.4B-scale layer, T=4096)" if args.workload == "prefill_4k"
+        else "prefill tokens/s (%s)" % args.workload,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded PCG64, distributions of the workload recipe)",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                   "chunk": 64, "path": args.path, "global_batch": w.B * world,
+                   "seq_len": w.T, "parallelism": "dp%d (independent sequences)" % world,
+                   "l2": "flushed before every timed step (512 MiB write+read); inputs > L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": achieved_gbs / hbm_peak, "traffic": None,
+                     "algorithmic_bytes": byts, "peak_source": peak_src},
+        "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
+                   "frac": achieved_tf / tc_peak, "algorithmic_flops": flops,
+                   "peak_source": peak_src + " (burst cuBLAS bf16)"},
+        "gpu_launches": args.steps,
+        "wall_s": wall,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if not args.no_decode:
+        res["decode"] = run_decode(args, rank, dev, stream, flush, peaks, peak_src, fn)
+    return res
+
+
+def measure_e2e(args, w, x, fn, dev, stream, world):
+    """Same metric through the public call with pinned host buffers: H2D of
+    the step's inputs, the prefill, D2H of o and hT, all inside the events."""
+    host = {k: x[k].pin_memory() for k in ("q", "k", "v", "g", "eta")}
+    dbuf = {k: torch.empty_like(host[k], device=dev) for k in host}
+    o_h = torch.empty((w.B, w.T, w.H, w.dv), dtype=w.torch_dtype).pin_memory()
+    h_h = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32).pin_memory()
+    o = torch.empty_like(o_h, device=dev)
+    hT = torch.empty_like(h_h, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + h_h.numel() * h_h.element_size()
+    n = max(2, min(args.steps, 5))
+    times = []
+    for i in range(n + 2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k in dbuf:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["eta"], x["eps"], None, o=o, hT=hT)
+        o_h.copy_(o, non_blocking=True)
+        h_h.copy_(hT, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            times.append(e0.elapsed_time(e1))
+    ms = allreduce_max(sum(times) / len(times), world, dev)
+    return {"value": w.B * w.T * world / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn):
+    """Decode: state = our prefill over the trailing prefix; then in-place steps."""
+    from delta_rule_linear_kla_b200 import api, inputs
+
+    w = inputs.DECODE.scaled(seed=inputs.DECODE.seed + 100 * rank)
+    nsteps = args.decode_steps
+    d = inputs.make_decode(w, steps=nsteps)
+    p = {k: v.to(dev) for k, v in d["prefix"].items()}
+    _, S = prefill_fn(p["q"], p["k"], p["v"], p["g"], p["eta"], d["eps"], None)
+    st = {k: v.to(dev) for k, v in d["steps"].items()}
+    o = torch.empty((w.B, w.H, w.dv), dtype=w.torch_dtype, device=dev)
+    for i in range(3):
+        api.decode_step(st["q"][i], st["k"][i], st["v"][i], st["g"][i], st["eta"][i], S,
+                        d["eps"], o=o)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(nsteps)]
+    torch.cuda.synchronize()
+    for i, (e0, e1) in enumerate(evs):
+        flush()
+        e0.record(stream)
+        api.decode_step(st["q"][i], st["k"][i], st["v"][i], st["g"][i], st["eta"][i], S,
+                        d["eps"], o=o)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / nsteps
+    state_bytes = 2 * w.B * w.H * w.dk * w.dv * 4
+    io_bytes = w.B * w.H * (2 * w.dk + 2 * w.dv) * 2 + w.B * w.H * 8
+    gbs = (state_bytes + io_bytes) / (ms / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    return {"metric": "decode tokens/s (B=64 H=16 d=128, 32K-token state)",
+            "value": w.B / (ms / 1e3), "unit": "tokens/s", "us_per_step": ms * 1e3,
+            "steps": nsteps, "l2": "flushed before every step",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                         "frac": gbs / peak, "traffic": None,
+                         "algorithmic_bytes": state_bytes + io_bytes,
+                         "peak_source": peak_src}}
+
+
+# ------------------------------------------------------------ reference
+def run_reference(args, world, rank):
+    """The fp64 oracle on the host cores, on a bounded sample of the workload."""
+    import oracle
+    from delta_rule_linear_kla_b200 import inputs
+
+    w = inputs.WORKLOADS[args.workload]
+    x = inputs.make_prefill(w)
+    cores = oracle.num_threads()
+    # sample: the first n_heads heads (b-major) of the workload, full length
+    nh = max(1, min(w.B * w.H, args.ref_heads or w.B * w.H))
+    B_s = max(1, min(w.B, (nh + w.H - 1) // w.H))
+    H_s = min(w.H, nh)
+    xs = {k: x[k][:B_s, :, :H_s].contiguous() for k in ("q", "k", "v", "g", "eta")}
+    h0 = None if x["h0"] is None else x["h0"][:B_s, :H_s].contiguous()
+    for _ in range(args.warmup if args.warmup < 2 else 1):
+        oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["eta"], x["eps"], h0)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["eta"], x["eps"], h0)
+        times.append(time.perf_counter() - t0)
+    t = sum(times) / len(times)
+    head_tokens = B_s * H_s * w.T
+    value = head_tokens / w.H / t  # tokens/s (a token = one position of all H heads)
+    sample = "%d of %d heads x T=%d of %s (first heads, full length)" % (
+        B_s * H_s, w.B * w.H, w.T, w.name)
+    return {"metric": "prefill tokens/s (0.4B-scale layer, T=4096)" if args.workload == "prefill_4k"
+            else "prefill tokens/s (%s)" % args.workload,
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded PCG64)", "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk,
+                       "dv": w.dv, "chunk": 64},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def cpu_baseline(args, budget_s=15.0):
+    """The oracle as it stands, timed on this host on a bounded sample."""
+    import oracle
+    from delta_rule_linear_kla_b200 import inputs
+
+    w = inputs.WORKLOADS[args.workload]
+    cores = oracle.num_threads()
+    nh = min(w.B * w.H, max(cores, 1))
+    B_s = max(1, (nh + w.H - 1) // w.H)
+    H_s = min(w.H, nh)
+    # probe the per-token cost, then size the sample to ~budget_s
+    T_probe = min(w.T, 256)
+    xs = inputs.make_prefill(w.scaled(B=B_s, T=T_probe, H=H_s))
+    t0 = time.perf_counter()
+    oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["eta"], xs["eps"], xs["h0"])
+    dt = time.perf_counter() - t0
+    T_s = int(min(w.T, max(T_probe, T_probe * budget_s / max(dt, 1e-3))))
+    xs = inputs.make_prefill(w.scaled(B=B_s, T=T_s, H=H_s))
+    t0 = time.perf_counter()
+    oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["eta"], xs["eps"], xs["h0"])
+    t = time.perf_counter() - t0
+    value = B_s * H_s * T_s / w.H / t
+    return {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "%d heads x T=%d drawn like %s (%.1f s of fp64 CPU work)"
+                      % (B_s * H_s, T_s, w.name, t)}
+
+
+# ---------------------------------------------------------- distributed
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def allreduce_max(x, world, dev):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_4k",
+                    choices=["prefill_4k", "prefill_65k", "stress", "tiny"])
+    ap.add_argument("--path", choices=["chunk", "recurrent"], default="chunk")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-heads", type=int, default=0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return 0
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=dev,
+                                             timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_ours(args, rank, world, dev)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

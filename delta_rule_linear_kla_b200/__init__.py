@@ -4,7 +4,8 @@ The public calls live in :mod:`delta_rule_linear_kla_b200.api`; they marshal
 torch tensors into the C ABI of ``libkla.so`` (declared in ``include/kla.h``),
 whose CUDA kernels do all of the arithmetic.
 """
-from .api import (chunk_fwd, decode_step, chunk_fwd_workspace_size,  # noqa: F401
-                  KLAError)
+from .api import (KLAError, check_device_error, chunk_fwd,  # noqa: F401
+                  chunk_fwd_workspace_size, decode_step, recurrent_fwd)
 
-__all__ = ["chunk_fwd", "decode_step", "chunk_fwd_workspace_size", "KLAError"]
+__all__ = ["chunk_fwd", "recurrent_fwd", "decode_step", "chunk_fwd_workspace_size",
+           "check_device_error", "KLAError"]

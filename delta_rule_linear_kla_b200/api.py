@@ -1,17 +1,134 @@
-"""Python binding of the KLA C ABI (filled in with the CUDA library)."""
+"""Python binding of the KLA C ABI (include/kla.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libkla.so.  Tensors must live on the current CUDA device; outputs
+are allocated here with torch (the library itself never allocates).
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import _native
+
+KLA_BF16, KLA_FP32 = 0, 1
+CHUNK = 64
+_DT = {torch.bfloat16: KLA_BF16, torch.float32: KLA_FP32}
 
 
 class KLAError(RuntimeError):
-    pass
+    """A non-OK kla_status returned by the library."""
+
+    def __init__(self, status: int, where: str):
+        msg = _native.lib().kla_status_string(status).decode()
+        super().__init__("%s: %s (status %d)" % (where, msg, status))
+        self.status = status
 
 
-def chunk_fwd(*a, **k):
-    raise KLAError("CUDA library not built yet")
+def _check(status: int, where: str):
+    if status != 0:
+        raise KLAError(status, where)
 
 
-def decode_step(*a, **k):
-    raise KLAError("CUDA library not built yet")
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
 
 
-def chunk_fwd_workspace_size(*a, **k):
-    raise KLAError("CUDA library not built yet")
+def _need(t, name, dtype=None, shape=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
+                             dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(_native.lib().kla_chunk_fwd_workspace_size(B, T, H, dk, dv, _DT[dtype]))
+
+
+def _prefill_args(q, k, v, g, eta, h0, o, hT, return_state):
+    _need(q, "q")
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v must be bfloat16 or float32")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", q.dtype, (B, T, H, dk))
+    _need(v, "v", q.dtype, (B, T, H, dv))
+    _need(g, "g", torch.float32, (B, T, H))
+    _need(eta, "eta", torch.float32, (B, T, H))
+    _need(h0, "h0", torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, (B, T, H, dv))
+    if hT is None and return_state:
+        hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(hT, "hT", torch.float32, (B, H, dk, dv))
+    return B, T, H, dk, dv, o, hT
+
+
+def chunk_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
+              return_state: bool = True, workspace=None,
+              stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise KLA prefill (kla_chunk_fwd).  Returns (o, hT)."""
+    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, eta, h0, o, hT, return_state)
+    need = chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _native.lib().kla_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0),
+        _ptr(o), _ptr(hT), B, T, H, dk, dv, CHUNK, _DT[q.dtype], _ptr(workspace),
+        ws_bytes, _stream(stream))
+    _check(st, "kla_chunk_fwd")
+    return o, hT
+
+
+def recurrent_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
+                  return_state: bool = True, stream=None):
+    """Token-serial KLA prefill on CUDA cores (kla_recurrent_fwd)."""
+    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, eta, h0, o, hT, return_state)
+    st = _native.lib().kla_recurrent_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0),
+        _ptr(o), _ptr(hT), B, T, H, dk, dv, _DT[q.dtype], _stream(stream))
+    _check(st, "kla_recurrent_fwd")
+    return o, hT
+
+
+def decode_step(q, k, v, g, eta, S, eps: float = 1e-6, *, o=None, stream=None):
+    """One decode token per sequence; S [B,H,dk,dv] fp32 is updated in place.
+    Returns o [B,H,dv]."""
+    _need(q, "q")
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v must be bfloat16 or float32")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", q.dtype, (B, H, dk))
+    _need(v, "v", q.dtype, (B, H, dv))
+    _need(g, "g", torch.float32, (B, H))
+    _need(eta, "eta", torch.float32, (B, H))
+    _need(S, "S", torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, (B, H, dv))
+    st = _native.lib().kla_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(S), _ptr(o),
+        B, H, dk, dv, _DT[q.dtype], _stream(stream))
+    _check(st, "kla_decode_step")
+    return o
+
+
+def check_device_error(stream=None):
+    """Synchronise and raise KLAError if a kernel reported a timed-out wait."""
+    _check(_native.lib().kla_check_device_error(_stream(stream)), "kla_check_device_error")

@@ -1,0 +1,183 @@
+// C ABI entry points of libkla.so: argument validation on the host, then a
+// launch on the caller's stream.  No entry point allocates device memory or
+// synchronises, except kla_check_device_error which is documented to.
+#include <string.h>
+
+#include "kla_common.cuh"
+#include "kla_chunk.h"
+
+namespace kla {
+
+// Device error word (see kla_common.cuh); read back by kla_check_device_error.
+__device__ unsigned int g_device_error = 0;
+
+static const int kMaxDevices = 64;
+static unsigned int* g_err_ptr[kMaxDevices];
+
+// Address of this device's error word (looked up once per device).
+unsigned int* device_error_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = (unsigned int*)p;
+  }
+  return g_err_ptr[dev];
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+static Range rng(const void* p, size_t bytes) {
+  return Range{(uintptr_t)p, (uintptr_t)p + bytes};
+}
+static bool overlap(Range a, Range b) {
+  return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi;
+}
+
+static bool head_dims_ok(int dk, int dv) {
+  return (dk == 64 && dv == 64) || (dk == 128 && dv == 128);
+}
+
+// Shared validation of the prefill entry points.
+static kla_status check_prefill(const void* q, const void* k, const void* v,
+                                const float* g, const float* eta, float eps,
+                                const float* h0, const void* o, const float* hT,
+                                int B, int T, int H, int dk, int dv, int dtype) {
+  if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return KLA_ERR_INVALID_ARG;
+  if (dtype != KLA_BF16 && dtype != KLA_FP32) return KLA_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || eps != eps) return KLA_ERR_INVALID_ARG;
+  if ((long long)B * T * H * (dk > dv ? dk : dv) >= (1LL << 40)) return KLA_ERR_INVALID_ARG;
+  if (T > 0 && (!q || !k || !v || !g || !eta || !o)) return KLA_ERR_INVALID_ARG;
+  if (T == 0 && hT == nullptr) return KLA_OK;
+  const void* ptrs[] = {q, k, v, g, eta, h0, o, hT};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KLA_ERR_INVALID_ARG;
+  if (!head_dims_ok(dk, dv)) return KLA_ERR_UNSUPPORTED;
+  const size_t es = dtype == KLA_BF16 ? 2 : 4;
+  const size_t ntok = (size_t)B * T * H;
+  if (o && T > 0) {
+    Range ro = rng(o, ntok * dv * es);
+    Range ins[] = {rng(q, ntok * dk * es), rng(k, ntok * dk * es), rng(v, ntok * dv * es),
+                   rng(g, ntok * 4), rng(eta, ntok * 4),
+                   rng(h0, h0 ? (size_t)B * H * dk * dv * 4 : 0),
+                   rng(hT, hT ? (size_t)B * H * dk * dv * 4 : 0)};
+    for (Range r : ins)
+      if (overlap(ro, r)) return KLA_ERR_INVALID_ARG;
+  }
+  if (hT && h0 && hT != h0) {
+    const size_t sb = (size_t)B * H * dk * dv * 4;
+    if (overlap(rng(hT, sb), rng(h0, sb))) return KLA_ERR_INVALID_ARG;
+  }
+  return KLA_OK;
+}
+
+// T == 0: the final state is the initial state.
+static kla_status empty_prefill(const float* h0, float* hT, int B, int H, int dk,
+                                int dv, cudaStream_t st) {
+  if (!hT) return KLA_OK;
+  const size_t sb = (size_t)B * H * dk * dv * sizeof(float);
+  cudaError_t e = h0 ? (hT == h0 ? cudaSuccess
+                                 : cudaMemcpyAsync(hT, h0, sb, cudaMemcpyDeviceToDevice, st))
+                     : cudaMemsetAsync(hT, 0, sb, st);
+  return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+}  // namespace kla
+
+using namespace kla;
+
+extern "C" {
+
+size_t kla_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int dtype) {
+  return chunk_workspace_bytes(B, T, H, dk, dv, dtype);
+}
+
+kla_status kla_chunk_fwd(const void* q, const void* k, const void* v,
+                         const float* g, const float* eta, float eps,
+                         const float* h0, void* o, float* hT, int B, int T, int H,
+                         int dk, int dv, int chunk, int dtype, void* workspace,
+                         size_t ws_bytes, void* stream) {
+  kla_status s = check_prefill(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype);
+  if (s != KLA_OK) return s;
+  if (chunk != KLA_CHUNK) return KLA_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (T == 0) return empty_prefill(h0, hT, B, H, dk, dv, st);
+  const size_t need = chunk_workspace_bytes(B, T, H, dk, dv, dtype);
+  if (ws_bytes < need || (need > 0 && workspace == nullptr)) return KLA_ERR_INVALID_ARG;
+  if (workspace && !aligned16(workspace)) return KLA_ERR_INVALID_ARG;
+  cudaError_t e;
+  if (dtype == KLA_FP32) {
+    e = launch_recurrent(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype, st);
+  } else {
+    unsigned int* err = device_error_ptr();
+    if (!err) return KLA_ERR_CUDA;
+    e = launch_chunk_tc(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, workspace,
+                        err, st);
+    if (e == cudaErrorNotSupported) return KLA_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+kla_status kla_recurrent_fwd(const void* q, const void* k, const void* v,
+                             const float* g, const float* eta, float eps,
+                             const float* h0, void* o, float* hT, int B, int T,
+                             int H, int dk, int dv, int dtype, void* stream) {
+  kla_status s = check_prefill(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype);
+  if (s != KLA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (T == 0) return empty_prefill(h0, hT, B, H, dk, dv, st);
+  cudaError_t e = launch_recurrent(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv,
+                                   dtype, st);
+  return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+kla_status kla_decode_step(const void* q, const void* k, const void* v,
+                           const float* g, const float* eta, float eps, float* S,
+                           void* o, int B, int H, int dk, int dv, int dtype,
+                           void* stream) {
+  if (B < 1 || H < 1) return KLA_ERR_INVALID_ARG;
+  if (dtype != KLA_BF16 && dtype != KLA_FP32) return KLA_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, g, eta, S, o};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return KLA_ERR_INVALID_ARG;
+  if (!head_dims_ok(dk, dv)) return KLA_ERR_UNSUPPORTED;
+  const size_t es = dtype == KLA_BF16 ? 2 : 4;
+  const size_t nh = (size_t)B * H;
+  Range ro = rng(o, nh * dv * es);
+  Range others[] = {rng(q, nh * dk * es), rng(k, nh * dk * es), rng(v, nh * dv * es),
+                    rng(g, nh * 4), rng(eta, nh * 4), rng(S, nh * dk * dv * 4)};
+  for (Range r : others)
+    if (overlap(ro, r)) return KLA_ERR_INVALID_ARG;
+  cudaError_t e = launch_decode(q, k, v, g, eta, eps, S, o, B, H, dk, dv, dtype,
+                                (cudaStream_t)stream);
+  return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+kla_status kla_check_device_error(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return KLA_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return KLA_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+    return KLA_ERR_CUDA;
+  return v ? KLA_ERR_TIMEOUT : KLA_OK;
+}
+
+const char* kla_status_string(int status) {
+  switch (status) {
+    case KLA_OK: return "ok";
+    case KLA_ERR_INVALID_ARG: return "invalid argument";
+    case KLA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KLA_ERR_CUDA: return "CUDA error";
+    case KLA_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int kla_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// Shared helpers of the KLA CUDA library: element loads/stores for the two
+// I/O types, warp reductions and the device error word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kla.h"
+
+namespace kla {
+
+// Device error word: one per device, owned by kla_api.cu, passed to kernels
+// as a pointer.  Bounded waits that give up set a bit instead of hanging.
+enum : unsigned int { KLA_DEVERR_TIMEOUT = 1u };
+
+__device__ __forceinline__ void report_timeout(unsigned int* err) {
+  atomicOr(err, KLA_DEVERR_TIMEOUT);
+}
+
+// Launchers (one per kernel family), all queue work on `st` only.
+cudaError_t launch_decode(const void* q, const void* k, const void* v,
+                          const float* g, const float* eta, float eps, float* S,
+                          void* o, int B, int H, int dk, int dv, int dtype,
+                          cudaStream_t st);
+cudaError_t launch_recurrent(const void* q, const void* k, const void* v,
+                             const float* g, const float* eta, float eps,
+                             const float* h0, void* o, float* hT, int B, int T,
+                             int H, int dk, int dv, int dtype, cudaStream_t st);
+
+template <typename T> struct IO;
+
+template <> struct IO<float> {
+  static __device__ __forceinline__ float ld(const float* p) { return *p; }
+  static __device__ __forceinline__ void st(float* p, float x) { *p = x; }
+  // 4 consecutive elements
+  static __device__ __forceinline__ float4 ld4(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+  }
+  static __device__ __forceinline__ void st4(float* p, float4 x) {
+    *reinterpret_cast<float4*>(p) = x;
+  }
+};
+
+template <> struct IO<__nv_bfloat16> {
+  static __device__ __forceinline__ float ld(const __nv_bfloat16* p) {
+    return __bfloat162float(*p);
+  }
+  static __device__ __forceinline__ void st(__nv_bfloat16* p, float x) {
+    *p = __float2bfloat16_rn(x);
+  }
+  static __device__ __forceinline__ float4 ld4(const __nv_bfloat16* p) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  }
+  static __device__ __forceinline__ void st4(__nv_bfloat16* p, float4 x) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(x.z, x.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+};
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+}  // namespace kla

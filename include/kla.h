@@ -1,0 +1,137 @@
+/*
+ * kla.h -- C ABI of the Kaczmarz Linear Attention (KLA) hot path on NVIDIA
+ * B200 (sm_100a).  Library: libkla.so (delta_rule_linear_kla_b200/).
+ *
+ * The method (h = S^T is stored, one [dk][dv] fp32 matrix per head):
+ *
+ *   beta_t = eta_t / (||k_t||_2^2 + eps)
+ *       -- "Kaczmarz Linear Attention" (arXiv 2605.08587 summary), Abstract:
+ *          the key-norm-normalised step size of the Kaczmarz projection.
+ *   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *   alpha_t = exp(g_t),   o_t = S_t q_t
+ *       -- "Deep Dive into KDA", section 2.2 (Gated DeltaNet), which the KLA
+ *          Abstract keeps except for beta; the erase factor is placed where
+ *          S (dv x dk) type-checks, and o reads the updated state.
+ *
+ * Conventions shared by every call:
+ *   * All tensors are device pointers, contiguous, row-major, 16-byte
+ *     aligned, on the current device, in the layouts stated per argument.
+ *   * The caller owns every buffer (including any workspace).  The library
+ *     allocates no device memory and never synchronises the stream: work is
+ *     queued on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream) and returns immediately.
+ *   * Arguments are validated on the host before anything is launched; a
+ *     bad argument returns KLA_ERR_INVALID_ARG or KLA_ERR_UNSUPPORTED and
+ *     leaves every buffer untouched.  A failed launch returns KLA_ERR_CUDA.
+ *     No call aborts, throws or prints.
+ *   * dtype selects the element type of q, k, v and o (KLA_BF16 or
+ *     KLA_FP32); g, eta, states are always fp32.  Arithmetic is fp32
+ *     (tensor-core products take bf16 operands with fp32 accumulation).
+ */
+#ifndef KLA_H_
+#define KLA_H_
+
+#include <stddef.h>
+
+/* Every entry point below is exported from libkla.so; the rest is hidden. */
+#if defined(__GNUC__)
+#define KLA_API __attribute__((visibility("default")))
+#else
+#define KLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KLA_OK = 0,
+    KLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, aliasing */
+    KLA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not 64/128) */
+    KLA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or launch failed   */
+    KLA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up            */
+} kla_status;
+
+typedef enum { KLA_BF16 = 0, KLA_FP32 = 1 } kla_dtype;
+
+/* Chunk length of the chunkwise prefill ("Deep Dive into KDA", section 3:
+ * the sequence is cut into chunks of C tokens).  Fixed at compile time. */
+#define KLA_CHUNK 64
+
+/*
+ * Prefill forward (chunkwise parallel form, "Deep Dive into KDA", section 3).
+ *
+ *   q, k    [B][T][H][dk]  dtype       queries, keys (keys are NOT normalised;
+ *                                      beta carries the key norm)
+ *   v       [B][T][H][dv]  dtype       values
+ *   g       [B][T][H]      fp32        log gate, alpha_t = exp(g_t)
+ *   eta     [B][T][H]      fp32        relaxation eta_t of the Kaczmarz step
+ *   eps                    fp32        added to ||k_t||^2 (KLA Abstract)
+ *   h0      [B][H][dk][dv] fp32        initial state h = S^T; NULL = zeros
+ *   o       [B][T][H][dv]  dtype       output, o_t = S_t q_t (written)
+ *   hT      [B][H][dk][dv] fp32        final state (written); NULL = not
+ *                                      returned.  hT may alias h0 exactly.
+ *   chunk   must equal KLA_CHUNK (else KLA_ERR_UNSUPPORTED)
+ *   workspace / ws_bytes: caller-owned device scratch of at least
+ *     kla_chunk_fwd_workspace_size(...) bytes (NULL allowed when that is 0).
+ *
+ * Supported: B, H >= 1; T >= 0 (T = 0 copies h0 to hT); dk = dv in {64, 128}.
+ * A ragged tail (T not a multiple of the chunk) is processed as if padded
+ * with g = 0, eta = 0, which is an exact identity step.
+ * o must not overlap any input.  bf16 runs the tcgen05 chunk kernel; fp32
+ * runs the token-serial CUDA-core kernel (kla_recurrent_fwd).
+ */
+KLA_API size_t kla_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int dtype);
+
+KLA_API kla_status kla_chunk_fwd(const void *q, const void *k, const void *v,
+                         const float *g, const float *eta, float eps,
+                         const float *h0, void *o, float *hT,
+                         int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Token-serial prefill on CUDA cores: the recurrence evaluated one token at
+ * a time in fp32 (same arguments and layouts as kla_chunk_fwd, no chunk and
+ * no workspace).  Exact-order fp32 evaluation, used for the fp32 I/O mode.
+ * Supported: dk, dv in {64, 128}.
+ */
+KLA_API kla_status kla_recurrent_fwd(const void *q, const void *k, const void *v,
+                             const float *g, const float *eta, float eps,
+                             const float *h0, void *o, float *hT,
+                             int B, int T, int H, int dk, int dv, int dtype,
+                             void *stream);
+
+/*
+ * One decode step for B sequences (one new token each), updating the state
+ * in place -- the recurrence above for a single t.
+ *
+ *   q, k  [B][H][dk] dtype;  v [B][H][dv] dtype
+ *   g, eta [B][H] fp32;  eps fp32
+ *   S     [B][H][dk][dv] fp32   state h = S^T, read and overwritten
+ *   o     [B][H][dv] dtype      o = S_t q (the updated state)
+ * Supported: dk, dv in {64, 128}.  o must not overlap S or the inputs.
+ */
+KLA_API kla_status kla_decode_step(const void *q, const void *k, const void *v,
+                           const float *g, const float *eta, float eps,
+                           float *S, void *o, int B, int H, int dk, int dv,
+                           int dtype, void *stream);
+
+/*
+ * Reads and clears the library's device error word for the current device
+ * after synchronising `stream`.  Kernels set it instead of hanging when a
+ * bounded wait on an mbarrier runs out (KLA_ERR_TIMEOUT).  Returns KLA_OK
+ * when no kernel reported a problem.
+ */
+KLA_API kla_status kla_check_device_error(void *stream);
+
+/* Static description of a status code (never NULL). */
+KLA_API const char *kla_status_string(int status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+KLA_API int kla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KLA_H_ */

@@ -1,0 +1,76 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+entry point include/kla.h declares, and rejects bad arguments on the host
+before any CUDA call (no compute call is made here)."""
+import ctypes
+
+import pytest
+
+from delta_rule_linear_kla_b200 import _native
+from delta_rule_linear_kla_b200 import build as kbuild
+
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+A = 1 << 20  # fake, 16-byte-aligned device addresses: never dereferenced here
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return _native.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _native.header_symbols()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_native.SIGNATURES)
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.kla_status_string(s)
+    assert lib.kla_status_string(99) == b"unknown status"
+    assert lib.kla_version() >= 100
+
+
+def _fwd(lib, q=A, k=2 * A, v=3 * A, g=4 * A, eta=5 * A, eps=1e-6, h0=None, o=6 * A,
+         hT=None, B=1, T=128, H=2, dk=128, dv=128, chunk=64, dtype=0, ws=None, wsb=0):
+    return lib.kla_chunk_fwd(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, chunk,
+                             dtype, ws, wsb, None)
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    assert _fwd(lib, q=None) == INVALID
+    assert _fwd(lib, o=None) == INVALID
+    assert _fwd(lib, k=2 * A + 8) == INVALID          # misaligned
+    assert _fwd(lib, B=0) == INVALID
+    assert _fwd(lib, T=-1) == INVALID
+    assert _fwd(lib, dtype=7) == INVALID
+    assert _fwd(lib, eps=-1.0) == INVALID
+    assert _fwd(lib, eps=float("nan")) == INVALID
+    assert _fwd(lib, o=A + 256) == INVALID             # o overlaps q
+    assert _fwd(lib, h0=7 * A, hT=7 * A + 1024) == INVALID  # partial state overlap
+    assert _fwd(lib, dk=96, dv=96) == UNSUPPORTED
+    assert _fwd(lib, dk=128, dv=64) == UNSUPPORTED
+    assert _fwd(lib, chunk=32) == UNSUPPORTED
+    assert lib.kla_recurrent_fwd(None, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, None, 6 * A,
+                                 None, 1, 4, 1, 64, 64, 1, None) == INVALID
+    assert lib.kla_recurrent_fwd(A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, None, 6 * A,
+                                 None, 1, 4, 1, 32, 32, 1, None) == UNSUPPORTED
+
+
+def test_decode_rejects_bad_arguments(lib):
+    args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, 6 * A, 7 * A, 2, 3, 128, 128, 0, None]
+    bad = list(args); bad[6] = None
+    assert lib.kla_decode_step(*bad) == INVALID
+    bad = list(args); bad[7] = 6 * A + 64            # o inside S
+    assert lib.kla_decode_step(*bad) == INVALID
+    bad = list(args); bad[10], bad[11] = 80, 80
+    assert lib.kla_decode_step(*bad) == UNSUPPORTED
+    bad = list(args); bad[8] = 0
+    assert lib.kla_decode_step(*bad) == INVALID
+
+
+def test_workspace_query(lib):
+    n = lib.kla_chunk_fwd_workspace_size(8, 4096, 8, 128, 128, 0)
+    assert n >= 0 and n < (1 << 34)
