@@ -17,6 +17,7 @@ after the prefill and reported under "decode".
 from __future__ import annotations
 
 import argparse
+import functools
 import json
 import os
 import statistics
@@ -83,7 +84,12 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.rows.append([c.strip() for c in line.split(",")])
+            self.rows.append((time.perf_counter(), [c.strip() for c in line.split(",")]))
+
+    def wait_first(self, timeout=3.0):
+        t0 = time.perf_counter()
+        while self.proc and not self.rows and time.perf_counter() - t0 < timeout:
+            time.sleep(0.02)
 
     def __exit__(self, *a):
         if self.proc:
@@ -93,10 +99,14 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, t_lo=None, t_hi=None):
+        """Median SM clock (upper half of the samples: under load) and the
+        throttle reasons seen between host times t_lo and t_hi."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in self.rows:
+        for ts, r in self.rows:
+            if (t_lo is not None and ts < t_lo) or (t_hi is not None and ts > t_hi):
+                continue
             try:
                 sm.append(float(r[1]))
                 mx = float(r[2])
@@ -133,32 +143,46 @@ def run_ours(args, rank, world, dev):
     w = w.scaled(seed=w.seed + 100 * rank)
     x = inputs.make_prefill(w)
     xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-    fn = api.chunk_fwd if args.path == "chunk" else api.recurrent_fwd
     o = torch.empty((w.B, w.T, w.H, w.dv), dtype=w.torch_dtype, device=dev)
     hT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    if args.path == "chunk":
+        nws = api.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype)
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+        fn = functools.partial(api.chunk_fwd, workspace=ws)
+    else:
+        fn = api.recurrent_fwd
     stream = torch.cuda.current_stream()
     flush = L2Flush(dev)
 
     def step():
         fn(xd["q"], xd["k"], xd["v"], xd["g"], xd["eta"], x["eps"], xd["h0"], o=o, hT=hT)
 
-    for _ in range(args.warmup):
+    clk = ClockSampler(dev.index).__enter__()
+    clk.wait_first()
+    # warm-up: at least W steps, and at least ~1 s of back-to-back steps so
+    # the clock samples that bracket the timed region are taken under load
+    t_load = time.perf_counter()
+    i = 0
+    while i < args.warmup or time.perf_counter() - t_load < 1.0:
         flush()
         step()
+        i += 1
+        if i % 8 == 0:
+            torch.cuda.synchronize()
     api.check_device_error()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clk:
-        t0 = time.perf_counter()
-        for e0, e1 in evs:
-            flush()
-            e0.record(stream)
-            step()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        wall = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    for e0, e1 in evs:
+        flush()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    t1 = time.perf_counter()
     barrier(world)
     api.check_device_error()
     ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
@@ -201,11 +225,15 @@ def run_ours(args, rank, world, dev):
                    "peak_source": peak_src + " (burst cuBLAS bf16)"},
         "gpu_launches": args.steps,
         "wall_s": wall,
-        "clocks": clk.summary(),
         "e2e": e2e,
     }
     if not args.no_decode:
-        res["decode"] = run_decode(args, rank, dev, stream, flush, peaks, peak_src, fn)
+        res["decode"] = run_decode(args, rank, dev, stream, flush, peaks, peak_src, fn, clk)
+    time.sleep(0.25)
+    clk.__exit__()
+    res["clocks"] = clk.summary(t_load, t1 + 0.15)
+    res["clocks"]["window"] = "samples from 1 s of back-to-back warm-up steps and the timed steps"
+    res["warmup_steps_run"] = i
     return res
 
 
@@ -239,7 +267,7 @@ def measure_e2e(args, w, x, fn, dev, stream, world):
             "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
-def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn):
+def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn, clk):
     """Decode: state = our prefill over the trailing prefix; then in-place steps."""
     from delta_rule_linear_kla_b200 import api, inputs
 
@@ -256,6 +284,7 @@ def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(nsteps)]
     torch.cuda.synchronize()
+    t0 = time.perf_counter()
     for i, (e0, e1) in enumerate(evs):
         flush()
         e0.record(stream)
@@ -263,6 +292,8 @@ def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn):
                         d["eps"], o=o)
         e1.record(stream)
     torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    api.check_device_error()
     ms = sum(a.elapsed_time(b) for a, b in evs) / nsteps
     state_bytes = 2 * w.B * w.H * w.dk * w.dv * 4
     io_bytes = w.B * w.H * (2 * w.dk + 2 * w.dv) * 2 + w.B * w.H * 8
@@ -271,6 +302,7 @@ def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn):
     return {"metric": "decode tokens/s (B=64 H=16 d=128, 32K-token state)",
             "value": w.B / (ms / 1e3), "unit": "tokens/s", "us_per_step": ms * 1e3,
             "steps": nsteps, "l2": "flushed before every step",
+            "clocks": clk.summary(t0, t1 + 0.15), "gpu_launches": nsteps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": None,
                          "algorithmic_bytes": state_bytes + io_bytes,

@@ -1,19 +1,34 @@
-// Host-side interface of the chunkwise tensor-core prefill (kla_chunk_tc.cu).
+// Host-side interface of the chunkwise tensor-core prefill.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
+#include <stdint.h>
 
 namespace kla {
 
-// Device scratch the chunk kernel needs for these sizes (bytes, 0 if none).
+// Bytes of one chunk's UT factors in the workspace: T' = T diag(beta) and
+// T'' = T diag(beta e^G), two 64x64 bf16 tiles stored exactly as the chain
+// kernel wants them in shared memory (128-byte swizzled rows).
+constexpr size_t kUtTileBytes = 2 * 64 * 64 * 2;
+
+// Device scratch the chunk path needs for these sizes (bytes, 0 if none).
 size_t chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
 
-// bf16 I/O chunkwise prefill.  Returns cudaErrorNotSupported for shapes the
-// kernel does not handle; `err` is this device's error word.
+// bf16 I/O chunkwise prefill (UT kernel, then the chain kernel).  Returns
+// cudaErrorNotSupported for shapes it does not handle; `err` is this
+// device's error word.
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v,
                             const float* g, const float* eta, float eps,
                             const float* h0, void* o, float* hT, int B, int T,
                             int H, int dk, int dv, void* workspace,
                             unsigned int* err, cudaStream_t st);
+
+// UT kernel alone: T', T'' of every chunk into `ws` (chunk-major order
+// ((b * H + h) * nchunks + n)).  `tm_k` maps k as [B][T][H][dk] bf16 with
+// 64 x 64 boxes and 128-byte swizzle.
+cudaError_t launch_ut(const CUtensorMap& tm_k, const float* g, const float* eta, float eps,
+                      uint8_t* ws, int B, int T, int H, int dk, unsigned int* err,
+                      cudaStream_t st);
 
 }  // namespace kla

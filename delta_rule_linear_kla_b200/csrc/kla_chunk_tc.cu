@@ -1,14 +1,466 @@
-// Chunkwise tensor-core prefill (placeholder until the tcgen05 kernel lands).
-#include "kla_common.cuh"
+// Chunkwise KLA prefill on sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Two kernels.  The UT kernel (kla_ut.cu) runs first, in parallel over every
+// chunk, and leaves T' = T diag(beta) and T'' = T diag(beta e^G) of each chunk
+// in the workspace, where T = (I + A)^{-1} and
+// A = strict_lower(diag(beta) K K^T (*) e^{G_r - G_s}).  The chain kernel here
+// then has one CTA per head (b, h) and 64-column slab of the state h = S^T
+// ([DK][DV] fp32), walking the sequence chunk by chunk (C = 64 tokens) with
+// its fp32 state slab in registers for the whole sequence.  Per chunk
+// ("Deep Dive into KDA", section 3, specialised to a scalar gate, with the
+// KLA step size of "Kaczmarz Linear Attention", Abstract):
+//
+//   G_r = sum_{j<=r} g_j  (in chunk)
+//   P  = lower_incl(Q K^T (*) e^{G_r - G_s})                       [MMA 1]
+//   W  = T'' K,  U = T' V     (T', T'' fetched from the workspace)  [MMA 2,3]
+//   V' = U - W h                                                    [MMA 4]
+//   O  = diag(e^G) Q h + P V'                                       [MMA 4,6]
+//   h <- e^{G_63} h + K^T diag(e^{G_63 - G_s}) V'                   [MMA 5]
+//
+// The decay ratios are only ever formed as masked differences of G (never
+// K / Gamma), so strong gates cannot overflow.  A ragged tail is zero-filled
+// by TMA and given g = eta = 0, an exact identity step.
+//
+// Every contraction is a single-CTA tcgen05.mma with M = 128 (products with
+// 64 output rows are stacked or padded to 128 lanes so TMEM lane = row):
+//   MMA 1  D_S[128x64]  = [K; Q] . K^T           A, B K-major (QK^T used)
+//   MMA 2  D_W[128xDK]  = [T''; P] . K           A K-major, B MN-major
+//   MMA 3  D_U[128x64]  = [T'; T''] . V          A K-major, B MN-major
+//   MMA 4  D_1[128x64]  = [W; e^G Q] . h         A K-major, B MN-major
+//   MMA 5  D_H[128x64]  = K^T . (decay V')       A, B MN-major
+//   MMA 6  D_1[64:128] += P . V'                 A K-major, B MN-major
+// (T' = T diag(beta), T'' = T diag(beta e^G); rows 64..127 of MMA 2/3 and
+// rows 0..63 of MMA 6 are don't-care lanes.)  Operands are bf16 in 128-byte
+// swizzled shared-memory panels, accumulators fp32 in TMEM.
+//
+// Every mbarrier wait is bounded (2 s of %globaltimer); on timeout the kernel
+// sets the device error word, drains its own TMA loads (bounded), frees TMEM
+// and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kla_chunk.h"
+#include "kla_common.cuh"
+#include "ptx_sm100.cuh"
+#include "kla_sync.cuh"
+#include "tile_sw128.cuh"
 
 namespace kla {
+namespace {
 
-size_t chunk_workspace_bytes(int, int, int, int, int, int) { return 0; }
+constexpr int C = 64;       // chunk length
+constexpr int BV = 64;      // state columns per CTA
+constexpr int NTHREADS = 128;
+constexpr uint32_t TMEM_COLS = 512;
+// TMEM column offsets of the accumulators
+constexpr uint32_t COL_S = 0, COL_W = 64, COL_U = 192, COL_1 = 256, COL_H = 320;
 
-cudaError_t launch_chunk_tc(const void*, const void*, const void*, const float*,
-                            const float*, float, const float*, void*, float*, int,
-                            int, int, int, int, void*, unsigned int*, cudaStream_t) {
+template <int DK>
+struct alignas(1024) ChunkSmem {
+  static constexpr int NP = DK / 64;  // 64-column panels of a key row
+  // [buffer][panel]: K rows 0..63 (8 KB) then Q rows 0..63 (8 KB)
+  uint8_t kq[2][NP][16384];
+  uint8_t v[2][8192];          // V slab, rows s, 64 columns
+  // [buffer]: T' (8 KB), T'' (8 KB) -- one bulk copy from the workspace --
+  // then P (8 KB).  MMA A operands take 128 rows starting at T' or T''.
+  uint8_t tpp[2][3][8192];
+  uint8_t wq[NP][16384];       // [W rows 0..63][e^G Q rows 64..127]
+  uint8_t hm[DK * 128];        // bf16 state slab, row i = key index
+  uint8_t vp[8192];            // V'
+  uint8_t vpd[8192];           // V' scaled by e^{G_63 - G_s}
+  float G[C];
+  uint64_t bar_tma[2];
+  uint64_t bar_mma;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int DK>
+__global__ void __launch_bounds__(NTHREADS, 1)
+chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+                 const float* __restrict__ eta, float eps, const float* __restrict__ h0,
+                 __nv_bfloat16* __restrict__ o, float* __restrict__ hT, int T, int H, int DV,
+                 const uint8_t* __restrict__ ws, unsigned int* err) {
+  using Smem = ChunkSmem<DK>;
+  constexpr int NP = Smem::NP;
+  extern __shared__ uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                     ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int slab = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
+  const int nchunks = (T + C - 1) / C;
+  const size_t head = (size_t)b * H + hh;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+
+  if (warp == 0) {
+    ptx::tmem_alloc(&s.tmem_base, TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  if (tid == 0) {
+    ptx::mbar_init(&s.bar_tma[0], 1);
+    ptx::mbar_init(&s.bar_tma[1], 1);
+    ptx::mbar_init(&s.bar_mma, 1);
+    ptx::mbar_init_fence();
+    ptx::prefetch_tensormap(&tm_q);
+    ptx::prefetch_tensormap(&tm_k);
+    ptx::prefetch_tensormap(&tm_v);
+    s.abort_flag = 0;
+  }
+
+  // fp32 state slab: thread i < DK owns row i (64 columns) for the whole run.
+  float hreg[BV];
+  if (tid < DK) {
+    if (h0) {
+      const float4* src = reinterpret_cast<const float4*>(h0 + (head * DK + tid) * DV + slab * BV);
+#pragma unroll
+      for (int j = 0; j < BV / 4; ++j) {
+        float4 x = src[j];
+        hreg[4 * j] = x.x; hreg[4 * j + 1] = x.y; hreg[4 * j + 2] = x.z; hreg[4 * j + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < BV; ++j) hreg[j] = 0.f;
+    }
+    sw128_store_row(s.hm, tid, hreg);
+  }
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tb = s.tmem_base;
+
+  constexpr uint32_t TMA_BYTES = (uint32_t)(2 * NP * 8192 + 8192 + kUtTileBytes);
+  const uint8_t* ws_head = ws + head * (size_t)nchunks * kUtTileBytes;
+  auto issue_tma = [&](int n, int buf) {
+    ptx::mbar_arrive_expect_tx(&s.bar_tma[buf], TMA_BYTES);
+    ptx::bulk_load(s.tpp[buf][0], ws_head + (size_t)n * kUtTileBytes, (uint32_t)kUtTileBytes,
+                   &s.bar_tma[buf]);
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      ptx::tma_load_4d(s.kq[buf][p], &tm_k, &s.bar_tma[buf], p * 64, hh, n * C, b);
+      ptx::tma_load_4d(s.kq[buf][p] + 8192, &tm_q, &s.bar_tma[buf], p * 64, hh, n * C, b);
+    }
+    ptx::tma_load_4d(s.v[buf], &tm_v, &s.bar_tma[buf], slab * BV, hh, n * C, b);
+  };
+  int tma_issued = 0;    // chunks whose loads were issued (meaningful on tid 0)
+  int tma_consumed = 0;  // chunks whose loads were waited for
+  if (tid == 0 && nchunks > 0) {
+    issue_tma(0, 0);
+    tma_issued = 1;
+  }
+
+  uint32_t mma_phase = 0;
+  bool ok = true;
+  // All threads wait on the same barrier; a timeout anywhere aborts all.
+  auto sync_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (!wait_bounded(bar, parity)) atomicExch(&s.abort_flag, 1);
+    __syncthreads();
+    return s.abort_flag == 0;
+  };
+  auto mma_wait = [&]() -> bool {
+    bool r = sync_wait(&s.bar_mma, mma_phase);
+    mma_phase ^= 1u;
+    ptx::tc_fence_after();
+    return r;
+  };
+
+#pragma unroll 1
+  for (int n = 0; n < nchunks && ok; ++n) {
+    const int buf = n & 1;
+    if (!sync_wait(&s.bar_tma[buf], (uint32_t)((n >> 1) & 1))) { ok = false; break; }
+    tma_consumed = n + 1;
+    if (tid == 0 && n + 1 < nchunks) {
+      issue_tma(n + 1, buf ^ 1);
+      tma_issued = n + 2;
+    }
+    const int t0 = n * C;
+
+    // ---- prologue: chunk-local inclusive cumsum G_r (threads 0..63)
+    if (tid < C) {
+      const int t = t0 + tid;
+      float gr = 0.f;
+      if (t < T) gr = g[((size_t)b * T + t) * H + hh];
+      float x = gr;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        float y = __shfl_up_sync(0xffffffffu, x, off);
+        if ((tid & 31) >= off) x += y;
+      }
+      s.G[tid] = x;
+    }
+    __syncthreads();
+    if (tid >= 32 && tid < C) s.G[tid] += s.G[31];
+    __syncthreads();
+
+    // ---- MMA 1: D_S = [K; Q] . K^T
+    if (tid == 0) {
+      ptx::tc_fence_after();
+      constexpr uint32_t id = ptx::idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+      for (int kk = 0; kk < DK / 16; ++kk) {
+        const uint32_t a = ptx::smem_u32(s.kq[buf][kk >> 2]) + (kk & 3) * 32;
+        ptx::mma_bf16(tb + COL_S, ptx::sdesc_sw128(a, 16, 1024), ptx::sdesc_sw128(a, 16, 1024),
+                      id, kk > 0);
+      }
+      ptx::mma_commit(&s.bar_mma);
+    }
+    if (!mma_wait()) { ok = false; break; }
+
+    // ---- P (rows 64..127, bf16 operand); rows 0..63 of D_S are unused
+    uint8_t* tp1 = s.tpp[buf][0];
+    uint8_t* tp2 = s.tpp[buf][1];
+    if (tid >= C) {
+      float srow[64];
+      ptx::tmem_ld32(tb + lane_base + COL_S, srow);
+      ptx::tmem_ld32(tb + lane_base + COL_S + 32, srow + 32);
+      const int r = tid - C;
+      const float Gr = s.G[r];
+#pragma unroll
+      for (int c = 0; c < C; ++c) srow[c] = (c <= r) ? srow[c] * __expf(Gr - s.G[c]) : 0.f;
+      sw128_store_row(s.tpp[buf][2], r, srow);
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+
+    // ---- MMA 2: D_W = [T''; P] . K ;  MMA 3: D_U = [T'; T''] . V
+    if (tid == 0) {
+      ptx::tc_fence_after();
+      constexpr uint32_t idw = ptx::idesc_bf16(128, DK, 0, 1);
+      constexpr uint32_t idu = ptx::idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk) {
+        const uint32_t a = ptx::smem_u32(tp2) + kk * 32;
+        const uint32_t bk = ptx::smem_u32(s.kq[buf][0]) + kk * 2048;
+        ptx::mma_bf16(tb + COL_W, ptx::sdesc_sw128(a, 16, 1024), ptx::sdesc_sw128(bk, 16384, 1024),
+                      idw, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk) {
+        const uint32_t a = ptx::smem_u32(tp1) + kk * 32;
+        const uint32_t bv = ptx::smem_u32(s.v[buf]) + kk * 2048;
+        ptx::mma_bf16(tb + COL_U, ptx::sdesc_sw128(a, 16, 1024), ptx::sdesc_sw128(bv, 1024, 1024),
+                      idu, kk > 0);
+      }
+      ptx::mma_commit(&s.bar_mma);
+    }
+    if (!mma_wait()) { ok = false; break; }
+
+    // ---- W rows -> wq rows 0..63; e^{G_r} q_r -> wq rows 64..127
+    if (tid < C) {
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        float w[64];
+        ptx::tmem_ld32(tb + lane_base + COL_W + p * 64, w);
+        ptx::tmem_ld32(tb + lane_base + COL_W + p * 64 + 32, w + 32);
+        sw128_store_row(s.wq[p], tid, w);
+      }
+    } else {
+      const int r = tid - C;
+      const float sc = __expf(s.G[r]);
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t off = 8192 + sw128_chunk_off(r, c);
+          float x[8];
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(s.kq[buf][p] + off), x);
+          uint4 u;
+          u.x = pack_bf16x2(x[0] * sc, x[1] * sc);
+          u.y = pack_bf16x2(x[2] * sc, x[3] * sc);
+          u.z = pack_bf16x2(x[4] * sc, x[5] * sc);
+          u.w = pack_bf16x2(x[6] * sc, x[7] * sc);
+          *reinterpret_cast<uint4*>(s.wq[p] + off) = u;
+        }
+      }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+
+    // ---- MMA 4: D_1 = [W; e^G Q] . h
+    if (tid == 0) {
+      ptx::tc_fence_after();
+      constexpr uint32_t id = ptx::idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+      for (int kk = 0; kk < DK / 16; ++kk) {
+        const uint32_t a = ptx::smem_u32(s.wq[kk >> 2]) + (kk & 3) * 32;
+        const uint32_t bh = ptx::smem_u32(s.hm) + kk * 2048;
+        ptx::mma_bf16(tb + COL_1, ptx::sdesc_sw128(a, 16, 1024), ptx::sdesc_sw128(bh, 1024, 1024),
+                      id, kk > 0);
+      }
+      ptx::mma_commit(&s.bar_mma);
+    }
+    if (!mma_wait()) { ok = false; break; }
+
+    // ---- V' = U - W h (rows 0..63), and its decayed copy for the state
+    if (tid < C) {
+      float u[64], wh[64];
+      ptx::tmem_ld32(tb + lane_base + COL_U, u);
+      ptx::tmem_ld32(tb + lane_base + COL_U + 32, u + 32);
+      ptx::tmem_ld32(tb + lane_base + COL_1, wh);
+      ptx::tmem_ld32(tb + lane_base + COL_1 + 32, wh + 32);
+#pragma unroll
+      for (int j = 0; j < 64; ++j) u[j] -= wh[j];
+      sw128_store_row(s.vp, tid, u);
+      const float dec = __expf(s.G[C - 1] - s.G[tid]);
+#pragma unroll
+      for (int j = 0; j < 64; ++j) u[j] *= dec;
+      sw128_store_row(s.vpd, tid, u);
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+
+    // ---- MMA 5: D_H = K^T . (decay V') ;  MMA 6: D_1 += [T''; P] . V'
+    if (tid == 0) {
+      ptx::tc_fence_after();
+      constexpr uint32_t idh = ptx::idesc_bf16(128, 64, 1, 1);
+      constexpr uint32_t ido = ptx::idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk) {
+        const uint32_t a = ptx::smem_u32(s.kq[buf][0]) + kk * 2048;
+        const uint32_t bv = ptx::smem_u32(s.vpd) + kk * 2048;
+        ptx::mma_bf16(tb + COL_H, ptx::sdesc_sw128(a, 16384, 1024), ptx::sdesc_sw128(bv, 1024, 1024),
+                      idh, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk) {
+        const uint32_t a = ptx::smem_u32(tp2) + kk * 32;
+        const uint32_t bv = ptx::smem_u32(s.vp) + kk * 2048;
+        ptx::mma_bf16(tb + COL_1, ptx::sdesc_sw128(a, 16, 1024), ptx::sdesc_sw128(bv, 1024, 1024),
+                      ido, 1);
+      }
+      ptx::mma_commit(&s.bar_mma);
+    }
+    if (!mma_wait()) { ok = false; break; }
+
+    // ---- state update (rows < DK) and output rows (lanes 64..127)
+    const float gC = __expf(s.G[C - 1]);
+    if (tid < DK) {
+      float dh[64];
+      ptx::tmem_ld32(tb + lane_base + COL_H, dh);
+      ptx::tmem_ld32(tb + lane_base + COL_H + 32, dh + 32);
+#pragma unroll
+      for (int j = 0; j < BV; ++j) hreg[j] = fmaf(gC, hreg[j], dh[j]);
+      sw128_store_row(s.hm, tid, hreg);
+    }
+    if (tid >= C) {
+      const int r = tid - C, t = t0 + r;
+      float ov[64];
+      ptx::tmem_ld32(tb + lane_base + COL_1, ov);
+      ptx::tmem_ld32(tb + lane_base + COL_1 + 32, ov + 32);
+      if (t < T) {
+        uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * T + t) * H + hh) * DV + slab * BV);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 u;
+          u.x = pack_bf16x2(ov[8 * c + 0], ov[8 * c + 1]);
+          u.y = pack_bf16x2(ov[8 * c + 2], ov[8 * c + 3]);
+          u.z = pack_bf16x2(ov[8 * c + 4], ov[8 * c + 5]);
+          u.w = pack_bf16x2(ov[8 * c + 6], ov[8 * c + 7]);
+          dst[c] = u;
+        }
+      }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
+
+  if (ok) {
+    if (hT && tid < DK) {
+      float4* dst = reinterpret_cast<float4*>(hT + (head * DK + tid) * DV + slab * BV);
+#pragma unroll
+      for (int j = 0; j < BV / 4; ++j)
+        dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
+    }
+  } else if (tid == 0) {
+    report_timeout(err);
+    // drain this CTA's own TMA loads still in flight (bounded), so no copy
+    // lands in shared memory after the CTA has gone
+    for (int n = tma_consumed; n < tma_issued; ++n) {
+      if (!wait_bounded(&s.bar_tma[n & 1], (uint32_t)((n >> 1) & 1))) break;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tb, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  }
+  return fn;
+}
+
+// [B][T][H][d] bf16 tensor, boxes of 64 (d) x 64 (t) for one (b, h).
+bool make_map(CUtensorMap* m, const void* base, int d, int H, int T, int B) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DK>
+cudaError_t launch_dk(const void* q, const void* k, const void* v, const float* g,
+                      const float* eta, float eps, const float* h0, void* o, float* hT, int B,
+                      int T, int H, int DV, uint8_t* ws, unsigned int* err, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, DK, H, T, B) || !make_map(&mk, k, DK, H, T, B) ||
+      !make_map(&mv, v, DV, H, T, B))
+    return cudaErrorInvalidValue;
+  cudaError_t eu = launch_ut(mk, g, eta, eps, ws, B, T, H, DK, err, st);
+  if (eu != cudaSuccess) return eu;
+  const size_t smem = sizeof(ChunkSmem<DK>) + 1024;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<DK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid(DV / BV, H, B);
+  chunk_fwd_kernel<DK><<<grid, NTHREADS, smem, st>>>(mq, mk, mv, g, eta, eps, h0,
+                                                     (__nv_bfloat16*)o, hT, T, H, DV, ws, err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
+  if (dtype != KLA_BF16 || B < 1 || H < 1 || T < 1 || dk != dv) return 0;
+  return (size_t)B * H * ((T + C - 1) / C) * kUtTileBytes;
+}
+
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
+                            const float* eta, float eps, const float* h0, void* o, float* hT,
+                            int B, int T, int H, int dk, int dv, void* workspace,
+                            unsigned int* err, cudaStream_t st) {
+  if (dk != dv) return cudaErrorNotSupported;
+  uint8_t* ws = (uint8_t*)workspace;
+  if (dk == 128) return launch_dk<128>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dv, ws, err, st);
+  if (dk == 64) return launch_dk<64>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dv, ws, err, st);
   return cudaErrorNotSupported;
 }
 

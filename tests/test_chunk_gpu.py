@@ -1,0 +1,115 @@
+"""tcgen05 chunkwise prefill (kla_chunk_fwd, bf16) against the fp64 oracle.
+
+Small shapes are compared element by element over the whole output; the
+full-size workloads run in the same launch configuration the benchmark times
+and are compared on sampled heads (each head is an independent recurrence,
+so the oracle can evaluate a few heads on their own)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from delta_rule_linear_kla_b200 import api, inputs
+
+from helpers import cuda, rel, worst_head_rel
+
+pytestmark = pytest.mark.gpu
+W = inputs.WORKLOADS
+TOL = 1e-2
+
+
+def _run(w, with_h0=None):
+    x = inputs.make_prefill(w, with_h0=with_h0)
+    xc = cuda(x)
+    o, hT = api.chunk_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"], xc["h0"])
+    api.check_device_error()
+    return x, o.cpu(), hT.cpu()
+
+
+def _full_check(w, with_h0=None):
+    x, o, hT = _run(w, with_h0)
+    o_ref, h_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"])
+    eo, eh = rel(o, o_ref), rel(hT, h_ref)
+    assert np.isfinite(oracle.f64(o)).all() and np.isfinite(oracle.f64(hT)).all()
+    assert eo < TOL and eh < TOL, (w, eo, eh, worst_head_rel(o, o_ref))
+
+
+@pytest.mark.parametrize("T", [1, 17, 64, 65, 130, 256])
+def test_layer_shapes_d128(T):
+    _full_check(W["prefill_4k"].scaled(B=2, T=T, H=2))
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 200])
+def test_with_initial_state_d128(T):
+    _full_check(W["prefill_4k"].scaled(B=1, T=T, H=3, seed=7), with_h0=True)
+
+
+@pytest.mark.parametrize("T", [1, 64, 129, 300])
+def test_stress_shapes_d64(T):
+    _full_check(W["stress"].scaled(B=2, T=T, H=3))
+
+
+def test_long_gates_small():
+    _full_check(W["prefill_65k"].scaled(T=700, H=2))
+
+
+def test_final_state_only_and_alias():
+    w = W["stress"].scaled(B=1, T=150, H=2)
+    x = inputs.make_prefill(w)
+    xc = cuda(x)
+    h = xc["h0"].clone()
+    o, hT = api.chunk_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"], h, hT=h)
+    torch.cuda.synchronize()
+    assert hT.data_ptr() == h.data_ptr()
+    _, h_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"])
+    assert rel(h, h_ref) < TOL
+    o2, none = api.chunk_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"],
+                             xc["h0"], return_state=False)
+    torch.cuda.synchronize()
+    assert none is None and torch.equal(o2, o)
+
+
+def test_deterministic():
+    w = W["prefill_4k"].scaled(B=1, T=300, H=2)
+    _, o1, h1 = _run(w)
+    _, o2, h2 = _run(w)
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+def _sampled(w, heads, with_h0=None):
+    """Full-size launch; oracle on the listed (b, h) heads only."""
+    x, o, hT = _run(w, with_h0)
+    errs = []
+    for (b, h) in heads:
+        sl = lambda t: t[b:b + 1, :, h:h + 1]
+        h0 = None if x["h0"] is None else x["h0"][b:b + 1, h:h + 1]
+        o_ref, h_ref = oracle.forward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]),
+                                      sl(x["eta"]), x["eps"], h0)
+        eo = rel(o[b:b + 1, :, h:h + 1], o_ref)
+        eh = rel(hT[b:b + 1, h:h + 1], h_ref)
+        errs.append((b, h, eo, eh))
+    assert all(e[2] < TOL and e[3] < TOL for e in errs), errs
+    return errs
+
+
+def test_full_size_layer_4k_sampled():
+    _sampled(W["prefill_4k"], [(0, 0), (3, 5), (7, 7)])
+
+
+def test_full_size_stress_sampled():
+    _sampled(W["stress"], [(0, 0), (1, 17), (3, 31)])
+
+
+def test_full_size_long_65k_sampled():
+    _sampled(W["prefill_65k"], [(0, 3), (0, 15)])
+
+
+def test_matches_token_serial_all_heads_4k():
+    """Property at full size over every head: the chunkwise kernel and the
+    token-serial kernel evaluate the same recurrence."""
+    w = W["prefill_4k"]
+    x = cuda(inputs.make_prefill(w))
+    o1, h1 = api.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"])
+    o2, h2 = api.recurrent_fwd(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"])
+    torch.cuda.synchronize()
+    assert rel(o1, o2) < TOL and rel(h1, h2) < TOL
