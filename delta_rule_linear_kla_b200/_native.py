@@ -22,6 +22,8 @@ SIGNATURES = {
                                _i, _i, _i, _i, _i, _i, _vp]),
     "kla_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp,
                              _i, _i, _i, _i, _i, _vp]),
+    "kla_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
+                                   _i, _i, _i, _i, _i, _i, _vp]),
     "kla_check_device_error": (_i, [_vp]),
     "kla_status_string": (ctypes.c_char_p, [_i]),
     "kla_version": (_i, []),

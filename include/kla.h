@@ -117,6 +117,37 @@ KLA_API kla_status kla_decode_step(const void *q, const void *k, const void *v,
                            int dtype, void *stream);
 
 /*
+ * Chunkwise prefill without any caller-provided device memory.
+ *
+ * No counterpart in the paper: this is a deployment convenience.  Some
+ * callers cannot hand the library scratch memory -- their device memory
+ * belongs to another allocator (e.g. a serving process's pre-reserved pool)
+ * or they may not allocate after start-up -- so this call runs
+ * kla_chunk_fwd (same arguments and layouts, chunk = KLA_CHUNK, dtype
+ * KLA_BF16 or KLA_FP32) with a fixed scratch array compiled into libkla.so
+ * instead of a workspace.  It allocates nothing itself.
+ *
+ *   Limit: B * H * ceil(T / KLA_CHUNK) <= KLA_NOALLOC_MAX_CHUNKS, else
+ *          KLA_ERR_UNSUPPORTED (checked before any CUDA call).
+ *   Memory: every GPU that loads libkla.so holds KLA_NOALLOC_SCRATCH_BYTES
+ *          for the life of the process.
+ *   First call on a device looks up the array's device address
+ *          (cudaGetSymbolAddress); make that first call before any stream
+ *          capture.
+ *   All calls share the one array, which keeps the previous call's contents
+ *          (nothing in it needs to start at zero).  Calls whose work overlaps
+ *          on the GPU (several streams or host threads at once) race on it:
+ *          issue them one after another.
+ */
+#define KLA_NOALLOC_MAX_CHUNKS 1024
+#define KLA_NOALLOC_SCRATCH_BYTES (KLA_NOALLOC_MAX_CHUNKS * 16384)
+KLA_API kla_status kla_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                 const float *g, const float *eta, float eps,
+                                 const float *h0, void *o, float *hT,
+                                 int B, int T, int H, int dk, int dv, int dtype,
+                                 void *stream);
+
+/*
  * Reads and clears the library's device error word for the current device
  * after synchronising `stream`.  Kernels set it instead of hanging when a
  * bounded wait on an mbarrier runs out (KLA_ERR_TIMEOUT).  Returns KLA_OK
