@@ -11,12 +11,11 @@
 // "Kaczmarz Linear Attention", Abstract):
 //
 //   G_r = sum_{j<=r} g_j  (in chunk)
-//   P  = lower_incl(Q K^T (*) e^{G_r - G_s})                          [MMA 1]
-//   W  = T'' K,  U = T' V                                             [MMA 2,3]
-//   X  = [W; Q] h          (rows 0..63: W h, rows 64..127: Q h)       [MMA 4]
-//   V' = U - W h
-//   h <- e^{G_63} h + K^T diag(e^{G_63 - G_s}) V'                      [MMA 5]
-//   O  = diag(e^G) Q h + P V'                                         [MMA 6]
+//   P  = lower_incl(Q K^T (*) e^{G_r - G_s})                        [MMA 1]
+//   W  = T'' K,  U = T' V                                           [MMA 2, 3]
+//   V' = U - W h  (and -Q h)  accumulated onto U in TMEM            [MMA 4]
+//   h <- e^{G_63} h + K^T diag(e^{G_63 - G_s}) V'                    [MMA 5]
+//   O  = diag(e^G) Q h + P V'                                       [MMA 6]
 //
 // The decay ratios are only formed as masked differences of G (never
 // K / Gamma), so strong gates cannot overflow.  A ragged tail is zero-filled
@@ -25,27 +24,34 @@
 // All contractions are single-CTA tcgen05.mma with M = 128, bf16 operands in
 // 128-byte swizzled shared-memory panels and fp32 accumulators in TMEM (lane
 // = row; 64-row products are stacked or padded to 128 lanes):
-//   MMA 1  D_S [128x64]  = [W_stale; Q] . K^T   A, B K-major  (lanes 64..127)
-//   MMA 2  D_W [128xDK]  = [T''; P] . K          B MN-major    (lanes 0..63)
-//   MMA 3  D_U [128x64]  = [T'; T''] . V         B MN-major    (lanes 0..63)
-//   MMA 4  D_X [128x64]  = [W; Q] . h            B MN-major
-//   MMA 5  D_H [128x64]  = K^T . (decay V')      A, B MN-major (lanes < DK)
-//   MMA 6  D_PV[128x64]  = [T''; P] . V'         B MN-major    (lanes 64..127)
+//   MMA 1  D_S [128x64]   = [W_stale; Q] . K^T   A, B K-major (lanes 64..127)
+//   MMA 2  D_W [128xDK]   = [T''; P] . K          B MN-major   (lanes 0..63)
+//   MMA 3  D_U [128x64]   = [T'; 0] . V           B MN-major
+//   MMA 4  D_U           += -[W; Q] . h           B MN-major   (negated A)
+//          -> lanes 0..63 hold V' = U - W h, lanes 64..127 hold -Q h
+//   MMA 5  D_H [128x64]   = K^T . (decay V')      A, B MN-major (lanes < DK)
+//   MMA 6  D_PV[128x64]   = [T''; P] . V'         B MN-major   (lanes 64..127)
 //
-// Warp roles (320 threads), synchronised only through mbarriers:
+// Warp roles (448 threads), synchronised only through mbarriers:
 //   warp 0      TMA producer: K, Q, V slab and the UT tiles of chunk n into
 //               stage n % 2 (double buffered).
-//   warp 1      MMA issuer (one thread).  Per iteration n it issues the chain
-//               MMAs of chunk n (4, then 5 and 6) interleaved with the
-//               state-independent MMAs of chunk n + 1 (1, then 2 and 3), so
-//               the tensor pipe works on chunk n + 1 while the chain warps
-//               run chunk n's epilogues.
-//   warps 2..5  "next-chunk" epilogues: the gate cumsum G, P (lanes 64..127)
-//               and W (lanes 0..63), written into the stage's P and W slots.
-//   warps 6..9  "chain" epilogues: V' (lanes 0..63), the state update (lanes
-//               < DK) and the output rows (lanes 64..127).
+//   warp 1      MMA issuer: the warp runs the schedule uniformly and one
+//               elected lane issues.  Per iteration n: MMA 4 of chunk n, then
+//               MMAs 2 and 1 of chunk n + 1 (they run while the chain warps
+//               form V'(n)), MMAs 5, 6 of chunk n, then MMA 3 of chunk n + 1
+//               (it runs while the state is updated).  The tensor pipe
+//               executes in issue order, so this keeps the chain's MMAs from
+//               queueing behind state-independent work.
+//   warps 2, 3, 14, 15  P of the next chunk (TMEM lanes 64..127) into the
+//               stage's P slot; warp 2 also computes the gate cumsum.
+//   warps 4, 5  W of the next chunk (TMEM lanes 0..63) into the W slot.
+//   warps 6..13 "chain" epilogues, split by state columns (warps 6..9 take
+//               columns 0..31, warps 10..13 columns 32..63): V' (lanes
+//               0..63), the state update (lanes < DK) and the output rows
+//               (lanes 64..127).
 // Every wait is bounded (about 2 s); on timeout the kernel raises the device
-// error word, stops all roles, drains its own TMA loads and frees TMEM.
+// error word, stops all roles, drains its own TMA loads and MMAs and frees
+// TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -60,21 +66,21 @@ namespace {
 
 constexpr int C = 64;       // chunk length
 constexpr int BV = 64;      // state columns per CTA
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 512;
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM column offsets of the accumulators
-constexpr uint32_t COL_S = 0, COL_W = 64, COL_U = 192 /* 2 buffers */, COL_X = 320,
+constexpr uint32_t COL_S = 0 /* 2 buffers */, COL_W = 128, COL_U = 256 /* 2 buffers */,
                    COL_H = 384, COL_PV = 448;
 
 // One pipeline stage.  Per 64-column key panel: [W rows | Q rows | K rows]
 // (8 KB each), so [W; Q] is one 128-row K-major operand.  Then the V slab and
-// [T' | T'' | P]: MMA A operands take 128 rows starting at T' or T''.
+// [T' | 0 | T'' | P]: 128-row MMA A operands [T'; 0] and [T''; P].
 template <int DK>
 struct alignas(1024) Stage {
   static constexpr int NP = DK / 64;
   uint8_t panel[NP][3][8192];
   uint8_t v[8192];
-  uint8_t tp[3][8192];
+  uint8_t tp[4][8192];
 };
 
 template <int DK>
@@ -82,12 +88,13 @@ struct alignas(1024) ChainSmem {
   Stage<DK> st[2];
   uint8_t hm[DK * 128];  // bf16 state slab (MMA 4 operand), row i = key index
   uint8_t vp[8192];      // V'
-  uint8_t vpd[8192];     // V' scaled by e^{G_63 - G_s}
+  uint8_t vpd[8192];     // V' scaled by e^{G_63 - G_s} (MMA 5 operand)
   float G[3][C];         // gate cumsum of chunk n in slot n % 3
+  alignas(16) float alpha[3][C];  // e^{g_s} of chunk n in slot n % 3
   uint64_t full[2], empty[2];
-  uint64_t bS, bWU, bX, bHP;             // MMA completions
-  uint64_t p_done, w_done, vp_ready;     // epilogue -> MMA
-  uint64_t u_free[2], x_free, h_done, pv_free;
+  uint64_t bS[2], bW, bX, bHP;           // MMA completions (bS per D_S buffer)
+  uint64_t p_done[2], w_done, vp_ready;  // epilogue -> MMA (p_done per D_S buffer)
+  uint64_t u_free[2], h_done, pv_free;
   uint64_t g_ready[3];
   uint64_t mma_drain;
   uint32_t tmem_base;
@@ -95,10 +102,12 @@ struct alignas(1024) ChainSmem {
 };
 
 enum Slot { SW = 0, SQ = 1, SK = 2 };
+enum TSlot { TP1 = 0, TZ = 1, TP2 = 2, TP = 3 };
 
 // Bounded wait that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag) {
+  if (ptx::mbar_test_wait(bar, parity)) return true;
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
@@ -117,9 +126,9 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(ptx::smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
+// Descriptor advance: the start address lives in the low bits, in 16-byte
+// units; a K step is 32 B (K-major) or 2048 B (MN-major).
+constexpr uint64_t KSTEP_K = 2, KSTEP_MN = 128;
 
 template <int DK>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -151,23 +160,26 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&s.full[i], 1);
       ptx::mbar_init(&s.empty[i], 1);
-      ptx::mbar_init(&s.u_free[i], 2);
+      ptx::mbar_init(&s.u_free[i], 8);
+      ptx::mbar_init(&s.bS[i], 1);
+      ptx::mbar_init(&s.p_done[i], 4);
     }
-    ptx::mbar_init(&s.bS, 1);
-    ptx::mbar_init(&s.bWU, 1);
+    for (int i = 0; i < 3; ++i) ptx::mbar_init(&s.g_ready[i], 1);
+    ptx::mbar_init(&s.bW, 1);
     ptx::mbar_init(&s.bX, 1);
     ptx::mbar_init(&s.bHP, 1);
-    ptx::mbar_init(&s.p_done, 2);
     ptx::mbar_init(&s.w_done, 2);
-    ptx::mbar_init(&s.vp_ready, 2);
-    ptx::mbar_init(&s.x_free, 4);
-    ptx::mbar_init(&s.h_done, 4);
-    ptx::mbar_init(&s.pv_free, 2);
-    for (int i = 0; i < 3; ++i) ptx::mbar_init(&s.g_ready[i], 2);
+    ptx::mbar_init(&s.vp_ready, 4);
+    ptx::mbar_init(&s.h_done, 8);
+    ptx::mbar_init(&s.pv_free, 4);
     ptx::mbar_init(&s.mma_drain, 1);
     ptx::mbar_init_fence();
     s.abort_flag = 0;
   }
+  // the zero blocks of both stages ([T'; 0] operand of MMA 3)
+  for (int i = tid; i < 2 * 8192 / 16; i += NTHREADS)
+    reinterpret_cast<uint4*>(s.st[i / 512].tp[TZ])[i % 512] = make_uint4(0, 0, 0, 0);
+  ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -189,9 +201,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           drained = n - 1;  // chunks up to n-2 fully consumed
         }
         Stage<DK>& S = s.st[st];
+        const uint8_t* src = ws_head + (size_t)n * kUtTileBytes;
         ptx::mbar_arrive_expect_tx(&s.full[st], BYTES);
-        ptx::bulk_load(S.tp[0], ws_head + (size_t)n * kUtTileBytes, (uint32_t)kUtTileBytes,
-                       &s.full[st]);
+        ptx::bulk_load(S.tp[TP1], src, 8192, &s.full[st]);
+        ptx::bulk_load(S.tp[TP2], src + 8192, 8192, &s.full[st]);
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
           ptx::tma_load_4d(S.panel[p][SK], &tm_k, &s.full[st], p * 64, hh, n * C, b);
@@ -199,6 +212,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
         ptx::tma_load_4d(S.v, &tm_v, &s.full[st], slab * BV, hh, n * C, b);
         issued = n + 1;
+        if (n + 2 < nchunks) {  // warm L2 two chunks ahead of the loads
+          const int m = n + 2;
+          ptx::bulk_prefetch_l2(ws_head + (size_t)m * kUtTileBytes, (uint32_t)kUtTileBytes);
+#pragma unroll
+          for (int p = 0; p < NP; ++p) {
+            ptx::tma_prefetch_l2_4d(&tm_k, p * 64, hh, m * C, b);
+            ptx::tma_prefetch_l2_4d(&tm_q, p * 64, hh, m * C, b);
+          }
+          ptx::tma_prefetch_l2_4d(&tm_v, slab * BV, hh, m * C, b);
+        }
       }
       if (*abort_flag) {
         // let this CTA's own copies land before the CTA goes away
@@ -208,271 +231,311 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
   } else if (warp == 1) {
     // ============================ MMA issuer ============================
-    if (lane == 0) {
-      constexpr uint32_t id_s = ptx::idesc_bf16(128, 64, 0, 0);
-      constexpr uint32_t id_w = ptx::idesc_bf16(128, DK, 0, 1);
-      constexpr uint32_t id_64 = ptx::idesc_bf16(128, 64, 0, 1);
-      constexpr uint32_t id_h = ptx::idesc_bf16(128, 64, 1, 1);
-      auto mma1 = [&](int n) {  // D_S = [W_stale; Q] K^T
-        Stage<DK>& S = s.st[n & 1];
+    constexpr uint32_t id_s = ptx::idesc_bf16(128, 64, 0, 0);
+    constexpr uint32_t id_w = ptx::idesc_bf16(128, DK, 0, 1);
+    constexpr uint32_t id_64 = ptx::idesc_bf16(128, 64, 0, 1);
+    constexpr uint32_t id_x = ptx::idesc_bf16(128, 64, 0, 1, /*neg_a=*/1);
+    constexpr uint32_t id_h = ptx::idesc_bf16(128, 64, 1, 1);
+    // descriptors of stage 0 / panel 0 (uniform across the warp); other
+    // stages and panels are fixed offsets in 16-byte units
+    constexpr uint64_t STG = sizeof(Stage<DK>) >> 4, PNL = PANEL >> 4;
+    const uint64_t dWQ = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SW]), 16, 1024);
+    const uint64_t dKk = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SK]), 16, 1024);
+    const uint64_t dKmn = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SK]), PANEL, 1024);
+    const uint64_t dT1 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP1]), 16, 1024);
+    const uint64_t dT2 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP2]), 16, 1024);
+    const uint64_t dV = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].v), 1024, 1024);
+    const uint64_t dH = ptx::sdesc_sw128(ptx::smem_u32(s.hm), 1024, 1024);
+    const uint64_t dVP = ptx::sdesc_sw128(ptx::smem_u32(s.vp), 1024, 1024);
+    const uint64_t dVPD = ptx::sdesc_sw128(ptx::smem_u32(s.vpd), 1024, 1024);
+
+    auto mma2 = [&](int n) {  // D_W = [T''; P_stale] K  (W in lanes 0..63)
+      const uint64_t so = (uint64_t)(n & 1) * STG;
+      if (ptx::elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) {
-          const uint32_t a = ptx::smem_u32(S.panel[kk >> 2][SW]) + (kk & 3) * 32;
-          const uint32_t bk = ptx::smem_u32(S.panel[kk >> 2][SK]) + (kk & 3) * 32;
-          ptx::mma_bf16(tb + COL_S, ptx::sdesc_sw128(a, 16, 1024), ptx::sdesc_sw128(bk, 16, 1024),
-                        id_s, kk > 0);
-        }
-        ptx::mma_commit(&s.bS);
-      };
-      auto mma23 = [&](int n) {  // D_W = [T''; P] K ;  D_U[n%2] = [T'; T''] V
-        Stage<DK>& S = s.st[n & 1];
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          const uint32_t a = ptx::smem_u32(S.tp[1]) + kk * 32;
-          const uint32_t bk = ptx::smem_u32(S.panel[0][SK]) + kk * 2048;
-          ptx::mma_bf16(tb + COL_W, ptx::sdesc_sw128(a, 16, 1024),
-                        ptx::sdesc_sw128(bk, PANEL, 1024), id_w, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          const uint32_t a = ptx::smem_u32(S.tp[0]) + kk * 32;
-          const uint32_t bv = ptx::smem_u32(S.v) + kk * 2048;
-          ptx::mma_bf16(tb + COL_U + 64 * (n & 1), ptx::sdesc_sw128(a, 16, 1024),
-                        ptx::sdesc_sw128(bv, 1024, 1024), id_64, kk > 0);
-        }
-        ptx::mma_commit(&s.bWU);
-      };
-      bool ok = nchunks > 0;
-      if (ok) ok = wait_or_abort(&s.full[0], 0, abort_flag);
-      if (ok) {
-        ptx::tc_fence_after();
-        mma1(0);
-        mma23(0);
+        for (int kk = 0; kk < C / 16; ++kk)
+          ptx::mma_bf16(tb + COL_W, dT2 + so + kk * KSTEP_K, dKmn + so + kk * KSTEP_MN, id_w,
+                        kk > 0);
+        ptx::mma_commit(&s.bW);
       }
-      for (int n = 0; n < nchunks && ok; ++n) {
-        Stage<DK>& S = s.st[n & 1];
-        const uint32_t par = (uint32_t)(n & 1);
-        // ---- MMA 4 (chunk n): needs W(n), h_n, and D_X free
-        if (!wait_or_abort(&s.w_done, par, abort_flag)) break;
-        if (!wait_or_abort(&s.h_done, par, abort_flag)) break;
-        if (n > 0 && !wait_or_abort(&s.x_free, par ^ 1u, abort_flag)) break;
-        ptx::tc_fence_after();
+      __syncwarp();
+    };
+    // D_S[n%2] = [W_stale; Q] K^T in two halves of the key dimension, placed
+    // in the two idle windows of the tensor pipe
+    auto mma1_half = [&](int n, int half) {
+      const uint64_t so = (uint64_t)(n & 1) * STG;
+      constexpr int KS = DK / 16, HS = KS / 2;
+      if (ptx::elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) {
-          const uint32_t a = ptx::smem_u32(S.panel[kk >> 2][SW]) + (kk & 3) * 32;
-          const uint32_t bh = ptx::smem_u32(s.hm) + kk * 2048;
-          ptx::mma_bf16(tb + COL_X, ptx::sdesc_sw128(a, 16, 1024),
-                        ptx::sdesc_sw128(bh, 1024, 1024), id_64, kk > 0);
+        for (int k2 = 0; k2 < HS; ++k2) {
+          const int kk = half * HS + k2;
+          ptx::mma_bf16(tb + COL_S + 64 * (n & 1), dWQ + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K,
+                        dKk + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K, id_s, kk > 0);
         }
-        ptx::mma_commit(&s.bX);
-        // ---- MMA 1 (chunk n+1): needs its data and D_S free (P(n) read)
-        if (!wait_or_abort(&s.p_done, par, abort_flag)) break;
-        if (n + 1 < nchunks) {
-          if (!wait_or_abort(&s.full[(n + 1) & 1], (uint32_t)(((n + 1) >> 1) & 1), abort_flag))
-            break;
-          ptx::tc_fence_after();
-          mma1(n + 1);
-        }
-        // ---- MMA 5, 6 (chunk n): need V'(n), P(n), D_PV free
-        if (!wait_or_abort(&s.vp_ready, par, abort_flag)) break;
-        if (n > 0 && !wait_or_abort(&s.pv_free, par ^ 1u, abort_flag)) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          const uint32_t a = ptx::smem_u32(S.panel[0][SK]) + kk * 2048;
-          const uint32_t bv = ptx::smem_u32(s.vpd) + kk * 2048;
-          ptx::mma_bf16(tb + COL_H, ptx::sdesc_sw128(a, PANEL, 1024),
-                        ptx::sdesc_sw128(bv, 1024, 1024), id_h, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          const uint32_t a = ptx::smem_u32(S.tp[1]) + kk * 32;
-          const uint32_t bv = ptx::smem_u32(s.vp) + kk * 2048;
-          ptx::mma_bf16(tb + COL_PV, ptx::sdesc_sw128(a, 16, 1024),
-                        ptx::sdesc_sw128(bv, 1024, 1024), id_64, kk > 0);
-        }
-        ptx::mma_commit(&s.bHP);
-        ptx::mma_commit(&s.empty[n & 1]);
-        // ---- MMA 2, 3 (chunk n+1): need D_W free (w_done(n) seen above) and
-        //      D_U[(n+1)%2] free (V'(n-1) done)
-        if (n + 1 < nchunks) {
-          if (n >= 1 &&
-              !wait_or_abort(&s.u_free[(n + 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), abort_flag))
-            break;
-          ptx::tc_fence_after();
-          mma23(n + 1);
-        }
+        if (half == 1) ptx::mma_commit(&s.bS[n & 1]);
       }
-      // every MMA this thread issued has finished before TMEM is released
-      ptx::mma_commit(&s.mma_drain);
-      wait_bounded(&s.mma_drain, 0);
+      __syncwarp();
+    };
+    auto mma3 = [&](int n) {  // D_U[n%2] = [T'; 0] V
+      const uint64_t so = (uint64_t)(n & 1) * STG;
+      if (ptx::elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+          ptx::mma_bf16(tb + COL_U + 64 * (n & 1), dT1 + so + kk * KSTEP_K, dV + so + kk * KSTEP_MN,
+                        id_64, kk > 0);
+      }
+      __syncwarp();
+    };
+    bool ok = nchunks > 0;
+    if (ok) ok = wait_or_abort(&s.full[0], 0, abort_flag);
+    if (ok) {
+      ptx::tc_fence_after();
+      mma2(0);
+      mma1_half(0, 0);
+      mma1_half(0, 1);
+      mma3(0);
     }
-  } else if (warp < 6) {
-    // ===================== next-chunk epilogues (P, W) ===================
-    const bool p_rows = row >= 64;  // warps 2, 3
+    for (int n = 0; n < nchunks && ok; ++n) {
+      const int st = n & 1;
+      const uint64_t so = (uint64_t)st * STG;
+      const uint32_t par = (uint32_t)(n & 1);
+      const bool more = n + 1 < nchunks;
+      // ---- MMA 4 (chunk n): needs W(n) and h_n (D_H of n-1 read)
+      if (!wait_or_abort(&s.w_done, par, abort_flag)) break;
+      if (!wait_or_abort(&s.h_done, par, abort_flag)) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk)
+          ptx::mma_bf16(tb + COL_U + 64 * st, dWQ + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K,
+                        dH + kk * KSTEP_MN, id_x, 1);
+        ptx::mma_commit(&s.bX);
+      }
+      __syncwarp();
+      // ---- while V'(n) is formed: W of chunk n+1 (needed by its MMA 4) and
+      //      its Q K^T (so P(n+1) has a whole chunk of slack).  D_W is free
+      //      (W(n) read above) and D_S[(n+1)%2] was read by P(n-1).
+      if (more) {
+        if (!wait_or_abort(&s.full[(n + 1) & 1], (uint32_t)(((n + 1) >> 1) & 1), abort_flag))
+          break;
+        ptx::tc_fence_after();
+        mma2(n + 1);
+        mma1_half(n + 1, 0);
+        mma1_half(n + 1, 1);
+      }
+      // ---- MMA 5, 6 (chunk n): need V'(n), P(n), D_PV free
+      if (!wait_or_abort(&s.p_done[n & 1], (uint32_t)((n >> 1) & 1), abort_flag)) break;
+      if (!wait_or_abort(&s.vp_ready, par, abort_flag)) break;
+      if (n > 0 && !wait_or_abort(&s.pv_free, par ^ 1u, abort_flag)) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+          ptx::mma_bf16(tb + COL_H, dKmn + so + kk * KSTEP_MN, dVPD + kk * KSTEP_MN, id_h, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+          ptx::mma_bf16(tb + COL_PV, dT2 + so + kk * KSTEP_K, dVP + kk * KSTEP_MN, id_64, kk > 0);
+        ptx::mma_commit(&s.bHP);
+        ptx::mma_commit(&s.empty[st]);
+      }
+      __syncwarp();
+      // ---- while the state is updated: U of chunk n+1 (D_U[(n+1)%2] was
+      //      used by chunk n-1); MMA 4 of n+1 accumulates onto it
+      if (more) {
+        if (n >= 1 &&
+            !wait_or_abort(&s.u_free[(n + 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), abort_flag))
+          break;
+        ptx::tc_fence_after();
+        mma3(n + 1);
+      }
+    }
+    // every MMA this warp issued has finished before TMEM is released
+    if (ptx::elect_one()) ptx::mma_commit(&s.mma_drain);
+    __syncwarp();
+    wait_bounded(&s.mma_drain, 0);
+  } else if (warp == 4 || warp == 5) {
+    // ===================== next-chunk epilogue: W =========================
+    // W rows 0..63 (TMEM lanes 0..63) -> the stage's W slot
+    for (int n = 0; n < nchunks; ++n) {
+      Stage<DK>& S = s.st[n & 1];
+      if (!wait_or_abort(&s.bW, (uint32_t)(n & 1), abort_flag)) break;
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float w[32];
+          ptx::tmem_ld32(tb + lane_base + COL_W + p * 64 + 32 * hf, w);
+          sw128_store_row32(S.panel[p][SW], row, hf, w);
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.w_done);
+    }
+  } else if (warp == 2 || warp == 3 || warp >= 14) {
+    // ===================== next-chunk epilogue: P =========================
+    // Warps 2, 3, 14, 15 (TMEM lanes 64..127); P row r: warps 2, 3 take
+    // columns 32..63, warps 14, 15 columns 0..31.  Warp 2 also computes the
+    // gate cumsum and alpha of the chunk (published through g_ready).
+    const int hc = (warp >= 14) ? 0 : 1;  // P column half
+    const int r = row - 64;
     for (int n = 0; n < nchunks; ++n) {
       Stage<DK>& S = s.st[n & 1];
       float* Gn = s.G[n % 3];
-      const uint32_t par = (uint32_t)(n & 1);
-      if (p_rows) {
-        // gate cumsum of chunk n (warps 2, 3: token r = row - 64)
-        const int r = row - 64, t = n * C + r;
-        float x = (t < T) ? g[((size_t)b * T + t) * H + hh] : 0.f;
+      if (warp == 2) {
+        // tokens lane and lane + 32 of chunk n
+        const int t0 = n * C + lane, t1 = t0 + 32;
+        const float g0 = (t0 < T) ? g[((size_t)b * T + t0) * H + hh] : 0.f;
+        const float g1 = (t1 < T) ? g[((size_t)b * T + t1) * H + hh] : 0.f;
+        float x0 = g0, x1 = g1;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, x, off);
-          if (lane >= off) x += y;
+          const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
+          const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
+          if (lane >= off) { x0 += y0; x1 += y1; }
         }
-        Gn[r] = x;
-        named_sync(1, 64);
-        if (r >= 32) Gn[r] = x + Gn[31];
-        named_sync(1, 64);
+        const float tot0 = __shfl_sync(0xffffffffu, x0, 31);
+        Gn[lane] = x0;
+        Gn[lane + 32] = x1 + tot0;
+        s.alpha[n % 3][lane] = __expf(g0);
+        s.alpha[n % 3][lane + 32] = __expf(g1);
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.g_ready[n % 3]);
-        // P row r
-        if (!wait_or_abort(&s.bS, par, abort_flag)) break;
-        ptx::tc_fence_after();
-        const float Gr = Gn[r];
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float srow[32];
-          ptx::tmem_ld32(tb + lane_base + COL_S + 32 * hf, srow);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int cc = 32 * hf + c;
-            srow[c] = (cc <= r) ? srow[c] * __expf(Gr - Gn[cc]) : 0.f;
-          }
-          sw128_store_row32(S.tp[2], r, hf, srow);
-        }
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.p_done);
       } else {
-        // W row `row` (0..63)
-        if (!wait_or_abort(&s.bWU, par, abort_flag)) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int p = 0; p < NP; ++p) {
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            float w[32];
-            ptx::tmem_ld32(tb + lane_base + COL_W + p * 64 + 32 * hf, w);
-            sw128_store_row32(S.panel[p][SW], row, hf, w);
-          }
-        }
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.w_done);
+        if (!wait_or_abort(&s.g_ready[n % 3], (uint32_t)((n / 3) & 1), abort_flag)) break;
       }
+      const float Gr = Gn[r];
+      const int c_hi = 32 * hc + 31;
+      float d = (r > c_hi) ? __expf(Gr - Gn[c_hi]) : 1.f;
+      float al[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 a4 = reinterpret_cast<const float4*>(&s.alpha[n % 3][32 * hc])[i];
+        al[4 * i] = a4.x; al[4 * i + 1] = a4.y; al[4 * i + 2] = a4.z; al[4 * i + 3] = a4.w;
+      }
+      // P row r, columns [32 hc, 32 hc + 32): e^{G_r - G_s} is the running
+      // product of alpha_j over s < j <= r, from the diagonal leftwards
+      // (every factor <= 1); the left half starts from e^{G_r - G_31}.
+      if (!wait_or_abort(&s.bS[n & 1], (uint32_t)((n >> 1) & 1), abort_flag)) break;
+      ptx::tc_fence_after();
+      float srow[32];
+      ptx::tmem_ld32(tb + lane_base + COL_S + 64 * (n & 1) + 32 * hc, srow);
+#pragma unroll
+      for (int c = 31; c >= 0; --c) {
+        const bool on = 32 * hc + c <= r;
+        srow[c] = on ? srow[c] * d : 0.f;
+        d = on ? d * al[c] : d;
+      }
+      sw128_store_row32(S.tp[TP], r, hc, srow);
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.p_done[n & 1]);
     }
-  } else {
+  } else if (warp >= 6 && warp < 14) {
     // ========================= chain epilogues ==========================
+    // warps 6..9 take state columns [0, 32) of the slab, warps 10..13
+    // columns [32, 64); within each group the lane groups give the rows.
+    const int grp = warp >= 10 ? 1 : 0, cg = 32 * grp;
     const bool has_h = row < DK;
-    float hreg[BV];
+    float hreg[32];
     if (has_h) {
       if (h0) {
         const float4* src =
-            reinterpret_cast<const float4*>(h0 + (head * DK + row) * DV + slab * BV);
+            reinterpret_cast<const float4*>(h0 + (head * DK + row) * DV + slab * BV + cg);
 #pragma unroll
-        for (int j = 0; j < BV / 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
           const float4 x = src[j];
           hreg[4 * j] = x.x; hreg[4 * j + 1] = x.y; hreg[4 * j + 2] = x.z; hreg[4 * j + 3] = x.w;
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < BV; ++j) hreg[j] = 0.f;
+        for (int j = 0; j < 32; ++j) hreg[j] = 0.f;
       }
-      sw128_store_row(s.hm, row, hreg);
+      sw128_store_row32(s.hm, row, grp, hreg);
       ptx::fence_proxy_async_smem();
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.h_done);  // h_0 is in place
-    const bool v_rows = row < 64;           // warps 8, 9
+    const bool v_rows = row < 64;
     bool ok = true;
     for (int n = 0; n < nchunks && ok; ++n) {
       const float* Gn = s.G[n % 3];
       const uint32_t par = (uint32_t)(n & 1);
+      const uint32_t col_u = COL_U + 64 * (n & 1);
       if (!wait_or_abort(&s.g_ready[n % 3], (uint32_t)((n / 3) & 1), abort_flag)) { ok = false; break; }
       const float gC = Gn[C - 1];
-      if (!wait_or_abort(&s.bX, par, abort_flag)) { ok = false; break; }
-      ptx::tc_fence_after();
       if (v_rows) {
-        // V'_r = U_r - (W h)_r, and its copy decayed to the chunk end
+        // V'_r = U_r - (W h)_r (already combined in TMEM) and its copy
+        // decayed to the chunk end for MMA 5
         const float dec = __expf(gC - Gn[row]);
+        if (!wait_or_abort(&s.bX, par, abort_flag)) { ok = false; break; }
+        ptx::tc_fence_after();
+        float u[32];
+        ptx::tmem_ld32(tb + lane_base + col_u + cg, u);
+        sw128_store_row32(s.vp, row, grp, u);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float u[32], x[32];
-          ptx::tmem_ld32(tb + lane_base + COL_U + 64 * (n & 1) + 32 * hf, u);
-          ptx::tmem_ld32(tb + lane_base + COL_X + 32 * hf, x);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) u[j] -= x[j];
-          sw128_store_row32(s.vp, row, hf, u);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) u[j] *= dec;
-          sw128_store_row32(s.vpd, row, hf, u);
-        }
+        for (int j = 0; j < 32; ++j) u[j] *= dec;
+        sw128_store_row32(s.vpd, row, grp, u);
         ptx::tc_fence_before();
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&s.u_free[n & 1]);
-          mbar_arrive(&s.x_free);
           mbar_arrive(&s.vp_ready);
+          mbar_arrive(&s.u_free[n & 1]);
         }
       }
+      // every read of G(n) happens before this warp's last arrival of chunk n
+      const float e_out = v_rows ? 0.f : -__expf(Gn[row - 64]);
       if (!wait_or_abort(&s.bHP, par, abort_flag)) { ok = false; break; }
       ptx::tc_fence_after();
       if (has_h) {
         const float a = __expf(gC);
+        float dh[32];
+        ptx::tmem_ld32(tb + lane_base + COL_H + cg, dh);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float dh[32];
-          ptx::tmem_ld32(tb + lane_base + COL_H + 32 * hf, dh);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) hreg[32 * hf + j] = fmaf(a, hreg[32 * hf + j], dh[j]);
-        }
-        sw128_store_row(s.hm, row, hreg);
+        for (int j = 0; j < 32; ++j) hreg[j] = fmaf(a, hreg[j], dh[j]);
+        sw128_store_row32(s.hm, row, grp, hreg);
         ptx::fence_proxy_async_smem();
       }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.h_done);  // h_{n+1} in place, D_H read
       if (!v_rows) {
-        // output row r = row - 64: o_r = e^{G_r} (Q h)_r + (P V')_r
+        // output row r = row - 64: o_r = e^{G_r} (Q h)_r + (P V')_r, with
+        // -(Q h)_r in lanes 64..127 of D_U
         const int r = row - 64, t = n * C + r;
-        const float e = __expf(Gn[r]);
-        uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * T + t) * H + hh) * DV + slab * BV);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float x[32], pv[32];
-          ptx::tmem_ld32(tb + lane_base + COL_X + 32 * hf, x);
-          ptx::tmem_ld32(tb + lane_base + COL_PV + 32 * hf, pv);
-          if (t < T) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint4 u4;
-              u4.x = pack_bf16x2(fmaf(e, x[8 * c + 0], pv[8 * c + 0]), fmaf(e, x[8 * c + 1], pv[8 * c + 1]));
-              u4.y = pack_bf16x2(fmaf(e, x[8 * c + 2], pv[8 * c + 2]), fmaf(e, x[8 * c + 3], pv[8 * c + 3]));
-              u4.z = pack_bf16x2(fmaf(e, x[8 * c + 4], pv[8 * c + 4]), fmaf(e, x[8 * c + 5], pv[8 * c + 5]));
-              u4.w = pack_bf16x2(fmaf(e, x[8 * c + 6], pv[8 * c + 6]), fmaf(e, x[8 * c + 7], pv[8 * c + 7]));
-              dst[4 * hf + c] = u4;
-            }
-          }
-        }
+        const float e = e_out;
+        float x[32], pv[32];
+        ptx::tmem_ld32(tb + lane_base + col_u + cg, x);
+        ptx::tmem_ld32(tb + lane_base + COL_PV + cg, pv);
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&s.x_free);
+          mbar_arrive(&s.u_free[n & 1]);
           mbar_arrive(&s.pv_free);
+        }
+        if (t < T) {
+          uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * T + t) * H + hh) * DV +
+                                                slab * BV + cg);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint4 u4;
+            u4.x = pack_bf16x2(fmaf(e, x[8 * c + 0], pv[8 * c + 0]), fmaf(e, x[8 * c + 1], pv[8 * c + 1]));
+            u4.y = pack_bf16x2(fmaf(e, x[8 * c + 2], pv[8 * c + 2]), fmaf(e, x[8 * c + 3], pv[8 * c + 3]));
+            u4.z = pack_bf16x2(fmaf(e, x[8 * c + 4], pv[8 * c + 4]), fmaf(e, x[8 * c + 5], pv[8 * c + 5]));
+            u4.w = pack_bf16x2(fmaf(e, x[8 * c + 6], pv[8 * c + 6]), fmaf(e, x[8 * c + 7], pv[8 * c + 7]));
+            dst[c] = u4;
+          }
         }
       }
     }
     if (ok && has_h && hT) {
-      float4* dst = reinterpret_cast<float4*>(hT + (head * DK + row) * DV + slab * BV);
+      float4* dst = reinterpret_cast<float4*>(hT + (head * DK + row) * DV + slab * BV + cg);
 #pragma unroll
-      for (int j = 0; j < BV / 4; ++j)
+      for (int j = 0; j < 8; ++j)
         dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
     }
   }

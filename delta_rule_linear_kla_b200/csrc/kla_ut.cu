@@ -12,7 +12,8 @@
 //
 // A CTA of 128 threads takes two chunks: their keys are stacked into one
 // 128-row operand so a single tcgen05.mma (M = N = 128) yields both Gram
-// matrices (the two diagonal 64x64 blocks of the product).  Thread t owns
+// matrices (the two diagonal 64x64 blocks of the product); the squared key
+// norms are their diagonals.  Thread t owns
 // row (t mod 64) of chunk (t / 64) for the A matrix, then column
 // (t mod 64) for the solve, which runs by forward substitution on CUDA cores
 // in fp32 with the column held in registers and the rows of A broadcast from
@@ -40,6 +41,7 @@ struct alignas(1024) UtSmem {
   float G[2][C];
   float beta[2][C];
   float eg[2][C];         // e^{G}
+  float eb[2][4][C];      // e^{G_{16 I} - G_s} for s < 16 I (row block I)
   uint64_t bar_tma, bar_mma;
   uint32_t tmem_base;
 };
@@ -120,16 +122,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   const uint32_t tb = s.tmem_base;
   bool ok = wait_bounded(&s.bar_tma, 0);
 
-  // ---- beta and the chunk-local inclusive cumsum of g
-  float n2 = 0.f;
-#pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    float x[64];
-    sw128_load_row(s.kk[p], tid, x);
-#pragma unroll
-    for (int i = 0; i < 64; ++i) n2 = fmaf(x[i], x[i], n2);
-  }
-  const float br = er / (n2 + eps);
+  // ---- chunk-local inclusive cumsum of g
   float gs = gr;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -137,12 +130,15 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
     if ((tid & 31) >= off) gs += y;
   }
   s.G[j][r] = gs;
-  s.beta[j][r] = br;
   __syncthreads();
   if (r >= 32) s.G[j][r] = gs + s.G[j][31];
   __syncthreads();
   const float Gr = s.G[j][r];
   s.eg[j][r] = __expf(Gr);
+  // decay from block starts: eb[j][I][s] = e^{G_{16I} - G_s}, s < 16 I
+#pragma unroll
+  for (int I = 1; I < 4; ++I)
+    if (r < 16 * I) s.eb[j][I][r] = __expf(s.G[j][16 * I] - s.G[j][r]);
 
   // ---- Gram matrices of both chunks in one MMA
   if (tid == 0 && ok) {
@@ -159,20 +155,35 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   if (ok) ok = wait_bounded(&s.bar_mma, 0);
   ptx::tc_fence_after();
 
-  // ---- A row r of chunk j
+  // ---- A row r of chunk j.  beta_r = eta_r / (||k_r||^2 + eps) takes the
+  // squared norm from the Gram diagonal.  Decays: within r's own 16-row block
+  // e^{G_r - G_s} directly; for earlier blocks e^{G_r - G_b} e^{G_b - G_s}
+  // with b = 16 * (r / 16) (both factors <= 1, never overflowing).
   if (ok) {
-    float srow[64];
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int I = r >> 4, b0 = 16 * I;
+    float srow[64];
     ptx::tmem_ld32(tb + lane_base + j * 64, srow);
     ptx::tmem_ld32(tb + lane_base + j * 64 + 32, srow + 32);
+    float diag = 0.f;
 #pragma unroll
-    for (int c4 = 0; c4 < C; c4 += 4) {
-      float4 a;
-      a.x = (c4 + 0 < r) ? br * srow[c4 + 0] * __expf(Gr - s.G[j][c4 + 0]) : 0.f;
-      a.y = (c4 + 1 < r) ? br * srow[c4 + 1] * __expf(Gr - s.G[j][c4 + 1]) : 0.f;
-      a.z = (c4 + 2 < r) ? br * srow[c4 + 2] * __expf(Gr - s.G[j][c4 + 2]) : 0.f;
-      a.w = (c4 + 3 < r) ? br * srow[c4 + 3] * __expf(Gr - s.G[j][c4 + 3]) : 0.f;
-      *reinterpret_cast<float4*>(&s.Af[j][r][c4]) = a;
+    for (int c = 0; c < 64; ++c) diag = (c == r) ? srow[c] : diag;
+    const float br = er / (diag + eps);
+    s.beta[j][r] = br;
+    const float cr = br * __expf(Gr - s.G[j][b0]);
+#pragma unroll
+    for (int c4 = 0; c4 < 64; c4 += 4) {
+      float a[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int sc = c4 + e;
+        float v;
+        if (sc < b0) v = cr * srow[sc] * s.eb[j][I][sc];
+        else if (sc < r) v = br * srow[sc] * __expf(Gr - s.G[j][sc]);
+        else v = 0.f;
+        a[e] = v;
+      }
+      *reinterpret_cast<float4*>(&s.Af[j][r][c4]) = make_float4(a[0], a[1], a[2], a[3]);
     }
   }
   ptx::tc_fence_before();
