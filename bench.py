@@ -134,6 +134,12 @@ class L2Flush:
         self.buf.sum()
 
 
+def metric_name(workload):
+    if workload == "prefill_4k":
+        return "prefill tokens/s (0.4B-scale layer, T=4096)"
+    return "prefill tokens/s (%s)" % workload
+
+
 # ------------------------------------------------------------- our arm
 def run_ours(args, rank, world, dev):
     from delta_rule_linear_kla_b200 import api, inputs
@@ -200,8 +206,7 @@ def run_ours(args, rank, world, dev):
     e2e = measure_e2e(args, w, x, fn, dev, stream, world)
 
     res = {
-        "metric": "prefill tokens/s (0.4B-scale layer, T=4096)" if args.workload == "prefill_4k"
-        else "prefill tokens/s (%s)" % args.workload,
+        "metric": metric_name(args.workload),
         "value": value,
         "unit": "tokens/s",
         "n_gpus": world,
@@ -223,7 +228,9 @@ def run_ours(args, rank, world, dev):
         "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
                    "frac": achieved_tf / tc_peak, "algorithmic_flops": flops,
                    "peak_source": peak_src + " (burst cuBLAS bf16)"},
-        "gpu_launches": args.steps,
+        # our kernels per step: UT transform + chain (chunk path), one
+        # token-serial kernel otherwise; the L2 flush is torch's, not counted
+        "gpu_launches": args.steps * (2 if args.path == "chunk" else 1),
         "wall_s": wall,
         "e2e": e2e,
     }
@@ -310,34 +317,61 @@ def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn, clk)
 
 
 # ------------------------------------------------------------ reference
-def run_reference(args, world, rank):
-    """The fp64 oracle on the host cores, on a bounded sample of the workload."""
+def oracle_sample(w, budget_s):
+    """Size a sample of workload ``w`` that costs the oracle about
+    ``budget_s`` seconds on this host: heads drawn like ``w`` (a multiple of
+    the oracle's thread count, up to B*H), length up to T, and whole repeats
+    of that when the full workload costs less than the budget."""
     import oracle
     from delta_rule_linear_kla_b200 import inputs
 
-    w = inputs.WORKLOADS[args.workload]
-    x = inputs.make_prefill(w)
     cores = oracle.num_threads()
-    # sample: the first n_heads heads (b-major) of the workload, full length
-    nh = max(1, min(w.B * w.H, args.ref_heads or w.B * w.H))
-    B_s = max(1, min(w.B, (nh + w.H - 1) // w.H))
+    nh_p = min(w.B * w.H, max(cores, 1))
+    T_p = min(w.T, 256)
+    xp = inputs.make_prefill(w.scaled(B=(nh_p + w.H - 1) // w.H, H=min(w.H, nh_p), T=T_p))
+    t0 = time.perf_counter()
+    oracle.forward(xp["q"], xp["k"], xp["v"], xp["g"], xp["eta"], xp["eps"], xp["h0"])
+    per_round = (time.perf_counter() - t0) / T_p  # s per token for nh_p heads in parallel
+    rounds = budget_s / max(per_round, 1e-9)       # affordable token-rounds of nh_p heads
+    T_s = int(min(w.T, max(T_p, rounds)))
+    groups = max(1, min((w.B * w.H) // nh_p, int(rounds / T_s)))
+    nh = min(w.B * w.H, groups * nh_p)
+    reps = max(1, min(64, int(rounds / (T_s * groups))))
     H_s = min(w.H, nh)
-    xs = {k: x[k][:B_s, :, :H_s].contiguous() for k in ("q", "k", "v", "g", "eta")}
-    h0 = None if x["h0"] is None else x["h0"][:B_s, :H_s].contiguous()
-    for _ in range(args.warmup if args.warmup < 2 else 1):
-        oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["eta"], x["eps"], h0)
-    times = []
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["eta"], x["eps"], h0)
-        times.append(time.perf_counter() - t0)
+    B_s = (nh + H_s - 1) // H_s
+    xs = inputs.make_prefill(w.scaled(B=B_s, H=H_s, T=T_s))
+    return xs, B_s, H_s, T_s, reps, cores
+
+
+def run_oracle_sample(xs, reps):
+    import oracle
+
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["eta"], xs["eps"], xs["h0"])
+    return time.perf_counter() - t0
+
+
+def sample_text(w, B_s, H_s, T_s, reps, t):
+    return "%d of %d heads x T=%d of %s, drawn with the same distributions, run %d time(s): " \
+           "%.1f s of fp64 CPU work" % (B_s * H_s, w.B * w.H, T_s, w.name, reps, t)
+
+
+def run_reference(args, world, rank):
+    """The fp64 oracle on the host cores; each step a bounded sample of the
+    workload sized so the whole run stays within a few minutes."""
+    from delta_rule_linear_kla_b200 import inputs
+
+    w = inputs.WORKLOADS[args.workload]
+    per_step = min(10.0, max(0.5, 100.0 / (args.steps + args.warmup)))
+    xs, B_s, H_s, T_s, reps, cores = oracle_sample(w, per_step)
+    for _ in range(args.warmup):
+        run_oracle_sample(xs, 1)
+    times = [run_oracle_sample(xs, reps) for _ in range(args.steps)]
     t = sum(times) / len(times)
-    head_tokens = B_s * H_s * w.T
-    value = head_tokens / w.H / t  # tokens/s (a token = one position of all H heads)
-    sample = "%d of %d heads x T=%d of %s (first heads, full length)" % (
-        B_s * H_s, w.B * w.H, w.T, w.name)
-    return {"metric": "prefill tokens/s (0.4B-scale layer, T=4096)" if args.workload == "prefill_4k"
-            else "prefill tokens/s (%s)" % args.workload,
+    value = B_s * H_s * T_s * reps / w.H / t  # a token = one position of all H heads
+    sample = sample_text(w, B_s, H_s, T_s, reps, t) + " per step"
+    return {"metric": metric_name(args.workload),
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -352,29 +386,14 @@ def run_reference(args, world, rank):
 
 def cpu_baseline(args, budget_s=15.0):
     """The oracle as it stands, timed on this host on a bounded sample."""
-    import oracle
     from delta_rule_linear_kla_b200 import inputs
 
     w = inputs.WORKLOADS[args.workload]
-    cores = oracle.num_threads()
-    nh = min(w.B * w.H, max(cores, 1))
-    B_s = max(1, (nh + w.H - 1) // w.H)
-    H_s = min(w.H, nh)
-    # probe the per-token cost, then size the sample to ~budget_s
-    T_probe = min(w.T, 256)
-    xs = inputs.make_prefill(w.scaled(B=B_s, T=T_probe, H=H_s))
-    t0 = time.perf_counter()
-    oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["eta"], xs["eps"], xs["h0"])
-    dt = time.perf_counter() - t0
-    T_s = int(min(w.T, max(T_probe, T_probe * budget_s / max(dt, 1e-3))))
-    xs = inputs.make_prefill(w.scaled(B=B_s, T=T_s, H=H_s))
-    t0 = time.perf_counter()
-    oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["eta"], xs["eps"], xs["h0"])
-    t = time.perf_counter() - t0
-    value = B_s * H_s * T_s / w.H / t
+    xs, B_s, H_s, T_s, reps, cores = oracle_sample(w, budget_s)
+    t = run_oracle_sample(xs, reps)
+    value = B_s * H_s * T_s * reps / w.H / t
     return {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": "%d heads x T=%d drawn like %s (%.1f s of fp64 CPU work)"
-                      % (B_s * H_s, T_s, w.name, t)}
+            "sample": sample_text(w, B_s, H_s, T_s, reps, t)}
 
 
 # ---------------------------------------------------------- distributed
@@ -403,7 +422,6 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-heads", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
