@@ -46,16 +46,62 @@ def load_peaks():
 
 # --------------------------------------------------------------- workloads
 def prefill_work(w):
-    """Algorithmic flops and minimum HBM bytes of one prefill."""
+    """Algorithmic flops and minimum HBM bytes of one whole prefill: q, k, v
+    read and o written once, g and eta read once, h0 read (when given) and
+    h_T written.  Dense tensor work per head-token: five (C x C x d) products
+    (K K^T, Q K^T, T'' K, T' V, P V') and three (C x d x d) ones (W h, Q h,
+    K^T V')."""
     C = 64
     d = w.dk
     es = 2 if w.dtype == "bf16" else 4
     ntok = w.B * w.T * w.H  # head-tokens
-    # dense tensor work per head-token: 5 (C x C x d) + 3 (C x d x d) products
     flops = ntok * (10 * C * d + 6 * d * d)
     state = w.B * w.H * w.dk * w.dv * 4
     byts = ntok * (2 * w.dk + 2 * w.dv) * es + ntok * 8 + state * (2 if w.kind == "stress" else 1)
     return flops, byts
+
+
+def stage_work(w):
+    """Algorithmic flops and bytes of each of the two kernels of one prefill.
+
+    UT transform: reads k, g, eta; writes the per-chunk factors T', T''
+    (2 x 64 x 64 bf16 per chunk); flops of K K^T.  State/output kernel:
+    reads q, k, v, g, h0 and the factors; writes o and h_T; flops of the
+    other seven products."""
+    C = 64
+    d = w.dk
+    es = 2
+    ntok = w.B * w.T * w.H
+    nchunk = w.B * w.H * ((w.T + C - 1) // C)
+    fac = nchunk * 2 * C * C * 2
+    state = w.B * w.H * w.dk * w.dv * 4
+    ut = {"flops": ntok * 2 * C * d, "bytes": ntok * w.dk * es + ntok * 8 + fac}
+    chain = {"flops": ntok * (8 * C * d + 6 * d * d),
+             "bytes": ntok * (2 * w.dk + 2 * w.dv) * es + ntok * 4 + fac
+             + state * (2 if w.kind == "stress" else 1)}
+    return ut, chain
+
+
+def profiled_traffic(kernel_file, profile):
+    """DRAM bytes per launch recorded by an ncu capture summarised under
+    profiles/, if the kernel source is unchanged since (same sha256)."""
+    import hashlib
+    src = os.path.join(ROOT, "delta_rule_linear_kla_b200", "csrc", kernel_file)
+    prof = os.path.join(ROOT, "profiles", profile)
+    if not (os.path.exists(src) and os.path.exists(prof)):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    rec = {}
+    for line in open(prof):
+        if ":" in line and line.startswith(("source-sha256", "dram-bytes-per-launch")):
+            k, v = line.split(":", 1)
+            rec[k.strip()] = v.strip()
+    if rec.get("source-sha256") != digest:
+        return None
+    try:
+        return int(rec["dram-bytes-per-launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 class ClockSampler:
@@ -151,7 +197,8 @@ def run_ours(args, rank, world, dev):
     xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     o = torch.empty((w.B, w.T, w.H, w.dv), dtype=w.torch_dtype, device=dev)
     hT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
-    if args.path == "chunk":
+    chunk = args.path == "chunk"
+    if chunk:
         nws = api.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype)
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
         fn = functools.partial(api.chunk_fwd, workspace=ws)
@@ -160,8 +207,16 @@ def run_ours(args, rank, world, dev):
     stream = torch.cuda.current_stream()
     flush = L2Flush(dev)
 
-    def step():
-        fn(xd["q"], xd["k"], xd["v"], xd["g"], xd["eta"], x["eps"], xd["h0"], o=o, hT=hT)
+    def step(mid=None):
+        # the chunk path as its two kernels (exactly what chunk_fwd launches),
+        # with an event between them when the split is being timed
+        if chunk:
+            api.chunk_ut_transform(xd["k"], xd["g"], xd["eta"], x["eps"], workspace=ws)
+            if mid is not None:
+                mid.record(stream)
+            api.chunk_state_fwd(xd["q"], xd["k"], xd["v"], xd["g"], ws, xd["h0"], o=o, hT=hT)
+        else:
+            fn(xd["q"], xd["k"], xd["v"], xd["g"], xd["eta"], x["eps"], xd["h0"], o=o, hT=hT)
 
     clk = ClockSampler(dev.index).__enter__()
     clk.wait_first()
@@ -176,31 +231,38 @@ def run_ours(args, rank, world, dev):
         if i % 8 == 0:
             torch.cuda.synchronize()
     api.check_device_error()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
            for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    for e0, e1 in evs:
+    for e0, em, e1 in evs:
         flush()
         e0.record(stream)
-        step()
+        step(em)
         e1.record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - t0
     t1 = time.perf_counter()
     barrier(world)
     api.check_device_error()
-    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    ms = sum(a.elapsed_time(b) for a, _, b in evs) / args.steps
     ms_max = allreduce_max(ms, world, dev)
+    # per-kernel launch durations over the same timed steps
+    ms_ut = sum(a.elapsed_time(m) for a, m, _ in evs) / args.steps if chunk else 0.0
+    ms_chain = sum(m.elapsed_time(b) for _, m, b in evs) / args.steps if chunk else ms
 
     tokens_per_rank = w.B * w.T
     value = tokens_per_rank * world / (ms_max / 1e3)
     flops, byts = prefill_work(w)
-    achieved_gbs = byts / (ms / 1e3) / 1e9
     achieved_tf = flops / (ms / 1e3) / 1e12
     hbm_peak = float(peaks["hbm_gbs"])
     tc_peak = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    if chunk:
+        ut_w, chain_w = stage_work(w)
+    else:
+        ut_w, chain_w = None, {"flops": flops, "bytes": byts}
+    chain_gbs = chain_w["bytes"] / (ms_chain / 1e3) / 1e9
 
     # end to end through the public API with host buffers (pinned)
     e2e = measure_e2e(args, w, x, fn, dev, stream, world)
@@ -222,18 +284,38 @@ def run_ours(args, rank, world, dev):
                    "chunk": 64, "path": args.path, "global_batch": w.B * world,
                    "seq_len": w.T, "parallelism": "dp%d (independent sequences)" % world,
                    "l2": "flushed before every timed step (512 MiB write+read); inputs > L2"},
-        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": achieved_gbs / hbm_peak, "traffic": None,
-                     "algorithmic_bytes": byts, "peak_source": peak_src},
+        # dominant kernel: the state/output (chain) kernel; its bytes at
+        # the measured copy bandwidth take longer than its flops at the
+        # measured bf16 rate, so it is HBM-bound at the roofline
+        "roofline": {"kernel": "chain_kernel" if chunk else "recurrent_kernel",
+                     "bound": "hbm", "achieved": chain_gbs, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": chain_gbs / hbm_peak,
+                     "traffic": profiled_traffic("kla_chunk_tc.cu",
+                                                 "chain_kernel_prefill_4k.md")
+                     if chunk and w.name == "prefill_4k" else None,
+                     "algorithmic_bytes": chain_w["bytes"], "us_per_launch": ms_chain * 1e3,
+                     "tensor_tflops": chain_w["flops"] / (ms_chain / 1e3) / 1e12,
+                     "peak_source": peak_src + " (burst copy)"},
+        # whole step against the dense bf16 tensor peak (tensor-pipe %)
         "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
                    "frac": achieved_tf / tc_peak, "algorithmic_flops": flops,
+                   "algorithmic_bytes": byts,
+                   "hbm_frac": byts / (ms / 1e3) / 1e9 / hbm_peak,
                    "peak_source": peak_src + " (burst cuBLAS bf16)"},
         # our kernels per step: UT transform + chain (chunk path), one
         # token-serial kernel otherwise; the L2 flush is torch's, not counted
-        "gpu_launches": args.steps * (2 if args.path == "chunk" else 1),
+        "gpu_launches": args.steps * (2 if chunk else 1),
         "wall_s": wall,
         "e2e": e2e,
     }
+    if chunk:
+        res["kernels"] = {
+            "ut_kernel": {"us_per_launch": ms_ut * 1e3, "algorithmic_bytes": ut_w["bytes"],
+                          "gbs": ut_w["bytes"] / (ms_ut / 1e3) / 1e9,
+                          "tflops": ut_w["flops"] / (ms_ut / 1e3) / 1e12},
+            "chain_kernel": {"us_per_launch": ms_chain * 1e3,
+                             "algorithmic_bytes": chain_w["bytes"], "gbs": chain_gbs,
+                             "tflops": chain_w["flops"] / (ms_chain / 1e3) / 1e12}}
     if not args.no_decode:
         res["decode"] = run_decode(args, rank, dev, stream, flush, peaks, peak_src, fn, clk)
     time.sleep(0.25)
@@ -310,8 +392,10 @@ def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn, clk)
             "value": w.B / (ms / 1e3), "unit": "tokens/s", "us_per_step": ms * 1e3,
             "steps": nsteps, "l2": "flushed before every step",
             "clocks": clk.summary(t0, t1 + 0.15), "gpu_launches": nsteps,
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                         "frac": gbs / peak, "traffic": None,
+            "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": gbs,
+                         "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": profiled_traffic("kla_decode.cu",
+                                                     "decode_kernel_decode_b64.md"),
                          "algorithmic_bytes": state_bytes + io_bytes,
                          "peak_source": peak_src}}
 

@@ -5,7 +5,8 @@ torch tensors into the C ABI of ``libkla.so`` (declared in ``include/kla.h``),
 whose CUDA kernels do all of the arithmetic.
 """
 from .api import (KLAError, check_device_error, chunk_fwd,  # noqa: F401
-                  chunk_fwd_workspace_size, decode_step, recurrent_fwd)
+                  chunk_fwd_workspace_size, chunk_state_fwd, chunk_ut_transform,
+                  decode_step, recurrent_fwd)
 
-__all__ = ["chunk_fwd", "recurrent_fwd", "decode_step", "chunk_fwd_workspace_size",
-           "check_device_error", "KLAError"]
+__all__ = ["chunk_fwd", "chunk_ut_transform", "chunk_state_fwd", "recurrent_fwd",
+           "decode_step", "chunk_fwd_workspace_size", "check_device_error", "KLAError"]

@@ -18,6 +18,9 @@ SIGNATURES = {
     "kla_chunk_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "kla_chunk_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
                            _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_chunk_ut_transform": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_chunk_state_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_recurrent_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
                                _i, _i, _i, _i, _i, _i, _vp]),
     "kla_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp,

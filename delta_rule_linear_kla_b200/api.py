@@ -95,6 +95,44 @@ def chunk_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
     return o, hT
 
 
+def _workspace(workspace, B, T, H, dk, dv, dtype, device):
+    need = chunk_fwd_workspace_size(B, T, H, dk, dv, dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def chunk_ut_transform(k, g, eta, eps: float = 1e-6, *, workspace=None, stream=None):
+    """First stage of the bf16 chunk prefill (kla_chunk_ut_transform): the
+    per-chunk factors T diag(beta), T diag(beta e^G) into the workspace,
+    which is returned."""
+    _need(k, "k", torch.bfloat16)
+    B, T, H, dk = k.shape
+    _need(g, "g", torch.float32, (B, T, H))
+    _need(eta, "eta", torch.float32, (B, T, H))
+    workspace, ws_bytes = _workspace(workspace, B, T, H, dk, dk, k.dtype, k.device)
+    st = _native.lib().kla_chunk_ut_transform(
+        _ptr(k), _ptr(g), _ptr(eta), float(eps), B, T, H, dk, KLA_BF16, _ptr(workspace),
+        ws_bytes, _stream(stream))
+    _check(st, "kla_chunk_ut_transform")
+    return workspace
+
+
+def chunk_state_fwd(q, k, v, g, workspace, h0=None, *, o=None, hT=None,
+                    return_state: bool = True, stream=None):
+    """Second stage of the bf16 chunk prefill (kla_chunk_state_fwd): the
+    state recurrence and outputs from a workspace made by chunk_ut_transform
+    of the same k and g.  Returns (o, hT)."""
+    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, g, h0, o, hT, return_state)
+    _need(workspace, "workspace", torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _native.lib().kla_chunk_state_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(h0), _ptr(o), _ptr(hT), B, T, H, dk, dv,
+        _DT[q.dtype], _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "kla_chunk_state_fwd")
+    return o, hT
+
+
 def recurrent_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
                   return_state: bool = True, stream=None):
     """Token-serial KLA prefill on CUDA cores (kla_recurrent_fwd)."""

@@ -8,8 +8,8 @@
 namespace kla {
 
 // Bytes of one chunk's UT factors in the workspace: T' = T diag(beta) and
-// T'' = T diag(beta e^G), two 64x64 bf16 tiles stored exactly as the chain
-// kernel wants them in shared memory (128-byte swizzled rows).
+// T'' = T diag(beta e^G), two 64x64 bf16 tiles stored transposed, exactly as
+// the chain kernel wants them in shared memory (128-byte swizzled rows).
 constexpr size_t kUtTileBytes = 2 * 64 * 64 * 2;
 
 // Device scratch the chunk path needs for these sizes (bytes, 0 if none).
@@ -23,6 +23,16 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v,
                             const float* h0, void* o, float* hT, int B, int T,
                             int H, int dk, int dv, void* workspace,
                             unsigned int* err, cudaStream_t st);
+
+// The two stages of launch_chunk_tc on their own: the UT transform of every
+// chunk into the workspace, then the chain kernel that reads it.
+cudaError_t launch_chunk_ut(const void* k, const float* g, const float* eta, float eps,
+                            int B, int T, int H, int dk, void* workspace, unsigned int* err,
+                            cudaStream_t st);
+cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, const float* g,
+                               const float* h0, void* o, float* hT, int B, int T, int H,
+                               int dk, int dv, const void* workspace, unsigned int* err,
+                               cudaStream_t st);
 
 // UT kernel alone: T', T'' of every chunk into `ws` (chunk-major order
 // ((b * H + h) * nchunks + n)).  `tm_k` maps k as [B][T][H][dk] bf16 with

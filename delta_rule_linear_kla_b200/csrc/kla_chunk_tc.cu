@@ -24,13 +24,18 @@
 // All contractions are single-CTA tcgen05.mma with M = 128, bf16 operands in
 // 128-byte swizzled shared-memory panels and fp32 accumulators in TMEM (lane
 // = row; 64-row products are stacked or padded to 128 lanes):
-//   MMA 1  D_S [128x64]   = [W_stale; Q] . K^T   A, B K-major (lanes 64..127)
-//   MMA 2  D_W [128xDK]   = [T''; P] . K          B MN-major   (lanes 0..63)
-//   MMA 3  D_U [128x64]   = [T'; 0] . V           B MN-major
+//   MMA 1  D_S [128x64]   = [Q; K] . Q^T          A, B K-major (lanes 64..127
+//                                                  hold K Q^T, i.e. P^T before
+//                                                  the mask and decays)
+//   MMA 2  D_W [128xDK]   = [T''; P] . K          A, B MN-major (lanes 0..63)
+//   MMA 3  D_U [128x64]   = [T'; 0] . V           A, B MN-major
 //   MMA 4  D_U           += -[W; Q] . h           B MN-major   (negated A)
 //          -> lanes 0..63 hold V' = U - W h, lanes 64..127 hold -Q h
 //   MMA 5  D_H [128x64]   = K^T . (decay V')      A, B MN-major (lanes < DK)
-//   MMA 6  D_PV[128x64]   = [T''; P] . V'         B MN-major   (lanes 64..127)
+//   MMA 6  D_PV[128x64]   = [T''; P] . V'         A, B MN-major (lanes 64..127)
+// The MN-major A operands [T'; 0] and [T''; P] are kept as the transposed
+// tiles T'^T, 0, T''^T and P^T, which the UT kernel and the P epilogue write
+// by rows.
 //
 // Warp roles (448 threads), synchronised only through mbarriers:
 //   warp 0      TMA producer: K, Q, V slab and the UT tiles of chunk n into
@@ -42,7 +47,7 @@
 //               (it runs while the state is updated).  The tensor pipe
 //               executes in issue order, so this keeps the chain's MMAs from
 //               queueing behind state-independent work.
-//   warps 2, 3, 14, 15  P of the next chunk (TMEM lanes 64..127) into the
+//   warps 2, 3, 14, 15  P^T of the next chunk (TMEM lanes 64..127) into the
 //               stage's P slot; warp 2 also computes the gate cumsum.
 //   warps 4, 5  W of the next chunk (TMEM lanes 0..63) into the W slot.
 //   warps 6..13 "chain" epilogues, split by state columns (warps 6..9 take
@@ -73,8 +78,9 @@ constexpr uint32_t COL_S = 0 /* 2 buffers */, COL_W = 128, COL_U = 256 /* 2 buff
                    COL_H = 384, COL_PV = 448;
 
 // One pipeline stage.  Per 64-column key panel: [W rows | Q rows | K rows]
-// (8 KB each), so [W; Q] is one 128-row K-major operand.  Then the V slab and
-// [T' | 0 | T'' | P]: 128-row MMA A operands [T'; 0] and [T''; P].
+// (8 KB each), so [W; Q] and [Q; K] are 128-row K-major operands.  Then the V
+// slab and [T'^T | 0 | T''^T | P^T]: the 128-row MN-major A operands [T'; 0]
+// and [T''; P] (two 64-column panels each, 8 KB apart).
 template <int DK>
 struct alignas(1024) Stage {
   static constexpr int NP = DK / 64;
@@ -232,18 +238,17 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   } else if (warp == 1) {
     // ============================ MMA issuer ============================
     constexpr uint32_t id_s = ptx::idesc_bf16(128, 64, 0, 0);
-    constexpr uint32_t id_w = ptx::idesc_bf16(128, DK, 0, 1);
-    constexpr uint32_t id_64 = ptx::idesc_bf16(128, 64, 0, 1);
+    constexpr uint32_t id_w = ptx::idesc_bf16(128, DK, 1, 1);
     constexpr uint32_t id_x = ptx::idesc_bf16(128, 64, 0, 1, /*neg_a=*/1);
-    constexpr uint32_t id_h = ptx::idesc_bf16(128, 64, 1, 1);
+    constexpr uint32_t id_mn = ptx::idesc_bf16(128, 64, 1, 1);
     // descriptors of stage 0 / panel 0 (uniform across the warp); other
     // stages and panels are fixed offsets in 16-byte units
     constexpr uint64_t STG = sizeof(Stage<DK>) >> 4, PNL = PANEL >> 4;
     const uint64_t dWQ = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SW]), 16, 1024);
-    const uint64_t dKk = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SK]), 16, 1024);
+    const uint64_t dQK = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SQ]), 16, 1024);
     const uint64_t dKmn = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SK]), PANEL, 1024);
-    const uint64_t dT1 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP1]), 16, 1024);
-    const uint64_t dT2 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP2]), 16, 1024);
+    const uint64_t dT1 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP1]), 8192, 1024);
+    const uint64_t dT2 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP2]), 8192, 1024);
     const uint64_t dV = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].v), 1024, 1024);
     const uint64_t dH = ptx::sdesc_sw128(ptx::smem_u32(s.hm), 1024, 1024);
     const uint64_t dVP = ptx::sdesc_sw128(ptx::smem_u32(s.vp), 1024, 1024);
@@ -254,14 +259,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          ptx::mma_bf16(tb + COL_W, dT2 + so + kk * KSTEP_K, dKmn + so + kk * KSTEP_MN, id_w,
+          ptx::mma_bf16(tb + COL_W, dT2 + so + kk * KSTEP_MN, dKmn + so + kk * KSTEP_MN, id_w,
                         kk > 0);
         ptx::mma_commit(&s.bW);
       }
       __syncwarp();
     };
-    // D_S[n%2] = [W_stale; Q] K^T in two halves of the key dimension, placed
-    // in the two idle windows of the tensor pipe
+    // D_S[n%2] = [Q; K] Q^T in two halves of the key dimension
     auto mma1_half = [&](int n, int half) {
       const uint64_t so = (uint64_t)(n & 1) * STG;
       constexpr int KS = DK / 16, HS = KS / 2;
@@ -269,8 +273,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
         for (int k2 = 0; k2 < HS; ++k2) {
           const int kk = half * HS + k2;
-          ptx::mma_bf16(tb + COL_S + 64 * (n & 1), dWQ + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K,
-                        dKk + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K, id_s, kk > 0);
+          const uint64_t off = so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K;
+          ptx::mma_bf16(tb + COL_S + 64 * (n & 1), dQK + off, dQK + off, id_s, kk > 0);
         }
         if (half == 1) ptx::mma_commit(&s.bS[n & 1]);
       }
@@ -281,8 +285,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          ptx::mma_bf16(tb + COL_U + 64 * (n & 1), dT1 + so + kk * KSTEP_K, dV + so + kk * KSTEP_MN,
-                        id_64, kk > 0);
+          ptx::mma_bf16(tb + COL_U + 64 * (n & 1), dT1 + so + kk * KSTEP_MN, dV + so + kk * KSTEP_MN,
+                        id_mn, kk > 0);
       }
       __syncwarp();
     };
@@ -331,10 +335,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          ptx::mma_bf16(tb + COL_H, dKmn + so + kk * KSTEP_MN, dVPD + kk * KSTEP_MN, id_h, kk > 0);
+          ptx::mma_bf16(tb + COL_H, dKmn + so + kk * KSTEP_MN, dVPD + kk * KSTEP_MN, id_mn, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          ptx::mma_bf16(tb + COL_PV, dT2 + so + kk * KSTEP_K, dVP + kk * KSTEP_MN, id_64, kk > 0);
+          ptx::mma_bf16(tb + COL_PV, dT2 + so + kk * KSTEP_MN, dVP + kk * KSTEP_MN, id_mn, kk > 0);
         ptx::mma_commit(&s.bHP);
         ptx::mma_commit(&s.empty[st]);
       }
@@ -375,12 +379,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       if (lane == 0) mbar_arrive(&s.w_done);
     }
   } else if (warp == 2 || warp == 3 || warp >= 14) {
-    // ===================== next-chunk epilogue: P =========================
-    // Warps 2, 3, 14, 15 (TMEM lanes 64..127); P row r: warps 2, 3 take
-    // columns 32..63, warps 14, 15 columns 0..31.  Warp 2 also computes the
-    // gate cumsum and alpha of the chunk (published through g_ready).
-    const int hc = (warp >= 14) ? 0 : 1;  // P column half
-    const int r = row - 64;
+    // ===================== next-chunk epilogue: P^T ======================
+    // Warps 2, 3, 14, 15 (TMEM lanes 64..127): lane 64 + s holds row s of
+    // K Q^T, i.e. column s of Q K^T.  Row s of P^T, query columns r >= s:
+    // warps 2, 3 take columns 32..63, warps 14, 15 columns 0..31.  Warp 2
+    // also computes the gate cumsum and alpha of the chunk (published
+    // through g_ready).
+    const int hc = (warp >= 14) ? 0 : 1;  // column half
+    const int sk = row - 64;               // key position s
+    const int c_lo = 32 * hc;
     for (int n = 0; n < nchunks; ++n) {
       Stage<DK>& S = s.st[n & 1];
       float* Gn = s.G[n % 3];
@@ -406,29 +413,27 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       } else {
         if (!wait_or_abort(&s.g_ready[n % 3], (uint32_t)((n / 3) & 1), abort_flag)) break;
       }
-      const float Gr = Gn[r];
-      const int c_hi = 32 * hc + 31;
-      float d = (r > c_hi) ? __expf(Gr - Gn[c_hi]) : 1.f;
+      // e^{G_r - G_s} for r >= s is the running product of alpha_j over
+      // s < j <= r (every factor <= 1); the right half starts from
+      // e^{G_32 - G_s}.
+      float d = (sk < c_lo) ? __expf(Gn[c_lo] - Gn[sk]) : 1.f;
       float al[32];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 a4 = reinterpret_cast<const float4*>(&s.alpha[n % 3][32 * hc])[i];
+        const float4 a4 = reinterpret_cast<const float4*>(&s.alpha[n % 3][c_lo])[i];
         al[4 * i] = a4.x; al[4 * i + 1] = a4.y; al[4 * i + 2] = a4.z; al[4 * i + 3] = a4.w;
       }
-      // P row r, columns [32 hc, 32 hc + 32): e^{G_r - G_s} is the running
-      // product of alpha_j over s < j <= r, from the diagonal leftwards
-      // (every factor <= 1); the left half starts from e^{G_r - G_31}.
       if (!wait_or_abort(&s.bS[n & 1], (uint32_t)((n >> 1) & 1), abort_flag)) break;
       ptx::tc_fence_after();
       float srow[32];
       ptx::tmem_ld32(tb + lane_base + COL_S + 64 * (n & 1) + 32 * hc, srow);
 #pragma unroll
-      for (int c = 31; c >= 0; --c) {
-        const bool on = 32 * hc + c <= r;
-        srow[c] = on ? srow[c] * d : 0.f;
-        d = on ? d * al[c] : d;
+      for (int c = 0; c < 32; ++c) {
+        const int rq = c_lo + c;
+        d = (c > 0 && rq > sk) ? d * al[c] : d;
+        srow[c] = (rq >= sk) ? srow[c] * d : 0.f;
       }
-      sw128_store_row32(S.tp[TP], r, hc, srow);
+      sw128_store_row32(S.tp[TP], sk, hc, srow);
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncwarp();
@@ -577,15 +582,13 @@ bool make_map(CUtensorMap* m, const void* base, int d, int H, int T, int B) {
 }
 
 template <int DK>
-cudaError_t launch_dk(const void* q, const void* k, const void* v, const float* g,
-                      const float* eta, float eps, const float* h0, void* o, float* hT, int B,
-                      int T, int H, int DV, uint8_t* ws, unsigned int* err, cudaStream_t st) {
+cudaError_t launch_chain_dk(const void* q, const void* k, const void* v, const float* g,
+                            const float* h0, void* o, float* hT, int B, int T, int H, int DV,
+                            const uint8_t* ws, unsigned int* err, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, DK, H, T, B) || !make_map(&mk, k, DK, H, T, B) ||
       !make_map(&mv, v, DV, H, T, B))
     return cudaErrorInvalidValue;
-  cudaError_t eu = launch_ut(mk, g, eta, eps, ws, B, T, H, DK, err, st);
-  if (eu != cudaSuccess) return eu;
   const size_t smem = sizeof(ChainSmem<DK>) + 1024;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -610,15 +613,34 @@ size_t chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
   return (size_t)B * H * ((T + C - 1) / C) * kUtTileBytes;
 }
 
+cudaError_t launch_chunk_ut(const void* k, const float* g, const float* eta, float eps,
+                            int B, int T, int H, int dk, void* workspace, unsigned int* err,
+                            cudaStream_t st) {
+  if (dk != 64 && dk != 128) return cudaErrorNotSupported;
+  CUtensorMap mk;
+  if (!make_map(&mk, k, dk, H, T, B)) return cudaErrorInvalidValue;
+  return launch_ut(mk, g, eta, eps, (uint8_t*)workspace, B, T, H, dk, err, st);
+}
+
+cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, const float* g,
+                               const float* h0, void* o, float* hT, int B, int T, int H,
+                               int dk, int dv, const void* workspace, unsigned int* err,
+                               cudaStream_t st) {
+  if (dk != dv) return cudaErrorNotSupported;
+  const uint8_t* ws = (const uint8_t*)workspace;
+  if (dk == 128) return launch_chain_dk<128>(q, k, v, g, h0, o, hT, B, T, H, dv, ws, err, st);
+  if (dk == 64) return launch_chain_dk<64>(q, k, v, g, h0, o, hT, B, T, H, dv, ws, err, st);
+  return cudaErrorNotSupported;
+}
+
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                             const float* eta, float eps, const float* h0, void* o, float* hT,
                             int B, int T, int H, int dk, int dv, void* workspace,
                             unsigned int* err, cudaStream_t st) {
-  if (dk != dv) return cudaErrorNotSupported;
-  uint8_t* ws = (uint8_t*)workspace;
-  if (dk == 128) return launch_dk<128>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dv, ws, err, st);
-  if (dk == 64) return launch_dk<64>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dv, ws, err, st);
-  return cudaErrorNotSupported;
+  if (dk != dv || (dk != 64 && dk != 128)) return cudaErrorNotSupported;
+  cudaError_t e = launch_chunk_ut(k, g, eta, eps, B, T, H, dk, workspace, err, st);
+  if (e != cudaSuccess) return e;
+  return launch_chunk_chain(q, k, v, g, h0, o, hT, B, T, H, dk, dv, workspace, err, st);
 }
 
 }  // namespace kla

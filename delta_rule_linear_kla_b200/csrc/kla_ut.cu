@@ -8,30 +8,36 @@
 //   beta_r = eta_r / (||k_r||^2 + eps),   G_r = sum_{j <= r} g_j (in chunk)
 //   A_rs   = beta_r (k_r . k_s) e^{G_r - G_s}   for s < r, else 0
 //   T      = (I + A)^{-1}                       (unit lower triangular)
-//   out:   T' = T diag(beta),  T'' = T diag(beta e^G)   (bf16)
+//   out:   T' = T diag(beta),  T'' = T diag(beta e^G), stored transposed
+//          (row c of each tile is column c of the factor), bf16
 //
 // The inverse is taken by blocks of 16 on the tensor cores.  With A_D the
 // four 16x16 diagonal blocks of A, A_O the rest (strictly block-lower) and
 // D = (I + A_D)^{-1}, one has I + A = (I + A_D)(I + D A_O), and N = D A_O is
 // strictly block-lower with N^4 = 0, so
 //
-//   T = (I + N)^{-1} D = (I - N + N^2 - N^3) D = D - N (D - N (D - N D)).
+//   T = (I + N)^{-1} D = (I - N + N^2 - N^3) D = D - N (D - N (D - N D)),
 //
+// evaluated on the transposes: X_0 = D, X_{i+1}^T = D^T - X_i^T N^T, T = X_3.
 // D (sixteen-row forward substitutions) is computed on CUDA cores in fp32;
 // N = D A_O and the three Horner products are tcgen05.mma kind::tf32 products
 // with fp32 accumulation.
 //
-// A CTA of 128 threads takes two chunks: every operand tile stacks them along
+// A CTA of 256 threads takes two chunks: every operand tile stacks them along
 // its 128 rows, so each product is one M = N = 128 MMA whose two diagonal
-// 64x64 blocks are the two chunks' results (thread t then owns row t).  The
+// 64x64 blocks are the two chunks' results.  Two threads share a row (its
+// TMEM lane): each owns one 32-column half of it.  The
 // squared key norms are the diagonals of the Gram matrices of the first
 // (bf16) MMA.  tf32 operands are K-major on both sides, so a B operand X is
-// stored as X^T (row c holds column c of X).  The decays e^{G_r - G_s} are
-// running products of alpha_j = e^{g_j} over s < j <= r (every factor <= 1).
+// stored as X^T (row c holds column c of X).  The orientation of every
+// product is chosen so that the row a thread holds is a row of the next
+// operand: every shared-memory write is a whole swizzled row.  The decays
+// e^{G_s - G_r} are running products of alpha_j = e^{g_j} over r < j <= s
+// (every factor <= 1).
 //
 // The factors are written to global memory already in the 128-byte swizzled
-// bf16 row layout the chain kernel's MMAs read, so it fetches them with one
-// bulk copy per chunk.
+// bf16 layout the chain kernel's MMAs read (as MN-major A operands), so it
+// fetches them with one bulk copy per chunk.
 #include "kla_chunk.h"
 #include "kla_common.cuh"
 #include "kla_sync.cuh"
@@ -42,26 +48,23 @@ namespace kla {
 namespace {
 
 constexpr int C = 64;
-constexpr int NT = 128;
+constexpr int NT = 256;
 constexpr uint32_t TILE = 128 * 64 * 4;  // one fp32 operand tile: 128 rows x 64 (32 KB)
 
-// fp32 operand tile, K-major with 128-byte swizzle: two panels of 32 columns,
-// each panel 128 rows x 128 B.  Byte offset of element (row, k).
-__device__ __forceinline__ uint32_t f32_off(int row, int k) {
-  const int p = k >> 5, b = (k & 31) * 4;
-  return (uint32_t)p * 16384u + (uint32_t)row * 128u + ((((b >> 4) ^ (row & 7)) & 7) << 4) +
-         (b & 15);
-}
+// An fp32 operand tile is K-major with 128-byte swizzle: two panels of 32
+// columns, each panel 128 rows x 128 B.
 
 template <int DK>
 struct alignas(1024) UtSmem {
   static constexpr int NP = DK / 64;
   // region 0: keys (bf16, per panel: chunk 0 rows then chunk 1 rows); after
-  //           the Gram MMA: D^T (fp32 B operand), later V2^T
+  //           the Gram MMA: D^T, later X_2^T (A operands)
   uint8_t r0[TILE > NP * 16384 ? TILE : NP * 16384];
-  uint8_t r1[TILE];           // A_O^T (B operand), later V1^T
-  uint8_t r2[TILE];           // D (A operand), later N (A operand)
-  float adiag[2][4][16][17];  // diagonal 16x16 blocks of A
+  uint8_t r1[TILE];           // A_O^T (B operand of N), then N (B operand)
+  uint8_t r2[TILE];           // D (A operand of N), later X_1^T
+  // diagonal 16x16 blocks of A, [row][column]; after the solve the same
+  // blocks of D (keeps two CTAs per SM within the shared memory)
+  float adiag[2][4][16][17];
   float G[2][C];
   float beta[2][C];
   float alpha[2][C];
@@ -97,38 +100,29 @@ __device__ __forceinline__ void issue_tf32_product(uint32_t d, const uint8_t* at
   }
 }
 
-__device__ __forceinline__ void st_f32(uint8_t* tile, int row, int k, float v) {
-  *reinterpret_cast<float*>(tile + f32_off(row, k)) = v;
+// Half row: the 32 values of `row` in panel `pan` (columns 32 pan .. 32 pan
+// + 31), as eight 16-byte stores.
+__device__ __forceinline__ void st_half(uint8_t* tile, int pan, int row, const float* v) {
+  uint8_t* base = tile + pan * 16384 + row * 128;
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch)
+    *reinterpret_cast<float4*>(base + (((ch ^ (row & 7)) & 7) << 4)) =
+        make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
 }
 
-// Column k of rows base_row + c (c = 0..63, base_row a multiple of 8): the
-// swizzle phase is c & 7, so the eight addresses per phase are precomputed
-// and every store is one STS with an immediate row offset.
-struct ColWriter {
-  uint8_t* p[8];
-  __device__ __forceinline__ ColWriter(uint8_t* tile, int base_row, int k) {
-    const int pan = k >> 5, b = (k & 31) * 4;
-    uint8_t* base = tile + pan * 16384 + base_row * 128 + (b & 15);
+// Column half `hf` of a 64-wide row that is zero outside the 16 values x of
+// block bb (columns 16 bb .. 16 bb + 15).
+__device__ __forceinline__ void block_half(float* v, const float* x, int bb, int hf) {
+  const bool lo = (bb >> 1) == hf && !(bb & 1), hi = (bb >> 1) == hf && (bb & 1);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) p[e] = base + ((((b >> 4) ^ e) & 7) << 4);
-  }
-  __device__ __forceinline__ void put(int c, float v) const {  // c compile-time
-    *reinterpret_cast<float*>(p[c & 7] + c * 128) = v;
-  }
-};
-
-// Row `row` (64 values) stored with 16-byte vector stores.
-__device__ __forceinline__ void st_row64(uint8_t* tile, int row, const float* v) {
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {  // 16-byte chunk q: columns 4q .. 4q+3
-    const int pan = q >> 3, ch = q & 7;
-    *reinterpret_cast<float4*>(tile + pan * 16384 + row * 128 + (((ch ^ (row & 7)) & 7) << 4)) =
-        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  for (int i = 0; i < 16; ++i) {
+    v[i] = lo ? x[i] : 0.f;
+    v[16 + i] = hi ? x[i] : 0.f;
   }
 }
 
 template <int DK>
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(NT, 2)
 ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
           const float* __restrict__ eta, float eps, uint8_t* __restrict__ ws, int T, int H,
           int nchunks, int total_chunks, unsigned int* err) {
@@ -138,58 +132,60 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                      ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j = tid >> 6, r = tid & 63;  // chunk slot and its row
-  const int ci0 = 2 * blockIdx.x;
-  const int nvalid = min(2, total_chunks - ci0);
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  // warps w and w + 4 share TMEM lane quarter w & 3 (tile row R); warp >> 2
+  // picks the 32-column half (= fp32 panel) of that row the thread owns
+  const int hf = warp >> 2;
+  const int R = 32 * (warp & 3) + lane;
+  const int j = R >> 6, r = R & 63;  // chunk slot and its row
+  const int npairs = (total_chunks + 1) / 2;
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+
+  // keys of pair `pr` (two chunks stacked) -> r0, on bar_tma
+  auto load_keys = [&](int pr) {
+    const int c0 = 2 * pr, nv = min(2, total_chunks - c0);
+    ptx::mbar_arrive_expect_tx(&s.bar_tma, (uint32_t)(nv * NP * 8192));
+    for (int jj = 0; jj < nv; ++jj) {
+      const int cj = c0 + jj, hd = cj / nchunks, nn = cj % nchunks;
+#pragma unroll
+      for (int p = 0; p < NP; ++p)
+        ptx::tma_load_4d(s.r0 + p * 16384 + jj * 8192, &tm_k, &s.bar_tma, p * 64, hd % H,
+                         nn * C, hd / H);
+    }
+  };
+  // gate and relaxation of my token in pair `pr` (zero beyond the sequence)
+  auto load_gates = [&](int pr, float& gv, float& ev) {
+    gv = 0.f;
+    ev = 0.f;
+    const int cj = 2 * pr + j;
+    if (pr < npairs && cj < total_chunks) {
+      const int hd = cj / nchunks, tt = (cj % nchunks) * C + r;
+      if (tt < T) {
+        const size_t tok = ((size_t)(hd / H) * T + tt) * H + hd % H;
+        gv = g[tok];
+        ev = eta[tok];
+      }
+    }
+  };
 
   if (warp == 0) {
     ptx::tmem_alloc(&s.tmem_base, 256);
     ptx::tmem_relinquish();
   }
   if (tid == 0) {
+    ptx::prefetch_tensormap(&tm_k);
     ptx::mbar_init(&s.bar_tma, 1);
     ptx::mbar_init(&s.bar_mma, 1);
     ptx::mbar_init_fence();
-    ptx::mbar_arrive_expect_tx(&s.bar_tma, (uint32_t)(nvalid * NP * 8192));
-    for (int jj = 0; jj < nvalid; ++jj) {
-      const int ci = ci0 + jj, head = ci / nchunks, n = ci % nchunks;
-      const int b = head / H, h = head % H;
-#pragma unroll
-      for (int p = 0; p < NP; ++p)
-        ptx::tma_load_4d(s.r0 + p * 16384 + jj * 8192, &tm_k, &s.bar_tma, p * 64, h, n * C, b);
-    }
+    if ((int)blockIdx.x < npairs) load_keys(blockIdx.x);
   }
-  // gate and relaxation of my token (zero beyond the sequence end)
-  const int ci = ci0 + j;
-  const bool valid = j < nvalid;
-  const int head = valid ? ci / nchunks : 0, n = valid ? ci % nchunks : 0;
-  const int t = n * C + r;
-  float gr = 0.f, er = 0.f;
-  if (valid && t < T) {
-    const int b = head / H, h = head % H;
-    const size_t tok = ((size_t)b * T + t) * H + h;
-    gr = g[tok];
-    er = eta[tok];
-  }
-  // chunk-local inclusive cumsum of g (warps 2j, 2j+1 hold chunk j)
-  float gs = gr;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const float y = __shfl_up_sync(0xffffffffu, gs, off);
-    if (lane >= off) gs += y;
-  }
-  s.G[j][r] = gs;
-  s.alpha[j][r] = __expf(gr);
+  float gr, er;
+  load_gates(blockIdx.x, gr, er);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (r >= 32) s.G[j][r] = gs + s.G[j][31];
   const uint32_t tb = s.tmem_base;
   const uint32_t t_gram = tb, t_prod = tb + 128;
-  bool ok = wait_bounded(&s.bar_tma, 0);
-  __syncthreads();
-
+  bool ok = true;
   uint32_t mma_phase = 0;
   auto mma_done = [&]() {
     __syncwarp();
@@ -197,6 +193,43 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
     mma_phase ^= 1u;
     ptx::tc_fence_after();
   };
+
+  uint32_t tma_phase = 0;
+  bool keys_in_flight = tid == 0 && (int)blockIdx.x < npairs;
+  // persistent: pairs blockIdx.x, blockIdx.x + gridDim.x, ...; the keys and
+  // gates of the next pair are fetched while this one is worked on.  Every
+  // thread takes the same number of trips (the exit test is block-uniform).
+#pragma unroll 1
+  for (int pair = blockIdx.x; pair < npairs; pair += gridDim.x) {
+  if (!__syncthreads_and(ok)) break;
+  const int ci0 = 2 * pair;
+  const int nvalid = min(2, total_chunks - ci0);
+  const int ci = ci0 + j;
+  const bool valid = j < nvalid;
+  float gn, en;  // next pair's gate and relaxation
+  load_gates(pair + gridDim.x, gn, en);
+  // chunk-local inclusive cumsum of g (lane quarters 2j, 2j+1 hold chunk j)
+  float gs = gr;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, gs, off);
+    if (lane >= off) gs += y;
+  }
+  __syncthreads();  // the previous pair's readers of G, alpha, beta are done
+  if (hf == 0) {
+    s.G[j][r] = gs;
+    s.alpha[j][r] = __expf(gr);
+  }
+  __syncthreads();
+  const float G31 = s.G[j][31];
+  __syncthreads();
+  if (hf == 0 && r >= 32) s.G[j][r] = gs + G31;
+  ok = wait_bounded(&s.bar_tma, tma_phase);
+  if (ok) {
+    tma_phase ^= 1u;
+    keys_in_flight = false;
+  }
+  __syncthreads();
 
   // ---- Gram matrices of both chunks: [K0; K1] [K0; K1]^T (bf16, fp32 acc)
   if (tid == 0 && ok) {
@@ -212,168 +245,157 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   }
   mma_done();
 
-  // ---- A row r of chunk j.  beta_r from the Gram diagonal; e^{G_r - G_s} for
-  // s < r as running products of alpha.  A_O^T -> r1 (row 64 j + c, column r);
-  // the diagonal block -> adiag.
+  // ---- beta_r from the Gram diagonal, then column r of A (A_sr for s > r):
+  // A_sr = beta_s (k_s . k_r) e^{G_s - G_r}, the decay a running product of
+  // alpha_s from s = r + 1 on (every factor <= 1); the right half starts from
+  // e^{G_31 - G_r}.  The Gram matrix is symmetric, so row r of it is also
+  // column r.  Column r of A_O is row r of A_O^T (B operand of N = D A_O,
+  // -> r1); the entries inside my diagonal block go to adiag.
   const int bb = r >> 4;  // my 16-row block
+  const int cq = r & 15;  // my position inside it
   {
-    float srow[64];
-    ptx::tmem_ld32(t_gram + lane_base + j * 64, srow);
-    ptx::tmem_ld32(t_gram + lane_base + j * 64 + 32, srow + 32);
-    float diag = 0.f;
+    float srow[32];
+    ptx::tmem_ld32(t_gram + lane_base + j * 64 + 32 * hf, srow);
+    if ((r >> 5) == hf) {
+      float diag = 0.f;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) diag = (c == r) ? srow[c] : diag;
-    const float br = er / (diag + eps);
-    s.beta[j][r] = br;
-    float d = br;  // beta_r e^{G_r - G_c}, built from c = r leftwards
-#pragma unroll
-    for (int c = 63; c >= 0; --c) {
-      d = (c < r) ? d * s.alpha[j][c + 1] : d;
-      srow[c] = (c < r) ? srow[c] * d : 0.f;
+      for (int c = 0; c < 32; ++c) diag = (32 * hf + c == r) ? srow[c] : diag;
+      s.beta[j][r] = er / (diag + eps);
     }
-    const ColWriter col(s.r1, 64 * j, r);
+    __syncthreads();
+    float d = (hf == 1 && r < 32) ? __expf(G31 - s.G[j][r]) : 1.f;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) col.put(c, ((c >> 4) == bb) ? 0.f : srow[c]);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float v = 0.f;
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) v = (blk == bb) ? srow[16 * blk + i] : v;
-      s.adiag[j][bb][r & 15][i] = v;
+    for (int c = 0; c < 32; ++c) {
+      const int sc = 32 * hf + c;
+      d = (sc > r) ? d * s.alpha[j][sc] : d;
+      srow[c] = (sc > r) ? s.beta[j][sc] * srow[c] * d : 0.f;
     }
+    if ((bb >> 1) == hf) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float v = (bb & 1) ? srow[16 + i] : srow[i];
+        s.adiag[j][bb][i][cq] = v;  // A_bb[i][cq]
+      }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) srow[c] = ((c >> 4) == (bb & 1)) ? 0.f : srow[c];
+    }
+    st_half(s.r1, hf, R, srow);
   }
-  ptx::tc_fence_before();
   __syncthreads();
 
-  // ---- D: thread r solves column (r & 15) of (I + A_bb)^{-1}, bb = r >> 4.
-  // Written as D^T (B operand, r0: the keys are dead) and D (A operand, r2).
+  // ---- D = (I + A_D)^{-1}: column cq of (I + A_bb)^{-1} by forward
+  // substitution (both threads of a row solve it; each keeps it for the
+  // Horner steps).  The column is row r of D^T (the first Horner A operand,
+  // -> r0: the keys are dead); rows of D (A operand of N, -> r2) are read
+  // back through the padded adiag, which then holds D's blocks.
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float acc = 0.f;
+#pragma unroll
+    for (int m = 0; m < i; ++m) acc = fmaf(s.adiag[j][bb][i][m], x[m], acc);
+    x[i] = (i == cq) ? 1.f : (i < cq ? 0.f : -acc);
+  }
   {
-    const int cq = r & 15;
-    float x[16];
+    float v[32];
+    block_half(v, x, bb, hf);
+    st_half(s.r0, hf, R, v);
+    __syncthreads();  // every solve has read A_D
+    if (hf == 0) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float acc = 0.f;
-#pragma unroll
-      for (int m = 0; m < i; ++m) acc = fmaf(s.adiag[j][bb][i][m], x[m], acc);
-      x[i] = (i == cq) ? 1.f : (i < cq ? 0.f : -acc);
+      for (int i = 0; i < 16; ++i) s.adiag[j][bb][i][cq] = x[i];
     }
-    // D^T row 64 j + r is column r of D_j: x in block bb, zero elsewhere
-    {
-      float v[64];
+    __syncthreads();
+    float y[16];
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[16 * blk + i] = (blk == bb) ? x[i] : 0.f;
-      st_row64(s.r0, 64 * j + r, v);
-    }
-    // D: element (16 bb + i, r) = x[i]; row r of D is zeroed outside its block
-    {
-      const ColWriter col(s.r2, 64 * j + 16 * bb, r);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) col.put(i, x[i]);
-    }
-#pragma unroll
-    for (int blk = 0; blk < 4; ++blk)
-      if (blk != bb)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ch = 4 * blk + q, pan = ch >> 3;
-          const int row = 64 * j + r;
-          *reinterpret_cast<float4*>(s.r2 + pan * 16384 + row * 128 +
-                                     ((((ch & 7) ^ (row & 7)) & 7) << 4)) =
-              make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+    for (int i = 0; i < 16; ++i) y[i] = s.adiag[j][bb][cq][i];
+    block_half(v, y, bb, hf);
+    st_half(s.r2, hf, R, v);
   }
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  // my row of D (its 16 non-zeros sit in block bb)
-  float drow[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    drow[i] = *reinterpret_cast<const float*>(s.r2 + f32_off(64 * j + r, 16 * bb + i));
 
-  // ---- N = D A_O  ->  r2 (A operand rows); D is dead afterwards
+  // ---- N = D A_O (lane R = row r of N) -> r1 as the Horner B operand (a
+  // K-major B operand X^T stored by rows is X = N, row-major)
   if (tid == 0 && ok) {
     issue_tf32_product(t_prod, s.r2, s.r1);
     ptx::mma_commit(&s.bar_mma);
   }
   mma_done();
   {
-    float v[64];
-    ptx::tmem_ld32(t_prod + lane_base + j * 64, v);
-    ptx::tmem_ld32(t_prod + lane_base + j * 64 + 32, v + 32);
-    ptx::tc_fence_before();
-    __syncthreads();  // everyone has read its row of D
-    st_row64(s.r2, 64 * j + r, v);
+    float v[32];
+    ptx::tmem_ld32(t_prod + lane_base + j * 64 + 32 * hf, v);
+    st_half(s.r1, hf, R, v);
   }
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
 
-  // ---- Horner: V1 = D - N D (-> r1 as V1^T), V2 = D - N V1 (-> r0 as V2^T),
-  // T = D - N V2
-  float trow[64];
+  // ---- Horner on the transposes: X_0 = D, X_{i+1}^T = D^T - X_i^T N^T, so
+  // lane R of each product is row r of X_{i+1}^T, which is the next A operand
+  // row as is.  X_1^T -> r2 (D is dead), X_2^T -> r0, T^T = X_3^T stays in
+  // registers (row r of T^T = column r of T).
+  float dcol[32];  // my half of column r of D (= row r of D^T)
+  block_half(dcol, x, bb, hf);
+  float trow[32];
 #pragma unroll 1
   for (int step = 0; step < 3; ++step) {
-    const uint8_t* bsrc = (step == 1) ? s.r1 : s.r0;
+    const uint8_t* asrc = (step == 1) ? s.r2 : s.r0;
     if (tid == 0 && ok) {
       ptx::tc_fence_after();
-      issue_tf32_product(t_prod, s.r2, bsrc);
+      issue_tf32_product(t_prod, asrc, s.r1);
       ptx::mma_commit(&s.bar_mma);
     }
     mma_done();
-    ptx::tmem_ld32(t_prod + lane_base + j * 64, trow);
-    ptx::tmem_ld32(t_prod + lane_base + j * 64 + 32, trow + 32);
+    // the last product has read r0: the next pair's keys may land there
+    if (step == 2 && tid == 0 && ok && pair + (int)gridDim.x < npairs) {
+      load_keys(pair + gridDim.x);
+      keys_in_flight = true;
+    }
+    ptx::tmem_ld32(t_prod + lane_base + j * 64 + 32 * hf, trow);
 #pragma unroll
-    for (int c = 0; c < 64; ++c) trow[c] = (((c >> 4) == bb) ? drow[c & 15] : 0.f) - trow[c];
+    for (int c = 0; c < 32; ++c) trow[c] = dcol[c] - trow[c];
     if (step < 2) {
-      uint8_t* bdst = (step == 0) ? s.r1 : s.r0;
-      ptx::tc_fence_before();
-      __syncthreads();  // the product that read the destination has finished
-      const ColWriter col(bdst, 64 * j, r);
-#pragma unroll
-      for (int c = 0; c < 64; ++c) col.put(c, trow[c]);
+      st_half(step == 0 ? s.r2 : s.r0, hf, R, trow);
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
     }
   }
 
-  // ---- T' and T'' rows -> workspace (swizzled bf16 rows, 128 B each)
+  // ---- outputs: row r of T'^T = beta_r (column r of T) and row r of T''^T =
+  // beta_r e^{G_r} (column r of T), swizzled bf16 rows of 128 B; this thread
+  // writes the four 16-byte chunks of its column half
   if (ok && valid) {
-    float row[64];
-#pragma unroll
-    for (int c = 0; c < 64; ++c) row[c] = trow[c] * s.beta[j][c];
+    const float b1 = s.beta[j][r], b2 = b1 * __expf(s.G[j][r]);
     uint8_t* dst = ws + (size_t)ci * kUtTileBytes;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
       uint4 u;
-      u.x = pack_bf16x2(row[8 * c + 0], row[8 * c + 1]);
-      u.y = pack_bf16x2(row[8 * c + 2], row[8 * c + 3]);
-      u.z = pack_bf16x2(row[8 * c + 4], row[8 * c + 5]);
-      u.w = pack_bf16x2(row[8 * c + 6], row[8 * c + 7]);
-      *reinterpret_cast<uint4*>(dst + sw128_chunk_off(r, c)) = u;
-    }
-    // e^{G_c} as a running product of alpha from the chunk start
-    float e = 1.f;
-#pragma unroll
-    for (int c = 0; c < 64; ++c) {
-      e *= s.alpha[j][c];
-      row[c] *= e;
+      u.x = pack_bf16x2(b1 * trow[8 * c + 0], b1 * trow[8 * c + 1]);
+      u.y = pack_bf16x2(b1 * trow[8 * c + 2], b1 * trow[8 * c + 3]);
+      u.z = pack_bf16x2(b1 * trow[8 * c + 4], b1 * trow[8 * c + 5]);
+      u.w = pack_bf16x2(b1 * trow[8 * c + 6], b1 * trow[8 * c + 7]);
+      *reinterpret_cast<uint4*>(dst + sw128_chunk_off(r, 4 * hf + c)) = u;
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
       uint4 u;
-      u.x = pack_bf16x2(row[8 * c + 0], row[8 * c + 1]);
-      u.y = pack_bf16x2(row[8 * c + 2], row[8 * c + 3]);
-      u.z = pack_bf16x2(row[8 * c + 4], row[8 * c + 5]);
-      u.w = pack_bf16x2(row[8 * c + 6], row[8 * c + 7]);
-      *reinterpret_cast<uint4*>(dst + 8192 + sw128_chunk_off(r, c)) = u;
+      u.x = pack_bf16x2(b2 * trow[8 * c + 0], b2 * trow[8 * c + 1]);
+      u.y = pack_bf16x2(b2 * trow[8 * c + 2], b2 * trow[8 * c + 3]);
+      u.z = pack_bf16x2(b2 * trow[8 * c + 4], b2 * trow[8 * c + 5]);
+      u.w = pack_bf16x2(b2 * trow[8 * c + 6], b2 * trow[8 * c + 7]);
+      *reinterpret_cast<uint4*>(dst + 8192 + sw128_chunk_off(r, 4 * hf + c)) = u;
     }
   }
-  if (!ok && tid == 0) report_timeout(err);
+  gr = gn;
+  er = en;
+  }  // pair loop
+  if (!ok) report_timeout(err);
+  // a wait gave up: let this CTA's own key copy land before it exits
+  if (keys_in_flight) wait_bounded(&s.bar_tma, tma_phase);
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -399,7 +421,15 @@ cudaError_t launch_ut_dk(const CUtensorMap& tm_k, const float* g, const float* e
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int grid = (total + 1) / 2;
+  // persistent grid: two CTAs per SM (the shared-memory limit), each taking
+  // every gridDim-th pair of chunks
+  static int sm_count[64] = {};
+  if (!sm_count[dev]) {
+    cudaError_t e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  const int npairs = (total + 1) / 2;
+  const int grid = npairs < 2 * sm_count[dev] ? npairs : 2 * sm_count[dev];
   ut_kernel<DK><<<grid, NT, smem, st>>>(tm_k, g, eta, eps, ws, T, H, nchunks, total, err);
   return cudaGetLastError();
 }

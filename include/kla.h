@@ -90,6 +90,37 @@ KLA_API kla_status kla_chunk_fwd(const void *q, const void *k, const void *v,
                          void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * The two stages of the bf16 kla_chunk_fwd, callable on their own (same
+ * layouts and conventions; kla_chunk_fwd is exactly the first call followed
+ * by the second on the same stream).  dtype must be KLA_BF16 (KLA_FP32 ->
+ * KLA_ERR_UNSUPPORTED); T >= 1; workspace as for kla_chunk_fwd.
+ *
+ * kla_chunk_ut_transform -- per chunk of KLA_CHUNK tokens ("Deep Dive into
+ *   KDA", section 3, with the KLA step size of the KLA Abstract):
+ *   beta_r = eta_r / (||k_r||^2 + eps), G_r = in-chunk inclusive cumsum of
+ *   g, A_rs = beta_r (k_r . k_s) e^{G_r - G_s} (s < r), T = (I + A)^{-1};
+ *   writes T diag(beta) and T diag(beta e^G) of every chunk (bf16, opaque
+ *   layout) into the workspace.  Reads k [B][T][H][dk], g, eta [B][T][H].
+ *   The workspace must not overlap k, g or eta.
+ *
+ * kla_chunk_state_fwd -- the inter-chunk state recurrence and the
+ *   intra-chunk outputs from those factors: per chunk U = T diag(beta) V,
+ *   W = T diag(beta e^G) K, V' = U - W h, o = e^G Q h + P V' (P the causal
+ *   decayed Q K^T, diagonal included), h <- e^{G_last} h + K^T diag(e^{G_last
+ *   - G}) V'.  Reads q, k, v, g (the same k and g the workspace was made
+ *   from), h0 (NULL = zeros) and the workspace; writes o and hT (NULL = not
+ *   returned, may alias h0).  o and hT must not overlap the workspace.
+ */
+KLA_API kla_status kla_chunk_ut_transform(const void *k, const float *g, const float *eta,
+                                  float eps, int B, int T, int H, int dk, int dtype,
+                                  void *workspace, size_t ws_bytes, void *stream);
+
+KLA_API kla_status kla_chunk_state_fwd(const void *q, const void *k, const void *v,
+                               const float *g, const float *h0, void *o, float *hT,
+                               int B, int T, int H, int dk, int dv, int dtype,
+                               const void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Token-serial prefill on CUDA cores: the recurrence evaluated one token at
  * a time in fp32 (same arguments and layouts as kla_chunk_fwd, no chunk and
  * no workspace).  Exact-order fp32 evaluation, used for the fp32 I/O mode.

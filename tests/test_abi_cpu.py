@@ -59,6 +59,32 @@ def test_prefill_rejects_bad_arguments(lib):
                                  None, 1, 4, 1, 32, 32, 1, None) == UNSUPPORTED
 
 
+def test_prefill_stages_reject_bad_arguments(lib):
+    ws, wsb = 8 * A, 1 << 22
+    ut = lambda **kw: lib.kla_chunk_ut_transform(
+        kw.get("k", 2 * A), kw.get("g", 4 * A), kw.get("eta", 5 * A), kw.get("eps", 1e-6),
+        kw.get("B", 1), kw.get("T", 128), kw.get("H", 2), kw.get("dk", 128),
+        kw.get("dtype", 0), kw.get("ws", ws), kw.get("wsb", wsb), None)
+    assert ut(k=None) == INVALID
+    assert ut(T=0) == INVALID
+    assert ut(ws=None) == INVALID
+    assert ut(wsb=16) == INVALID                       # workspace too small
+    assert ut(ws=2 * A + 64) == INVALID                # workspace overlaps k
+    assert ut(dk=96) == UNSUPPORTED
+    assert ut(dtype=1) == UNSUPPORTED                  # fp32 I/O has no stages
+    st = lambda **kw: lib.kla_chunk_state_fwd(
+        kw.get("q", A), kw.get("k", 2 * A), kw.get("v", 3 * A), kw.get("g", 4 * A),
+        kw.get("h0", None), kw.get("o", 6 * A), kw.get("hT", None), kw.get("B", 1),
+        kw.get("T", 128), kw.get("H", 2), kw.get("dk", 128), kw.get("dv", 128),
+        kw.get("dtype", 0), kw.get("ws", ws), kw.get("wsb", wsb), None)
+    assert st(q=None) == INVALID
+    assert st(o=A + 256) == INVALID                    # o overlaps q
+    assert st(o=ws + 1024) == INVALID                  # o overlaps the workspace
+    assert st(wsb=16) == INVALID
+    assert st(dk=128, dv=64) == UNSUPPORTED
+    assert st(dtype=1) == UNSUPPORTED
+
+
 def test_decode_rejects_bad_arguments(lib):
     args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, 6 * A, 7 * A, 2, 3, 128, 128, 0, None]
     bad = list(args); bad[6] = None

@@ -69,6 +69,19 @@ def test_final_state_only_and_alias():
     assert none is None and torch.equal(o2, o)
 
 
+def test_two_stages_equal_one_call():
+    """kla_chunk_ut_transform then kla_chunk_state_fwd is the same computation
+    as kla_chunk_fwd (bit for bit), including a ragged tail and h0."""
+    w = W["stress"].scaled(B=2, T=200, H=3)
+    x = inputs.make_prefill(w)
+    xc = cuda(x)
+    o1, h1 = api.chunk_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"], xc["h0"])
+    ws = api.chunk_ut_transform(xc["k"], xc["g"], xc["eta"], x["eps"])
+    o2, h2 = api.chunk_state_fwd(xc["q"], xc["k"], xc["v"], xc["g"], ws, xc["h0"])
+    api.check_device_error()
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
 def test_deterministic():
     w = W["prefill_4k"].scaled(B=1, T=300, H=2)
     _, o1, h1 = _run(w)
