@@ -11,45 +11,48 @@
 // "Kaczmarz Linear Attention", Abstract):
 //
 //   G_r = sum_{j<=r} g_j  (in chunk)
-//   P  = lower_incl(Q K^T (*) e^{G_r - G_s})                        [MMA 1]
 //   W  = T'' K,  U = T' V                                           [MMA 2, 3]
+//   P  = lower_incl(Q K^T (*) e^{G_r - G_s})                        [MMA 1]
 //   V' = U - W h  (and -Q h)  accumulated onto U in TMEM            [MMA 4]
 //   h <- e^{G_63} h + K^T diag(e^{G_63 - G_s}) V'                    [MMA 5]
 //   O  = diag(e^G) Q h + P V'                                       [MMA 6]
 //
-// The decay ratios are only formed as masked differences of G (never
-// K / Gamma), so strong gates cannot overflow.  A ragged tail is zero-filled
-// by TMA and given g = 0 (and eta = 0 in the UT kernel): an identity step.
+// The decay ratios are only formed as masked differences of G or running
+// products of alpha (never K / Gamma), so strong gates cannot overflow.  A
+// ragged tail is zero-filled by TMA and given g = 0 (and eta = 0 in the UT
+// kernel): an identity step.
 //
-// All contractions are single-CTA tcgen05.mma with M = 128, bf16 operands in
-// 128-byte swizzled shared-memory panels and fp32 accumulators in TMEM (lane
-// = row; 64-row products are stacked or padded to 128 lanes):
-//   MMA 1  D_S [128x64]   = [Q; K] . Q^T          A, B K-major (lanes 64..127
-//                                                  hold K Q^T, i.e. P^T before
-//                                                  the mask and decays)
-//   MMA 2  D_W [128xDK]   = [T''; P] . K          A, B MN-major (lanes 0..63)
+// All contractions are single-CTA tcgen05.mma with M = 128 and fp32
+// accumulators in TMEM (lane = row; 64-row products are stacked or padded to
+// 128 lanes).  [W; Q] is kept in TMEM as the A operand of MMAs 4 and 1 (Q
+// copied in by tcgen05.cp in the tensor pipe, W written by its epilogue), so
+// those two read only their B operand from shared memory; the others take
+// bf16 operands from 128-byte swizzled shared-memory tiles:
+//   MMA 2  D_W [128xDK]   = [T''; 0] . K          A, B MN-major (W: lanes 0..63)
 //   MMA 3  D_U [128x64]   = [T'; 0] . V           A, B MN-major
-//   MMA 4  D_U           += -[W; Q] . h           B MN-major   (negated A)
+//   MMA 1  D_S [128x64]   = [W; Q] . K^T          A in TMEM, B K-major
+//                                                  (lanes 64..127: Q K^T)
+//   MMA 4  D_U           += -[W; Q] . h           A in TMEM, B MN-major
 //          -> lanes 0..63 hold V' = U - W h, lanes 64..127 hold -Q h
 //   MMA 5  D_H [128x64]   = K^T . (decay V')      A, B MN-major (lanes < DK)
-//   MMA 6  D_PV[128x64]   = [T''; P] . V'         A, B MN-major (lanes 64..127)
-// The MN-major A operands [T'; 0] and [T''; P] are kept as the transposed
-// tiles T'^T, 0, T''^T and P^T, which the UT kernel and the P epilogue write
-// by rows.
+//   MMA 6  D_PV[128x64]   = [0; P] . V'           A K-major, B MN-major
+//                                                  (lanes 64..127)
 //
-// Warp roles (448 threads), synchronised only through mbarriers:
-//   warp 0      TMA producer: K, Q, V slab and the UT tiles of chunk n into
+// Warp roles (512 threads), synchronised only through mbarriers:
+//   warp 0      TMA producer: Q, K, V slab and the UT tiles of chunk n into
 //               stage n % 2 (double buffered).
 //   warp 1      MMA issuer: the warp runs the schedule uniformly and one
-//               elected lane issues.  Per iteration n: MMA 4 of chunk n, then
-//               MMAs 2 and 1 of chunk n + 1 (they run while the chain warps
-//               form V'(n)), MMAs 5, 6 of chunk n, then MMA 3 of chunk n + 1
-//               (it runs while the state is updated).  The tensor pipe
-//               executes in issue order, so this keeps the chain's MMAs from
-//               queueing behind state-independent work.
-//   warps 2, 3, 14, 15  P^T of the next chunk (TMEM lanes 64..127) into the
-//               stage's P slot; warp 2 also computes the gate cumsum.
-//   warps 4, 5  W of the next chunk (TMEM lanes 0..63) into the W slot.
+//               elected lane issues.  Per iteration n: MMA 4 of chunk n, the
+//               copy of Q(n + 1) into TMEM and MMA 2 of chunk n + 1 (they run
+//               while V'(n) is formed), MMA 5 and MMA 6 of chunk n, then MMAs
+//               3 and 1 of chunk n + 1 (they run while the state is
+//               updated).  The tensor pipe executes in issue order, so the
+//               state chain's MMAs never queue behind more than one
+//               state-independent product.
+//   warps 4, 5  W of the next chunk: D_W (lanes 0..63) -> bf16 -> [W; Q] in
+//               TMEM.
+//   warps 2, 3, 14, 15  P of the next chunk (TMEM lanes 64..127) into the
+//               stage's P tile; warp 2 also computes the gate cumsum.
 //   warps 6..13 "chain" epilogues, split by state columns (warps 6..9 take
 //               columns 0..31, warps 10..13 columns 32..63): V' (lanes
 //               0..63), the state update (lanes < DK) and the output rows
@@ -73,18 +76,20 @@ constexpr int C = 64;       // chunk length
 constexpr int BV = 64;      // state columns per CTA
 constexpr int NTHREADS = 512;
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM column offsets of the accumulators
-constexpr uint32_t COL_S = 0 /* 2 buffers */, COL_W = 128, COL_U = 256 /* 2 buffers */,
-                   COL_H = 384, COL_PV = 448;
+// TMEM column offsets: accumulators, then the [W; Q] A operand (DK / 2
+// columns of packed bf16 pairs)
+constexpr uint32_t COL_S = 0, COL_W = 64, COL_U = 192 /* 2 buffers */, COL_H = 320,
+                   COL_PV = 384, COL_A = 448;
 
-// One pipeline stage.  Per 64-column key panel: [W rows | Q rows | K rows]
-// (8 KB each), so [W; Q] and [Q; K] are 128-row K-major operands.  Then the V
-// slab and [T'^T | 0 | T''^T | P^T]: the 128-row MN-major A operands [T'; 0]
-// and [T''; P] (two 64-column panels each, 8 KB apart).
+// One pipeline stage.  Per 64-column key panel: [K rows | Q rows] (8 KB
+// each), so the 128 rows from K are [K; Q], whose copy into TMEM puts Q in
+// lanes 64..127.  Then the V slab and [T'^T | T''^T | 0 | P]: the MN-major A
+// operands [T'; 0] (leading offset 16 KB) and [T''; 0] (8 KB), and the
+// K-major A operand [0; P].
 template <int DK>
 struct alignas(1024) Stage {
   static constexpr int NP = DK / 64;
-  uint8_t panel[NP][3][8192];
+  uint8_t panel[NP][2][8192];
   uint8_t v[8192];
   uint8_t tp[4][8192];
 };
@@ -98,8 +103,8 @@ struct alignas(1024) ChainSmem {
   float G[3][C];         // gate cumsum of chunk n in slot n % 3
   alignas(16) float alpha[3][C];  // e^{g_s} of chunk n in slot n % 3
   uint64_t full[2], empty[2];
-  uint64_t bS[2], bW, bX, bHP;           // MMA completions (bS per D_S buffer)
-  uint64_t p_done[2], w_done, vp_ready;  // epilogue -> MMA (p_done per D_S buffer)
+  uint64_t bS, bW, bX, bH, bHP;          // MMA completions
+  uint64_t p_done, w_done, vp_ready;
   uint64_t u_free[2], h_done, pv_free;
   uint64_t g_ready[3];
   uint64_t mma_drain;
@@ -107,8 +112,8 @@ struct alignas(1024) ChainSmem {
   int abort_flag;
 };
 
-enum Slot { SW = 0, SQ = 1, SK = 2 };
-enum TSlot { TP1 = 0, TZ = 1, TP2 = 2, TP = 3 };
+enum Slot { SK = 0, SQ = 1 };
+enum TSlot { TP1 = 0, TP2 = 1, TZ = 2, TP = 3 };
 
 // Bounded wait that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
@@ -145,7 +150,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
              unsigned int* err) {
   using Smem = ChainSmem<DK>;
   constexpr int NP = Stage<DK>::NP;
-  constexpr uint32_t PANEL = 3 * 8192;  // byte stride between key panels
+  constexpr uint32_t PANEL = 2 * 8192;  // byte stride between key panels
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                      ~uintptr_t(1023));
@@ -167,13 +172,14 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       ptx::mbar_init(&s.full[i], 1);
       ptx::mbar_init(&s.empty[i], 1);
       ptx::mbar_init(&s.u_free[i], 8);
-      ptx::mbar_init(&s.bS[i], 1);
-      ptx::mbar_init(&s.p_done[i], 4);
     }
     for (int i = 0; i < 3; ++i) ptx::mbar_init(&s.g_ready[i], 1);
+    ptx::mbar_init(&s.bS, 1);
     ptx::mbar_init(&s.bW, 1);
     ptx::mbar_init(&s.bX, 1);
+    ptx::mbar_init(&s.bH, 1);
     ptx::mbar_init(&s.bHP, 1);
+    ptx::mbar_init(&s.p_done, 4);
     ptx::mbar_init(&s.w_done, 2);
     ptx::mbar_init(&s.vp_ready, 4);
     ptx::mbar_init(&s.h_done, 8);
@@ -182,7 +188,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     ptx::mbar_init_fence();
     s.abort_flag = 0;
   }
-  // the zero blocks of both stages ([T'; 0] operand of MMA 3)
+  // the zero tiles of both stages
   for (int i = tid; i < 2 * 8192 / 16; i += NTHREADS)
     reinterpret_cast<uint4*>(s.st[i / 512].tp[TZ])[i % 512] = make_uint4(0, 0, 0, 0);
   ptx::fence_proxy_async_smem();
@@ -237,24 +243,27 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
   } else if (warp == 1) {
     // ============================ MMA issuer ============================
-    constexpr uint32_t id_s = ptx::idesc_bf16(128, 64, 0, 0);
     constexpr uint32_t id_w = ptx::idesc_bf16(128, DK, 1, 1);
-    constexpr uint32_t id_x = ptx::idesc_bf16(128, 64, 0, 1, /*neg_a=*/1);
     constexpr uint32_t id_mn = ptx::idesc_bf16(128, 64, 1, 1);
+    constexpr uint32_t id_s = ptx::idesc_bf16(128, 64, 0, 0);
+    constexpr uint32_t id_x = ptx::idesc_bf16(128, 64, 0, 1, /*neg_a=*/1);
+    constexpr uint32_t id_pv = ptx::idesc_bf16(128, 64, 0, 1);
     // descriptors of stage 0 / panel 0 (uniform across the warp); other
     // stages and panels are fixed offsets in 16-byte units
     constexpr uint64_t STG = sizeof(Stage<DK>) >> 4, PNL = PANEL >> 4;
-    const uint64_t dWQ = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SW]), 16, 1024);
-    const uint64_t dQK = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SQ]), 16, 1024);
+    const uint64_t dKk = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SK]), 16, 1024);
+    // (the same descriptor read as 128 rows is [K; Q], the source of the Q copy)
     const uint64_t dKmn = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SK]), PANEL, 1024);
-    const uint64_t dT1 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP1]), 8192, 1024);
+    const uint64_t dT1 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP1]), 2 * 8192, 1024);
     const uint64_t dT2 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP2]), 8192, 1024);
+    const uint64_t dZP = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TZ]), 16, 1024);
     const uint64_t dV = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].v), 1024, 1024);
     const uint64_t dH = ptx::sdesc_sw128(ptx::smem_u32(s.hm), 1024, 1024);
     const uint64_t dVP = ptx::sdesc_sw128(ptx::smem_u32(s.vp), 1024, 1024);
     const uint64_t dVPD = ptx::sdesc_sw128(ptx::smem_u32(s.vpd), 1024, 1024);
+    const uint32_t tA = tb + COL_A;
 
-    auto mma2 = [&](int n) {  // D_W = [T''; P_stale] K  (W in lanes 0..63)
+    auto mma2 = [&](int n) {  // D_W = [T''; 0] K  (W in lanes 0..63)
       const uint64_t so = (uint64_t)(n & 1) * STG;
       if (ptx::elect_one()) {
 #pragma unroll
@@ -265,28 +274,35 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       }
       __syncwarp();
     };
-    // D_S[n%2] = [Q; K] Q^T in two halves of the key dimension
-    auto mma1_half = [&](int n, int half) {
-      const uint64_t so = (uint64_t)(n & 1) * STG;
-      constexpr int KS = DK / 16, HS = KS / 2;
-      if (ptx::elect_one()) {
-#pragma unroll
-        for (int k2 = 0; k2 < HS; ++k2) {
-          const int kk = half * HS + k2;
-          const uint64_t off = so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K;
-          ptx::mma_bf16(tb + COL_S + 64 * (n & 1), dQK + off, dQK + off, id_s, kk > 0);
-        }
-        if (half == 1) ptx::mma_commit(&s.bS[n & 1]);
-      }
-      __syncwarp();
-    };
     auto mma3 = [&](int n) {  // D_U[n%2] = [T'; 0] V
       const uint64_t so = (uint64_t)(n & 1) * STG;
       if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          ptx::mma_bf16(tb + COL_U + 64 * (n & 1), dT1 + so + kk * KSTEP_MN, dV + so + kk * KSTEP_MN,
-                        id_mn, kk > 0);
+          ptx::mma_bf16(tb + COL_U + 64 * (n & 1), dT1 + so + kk * KSTEP_MN,
+                        dV + so + kk * KSTEP_MN, id_mn, kk > 0);
+      }
+      __syncwarp();
+    };
+    // [K(n); Q(n)] -> TMEM [W; Q] (lanes 0..63 get K, overwritten by W(n)
+    // later: the W epilogue waits for MMA 2 of n, which is behind this copy)
+    auto copy_q = [&](int n) {
+      const uint64_t so = (uint64_t)(n & 1) * STG;
+      if (ptx::elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk)
+          ptx::tmem_cp_128x256b(tA + 8 * kk, dKk + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K);
+      }
+      __syncwarp();
+    };
+    auto mma1 = [&](int n) {  // D_S = [W; Q] K^T  (Q K^T in lanes 64..127)
+      const uint64_t so = (uint64_t)(n & 1) * STG;
+      if (ptx::elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk)
+          ptx::mma_bf16_ta(tb + COL_S, tA + 8 * kk,
+                           dKk + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K, id_s, kk > 0);
+        ptx::mma_commit(&s.bS);
       }
       __syncwarp();
     };
@@ -294,63 +310,77 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     if (ok) ok = wait_or_abort(&s.full[0], 0, abort_flag);
     if (ok) {
       ptx::tc_fence_after();
+      copy_q(0);
       mma2(0);
-      mma1_half(0, 0);
-      mma1_half(0, 1);
       mma3(0);
+      ok = wait_or_abort(&s.w_done, 0, abort_flag);
+      if (ok) {
+        ptx::tc_fence_after();
+        mma1(0);
+      }
     }
     for (int n = 0; n < nchunks && ok; ++n) {
       const int st = n & 1;
       const uint64_t so = (uint64_t)st * STG;
       const uint32_t par = (uint32_t)(n & 1);
       const bool more = n + 1 < nchunks;
-      // ---- MMA 4 (chunk n): needs W(n) and h_n (D_H of n-1 read)
+      // ---- MMA 4 (chunk n): needs [W(n); Q(n)] in TMEM and h_n (D_H of
+      //      n-1 read)
       if (!wait_or_abort(&s.w_done, par, abort_flag)) break;
       if (!wait_or_abort(&s.h_done, par, abort_flag)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
-          ptx::mma_bf16(tb + COL_U + 64 * st, dWQ + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K,
-                        dH + kk * KSTEP_MN, id_x, 1);
+          ptx::mma_bf16_ta(tb + COL_U + 64 * st, tA + 8 * kk, dH + kk * KSTEP_MN, id_x, 1);
         ptx::mma_commit(&s.bX);
       }
       __syncwarp();
-      // ---- while V'(n) is formed: W of chunk n+1 (needed by its MMA 4) and
-      //      its Q K^T (so P(n+1) has a whole chunk of slack).  D_W is free
-      //      (W(n) read above) and D_S[(n+1)%2] was read by P(n-1).
+      // ---- while V'(n) is formed: Q(n+1) into TMEM (MMA 4 of n, the last
+      //      reader of [W; Q](n), is ahead of it in the pipe) and W of chunk
+      //      n+1 (needed by its MMA 4; D_W was read before w_done(n))
       if (more) {
         if (!wait_or_abort(&s.full[(n + 1) & 1], (uint32_t)(((n + 1) >> 1) & 1), abort_flag))
           break;
         ptx::tc_fence_after();
+        copy_q(n + 1);
         mma2(n + 1);
-        mma1_half(n + 1, 0);
-        mma1_half(n + 1, 1);
       }
-      // ---- MMA 5, 6 (chunk n): need V'(n), P(n), D_PV free
-      if (!wait_or_abort(&s.p_done[n & 1], (uint32_t)((n >> 1) & 1), abort_flag)) break;
+      // ---- MMA 5 (state), committed on its own so the update starts at once
       if (!wait_or_abort(&s.vp_ready, par, abort_flag)) break;
-      if (n > 0 && !wait_or_abort(&s.pv_free, par ^ 1u, abort_flag)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
           ptx::mma_bf16(tb + COL_H, dKmn + so + kk * KSTEP_MN, dVPD + kk * KSTEP_MN, id_mn, kk > 0);
+        ptx::mma_commit(&s.bH);
+      }
+      __syncwarp();
+      // ---- MMA 6 (chunk n): needs P(n) and D_PV free (outputs of n-1 read)
+      if (!wait_or_abort(&s.p_done, par, abort_flag)) break;
+      if (n > 0 && !wait_or_abort(&s.pv_free, par ^ 1u, abort_flag)) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          ptx::mma_bf16(tb + COL_PV, dT2 + so + kk * KSTEP_MN, dVP + kk * KSTEP_MN, id_mn, kk > 0);
+          ptx::mma_bf16(tb + COL_PV, dZP + so + kk * KSTEP_K, dVP + kk * KSTEP_MN, id_pv, kk > 0);
         ptx::mma_commit(&s.bHP);
         ptx::mma_commit(&s.empty[st]);
       }
       __syncwarp();
-      // ---- while the state is updated: U of chunk n+1 (D_U[(n+1)%2] was
-      //      used by chunk n-1); MMA 4 of n+1 accumulates onto it
       if (more) {
+        // ---- while the state is updated: U of chunk n+1 (D_U[(n+1)%2] was
+        //      used by chunk n-1; MMA 4 of n+1 accumulates onto it) ...
         if (n >= 1 &&
             !wait_or_abort(&s.u_free[(n + 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), abort_flag))
           break;
         ptx::tc_fence_after();
         mma3(n + 1);
+        // ... and Q K^T of chunk n+1: D_S was read by P(n) (waited above),
+        // [W(n+1); Q(n+1)] is in TMEM
+        if (!wait_or_abort(&s.w_done, par ^ 1u, abort_flag)) break;
+        ptx::tc_fence_after();
+        mma1(n + 1);
       }
     }
     // every MMA this warp issued has finished before TMEM is released
@@ -359,43 +389,48 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     wait_bounded(&s.mma_drain, 0);
   } else if (warp == 4 || warp == 5) {
     // ===================== next-chunk epilogue: W =========================
-    // W rows 0..63 (TMEM lanes 0..63) -> the stage's W slot
+    // W rows 0..63 (TMEM lanes 0..63) -> packed bf16 -> [W; Q] in TMEM
     for (int n = 0; n < nchunks; ++n) {
-      Stage<DK>& S = s.st[n & 1];
       if (!wait_or_abort(&s.bW, (uint32_t)(n & 1), abort_flag)) break;
       ptx::tc_fence_after();
 #pragma unroll
       for (int p = 0; p < NP; ++p) {
+        uint32_t pk[32];
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           float w[32];
           ptx::tmem_ld32(tb + lane_base + COL_W + p * 64 + 32 * hf, w);
-          sw128_store_row32(S.panel[p][SW], row, hf, w);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[16 * hf + i] = pack_bf16x2(w[2 * i], w[2 * i + 1]);
         }
+        ptx::tmem_st32(tb + lane_base + COL_A + 32 * p, pk);
       }
-      ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.w_done);
     }
   } else if (warp == 2 || warp == 3 || warp >= 14) {
-    // ===================== next-chunk epilogue: P^T ======================
-    // Warps 2, 3, 14, 15 (TMEM lanes 64..127): lane 64 + s holds row s of
-    // K Q^T, i.e. column s of Q K^T.  Row s of P^T, query columns r >= s:
-    // warps 2, 3 take columns 32..63, warps 14, 15 columns 0..31.  Warp 2
-    // also computes the gate cumsum and alpha of the chunk (published
-    // through g_ready).
-    const int hc = (warp >= 14) ? 0 : 1;  // column half
-    const int sk = row - 64;               // key position s
-    const int c_lo = 32 * hc;
+    // ===================== next-chunk epilogue: P =========================
+    // Warps 2, 3, 14, 15 (TMEM lanes 64..127, row r = lane row - 64); warps
+    // 2, 3 take columns 32..63, warps 14, 15 columns 0..31.  Warp 2 also
+    // computes the gate cumsum and alpha of the chunk (published through
+    // g_ready), loading the next chunk's gates one chunk ahead.
+    const int hc = (warp >= 14) ? 0 : 1;
+    const int r = row - 64;
+    float gn0 = 0.f, gn1 = 0.f;
+    if (warp == 2 && nchunks > 0) {
+      gn0 = (lane < T) ? g[((size_t)b * T + lane) * H + hh] : 0.f;
+      gn1 = (lane + 32 < T) ? g[((size_t)b * T + lane + 32) * H + hh] : 0.f;
+    }
     for (int n = 0; n < nchunks; ++n) {
       Stage<DK>& S = s.st[n & 1];
       float* Gn = s.G[n % 3];
       if (warp == 2) {
-        // tokens lane and lane + 32 of chunk n
-        const int t0 = n * C + lane, t1 = t0 + 32;
-        const float g0 = (t0 < T) ? g[((size_t)b * T + t0) * H + hh] : 0.f;
-        const float g1 = (t1 < T) ? g[((size_t)b * T + t1) * H + hh] : 0.f;
+        const float g0 = gn0, g1 = gn1;
+        // next chunk's gates (tokens lane, lane + 32), used one chunk later
+        const int t0 = (n + 1) * C + lane, t1 = t0 + 32;
+        gn0 = (t0 < T) ? g[((size_t)b * T + t0) * H + hh] : 0.f;
+        gn1 = (t1 < T) ? g[((size_t)b * T + t1) * H + hh] : 0.f;
         float x0 = g0, x1 = g1;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -413,31 +448,34 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       } else {
         if (!wait_or_abort(&s.g_ready[n % 3], (uint32_t)((n / 3) & 1), abort_flag)) break;
       }
-      // e^{G_r - G_s} for r >= s is the running product of alpha_j over
-      // s < j <= r (every factor <= 1); the right half starts from
-      // e^{G_32 - G_s}.
-      float d = (sk < c_lo) ? __expf(Gn[c_lo] - Gn[sk]) : 1.f;
+      // ---- P row r, columns [32 hc, 32 hc + 32): e^{G_r - G_s} is the
+      //      running product of alpha_j over s < j <= r, from the diagonal
+      //      leftwards (every factor <= 1); the left half starts from
+      //      e^{G_r - G_31}.
+      const float Gr = Gn[r];
+      const int c_hi = 32 * hc + 31;
+      float d = (r > c_hi) ? __expf(Gr - Gn[c_hi]) : 1.f;
       float al[32];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 a4 = reinterpret_cast<const float4*>(&s.alpha[n % 3][c_lo])[i];
+        const float4 a4 = reinterpret_cast<const float4*>(&s.alpha[n % 3][32 * hc])[i];
         al[4 * i] = a4.x; al[4 * i + 1] = a4.y; al[4 * i + 2] = a4.z; al[4 * i + 3] = a4.w;
       }
-      if (!wait_or_abort(&s.bS[n & 1], (uint32_t)((n >> 1) & 1), abort_flag)) break;
+      if (!wait_or_abort(&s.bS, (uint32_t)(n & 1), abort_flag)) break;
       ptx::tc_fence_after();
       float srow[32];
-      ptx::tmem_ld32(tb + lane_base + COL_S + 64 * (n & 1) + 32 * hc, srow);
+      ptx::tmem_ld32(tb + lane_base + COL_S + 32 * hc, srow);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int rq = c_lo + c;
-        d = (c > 0 && rq > sk) ? d * al[c] : d;
-        srow[c] = (rq >= sk) ? srow[c] * d : 0.f;
+      for (int c = 31; c >= 0; --c) {
+        const bool on = 32 * hc + c <= r;
+        srow[c] = on ? srow[c] * d : 0.f;
+        d = on ? d * al[c] : d;
       }
-      sw128_store_row32(S.tp[TP], sk, hc, srow);
+      sw128_store_row32(S.tp[TP], r, hc, srow);
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.p_done[n & 1]);
+      if (lane == 0) mbar_arrive(&s.p_done);
     }
   } else if (warp >= 6 && warp < 14) {
     // ========================= chain epilogues ==========================
@@ -494,7 +532,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       }
       // every read of G(n) happens before this warp's last arrival of chunk n
       const float e_out = v_rows ? 0.f : -__expf(Gn[row - 64]);
-      if (!wait_or_abort(&s.bHP, par, abort_flag)) { ok = false; break; }
+      if (!wait_or_abort(&s.bH, par, abort_flag)) { ok = false; break; }
       ptx::tc_fence_after();
       if (has_h) {
         const float a = __expf(gC);
@@ -513,6 +551,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // -(Q h)_r in lanes 64..127 of D_U
         const int r = row - 64, t = n * C + r;
         const float e = e_out;
+        if (!wait_or_abort(&s.bHP, par, abort_flag)) { ok = false; break; }
+        ptx::tc_fence_after();
         float x[32], pv[32];
         ptx::tmem_ld32(tb + lane_base + col_u + cg, x);
         ptx::tmem_ld32(tb + lane_base + COL_PV + cg, pv);

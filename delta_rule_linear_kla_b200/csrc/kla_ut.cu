@@ -19,21 +19,24 @@
 //   T = (I + N)^{-1} D = (I - N + N^2 - N^3) D = D - N (D - N (D - N D)),
 //
 // evaluated on the transposes: X_0 = D, X_{i+1}^T = D^T - X_i^T N^T, T = X_3.
-// D (sixteen-row forward substitutions) is computed on CUDA cores in fp32;
-// N = D A_O and the three Horner products are tcgen05.mma kind::tf32 products
-// with fp32 accumulation.
+// D (sixteen-row forward substitutions) and every combination are fp32 on
+// CUDA cores; N = D A_O and the three Horner products are tcgen05.mma
+// products of bf16 operands with fp32 accumulation.  Rounding those operands
+// to bf16 moves the final outputs far less than the bf16 rounding of T' and
+// T'' themselves, which the state kernel consumes as bf16 anyway.
 //
-// A CTA of 256 threads takes two chunks: every operand tile stacks them along
+// A CTA of 128 threads takes two chunks: every operand tile stacks them along
 // its 128 rows, so each product is one M = N = 128 MMA whose two diagonal
-// 64x64 blocks are the two chunks' results.  Two threads share a row (its
-// TMEM lane): each owns one 32-column half of it.  The
-// squared key norms are the diagonals of the Gram matrices of the first
-// (bf16) MMA.  tf32 operands are K-major on both sides, so a B operand X is
-// stored as X^T (row c holds column c of X).  The orientation of every
-// product is chosen so that the row a thread holds is a row of the next
-// operand: every shared-memory write is a whole swizzled row.  The decays
-// e^{G_s - G_r} are running products of alpha_j = e^{g_j} over r < j <= s
-// (every factor <= 1).
+// 64x64 blocks are the two chunks' results (thread t owns row t).  The
+// squared key norms are the diagonals of the Gram matrices of the first MMA.
+// Operands are K-major on both sides, so a B operand X is stored as X^T (row
+// c holds column c of X).  The orientation of every product is chosen so
+// that the row a thread holds is a row of the next operand: every
+// shared-memory write is a whole swizzled row.  The decays e^{G_s - G_r} are
+// running products of alpha_j = e^{g_j} over r < j <= s (every factor <= 1).
+// Two 16 KB operand tiles and the key tile are all the shared memory a CTA
+// needs, so three CTAs share an SM; each is persistent over pairs of chunks
+// and fetches the next pair's keys and gates while it works.
 //
 // The factors are written to global memory already in the 128-byte swizzled
 // bf16 layout the chain kernel's MMAs read (as MN-major A operands), so it
@@ -48,22 +51,19 @@ namespace kla {
 namespace {
 
 constexpr int C = 64;
-constexpr int NT = 256;
-constexpr uint32_t TILE = 128 * 64 * 4;  // one fp32 operand tile: 128 rows x 64 (32 KB)
-
-// An fp32 operand tile is K-major with 128-byte swizzle: two panels of 32
-// columns, each panel 128 rows x 128 B.
+constexpr int NT = 128;
+constexpr int CTAS_PER_SM = 3;
+constexpr uint32_t TILE = 128 * 64 * 2;  // one bf16 operand tile: 128 rows x 64 (16 KB)
 
 template <int DK>
 struct alignas(1024) UtSmem {
   static constexpr int NP = DK / 64;
-  // region 0: keys (bf16, per panel: chunk 0 rows then chunk 1 rows); after
-  //           the Gram MMA: D^T, later X_2^T (A operands)
-  uint8_t r0[TILE > NP * 16384 ? TILE : NP * 16384];
-  uint8_t r1[TILE];           // A_O^T (B operand of N), then N (B operand)
-  uint8_t r2[TILE];           // D (A operand of N), later X_1^T
+  // keys (per 64-column panel: chunk 0 rows then chunk 1 rows); after the
+  // Gram MMA its first tile holds A_O^T, then N (B operands)
+  uint8_t r0[NP * TILE];
+  uint8_t r1[TILE];  // D (A operand of N), then X_i^T (Horner A operands)
   // diagonal 16x16 blocks of A, [row][column]; after the solve the same
-  // blocks of D (keeps two CTAs per SM within the shared memory)
+  // blocks of D
   float adiag[2][4][16][17];
   float G[2][C];
   float beta[2][C];
@@ -72,57 +72,17 @@ struct alignas(1024) UtSmem {
   uint32_t tmem_base;
 };
 
-__device__ __forceinline__ void mma_tf32(uint32_t d, uint64_t a, uint64_t b, uint32_t id,
-                                         uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(id), "r"(acc)
-      : "memory");
-}
-
-// idesc of kind::tf32: D f32, A and B tf32 (format 2), both K-major.
-constexpr uint32_t idesc_tf32(int M, int N) {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-// D_out(128x128, TMEM) = Atile(128x64) . Btile^T, both tiles K-major fp32.
-__device__ __forceinline__ void issue_tf32_product(uint32_t d, const uint8_t* at,
-                                                   const uint8_t* bt) {
-  constexpr uint32_t id = idesc_tf32(128, 128);
+// D (TMEM, 128 x 128 fp32) = Atile (128 x 64) . Btile^T, both bf16 K-major.
+__device__ __forceinline__ void issue_product(uint32_t d, const uint8_t* at, const uint8_t* bt) {
+  constexpr uint32_t id = ptx::idesc_bf16(128, 128, 0, 0);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {  // K = 8 per instruction
-    const uint32_t off = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-    mma_tf32(d, ptx::sdesc_sw128(ptx::smem_u32(at) + off, 16, 1024),
-             ptx::sdesc_sw128(ptx::smem_u32(bt) + off, 16, 1024), id, kk > 0);
-  }
-}
-
-// Half row: the 32 values of `row` in panel `pan` (columns 32 pan .. 32 pan
-// + 31), as eight 16-byte stores.
-__device__ __forceinline__ void st_half(uint8_t* tile, int pan, int row, const float* v) {
-  uint8_t* base = tile + pan * 16384 + row * 128;
-#pragma unroll
-  for (int ch = 0; ch < 8; ++ch)
-    *reinterpret_cast<float4*>(base + (((ch ^ (row & 7)) & 7) << 4)) =
-        make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
-}
-
-// Column half `hf` of a 64-wide row that is zero outside the 16 values x of
-// block bb (columns 16 bb .. 16 bb + 15).
-__device__ __forceinline__ void block_half(float* v, const float* x, int bb, int hf) {
-  const bool lo = (bb >> 1) == hf && !(bb & 1), hi = (bb >> 1) == hf && (bb & 1);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    v[i] = lo ? x[i] : 0.f;
-    v[16 + i] = hi ? x[i] : 0.f;
-  }
+  for (int kk = 0; kk < C / 16; ++kk)  // K = 16 per instruction
+    ptx::mma_bf16(d, ptx::sdesc_sw128(ptx::smem_u32(at) + kk * 32, 16, 1024),
+                  ptx::sdesc_sw128(ptx::smem_u32(bt) + kk * 32, 16, 1024), id, kk > 0);
 }
 
 template <int DK>
-__global__ void __launch_bounds__(NT, 2)
+__global__ void __launch_bounds__(NT, CTAS_PER_SM)
 ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
           const float* __restrict__ eta, float eps, uint8_t* __restrict__ ws, int T, int H,
           int nchunks, int total_chunks, unsigned int* err) {
@@ -132,13 +92,9 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                      ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // warps w and w + 4 share TMEM lane quarter w & 3 (tile row R); warp >> 2
-  // picks the 32-column half (= fp32 panel) of that row the thread owns
-  const int hf = warp >> 2;
-  const int R = 32 * (warp & 3) + lane;
-  const int j = R >> 6, r = R & 63;  // chunk slot and its row
+  const int j = tid >> 6, r = tid & 63;  // chunk slot and its row
   const int npairs = (total_chunks + 1) / 2;
-  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
   // keys of pair `pr` (two chunks stacked) -> r0, on bar_tma
   auto load_keys = [&](int pr) {
@@ -148,7 +104,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
       const int cj = c0 + jj, hd = cj / nchunks, nn = cj % nchunks;
 #pragma unroll
       for (int p = 0; p < NP; ++p)
-        ptx::tma_load_4d(s.r0 + p * 16384 + jj * 8192, &tm_k, &s.bar_tma, p * 64, hd % H,
+        ptx::tma_load_4d(s.r0 + p * TILE + jj * 8192, &tm_k, &s.bar_tma, p * 64, hd % H,
                          nn * C, hd / H);
     }
   };
@@ -168,7 +124,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   };
 
   if (warp == 0) {
-    ptx::tmem_alloc(&s.tmem_base, 256);
+    ptx::tmem_alloc(&s.tmem_base, 128);
     ptx::tmem_relinquish();
   }
   if (tid == 0) {
@@ -183,9 +139,10 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const uint32_t tb = s.tmem_base;
-  const uint32_t t_gram = tb, t_prod = tb + 128;
+  // one 128-column accumulator: the Gram matrices, then every product
+  const uint32_t tacc = s.tmem_base;
   bool ok = true;
+
   uint32_t mma_phase = 0;
   auto mma_done = [&]() {
     __syncwarp();
@@ -193,205 +150,196 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
     mma_phase ^= 1u;
     ptx::tc_fence_after();
   };
+  // row `R` of the accumulator's diagonal block for my chunk
+  auto ld_row = [&](float* v) {
+    ptx::tmem_ld32(tacc + lane_base + j * 64, v);
+    ptx::tmem_ld32(tacc + lane_base + j * 64 + 32, v + 32);
+  };
 
   uint32_t tma_phase = 0;
   bool keys_in_flight = tid == 0 && (int)blockIdx.x < npairs;
-  // persistent: pairs blockIdx.x, blockIdx.x + gridDim.x, ...; the keys and
-  // gates of the next pair are fetched while this one is worked on.  Every
-  // thread takes the same number of trips (the exit test is block-uniform).
+  // persistent: pairs blockIdx.x, blockIdx.x + gridDim.x, ...  Every thread
+  // takes the same number of trips (the exit test is block-uniform).
 #pragma unroll 1
   for (int pair = blockIdx.x; pair < npairs; pair += gridDim.x) {
-  if (!__syncthreads_and(ok)) break;
-  const int ci0 = 2 * pair;
-  const int nvalid = min(2, total_chunks - ci0);
-  const int ci = ci0 + j;
-  const bool valid = j < nvalid;
-  float gn, en;  // next pair's gate and relaxation
-  load_gates(pair + gridDim.x, gn, en);
-  // chunk-local inclusive cumsum of g (lane quarters 2j, 2j+1 hold chunk j)
-  float gs = gr;
+    if (!__syncthreads_and(ok)) break;
+    const int ci = 2 * pair + j;
+    const bool valid = ci < total_chunks;
+    float gn, en;  // next pair's gate and relaxation
+    load_gates(pair + gridDim.x, gn, en);
+    // chunk-local inclusive cumsum of g (warps 2j, 2j+1 hold chunk j)
+    float gs = gr;
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const float y = __shfl_up_sync(0xffffffffu, gs, off);
-    if (lane >= off) gs += y;
-  }
-  __syncthreads();  // the previous pair's readers of G, alpha, beta are done
-  if (hf == 0) {
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, gs, off);
+      if (lane >= off) gs += y;
+    }
+    __syncthreads();  // the previous pair's readers of G, alpha, beta are done
     s.G[j][r] = gs;
     s.alpha[j][r] = __expf(gr);
-  }
-  __syncthreads();
-  const float G31 = s.G[j][31];
-  __syncthreads();
-  if (hf == 0 && r >= 32) s.G[j][r] = gs + G31;
-  ok = wait_bounded(&s.bar_tma, tma_phase);
-  if (ok) {
-    tma_phase ^= 1u;
-    keys_in_flight = false;
-  }
-  __syncthreads();
-
-  // ---- Gram matrices of both chunks: [K0; K1] [K0; K1]^T (bf16, fp32 acc)
-  if (tid == 0 && ok) {
+    __syncthreads();
+    const float G31 = s.G[j][31];
+    if (r >= 32) s.G[j][r] = gs + G31;
+    ok = wait_bounded(&s.bar_tma, tma_phase);
+    if (ok) {
+      tma_phase ^= 1u;
+      keys_in_flight = false;
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
     ptx::tc_fence_after();
-    constexpr uint32_t id = ptx::idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-    for (int kk = 0; kk < DK / 16; ++kk) {
-      const uint32_t a = ptx::smem_u32(s.r0 + (kk >> 2) * 16384) + (kk & 3) * 32;
-      ptx::mma_bf16(t_gram, ptx::sdesc_sw128(a, 16, 1024), ptx::sdesc_sw128(a, 16, 1024), id,
-                    kk > 0);
-    }
-    ptx::mma_commit(&s.bar_mma);
-  }
-  mma_done();
 
-  // ---- beta_r from the Gram diagonal, then column r of A (A_sr for s > r):
-  // A_sr = beta_s (k_s . k_r) e^{G_s - G_r}, the decay a running product of
-  // alpha_s from s = r + 1 on (every factor <= 1); the right half starts from
-  // e^{G_31 - G_r}.  The Gram matrix is symmetric, so row r of it is also
-  // column r.  Column r of A_O is row r of A_O^T (B operand of N = D A_O,
-  // -> r1); the entries inside my diagonal block go to adiag.
-  const int bb = r >> 4;  // my 16-row block
-  const int cq = r & 15;  // my position inside it
-  {
-    float srow[32];
-    ptx::tmem_ld32(t_gram + lane_base + j * 64 + 32 * hf, srow);
-    if ((r >> 5) == hf) {
-      float diag = 0.f;
-#pragma unroll
-      for (int c = 0; c < 32; ++c) diag = (32 * hf + c == r) ? srow[c] : diag;
-      s.beta[j][r] = er / (diag + eps);
-    }
-    __syncthreads();
-    float d = (hf == 1 && r < 32) ? __expf(G31 - s.G[j][r]) : 1.f;
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const int sc = 32 * hf + c;
-      d = (sc > r) ? d * s.alpha[j][sc] : d;
-      srow[c] = (sc > r) ? s.beta[j][sc] * srow[c] * d : 0.f;
-    }
-    if ((bb >> 1) == hf) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float v = (bb & 1) ? srow[16 + i] : srow[i];
-        s.adiag[j][bb][i][cq] = v;  // A_bb[i][cq]
-      }
-#pragma unroll
-      for (int c = 0; c < 32; ++c) srow[c] = ((c >> 4) == (bb & 1)) ? 0.f : srow[c];
-    }
-    st_half(s.r1, hf, R, srow);
-  }
-  __syncthreads();
-
-  // ---- D = (I + A_D)^{-1}: column cq of (I + A_bb)^{-1} by forward
-  // substitution (both threads of a row solve it; each keeps it for the
-  // Horner steps).  The column is row r of D^T (the first Horner A operand,
-  // -> r0: the keys are dead); rows of D (A operand of N, -> r2) are read
-  // back through the padded adiag, which then holds D's blocks.
-  float x[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float acc = 0.f;
-#pragma unroll
-    for (int m = 0; m < i; ++m) acc = fmaf(s.adiag[j][bb][i][m], x[m], acc);
-    x[i] = (i == cq) ? 1.f : (i < cq ? 0.f : -acc);
-  }
-  {
-    float v[32];
-    block_half(v, x, bb, hf);
-    st_half(s.r0, hf, R, v);
-    __syncthreads();  // every solve has read A_D
-    if (hf == 0) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) s.adiag[j][bb][i][cq] = x[i];
-    }
-    __syncthreads();
-    float y[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = s.adiag[j][bb][cq][i];
-    block_half(v, y, bb, hf);
-    st_half(s.r2, hf, R, v);
-  }
-  ptx::fence_proxy_async_smem();
-  ptx::tc_fence_before();
-  __syncthreads();
-  ptx::tc_fence_after();
-
-  // ---- N = D A_O (lane R = row r of N) -> r1 as the Horner B operand (a
-  // K-major B operand X^T stored by rows is X = N, row-major)
-  if (tid == 0 && ok) {
-    issue_tf32_product(t_prod, s.r2, s.r1);
-    ptx::mma_commit(&s.bar_mma);
-  }
-  mma_done();
-  {
-    float v[32];
-    ptx::tmem_ld32(t_prod + lane_base + j * 64 + 32 * hf, v);
-    st_half(s.r1, hf, R, v);
-  }
-  ptx::fence_proxy_async_smem();
-  ptx::tc_fence_before();
-  __syncthreads();
-
-  // ---- Horner on the transposes: X_0 = D, X_{i+1}^T = D^T - X_i^T N^T, so
-  // lane R of each product is row r of X_{i+1}^T, which is the next A operand
-  // row as is.  X_1^T -> r2 (D is dead), X_2^T -> r0, T^T = X_3^T stays in
-  // registers (row r of T^T = column r of T).
-  float dcol[32];  // my half of column r of D (= row r of D^T)
-  block_half(dcol, x, bb, hf);
-  float trow[32];
-#pragma unroll 1
-  for (int step = 0; step < 3; ++step) {
-    const uint8_t* asrc = (step == 1) ? s.r2 : s.r0;
+    // ---- Gram matrices of both chunks: [K0; K1] [K0; K1]^T
     if (tid == 0 && ok) {
-      ptx::tc_fence_after();
-      issue_tf32_product(t_prod, asrc, s.r1);
+      constexpr uint32_t id = ptx::idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+      for (int kk = 0; kk < DK / 16; ++kk) {
+        const uint32_t a = ptx::smem_u32(s.r0 + (kk >> 2) * TILE) + (kk & 3) * 32;
+        ptx::mma_bf16(tacc, ptx::sdesc_sw128(a, 16, 1024), ptx::sdesc_sw128(a, 16, 1024), id,
+                      kk > 0);
+      }
       ptx::mma_commit(&s.bar_mma);
     }
     mma_done();
-    // the last product has read r0: the next pair's keys may land there
-    if (step == 2 && tid == 0 && ok && pair + (int)gridDim.x < npairs) {
-      load_keys(pair + gridDim.x);
-      keys_in_flight = true;
-    }
-    ptx::tmem_ld32(t_prod + lane_base + j * 64 + 32 * hf, trow);
-#pragma unroll
-    for (int c = 0; c < 32; ++c) trow[c] = dcol[c] - trow[c];
-    if (step < 2) {
-      st_half(step == 0 ? s.r2 : s.r0, hf, R, trow);
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      __syncthreads();
-    }
-  }
 
-  // ---- outputs: row r of T'^T = beta_r (column r of T) and row r of T''^T =
-  // beta_r e^{G_r} (column r of T), swizzled bf16 rows of 128 B; this thread
-  // writes the four 16-byte chunks of its column half
-  if (ok && valid) {
-    const float b1 = s.beta[j][r], b2 = b1 * __expf(s.G[j][r]);
-    uint8_t* dst = ws + (size_t)ci * kUtTileBytes;
+    // ---- beta_r from the Gram diagonal, then column r of A (A_sr for s > r):
+    // A_sr = beta_s (k_s . k_r) e^{G_s - G_r}, the decay a running product of
+    // alpha_s from s = r + 1 on (every factor <= 1).  The Gram matrix is
+    // symmetric, so row r of it is also column r.  Column r of A_O is row r
+    // of A_O^T (B operand of N = D A_O, -> r0: the keys are dead); the
+    // entries inside my diagonal block go to adiag.
+    const int bb = r >> 4;  // my 16-row block
+    const int cq = r & 15;  // my position inside it
+    {
+      float srow[64];
+      ld_row(srow);
+      float diag = 0.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint4 u;
-      u.x = pack_bf16x2(b1 * trow[8 * c + 0], b1 * trow[8 * c + 1]);
-      u.y = pack_bf16x2(b1 * trow[8 * c + 2], b1 * trow[8 * c + 3]);
-      u.z = pack_bf16x2(b1 * trow[8 * c + 4], b1 * trow[8 * c + 5]);
-      u.w = pack_bf16x2(b1 * trow[8 * c + 6], b1 * trow[8 * c + 7]);
-      *reinterpret_cast<uint4*>(dst + sw128_chunk_off(r, 4 * hf + c)) = u;
-    }
+      for (int c = 0; c < 64; ++c) diag = (c == r) ? srow[c] : diag;
+      s.beta[j][r] = er / (diag + eps);
+      ptx::tc_fence_before();
+      __syncthreads();  // beta complete; every thread has read the Gram row
+      float d = 1.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint4 u;
-      u.x = pack_bf16x2(b2 * trow[8 * c + 0], b2 * trow[8 * c + 1]);
-      u.y = pack_bf16x2(b2 * trow[8 * c + 2], b2 * trow[8 * c + 3]);
-      u.z = pack_bf16x2(b2 * trow[8 * c + 4], b2 * trow[8 * c + 5]);
-      u.w = pack_bf16x2(b2 * trow[8 * c + 6], b2 * trow[8 * c + 7]);
-      *reinterpret_cast<uint4*>(dst + 8192 + sw128_chunk_off(r, 4 * hf + c)) = u;
+      for (int c = 0; c < 64; ++c) {
+        d = (c > r) ? d * s.alpha[j][c] : d;
+        srow[c] = (c > r) ? s.beta[j][c] * srow[c] * d : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float v = 0.f;
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) v = (blk == bb) ? srow[16 * blk + i] : v;
+        s.adiag[j][bb][i][cq] = v;  // A_bb[i][cq]
+      }
+#pragma unroll
+      for (int c = 0; c < 64; ++c) srow[c] = ((c >> 4) == bb) ? 0.f : srow[c];
+      sw128_store_row(s.r0, tid, srow);
     }
-  }
-  gr = gn;
-  er = en;
+    __syncthreads();
+
+    // ---- D = (I + A_D)^{-1}: thread r solves column cq of (I + A_bb)^{-1}
+    // by forward substitution and keeps it (it is row r of D^T); rows of D
+    // (A operand of N, -> r1) are read back through the padded adiag, which
+    // then holds D's blocks.
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float acc = 0.f;
+#pragma unroll
+      for (int m = 0; m < i; ++m) acc = fmaf(s.adiag[j][bb][i][m], x[m], acc);
+      x[i] = (i == cq) ? 1.f : (i < cq ? 0.f : -acc);
+    }
+    __syncthreads();  // every solve has read A_D
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s.adiag[j][bb][i][cq] = x[i];
+    __syncthreads();
+    {
+      float v[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) v[c] = ((c >> 4) == bb) ? s.adiag[j][bb][cq][c & 15] : 0.f;
+      sw128_store_row(s.r1, tid, v);
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+
+    // ---- N = D A_O (lane t = row r of N) -> r0 as the Horner B operand (a
+    // K-major B operand X^T stored by rows is X = N, row-major); D^T -> r1
+    // as the first Horner A operand
+    if (tid == 0 && ok) {
+      issue_product(tacc, s.r1, s.r0);
+      ptx::mma_commit(&s.bar_mma);
+    }
+    mma_done();
+    {
+      float v[64];
+      ld_row(v);
+      sw128_store_row(s.r0, tid, v);
+#pragma unroll
+      for (int c = 0; c < 64; ++c) v[c] = ((c >> 4) == bb) ? x[c & 15] : 0.f;
+      sw128_store_row(s.r1, tid, v);
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+
+    // ---- Horner on the transposes: X_0 = D, X_{i+1}^T = D^T - X_i^T N^T, so
+    // lane t of each product is row r of X_{i+1}^T, the next A operand row as
+    // is (written in place: the product that read r1 has finished).  T^T =
+    // X_3^T stays in registers (row r of T^T = column r of T).
+    float trow[64];
+#pragma unroll 1
+    for (int step = 0; step < 3; ++step) {
+      if (tid == 0 && ok) {
+        ptx::tc_fence_after();
+        issue_product(tacc, s.r1, s.r0);
+        ptx::mma_commit(&s.bar_mma);
+      }
+      mma_done();
+      // the last product has read r0: the next pair's keys may land there
+      if (step == 2 && tid == 0 && ok && pair + (int)gridDim.x < npairs) {
+        load_keys(pair + gridDim.x);
+        keys_in_flight = true;
+      }
+      ld_row(trow);
+#pragma unroll
+      for (int c = 0; c < 64; ++c) trow[c] = (((c >> 4) == bb) ? x[c & 15] : 0.f) - trow[c];
+      if (step < 2) {
+        sw128_store_row(s.r1, tid, trow);
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+      }
+    }
+
+    // ---- outputs: row r of T'^T = beta_r (column r of T) and row r of
+    // T''^T = beta_r e^{G_r} (column r of T), swizzled bf16 rows of 128 B
+    if (ok && valid) {
+      const float b1 = s.beta[j][r], b2 = b1 * __expf(s.G[j][r]);
+      uint8_t* dst = ws + (size_t)ci * kUtTileBytes;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 u;
+        u.x = pack_bf16x2(b1 * trow[8 * c + 0], b1 * trow[8 * c + 1]);
+        u.y = pack_bf16x2(b1 * trow[8 * c + 2], b1 * trow[8 * c + 3]);
+        u.z = pack_bf16x2(b1 * trow[8 * c + 4], b1 * trow[8 * c + 5]);
+        u.w = pack_bf16x2(b1 * trow[8 * c + 6], b1 * trow[8 * c + 7]);
+        *reinterpret_cast<uint4*>(dst + sw128_chunk_off(r, c)) = u;
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 u;
+        u.x = pack_bf16x2(b2 * trow[8 * c + 0], b2 * trow[8 * c + 1]);
+        u.y = pack_bf16x2(b2 * trow[8 * c + 2], b2 * trow[8 * c + 3]);
+        u.z = pack_bf16x2(b2 * trow[8 * c + 4], b2 * trow[8 * c + 5]);
+        u.w = pack_bf16x2(b2 * trow[8 * c + 6], b2 * trow[8 * c + 7]);
+        *reinterpret_cast<uint4*>(dst + 8192 + sw128_chunk_off(r, c)) = u;
+      }
+    }
+    gr = gn;
+    er = en;
   }  // pair loop
   if (!ok) report_timeout(err);
   // a wait gave up: let this CTA's own key copy land before it exits
@@ -400,7 +348,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   __syncthreads();
   if (warp == 0) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tb, 256);
+    ptx::tmem_dealloc(tacc, 128);
   }
 }
 
@@ -421,15 +369,15 @@ cudaError_t launch_ut_dk(const CUtensorMap& tm_k, const float* g, const float* e
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  // persistent grid: two CTAs per SM (the shared-memory limit), each taking
-  // every gridDim-th pair of chunks
+  // persistent grid: CTAS_PER_SM CTAs per SM, each taking every gridDim-th
+  // pair of chunks
   static int sm_count[64] = {};
   if (!sm_count[dev]) {
     cudaError_t e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
   }
   const int npairs = (total + 1) / 2;
-  const int grid = npairs < 2 * sm_count[dev] ? npairs : 2 * sm_count[dev];
+  const int grid = npairs < CTAS_PER_SM * sm_count[dev] ? npairs : CTAS_PER_SM * sm_count[dev];
   ut_kernel<DK><<<grid, NT, smem, st>>>(tm_k, g, eta, eps, ws, T, H, nchunks, total, err);
   return cudaGetLastError();
 }

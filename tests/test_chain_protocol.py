@@ -44,11 +44,11 @@ def build(N):
 
     for i in range(2):
         B(("full", i), 1); B(("empty", i), 1); B(("u_free", i), 8)
-        B(("bS", i), 1); B(("p_done", i), 4)
     for i in range(3):
         B(("g_ready", i), 1)
-    for name, c in [("bW", 1), ("bX", 1), ("bHP", 1), ("w_done", 2), ("vp_ready", 4),
-                    ("h_done", 8), ("pv_free", 4)]:
+    for name, c in [("bS", 1), ("bW", 1), ("bX", 1), ("bH", 1), ("bHP", 1), ("p_done", 4),
+                    ("w_done", 2), ("vp_ready", 4), ("h_done", 8),
+                    ("pv_free", 4)]:
         B(name, c)
 
     W = lambda bar, k: ("wait", bar, k)
@@ -65,23 +65,29 @@ def build(N):
         prod.append(("tma", n))
     roles["producer"] = prod
 
-    m = [W(("full", 0), 0), I("mma2", 0), Cm("bW"), I("mma1", 0), Cm(("bS", 0)), I("mma3", 0)]
+    m = [W(("full", 0), 0), I("cpq", 0), I("mma2", 0), Cm("bW"), I("mma3", 0),
+         W("w_done", 0), I("mma1", 0), Cm("bS")]
     for n in range(N):
         more = n + 1 < N
         m += [W("w_done", n), W("h_done", n), I("mma4", n), Cm("bX")]
         if more:
-            m += [W(("full", (n + 1) & 1), (n + 1) >> 1), I("mma2", n + 1), Cm("bW"),
-                  I("mma1", n + 1), Cm(("bS", (n + 1) & 1))]
-        m += [W(("p_done", n & 1), n >> 1), W("vp_ready", n)]
+            m += [W(("full", (n + 1) & 1), (n + 1) >> 1), I("cpq", n + 1), I("mma2", n + 1),
+                  Cm("bW")]
+        m += [W("vp_ready", n), I("mma5", n), Cm("bH"), W("p_done", n)]
         if n > 0:
             m.append(W("pv_free", n - 1))
-        m += [I("mma56", n), Cm("bHP"), Cm(("empty", n & 1))]
+        m += [I("mma6", n), Cm("bHP"), Cm(("empty", n & 1))]
         if more:
             if n >= 1:
                 m.append(W(("u_free", (n + 1) & 1), (n - 1) >> 1))
-            m.append(I("mma3", n + 1))
+            m += [I("mma3", n + 1), W("w_done", n + 1), I("mma1", n + 1), Cm("bS")]
     roles["mma"] = m
 
+    for w in (4, 5):
+        seq = []
+        for n in range(N):
+            seq += [W("bW", n), Do("W", n), A("w_done")]
+        roles[f"w{w}"] = seq
     for w in (2, 3, 14, 15):
         seq = []
         for n in range(N):
@@ -89,13 +95,8 @@ def build(N):
                 seq += [Do("G", n), A(("g_ready", n % 3))]
             else:
                 seq.append(W(("g_ready", n % 3), n // 3))
-            seq += [Do("readG", n), W(("bS", n & 1), n >> 1), Do("P", n), A(("p_done", n & 1))]
+            seq += [Do("readG", n), W("bS", n), Do("P", n), A("p_done")]
         roles[f"p{w}"] = seq
-    for w in (4, 5):
-        seq = []
-        for n in range(N):
-            seq += [W("bW", n), Do("W", n), A("w_done")]
-        roles[f"w{w}"] = seq
     for w in range(6, 14):
         v_rows = (w & 3) < 2
         seq = [A("h_done")]
@@ -103,9 +104,9 @@ def build(N):
             seq += [W(("g_ready", n % 3), n // 3), Do("readG", n)]
             if v_rows:
                 seq += [W("bX", n), Do("Vp", n), A("vp_ready"), A(("u_free", n & 1))]
-            seq += [W("bHP", n), Do("h", n), A("h_done")]
+            seq += [W("bH", n), Do("h", n), A("h_done")]
             if not v_rows:
-                seq += [Do("o", n), A(("u_free", n & 1)), A("pv_free")]
+                seq += [W("bHP", n), Do("o", n), A(("u_free", n & 1)), A("pv_free")]
         roles[f"c{w}"] = seq
     return bars, roles
 
@@ -131,32 +132,44 @@ def run(N, seed):
 
     def check_issue(tag, n):
         # TMEM / smem reuse before the previous user is done
-        if tag == "mma1" and n >= 2 and not finished("P", n - 2, 4):
-            raise Hazard(f"D_S[{n % 2}] overwritten by chunk {n} before P({n - 2}) read it")
+        if tag == "mma1":
+            if n >= 1 and not finished("P", n - 1, 4):
+                raise Hazard(f"D_S overwritten by chunk {n} before P({n - 1}) read it")
+            if not finished("W", n, 2):
+                raise Hazard(f"MMA 1 of {n} before [W; Q]({n}) is in TMEM")
         if tag == "mma2" and n >= 1 and not finished("W", n - 1, 2):
             raise Hazard(f"D_W overwritten by chunk {n} before W({n - 1}) was read")
         if tag == "mma3" and n >= 2 and not (finished("Vp", n - 2, 4) and finished("o", n - 2, 4)):
             raise Hazard(f"D_U[{n % 2}] overwritten by chunk {n} while chunk {n - 2} uses it")
         if tag == "mma4":
             if not finished("W", n, 2):
-                raise Hazard(f"MMA 4 of {n} before W({n}) is written")
+                raise Hazard(f"MMA 4 of {n} before [W; Q]({n}) is in TMEM")
             if n >= 1 and not finished("h", n - 1, 8):
                 raise Hazard(f"MMA 4 of {n} before h_{n} is written")
-        if tag == "mma56":
+        if tag == "mma5":
+            if not finished("Vp", n, 4):
+                raise Hazard(f"MMA 5 of {n} before V'({n})")
+            if n >= 1 and not finished("h", n - 1, 8):
+                raise Hazard(f"D_H of {n} overwritten before chunk {n - 1} read it")
+        if tag == "mma6":
             if not (finished("Vp", n, 4) and finished("P", n, 4)):
-                raise Hazard(f"MMA 5/6 of {n} before V'({n}) / P({n})")
-            if n >= 1 and not (finished("h", n - 1, 8) and finished("o", n - 1, 4)):
-                raise Hazard(f"D_H / D_PV of {n} overwritten before chunk {n - 1} read them")
+                raise Hazard(f"MMA 6 of {n} before V'({n}) / P({n})")
+            if n >= 1 and not finished("o", n - 1, 4):
+                raise Hazard(f"D_PV of {n} overwritten before chunk {n - 1} read it")
 
     def check_do(tag, n):
-        if tag == "Vp" and n >= 1 and ("mma56", n - 1) not in done_mma:
+        if tag == "Vp" and n >= 1 and not {("mma5", n - 1), ("mma6", n - 1)} <= done_mma:
             raise Hazard(f"V'({n}) overwrites vp/vpd while MMA 5/6 of {n - 1} may read them")
-        if tag == "h" and ("mma4", n) not in done_mma:
+        if tag == "h" and not {("mma4", n), ("mma5", n)} <= done_mma:
             raise Hazard(f"h_{n + 1} written while MMA 4 of {n} may read h_{n}")
-        if tag == "W" and n >= 2 and ("mma4", n - 2) not in done_mma:
-            raise Hazard(f"W({n}) overwrites the W slot of chunk {n - 2} in use")
-        if tag == "P" and n >= 2 and ("mma56", n - 2) not in done_mma:
+        if tag == "W" and n >= 1 and ("mma4", n - 1) not in done_mma:
+            raise Hazard(f"W({n}) overwrites [W; Q] while MMA 4 of {n - 1} may read it")
+        if tag == "W" and ("cpq", n) not in done_mma:
+            raise Hazard(f"W({n}) written before the copy of [K; Q]({n}) that it overwrites")
+        if tag == "P" and n >= 2 and ("mma6", n - 2) not in done_mma:
             raise Hazard(f"P({n}) overwrites the P slot of chunk {n - 2} in use")
+        if tag == "P" and ("mma1", n) not in done_mma:
+            raise Hazard(f"P({n}) read before Q K^T of {n} finished")
         if tag == "G":
             old = G_written.get(n % 3)
             if old is not None and G_readers.get(old, 0) < 4 + 8:
@@ -218,15 +231,16 @@ def run(N, seed):
             pipe.append(("commit", st[1]))
         elif st[0] == "tma":
             n = st[1]
-            if n >= 2 and ("mma56", n - 2) not in done_mma:
+            if n >= 2 and not {("mma5", n - 2), ("mma6", n - 2)} <= done_mma:
                 raise Hazard(f"stage of chunk {n} reloaded while chunk {n - 2} uses it")
+            tma_done.pop(n - 2, None)
             tma.append(n)
         elif st[0] == "do":
             check_do(st[1], st[2])
             did[(st[1], st[2])] = did.get((st[1], st[2]), 0) + 1
     stuck = {r: roles[r][pc[r]] for r in roles if pc[r] < len(roles[r])}
     assert not stuck, f"deadlock: {stuck}"
-    assert ("mma56", N - 1) in done_mma
+    assert ("mma6", N - 1) in done_mma
 
 
 @pytest.mark.parametrize("N", [1, 2, 3, 4, 7, 12])
