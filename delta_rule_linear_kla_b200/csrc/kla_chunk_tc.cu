@@ -22,17 +22,14 @@
 // ragged tail is zero-filled by TMA and given g = 0 (and eta = 0 in the UT
 // kernel): an identity step.
 //
-// All contractions are single-CTA tcgen05.mma with M = 128 and fp32
-// accumulators in TMEM (lane = row; 64-row products are stacked or padded to
-// 128 lanes).  [W; Q] is kept in TMEM as the A operand of MMAs 4 and 1 (Q
-// copied in by tcgen05.cp in the tensor pipe, W written by its epilogue), so
-// those two read only their B operand from shared memory; the others take
-// bf16 operands from 128-byte swizzled shared-memory tiles:
+// All contractions are single-CTA tcgen05.mma with M = 128, bf16 operands in
+// 128-byte swizzled shared-memory tiles and fp32 accumulators in TMEM (lane
+// = row; 64-row products are stacked or padded to 128 lanes):
 //   MMA 2  D_W [128xDK]   = [T''; 0] . K          A, B MN-major (W: lanes 0..63)
 //   MMA 3  D_U [128x64]   = [T'; 0] . V           A, B MN-major
-//   MMA 1  D_S [128x64]   = [W; Q] . K^T          A in TMEM, B K-major
+//   MMA 1  D_S [128x64]   = [W; Q] . K^T          A, B K-major
 //                                                  (lanes 64..127: Q K^T)
-//   MMA 4  D_U           += -[W; Q] . h           A in TMEM, B MN-major
+//   MMA 4  D_U           += -[W; Q] . h           B MN-major (negated A)
 //          -> lanes 0..63 hold V' = U - W h, lanes 64..127 hold -Q h
 //   MMA 5  D_H [128x64]   = K^T . (decay V')      A, B MN-major (lanes < DK)
 //   MMA 6  D_PV[128x64]   = [0; P] . V'           A K-major, B MN-major
@@ -42,15 +39,14 @@
 //   warp 0      TMA producer: Q, K, V slab and the UT tiles of chunk n into
 //               stage n % 2 (double buffered).
 //   warp 1      MMA issuer: the warp runs the schedule uniformly and one
-//               elected lane issues.  Per iteration n: MMA 4 of chunk n, the
-//               copy of Q(n + 1) into TMEM and MMA 2 of chunk n + 1 (they run
-//               while V'(n) is formed), MMA 5 and MMA 6 of chunk n, then MMAs
-//               3 and 1 of chunk n + 1 (they run while the state is
-//               updated).  The tensor pipe executes in issue order, so the
+//               elected lane issues.  Per iteration n: MMA 4 of chunk n, MMA 2
+//               of chunk n + 1 (it runs while V'(n) is formed), MMA 5 and
+//               MMA 6 of chunk n, then MMAs 3 and 1 of chunk n + 1 (they run
+//               while the state is updated).  The tensor pipe executes in issue order, so the
 //               state chain's MMAs never queue behind more than one
 //               state-independent product.
-//   warps 4, 5  W of the next chunk: D_W (lanes 0..63) -> bf16 -> [W; Q] in
-//               TMEM.
+//   warps 4, 5  W of the next chunk: D_W (lanes 0..63) -> bf16 -> the
+//               stage's W rows.
 //   warps 2, 3, 14, 15  P of the next chunk (TMEM lanes 64..127) into the
 //               stage's P tile; warp 2 also computes the gate cumsum.
 //   warps 6..13 "chain" epilogues, split by state columns (warps 6..9 take
@@ -76,20 +72,18 @@ constexpr int C = 64;       // chunk length
 constexpr int BV = 64;      // state columns per CTA
 constexpr int NTHREADS = 512;
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM column offsets: accumulators, then the [W; Q] A operand (DK / 2
-// columns of packed bf16 pairs)
+// TMEM column offsets of the accumulators
 constexpr uint32_t COL_S = 0, COL_W = 64, COL_U = 192 /* 2 buffers */, COL_H = 320,
-                   COL_PV = 384, COL_A = 448;
+                   COL_PV = 384;
 
-// One pipeline stage.  Per 64-column key panel: [K rows | Q rows] (8 KB
-// each), so the 128 rows from K are [K; Q], whose copy into TMEM puts Q in
-// lanes 64..127.  Then the V slab and [T'^T | T''^T | 0 | P]: the MN-major A
+// One pipeline stage.  Per 64-column key panel: [W rows | Q rows | K rows]
+// (8 KB each), so [W; Q] is one 128-row K-major operand.  Then the V slab and [T'^T | T''^T | 0 | P]: the MN-major A
 // operands [T'; 0] (leading offset 16 KB) and [T''; 0] (8 KB), and the
 // K-major A operand [0; P].
 template <int DK>
 struct alignas(1024) Stage {
   static constexpr int NP = DK / 64;
-  uint8_t panel[NP][2][8192];
+  uint8_t panel[NP][3][8192];
   uint8_t v[8192];
   uint8_t tp[4][8192];
 };
@@ -112,7 +106,7 @@ struct alignas(1024) ChainSmem {
   int abort_flag;
 };
 
-enum Slot { SK = 0, SQ = 1 };
+enum Slot { SW = 0, SQ = 1, SK = 2 };
 enum TSlot { TP1 = 0, TP2 = 1, TZ = 2, TP = 3 };
 
 // Bounded wait that also gives up as soon as another role has aborted.
@@ -150,7 +144,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
              unsigned int* err) {
   using Smem = ChainSmem<DK>;
   constexpr int NP = Stage<DK>::NP;
-  constexpr uint32_t PANEL = 2 * 8192;  // byte stride between key panels
+  constexpr uint32_t PANEL = 3 * 8192;  // byte stride between key panels
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                      ~uintptr_t(1023));
@@ -251,8 +245,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // descriptors of stage 0 / panel 0 (uniform across the warp); other
     // stages and panels are fixed offsets in 16-byte units
     constexpr uint64_t STG = sizeof(Stage<DK>) >> 4, PNL = PANEL >> 4;
+    const uint64_t dWQ = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SW]), 16, 1024);
     const uint64_t dKk = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SK]), 16, 1024);
-    // (the same descriptor read as 128 rows is [K; Q], the source of the Q copy)
     const uint64_t dKmn = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].panel[0][SK]), PANEL, 1024);
     const uint64_t dT1 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP1]), 2 * 8192, 1024);
     const uint64_t dT2 = ptx::sdesc_sw128(ptx::smem_u32(s.st[0].tp[TP2]), 8192, 1024);
@@ -261,7 +255,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const uint64_t dH = ptx::sdesc_sw128(ptx::smem_u32(s.hm), 1024, 1024);
     const uint64_t dVP = ptx::sdesc_sw128(ptx::smem_u32(s.vp), 1024, 1024);
     const uint64_t dVPD = ptx::sdesc_sw128(ptx::smem_u32(s.vpd), 1024, 1024);
-    const uint32_t tA = tb + COL_A;
 
     auto mma2 = [&](int n) {  // D_W = [T''; 0] K  (W in lanes 0..63)
       const uint64_t so = (uint64_t)(n & 1) * STG;
@@ -284,24 +277,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       }
       __syncwarp();
     };
-    // [K(n); Q(n)] -> TMEM [W; Q] (lanes 0..63 get K, overwritten by W(n)
-    // later: the W epilogue waits for MMA 2 of n, which is behind this copy)
-    auto copy_q = [&](int n) {
-      const uint64_t so = (uint64_t)(n & 1) * STG;
-      if (ptx::elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk)
-          ptx::tmem_cp_128x256b(tA + 8 * kk, dKk + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K);
-      }
-      __syncwarp();
-    };
     auto mma1 = [&](int n) {  // D_S = [W; Q] K^T  (Q K^T in lanes 64..127)
       const uint64_t so = (uint64_t)(n & 1) * STG;
       if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
-          ptx::mma_bf16_ta(tb + COL_S, tA + 8 * kk,
-                           dKk + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K, id_s, kk > 0);
+          ptx::mma_bf16(tb + COL_S, dWQ + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K,
+                        dKk + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K, id_s, kk > 0);
         ptx::mma_commit(&s.bS);
       }
       __syncwarp();
@@ -310,7 +292,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     if (ok) ok = wait_or_abort(&s.full[0], 0, abort_flag);
     if (ok) {
       ptx::tc_fence_after();
-      copy_q(0);
       mma2(0);
       mma3(0);
       ok = wait_or_abort(&s.w_done, 0, abort_flag);
@@ -324,26 +305,24 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const uint64_t so = (uint64_t)st * STG;
       const uint32_t par = (uint32_t)(n & 1);
       const bool more = n + 1 < nchunks;
-      // ---- MMA 4 (chunk n): needs [W(n); Q(n)] in TMEM and h_n (D_H of
-      //      n-1 read)
+      // ---- MMA 4 (chunk n): needs W(n) and h_n (D_H of n-1 read)
       if (!wait_or_abort(&s.w_done, par, abort_flag)) break;
       if (!wait_or_abort(&s.h_done, par, abort_flag)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
-          ptx::mma_bf16_ta(tb + COL_U + 64 * st, tA + 8 * kk, dH + kk * KSTEP_MN, id_x, 1);
+          ptx::mma_bf16(tb + COL_U + 64 * st, dWQ + so + (kk >> 2) * PNL + (kk & 3) * KSTEP_K,
+                        dH + kk * KSTEP_MN, id_x, 1);
         ptx::mma_commit(&s.bX);
       }
       __syncwarp();
-      // ---- while V'(n) is formed: Q(n+1) into TMEM (MMA 4 of n, the last
-      //      reader of [W; Q](n), is ahead of it in the pipe) and W of chunk
-      //      n+1 (needed by its MMA 4; D_W was read before w_done(n))
+      // ---- while V'(n) is formed: W of chunk n+1 (needed by its MMA 4);
+      //      D_W was read before w_done(n)
       if (more) {
         if (!wait_or_abort(&s.full[(n + 1) & 1], (uint32_t)(((n + 1) >> 1) & 1), abort_flag))
           break;
         ptx::tc_fence_after();
-        copy_q(n + 1);
         mma2(n + 1);
       }
       // ---- MMA 5 (state), committed on its own so the update starts at once
@@ -376,8 +355,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           break;
         ptx::tc_fence_after();
         mma3(n + 1);
-        // ... and Q K^T of chunk n+1: D_S was read by P(n) (waited above),
-        // [W(n+1); Q(n+1)] is in TMEM
+        // ... and Q K^T of chunk n+1: D_S was read by P(n) (waited above);
+        // waiting for W(n+1) keeps its rows from changing under the read
         if (!wait_or_abort(&s.w_done, par ^ 1u, abort_flag)) break;
         ptx::tc_fence_after();
         mma1(n + 1);
@@ -389,22 +368,21 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     wait_bounded(&s.mma_drain, 0);
   } else if (warp == 4 || warp == 5) {
     // ===================== next-chunk epilogue: W =========================
-    // W rows 0..63 (TMEM lanes 0..63) -> packed bf16 -> [W; Q] in TMEM
+    // W rows 0..63 (TMEM lanes 0..63) -> the stage's W slot (bf16)
     for (int n = 0; n < nchunks; ++n) {
+      Stage<DK>& S = s.st[n & 1];
       if (!wait_or_abort(&s.bW, (uint32_t)(n & 1), abort_flag)) break;
       ptx::tc_fence_after();
 #pragma unroll
       for (int p = 0; p < NP; ++p) {
-        uint32_t pk[32];
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           float w[32];
           ptx::tmem_ld32(tb + lane_base + COL_W + p * 64 + 32 * hf, w);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[16 * hf + i] = pack_bf16x2(w[2 * i], w[2 * i + 1]);
+          sw128_store_row32(S.panel[p][SW], row, hf, w);
         }
-        ptx::tmem_st32(tb + lane_base + COL_A + 32 * p, pk);
       }
+      ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.w_done);

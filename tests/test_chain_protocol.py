@@ -65,14 +65,13 @@ def build(N):
         prod.append(("tma", n))
     roles["producer"] = prod
 
-    m = [W(("full", 0), 0), I("cpq", 0), I("mma2", 0), Cm("bW"), I("mma3", 0),
+    m = [W(("full", 0), 0), I("mma2", 0), Cm("bW"), I("mma3", 0),
          W("w_done", 0), I("mma1", 0), Cm("bS")]
     for n in range(N):
         more = n + 1 < N
         m += [W("w_done", n), W("h_done", n), I("mma4", n), Cm("bX")]
         if more:
-            m += [W(("full", (n + 1) & 1), (n + 1) >> 1), I("cpq", n + 1), I("mma2", n + 1),
-                  Cm("bW")]
+            m += [W(("full", (n + 1) & 1), (n + 1) >> 1), I("mma2", n + 1), Cm("bW")]
         m += [W("vp_ready", n), I("mma5", n), Cm("bH"), W("p_done", n)]
         if n > 0:
             m.append(W("pv_free", n - 1))
@@ -162,10 +161,8 @@ def run(N, seed):
             raise Hazard(f"V'({n}) overwrites vp/vpd while MMA 5/6 of {n - 1} may read them")
         if tag == "h" and not {("mma4", n), ("mma5", n)} <= done_mma:
             raise Hazard(f"h_{n + 1} written while MMA 4 of {n} may read h_{n}")
-        if tag == "W" and n >= 1 and ("mma4", n - 1) not in done_mma:
-            raise Hazard(f"W({n}) overwrites [W; Q] while MMA 4 of {n - 1} may read it")
-        if tag == "W" and ("cpq", n) not in done_mma:
-            raise Hazard(f"W({n}) written before the copy of [K; Q]({n}) that it overwrites")
+        if tag == "W" and n >= 2 and not {("mma4", n - 2), ("mma1", n - 2)} <= done_mma:
+            raise Hazard(f"W({n}) overwrites the W slot while chunk {n - 2} may read it")
         if tag == "P" and n >= 2 and ("mma6", n - 2) not in done_mma:
             raise Hazard(f"P({n}) overwrites the P slot of chunk {n - 2} in use")
         if tag == "P" and ("mma1", n) not in done_mma:
