@@ -34,8 +34,8 @@
 // that the row a thread holds is a row of the next operand: every
 // shared-memory write is a whole swizzled row.  The decays e^{G_s - G_r} are
 // running products of alpha_j = e^{g_j} over r < j <= s (every factor <= 1).
-// Two 16 KB operand tiles and the key tile are all the shared memory a CTA
-// needs, so three CTAs share an SM; each is persistent over pairs of chunks
+// The key tile and one 16 KB operand tile are all the shared memory a CTA
+// needs, so four CTAs share an SM; each is persistent over pairs of chunks
 // and fetches the next pair's keys and gates while it works.
 //
 // The factors are written to global memory already in the 128-byte swizzled
@@ -52,19 +52,24 @@ namespace {
 
 constexpr int C = 64;
 constexpr int NT = 128;
-constexpr int CTAS_PER_SM = 3;
+constexpr int CTAS_PER_SM = 4;
 constexpr uint32_t TILE = 128 * 64 * 2;  // one bf16 operand tile: 128 rows x 64 (16 KB)
+
+// Diagonal 16x16 blocks of A ([row][column], padded), later the same blocks
+// of D; kept in the second tile of r0, which is idle from the Gram MMA until
+// the next pair's keys arrive.
+typedef float DiagBlocks[2][4][16][17];
+static_assert(sizeof(DiagBlocks) <= TILE, "diagonal blocks fit one tile");
 
 template <int DK>
 struct alignas(1024) UtSmem {
   static constexpr int NP = DK / 64;
+  static constexpr int R0_TILES = NP < 2 ? 2 : NP;
   // keys (per 64-column panel: chunk 0 rows then chunk 1 rows); after the
-  // Gram MMA its first tile holds A_O^T, then N (B operands)
-  uint8_t r0[NP * TILE];
+  // Gram MMA its first tile holds A_O^T, then N (B operands), its second
+  // tile the diagonal blocks
+  uint8_t r0[R0_TILES * TILE];
   uint8_t r1[TILE];  // D (A operand of N), then X_i^T (Horner A operands)
-  // diagonal 16x16 blocks of A, [row][column]; after the solve the same
-  // blocks of D
-  float adiag[2][4][16][17];
   float G[2][C];
   float beta[2][C];
   float alpha[2][C];
@@ -81,6 +86,17 @@ __device__ __forceinline__ void issue_product(uint32_t d, const uint8_t* at, con
                   ptx::sdesc_sw128(ptx::smem_u32(bt) + kk * 32, 16, 1024), id, kk > 0);
 }
 
+// Column half hf (32 values) of a 64-wide row that is zero outside the 16
+// values x of block bb.
+__device__ __forceinline__ void block_half(float* v, const float* x, int bb, int hf) {
+  const bool lo = (bb >> 1) == hf && !(bb & 1), hi = (bb >> 1) == hf && (bb & 1);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    v[i] = lo ? x[i] : 0.f;
+    v[16 + i] = hi ? x[i] : 0.f;
+  }
+}
+
 template <int DK>
 __global__ void __launch_bounds__(NT, CTAS_PER_SM)
 ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
@@ -91,6 +107,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                      ~uintptr_t(1023));
+  DiagBlocks& adiag = *reinterpret_cast<DiagBlocks*>(s.r0 + TILE);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = tid >> 6, r = tid & 63;  // chunk slot and its row
   const int npairs = (total_chunks + 1) / 2;
@@ -150,10 +167,9 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
     mma_phase ^= 1u;
     ptx::tc_fence_after();
   };
-  // row `R` of the accumulator's diagonal block for my chunk
-  auto ld_row = [&](float* v) {
-    ptx::tmem_ld32(tacc + lane_base + j * 64, v);
-    ptx::tmem_ld32(tacc + lane_base + j * 64 + 32, v + 32);
+  // column half hf of row t of the accumulator's diagonal block (my chunk)
+  auto ld_half = [&](int hf, float* v) {
+    ptx::tmem_ld32(tacc + lane_base + j * 64 + 32 * hf, v);
   };
 
   uint32_t tma_phase = 0;
@@ -206,37 +222,40 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
     // A_sr = beta_s (k_s . k_r) e^{G_s - G_r}, the decay a running product of
     // alpha_s from s = r + 1 on (every factor <= 1).  The Gram matrix is
     // symmetric, so row r of it is also column r.  Column r of A_O is row r
-    // of A_O^T (B operand of N = D A_O, -> r0: the keys are dead); the
-    // entries inside my diagonal block go to adiag.
+    // of A_O^T (B operand of N = D A_O, -> first tile of r0: the keys are
+    // dead); the entries inside my diagonal block go to adiag.
     const int bb = r >> 4;  // my 16-row block
     const int cq = r & 15;  // my position inside it
     {
-      float srow[64];
-      ld_row(srow);
+      float v[32];
+      ld_half(r >> 5, v);
       float diag = 0.f;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) diag = (c == r) ? srow[c] : diag;
+      for (int c = 0; c < 32; ++c) diag = (c == (r & 31)) ? v[c] : diag;
       s.beta[j][r] = er / (diag + eps);
-      ptx::tc_fence_before();
-      __syncthreads();  // beta complete; every thread has read the Gram row
+      __syncthreads();  // beta complete
       float d = 1.f;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        d = (c > r) ? d * s.alpha[j][c] : d;
-        srow[c] = (c > r) ? s.beta[j][c] * srow[c] * d : 0.f;
+      for (int hf = 0; hf < 2; ++hf) {
+        ld_half(hf, v);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int sc = 32 * hf + c;
+          d = (sc > r) ? d * s.alpha[j][sc] : d;
+          v[c] = (sc > r) ? s.beta[j][sc] * v[c] * d : 0.f;
+        }
+        if ((bb >> 1) == hf) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            adiag[j][bb][i][cq] = (bb & 1) ? v[16 + i] : v[i];  // A_bb[i][cq]
+            if (bb & 1) v[16 + i] = 0.f; else v[i] = 0.f;
+          }
+        }
+        sw128_store_row32(s.r0, tid, hf, v);
       }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float v = 0.f;
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) v = (blk == bb) ? srow[16 * blk + i] : v;
-        s.adiag[j][bb][i][cq] = v;  // A_bb[i][cq]
-      }
-#pragma unroll
-      for (int c = 0; c < 64; ++c) srow[c] = ((c >> 4) == bb) ? 0.f : srow[c];
-      sw128_store_row(s.r0, tid, srow);
     }
-    __syncthreads();
+    ptx::tc_fence_before();
+    __syncthreads();  // every thread has read the Gram row; A_O^T, A_D complete
 
     // ---- D = (I + A_D)^{-1}: thread r solves column cq of (I + A_bb)^{-1}
     // by forward substitution and keeps it (it is row r of D^T); rows of D
@@ -247,18 +266,22 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
     for (int i = 0; i < 16; ++i) {
       float acc = 0.f;
 #pragma unroll
-      for (int m = 0; m < i; ++m) acc = fmaf(s.adiag[j][bb][i][m], x[m], acc);
+      for (int m = 0; m < i; ++m) acc = fmaf(adiag[j][bb][i][m], x[m], acc);
       x[i] = (i == cq) ? 1.f : (i < cq ? 0.f : -acc);
     }
     __syncthreads();  // every solve has read A_D
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s.adiag[j][bb][i][cq] = x[i];
+    for (int i = 0; i < 16; ++i) adiag[j][bb][i][cq] = x[i];
     __syncthreads();
     {
-      float v[64];
+      float y[16], v[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) v[c] = ((c >> 4) == bb) ? s.adiag[j][bb][cq][c & 15] : 0.f;
-      sw128_store_row(s.r1, tid, v);
+      for (int i = 0; i < 16; ++i) y[i] = adiag[j][bb][cq][i];
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        block_half(v, y, bb, hf);
+        sw128_store_row32(s.r1, tid, hf, v);
+      }
     }
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
@@ -273,13 +296,13 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
       ptx::mma_commit(&s.bar_mma);
     }
     mma_done();
-    {
-      float v[64];
-      ld_row(v);
-      sw128_store_row(s.r0, tid, v);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) v[c] = ((c >> 4) == bb) ? x[c & 15] : 0.f;
-      sw128_store_row(s.r1, tid, v);
+    for (int hf = 0; hf < 2; ++hf) {
+      float v[32];
+      ld_half(hf, v);
+      sw128_store_row32(s.r0, tid, hf, v);
+      block_half(v, x, bb, hf);
+      sw128_store_row32(s.r1, tid, hf, v);
     }
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
@@ -287,9 +310,8 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
 
     // ---- Horner on the transposes: X_0 = D, X_{i+1}^T = D^T - X_i^T N^T, so
     // lane t of each product is row r of X_{i+1}^T, the next A operand row as
-    // is (written in place: the product that read r1 has finished).  T^T =
-    // X_3^T stays in registers (row r of T^T = column r of T).
-    float trow[64];
+    // is (written in place: the product that read r1 has finished).  The
+    // last one, row r of T^T = column r of T, goes straight to the outputs.
 #pragma unroll 1
     for (int step = 0; step < 3; ++step) {
       if (tid == 0 && ok) {
@@ -298,20 +320,25 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
         ptx::mma_commit(&s.bar_mma);
       }
       mma_done();
-      // the last product has read r0: the next pair's keys may land there
-      if (step == 2 && tid == 0 && ok && pair + (int)gridDim.x < npairs) {
-        load_keys(pair + gridDim.x);
-        keys_in_flight = true;
-      }
-      ld_row(trow);
-#pragma unroll
-      for (int c = 0; c < 64; ++c) trow[c] = (((c >> 4) == bb) ? x[c & 15] : 0.f) - trow[c];
       if (step < 2) {
-        sw128_store_row(s.r1, tid, trow);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32], dc[32];
+          ld_half(hf, v);
+          block_half(dc, x, bb, hf);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) v[c] = dc[c] - v[c];
+          sw128_store_row32(s.r1, tid, hf, v);
+        }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncthreads();
       }
+    }
+    // the last product has read r0: the next pair's keys may land there
+    if (tid == 0 && ok && pair + (int)gridDim.x < npairs) {
+      load_keys(pair + gridDim.x);
+      keys_in_flight = true;
     }
 
     // ---- outputs: row r of T'^T = beta_r (column r of T) and row r of
@@ -320,22 +347,26 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
       const float b1 = s.beta[j][r], b2 = b1 * __expf(s.G[j][r]);
       uint8_t* dst = ws + (size_t)ci * kUtTileBytes;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 u;
-        u.x = pack_bf16x2(b1 * trow[8 * c + 0], b1 * trow[8 * c + 1]);
-        u.y = pack_bf16x2(b1 * trow[8 * c + 2], b1 * trow[8 * c + 3]);
-        u.z = pack_bf16x2(b1 * trow[8 * c + 4], b1 * trow[8 * c + 5]);
-        u.w = pack_bf16x2(b1 * trow[8 * c + 6], b1 * trow[8 * c + 7]);
-        *reinterpret_cast<uint4*>(dst + sw128_chunk_off(r, c)) = u;
-      }
+      for (int hf = 0; hf < 2; ++hf) {
+        float v[32], dc[32];
+        ld_half(hf, v);
+        block_half(dc, x, bb, hf);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 u;
-        u.x = pack_bf16x2(b2 * trow[8 * c + 0], b2 * trow[8 * c + 1]);
-        u.y = pack_bf16x2(b2 * trow[8 * c + 2], b2 * trow[8 * c + 3]);
-        u.z = pack_bf16x2(b2 * trow[8 * c + 4], b2 * trow[8 * c + 5]);
-        u.w = pack_bf16x2(b2 * trow[8 * c + 6], b2 * trow[8 * c + 7]);
-        *reinterpret_cast<uint4*>(dst + 8192 + sw128_chunk_off(r, c)) = u;
+        for (int c = 0; c < 32; ++c) v[c] = dc[c] - v[c];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 u;
+          u.x = pack_bf16x2(b1 * v[8 * c + 0], b1 * v[8 * c + 1]);
+          u.y = pack_bf16x2(b1 * v[8 * c + 2], b1 * v[8 * c + 3]);
+          u.z = pack_bf16x2(b1 * v[8 * c + 4], b1 * v[8 * c + 5]);
+          u.w = pack_bf16x2(b1 * v[8 * c + 6], b1 * v[8 * c + 7]);
+          *reinterpret_cast<uint4*>(dst + sw128_chunk_off(r, 4 * hf + c)) = u;
+          u.x = pack_bf16x2(b2 * v[8 * c + 0], b2 * v[8 * c + 1]);
+          u.y = pack_bf16x2(b2 * v[8 * c + 2], b2 * v[8 * c + 3]);
+          u.z = pack_bf16x2(b2 * v[8 * c + 4], b2 * v[8 * c + 5]);
+          u.w = pack_bf16x2(b2 * v[8 * c + 6], b2 * v[8 * c + 7]);
+          *reinterpret_cast<uint4*>(dst + 8192 + sw128_chunk_off(r, 4 * hf + c)) = u;
+        }
       }
     }
     gr = gn;
