@@ -98,7 +98,7 @@ struct alignas(1024) ChainSmem {
   alignas(16) float alpha[3][C];  // e^{g_s} of chunk n in slot n % 3
   uint64_t full[2], empty[2];
   uint64_t bS, bW, bX, bH, bHP;          // MMA completions
-  uint64_t p_done, w_done, vp_ready;
+  uint64_t p_done, w_done, vpd_ready, vp_ready;
   uint64_t u_free[2], h_done, pv_free;
   uint64_t g_ready[3];
   uint64_t mma_drain;
@@ -175,6 +175,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     ptx::mbar_init(&s.bHP, 1);
     ptx::mbar_init(&s.p_done, 4);
     ptx::mbar_init(&s.w_done, 2);
+    ptx::mbar_init(&s.vpd_ready, 4);
     ptx::mbar_init(&s.vp_ready, 4);
     ptx::mbar_init(&s.h_done, 8);
     ptx::mbar_init(&s.pv_free, 4);
@@ -326,7 +327,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         mma2(n + 1);
       }
       // ---- MMA 5 (state), committed on its own so the update starts at once
-      if (!wait_or_abort(&s.vp_ready, par, abort_flag)) break;
+      if (!wait_or_abort(&s.vpd_ready, par, abort_flag)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
@@ -335,7 +336,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         ptx::mma_commit(&s.bH);
       }
       __syncwarp();
-      // ---- MMA 6 (chunk n): needs P(n) and D_PV free (outputs of n-1 read)
+      // ---- MMA 6 (chunk n): needs V'(n), P(n) and D_PV free (outputs of n-1
+      //      read)
+      if (!wait_or_abort(&s.vp_ready, par, abort_flag)) break;
       if (!wait_or_abort(&s.p_done, par, abort_flag)) break;
       if (n > 0 && !wait_or_abort(&s.pv_free, par ^ 1u, abort_flag)) break;
       ptx::tc_fence_after();
@@ -494,19 +497,23 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const float dec = __expf(gC - Gn[row]);
         if (!wait_or_abort(&s.bX, par, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
-        float u[32];
+        float u[32], ud[32];
         ptx::tmem_ld32(tb + lane_base + col_u + cg, u);
-        sw128_store_row32(s.vp, row, grp, u);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) u[j] *= dec;
-        sw128_store_row32(s.vpd, row, grp, u);
         ptx::tc_fence_before();
+        // the decayed copy first: it feeds MMA 5, the next link of the chain
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ud[j] = u[j] * dec;
+        sw128_store_row32(s.vpd, row, grp, ud);
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&s.vp_ready);
+          mbar_arrive(&s.vpd_ready);
           mbar_arrive(&s.u_free[n & 1]);
         }
+        sw128_store_row32(s.vp, row, grp, u);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.vp_ready);
       }
       // every read of G(n) happens before this warp's last arrival of chunk n
       const float e_out = v_rows ? 0.f : -__expf(Gn[row - 64]);

@@ -47,7 +47,7 @@ def build(N):
     for i in range(3):
         B(("g_ready", i), 1)
     for name, c in [("bS", 1), ("bW", 1), ("bX", 1), ("bH", 1), ("bHP", 1), ("p_done", 4),
-                    ("w_done", 2), ("vp_ready", 4), ("h_done", 8),
+                    ("w_done", 2), ("vpd_ready", 4), ("vp_ready", 4), ("h_done", 8),
                     ("pv_free", 4)]:
         B(name, c)
 
@@ -72,7 +72,7 @@ def build(N):
         m += [W("w_done", n), W("h_done", n), I("mma4", n), Cm("bX")]
         if more:
             m += [W(("full", (n + 1) & 1), (n + 1) >> 1), I("mma2", n + 1), Cm("bW")]
-        m += [W("vp_ready", n), I("mma5", n), Cm("bH"), W("p_done", n)]
+        m += [W("vpd_ready", n), I("mma5", n), Cm("bH"), W("vp_ready", n), W("p_done", n)]
         if n > 0:
             m.append(W("pv_free", n - 1))
         m += [I("mma6", n), Cm("bHP"), Cm(("empty", n & 1))]
@@ -102,7 +102,8 @@ def build(N):
         for n in range(N):
             seq += [W(("g_ready", n % 3), n // 3), Do("readG", n)]
             if v_rows:
-                seq += [W("bX", n), Do("Vp", n), A("vp_ready"), A(("u_free", n & 1))]
+                seq += [W("bX", n), Do("Vpd", n), A("vpd_ready"), A(("u_free", n & 1)),
+                        Do("Vp", n), A("vp_ready")]
             seq += [W("bH", n), Do("h", n), A("h_done")]
             if not v_rows:
                 seq += [W("bHP", n), Do("o", n), A(("u_free", n & 1)), A("pv_free")]
@@ -146,7 +147,7 @@ def run(N, seed):
             if n >= 1 and not finished("h", n - 1, 8):
                 raise Hazard(f"MMA 4 of {n} before h_{n} is written")
         if tag == "mma5":
-            if not finished("Vp", n, 4):
+            if not finished("Vpd", n, 4):
                 raise Hazard(f"MMA 5 of {n} before V'({n})")
             if n >= 1 and not finished("h", n - 1, 8):
                 raise Hazard(f"D_H of {n} overwritten before chunk {n - 1} read it")
@@ -157,8 +158,10 @@ def run(N, seed):
                 raise Hazard(f"D_PV of {n} overwritten before chunk {n - 1} read it")
 
     def check_do(tag, n):
-        if tag == "Vp" and n >= 1 and not {("mma5", n - 1), ("mma6", n - 1)} <= done_mma:
-            raise Hazard(f"V'({n}) overwrites vp/vpd while MMA 5/6 of {n - 1} may read them")
+        if tag == "Vpd" and n >= 1 and ("mma5", n - 1) not in done_mma:
+            raise Hazard(f"V'({n}) overwrites vpd while MMA 5 of {n - 1} may read it")
+        if tag == "Vp" and n >= 1 and ("mma6", n - 1) not in done_mma:
+            raise Hazard(f"V'({n}) overwrites vp while MMA 6 of {n - 1} may read it")
         if tag == "h" and not {("mma4", n), ("mma5", n)} <= done_mma:
             raise Hazard(f"h_{n + 1} written while MMA 4 of {n} may read h_{n}")
         if tag == "W" and n >= 2 and not {("mma4", n - 2), ("mma1", n - 2)} <= done_mma:

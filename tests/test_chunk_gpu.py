@@ -126,3 +126,46 @@ def test_matches_token_serial_all_heads_4k():
     o2, h2 = api.recurrent_fwd(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"])
     torch.cuda.synchronize()
     assert rel(o1, o2) < TOL and rel(h1, h2) < TOL
+
+
+def _degenerate(w, seed):
+    """Inputs of workload ``w`` with degenerate tokens mixed in: zero keys
+    (beta = eta / eps), eta = 0 (pure decay), g = 0 (no decay), a forget
+    strong enough to wipe the state (g = -40), zero queries and values."""
+    x = inputs.make_prefill(w)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    B, T, H = x["g"].shape
+    pick = lambda p: torch.from_numpy(rng.random((B, T, H)) < p)
+    zk, ze, zg, wipe, zq, zv = (pick(p) for p in (0.05, 0.05, 0.1, 0.01, 0.05, 0.05))
+    x["k"][zk] = 0
+    x["q"][zq] = 0
+    x["v"][zv] = 0
+    x["eta"][ze] = 0.0
+    x["g"][zg] = 0.0
+    x["g"][wipe] = -40.0
+    return x
+
+
+@pytest.mark.parametrize("name,T", [("prefill_4k", 300), ("stress", 257)])
+def test_degenerate_tokens(name, T):
+    w = W[name].scaled(B=1, T=T, H=2)
+    x = _degenerate(w, 7)
+    xc = cuda(x)
+    o, hT = api.chunk_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"], xc["h0"])
+    api.check_device_error()
+    o_ref, h_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"])
+    assert np.isfinite(oracle.f64(o.cpu())).all() and np.isfinite(oracle.f64(hT.cpu())).all()
+    assert rel(o.cpu(), o_ref) < TOL and rel(hT.cpu(), h_ref) < TOL
+
+
+def test_all_keys_zero_is_pure_decay():
+    """Every key zero: no write ever lands, h_T = e^{sum g} h0 exactly as the
+    recurrence says, and o_t = e^{G_t} h0^T q_t."""
+    w = W["stress"].scaled(B=1, T=130, H=2)
+    x = inputs.make_prefill(w)
+    x["k"].zero_()
+    xc = cuda(x)
+    o, hT = api.chunk_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"], xc["h0"])
+    api.check_device_error()
+    o_ref, h_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"])
+    assert rel(o.cpu(), o_ref) < TOL and rel(hT.cpu(), h_ref) < TOL

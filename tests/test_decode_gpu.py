@@ -61,3 +61,27 @@ def test_decode_fp32_tight():
     w = inputs.DECODE.scaled(B=4, H=4, dtype="fp32", prefix_tokens=32)
     eo, eS, edS = _run(w, 20, "fp32")
     assert eo < 1e-4 and eS < 1e-4 and edS < 1e-4, (eo, eS, edS)
+
+
+def test_decode_degenerate_tokens():
+    """Zero keys (beta = eta / eps: no write lands), eta = 0 (pure decay),
+    g = 0 (no decay) and g = -40 (the state is wiped), per (b, h)."""
+    w = inputs.DECODE.scaled(B=4, H=4, prefix_tokens=32)
+    d = inputs.make_decode(w, steps=4)
+    st = d["steps"]
+    st["k"][0, 0] = 0
+    st["eta"][1, 1] = 0.0
+    st["g"][2, 2] = 0.0
+    st["g"][3, 3] = -40.0
+    S0 = oracle_decode_state(d)
+    S = cuda(S0.clone())
+    Sref = oracle.f64(S0)
+    for i in range(4):
+        q, k, v, g, e = (cuda(st[n][i]) for n in ("q", "k", "v", "g", "eta"))
+        o = api.decode_step(q, k, v, g, e, S, eps=d["eps"])
+        o_ref, Sref = oracle.decode_step(st["q"][i], st["k"][i], st["v"][i], st["g"][i],
+                                         st["eta"][i], d["eps"], Sref)
+        assert np.isfinite(oracle.f64(o)).all()
+        assert rel(o, o_ref) < TOL["bf16"]
+    torch.cuda.synchronize()
+    assert rel(S, Sref) < TOL["bf16"]
