@@ -23,6 +23,10 @@ SIGNATURES = {
                                  _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_recurrent_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
                                _i, _i, _i, _i, _i, _i, _vp]),
+    "kla_gdn_chunk_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                               _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_gdn_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _i, _i, _i, _i, _i, _vp]),
     "kla_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp,
                              _i, _i, _i, _i, _i, _vp]),
     "kla_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,

@@ -167,6 +167,45 @@ def decode_step(q, k, v, g, eta, S, eps: float = 1e-6, *, o=None, stream=None):
     return o
 
 
+def gdn_chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, hT=None, return_state: bool = True,
+                  workspace=None, stream=None):
+    """Gated DeltaNet prefill (kla_gdn_chunk_fwd): beta [B,T,H] fp32 is the
+    step size itself.  Returns (o, hT)."""
+    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, beta, h0, o, hT, return_state)
+    need = chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _native.lib().kla_gdn_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT),
+        B, T, H, dk, dv, CHUNK, _DT[q.dtype], _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "kla_gdn_chunk_fwd")
+    return o, hT
+
+
+def gdn_decode_step(q, k, v, g, beta, S, *, o=None, stream=None):
+    """One Gated DeltaNet decode token per sequence (kla_gdn_decode_step);
+    S is updated in place.  Returns o [B,H,dv]."""
+    _need(q, "q")
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v must be bfloat16 or float32")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", q.dtype, (B, H, dk))
+    _need(v, "v", q.dtype, (B, H, dv))
+    _need(g, "g", torch.float32, (B, H))
+    _need(beta, "beta", torch.float32, (B, H))
+    _need(S, "S", torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, (B, H, dv))
+    st = _native.lib().kla_gdn_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o), B, H, dk, dv,
+        _DT[q.dtype], _stream(stream))
+    _check(st, "kla_gdn_decode_step")
+    return o
+
+
 def check_device_error(stream=None):
     """Synchronise and raise KLAError if a kernel reported a timed-out wait."""
     _check(_native.lib().kla_check_device_error(_stream(stream)), "kla_check_device_error")

@@ -96,12 +96,16 @@ size_t kla_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int dty
   return chunk_workspace_bytes(B, T, H, dk, dv, dtype);
 }
 
-kla_status kla_chunk_fwd(const void* q, const void* k, const void* v,
-                         const float* g, const float* eta, float eps,
-                         const float* h0, void* o, float* hT, int B, int T, int H,
-                         int dk, int dv, int chunk, int dtype, void* workspace,
-                         size_t ws_bytes, void* stream) {
-  kla_status s = check_prefill(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype);
+}  // extern "C"
+
+// Prefill with the KLA step size, or (eps == kBetaGiven) with beta given.
+static kla_status chunk_fwd_impl(const void* q, const void* k, const void* v,
+                                 const float* g, const float* eta, float eps,
+                                 const float* h0, void* o, float* hT, int B, int T, int H,
+                                 int dk, int dv, int chunk, int dtype, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  kla_status s = check_prefill(q, k, v, g, eta, eps < 0.f ? 0.f : eps, h0, o, hT, B, T, H,
+                               dk, dv, dtype);
   if (s != KLA_OK) return s;
   if (chunk != KLA_CHUNK) return KLA_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
@@ -120,6 +124,26 @@ kla_status kla_chunk_fwd(const void* q, const void* k, const void* v,
     if (e == cudaErrorNotSupported) return KLA_ERR_UNSUPPORTED;
   }
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+extern "C" {
+
+kla_status kla_chunk_fwd(const void* q, const void* k, const void* v,
+                         const float* g, const float* eta, float eps,
+                         const float* h0, void* o, float* hT, int B, int T, int H,
+                         int dk, int dv, int chunk, int dtype, void* workspace,
+                         size_t ws_bytes, void* stream) {
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  return chunk_fwd_impl(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, chunk, dtype,
+                        workspace, ws_bytes, stream);
+}
+
+kla_status kla_gdn_chunk_fwd(const void* q, const void* k, const void* v,
+                             const float* g, const float* beta, const float* h0, void* o,
+                             float* hT, int B, int T, int H, int dk, int dv, int chunk,
+                             int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  return chunk_fwd_impl(q, k, v, g, beta, kBetaGiven, h0, o, hT, B, T, H, dk, dv, chunk, dtype,
+                        workspace, ws_bytes, stream);
 }
 
 // Shared checks of the two prefill stages (bf16 chunk path only).
@@ -193,13 +217,15 @@ kla_status kla_recurrent_fwd(const void* q, const void* k, const void* v,
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
 
-kla_status kla_decode_step(const void* q, const void* k, const void* v,
-                           const float* g, const float* eta, float eps, float* S,
-                           void* o, int B, int H, int dk, int dv, int dtype,
-                           void* stream) {
+}  // extern "C"
+
+// One decode step with the KLA step size, or (eps == kBetaGiven) beta given.
+static kla_status decode_impl(const void* q, const void* k, const void* v,
+                              const float* g, const float* eta, float eps, float* S,
+                              void* o, int B, int H, int dk, int dv, int dtype,
+                              void* stream) {
   if (B < 1 || H < 1) return KLA_ERR_INVALID_ARG;
   if (dtype != KLA_BF16 && dtype != KLA_FP32) return KLA_ERR_INVALID_ARG;
-  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, g, eta, S, o};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return KLA_ERR_INVALID_ARG;
@@ -214,6 +240,22 @@ kla_status kla_decode_step(const void* q, const void* k, const void* v,
   cudaError_t e = launch_decode(q, k, v, g, eta, eps, S, o, B, H, dk, dv, dtype,
                                 (cudaStream_t)stream);
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+extern "C" {
+
+kla_status kla_decode_step(const void* q, const void* k, const void* v,
+                           const float* g, const float* eta, float eps, float* S,
+                           void* o, int B, int H, int dk, int dv, int dtype,
+                           void* stream) {
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  return decode_impl(q, k, v, g, eta, eps, S, o, B, H, dk, dv, dtype, stream);
+}
+
+kla_status kla_gdn_decode_step(const void* q, const void* k, const void* v,
+                               const float* g, const float* beta, float* S, void* o, int B,
+                               int H, int dk, int dv, int dtype, void* stream) {
+  return decode_impl(q, k, v, g, beta, kBetaGiven, S, o, B, H, dk, dv, dtype, stream);
 }
 
 kla_status kla_check_device_error(void* stream) {

@@ -18,6 +18,15 @@ __device__ __forceinline__ void report_timeout(unsigned int* err) {
   atomicOr(err, KLA_DEVERR_TIMEOUT);
 }
 
+// eps value that selects the gated-delta form inside the kernels: beta_t is
+// then the per-token input itself (the `eta` argument) instead of
+// eta_t / (||k_t||^2 + eps).  The C ABI never passes a negative eps otherwise.
+constexpr float kBetaGiven = -1.0f;
+
+__device__ __forceinline__ float step_size(float eta, float knorm2, float eps) {
+  return eps < 0.f ? eta : eta / (knorm2 + eps);
+}
+
 // Launchers (one per kernel family), all queue work on `st` only.
 cudaError_t launch_decode(const void* q, const void* k, const void* v,
                           const float* g, const float* eta, float eps, float* S,

@@ -91,7 +91,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k,
   __syncthreads();
 
   const float alpha = expf(g[head]);
-  const float beta = eta[head] / (kq_sh[0] + eps);
+  const float beta = step_size(eta[head], kq_sh[0], eps);
   if (tid < CW) {
     float r = 0.f, s = 0.f;
 #pragma unroll

@@ -67,7 +67,7 @@ recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k,
     r += __shfl_xor_sync(0xffffffffu, r, 8);
     r += __shfl_xor_sync(0xffffffffu, r, 16);
     const float alpha = expf(gt);
-    const float beta = et / (n2 + eps);
+    const float beta = step_size(et, n2, eps);
     const float u = beta * (vj - alpha * r);
     float s = 0.f;
 #pragma unroll

@@ -232,7 +232,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
       float diag = 0.f;
 #pragma unroll
       for (int c = 0; c < 32; ++c) diag = (c == (r & 31)) ? v[c] : diag;
-      s.beta[j][r] = er / (diag + eps);
+      s.beta[j][r] = step_size(er, diag, eps);
       __syncthreads();  // beta complete
       float d = 1.f;
 #pragma unroll

@@ -148,6 +148,26 @@ KLA_API kla_status kla_decode_step(const void *q, const void *k, const void *v,
                            int dtype, void *stream);
 
 /*
+ * Gated DeltaNet form: the same recurrence with the step size beta_t given
+ * per token instead of derived from the key norm ("Deep Dive into KDA",
+ * section 2.2; "Kaczmarz Linear Attention", Abstract, describes KLA as this
+ * rule with beta_t = eta_t / (||k_t||^2 + eps)).  Arguments, layouts, limits
+ * and errors are those of kla_chunk_fwd / kla_decode_step with `beta`
+ * ([B][T][H] resp. [B][H] fp32, any real value) in place of eta and no eps;
+ * the workspace size is kla_chunk_fwd_workspace_size's.  Runs the same
+ * kernels.
+ */
+KLA_API kla_status kla_gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                             const float *g, const float *beta, const float *h0,
+                             void *o, float *hT, int B, int T, int H, int dk, int dv,
+                             int chunk, int dtype, void *workspace, size_t ws_bytes,
+                             void *stream);
+
+KLA_API kla_status kla_gdn_decode_step(const void *q, const void *k, const void *v,
+                               const float *g, const float *beta, float *S, void *o,
+                               int B, int H, int dk, int dv, int dtype, void *stream);
+
+/*
  * Chunkwise prefill without any caller-provided device memory.
  *
  * No counterpart in the paper: this is a deployment convenience.  Some

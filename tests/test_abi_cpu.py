@@ -85,6 +85,24 @@ def test_prefill_stages_reject_bad_arguments(lib):
     assert st(dtype=1) == UNSUPPORTED
 
 
+def test_gdn_entry_points_reject_bad_arguments(lib):
+    gdn = lambda **kw: lib.kla_gdn_chunk_fwd(
+        kw.get("q", A), kw.get("k", 2 * A), kw.get("v", 3 * A), kw.get("g", 4 * A),
+        kw.get("beta", 5 * A), None, kw.get("o", 6 * A), None, 1, kw.get("T", 128), 2,
+        kw.get("dk", 128), kw.get("dv", 128), kw.get("chunk", 64), kw.get("dtype", 0),
+        None, 0, None)
+    assert gdn(beta=None) == INVALID
+    assert gdn(o=A + 256) == INVALID                   # o overlaps q
+    assert gdn(dk=96, dv=96) == UNSUPPORTED
+    assert gdn(chunk=32) == UNSUPPORTED
+    assert gdn(dtype=0) == INVALID                     # bf16 needs a workspace
+    args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 7 * A, 2, 3, 128, 128, 0, None]
+    bad = list(args); bad[4] = None
+    assert lib.kla_gdn_decode_step(*bad) == INVALID
+    bad = list(args); bad[9], bad[10] = 80, 80
+    assert lib.kla_gdn_decode_step(*bad) == UNSUPPORTED
+
+
 def test_decode_rejects_bad_arguments(lib):
     args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, 6 * A, 7 * A, 2, 3, 128, 128, 0, None]
     bad = list(args); bad[6] = None
