@@ -202,8 +202,13 @@ def run_ours(args, rank, world, dev):
         nws = api.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype)
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
         fn = functools.partial(api.chunk_fwd, workspace=ws)
+        # UT kernel, then one chain launch, or three for a cut chain
+        # (segment transitions, start states, outputs)
+        nseg = api.chunk_fwd_segments(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, nws)
+        launches_per_step = 1 + (3 if nseg > 1 else 1)
     else:
         fn = api.recurrent_fwd
+        nseg, launches_per_step = 0, 1
     stream = torch.cuda.current_stream()
     flush = L2Flush(dev)
 
@@ -280,7 +285,8 @@ def run_ours(args, rank, world, dev):
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded PCG64, distributions of the workload recipe)",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
-                   "chunk": 64, "path": args.path, "global_batch": w.B * world,
+                   "chunk": 64, "path": args.path, "chain_segments": nseg,
+                   "global_batch": w.B * world,
                    "seq_len": w.T, "parallelism": "dp%d (independent sequences)" % world,
                    "l2": "flushed before every timed step (512 MiB write+read); inputs > L2"},
         # dominant kernel: the state/output (chain) kernel; its bytes at
@@ -301,9 +307,10 @@ def run_ours(args, rank, world, dev):
                    "algorithmic_bytes": byts,
                    "hbm_frac": byts / (ms / 1e3) / 1e9 / hbm_peak,
                    "peak_source": peak_src + " (burst cuBLAS bf16)"},
-        # our kernels per step: UT transform + chain (chunk path), one
-        # token-serial kernel otherwise; the L2 flush is torch's, not counted
-        "gpu_launches": args.steps * (2 if chunk else 1),
+        # our kernels per step: UT transform + chain (chunk path; three
+        # launches for a cut chain), one token-serial kernel otherwise; the
+        # L2 flush is torch's, not counted
+        "gpu_launches": args.steps * launches_per_step,
         "wall_s": wall,
         "e2e": e2e,
     }
@@ -315,6 +322,10 @@ def run_ours(args, rank, world, dev):
             "chain_kernel": {"us_per_launch": ms_chain * 1e3,
                              "algorithmic_bytes": chain_w["bytes"], "gbs": chain_gbs,
                              "tflops": chain_w["flops"] / (ms_chain / 1e3) / 1e12}}
+        if nseg > 1:
+            # the cut chain: its time spans its three launches
+            res["kernels"]["chain_kernel"]["launches"] = (
+                "%d segments: transitions, start states, outputs" % nseg)
     if not args.no_decode:
         res["decode"] = run_decode(args, rank, dev, stream, flush, peaks, peak_src, fn, clk)
     time.sleep(0.25)

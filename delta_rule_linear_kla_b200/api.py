@@ -58,6 +58,15 @@ def chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
     return int(_native.lib().kla_chunk_fwd_workspace_size(B, T, H, dk, dv, _DT[dtype]))
 
 
+def chunk_fwd_segments(B: int, T: int, H: int, dk: int, dv: int,
+                       dtype: torch.dtype = torch.bfloat16, ws_bytes: Optional[int] = None) -> int:
+    """Segments the bf16 state chain runs in (1 = uncut, 0 = not the chunk
+    path); ws_bytes defaults to the full workspace size."""
+    if ws_bytes is None:
+        ws_bytes = chunk_fwd_workspace_size(B, T, H, dk, dv, dtype)
+    return int(_native.lib().kla_chunk_fwd_segments(B, T, H, dk, dv, _DT[dtype], ws_bytes))
+
+
 def _prefill_args(q, k, v, g, eta, h0, o, hT, return_state):
     _need(q, "q")
     if q.dtype not in _DT:

@@ -75,6 +75,23 @@ static kla_status check_prefill(const void* q, const void* k, const void* v,
   return KLA_OK;
 }
 
+// True when [ws, ws + used) overlaps any argument of a prefill call.
+static bool workspace_overlaps(const void* ws, size_t used, const void* q, const void* k,
+                               const void* v, const float* g, const float* eta,
+                               const float* h0, const void* o, const float* hT, int B, int T,
+                               int H, int dk, int dv, int dtype) {
+  const size_t es = dtype == KLA_BF16 ? 2 : 4;
+  const size_t ntok = (size_t)B * T * H, sb = (size_t)B * H * dk * dv * 4;
+  const Range rw = rng(ws, used);
+  const Range args[] = {rng(q, ntok * dk * es), rng(k, ntok * dk * es), rng(v, ntok * dv * es),
+                        rng(g, ntok * 4),       rng(eta, eta ? ntok * 4 : 0),
+                        rng(h0, h0 ? sb : 0),   rng(o, ntok * dv * es),
+                        rng(hT, hT ? sb : 0)};
+  for (Range r : args)
+    if (overlap(rw, r)) return true;
+  return false;
+}
+
 // T == 0: the final state is the initial state.
 static kla_status empty_prefill(const float* h0, float* hT, int B, int H, int dk,
                                 int dv, cudaStream_t st) {
@@ -96,6 +113,11 @@ size_t kla_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int dty
   return chunk_workspace_bytes(B, T, H, dk, dv, dtype);
 }
 
+int kla_chunk_fwd_segments(int B, int T, int H, int dk, int dv, int dtype, size_t ws_bytes) {
+  if (!head_dims_ok(dk, dv) || chunk_ut_workspace_bytes(B, T, H, dk, dv, dtype) == 0) return 0;
+  return chunk_chain_segments(B, T, H, dk, dv, ws_bytes);
+}
+
 }  // extern "C"
 
 // Prefill with the KLA step size, or (eps == kBetaGiven) with beta given.
@@ -110,16 +132,22 @@ static kla_status chunk_fwd_impl(const void* q, const void* k, const void* v,
   if (chunk != KLA_CHUNK) return KLA_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
   if (T == 0) return empty_prefill(h0, hT, B, H, dk, dv, st);
-  const size_t need = chunk_workspace_bytes(B, T, H, dk, dv, dtype);
+  // the UT factors are required; the segment states (the rest of
+  // kla_chunk_fwd_workspace_size) only enable the segmented chain
+  const size_t need = chunk_ut_workspace_bytes(B, T, H, dk, dv, dtype);
   if (ws_bytes < need || (need > 0 && workspace == nullptr)) return KLA_ERR_INVALID_ARG;
   if (workspace && !aligned16(workspace)) return KLA_ERR_INVALID_ARG;
+  if (need > 0 && workspace_overlaps(workspace, chunk_workspace_used(B, T, H, dk, dv, dtype,
+                                                                     ws_bytes),
+                                     q, k, v, g, eta, h0, o, hT, B, T, H, dk, dv, dtype))
+    return KLA_ERR_INVALID_ARG;
   cudaError_t e;
   if (dtype == KLA_FP32) {
     e = launch_recurrent(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype, st);
   } else {
     unsigned int* err = device_error_ptr();
     if (!err) return KLA_ERR_CUDA;
-    e = launch_chunk_tc(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, workspace,
+    e = launch_chunk_tc(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, workspace, ws_bytes,
                         err, st);
     if (e == cudaErrorNotSupported) return KLA_ERR_UNSUPPORTED;
   }
@@ -151,7 +179,7 @@ static kla_status check_stage(int T, int dtype, void* workspace, size_t ws_bytes
                               int dk, int dv) {
   if (dtype != KLA_BF16) return dtype == KLA_FP32 ? KLA_ERR_UNSUPPORTED : KLA_ERR_INVALID_ARG;
   if (T < 1) return KLA_ERR_INVALID_ARG;
-  const size_t need = chunk_workspace_bytes(B, T, H, dk, dv, dtype);
+  const size_t need = chunk_ut_workspace_bytes(B, T, H, dk, dv, dtype);
   if (need == 0 || ws_bytes < need || workspace == nullptr || !aligned16(workspace))
     return KLA_ERR_INVALID_ARG;
   return KLA_OK;
@@ -170,7 +198,7 @@ kla_status kla_chunk_ut_transform(const void* k, const float* g, const float* et
   kla_status s = check_stage(T, dtype, workspace, ws_bytes, B, H, dk, dk);
   if (s != KLA_OK) return s;
   const size_t ntok = (size_t)B * T * H;
-  Range rw = rng(workspace, chunk_workspace_bytes(B, T, H, dk, dk, dtype));
+  Range rw = rng(workspace, chunk_ut_workspace_bytes(B, T, H, dk, dk, dtype));
   if (overlap(rw, rng(k, ntok * dk * 2)) || overlap(rw, rng(g, ntok * 4)) ||
       overlap(rw, rng(eta, ntok * 4)))
     return KLA_ERR_INVALID_ARG;
@@ -184,22 +212,20 @@ kla_status kla_chunk_ut_transform(const void* k, const float* g, const float* et
 
 kla_status kla_chunk_state_fwd(const void* q, const void* k, const void* v, const float* g,
                                const float* h0, void* o, float* hT, int B, int T, int H,
-                               int dk, int dv, int dtype, const void* workspace,
+                               int dk, int dv, int dtype, void* workspace,
                                size_t ws_bytes, void* stream) {
   // eta only enters through the workspace; validate with a stand-in pointer
   kla_status s = check_prefill(q, k, v, g, g, 0.f, h0, o, hT, B, T, H, dk, dv, dtype);
   if (s != KLA_OK) return s;
-  s = check_stage(T, dtype, const_cast<void*>(workspace), ws_bytes, B, H, dk, dv);
+  s = check_stage(T, dtype, workspace, ws_bytes, B, H, dk, dv);
   if (s != KLA_OK) return s;
-  const size_t ntok = (size_t)B * T * H;
-  Range rw = rng(workspace, chunk_workspace_bytes(B, T, H, dk, dv, dtype));
-  if (overlap(rw, rng(o, ntok * dv * 2)) ||
-      (hT && overlap(rw, rng(hT, (size_t)B * H * dk * dv * 4))))
+  if (workspace_overlaps(workspace, chunk_workspace_used(B, T, H, dk, dv, dtype, ws_bytes), q,
+                         k, v, g, nullptr, h0, o, hT, B, T, H, dk, dv, dtype))
     return KLA_ERR_INVALID_ARG;
   unsigned int* err = device_error_ptr();
   if (!err) return KLA_ERR_CUDA;
-  cudaError_t e = launch_chunk_chain(q, k, v, g, h0, o, hT, B, T, H, dk, dv, workspace, err,
-                                     (cudaStream_t)stream);
+  cudaError_t e = launch_chunk_chain(q, k, v, g, h0, o, hT, B, T, H, dk, dv, workspace,
+                                     ws_bytes, err, (cudaStream_t)stream);
   if (e == cudaErrorNotSupported) return KLA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }

@@ -12,8 +12,17 @@ namespace kla {
 // the chain kernel wants them in shared memory (128-byte swizzled rows).
 constexpr size_t kUtTileBytes = 2 * 64 * 64 * 2;
 
-// Device scratch the chunk path needs for these sizes (bytes, 0 if none).
+// Device scratch the chunk path needs for these sizes (bytes, 0 if none):
+// the UT factors of every chunk and, when the state chain is cut into
+// segments, the segment states.
 size_t chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
+// The UT factors alone (the least a workspace must hold).
+size_t chunk_ut_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
+// Bytes of a workspace of ws_bytes that the chunk path touches: all of
+// chunk_workspace_bytes when it fits (segmented chain), else the UT factors.
+size_t chunk_workspace_used(int B, int T, int H, int dk, int dv, int dtype, size_t ws_bytes);
+// Segments the state chain runs in for a workspace of ws_bytes (1 = uncut).
+int chunk_chain_segments(int B, int T, int H, int dk, int dv, size_t ws_bytes);
 
 // bf16 I/O chunkwise prefill (UT kernel, then the chain kernel).  Returns
 // cudaErrorNotSupported for shapes it does not handle; `err` is this
@@ -21,7 +30,7 @@ size_t chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v,
                             const float* g, const float* eta, float eps,
                             const float* h0, void* o, float* hT, int B, int T,
-                            int H, int dk, int dv, void* workspace,
+                            int H, int dk, int dv, void* workspace, size_t ws_bytes,
                             unsigned int* err, cudaStream_t st);
 
 // The two stages of launch_chunk_tc on their own: the UT transform of every
@@ -29,10 +38,12 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v,
 cudaError_t launch_chunk_ut(const void* k, const float* g, const float* eta, float eps,
                             int B, int T, int H, int dk, void* workspace, unsigned int* err,
                             cudaStream_t st);
+// The chain is cut into segments (a sequence-parallel schedule for few heads
+// and long sequences) when ws_bytes also covers the segment states.
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, const float* g,
                                const float* h0, void* o, float* hT, int B, int T, int H,
-                               int dk, int dv, const void* workspace, unsigned int* err,
-                               cudaStream_t st);
+                               int dk, int dv, void* workspace, size_t ws_bytes,
+                               unsigned int* err, cudaStream_t st);
 
 // UT kernel alone: T', T'' of every chunk into `ws` (chunk-major order
 // ((b * H + h) * nchunks + n)).  `tm_k` maps k as [B][T][H][dk] bf16 with

@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
              const float* __restrict__ h0, __nv_bfloat16* __restrict__ o,
-             float* __restrict__ hT, int T, int H, int DV, const uint8_t* __restrict__ ws,
+             float* __restrict__ hT, float* __restrict__ phi, int T, int H, int DV,
+             int nseg, int seg_chunks, int mode, const uint8_t* __restrict__ ws,
              unsigned int* err) {
   using Smem = ChainSmem<DK>;
   constexpr int NP = Stage<DK>::NP;
@@ -150,9 +151,22 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                                      ~uintptr_t(1023));
   volatile int* abort_flag = &s.abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int slab = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
-  const int nchunks = (T + C - 1) / C;
+  const int hh = blockIdx.y, b = blockIdx.z / nseg, seg = blockIdx.z % nseg;
+  // Segment `seg` of the sequence: chunks n0 .. n0 + nchunks - 1 (the loop
+  // index n below counts chunks within the segment; n0 + n addresses data).
+  const int nchunks_all = (T + C - 1) / C;
+  const int n0 = seg * seg_chunks;
+  const int nchunks = min(seg_chunks, nchunks_all - n0);
   const size_t head = (size_t)b * H + hh;
+  const size_t sidx = ((size_t)b * nseg + seg) * H + hh;  // per-segment state index
+  // mode 0: outputs; the initial state is h0[sidx] (NULL = zeros) and the
+  // last segment writes h_T to hT[head].  mode 1 (segment transitions, no
+  // outputs): slabs below DV / BV run from a zero state and leave the end
+  // state E in hT[sidx]; the others propagate the identity with V = 0 and
+  // leave Phi (the segment's transition, [DK][DK]) in phi[sidx].
+  const int nvs = DV / BV;
+  const bool phi_slab = mode == 1 && (int)blockIdx.x >= nvs;
+  const int slab = phi_slab ? (int)blockIdx.x - nvs : (int)blockIdx.x;
   // TMEM lane group this warp may access, and the row it stands for
   const int row = 32 * (warp & 3) + lane;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
@@ -183,9 +197,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     ptx::mbar_init_fence();
     s.abort_flag = 0;
   }
-  // the zero tiles of both stages
-  for (int i = tid; i < 2 * 8192 / 16; i += NTHREADS)
+  // the zero tiles of both stages (and, with V = 0, the V slabs)
+  for (int i = tid; i < 2 * 8192 / 16; i += NTHREADS) {
     reinterpret_cast<uint4*>(s.st[i / 512].tp[TZ])[i % 512] = make_uint4(0, 0, 0, 0);
+    if (phi_slab) reinterpret_cast<uint4*>(s.st[i / 512].v)[i % 512] = make_uint4(0, 0, 0, 0);
+  }
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
@@ -198,8 +214,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       ptx::prefetch_tensormap(&tm_q);
       ptx::prefetch_tensormap(&tm_k);
       ptx::prefetch_tensormap(&tm_v);
-      constexpr uint32_t BYTES = (uint32_t)(2 * NP * 8192 + 8192 + kUtTileBytes);
-      const uint8_t* ws_head = ws + head * (size_t)nchunks * kUtTileBytes;
+      const uint32_t BYTES = (uint32_t)(2 * NP * 8192 + (phi_slab ? 0 : 8192) + kUtTileBytes);
+      const uint8_t* ws_head = ws + (head * (size_t)nchunks_all + n0) * kUtTileBytes;
       int issued = 0, drained = 0;
       for (int n = 0; n < nchunks; ++n) {
         const int st = n & 1;
@@ -214,20 +230,21 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         ptx::bulk_load(S.tp[TP2], src + 8192, 8192, &s.full[st]);
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-          ptx::tma_load_4d(S.panel[p][SK], &tm_k, &s.full[st], p * 64, hh, n * C, b);
-          ptx::tma_load_4d(S.panel[p][SQ], &tm_q, &s.full[st], p * 64, hh, n * C, b);
+          ptx::tma_load_4d(S.panel[p][SK], &tm_k, &s.full[st], p * 64, hh, (n0 + n) * C, b);
+          ptx::tma_load_4d(S.panel[p][SQ], &tm_q, &s.full[st], p * 64, hh, (n0 + n) * C, b);
         }
-        ptx::tma_load_4d(S.v, &tm_v, &s.full[st], slab * BV, hh, n * C, b);
+        if (!phi_slab)
+          ptx::tma_load_4d(S.v, &tm_v, &s.full[st], slab * BV, hh, (n0 + n) * C, b);
         issued = n + 1;
         if (n + 2 < nchunks) {  // warm L2 two chunks ahead of the loads
           const int m = n + 2;
           ptx::bulk_prefetch_l2(ws_head + (size_t)m * kUtTileBytes, (uint32_t)kUtTileBytes);
 #pragma unroll
           for (int p = 0; p < NP; ++p) {
-            ptx::tma_prefetch_l2_4d(&tm_k, p * 64, hh, m * C, b);
-            ptx::tma_prefetch_l2_4d(&tm_q, p * 64, hh, m * C, b);
+            ptx::tma_prefetch_l2_4d(&tm_k, p * 64, hh, (n0 + m) * C, b);
+            ptx::tma_prefetch_l2_4d(&tm_q, p * 64, hh, (n0 + m) * C, b);
           }
-          ptx::tma_prefetch_l2_4d(&tm_v, slab * BV, hh, m * C, b);
+          if (!phi_slab) ptx::tma_prefetch_l2_4d(&tm_v, slab * BV, hh, (n0 + m) * C, b);
         }
       }
       if (*abort_flag) {
@@ -400,8 +417,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const int r = row - 64;
     float gn0 = 0.f, gn1 = 0.f;
     if (warp == 2 && nchunks > 0) {
-      gn0 = (lane < T) ? g[((size_t)b * T + lane) * H + hh] : 0.f;
-      gn1 = (lane + 32 < T) ? g[((size_t)b * T + lane + 32) * H + hh] : 0.f;
+      const int t0 = n0 * C + lane, t1 = t0 + 32;
+      gn0 = (t0 < T) ? g[((size_t)b * T + t0) * H + hh] : 0.f;
+      gn1 = (t1 < T) ? g[((size_t)b * T + t1) * H + hh] : 0.f;
     }
     for (int n = 0; n < nchunks; ++n) {
       Stage<DK>& S = s.st[n & 1];
@@ -409,7 +427,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       if (warp == 2) {
         const float g0 = gn0, g1 = gn1;
         // next chunk's gates (tokens lane, lane + 32), used one chunk later
-        const int t0 = (n + 1) * C + lane, t1 = t0 + 32;
+        const int t0 = (n0 + n + 1) * C + lane, t1 = t0 + 32;
         gn0 = (t0 < T) ? g[((size_t)b * T + t0) * H + hh] : 0.f;
         gn1 = (t1 < T) ? g[((size_t)b * T + t1) * H + hh] : 0.f;
         float x0 = g0, x1 = g1;
@@ -466,9 +484,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const bool has_h = row < DK;
     float hreg[32];
     if (has_h) {
-      if (h0) {
+      if (phi_slab) {  // identity columns slab * BV + cg ..
+#pragma unroll
+        for (int j = 0; j < 32; ++j) hreg[j] = (row == slab * BV + cg + j) ? 1.f : 0.f;
+      } else if (h0 && mode == 0) {
         const float4* src =
-            reinterpret_cast<const float4*>(h0 + (head * DK + row) * DV + slab * BV + cg);
+            reinterpret_cast<const float4*>(h0 + (sidx * DK + row) * DV + slab * BV + cg);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float4 x = src[j];
@@ -534,7 +555,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       if (!v_rows) {
         // output row r = row - 64: o_r = e^{G_r} (Q h)_r + (P V')_r, with
         // -(Q h)_r in lanes 64..127 of D_U
-        const int r = row - 64, t = n * C + r;
+        const int r = row - 64, t = (n0 + n) * C + r;
         const float e = e_out;
         if (!wait_or_abort(&s.bHP, par, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
@@ -547,7 +568,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           mbar_arrive(&s.u_free[n & 1]);
           mbar_arrive(&s.pv_free);
         }
-        if (t < T) {
+        if (t < T && mode == 0) {
           uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * T + t) * H + hh) * DV +
                                                 slab * BV + cg);
 #pragma unroll
@@ -562,8 +583,20 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
       }
     }
-    if (ok && has_h && hT) {
-      float4* dst = reinterpret_cast<float4*>(hT + (head * DK + row) * DV + slab * BV + cg);
+    // the state this CTA ends with: h_T (last segment), E or Phi
+    float* out = nullptr;
+    size_t oidx = 0;
+    int ostride = DV;
+    if (mode == 0 && seg == nseg - 1) {
+      out = hT;
+      oidx = head;
+    } else if (mode == 1) {
+      out = phi_slab ? phi : hT;
+      oidx = sidx;
+      ostride = phi_slab ? DK : DV;
+    }
+    if (ok && has_h && out) {
+      float4* dst = reinterpret_cast<float4*>(out + (oidx * DK + row) * ostride + slab * BV + cg);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
@@ -606,9 +639,54 @@ bool make_map(CUtensorMap* m, const void* base, int d, int H, int T, int B) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Start state of every segment: h(0) = h0 (NULL = zeros), h(s + 1) =
+// Phi_s h(s) + E_s, for one head and 64-column slab per CTA, fp32 on CUDA
+// cores (nseg - 1 products of [DK][DK] by [DK][64]).  E and Phi hold the
+// nseg - 1 first segments ([B][nseg - 1][H]), hstart all nseg ([B][nseg][H]).
+// Thread t owns row t / 2 and 32 columns of the slab; the slab itself stays
+// in shared memory.
+template <int DK>
+__global__ void __launch_bounds__(2 * DK)
+segment_start_kernel(const float* __restrict__ h0, const float* __restrict__ E,
+                     const float* __restrict__ Phi, float* __restrict__ hstart, int H, int DV,
+                     int nseg) {
+  __shared__ float hs[DK][BV];
+  const int slab = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
+  const int i = threadIdx.x >> 1, c0 = 32 * (threadIdx.x & 1);
+  const size_t head = (size_t)b * H + hh;
+  float acc[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c)
+    acc[c] = h0 ? h0[(head * DK + i) * DV + slab * BV + c0 + c] : 0.f;
+  for (int sg = 0; sg < nseg; ++sg) {
+    const size_t sidx = ((size_t)b * nseg + sg) * H + hh;
+    if (sg > 0) {
+      const size_t pidx = ((size_t)b * (nseg - 1) + sg - 1) * H + hh;  // segment sg - 1
+      const float* ph = Phi + (pidx * DK + i) * DK;
+      const float* e = E + (pidx * DK + i) * DV + slab * BV + c0;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) acc[c] = e[c];
+#pragma unroll 4
+      for (int kq = 0; kq < DK; ++kq) {
+        const float a = ph[kq];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) acc[c] = fmaf(a, hs[kq][c0 + c], acc[c]);
+      }
+      __syncthreads();  // everyone has read h(sg - 1)
+    }
+#pragma unroll
+    for (int c = 0; c < 32; ++c) hs[i][c0 + c] = acc[c];
+    float* dst = hstart + (sidx * DK + i) * DV + slab * BV + c0;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) dst[c] = acc[c];
+    __syncthreads();
+  }
+}
+
 template <int DK>
 cudaError_t launch_chain_dk(const void* q, const void* k, const void* v, const float* g,
-                            const float* h0, void* o, float* hT, int B, int T, int H, int DV,
+                            const float* h0, void* o, float* hT, float* phi, int B, int T,
+                            int H, int DV, int nseg, int seg_chunks, int mode,
                             const uint8_t* ws, unsigned int* err, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, DK, H, T, B) || !make_map(&mk, k, DK, H, T, B) ||
@@ -625,17 +703,74 @@ cudaError_t launch_chain_dk(const void* q, const void* k, const void* v, const f
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid(DV / BV, H, B);
-  chain_kernel<DK><<<grid, NTHREADS, smem, st>>>(mq, mk, mv, g, h0, (__nv_bfloat16*)o, hT, T,
-                                                 H, DV, ws, err);
+  dim3 grid((mode == 1 ? DV + DK : DV) / BV, H, B * nseg);
+  chain_kernel<DK><<<grid, NTHREADS, smem, st>>>(mq, mk, mv, g, h0, (__nv_bfloat16*)o, hT, phi,
+                                                 T, H, DV, nseg, seg_chunks, mode, ws, err);
   return cudaGetLastError();
+}
+
+// Number of segments the sequence is cut into for the state chain.  One CTA
+// per (head, 64-column slab) walks its chunks in sequence, so with few heads
+// most SMs idle; cutting the sequence into S segments runs S times as many
+// CTAs, at the price of a first pass over segments 0 .. S-2 that also carries
+// the dk identity columns (the segment transitions) and of a small combine.
+// Cost model in units of "one chunk step of one wave of CTAs" on the 148 SMs
+// of a B200; segments keep at least 8 chunks.
+constexpr int kSmTarget = 148;
+int chain_segments(int B, int T, int H, int dk, int dv) {
+  const int nchunks = (T + C - 1) / C;
+  const long p3 = (long)B * H * (dv / BV);          // CTAs per segment, outputs
+  const long p1 = (long)B * H * ((dv + dk) / BV);   // CTAs per segment, pass 1
+  auto waves = [](long ctas) { return (ctas + kSmTarget - 1) / kSmTarget; };
+  long best = waves(p3) * nchunks;
+  int best_s = 1;
+  for (int sg = 2; sg <= 64 && nchunks / sg >= 8; ++sg) {
+    const long len = (nchunks + sg - 1) / sg;
+    if ((sg - 1) * len >= nchunks) continue;  // the last segment would be empty
+    const long cost = (waves((sg - 1) * p1) + waves(sg * p3)) * len;
+    if (cost * 5 < best * 4) {  // a clear gain only
+      best = cost;
+      best_s = sg;
+    }
+  }
+  return best_s;
+}
+
+size_t ut_workspace_bytes(int B, int T, int H) {
+  return (size_t)B * H * ((T + C - 1) / C) * kUtTileBytes;
+}
+
+// Segment buffers after the UT factors: E and the start states
+// [B * S * H][dk][dv], Phi [B * S * H][dk][dk] (fp32).
+size_t segment_bytes(int B, int T, int H, int dk, int dv) {
+  const int sg = chain_segments(B, T, H, dk, dv);
+  if (sg == 1) return 0;
+  const size_t n = (size_t)B * sg * H;
+  return n * ((size_t)2 * dk * dv + (size_t)dk * dk) * sizeof(float);
 }
 
 }  // namespace
 
 size_t chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
   if (dtype != KLA_BF16 || B < 1 || H < 1 || T < 1 || dk != dv) return 0;
-  return (size_t)B * H * ((T + C - 1) / C) * kUtTileBytes;
+  return ut_workspace_bytes(B, T, H) + segment_bytes(B, T, H, dk, dv);
+}
+
+size_t chunk_ut_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
+  if (dtype != KLA_BF16 || B < 1 || H < 1 || T < 1 || dk != dv) return 0;
+  return ut_workspace_bytes(B, T, H);
+}
+
+int chunk_chain_segments(int B, int T, int H, int dk, int dv, size_t ws_bytes) {
+  const int sg = chain_segments(B, T, H, dk, dv);
+  return sg > 1 && ws_bytes >= ut_workspace_bytes(B, T, H) + segment_bytes(B, T, H, dk, dv)
+             ? sg
+             : 1;
+}
+
+size_t chunk_workspace_used(int B, int T, int H, int dk, int dv, int dtype, size_t ws_bytes) {
+  const size_t full = chunk_workspace_bytes(B, T, H, dk, dv, dtype);
+  return ws_bytes >= full ? full : chunk_ut_workspace_bytes(B, T, H, dk, dv, dtype);
 }
 
 cudaError_t launch_chunk_ut(const void* k, const float* g, const float* eta, float eps,
@@ -647,25 +782,67 @@ cudaError_t launch_chunk_ut(const void* k, const float* g, const float* eta, flo
   return launch_ut(mk, g, eta, eps, (uint8_t*)workspace, B, T, H, dk, err, st);
 }
 
+// The chain in S segments: pass 1 (E, Phi of segments 0 .. S-2), the start
+// states, pass 2 (outputs of every segment from its start state).
+template <int DK>
+static cudaError_t launch_segmented(const void* q, const void* k, const void* v, const float* g,
+                                    const float* h0, void* o, float* hT, int B, int T, int H,
+                                    int sg, uint8_t* ws, unsigned int* err, cudaStream_t st);
+
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, const float* g,
                                const float* h0, void* o, float* hT, int B, int T, int H,
-                               int dk, int dv, const void* workspace, unsigned int* err,
-                               cudaStream_t st) {
+                               int dk, int dv, void* workspace, size_t ws_bytes,
+                               unsigned int* err, cudaStream_t st) {
   if (dk != dv) return cudaErrorNotSupported;
+  const int sg = chunk_chain_segments(B, T, H, dk, dv, ws_bytes);
+  if (sg > 1) {
+    uint8_t* wsm = (uint8_t*)workspace;
+    if (dk == 128) return launch_segmented<128>(q, k, v, g, h0, o, hT, B, T, H, sg, wsm, err, st);
+    return launch_segmented<64>(q, k, v, g, h0, o, hT, B, T, H, sg, wsm, err, st);
+  }
   const uint8_t* ws = (const uint8_t*)workspace;
-  if (dk == 128) return launch_chain_dk<128>(q, k, v, g, h0, o, hT, B, T, H, dv, ws, err, st);
-  if (dk == 64) return launch_chain_dk<64>(q, k, v, g, h0, o, hT, B, T, H, dv, ws, err, st);
+  const int nchunks = (T + C - 1) / C;
+  if (dk == 128)
+    return launch_chain_dk<128>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks, 0, ws,
+                                err, st);
+  if (dk == 64)
+    return launch_chain_dk<64>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks, 0, ws,
+                               err, st);
   return cudaErrorNotSupported;
+}
+
+template <int DK>
+static cudaError_t launch_segmented(const void* q, const void* k, const void* v, const float* g,
+                                    const float* h0, void* o, float* hT, int B, int T, int H,
+                                    int sg, uint8_t* ws, unsigned int* err, cudaStream_t st) {
+  constexpr int DV = DK;
+  const int nchunks = (T + C - 1) / C;
+  const int len = (nchunks + sg - 1) / sg;
+  const size_t n = (size_t)B * sg * H;
+  float* E = reinterpret_cast<float*>(ws + ut_workspace_bytes(B, T, H));
+  float* hstart = E + n * DK * DV;
+  float* Phi = hstart + n * DK * DV;
+  // pass 1 covers segments 0 .. S-2 (launched as S - 1 segments of `len`
+  // chunks, so E and Phi are laid out [B][S - 1][H])
+  cudaError_t e = launch_chain_dk<DK>(q, k, v, g, nullptr, nullptr, E, Phi, B, T, H, DV,
+                                      sg - 1, len, 1, ws, err, st);
+  if (e != cudaSuccess) return e;
+  segment_start_kernel<DK><<<dim3(DV / BV, H, B), 2 * DK, 0, st>>>(h0, E, Phi, hstart, H, DV, sg);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_chain_dk<DK>(q, k, v, g, hstart, o, hT, nullptr, B, T, H, DV, sg, len, 0, ws,
+                             err, st);
 }
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                             const float* eta, float eps, const float* h0, void* o, float* hT,
                             int B, int T, int H, int dk, int dv, void* workspace,
-                            unsigned int* err, cudaStream_t st) {
+                            size_t ws_bytes, unsigned int* err, cudaStream_t st) {
   if (dk != dv || (dk != 64 && dk != 128)) return cudaErrorNotSupported;
   cudaError_t e = launch_chunk_ut(k, g, eta, eps, B, T, H, dk, workspace, err, st);
   if (e != cudaSuccess) return e;
-  return launch_chunk_chain(q, k, v, g, h0, o, hT, B, T, H, dk, dv, workspace, err, st);
+  return launch_chunk_chain(q, k, v, g, h0, o, hT, B, T, H, dk, dv, workspace, ws_bytes, err,
+                            st);
 }
 
 }  // namespace kla

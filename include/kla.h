@@ -72,8 +72,14 @@ typedef enum { KLA_BF16 = 0, KLA_FP32 = 1 } kla_dtype;
  *   hT      [B][H][dk][dv] fp32        final state (written); NULL = not
  *                                      returned.  hT may alias h0 exactly.
  *   chunk   must equal KLA_CHUNK (else KLA_ERR_UNSUPPORTED)
- *   workspace / ws_bytes: caller-owned device scratch of at least
- *     kla_chunk_fwd_workspace_size(...) bytes (NULL allowed when that is 0).
+ *   workspace / ws_bytes: caller-owned device scratch of
+ *     kla_chunk_fwd_workspace_size(...) bytes (NULL allowed when that is 0):
+ *     the per-chunk factors (B * H * ceil(T / KLA_CHUNK) * 16384 bytes, the
+ *     least accepted, else KLA_ERR_INVALID_ARG) followed, for few heads and
+ *     long sequences, by the states of the sequence segments the state chain
+ *     is cut into (run in parallel).  A workspace smaller than the full size
+ *     but holding the factors runs the chain uncut.  It must not overlap any
+ *     other argument.
  *
  * Supported: B, H >= 1; T >= 0 (T = 0 copies h0 to hT); dk = dv in {64, 128}.
  * A ragged tail (T not a multiple of the chunk) is processed as if padded
@@ -82,6 +88,18 @@ typedef enum { KLA_BF16 = 0, KLA_FP32 = 1 } kla_dtype;
  * runs the token-serial CUDA-core kernel (kla_recurrent_fwd).
  */
 KLA_API size_t kla_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int dtype);
+
+/*
+ * Number of sequence segments the bf16 state chain of kla_chunk_fwd (and of
+ * kla_chunk_state_fwd, kla_gdn_chunk_fwd) runs in for these sizes and a
+ * workspace of ws_bytes: 1 = one pass over the whole sequence (one chain
+ * kernel launch); S > 1 = the segment transitions of segments 0 .. S-2, a
+ * start-state kernel, then the outputs of all S segments (three launches).
+ * 0 when the bf16 chunk path does not apply (fp32 I/O, bad sizes).
+ * Informational: the entry points choose by themselves.
+ */
+KLA_API int kla_chunk_fwd_segments(int B, int T, int H, int dk, int dv, int dtype,
+                                   size_t ws_bytes);
 
 KLA_API kla_status kla_chunk_fwd(const void *q, const void *k, const void *v,
                          const float *g, const float *eta, float eps,
@@ -109,7 +127,10 @@ KLA_API kla_status kla_chunk_fwd(const void *q, const void *k, const void *v,
  *   decayed Q K^T, diagonal included), h <- e^{G_last} h + K^T diag(e^{G_last
  *   - G}) V'.  Reads q, k, v, g (the same k and g the workspace was made
  *   from), h0 (NULL = zeros) and the workspace; writes o and hT (NULL = not
- *   returned, may alias h0).  o and hT must not overlap the workspace.
+ *   returned, may alias h0).  It writes the workspace past the factors
+ *   (the segment states) when ws_bytes is kla_chunk_fwd_workspace_size's;
+ *   the factors themselves are left as they are.  No other argument may
+ *   overlap the workspace.
  */
 KLA_API kla_status kla_chunk_ut_transform(const void *k, const float *g, const float *eta,
                                   float eps, int B, int T, int H, int dk, int dtype,
@@ -118,7 +139,7 @@ KLA_API kla_status kla_chunk_ut_transform(const void *k, const float *g, const f
 KLA_API kla_status kla_chunk_state_fwd(const void *q, const void *k, const void *v,
                                const float *g, const float *h0, void *o, float *hT,
                                int B, int T, int H, int dk, int dv, int dtype,
-                               const void *workspace, size_t ws_bytes, void *stream);
+                               void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * Token-serial prefill on CUDA cores: the recurrence evaluated one token at
@@ -179,7 +200,8 @@ KLA_API kla_status kla_gdn_decode_step(const void *q, const void *k, const void 
  * instead of a workspace.  It allocates nothing itself.
  *
  *   Limit: B * H * ceil(T / KLA_CHUNK) <= KLA_NOALLOC_MAX_CHUNKS, else
- *          KLA_ERR_UNSUPPORTED (checked before any CUDA call).
+ *          KLA_ERR_UNSUPPORTED (checked before any CUDA call).  The state
+ *          chain is cut into segments only where their states also fit.
  *   Memory: every GPU that loads libkla.so holds KLA_NOALLOC_SCRATCH_BYTES
  *          for the life of the process.
  *   First call on a device looks up the array's device address

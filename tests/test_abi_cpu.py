@@ -115,6 +115,37 @@ def test_decode_rejects_bad_arguments(lib):
     assert lib.kla_decode_step(*bad) == INVALID
 
 
+def _ut_bytes(B, T, H):
+    return B * H * ((T + 63) // 64) * 16384  # two 64 x 64 bf16 factors per chunk
+
+
 def test_workspace_query(lib):
-    n = lib.kla_chunk_fwd_workspace_size(8, 4096, 8, 128, 128, 0)
-    assert n >= 0 and n < (1 << 34)
+    # enough heads to fill the GPU: the chain runs uncut, factors only
+    assert lib.kla_chunk_fwd_workspace_size(8, 4096, 8, 128, 128, 0) == _ut_bytes(8, 4096, 8)
+    # few heads and a long sequence: per-segment states (E, start state,
+    # transition) follow the factors, for between 2 and 64 segments
+    n = lib.kla_chunk_fwd_workspace_size(1, 65536, 16, 128, 128, 0)
+    per_seg = 16 * (2 * 128 * 128 + 128 * 128) * 4
+    extra = n - _ut_bytes(1, 65536, 16)
+    assert extra > 0 and extra % per_seg == 0 and 2 <= extra // per_seg <= 64
+    assert lib.kla_chunk_fwd_segments(1, 65536, 16, 128, 128, 0, n) == extra // per_seg
+    assert lib.kla_chunk_fwd_segments(1, 65536, 16, 128, 128, 0, n - 16) == 1  # no room: uncut
+    assert lib.kla_chunk_fwd_segments(8, 4096, 8, 128, 128, 0, 1 << 40) == 1
+    assert lib.kla_chunk_fwd_segments(1, 65536, 16, 128, 128, 1, n) == 0  # fp32 I/O
+    assert lib.kla_chunk_fwd_segments(1, 65536, 16, 96, 96, 0, n) == 0
+    # short sequences are never cut (segments keep at least 8 chunks)
+    assert lib.kla_chunk_fwd_workspace_size(1, 64 * 15, 1, 64, 64, 0) == _ut_bytes(1, 960, 1)
+    assert lib.kla_chunk_fwd_workspace_size(1, 65536, 16, 128, 128, 1) == 0  # fp32: none
+
+
+def test_prefill_workspace_checks(lib):
+    ws = 8 * A
+    assert _fwd(lib, ws=ws, wsb=_ut_bytes(1, 128, 2) - 16) == INVALID  # factors do not fit
+    assert _fwd(lib, ws=2 * A, wsb=1 << 22) == INVALID                 # overlaps k
+    # a cut chain (B=1, T=1536, H=1, d=64): the factors end right where o
+    # starts, so only the segment states past them would overlap o
+    T, d = 1536, 64
+    full = lib.kla_chunk_fwd_workspace_size(1, T, 1, d, d, 0)
+    ut = _ut_bytes(1, T, 1)
+    assert full > ut
+    assert _fwd(lib, ws=6 * A - ut, wsb=full, T=T, H=1, dk=d, dv=d) == INVALID

@@ -53,6 +53,37 @@ def test_long_gates_small():
     _full_check(W["prefill_65k"].scaled(T=700, H=2))
 
 
+def _ut_bytes(w):
+    return w.B * w.H * ((w.T + 63) // 64) * 16384
+
+
+# Few heads and long sequences: the state chain is cut into segments that run
+# in parallel (transitions, start states, then outputs per segment).  The
+# shapes give several segments of at least 8 chunks and a ragged tail.
+SEGMENTED = [("prefill_4k", 1, 4000, 2, True), ("stress", 2, 2000, 1, False),
+             ("stress", 1, 1536, 1, True), ("prefill_65k", 1, 2500, 3, True)]
+
+
+@pytest.mark.parametrize("name,B,T,H,h0", SEGMENTED)
+def test_segmented_chain(name, B, T, H, h0):
+    w = W[name].scaled(B=B, T=T, H=H, seed=17)
+    assert api.chunk_fwd_segments(w.B, w.T, w.H, w.dk, w.dv) > 1
+    _full_check(w, with_h0=h0)
+
+
+@pytest.mark.parametrize("name,B,T,H,h0", SEGMENTED[:2])
+def test_segmented_equals_uncut_chain(name, B, T, H, h0):
+    """The same factors through the cut chain (full workspace) and the uncut
+    one (a workspace holding the factors only) agree to rounding."""
+    w = W[name].scaled(B=B, T=T, H=H, seed=19)
+    x = cuda(inputs.make_prefill(w, with_h0=h0))
+    ws = api.chunk_ut_transform(x["k"], x["g"], x["eta"], x["eps"])
+    o1, h1 = api.chunk_state_fwd(x["q"], x["k"], x["v"], x["g"], ws, x["h0"])
+    o2, h2 = api.chunk_state_fwd(x["q"], x["k"], x["v"], x["g"], ws[:_ut_bytes(w)], x["h0"])
+    api.check_device_error()
+    assert rel(o1.cpu(), o2.cpu()) < 2e-3 and rel(h1.cpu(), h2.cpu()) < 2e-3
+
+
 def test_final_state_only_and_alias():
     w = W["stress"].scaled(B=1, T=150, H=2)
     x = inputs.make_prefill(w)

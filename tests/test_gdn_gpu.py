@@ -20,10 +20,13 @@ def _beta(shape, seed):
     return torch.from_numpy((1.0 / (1.0 + np.exp(-rng.normal(size=shape)))).astype(np.float32))
 
 
-@pytest.mark.parametrize("name,T,dt", [("prefill_4k", 200, "bf16"), ("stress", 130, "bf16"),
-                                       ("tiny", 150, "fp32")])
-def test_gdn_prefill(name, T, dt):
-    w = inputs.WORKLOADS[name].scaled(B=2, T=T, H=2, dtype=dt)
+@pytest.mark.parametrize("name,B,T,H,dt", [("prefill_4k", 2, 200, 2, "bf16"),
+                                           ("stress", 2, 130, 2, "bf16"),
+                                           ("tiny", 2, 150, 2, "fp32"),
+                                           # long and few heads: the cut state chain
+                                           ("prefill_4k", 1, 3000, 1, "bf16")])
+def test_gdn_prefill(name, B, T, H, dt):
+    w = inputs.WORKLOADS[name].scaled(B=B, T=T, H=H, dtype=dt)
     x = inputs.make_prefill(w)
     # GDN is used with normalised keys; keep them at unit norm
     kf = x["k"].float()
