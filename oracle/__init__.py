@@ -12,6 +12,10 @@ Sources of each formula (page title, section):
   * S_t = alpha_t S_{t-1}(I - beta_t k_t k_t^T) + beta_t v_t k_t^T, o_t = S_t q_t:
     "Deep Dive into KDA", section 2.2 (Gated DeltaNet), which the KLA Abstract
     says KLA keeps unchanged apart from beta.
+  * per-channel gate: S_t = (I - beta_t k_t k_t^T) Diag(a_t) S_{t-1}
+    + beta_t v_t k_t^T, a_t = exp(g_t) per key channel (decay first, then the
+    erase reads the decayed state): "Deep Dive into KDA", section 2.3 (KDA);
+    the KLA Abstract names a preconditioned KDA (beta from the key norm).
 
 Arrays follow the library's layouts: q, k ``[B, T, H, dk]``; v, o
 ``[B, T, H, dv]``; g, eta ``[B, T, H]``; states ``[B, H, dk, dv]`` holding
@@ -61,6 +65,8 @@ def _load():
     lib.kla_oracle_forward.argtypes = [dp, dp, dp, dp, dp, ctypes.c_double,
                                        dp, dp, dp, i, i, i, i, i]
     lib.kla_oracle_forward.restype = None
+    lib.kla_oracle_kda.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i]
+    lib.kla_oracle_kda.restype = None
     lib.kla_oracle_num_threads.argtypes = []
     lib.kla_oracle_num_threads.restype = i
     _lib = lib
@@ -126,6 +132,38 @@ def forward(q, k, v, g, eta, eps: float, h0=None):
                                float(eps), _ptr(h0), _ptr(o), _ptr(hT),
                                B, T, H, dk, dv)
     return o, hT
+
+
+def kda(q, k, v, g, beta_, h0=None):
+    """Delta rule with a per-channel gate (KDA form), beta given per token:
+    g [B,T,H,dk] (log-gate per key channel), beta [B,T,H].  Returns (o, hT)
+    in fp64."""
+    q, k, v, g, beta_, h0 = map(f64, (q, k, v, g, beta_, h0))
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    assert q.shape == k.shape and v.shape[:3] == (B, T, H)
+    assert g.shape == (B, T, H, dk) and beta_.shape == (B, T, H)
+    if h0 is not None:
+        assert h0.shape == (B, H, dk, dv)
+    o = np.empty((B, T, H, dv), dtype=np.float64)
+    hT = np.empty((B, H, dk, dv), dtype=np.float64)
+    _load().kla_oracle_kda(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta_), _ptr(h0),
+                           _ptr(o), _ptr(hT), B, T, H, dk, dv)
+    return o, hT
+
+
+def kda_forward(q, k, v, g, eta, eps: float, h0=None):
+    """KLA with the per-channel gate (preconditioned KDA): beta from the key
+    norm, then :func:`kda`.  g is [B,T,H,dk].  Returns (o, hT) in fp64."""
+    return kda(q, k, v, g, beta(k, eta, eps), h0)
+
+
+def kda_decode_step(q, k, v, g, eta, eps: float, S):
+    """One per-channel-gated decode token: g [B,H,dk].  Returns (o, S_new)."""
+    q, k, v, g, eta, S = map(f64, (q, k, v, g, eta, S))
+    o, S_new = kda_forward(q[:, None], k[:, None], v[:, None], g[:, None],
+                           eta[:, None], eps, S)
+    return o[:, 0], S_new
 
 
 def decode_step(q, k, v, g, eta, eps: float, S):

@@ -26,9 +26,19 @@
  * + beta k v^T  and  alpha (I - beta k k^T) h + beta k v^T
  *  = alpha h + k (beta v - alpha beta k^T h)^T.
  *
+ * Per-channel gate (KDA, "Deep Dive into KDA", section 2.3; the KLA Abstract
+ * lists a preconditioned KDA among its variants):
+ *   S_t = (I - beta_t k_t k_t^T) Diag(a_t) S_{t-1} + beta_t v_t k_t^T,
+ *   a_t = exp(g_t) with g_t one log-gate per key channel.
+ * The page's orientation is garbled the same way as the GDN line; with S
+ * mapping keys to values the diagonal acts on the key side, and the page's
+ * order is kept: decay first, then the erase reads the decayed state.  In
+ * h-form, per token:  h <- Diag(a) h  (row i scaled by a_i);  r = h^T k;
+ *                     u = beta (v - r);  h <- h + k u^T;  o = h^T q.
+ *
  * Layouts (row-major, contiguous):
  *   q, k : [B][T][H][dk]     v, o : [B][T][H][dv]
- *   g, eta, beta : [B][T][H]
+ *   g, eta, beta : [B][T][H]  (per-channel gate: g is [B][T][H][dk])
  *   h0, hT : [B][H][dk][dv]  (h0 may be NULL = zeros; hT may be NULL)
  * Heads (b, h) are independent; OpenMP runs them in parallel.
  */
@@ -116,6 +126,60 @@ void kla_oracle_forward(const double *q, const double *k, const double *v,
     kla_oracle_beta(k, eta, eps, beta, B, T, H, dk);
     kla_oracle_gated_delta(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv);
     free(beta);
+}
+
+/* The delta rule with a per-channel gate (KDA form), beta given per token. */
+void kla_oracle_kda(const double *q, const double *k, const double *v,
+                    const double *g, const double *beta,
+                    const double *h0, double *o, double *hT,
+                    int B, int T, int H, int dk, int dv)
+{
+    int nheads = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < nheads; ++bh) {
+        int b = bh / H, hh = bh % H;
+        double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+        double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+        if (h0)
+            memcpy(S, h0 + (size_t)bh * dk * dv, sizeof(double) * (size_t)dk * dv);
+        else
+            memset(S, 0, sizeof(double) * (size_t)dk * dv);
+        for (int t = 0; t < T; ++t) {
+            size_t tok = ((size_t)b * T + t) * H + hh;
+            const double *kt = k + tok * dk;
+            const double *qt = q + tok * dk;
+            const double *vt = v + tok * dv;
+            const double *gt = g + tok * dk;
+            double bt = beta[tok];
+            /* Diag(a_t) S_{t-1}: row i of h (key channel i) times exp(g_i) */
+            for (int i = 0; i < dk; ++i) {
+                double a = exp(gt[i]);
+                double *Si = S + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) Si[j] *= a;
+            }
+            /* u = beta (v - h^T k), from the decayed state */
+            for (int j = 0; j < dv; ++j) u[j] = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                const double *Si = S + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) u[j] += Si[j] * kt[i];
+            }
+            for (int j = 0; j < dv; ++j) u[j] = bt * (vt[j] - u[j]);
+            /* h += k u^T; o = h^T q with the updated state */
+            for (int i = 0; i < dk; ++i) {
+                double *Si = S + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) Si[j] += kt[i] * u[j];
+            }
+            double *ot = o + tok * dv;
+            for (int j = 0; j < dv; ++j) ot[j] = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                const double *Si = S + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) ot[j] += Si[j] * qt[i];
+            }
+        }
+        if (hT) memcpy(hT + (size_t)bh * dk * dv, S, sizeof(double) * (size_t)dk * dv);
+        free(S);
+        free(u);
+    }
 }
 
 /* Number of OpenMP threads a parallel region would use (for reporting). */
