@@ -32,6 +32,14 @@ SIGNATURES = {
                              _i, _i, _i, _i, _i, _vp]),
     "kla_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
                                    _i, _i, _i, _i, _i, _i, _vp]),
+    "kla_kda_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
+                         _i, _i, _i, _i, _i, _i, _vp]),
+    "kla_kda_fwd_beta": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                              _i, _i, _i, _i, _i, _i, _vp]),
+    "kla_kda_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp,
+                                 _i, _i, _i, _i, _i, _vp]),
+    "kla_kda_decode_step_beta": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _i, _i, _i, _i, _i, _vp]),
     "kla_check_device_error": (_i, [_vp]),
     "kla_status_string": (ctypes.c_char_p, [_i]),
     "kla_version": (_i, []),

@@ -215,6 +215,70 @@ def gdn_decode_step(q, k, v, g, beta, S, *, o=None, stream=None):
     return o
 
 
+def _kda_prefill(fn, name, q, k, v, g, step, eps, h0, o, hT, return_state, stream):
+    # the per-token arguments as for chunk_fwd; g is checked on its own
+    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, None, step, h0, o, hT, return_state)
+    if g is None:
+        raise ValueError("g must be a CUDA tensor")
+    _need(g, "g", torch.float32, (B, T, H, dk))
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
+    if eps is not None:
+        args.append(float(eps))
+    st = fn(*args, _ptr(h0), _ptr(o), _ptr(hT), B, T, H, dk, dv, _DT[q.dtype],
+            _stream(stream))
+    _check(st, name)
+    return o, hT
+
+
+def kda_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
+            return_state: bool = True, stream=None):
+    """KLA prefill with a per-channel gate (kla_kda_fwd): g [B,T,H,dk] fp32,
+    one log-gate per key channel.  Returns (o, hT)."""
+    return _kda_prefill(_native.lib().kla_kda_fwd, "kla_kda_fwd", q, k, v, g, eta, eps, h0,
+                        o, hT, return_state, stream)
+
+
+def kda_fwd_beta(q, k, v, g, beta, h0=None, *, o=None, hT=None, return_state: bool = True,
+                 stream=None):
+    """Per-channel-gated prefill with beta given per token (kla_kda_fwd_beta)."""
+    return _kda_prefill(_native.lib().kla_kda_fwd_beta, "kla_kda_fwd_beta", q, k, v, g, beta,
+                        None, h0, o, hT, return_state, stream)
+
+
+def _kda_decode(fn, name, q, k, v, g, step, eps, S, o, stream):
+    _need(q, "q")
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v must be bfloat16 or float32")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", q.dtype, (B, H, dk))
+    _need(v, "v", q.dtype, (B, H, dv))
+    _need(g, "g", torch.float32, (B, H, dk))
+    _need(step, "eta" if eps is not None else "beta", torch.float32, (B, H))
+    _need(S, "S", torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, (B, H, dv))
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
+    if eps is not None:
+        args.append(float(eps))
+    _check(fn(*args, _ptr(S), _ptr(o), B, H, dk, dv, _DT[q.dtype], _stream(stream)), name)
+    return o
+
+
+def kda_decode_step(q, k, v, g, eta, S, eps: float = 1e-6, *, o=None, stream=None):
+    """One per-channel-gated decode token (kla_kda_decode_step): g [B,H,dk];
+    S is updated in place.  Returns o [B,H,dv]."""
+    return _kda_decode(_native.lib().kla_kda_decode_step, "kla_kda_decode_step", q, k, v, g,
+                       eta, eps, S, o, stream)
+
+
+def kda_decode_step_beta(q, k, v, g, beta, S, *, o=None, stream=None):
+    """Per-channel-gated decode token with beta given (kla_kda_decode_step_beta)."""
+    return _kda_decode(_native.lib().kla_kda_decode_step_beta, "kla_kda_decode_step_beta",
+                       q, k, v, g, beta, None, S, o, stream)
+
+
 def check_device_error(stream=None):
     """Synchronise and raise KLAError if a kernel reported a timed-out wait."""
     _check(_native.lib().kla_check_device_error(_stream(stream)), "kla_check_device_error")

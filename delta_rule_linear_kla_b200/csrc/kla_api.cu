@@ -42,11 +42,13 @@ static bool head_dims_ok(int dk, int dv) {
   return (dk == 64 && dv == 64) || (dk == 128 && dv == 128);
 }
 
-// Shared validation of the prefill entry points.
+// Shared validation of the prefill entry points; gdim = log-gates per token
+// (1, or dk for the per-channel gate).
 static kla_status check_prefill(const void* q, const void* k, const void* v,
                                 const float* g, const float* eta, float eps,
                                 const float* h0, const void* o, const float* hT,
-                                int B, int T, int H, int dk, int dv, int dtype) {
+                                int B, int T, int H, int dk, int dv, int dtype,
+                                int gdim = 1) {
   if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return KLA_ERR_INVALID_ARG;
   if (dtype != KLA_BF16 && dtype != KLA_FP32) return KLA_ERR_INVALID_ARG;
   if (!(eps >= 0.0f) || eps != eps) return KLA_ERR_INVALID_ARG;
@@ -58,18 +60,18 @@ static kla_status check_prefill(const void* q, const void* k, const void* v,
     if (p && !aligned16(p)) return KLA_ERR_INVALID_ARG;
   if (!head_dims_ok(dk, dv)) return KLA_ERR_UNSUPPORTED;
   const size_t es = dtype == KLA_BF16 ? 2 : 4;
-  const size_t ntok = (size_t)B * T * H;
-  if (o && T > 0) {
-    Range ro = rng(o, ntok * dv * es);
+  const size_t ntok = (size_t)B * T * H, sb = (size_t)B * H * dk * dv * 4;
+  if (T > 0) {
+    // o and hT are written: neither may overlap an input (hT may alias h0
+    // exactly) or the other
     Range ins[] = {rng(q, ntok * dk * es), rng(k, ntok * dk * es), rng(v, ntok * dv * es),
-                   rng(g, ntok * 4), rng(eta, ntok * 4),
-                   rng(h0, h0 ? (size_t)B * H * dk * dv * 4 : 0),
-                   rng(hT, hT ? (size_t)B * H * dk * dv * 4 : 0)};
+                   rng(g, ntok * gdim * 4), rng(eta, ntok * 4)};
+    Range ro = rng(o, ntok * dv * es), rh = rng(hT, hT ? sb : 0);
     for (Range r : ins)
-      if (overlap(ro, r)) return KLA_ERR_INVALID_ARG;
+      if (overlap(ro, r) || overlap(rh, r)) return KLA_ERR_INVALID_ARG;
+    if (overlap(ro, rng(h0, h0 ? sb : 0)) || overlap(ro, rh)) return KLA_ERR_INVALID_ARG;
   }
   if (hT && h0 && hT != h0) {
-    const size_t sb = (size_t)B * H * dk * dv * 4;
     if (overlap(rng(hT, sb), rng(h0, sb))) return KLA_ERR_INVALID_ARG;
   }
   return KLA_OK;
@@ -143,7 +145,7 @@ static kla_status chunk_fwd_impl(const void* q, const void* k, const void* v,
     return KLA_ERR_INVALID_ARG;
   cudaError_t e;
   if (dtype == KLA_FP32) {
-    e = launch_recurrent(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype, st);
+    e = launch_recurrent(q, k, v, g, false, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype, st);
   } else {
     unsigned int* err = device_error_ptr();
     if (!err) return KLA_ERR_CUDA;
@@ -238,18 +240,53 @@ kla_status kla_recurrent_fwd(const void* q, const void* k, const void* v,
   if (s != KLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   if (T == 0) return empty_prefill(h0, hT, B, H, dk, dv, st);
-  cudaError_t e = launch_recurrent(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv,
+  cudaError_t e = launch_recurrent(q, k, v, g, false, eta, eps, h0, o, hT, B, T, H, dk, dv,
                                    dtype, st);
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
 
 }  // extern "C"
 
-// One decode step with the KLA step size, or (eps == kBetaGiven) beta given.
+// Prefill with the per-channel gate (token-serial kernel), KLA step size or
+// (eps == kBetaGiven) beta given.
+static kla_status kda_fwd_impl(const void* q, const void* k, const void* v, const float* g,
+                               const float* eta, float eps, const float* h0, void* o,
+                               float* hT, int B, int T, int H, int dk, int dv, int dtype,
+                               void* stream) {
+  kla_status s = check_prefill(q, k, v, g, eta, eps < 0.f ? 0.f : eps, h0, o, hT, B, T, H,
+                               dk, dv, dtype, dk);
+  if (s != KLA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (T == 0) return empty_prefill(h0, hT, B, H, dk, dv, st);
+  cudaError_t e = launch_recurrent(q, k, v, g, true, eta, eps, h0, o, hT, B, T, H, dk, dv,
+                                   dtype, st);
+  return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+extern "C" {
+
+kla_status kla_kda_fwd(const void* q, const void* k, const void* v, const float* g,
+                       const float* eta, float eps, const float* h0, void* o, float* hT,
+                       int B, int T, int H, int dk, int dv, int dtype, void* stream) {
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  return kda_fwd_impl(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype, stream);
+}
+
+kla_status kla_kda_fwd_beta(const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, const float* h0, void* o, float* hT, int B,
+                            int T, int H, int dk, int dv, int dtype, void* stream) {
+  return kda_fwd_impl(q, k, v, g, beta, kBetaGiven, h0, o, hT, B, T, H, dk, dv, dtype,
+                      stream);
+}
+
+}  // extern "C"
+
+// One decode step with the KLA step size, or (eps == kBetaGiven) beta given;
+// a per-channel gate when vector_gate (g [B][H][dk]).
 static kla_status decode_impl(const void* q, const void* k, const void* v,
                               const float* g, const float* eta, float eps, float* S,
                               void* o, int B, int H, int dk, int dv, int dtype,
-                              void* stream) {
+                              void* stream, bool vector_gate = false) {
   if (B < 1 || H < 1) return KLA_ERR_INVALID_ARG;
   if (dtype != KLA_BF16 && dtype != KLA_FP32) return KLA_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, g, eta, S, o};
@@ -259,11 +296,13 @@ static kla_status decode_impl(const void* q, const void* k, const void* v,
   const size_t es = dtype == KLA_BF16 ? 2 : 4;
   const size_t nh = (size_t)B * H;
   Range ro = rng(o, nh * dv * es);
-  Range others[] = {rng(q, nh * dk * es), rng(k, nh * dk * es), rng(v, nh * dv * es),
-                    rng(g, nh * 4), rng(eta, nh * 4), rng(S, nh * dk * dv * 4)};
-  for (Range r : others)
-    if (overlap(ro, r)) return KLA_ERR_INVALID_ARG;
-  cudaError_t e = launch_decode(q, k, v, g, eta, eps, S, o, B, H, dk, dv, dtype,
+  Range rs = rng(S, nh * dk * dv * 4);
+  Range ins[] = {rng(q, nh * dk * es), rng(k, nh * dk * es), rng(v, nh * dv * es),
+                 rng(g, nh * (vector_gate ? dk : 1) * 4), rng(eta, nh * 4)};
+  if (overlap(ro, rs)) return KLA_ERR_INVALID_ARG;
+  for (Range r : ins)
+    if (overlap(ro, r) || overlap(rs, r)) return KLA_ERR_INVALID_ARG;
+  cudaError_t e = launch_decode(q, k, v, g, vector_gate, eta, eps, S, o, B, H, dk, dv, dtype,
                                 (cudaStream_t)stream);
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
@@ -282,6 +321,19 @@ kla_status kla_gdn_decode_step(const void* q, const void* k, const void* v,
                                const float* g, const float* beta, float* S, void* o, int B,
                                int H, int dk, int dv, int dtype, void* stream) {
   return decode_impl(q, k, v, g, beta, kBetaGiven, S, o, B, H, dk, dv, dtype, stream);
+}
+
+kla_status kla_kda_decode_step(const void* q, const void* k, const void* v, const float* g,
+                               const float* eta, float eps, float* S, void* o, int B, int H,
+                               int dk, int dv, int dtype, void* stream) {
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  return decode_impl(q, k, v, g, eta, eps, S, o, B, H, dk, dv, dtype, stream, true);
+}
+
+kla_status kla_kda_decode_step_beta(const void* q, const void* k, const void* v,
+                                    const float* g, const float* beta, float* S, void* o,
+                                    int B, int H, int dk, int dv, int dtype, void* stream) {
+  return decode_impl(q, k, v, g, beta, kBetaGiven, S, o, B, H, dk, dv, dtype, stream, true);
 }
 
 kla_status kla_check_device_error(void* stream) {

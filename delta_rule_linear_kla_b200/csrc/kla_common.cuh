@@ -28,12 +28,14 @@ __device__ __forceinline__ float step_size(float eta, float knorm2, float eps) {
 }
 
 // Launchers (one per kernel family), all queue work on `st` only.
+// vector_gate: g holds one log-gate per key channel (KDA form) instead of one
+// per token / head.
 cudaError_t launch_decode(const void* q, const void* k, const void* v,
-                          const float* g, const float* eta, float eps, float* S,
-                          void* o, int B, int H, int dk, int dv, int dtype,
+                          const float* g, bool vector_gate, const float* eta, float eps,
+                          float* S, void* o, int B, int H, int dk, int dv, int dtype,
                           cudaStream_t st);
 cudaError_t launch_recurrent(const void* q, const void* k, const void* v,
-                             const float* g, const float* eta, float eps,
+                             const float* g, bool vector_gate, const float* eta, float eps,
                              const float* h0, void* o, float* hT, int B, int T,
                              int H, int dk, int dv, int dtype, cudaStream_t st);
 

@@ -8,8 +8,11 @@
 //   h <- alpha h + k u^T              (one write of the state)
 //   o = h_new^T q = alpha s + u (k . q)
 // which is one step of the gated delta rule ("Deep Dive into KDA",
-// section 2.2) with o read from the updated state.  Columns of h are
-// independent, so a CTA owns one head and a slab of CW columns.
+// section 2.2) with o read from the updated state.  With a per-channel gate
+// (KDA form, same page, section 2.3) the rows of h are scaled by
+// a_i = exp(g_i) as they are loaded and the step above runs on the decayed
+// state with alpha = 1.  Columns of h are independent, so a CTA owns one head
+// and a slab of CW columns.
 //
 // The state is the only large operand (DK*DV*4 bytes per head, read once and
 // written once with 128-bit accesses); the kernel is a pure HBM stream, so
@@ -20,7 +23,8 @@
 
 namespace kla {
 
-template <typename T, int DK, int DV, int CW, int NT>
+// VG: g is per key channel ([B][H][DK]) instead of per head.
+template <typename T, int DK, int DV, int CW, int NT, bool VG>
 __global__ void __launch_bounds__(NT)
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k,
               const T* __restrict__ v, const float* __restrict__ g,
@@ -60,6 +64,13 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k,
     kr[m] = IO<T>::ld(kp + row0 + m * RPP);
     qr[m] = IO<T>::ld(qp + row0 + m * RPP);
   }
+  if constexpr (VG) {  // Diag(a) h: row i of the state times exp(g_i)
+#pragma unroll
+    for (int m = 0; m < RT; ++m) {
+      const float a = expf(g[(size_t)head * DK + row0 + m * RPP]);
+      hv[m].x *= a; hv[m].y *= a; hv[m].z *= a; hv[m].w *= a;
+    }
+  }
 
   // ||k||^2 and k.q over the full key dimension (warp 0).
   if (tid < 32) {
@@ -90,7 +101,7 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k,
   *reinterpret_cast<float4*>(&red_s[row0][4 * c4]) = ps;
   __syncthreads();
 
-  const float alpha = expf(g[head]);
+  const float alpha = VG ? 1.f : expf(g[head]);
   const float beta = step_size(eta[head], kq_sh[0], eps);
   if (tid < CW) {
     float r = 0.f, s = 0.f;
@@ -119,31 +130,37 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k,
 
 template <typename T, int DK, int DV>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v,
-                                   const float* g, const float* eta, float eps,
-                                   float* S, void* o, int B, int H,
+                                   const float* g, bool vector_gate, const float* eta,
+                                   float eps, float* S, void* o, int B, int H,
                                    cudaStream_t st) {
   constexpr int CW = (DV >= 128) ? 64 : DV;
   constexpr int NT = 256;
   const int grid = B * H * (DV / CW);
-  decode_kernel<T, DK, DV, CW, NT><<<grid, NT, 0, st>>>(
-      (const T*)q, (const T*)k, (const T*)v, g, eta, eps, S, (T*)o, H);
+  if (vector_gate)
+    decode_kernel<T, DK, DV, CW, NT, true><<<grid, NT, 0, st>>>(
+        (const T*)q, (const T*)k, (const T*)v, g, eta, eps, S, (T*)o, H);
+  else
+    decode_kernel<T, DK, DV, CW, NT, false><<<grid, NT, 0, st>>>(
+        (const T*)q, (const T*)k, (const T*)v, g, eta, eps, S, (T*)o, H);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v,
-                          const float* g, const float* eta, float eps, float* S,
-                          void* o, int B, int H, int dk, int dv, int dtype,
+                          const float* g, bool vector_gate, const float* eta, float eps,
+                          float* S, void* o, int B, int H, int dk, int dv, int dtype,
                           cudaStream_t st) {
+  const bool vg = vector_gate;
   if (dtype == KLA_BF16) {
     if (dk == 128 && dv == 128)
-      return launch_decode_t<__nv_bfloat16, 128, 128>(q, k, v, g, eta, eps, S, o, B, H, st);
+      return launch_decode_t<__nv_bfloat16, 128, 128>(q, k, v, g, vg, eta, eps, S, o, B, H,
+                                                      st);
     if (dk == 64 && dv == 64)
-      return launch_decode_t<__nv_bfloat16, 64, 64>(q, k, v, g, eta, eps, S, o, B, H, st);
+      return launch_decode_t<__nv_bfloat16, 64, 64>(q, k, v, g, vg, eta, eps, S, o, B, H, st);
   } else {
     if (dk == 128 && dv == 128)
-      return launch_decode_t<float, 128, 128>(q, k, v, g, eta, eps, S, o, B, H, st);
+      return launch_decode_t<float, 128, 128>(q, k, v, g, vg, eta, eps, S, o, B, H, st);
     if (dk == 64 && dv == 64)
-      return launch_decode_t<float, 64, 64>(q, k, v, g, eta, eps, S, o, B, H, st);
+      return launch_decode_t<float, 64, 64>(q, k, v, g, vg, eta, eps, S, o, B, H, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -33,6 +33,10 @@ prefilled state):
                  precision.
 
 eps = 1e-6 and chunk C = 64 everywhere.
+
+Per-channel gates (the KDA form) replace g by one log-gate per key channel,
+drawn by :func:`channel_gates`: g = -softplus(N(3, 1.5)) i.i.d. per channel,
+so most channels forget slowly (alpha ~ 0.95) and a tail forgets fast.
 """
 from __future__ import annotations
 
@@ -141,6 +145,13 @@ def _draw_tokens(rng, kind, B, T, H, dk, dv):
     else:
         raise ValueError(kind)
     return q, k, v, g.astype(np.float32), eta.astype(np.float32)
+
+
+def channel_gates(shape, seed: int) -> torch.Tensor:
+    """Per-key-channel log-gates of the given shape (last axis = channel),
+    fp32: g = -softplus(N(3, 1.5)), drawn from their own seeded stream."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return torch.from_numpy((-_softplus(rng.normal(3.0, 1.5, shape))).astype(np.float32))
 
 
 def make_prefill(w: Workload, with_h0: Optional[bool] = None):

@@ -189,6 +189,44 @@ KLA_API kla_status kla_gdn_decode_step(const void *q, const void *k, const void 
                                int B, int H, int dk, int dv, int dtype, void *stream);
 
 /*
+ * Per-channel gate (KDA form, "Deep Dive into KDA", section 2.3; the
+ * "Kaczmarz Linear Attention" Abstract lists its preconditioned variant):
+ *
+ *   h_t = (I - beta_t k_t k_t^T) Diag(a_t) h_{t-1} + beta_t k_t v_t^T,
+ *   a_t = exp(g_t),  o_t = h_t^T q_t   (h = S^T, [dk][dv] per head)
+ *
+ * with one log-gate per key channel: g is [B][T][H][dk] fp32 for the
+ * prefill and [B][H][dk] fp32 for the decode step (any value <= 0 is
+ * meaningful; larger values grow the state).  Row i of the state decays by
+ * a_{t,i} before the erase reads it.  beta_t = eta_t / (||k_t||^2 + eps) for
+ * kla_kda_fwd / kla_kda_decode_step; given per token ([B][T][H] resp.
+ * [B][H] fp32) for the _beta variants.  Every other argument, layout, limit
+ * and error is that of kla_recurrent_fwd resp. kla_decode_step (dtype bf16
+ * or fp32; dk = dv in {64, 128}; o and the written states must not overlap
+ * any input, hT may alias h0).  The prefill runs the token-serial CUDA-core
+ * kernel (fp32 arithmetic); the decode step the same one-pass state kernel
+ * as kla_decode_step.
+ */
+KLA_API kla_status kla_kda_fwd(const void *q, const void *k, const void *v,
+                               const float *g, const float *eta, float eps,
+                               const float *h0, void *o, float *hT,
+                               int B, int T, int H, int dk, int dv, int dtype,
+                               void *stream);
+KLA_API kla_status kla_kda_fwd_beta(const void *q, const void *k, const void *v,
+                                    const float *g, const float *beta,
+                                    const float *h0, void *o, float *hT,
+                                    int B, int T, int H, int dk, int dv, int dtype,
+                                    void *stream);
+KLA_API kla_status kla_kda_decode_step(const void *q, const void *k, const void *v,
+                                       const float *g, const float *eta, float eps,
+                                       float *S, void *o, int B, int H, int dk, int dv,
+                                       int dtype, void *stream);
+KLA_API kla_status kla_kda_decode_step_beta(const void *q, const void *k, const void *v,
+                                            const float *g, const float *beta, float *S,
+                                            void *o, int B, int H, int dk, int dv,
+                                            int dtype, void *stream);
+
+/*
  * Chunkwise prefill without any caller-provided device memory.
  *
  * No counterpart in the paper: this is a deployment convenience.  Some

@@ -103,6 +103,31 @@ def test_gdn_entry_points_reject_bad_arguments(lib):
     assert lib.kla_gdn_decode_step(*bad) == UNSUPPORTED
 
 
+def test_kda_entry_points_reject_bad_arguments(lib):
+    """Per-channel gate: g is [B][T][H][dk] (prefill) / [B][H][dk] (decode)."""
+    kda = lambda **kw: lib.kla_kda_fwd(
+        kw.get("q", A), kw.get("k", 2 * A), kw.get("v", 3 * A), kw.get("g", 4 * A),
+        kw.get("eta", 5 * A), kw.get("eps", 1e-6), None, kw.get("o", 6 * A), kw.get("hT", None),
+        1, kw.get("T", 128), 2, kw.get("dk", 128), kw.get("dv", 128), kw.get("dtype", 0), None)
+    assert kda(g=None) == INVALID
+    assert kda(eps=-1.0) == INVALID
+    assert kda(dk=96, dv=96) == UNSUPPORTED
+    # 1 x 128 x 2 x 128 fp32 gates = 128 KiB: o placed inside that range
+    assert kda(o=4 * A + 64 * 1024) == INVALID
+    assert kda(hT=4 * A + 64 * 1024) == INVALID        # written state over the gates
+    assert lib.kla_kda_fwd_beta(A, 2 * A, 3 * A, 4 * A, None, None, 6 * A, None, 1, 4, 1,
+                                64, 64, 1, None) == INVALID
+    args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, 6 * A, 7 * A, 2, 3, 128, 128, 0, None]
+    bad = list(args); bad[7] = 4 * A + 2048          # o inside the 3 KiB of gates
+    assert lib.kla_kda_decode_step(*bad) == INVALID
+    bad = list(args); bad[5] = -1.0
+    assert lib.kla_kda_decode_step(*bad) == INVALID
+    bad = list(args); bad[10], bad[11] = 80, 80
+    assert lib.kla_kda_decode_step(*bad) == UNSUPPORTED
+    bargs = [A, 2 * A, 3 * A, 4 * A, None, 6 * A, 7 * A, 2, 3, 128, 128, 0, None]
+    assert lib.kla_kda_decode_step_beta(*bargs) == INVALID
+
+
 def test_decode_rejects_bad_arguments(lib):
     args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, 6 * A, 7 * A, 2, 3, 128, 128, 0, None]
     bad = list(args); bad[6] = None

@@ -1,0 +1,117 @@
+"""Per-channel gate (KDA form, "Deep Dive into KDA", section 2.3, with the
+KLA step size or beta given) on the GPU against the fp64 oracle: the
+token-serial prefill kernel (bf16 and fp32 I/O) and the decode step."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from delta_rule_linear_kla_b200 import api, inputs
+
+from helpers import TOL, cuda, rel
+
+pytestmark = pytest.mark.gpu
+
+
+def _prefill_inputs(name, B, T, H, dt, seed, with_h0=True):
+    w = inputs.WORKLOADS[name].scaled(B=B, T=T, H=H, dtype=dt, seed=seed)
+    x = inputs.make_prefill(w, with_h0=with_h0)
+    x["gv"] = inputs.channel_gates((B, T, H, w.dk), seed + 1)
+    return w, x
+
+
+@pytest.mark.parametrize("name,T,dt", [("prefill_4k", 1, "bf16"), ("prefill_4k", 130, "bf16"),
+                                       ("stress", 97, "bf16"), ("tiny", 150, "fp32"),
+                                       ("prefill_4k", 70, "fp32")])
+def test_kda_prefill(name, T, dt):
+    w, x = _prefill_inputs(name, 2, T, 2, dt, 41)
+    xc = cuda(x)
+    o, hT = api.kda_fwd(xc["q"], xc["k"], xc["v"], xc["gv"], xc["eta"], x["eps"], xc["h0"])
+    api.check_device_error()
+    o_ref, h_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["gv"], x["eta"], x["eps"],
+                                      x["h0"])
+    assert rel(o.cpu(), o_ref) < TOL[dt] and rel(hT.cpu(), h_ref) < TOL[dt]
+
+
+def test_kda_prefill_beta_given():
+    w, x = _prefill_inputs("prefill_4k", 1, 90, 3, "bf16", 43)
+    kf = x["k"].float()
+    k = (kf / kf.norm(dim=-1, keepdim=True).clamp_min(1e-6)).to(x["k"].dtype)
+    rng = np.random.Generator(np.random.PCG64(44))
+    beta = torch.from_numpy((1 / (1 + np.exp(-rng.normal(size=(1, 90, 3))))).astype(np.float32))
+    xc = cuda(x)
+    o, hT = api.kda_fwd_beta(xc["q"], cuda(k), xc["v"], xc["gv"], cuda(beta), xc["h0"])
+    api.check_device_error()
+    o_ref, h_ref = oracle.kda(x["q"], k, x["v"], x["gv"], beta, x["h0"])
+    assert rel(o.cpu(), o_ref) < TOL["bf16"] and rel(hT.cpu(), h_ref) < TOL["bf16"]
+
+
+def test_uniform_channel_gate_equals_scalar_gate_kernel():
+    """A gate equal on every channel is the scalar gate: the per-channel
+    token-serial kernel agrees with the scalar one to fp32 rounding."""
+    w, x = _prefill_inputs("tiny", 1, 200, 2, "fp32", 45)
+    gv = x["g"][..., None].expand(-1, -1, -1, w.dk).contiguous()
+    xc = cuda(x)
+    o1, h1 = api.kda_fwd(xc["q"], xc["k"], xc["v"], cuda(gv), xc["eta"], x["eps"], xc["h0"])
+    o2, h2 = api.recurrent_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"],
+                               xc["h0"])
+    torch.cuda.synchronize()
+    assert rel(o1.cpu(), o2.cpu()) < 1e-5 and rel(h1.cpu(), h2.cpu()) < 1e-5
+
+
+def test_kda_prefill_wiped_channels_and_empty():
+    """Channels whose gate wipes them (g = -200: a = 0) and a zero-length
+    prefill (hT = h0)."""
+    w, x = _prefill_inputs("prefill_4k", 1, 80, 2, "fp32", 47)
+    x["gv"][0, 10:20, :, ::7] = -200.0
+    xc = cuda(x)
+    o, hT = api.kda_fwd(xc["q"], xc["k"], xc["v"], xc["gv"], xc["eta"], x["eps"], xc["h0"])
+    api.check_device_error()
+    o_ref, h_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["gv"], x["eta"], x["eps"],
+                                      x["h0"])
+    assert rel(o.cpu(), o_ref) < TOL["fp32"] and rel(hT.cpu(), h_ref) < TOL["fp32"]
+    q0 = xc["q"][:, :0].contiguous()
+    _, h_empty = api.kda_fwd(q0, q0, xc["v"][:, :0].contiguous(),
+                             xc["gv"][:, :0].contiguous(), xc["eta"][:, :0].contiguous(),
+                             x["eps"], xc["h0"])
+    torch.cuda.synchronize()
+    assert torch.equal(h_empty, xc["h0"])
+
+
+@pytest.mark.parametrize("dt,d", [("bf16", 128), ("fp32", 128), ("bf16", 64)])
+def test_kda_decode(dt, d):
+    w = inputs.DECODE.scaled(B=3, H=4, dk=d, dv=d, dtype=dt, prefix_tokens=24)
+    dd = inputs.make_decode(w, steps=5)
+    st = dd["steps"]
+    gv = inputs.channel_gates((5, w.B, w.H, d), 49)
+    rng = np.random.Generator(np.random.PCG64(50))
+    S0 = torch.from_numpy(rng.normal(0, 0.1, (w.B, w.H, d, d)).astype(np.float32))
+    S = cuda(S0.clone())
+    Sref = oracle.f64(S0)
+    for i in range(5):
+        args = [st[n][i] for n in ("q", "k", "v")]
+        o = api.kda_decode_step(*(cuda(a) for a in args), cuda(gv[i]), cuda(st["eta"][i]), S,
+                                dd["eps"])
+        o_ref, Sref = oracle.kda_decode_step(*args, gv[i], st["eta"][i], dd["eps"], Sref)
+        assert rel(o.cpu(), o_ref) < TOL[dt]
+    api.check_device_error()
+    assert rel(S.cpu(), Sref) < TOL["fp32"]
+
+
+def test_kda_decode_beta_given():
+    w = inputs.DECODE.scaled(B=2, H=3, dtype="bf16", prefix_tokens=24)
+    dd = inputs.make_decode(w, steps=3)
+    st = dd["steps"]
+    gv = inputs.channel_gates((3, w.B, w.H, w.dk), 51)
+    rng = np.random.Generator(np.random.PCG64(52))
+    beta = torch.from_numpy(rng.uniform(0.0, 1.0, (3, w.B, w.H)).astype(np.float32))
+    S = cuda(torch.zeros(w.B, w.H, w.dk, w.dv))
+    Sref = np.zeros((w.B, w.H, w.dk, w.dv))
+    for i in range(3):
+        args = [st[n][i] for n in ("q", "k", "v")]
+        o = api.kda_decode_step_beta(*(cuda(a) for a in args), cuda(gv[i]), cuda(beta[i]), S)
+        o_ref, Sref = oracle.kda(*(a[:, None] for a in args), gv[i][:, None], beta[i][:, None],
+                                 Sref)
+        assert rel(o.cpu(), o_ref[:, 0]) < TOL["bf16"]
+    torch.cuda.synchronize()
+    assert rel(S.cpu(), Sref) < TOL["fp32"]
