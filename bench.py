@@ -328,6 +328,8 @@ def run_ours(args, rank, world, dev):
                 "%d segments: transitions, start states, outputs" % nseg)
     if not args.no_decode:
         res["decode"] = run_decode(args, rank, dev, stream, flush, peaks, peak_src, fn, clk)
+    if not args.no_kda and w.dtype == "bf16":
+        res["kda_prefill"] = run_kda_prefill(w, dev, stream, flush, peaks, peak_src)
     time.sleep(0.25)
     clk.__exit__()
     res["clocks"] = clk.summary(t_load, t1 + 0.15)
@@ -337,33 +339,54 @@ def run_ours(args, rank, world, dev):
 
 
 def measure_e2e(args, w, x, fn, dev, stream, world):
-    """Same metric through the public call with pinned host buffers: H2D of
-    the step's inputs, the prefill, D2H of o and hT, all inside the events."""
+    """Same metric end to end from pinned host buffers: H2D of the step's
+    inputs, the prefill, D2H of o and hT, all inside the events.  The chunk
+    path goes through the C ABI's host-buffer entry point
+    (kla_chunk_fwd_host), which pipelines the copies against the kernels
+    sequence by sequence; the token-serial path copies, runs and copies back
+    in turn."""
+    from delta_rule_linear_kla_b200 import api
+
     host = {k: x[k].pin_memory() for k in ("q", "k", "v", "g", "eta")}
-    dbuf = {k: torch.empty_like(host[k], device=dev) for k in host}
     o_h = torch.empty((w.B, w.T, w.H, w.dv), dtype=w.torch_dtype).pin_memory()
     h_h = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32).pin_memory()
-    o = torch.empty_like(o_h, device=dev)
-    hT = torch.empty_like(h_h, device=dev)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = o_h.numel() * o_h.element_size() + h_h.numel() * h_h.element_size()
+    if args.path == "chunk":
+        need = api.chunk_fwd_host_staging_size(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype)
+        staging = torch.empty(need, dtype=torch.uint8, device=dev)
+
+        def step():
+            api.chunk_fwd_host(host["q"], host["k"], host["v"], host["g"], host["eta"],
+                               x["eps"], None, o=o_h, hT=h_h, staging=staging, stream=stream)
+        how = "kla_chunk_fwd_host (copies pipelined per sequence against the kernels)"
+    else:
+        dbuf = {k: torch.empty_like(host[k], device=dev) for k in host}
+        o = torch.empty_like(o_h, device=dev)
+        hT = torch.empty_like(h_h, device=dev)
+
+        def step():
+            for k in dbuf:
+                dbuf[k].copy_(host[k], non_blocking=True)
+            fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["eta"], x["eps"], None, o=o,
+               hT=hT)
+            o_h.copy_(o, non_blocking=True)
+            h_h.copy_(hT, non_blocking=True)
+        how = "H2D copies, kla_recurrent_fwd, D2H copies in turn"
     n = max(2, min(args.steps, 5))
     times = []
     for i in range(n + 2):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for k in dbuf:
-            dbuf[k].copy_(host[k], non_blocking=True)
-        fn(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["eta"], x["eps"], None, o=o, hT=hT)
-        o_h.copy_(o, non_blocking=True)
-        h_h.copy_(hT, non_blocking=True)
+        step()
         e1.record(stream)
         torch.cuda.synchronize()
         if i >= 2:
             times.append(e0.elapsed_time(e1))
     ms = allreduce_max(sum(times) / len(times), world, dev)
     return {"value": w.B * w.T * world / (ms / 1e3), "unit": "tokens/s",
-            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "path": how}
 
 
 def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn, clk):
@@ -398,6 +421,28 @@ def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn, clk)
     io_bytes = w.B * w.H * (2 * w.dk + 2 * w.dv) * 2 + w.B * w.H * 8
     gbs = (state_bytes + io_bytes) / (ms / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
+
+    # the same steps with a per-channel gate (KDA form): 16 gate sets of
+    # [B, H, dk] drawn once and cycled (the gate values do not change the
+    # work); one more [B, H, dk] fp32 read per step than the scalar gate
+    gv = inputs.channel_gates((16, w.B, w.H, w.dk), w.seed + 7).to(dev)
+    kevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(nsteps)]
+    for i in range(3):
+        api.kda_decode_step(st["q"][i], st["k"][i], st["v"][i], gv[i % 16], st["eta"][i], S,
+                            d["eps"], o=o)
+    torch.cuda.synchronize()
+    for i, (e0, e1) in enumerate(kevs):
+        flush()
+        e0.record(stream)
+        api.kda_decode_step(st["q"][i], st["k"][i], st["v"][i], gv[i % 16], st["eta"][i], S,
+                            d["eps"], o=o)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    api.check_device_error()
+    kms = sum(a.elapsed_time(b) for a, b in kevs) / nsteps
+    kbytes = state_bytes + io_bytes + w.B * w.H * (w.dk - 1) * 4
+    kgbs = kbytes / (kms / 1e3) / 1e9
     return {"metric": "decode tokens/s (B=64 H=16 d=128, 32K-token state)",
             "value": w.B / (ms / 1e3), "unit": "tokens/s", "us_per_step": ms * 1e3,
             "steps": nsteps, "l2": "flushed before every step",
@@ -407,6 +452,53 @@ def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn, clk)
                          "traffic": profiled_traffic("kla_decode.cu",
                                                      "decode_kernel_decode_b64.md"),
                          "algorithmic_bytes": state_bytes + io_bytes,
+                         "peak_source": peak_src},
+            "per_channel_gate": {
+                "value": w.B / (kms / 1e3), "unit": "tokens/s", "us_per_step": kms * 1e3,
+                "steps": nsteps, "gpu_launches": nsteps,
+                "roofline": {"kernel": "decode_kernel (per-channel gate)", "bound": "hbm",
+                             "achieved": kgbs, "peak": peak, "unit": "GB/s",
+                             "frac": kgbs / peak, "traffic": None,
+                             "algorithmic_bytes": kbytes, "peak_source": peak_src}}}
+
+
+def run_kda_prefill(w, dev, stream, flush, peaks, peak_src, steps=3):
+    """The per-channel-gate prefill (token-serial kernel) on the same
+    workload's q, k, v, eta with per-channel gates: time per launch and
+    achieved GB/s of its algorithmic bytes (q, k, v, o, the [B,T,H,dk] gates,
+    eta, h_T)."""
+    from delta_rule_linear_kla_b200 import api, inputs
+
+    x = inputs.make_prefill(w)
+    xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    gv = inputs.channel_gates((w.B, w.T, w.H, w.dk), w.seed + 11).to(dev)
+    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=w.torch_dtype, device=dev)
+    hT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    run = lambda: api.kda_fwd(xd["q"], xd["k"], xd["v"], gv, xd["eta"], x["eps"], xd["h0"],
+                              o=o, hT=hT)
+    run()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for e0, e1 in evs:
+        flush()
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    api.check_device_error()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    es = 2 if w.dtype == "bf16" else 4
+    ntok = w.B * w.T * w.H
+    byts = ntok * (2 * w.dk + 2 * w.dv) * es + ntok * (w.dk + 1) * 4 + w.B * w.H * w.dk * w.dv * 4
+    gbs = byts / (ms / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    return {"metric": "prefill tokens/s, per-channel gate, token-serial kernel (%s)" % w.name,
+            "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_launch": ms,
+            "launches": steps, "path": "token-serial (CUDA cores, fp32 arithmetic)",
+            "roofline": {"kernel": "recurrent_kernel (per-channel gate)", "bound": "hbm",
+                         "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "algorithmic_bytes": byts,
                          "peak_source": peak_src}}
 
 
@@ -527,6 +619,8 @@ def main():
     ap.add_argument("--path", choices=["chunk", "recurrent"], default="chunk")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-kda", action="store_true",
+                    help="skip the per-channel-gate (KDA form) prefill measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -215,6 +215,57 @@ def gdn_decode_step(q, k, v, g, beta, S, *, o=None, stream=None):
     return o
 
 
+def _need_host(t, name, dtype, shape):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise ValueError("%s must be a host (CPU) tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must be %s of shape %s" % (name, dtype, tuple(shape)))
+
+
+def chunk_fwd_host_staging_size(B: int, T: int, H: int, dk: int, dv: int,
+                                dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(_native.lib().kla_chunk_fwd_host_staging_size(B, T, H, dk, dv, _DT[dtype]))
+
+
+def chunk_fwd_host(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
+                   return_state: bool = True, staging=None, device=None, stream=None):
+    """Prefill from host tensors (kla_chunk_fwd_host): the copies to and
+    from the device are pipelined against the kernels.  Inputs and outputs
+    are CPU tensors (pin them for the copies to overlap; outputs allocated
+    here are pinned).  Only enqueues work: synchronise ``stream`` before
+    reading o, hT.  Returns (o, hT)."""
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v must be bfloat16 or float32")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n, dt, sh in ((q, "q", q.dtype, (B, T, H, dk)), (k, "k", q.dtype, (B, T, H, dk)),
+                         (v, "v", q.dtype, (B, T, H, dv)), (g, "g", torch.float32, (B, T, H)),
+                         (eta, "eta", torch.float32, (B, T, H)),
+                         (h0, "h0", torch.float32, (B, H, dk, dv))):
+        _need_host(t, n, dt, sh)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, pin_memory=True)
+    _need_host(o, "o", q.dtype, (B, T, H, dv))
+    if hT is None and return_state:
+        hT = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
+    _need_host(hT, "hT", torch.float32, (B, H, dk, dv))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    need = chunk_fwd_host_staging_size(B, T, H, dk, dv, q.dtype)
+    if staging is None:
+        staging = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _need(staging, "staging", torch.uint8)
+    st = _native.lib().kla_chunk_fwd_host(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0), _ptr(o),
+        _ptr(hT), B, T, H, dk, dv, _DT[q.dtype], _ptr(staging),
+        staging.numel() * staging.element_size(), _stream(stream))
+    _check(st, "kla_chunk_fwd_host")
+    return o, hT
+
+
 def _kda_prefill(fn, name, q, k, v, g, step, eps, h0, o, hT, return_state, stream):
     # the per-token arguments as for chunk_fwd; g is checked on its own
     B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, None, step, h0, o, hT, return_state)

@@ -25,7 +25,7 @@ namespace kla {
 
 // VG: g is per key channel ([B][H][DK]) instead of per head.
 template <typename T, int DK, int DV, int CW, int NT, bool VG>
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(NT, 65536 / (NT * 64))  // <= 64 registers: 4 CTAs/SM
 decode_kernel(const T* __restrict__ q, const T* __restrict__ k,
               const T* __restrict__ v, const float* __restrict__ g,
               const float* __restrict__ eta, float eps, float* __restrict__ S,

@@ -15,7 +15,8 @@
  *
  * Conventions shared by every call:
  *   * All tensors are device pointers, contiguous, row-major, 16-byte
- *     aligned, on the current device, in the layouts stated per argument.
+ *     aligned, on the current device, in the layouts stated per argument
+ *     (kla_chunk_fwd_host alone takes host pointers).
  *   * The caller owns every buffer (including any workspace).  The library
  *     allocates no device memory and never synchronises the stream: work is
  *     queued on `stream` (a cudaStream_t passed as void*; NULL = legacy
@@ -225,6 +226,31 @@ KLA_API kla_status kla_kda_decode_step_beta(const void *q, const void *k, const 
                                             const float *g, const float *beta, float *S,
                                             void *o, int B, int H, int dk, int dv,
                                             int dtype, void *stream);
+
+/*
+ * Prefill from HOST buffers, end to end: the same computation as
+ * kla_chunk_fwd with q, k, v, g, eta, h0 (nullable), o and hT (nullable) in
+ * host memory (same layouts; page-locked memory is needed for the copies to
+ * run asynchronously and overlap).  T >= 1.
+ *
+ * The batch is cut into pieces of whole sequences; each piece is copied to a
+ * staging slot in `staging` (caller-owned device memory of
+ * kla_chunk_fwd_host_staging_size(...) bytes, 256-byte aligned, else
+ * KLA_ERR_INVALID_ARG), its prefill runs on `stream`, and its outputs are
+ * copied back, with the copy-in of the next piece and the copy-out of the
+ * previous one overlapping the kernels (two copy streams per device, created
+ * on first use and kept).  The call only enqueues work: the host buffers
+ * must stay valid, and o / hT may be read only once `stream` has passed the
+ * call (e.g. after cudaStreamSynchronize).  Calls that share a staging
+ * buffer are ordered by `stream`.  Limits and errors otherwise as
+ * kla_chunk_fwd.
+ */
+KLA_API size_t kla_chunk_fwd_host_staging_size(int B, int T, int H, int dk, int dv, int dtype);
+KLA_API kla_status kla_chunk_fwd_host(const void *q, const void *k, const void *v,
+                                      const float *g, const float *eta, float eps,
+                                      const float *h0, void *o, float *hT,
+                                      int B, int T, int H, int dk, int dv, int dtype,
+                                      void *staging, size_t staging_bytes, void *stream);
 
 /*
  * Chunkwise prefill without any caller-provided device memory.

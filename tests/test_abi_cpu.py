@@ -128,6 +128,28 @@ def test_kda_entry_points_reject_bad_arguments(lib):
     assert lib.kla_kda_decode_step_beta(*bargs) == INVALID
 
 
+def test_host_prefill_rejects_bad_arguments(lib):
+    """kla_chunk_fwd_host: host pointers, a device staging buffer; every
+    check below returns before any CUDA call."""
+    need = lib.kla_chunk_fwd_host_staging_size(3, 100, 2, 64, 64, 0)
+    assert need > 0
+    assert lib.kla_chunk_fwd_host_staging_size(3, 0, 2, 64, 64, 0) == 0
+    assert lib.kla_chunk_fwd_host_staging_size(3, 100, 2, 64, 64, 5) == 0
+    host = lambda **kw: lib.kla_chunk_fwd_host(
+        kw.get("q", A), kw.get("k", 2 * A), kw.get("v", 3 * A), kw.get("g", 4 * A),
+        kw.get("eta", 5 * A), kw.get("eps", 1e-6), None, kw.get("o", 6 * A), None, 3,
+        kw.get("T", 100), 2, kw.get("dk", 64), kw.get("dv", 64), 0, kw.get("st", 64 * A),
+        kw.get("stb", need), None)
+    assert host(q=None) == INVALID
+    assert host(o=None) == INVALID
+    assert host(T=0) == INVALID
+    assert host(eps=-1.0) == INVALID
+    assert host(st=64 * A + 16) == INVALID             # staging not 256-byte aligned
+    assert host(stb=need - 1) == INVALID               # staging too small
+    assert host(st=None) == INVALID
+    assert host(dk=96, dv=96) == UNSUPPORTED
+
+
 def test_decode_rejects_bad_arguments(lib):
     args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, 6 * A, 7 * A, 2, 3, 128, 128, 0, None]
     bad = list(args); bad[6] = None
