@@ -44,6 +44,7 @@ SIGNATURES = {
     "kla_kda_decode_step_beta": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                       _i, _i, _i, _i, _i, _vp]),
     "kla_check_device_error": (_i, [_vp]),
+    "kla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "kla_status_string": (ctypes.c_char_p, [_i]),
     "kla_version": (_i, []),
 }

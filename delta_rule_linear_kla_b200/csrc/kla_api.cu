@@ -5,6 +5,7 @@
 
 #include "kla_common.cuh"
 #include "kla_chunk.h"
+#include "kla_sync.cuh"
 
 namespace kla {
 
@@ -334,6 +335,31 @@ kla_status kla_kda_decode_step_beta(const void* q, const void* k, const void* v,
                                     const float* g, const float* beta, float* S, void* o,
                                     int B, int H, int dk, int dv, int dtype, void* stream) {
   return decode_impl(q, k, v, g, beta, kBetaGiven, S, o, B, H, dk, dv, dtype, stream, true);
+}
+
+}  // extern "C"
+
+namespace kla {
+// One thread waits, with the kernels' bounded wait, on an mbarrier phase
+// that nothing completes (no thread arrives); when the limit runs out it
+// reports a timeout through the device error word, exactly as a stuck
+// tensor-core kernel would, and returns.
+__global__ void selftest_wait_kernel(uint64_t limit_ns, unsigned int* err) {
+  __shared__ uint64_t bar;
+  ptx::mbar_init(&bar, 1);
+  ptx::mbar_init_fence();
+  if (!wait_bounded_ns(&bar, 0, limit_ns)) report_timeout(err);
+}
+}  // namespace kla
+
+extern "C" {
+
+kla_status kla_selftest_wait_timeout(unsigned int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 10000) return KLA_ERR_INVALID_ARG;
+  unsigned int* err = device_error_ptr();
+  if (!err) return KLA_ERR_CUDA;
+  selftest_wait_kernel<<<1, 1, 0, (cudaStream_t)stream>>>((uint64_t)limit_ms * 1000000ull, err);
+  return cudaGetLastError() == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
 
 kla_status kla_check_device_error(void* stream) {

@@ -16,16 +16,22 @@ __device__ __forceinline__ uint64_t globaltimer() {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Returns false if the phase with `parity` did not complete within the limit.
-__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
+// Returns false if the phase with `parity` did not complete within
+// `limit_ns` nanoseconds of %globaltimer.
+__device__ __forceinline__ bool wait_bounded_ns(uint64_t* bar, uint32_t parity,
+                                                uint64_t limit_ns) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (ptx::mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    if (globaltimer() - t0 > limit_ns) return false;
   }
+}
+
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
+  return wait_bounded_ns(bar, parity, kWaitLimitNs);
 }
 
 }  // namespace kla

@@ -292,6 +292,17 @@ KLA_API kla_status kla_chunk_fwd_noalloc(const void *q, const void *k, const voi
  */
 KLA_API kla_status kla_check_device_error(void *stream);
 
+/*
+ * Self-test of that path, for failure-detection tests: launches one thread
+ * that waits, with the same bounded mbarrier wait the tensor-core kernels
+ * use, on a phase nothing ever completes, gives up after `limit_ms`
+ * milliseconds (1 .. 10000, else KLA_ERR_INVALID_ARG), sets the device
+ * error word and returns.  The next kla_check_device_error on that stream
+ * reports KLA_ERR_TIMEOUT; the context stays usable.  No fault, trap or
+ * hang is involved.
+ */
+KLA_API kla_status kla_selftest_wait_timeout(unsigned int limit_ms, void *stream);
+
 /* Static description of a status code (never NULL). */
 KLA_API const char *kla_status_string(int status);
 

@@ -166,6 +166,11 @@ def _ut_bytes(B, T, H):
     return B * H * ((T + 63) // 64) * 16384  # two 64 x 64 bf16 factors per chunk
 
 
+def test_selftest_rejects_bad_limits(lib):
+    assert lib.kla_selftest_wait_timeout(0, None) == INVALID
+    assert lib.kla_selftest_wait_timeout(10001, None) == INVALID
+
+
 def test_workspace_query(lib):
     # enough heads to fill the GPU: the chain runs uncut, factors only
     assert lib.kla_chunk_fwd_workspace_size(8, 4096, 8, 128, 128, 0) == _ut_bytes(8, 4096, 8)
