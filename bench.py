@@ -463,10 +463,10 @@ def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn, clk)
 
 
 def run_kda_prefill(w, dev, stream, flush, peaks, peak_src, steps=3):
-    """The per-channel-gate prefill (token-serial kernel) on the same
-    workload's q, k, v, eta with per-channel gates: time per launch and
-    achieved GB/s of its algorithmic bytes (q, k, v, o, the [B,T,H,dk] gates,
-    eta, h_T)."""
+    """The per-channel-gate prefill (chunk path: per-chunk factor kernel,
+    then the tensor-core state kernel) on the same workload's q, k, v, eta
+    with per-channel gates: time per call and achieved GB/s of its
+    algorithmic bytes (q, k, v, o, the [B,T,H,dk] gates, eta, h_T)."""
     from delta_rule_linear_kla_b200 import api, inputs
 
     x = inputs.make_prefill(w)
@@ -474,8 +474,11 @@ def run_kda_prefill(w, dev, stream, flush, peaks, peak_src, steps=3):
     gv = inputs.channel_gates((w.B, w.T, w.H, w.dk), w.seed + 11).to(dev)
     o = torch.empty((w.B, w.T, w.H, w.dv), dtype=w.torch_dtype, device=dev)
     hT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
-    run = lambda: api.kda_fwd(xd["q"], xd["k"], xd["v"], gv, xd["eta"], x["eps"], xd["h0"],
-                              o=o, hT=hT)
+    ws = torch.empty(max(1, api.kda_chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv,
+                                                             w.torch_dtype)),
+                     dtype=torch.uint8, device=dev)
+    run = lambda: api.kda_chunk_fwd(xd["q"], xd["k"], xd["v"], gv, xd["eta"], x["eps"],
+                                    xd["h0"], o=o, hT=hT, workspace=ws)
     run()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -493,10 +496,12 @@ def run_kda_prefill(w, dev, stream, flush, peaks, peak_src, steps=3):
     byts = ntok * (2 * w.dk + 2 * w.dv) * es + ntok * (w.dk + 1) * 4 + w.B * w.H * w.dk * w.dv * 4
     gbs = byts / (ms / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
-    return {"metric": "prefill tokens/s, per-channel gate, token-serial kernel (%s)" % w.name,
-            "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_launch": ms,
-            "launches": steps, "path": "token-serial (CUDA cores, fp32 arithmetic)",
-            "roofline": {"kernel": "recurrent_kernel (per-channel gate)", "bound": "hbm",
+    return {"metric": "prefill tokens/s, per-channel gate (%s)" % w.name,
+            "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
+            "calls": steps,
+            "path": "kda_prep_kernel (per-chunk factors, CUDA cores fp32) + chain_kernel "
+                    "(KDA mode, tcgen05)",
+            "roofline": {"kernel": "whole call", "bound": "hbm",
                          "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "traffic": None, "algorithmic_bytes": byts,
                          "peak_source": peak_src}}

@@ -35,6 +35,11 @@ SIGNATURES = {
     "kla_chunk_fwd_host_staging_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "kla_chunk_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
                                 _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_kda_chunk_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "kla_kda_chunk_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
+                               _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_kda_chunk_fwd_beta": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                    _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_kda_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
                          _i, _i, _i, _i, _i, _i, _vp]),
     "kla_kda_fwd_beta": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,

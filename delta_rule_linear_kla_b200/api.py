@@ -296,6 +296,44 @@ def kda_fwd_beta(q, k, v, g, beta, h0=None, *, o=None, hT=None, return_state: bo
                         None, h0, o, hT, return_state, stream)
 
 
+def kda_chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
+                                 dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(_native.lib().kla_kda_chunk_fwd_workspace_size(B, T, H, dk, dv, _DT[dtype]))
+
+
+def _kda_chunk(fn, name, q, k, v, g, step, eps, h0, o, hT, return_state, workspace, stream):
+    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, None, step, h0, o, hT, return_state)
+    if g is None:
+        raise ValueError("g must be a CUDA tensor")
+    _need(g, "g", torch.float32, (B, T, H, dk))
+    need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
+    if eps is not None:
+        args.append(float(eps))
+    st = fn(*args, _ptr(h0), _ptr(o), _ptr(hT), B, T, H, dk, dv, CHUNK, _DT[q.dtype],
+            _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, name)
+    return o, hT
+
+
+def kda_chunk_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
+                  return_state: bool = True, workspace=None, stream=None):
+    """Per-channel-gate prefill as chunks (kla_kda_chunk_fwd): g [B,T,H,dk]
+    fp32.  bf16 runs the tensor-core chunk path.  Returns (o, hT)."""
+    return _kda_chunk(_native.lib().kla_kda_chunk_fwd, "kla_kda_chunk_fwd", q, k, v, g, eta,
+                      eps, h0, o, hT, return_state, workspace, stream)
+
+
+def kda_chunk_fwd_beta(q, k, v, g, beta, h0=None, *, o=None, hT=None, return_state: bool = True,
+                       workspace=None, stream=None):
+    """kda_chunk_fwd with beta given per token (kla_kda_chunk_fwd_beta)."""
+    return _kda_chunk(_native.lib().kla_kda_chunk_fwd_beta, "kla_kda_chunk_fwd_beta", q, k, v,
+                      g, beta, None, h0, o, hT, return_state, workspace, stream)
+
+
 def _kda_decode(fn, name, q, k, v, g, step, eps, S, o, stream):
     _need(q, "q")
     if q.dtype not in _DT:

@@ -248,6 +248,41 @@ kla_status kla_recurrent_fwd(const void* q, const void* k, const void* v,
 
 }  // extern "C"
 
+// Prefill with the per-channel gate as chunks: bf16 runs the per-chunk
+// factor kernel and the chain kernel's KDA mode, fp32 the token-serial
+// kernel; KLA step size or (eps == kBetaGiven) beta given.
+static kla_status kda_chunk_impl(const void* q, const void* k, const void* v, const float* g,
+                                 const float* eta, float eps, const float* h0, void* o,
+                                 float* hT, int B, int T, int H, int dk, int dv, int chunk,
+                                 int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  kla_status s = check_prefill(q, k, v, g, eta, eps < 0.f ? 0.f : eps, h0, o, hT, B, T, H,
+                               dk, dv, dtype, dk);
+  if (s != KLA_OK) return s;
+  if (chunk != KLA_CHUNK) return KLA_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (T == 0) return empty_prefill(h0, hT, B, H, dk, dv, st);
+  if (dtype == KLA_FP32) {
+    cudaError_t e = launch_recurrent(q, k, v, g, true, eta, eps, h0, o, hT, B, T, H, dk, dv,
+                                     dtype, st);
+    return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+  }
+  // the per-chunk factors are required; the segment states after them only
+  // enable the cut state chain
+  const size_t full = kda_chunk_workspace_bytes(B, T, H, dk, dv, dtype);
+  const size_t tiles = (size_t)B * H * ((T + KLA_CHUNK - 1) / KLA_CHUNK) *
+                       kda_tile_offsets(dk).total;
+  if (!workspace || ws_bytes < tiles || !aligned16(workspace)) return KLA_ERR_INVALID_ARG;
+  if (workspace_overlaps(workspace, ws_bytes >= full ? full : tiles, q, k, v, g, eta, h0, o, hT,
+                         B, T, H, dk, dv, dtype))
+    return KLA_ERR_INVALID_ARG;
+  unsigned int* err = device_error_ptr();
+  if (!err) return KLA_ERR_CUDA;
+  cudaError_t e = launch_kda_chunk(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, workspace,
+                                   ws_bytes, err, st);
+  if (e == cudaErrorNotSupported) return KLA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
 // Prefill with the per-channel gate (token-serial kernel), KLA step size or
 // (eps == kBetaGiven) beta given.
 static kla_status kda_fwd_impl(const void* q, const void* k, const void* v, const float* g,
@@ -271,6 +306,27 @@ kla_status kla_kda_fwd(const void* q, const void* k, const void* v, const float*
                        int B, int T, int H, int dk, int dv, int dtype, void* stream) {
   if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
   return kda_fwd_impl(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype, stream);
+}
+
+size_t kla_kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int dtype) {
+  return kda_chunk_workspace_bytes(B, T, H, dk, dv, dtype);
+}
+
+kla_status kla_kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                             const float* eta, float eps, const float* h0, void* o, float* hT,
+                             int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  return kda_chunk_impl(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, chunk, dtype,
+                        workspace, ws_bytes, stream);
+}
+
+kla_status kla_kda_chunk_fwd_beta(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const float* h0, void* o, float* hT, int B,
+                                  int T, int H, int dk, int dv, int chunk, int dtype,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  return kda_chunk_impl(q, k, v, g, beta, kBetaGiven, h0, o, hT, B, T, H, dk, dv, chunk, dtype,
+                        workspace, ws_bytes, stream);
 }
 
 kla_status kla_kda_fwd_beta(const void* q, const void* k, const void* v, const float* g,

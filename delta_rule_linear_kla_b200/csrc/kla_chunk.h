@@ -45,6 +45,34 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, cons
                                int dk, int dv, void* workspace, size_t ws_bytes,
                                unsigned int* err, cudaStream_t st);
 
+// Per-chunk factors of the per-channel-gate (KDA form) path, one tile per
+// chunk in chunk-major order: byte offsets of T'^T, P, W, Q o e^G,
+// K o e^{G_last - G} (64 x dk bf16 each in 64-column swizzled panels; the
+// first two 64 x 64) and e^{G_last} (dk fp32), and the tile's total size.
+struct KdaTileOffsets {
+  uint32_t tp, p, w, q, k, d, total;
+};
+__host__ __device__ constexpr KdaTileOffsets kda_tile_offsets(int dk) {
+  return KdaTileOffsets{0u,
+                        8192u,
+                        16384u,
+                        16384u + (uint32_t)(dk / 64) * 8192u,
+                        16384u + 2u * (uint32_t)(dk / 64) * 8192u,
+                        16384u + 3u * (uint32_t)(dk / 64) * 8192u,
+                        16384u + 3u * (uint32_t)(dk / 64) * 8192u + 1024u};
+}
+
+// The per-channel-gate chunk prefill: per-chunk factors (CUDA cores, fp32,
+// every chunk of every head in parallel), then the chain kernel in its KDA
+// mode.  g is [B][T][H][dk]; eps < 0 selects beta given (in eta).
+cudaError_t launch_kda_prep(const void* q, const void* k, const float* g, const float* eta,
+                            float eps, int B, int T, int H, int dk, void* ws, cudaStream_t st);
+cudaError_t launch_kda_chunk(const void* q, const void* k, const void* v, const float* g,
+                             const float* eta, float eps, const float* h0, void* o, float* hT,
+                             int B, int T, int H, int dk, int dv, void* workspace,
+                             size_t ws_bytes, unsigned int* err, cudaStream_t st);
+size_t kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
+
 // UT kernel alone: T', T'' of every chunk into `ws` (chunk-major order
 // ((b * H + h) * nchunks + n)).  `tm_k` maps k as [B][T][H][dk] bf16 with
 // 64 x 64 boxes and 128-byte swizzle.

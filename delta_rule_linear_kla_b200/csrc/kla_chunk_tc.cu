@@ -96,6 +96,7 @@ struct alignas(1024) ChainSmem {
   uint8_t vpd[8192];     // V' scaled by e^{G_63 - G_s} (MMA 5 operand)
   float G[3][C];         // gate cumsum of chunk n in slot n % 3
   alignas(16) float alpha[3][C];  // e^{g_s} of chunk n in slot n % 3
+  float kdec[3][128];    // per-channel gate: e^{G_last} of chunk n in slot n % 3
   uint64_t full[2], empty[2];
   uint64_t bS, bW, bX, bH, bHP;          // MMA completions
   uint64_t p_done, w_done, vpd_ready, vp_ready;
@@ -135,7 +136,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // units; a K step is 32 B (K-major) or 2048 B (MN-major).
 constexpr uint64_t KSTEP_K = 2, KSTEP_MN = 128;
 
-template <int DK>
+// KDA: the per-channel-gate form.  The stage then holds W, P, Q o e^G and
+// K o e^{G_last - G} as made per chunk by kda_prep_kernel (bulk copies; no
+// Q K^T or W products, no W or P epilogues), the state decays row by row with
+// e^{G_last}, and the outputs take no e^{G} factor (it is in Q o e^G).
+template <int DK, bool KDA>
 __global__ void __launch_bounds__(NTHREADS, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
@@ -214,8 +219,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       ptx::prefetch_tensormap(&tm_q);
       ptx::prefetch_tensormap(&tm_k);
       ptx::prefetch_tensormap(&tm_v);
-      const uint32_t BYTES = (uint32_t)(2 * NP * 8192 + (phi_slab ? 0 : 8192) + kUtTileBytes);
-      const uint8_t* ws_head = ws + (head * (size_t)nchunks_all + n0) * kUtTileBytes;
+      constexpr KdaTileOffsets KO = kda_tile_offsets(DK);
+      constexpr uint32_t TILE = KDA ? KO.total : (uint32_t)kUtTileBytes;
+      const uint32_t BYTES =
+          KDA ? (uint32_t)(2 * 8192 + 3 * NP * 8192 + DK * 4 + (phi_slab ? 0 : 8192))
+              : (uint32_t)(2 * NP * 8192 + (phi_slab ? 0 : 8192) + kUtTileBytes);
+      const uint8_t* ws_head = ws + (head * (size_t)nchunks_all + n0) * TILE;
       int issued = 0, drained = 0;
       for (int n = 0; n < nchunks; ++n) {
         const int st = n & 1;
@@ -224,25 +233,39 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           drained = n - 1;  // chunks up to n-2 fully consumed
         }
         Stage<DK>& S = s.st[st];
-        const uint8_t* src = ws_head + (size_t)n * kUtTileBytes;
+        const uint8_t* src = ws_head + (size_t)n * TILE;
         ptx::mbar_arrive_expect_tx(&s.full[st], BYTES);
-        ptx::bulk_load(S.tp[TP1], src, 8192, &s.full[st]);
-        ptx::bulk_load(S.tp[TP2], src + 8192, 8192, &s.full[st]);
+        if constexpr (KDA) {
+          ptx::bulk_load(S.tp[TP1], src + KO.tp, 8192, &s.full[st]);
+          ptx::bulk_load(S.tp[TP], src + KO.p, 8192, &s.full[st]);
+          ptx::bulk_load(S.tp[TP2], src + KO.d, DK * 4, &s.full[st]);  // e^{G_last}
 #pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          ptx::tma_load_4d(S.panel[p][SK], &tm_k, &s.full[st], p * 64, hh, (n0 + n) * C, b);
-          ptx::tma_load_4d(S.panel[p][SQ], &tm_q, &s.full[st], p * 64, hh, (n0 + n) * C, b);
+          for (int p = 0; p < NP; ++p) {
+            ptx::bulk_load(S.panel[p][SW], src + KO.w + p * 8192, 8192, &s.full[st]);
+            ptx::bulk_load(S.panel[p][SQ], src + KO.q + p * 8192, 8192, &s.full[st]);
+            ptx::bulk_load(S.panel[p][SK], src + KO.k + p * 8192, 8192, &s.full[st]);
+          }
+        } else {
+          ptx::bulk_load(S.tp[TP1], src, 8192, &s.full[st]);
+          ptx::bulk_load(S.tp[TP2], src + 8192, 8192, &s.full[st]);
+#pragma unroll
+          for (int p = 0; p < NP; ++p) {
+            ptx::tma_load_4d(S.panel[p][SK], &tm_k, &s.full[st], p * 64, hh, (n0 + n) * C, b);
+            ptx::tma_load_4d(S.panel[p][SQ], &tm_q, &s.full[st], p * 64, hh, (n0 + n) * C, b);
+          }
         }
         if (!phi_slab)
           ptx::tma_load_4d(S.v, &tm_v, &s.full[st], slab * BV, hh, (n0 + n) * C, b);
         issued = n + 1;
         if (n + 2 < nchunks) {  // warm L2 two chunks ahead of the loads
           const int m = n + 2;
-          ptx::bulk_prefetch_l2(ws_head + (size_t)m * kUtTileBytes, (uint32_t)kUtTileBytes);
+          ptx::bulk_prefetch_l2(ws_head + (size_t)m * TILE, TILE);
+          if constexpr (!KDA) {
 #pragma unroll
-          for (int p = 0; p < NP; ++p) {
-            ptx::tma_prefetch_l2_4d(&tm_k, p * 64, hh, (n0 + m) * C, b);
-            ptx::tma_prefetch_l2_4d(&tm_q, p * 64, hh, (n0 + m) * C, b);
+            for (int p = 0; p < NP; ++p) {
+              ptx::tma_prefetch_l2_4d(&tm_k, p * 64, hh, (n0 + m) * C, b);
+              ptx::tma_prefetch_l2_4d(&tm_q, p * 64, hh, (n0 + m) * C, b);
+            }
           }
           if (!phi_slab) ptx::tma_prefetch_l2_4d(&tm_v, slab * BV, hh, (n0 + m) * C, b);
         }
@@ -310,12 +333,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     if (ok) ok = wait_or_abort(&s.full[0], 0, abort_flag);
     if (ok) {
       ptx::tc_fence_after();
-      mma2(0);
-      mma3(0);
-      ok = wait_or_abort(&s.w_done, 0, abort_flag);
-      if (ok) {
-        ptx::tc_fence_after();
-        mma1(0);
+      if constexpr (KDA) {
+        mma3(0);
+      } else {
+        mma2(0);
+        mma3(0);
+        ok = wait_or_abort(&s.w_done, 0, abort_flag);
+        if (ok) {
+          ptx::tc_fence_after();
+          mma1(0);
+        }
       }
     }
     for (int n = 0; n < nchunks && ok; ++n) {
@@ -324,7 +351,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const uint32_t par = (uint32_t)(n & 1);
       const bool more = n + 1 < nchunks;
       // ---- MMA 4 (chunk n): needs W(n) and h_n (D_H of n-1 read)
-      if (!wait_or_abort(&s.w_done, par, abort_flag)) break;
+      if (!KDA && !wait_or_abort(&s.w_done, par, abort_flag)) break;
       if (!wait_or_abort(&s.h_done, par, abort_flag)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
@@ -341,7 +368,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (!wait_or_abort(&s.full[(n + 1) & 1], (uint32_t)(((n + 1) >> 1) & 1), abort_flag))
           break;
         ptx::tc_fence_after();
-        mma2(n + 1);
+        if constexpr (!KDA) mma2(n + 1);
       }
       // ---- MMA 5 (state), committed on its own so the update starts at once
       if (!wait_or_abort(&s.vpd_ready, par, abort_flag)) break;
@@ -349,14 +376,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       if (ptx::elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          ptx::mma_bf16(tb + COL_H, dKmn + so + kk * KSTEP_MN, dVPD + kk * KSTEP_MN, id_mn, kk > 0);
+          ptx::mma_bf16(tb + COL_H, dKmn + so + kk * KSTEP_MN, (KDA ? dVP : dVPD) + kk * KSTEP_MN,
+                        id_mn, kk > 0);
         ptx::mma_commit(&s.bH);
       }
       __syncwarp();
       // ---- MMA 6 (chunk n): needs V'(n), P(n) and D_PV free (outputs of n-1
       //      read)
       if (!wait_or_abort(&s.vp_ready, par, abort_flag)) break;
-      if (!wait_or_abort(&s.p_done, par, abort_flag)) break;
+      if (!KDA && !wait_or_abort(&s.p_done, par, abort_flag)) break;
       if (n > 0 && !wait_or_abort(&s.pv_free, par ^ 1u, abort_flag)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
@@ -375,11 +403,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           break;
         ptx::tc_fence_after();
         mma3(n + 1);
-        // ... and Q K^T of chunk n+1: D_S was read by P(n) (waited above);
-        // waiting for W(n+1) keeps its rows from changing under the read
-        if (!wait_or_abort(&s.w_done, par ^ 1u, abort_flag)) break;
-        ptx::tc_fence_after();
-        mma1(n + 1);
+        if constexpr (!KDA) {
+          // ... and Q K^T of chunk n+1: D_S was read by P(n) (waited above);
+          // waiting for W(n+1) keeps its rows from changing under the read
+          if (!wait_or_abort(&s.w_done, par ^ 1u, abort_flag)) break;
+          ptx::tc_fence_after();
+          mma1(n + 1);
+        }
       }
     }
     // every MMA this warp issued has finished before TMEM is released
@@ -389,7 +419,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   } else if (warp == 4 || warp == 5) {
     // ===================== next-chunk epilogue: W =========================
     // W rows 0..63 (TMEM lanes 0..63) -> the stage's W slot (bf16)
-    for (int n = 0; n < nchunks; ++n) {
+    for (int n = 0; n < (KDA ? 0 : nchunks); ++n) {
       Stage<DK>& S = s.st[n & 1];
       if (!wait_or_abort(&s.bW, (uint32_t)(n & 1), abort_flag)) break;
       ptx::tc_fence_after();
@@ -415,13 +445,24 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // g_ready), loading the next chunk's gates one chunk ahead.
     const int hc = (warp >= 14) ? 0 : 1;
     const int r = row - 64;
+    if constexpr (KDA) {
+      // the chunk decay e^{G_last} (one per key channel) arrives with the
+      // stage; warp 2 publishes it through the g_ready ring
+      for (int n = 0; n < (warp == 2 ? nchunks : 0); ++n) {
+        if (!wait_or_abort(&s.full[n & 1], (uint32_t)((n >> 1) & 1), abort_flag)) break;
+        const float* dsrc = reinterpret_cast<const float*>(s.st[n & 1].tp[TP2]);
+        for (int i = lane; i < DK; i += 32) s.kdec[n % 3][i] = dsrc[i];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.g_ready[n % 3]);
+      }
+    }
     float gn0 = 0.f, gn1 = 0.f;
-    if (warp == 2 && nchunks > 0) {
+    if (!KDA && warp == 2 && nchunks > 0) {
       const int t0 = n0 * C + lane, t1 = t0 + 32;
       gn0 = (t0 < T) ? g[((size_t)b * T + t0) * H + hh] : 0.f;
       gn1 = (t1 < T) ? g[((size_t)b * T + t1) * H + hh] : 0.f;
     }
-    for (int n = 0; n < nchunks; ++n) {
+    for (int n = 0; n < (KDA ? 0 : nchunks); ++n) {
       Stage<DK>& S = s.st[n & 1];
       float* Gn = s.G[n % 3];
       if (warp == 2) {
@@ -511,8 +552,23 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const uint32_t par = (uint32_t)(n & 1);
       const uint32_t col_u = COL_U + 64 * (n & 1);
       if (!wait_or_abort(&s.g_ready[n % 3], (uint32_t)((n / 3) & 1), abort_flag)) { ok = false; break; }
-      const float gC = Gn[C - 1];
-      if (v_rows) {
+      const float gC = KDA ? 0.f : Gn[C - 1];
+      if (v_rows && KDA) {
+        // V' = U - W h (combined in TMEM); the keys of MMA 5 carry the decay
+        if (!wait_or_abort(&s.bX, par, abort_flag)) { ok = false; break; }
+        ptx::tc_fence_after();
+        float u[32];
+        ptx::tmem_ld32(tb + lane_base + col_u + cg, u);
+        ptx::tc_fence_before();
+        sw128_store_row32(s.vp, row, grp, u);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&s.vpd_ready);
+          mbar_arrive(&s.u_free[n & 1]);
+          mbar_arrive(&s.vp_ready);
+        }
+      } else if (v_rows) {
         // V'_r = U_r - (W h)_r (already combined in TMEM) and its copy
         // decayed to the chunk end for MMA 5
         const float dec = __expf(gC - Gn[row]);
@@ -537,11 +593,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (lane == 0) mbar_arrive(&s.vp_ready);
       }
       // every read of G(n) happens before this warp's last arrival of chunk n
-      const float e_out = v_rows ? 0.f : -__expf(Gn[row - 64]);
+      const float e_out = v_rows ? 0.f : (KDA ? -1.f : -__expf(Gn[row - 64]));
       if (!wait_or_abort(&s.bH, par, abort_flag)) { ok = false; break; }
       ptx::tc_fence_after();
       if (has_h) {
-        const float a = __expf(gC);
+        const float a = KDA ? s.kdec[n % 3][row] : __expf(gC);
         float dh[32];
         ptx::tmem_ld32(tb + lane_base + COL_H + cg, dh);
 #pragma unroll
@@ -683,7 +739,7 @@ segment_start_kernel(const float* __restrict__ h0, const float* __restrict__ E,
   }
 }
 
-template <int DK>
+template <int DK, bool KDA>
 cudaError_t launch_chain_dk(const void* q, const void* k, const void* v, const float* g,
                             const float* h0, void* o, float* hT, float* phi, int B, int T,
                             int H, int DV, int nseg, int seg_chunks, int mode,
@@ -698,14 +754,15 @@ cudaError_t launch_chain_dk(const void* q, const void* k, const void* v, const f
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(chain_kernel<DK>,
+    cudaError_t e = cudaFuncSetAttribute(chain_kernel<DK, KDA>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   dim3 grid((mode == 1 ? DV + DK : DV) / BV, H, B * nseg);
-  chain_kernel<DK><<<grid, NTHREADS, smem, st>>>(mq, mk, mv, g, h0, (__nv_bfloat16*)o, hT, phi,
-                                                 T, H, DV, nseg, seg_chunks, mode, ws, err);
+  chain_kernel<DK, KDA><<<grid, NTHREADS, smem, st>>>(mq, mk, mv, g, h0, (__nv_bfloat16*)o, hT,
+                                                      phi, T, H, DV, nseg, seg_chunks, mode, ws,
+                                                      err);
   return cudaGetLastError();
 }
 
@@ -783,11 +840,13 @@ cudaError_t launch_chunk_ut(const void* k, const float* g, const float* eta, flo
 }
 
 // The chain in S segments: pass 1 (E, Phi of segments 0 .. S-2), the start
-// states, pass 2 (outputs of every segment from its start state).
-template <int DK>
+// states, pass 2 (outputs of every segment from its start state).  The
+// segment buffers follow the `tiles` bytes of per-chunk factors.
+template <int DK, bool KDA>
 static cudaError_t launch_segmented(const void* q, const void* k, const void* v, const float* g,
                                     const float* h0, void* o, float* hT, int B, int T, int H,
-                                    int sg, uint8_t* ws, unsigned int* err, cudaStream_t st);
+                                    int sg, uint8_t* ws, size_t tiles, unsigned int* err,
+                                    cudaStream_t st);
 
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, const float* g,
                                const float* h0, void* o, float* hT, int B, int T, int H,
@@ -797,41 +856,45 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, cons
   const int sg = chunk_chain_segments(B, T, H, dk, dv, ws_bytes);
   if (sg > 1) {
     uint8_t* wsm = (uint8_t*)workspace;
-    if (dk == 128) return launch_segmented<128>(q, k, v, g, h0, o, hT, B, T, H, sg, wsm, err, st);
-    return launch_segmented<64>(q, k, v, g, h0, o, hT, B, T, H, sg, wsm, err, st);
+    const size_t tiles = ut_workspace_bytes(B, T, H);
+    if (dk == 128)
+      return launch_segmented<128, false>(q, k, v, g, h0, o, hT, B, T, H, sg, wsm, tiles, err,
+                                          st);
+    return launch_segmented<64, false>(q, k, v, g, h0, o, hT, B, T, H, sg, wsm, tiles, err, st);
   }
   const uint8_t* ws = (const uint8_t*)workspace;
   const int nchunks = (T + C - 1) / C;
   if (dk == 128)
-    return launch_chain_dk<128>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks, 0, ws,
-                                err, st);
+    return launch_chain_dk<128, false>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks,
+                                       0, ws, err, st);
   if (dk == 64)
-    return launch_chain_dk<64>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks, 0, ws,
-                               err, st);
+    return launch_chain_dk<64, false>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks,
+                                      0, ws, err, st);
   return cudaErrorNotSupported;
 }
 
-template <int DK>
+template <int DK, bool KDA>
 static cudaError_t launch_segmented(const void* q, const void* k, const void* v, const float* g,
                                     const float* h0, void* o, float* hT, int B, int T, int H,
-                                    int sg, uint8_t* ws, unsigned int* err, cudaStream_t st) {
+                                    int sg, uint8_t* ws, size_t tiles, unsigned int* err,
+                                    cudaStream_t st) {
   constexpr int DV = DK;
   const int nchunks = (T + C - 1) / C;
   const int len = (nchunks + sg - 1) / sg;
   const size_t n = (size_t)B * sg * H;
-  float* E = reinterpret_cast<float*>(ws + ut_workspace_bytes(B, T, H));
+  float* E = reinterpret_cast<float*>(ws + tiles);
   float* hstart = E + n * DK * DV;
   float* Phi = hstart + n * DK * DV;
   // pass 1 covers segments 0 .. S-2 (launched as S - 1 segments of `len`
   // chunks, so E and Phi are laid out [B][S - 1][H])
-  cudaError_t e = launch_chain_dk<DK>(q, k, v, g, nullptr, nullptr, E, Phi, B, T, H, DV,
-                                      sg - 1, len, 1, ws, err, st);
+  cudaError_t e = launch_chain_dk<DK, KDA>(q, k, v, g, nullptr, nullptr, E, Phi, B, T, H, DV,
+                                           sg - 1, len, 1, ws, err, st);
   if (e != cudaSuccess) return e;
   segment_start_kernel<DK><<<dim3(DV / BV, H, B), 2 * DK, 0, st>>>(h0, E, Phi, hstart, H, DV, sg);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_chain_dk<DK>(q, k, v, g, hstart, o, hT, nullptr, B, T, H, DV, sg, len, 0, ws,
-                             err, st);
+  return launch_chain_dk<DK, KDA>(q, k, v, g, hstart, o, hT, nullptr, B, T, H, DV, sg, len, 0,
+                                  ws, err, st);
 }
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
@@ -843,6 +906,42 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
   if (e != cudaSuccess) return e;
   return launch_chunk_chain(q, k, v, g, h0, o, hT, B, T, H, dk, dv, workspace, ws_bytes, err,
                             st);
+}
+
+// ---------------------------------------------------- per-channel gate
+namespace {
+size_t kda_tiles_bytes(int B, int T, int H, int dk) {
+  return (size_t)B * H * ((T + C - 1) / C) * kda_tile_offsets(dk).total;
+}
+}  // namespace
+
+size_t kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
+  if (dtype != KLA_BF16 || B < 1 || H < 1 || T < 1 || dk != dv || (dk != 64 && dk != 128))
+    return 0;
+  return kda_tiles_bytes(B, T, H, dk) + segment_bytes(B, T, H, dk, dv);
+}
+
+cudaError_t launch_kda_chunk(const void* q, const void* k, const void* v, const float* g,
+                             const float* eta, float eps, const float* h0, void* o, float* hT,
+                             int B, int T, int H, int dk, int dv, void* workspace,
+                             size_t ws_bytes, unsigned int* err, cudaStream_t st) {
+  if (dk != dv || (dk != 64 && dk != 128)) return cudaErrorNotSupported;
+  cudaError_t e = launch_kda_prep(q, k, g, eta, eps, B, T, H, dk, workspace, st);
+  if (e != cudaSuccess) return e;
+  const size_t tiles = kda_tiles_bytes(B, T, H, dk);
+  const int sg = chain_segments(B, T, H, dk, dv);
+  uint8_t* ws = (uint8_t*)workspace;
+  if (sg > 1 && ws_bytes >= tiles + segment_bytes(B, T, H, dk, dv)) {
+    if (dk == 128)
+      return launch_segmented<128, true>(q, k, v, g, h0, o, hT, B, T, H, sg, ws, tiles, err, st);
+    return launch_segmented<64, true>(q, k, v, g, h0, o, hT, B, T, H, sg, ws, tiles, err, st);
+  }
+  const int nchunks = (T + C - 1) / C;
+  if (dk == 128)
+    return launch_chain_dk<128, true>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks, 0,
+                                      ws, err, st);
+  return launch_chain_dk<64, true>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks, 0,
+                                   ws, err, st);
 }
 
 }  // namespace kla

@@ -115,3 +115,86 @@ def test_kda_decode_beta_given():
         assert rel(o.cpu(), o_ref[:, 0]) < TOL["bf16"]
     torch.cuda.synchronize()
     assert rel(S.cpu(), Sref) < TOL["fp32"]
+
+
+# ------------------------------------------------- chunk path (tensor cores)
+@pytest.mark.parametrize("name,B,T,H,h0", [("prefill_4k", 2, 130, 2, True),
+                                           ("prefill_4k", 1, 1, 2, False),
+                                           ("prefill_4k", 1, 64, 3, True),
+                                           ("stress", 2, 97, 3, True),
+                                           ("stress", 1, 300, 2, False)])
+def test_kda_chunk_prefill(name, B, T, H, h0):
+    w, x = _prefill_inputs(name, B, T, H, "bf16", 91, with_h0=h0)
+    xc = cuda(x)
+    o, hT = api.kda_chunk_fwd(xc["q"], xc["k"], xc["v"], xc["gv"], xc["eta"], x["eps"],
+                              xc["h0"])
+    api.check_device_error()
+    o_ref, h_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["gv"], x["eta"], x["eps"],
+                                      x["h0"])
+    assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
+    assert rel(o.cpu(), o_ref) < TOL["bf16"] and rel(hT.cpu(), h_ref) < TOL["bf16"]
+
+
+def test_kda_chunk_strong_and_zero_gates():
+    """Channels that wipe the state (g down to -60 per token), channels that
+    never decay (g = 0) and mixtures inside one chunk: every decay factor the
+    chunk path forms is e^{difference} <= 1, so nothing overflows."""
+    w, x = _prefill_inputs("prefill_4k", 1, 200, 2, "bf16", 93, with_h0=True)
+    gv = x["gv"]
+    gv[..., :16] = 0.0
+    gv[0, 30:40, :, 16:48] = -60.0
+    gv[0, :, :, 100:] = -8.0
+    xc = cuda(x)
+    o, hT = api.kda_chunk_fwd(xc["q"], xc["k"], xc["v"], xc["gv"], xc["eta"], x["eps"],
+                              xc["h0"])
+    api.check_device_error()
+    o_ref, h_ref = oracle.kda_forward(x["q"], x["k"], x["v"], gv, x["eta"], x["eps"], x["h0"])
+    assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
+    assert rel(o.cpu(), o_ref) < TOL["bf16"] and rel(hT.cpu(), h_ref) < TOL["bf16"]
+
+
+def test_kda_chunk_beta_given_and_fp32():
+    w, x = _prefill_inputs("prefill_4k", 2, 150, 2, "bf16", 95, with_h0=True)
+    rng = np.random.Generator(np.random.PCG64(96))
+    beta = torch.from_numpy(rng.uniform(0.0, 1.0, (2, 150, 2)).astype(np.float32))
+    kf = x["k"].float()
+    k = (kf / kf.norm(dim=-1, keepdim=True).clamp_min(1e-6)).to(torch.bfloat16)
+    xc = cuda(x)
+    o, hT = api.kda_chunk_fwd_beta(xc["q"], cuda(k), xc["v"], xc["gv"], cuda(beta), xc["h0"])
+    api.check_device_error()
+    o_ref, h_ref = oracle.kda(x["q"], k, x["v"], x["gv"], beta, x["h0"])
+    assert rel(o.cpu(), o_ref) < TOL["bf16"] and rel(hT.cpu(), h_ref) < TOL["bf16"]
+    # fp32 I/O goes to the token-serial kernel through the same entry point
+    w2, x2 = _prefill_inputs("tiny", 1, 90, 2, "fp32", 97, with_h0=True)
+    x2c = cuda(x2)
+    o2, h2 = api.kda_chunk_fwd(x2c["q"], x2c["k"], x2c["v"], x2c["gv"], x2c["eta"], x2["eps"],
+                               x2c["h0"])
+    torch.cuda.synchronize()
+    o2_ref, h2_ref = oracle.kda_forward(x2["q"], x2["k"], x2["v"], x2["gv"], x2["eta"],
+                                        x2["eps"], x2["h0"])
+    assert rel(o2.cpu(), o2_ref) < TOL["fp32"] and rel(h2.cpu(), h2_ref) < TOL["fp32"]
+
+
+def test_kda_chunk_segmented_chain():
+    """Few heads, long sequence: the cut state chain in the per-channel form."""
+    w, x = _prefill_inputs("prefill_4k", 1, 4000, 2, "bf16", 99, with_h0=True)
+    assert api.chunk_fwd_segments(1, 4000, 2, w.dk, w.dv) > 1
+    xc = cuda(x)
+    o, hT = api.kda_chunk_fwd(xc["q"], xc["k"], xc["v"], xc["gv"], xc["eta"], x["eps"],
+                              xc["h0"])
+    api.check_device_error()
+    o_ref, h_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["gv"], x["eta"], x["eps"],
+                                      x["h0"])
+    assert rel(o.cpu(), o_ref) < TOL["bf16"] and rel(hT.cpu(), h_ref) < TOL["bf16"]
+
+
+def test_kda_chunk_matches_token_serial_4k_sampled():
+    """The full 4K shape in the benchmark's launch configuration: the chunk
+    path against the token-serial kernel on every head (same recurrence)."""
+    w = inputs.WORKLOADS["prefill_4k"]
+    x = cuda(inputs.make_prefill(w))
+    gv = cuda(inputs.channel_gates((w.B, w.T, w.H, w.dk), w.seed + 11))
+    o1, h1 = api.kda_chunk_fwd(x["q"], x["k"], x["v"], gv, x["eta"], x["eps"])
+    o2, h2 = api.kda_fwd(x["q"], x["k"], x["v"], gv, x["eta"], x["eps"])
+    api.check_device_error()
+    assert rel(o1, o2) < TOL["bf16"] and rel(h1, h2) < TOL["bf16"]
