@@ -26,6 +26,12 @@
 // stage wants (128-byte swizzled bf16 rows, fetched with bulk copies):
 //   [T'^T][P][W panels][Q o e^G panels][K o e^{G_last - G} panels][e^{G_last}]
 // (see kda_tile_offsets in kla_chunk.h).
+//
+// A and P inside each 16-token sub-block are summed with one exponential per
+// (pair, channel) in fp32; between sub-blocks the decay factors through the
+// sub-block's first row (both factors <= 1) and those entries, like W, are
+// bf16 warp-level tensor-core products with fp32 sums -- the same operand
+// rounding the scalar-gate path applies to its Gram matrix and W.
 #include "kla_chunk.h"
 #include "kla_common.cuh"
 #include "tile_sw128.cuh"
@@ -34,36 +40,82 @@ namespace kla {
 namespace {
 
 constexpr int C = 64;
-constexpr int NT = 512;
+constexpr int NT = 256;
 constexpr int SB = 16;  // sub-block of rows sharing one decay reference
 
-// fp32 rows are padded to an odd number of words so that threads reading
-// different rows at the same channel hit different banks.
+// Shared memory, two CTAs per SM.  fp32 rows are padded to an odd number of
+// words and bf16 operand rows by 8 elements, so that the threads of a warp
+// reading different rows at one channel (or the fragment loads of a
+// tensor-core product) hit distinct banks.  The union follows the
+// lifetimes: q, the sub-block operands and A live until T is formed; T and
+// the operands of W after that (T's rows overlap only q and the sub-block
+// operands, never A, which other warps may still be reading while T is
+// written).
 template <int DK>
 struct KdaPrepSmem {
-  float k[C][DK + 1];          // keys, token-major
-  float g[C][DK + 1];          // G (in-chunk cumsum of the gate), token-major
-  __nv_bfloat16 q[C][DK + 2];  // queries, token-major
+  __nv_bfloat16 k[C][DK + 2];  // keys, token-major (the bf16 inputs, exact)
+  float g[C][DK + 1];          // G, the in-chunk cumsum of the gate, token-major
   union {
     struct {
-      float xk[SB][DK + 1];   // k_ri e^{G_ri - G_ref,i}, rows of one sub-block
-      float xq[SB][DK + 1];   // q_ri e^{G_ri - G_ref,i}
-      float y[DK][3 * SB + 1];  // k_si e^{G_ref,i - G_si}, s before the sub-block
-    } ap;
-    float khat[C][DK + 1];  // k_si e^{G_si} (W)
+      __nv_bfloat16 q[C][DK + 2];       // queries, token-major
+      __nv_bfloat16 x[2 * SB][DK + 8];  // rows of one sub-block: k_ri e^{G_ri - G_ref,i},
+                                        // then q_ri e^{G_ri - G_ref,i}
+      __nv_bfloat16 y[3 * SB][DK + 8];  // k_si e^{G_ref,i - G_si}, s before the sub-block
+      float a[C][C + 1];                // A, row r column s
+    } p1;
+    struct {
+      float t[C][C + 1];            // T = (I + A)^{-1}, then T' = T diag(beta)
+      __nv_bfloat16 tb[C][C + 8];   // T', bf16
+      __nv_bfloat16 kc[DK][C + 8];  // k_si e^{G_si}, channel-major
+    } p2;
   } u;
-  float a[C][C + 1];  // A, row r column s
-  float t[C][C + 1];  // T = (I + A)^{-1}, then T' = T diag(beta)
   float beta[C];
 };
+
+// One warp-level tensor-core product D (16 x 8, fp32) += A (16 x 16) B (16 x 8),
+// bf16 operands.  A is taken from a row-major tile (rows m0 .. m0 + 15,
+// columns k0 .. k0 + 15), B from a tile holding B^T row-major (rows = the 8
+// columns n0 .. n0 + 7 of B, columns k0 .. k0 + 15); `lda`, `ldb` elements
+// per row.  Fragment ownership (PTX ISA, mma.m16n8k16): lane
+// (g = lane / 4, t = lane % 4) holds A rows g and g + 8 at columns 2t, 2t + 1
+// and 2t + 8, 2t + 9, B column n = g at rows 2t, 2t + 1 and 2t + 8, 2t + 9,
+// and D rows g, g + 8 at columns 2t, 2t + 1.  The sub-block products here are
+// 16 to 64 wide: too small for the CTA-level tcgen05 products and their
+// tensor-memory round trip, a natural fit for warp-level products.
+__device__ __forceinline__ void mma_16x8x16(float* d, const __nv_bfloat16* a, int lda, int m0,
+                                            const __nv_bfloat16* bt, int ldb, int n0, int k0,
+                                            int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  auto w32 = [](const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); };
+  const uint32_t a0 = w32(a + (m0 + g) * lda + k0 + 2 * t);
+  const uint32_t a1 = w32(a + (m0 + g + 8) * lda + k0 + 2 * t);
+  const uint32_t a2 = w32(a + (m0 + g) * lda + k0 + 2 * t + 8);
+  const uint32_t a3 = w32(a + (m0 + g + 8) * lda + k0 + 2 * t + 8);
+  const uint32_t b0 = w32(bt + (n0 + g) * ldb + k0 + 2 * t);
+  const uint32_t b1 = w32(bt + (n0 + g) * ldb + k0 + 2 * t + 8);
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
 __device__ __forceinline__ void store_bf16_at(uint8_t* tile, int row, int col, float x) {
   reinterpret_cast<__nv_bfloat16*>(tile)[(sw128_chunk_off(row, col >> 3) >> 1) + (col & 7)] =
       __float2bfloat16_rn(x);
 }
 
+__device__ __forceinline__ uint4 pack8(const float* x) {
+  uint4 u;
+  u.x = pack_bf16x2(x[0], x[1]);
+  u.y = pack_bf16x2(x[2], x[3]);
+  u.z = pack_bf16x2(x[4], x[5]);
+  u.w = pack_bf16x2(x[6], x[7]);
+  return u;
+}
+
 template <int DK>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT, 2)
 kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                 const float* __restrict__ g, const float* __restrict__ eta, float eps,
                 uint8_t* __restrict__ ws, int T, int H, int nchunks) {
@@ -85,22 +137,17 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     const int tok = p / (DK / 4), i0 = (p % (DK / 4)) * 4, t = t0 + tok;
     const size_t base = (((size_t)b * T + t) * H + hh) * DK + i0;
     float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
-    float kx[4] = {0.f, 0.f, 0.f, 0.f};
-    uint2 qv = make_uint2(0, 0);
+    uint2 kv = make_uint2(0, 0), qv = make_uint2(0, 0);
     if (t < T) {
       gv = *reinterpret_cast<const float4*>(g + base);
-      const uint2 kv = *reinterpret_cast<const uint2*>(k + base);
-      const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(&kv);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) kx[j] = __bfloat162float(kb[j]);
+      kv = *reinterpret_cast<const uint2*>(k + base);
       qv = *reinterpret_cast<const uint2*>(q + base);
     }
     s.g[tok][i0] = gv.x; s.g[tok][i0 + 1] = gv.y; s.g[tok][i0 + 2] = gv.z; s.g[tok][i0 + 3] = gv.w;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) s.k[tok][i0 + j] = kx[j];
-    const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(&qv);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) s.q[tok][i0 + j] = qb[j];
+    *reinterpret_cast<uint32_t*>(&s.k[tok][i0]) = kv.x;
+    *reinterpret_cast<uint32_t*>(&s.k[tok][i0 + 2]) = kv.y;
+    *reinterpret_cast<uint32_t*>(&s.u.p1.q[tok][i0]) = qv.x;
+    *reinterpret_cast<uint32_t*>(&s.u.p1.q[tok][i0 + 2]) = qv.y;
   }
   __syncthreads();
 
@@ -111,14 +158,29 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
       acc += s.g[tok][tid];
       s.g[tok][tid] = acc;
     }
-  } else if (tid >= 256 && tid < 256 + C) {
-    const int tok = tid - 256, t = t0 + tok;
+  } else if (tid >= 128 && tid < 128 + C) {
+    const int tok = tid - 128, t = t0 + tok;
     float n2 = 0.f;
-    for (int i = 0; i < DK; ++i) n2 = fmaf(s.k[tok][i], s.k[tok][i], n2);
+    for (int i = 0; i < DK; ++i) {
+      const float x = __bfloat162float(s.k[tok][i]);
+      n2 = fmaf(x, x, n2);
+    }
     const size_t tk = ((size_t)b * T + t) * H + hh;
     s.beta[tok] = t < T ? step_size(eta[tk], n2, eps) : 0.f;
   }
   __syncthreads();
+
+  // ---- Q o e^{G} (token rows in 64-column panels), written while the
+  // queries are still in shared memory
+  for (int p = tid; p < C * (DK / 8); p += NT) {
+    const int tok = p / (DK / 8), i0 = (p % (DK / 8)) * 8;
+    float x[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+      x[jj] = __bfloat162float(s.u.p1.q[tok][i0 + jj]) * __expf(s.g[tok][i0 + jj]);
+    *reinterpret_cast<uint4*>(out + off.q + (i0 / 64) * 8192 +
+                              sw128_chunk_off(tok, (i0 % 64) / 8)) = pack8(x);
+  }
 
   // ---- diagonal sub-blocks of A (s < r) and P (s <= r), both tokens in one
   // sub-block: one thread per pair, one exponential per channel
@@ -134,136 +196,142 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     float aa = 0.f, pp = 0.f;
 #pragma unroll 4
     for (int i = 0; i < DK; ++i) {
-      const float x = s.k[sc][i] * __expf(s.g[r][i] - s.g[sc][i]);
-      aa = fmaf(s.k[r][i], x, aa);
-      pp = fmaf(__bfloat162float(s.q[r][i]), x, pp);
+      const float x = __bfloat162float(s.k[sc][i]) * __expf(s.g[r][i] - s.g[sc][i]);
+      aa = fmaf(__bfloat162float(s.k[r][i]), x, aa);
+      pp = fmaf(__bfloat162float(s.u.p1.q[r][i]), x, pp);
     }
-    s.a[r][sc] = sc < r ? s.beta[r] * aa : 0.f;
+    s.u.p1.a[r][sc] = sc < r ? s.beta[r] * aa : 0.f;
     store_bf16_at(outP, r, sc, pp);
   }
   // zeros of A and P above the diagonal (s > r)
   for (int p = tid; p < C * C; p += NT) {
     const int r = p / C, sc = p % C;
     if (sc > r) {
-      s.a[r][sc] = 0.f;
+      s.u.p1.a[r][sc] = 0.f;
       store_bf16_at(outP, r, sc, 0.f);
     }
   }
   // ---- off-diagonal sub-blocks: for row sub-block R and s < 16 R the decay
   // factors through the reference G_ref = G at the sub-block's first row:
-  // e^{G_ri - G_si} = e^{G_ri - G_ref,i} e^{G_ref,i - G_si}, both <= 1.
+  // e^{G_ri - G_si} = e^{G_ri - G_ref,i} e^{G_ref,i - G_si}, both <= 1, so
+  // these entries are dot products of pre-scaled rows (bf16, fp32 sums)
   for (int R = 1; R < C / SB; ++R) {
     const int r0 = R * SB, ns = r0;
-    __syncthreads();  // the previous sub-block's products have read xk, xq, y
+    __syncthreads();  // the previous sub-block's products have read x, y
     for (int p = tid; p < SB * DK; p += NT) {
       const int rl = p / DK, i = p % DK;
       const float e = __expf(s.g[r0 + rl][i] - s.g[r0][i]);
-      s.u.ap.xk[rl][i] = s.k[r0 + rl][i] * e;
-      s.u.ap.xq[rl][i] = __bfloat162float(s.q[r0 + rl][i]) * e;
+      s.u.p1.x[rl][i] = __float2bfloat16_rn(__bfloat162float(s.k[r0 + rl][i]) * e);
+      s.u.p1.x[SB + rl][i] = __float2bfloat16_rn(__bfloat162float(s.u.p1.q[r0 + rl][i]) * e);
     }
     for (int p = tid; p < ns * DK; p += NT) {
       const int sc = p / DK, i = p % DK;
-      s.u.ap.y[i][sc] = s.k[sc][i] * __expf(s.g[r0][i] - s.g[sc][i]);
+      s.u.p1.y[sc][i] =
+          __float2bfloat16_rn(__bfloat162float(s.k[sc][i]) * __expf(s.g[r0][i] - s.g[sc][i]));
     }
     __syncthreads();
-    // warp w: row r0 + w; lanes: columns lane, lane + 32 (< ns)
-    {
-      const int rl = warp, r = r0 + rl;
-      const int s0 = lane, s1 = lane + 32;
-      const bool on0 = s0 < ns, on1 = s1 < ns;
-      float a0 = 0.f, a1 = 0.f, p0 = 0.f, p1 = 0.f;
-#pragma unroll 4
-      for (int i = 0; i < DK; ++i) {
-        const float xk = s.u.ap.xk[rl][i], xq = s.u.ap.xq[rl][i];
-        const float y0 = on0 ? s.u.ap.y[i][s0] : 0.f;
-        const float y1 = on1 ? s.u.ap.y[i][s1] : 0.f;
-        a0 = fmaf(xk, y0, a0);
-        p0 = fmaf(xq, y0, p0);
-        a1 = fmaf(xk, y1, a1);
-        p1 = fmaf(xq, y1, p1);
-      }
-      const float br = s.beta[r];
-      if (on0) {
-        s.a[r][s0] = br * a0;
-        store_bf16_at(outP, r, s0, p0);
-      }
-      if (on1) {
-        s.a[r][s1] = br * a1;
-        store_bf16_at(outP, r, s1, p1);
+    // [A rows; P rows] (32 x ns) = x (32 x DK) y^T, in 16 x 8 tiles
+    const int ntile = ns / 8;
+    for (int task = warp; task < 2 * ntile; task += NT / 32) {
+      const int mt = task / ntile, nt = task % ntile;
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k0 = 0; k0 < DK; k0 += 16)
+        mma_16x8x16(d, &s.u.p1.x[0][0], DK + 8, 16 * mt, &s.u.p1.y[0][0], DK + 8, 8 * nt, k0,
+                    lane);
+      const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = r0 + gq + 8 * (e >> 1), sc = 8 * nt + 2 * tq + (e & 1);
+        if (mt == 0)
+          s.u.p1.a[r][sc] = s.beta[r] * d[e];
+        else
+          store_bf16_at(outP, r, sc, d[e]);
       }
     }
   }
   __syncthreads();
 
-  // ---- T = (I + A)^{-1} by forward substitution, eight threads per column
-  // c (they split the sum over m and combine it with three shuffles)
+  // ---- T = (I + A)^{-1} by forward substitution, four threads per column
+  // c: thread j keeps T[m][c] for m = j, j + 4, ... in registers; the four
+  // split the sum over m and combine it with two shuffles
   {
-    const int c = tid >> 3, j = tid & 7;
-    for (int r = 0; r < C; ++r) {
+    constexpr int TPC = NT / C;  // threads per column
+    const int c = tid / TPC, j = tid % TPC;
+    float tc[C / TPC];
+#pragma unroll
+    for (int u = 0; u < C / TPC; ++u) tc[u] = (TPC * u + j == c) ? 1.f : 0.f;
+    for (int r = 1; r < C; ++r) {  // uniform over the warp (eight columns)
       float part = 0.f;
-      if (r > c)
-        for (int m = c + j; m < r; m += 8) part = fmaf(s.a[r][m], s.t[m][c], part);
-      part += __shfl_xor_sync(0xffffffffu, part, 1);
-      part += __shfl_xor_sync(0xffffffffu, part, 2);
-      part += __shfl_xor_sync(0xffffffffu, part, 4);
-      if (j == 0) s.t[r][c] = r < c ? 0.f : (r == c ? 1.f : -part);
-      __syncwarp();
+#pragma unroll
+      for (int u = 0; u < C / TPC; ++u) {
+        const int m = TPC * u + j;
+        if (m >= c && m < r) part = fmaf(s.u.p1.a[r][m], tc[u], part);
+      }
+#pragma unroll
+      for (int w = 1; w < TPC; w <<= 1) part += __shfl_xor_sync(0xffffffffu, part, w, TPC);
+#pragma unroll
+      for (int u = 0; u < C / TPC; ++u)
+        if (r > c && TPC * u + j == r) tc[u] = -part;
     }
+    __syncthreads();  // every thread is done reading A: T may go over q
+#pragma unroll
+    for (int u = 0; u < C / TPC; ++u) s.u.p2.t[TPC * u + j][c] = tc[u] * s.beta[c];
   }
   __syncthreads();
-  // T' = T diag(beta), in place
-  for (int p = tid; p < C * C; p += NT) s.t[p / C][p % C] *= s.beta[p % C];
-  __syncthreads();
 
-  // ---- T'^T rows (row c = column c of T'), K o e^{G_last - G},
-  // e^{G_last}, Q o e^{G}, and K o e^{G} for W
+  // ---- T'^T rows (row c = column c of T'), K o e^{G_last - G}, e^{G_last},
+  // and the bf16 operands of W
   if (tid < C) {
     float col[C];
 #pragma unroll
-    for (int r = 0; r < C; ++r) col[r] = s.t[r][tid];
+    for (int r = 0; r < C; ++r) col[r] = s.u.p2.t[r][tid];
     sw128_store_row(out + off.tp, tid, col);
   }
   for (int p = tid; p < C * (DK / 8); p += NT) {
     const int tok = p / (DK / 8), i0 = (p % (DK / 8)) * 8;
-    float xk[8], xq[8];
+    float x[8];
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
       const int i = i0 + jj;
-      xk[jj] = s.k[tok][i] * __expf(s.g[C - 1][i] - s.g[tok][i]);
-      xq[jj] = __bfloat162float(s.q[tok][i]) * __expf(s.g[tok][i]);
+      x[jj] = __bfloat162float(s.k[tok][i]) * __expf(s.g[C - 1][i] - s.g[tok][i]);
     }
-    uint4 uk, uq;
-    uk.x = pack_bf16x2(xk[0], xk[1]); uk.y = pack_bf16x2(xk[2], xk[3]);
-    uk.z = pack_bf16x2(xk[4], xk[5]); uk.w = pack_bf16x2(xk[6], xk[7]);
-    uq.x = pack_bf16x2(xq[0], xq[1]); uq.y = pack_bf16x2(xq[2], xq[3]);
-    uq.z = pack_bf16x2(xq[4], xq[5]); uq.w = pack_bf16x2(xq[6], xq[7]);
-    const uint32_t o16 = (i0 / 64) * 8192 + sw128_chunk_off(tok, (i0 % 64) / 8);
-    *reinterpret_cast<uint4*>(out + off.k + o16) = uk;
-    *reinterpret_cast<uint4*>(out + off.q + o16) = uq;
+    *reinterpret_cast<uint4*>(out + off.k + (i0 / 64) * 8192 +
+                              sw128_chunk_off(tok, (i0 % 64) / 8)) = pack8(x);
   }
   if (tid < DK) reinterpret_cast<float*>(out + off.d)[tid] = __expf(s.g[C - 1][tid]);
-  for (int p = tid; p < C * DK; p += NT) {
-    const int tok = p / DK, i = p % DK;
-    s.u.khat[tok][i] = s.k[tok][i] * __expf(s.g[tok][i]);
+  for (int p = tid; p < C * C; p += NT)
+    s.u.p2.tb[p / C][p % C] = __float2bfloat16_rn(s.u.p2.t[p / C][p % C]);
+  for (int p = tid; p < C * DK; p += NT) {  // threads on consecutive tokens
+    const int tok = p % C, i = p / C;
+    s.u.p2.kc[i][tok] = __float2bfloat16_rn(__bfloat162float(s.k[tok][i]) * __expf(s.g[tok][i]));
   }
   __syncthreads();
 
-  // ---- W = T' (K o e^{G}): thread on channel i and four rows at a time
+  // ---- W = T' (K o e^{G}) (64 x DK): warp w takes the 16 rows 16 (w % 4)
+  // and NTW column tiles of 8 from 8 NTW (w / 4)
   {
-    constexpr int RG = NT / DK;  // row groups
-    const int i = tid % DK, rg = tid / DK;
-    uint8_t* outW = out + off.w + (i / 64) * 8192;
-    const int ic = i % 64;
-    for (int r0 = 4 * rg; r0 < C; r0 += 4 * RG) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int sc = 0; sc <= r0 + 3; ++sc) {
-        const float kh = s.u.khat[sc][i];
+    constexpr int NTW = DK / 16;
+    const int mt = warp & 3, nt0 = (warp >> 2) * NTW;
+    float d[NTW][4];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) acc[jj] = fmaf(s.t[r0 + jj][sc], kh, acc[jj]);
+    for (int q2 = 0; q2 < NTW; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d[q2][e] = 0.f;
+#pragma unroll
+    for (int k0 = 0; k0 < C; k0 += 16)
+#pragma unroll
+      for (int q2 = 0; q2 < NTW; ++q2)
+        mma_16x8x16(d[q2], &s.u.p2.tb[0][0], C + 8, 16 * mt, &s.u.p2.kc[0][0], C + 8,
+                    8 * (nt0 + q2), k0, lane);
+    const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int q2 = 0; q2 < NTW; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = 16 * mt + gq + 8 * (e >> 1), i = 8 * (nt0 + q2) + 2 * tq + (e & 1);
+        store_bf16_at(out + off.w + (i / 64) * 8192, r, i % 64, d[q2][e]);
       }
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) store_bf16_at(outW, r0 + jj, ic, acc[jj]);
-    }
   }
 }
 
