@@ -269,7 +269,7 @@ def run_ours(args, rank, world, dev):
     chain_gbs = chain_w["bytes"] / (ms_chain / 1e3) / 1e9
 
     # end to end through the public API with host buffers (pinned)
-    e2e = measure_e2e(args, w, x, fn, dev, stream, world)
+    e2e = None if args.no_e2e else measure_e2e(args, w, x, fn, dev, stream, world)
 
     res = {
         "metric": metric_name(args.workload),
@@ -499,8 +499,8 @@ def run_kda_prefill(w, dev, stream, flush, peaks, peak_src, steps=3):
     return {"metric": "prefill tokens/s, per-channel gate (%s)" % w.name,
             "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
             "calls": steps,
-            "path": "kda_prep_kernel (per-chunk factors, CUDA cores fp32) + chain_kernel "
-                    "(KDA mode, tcgen05)",
+            "path": "kda_prep_kernel (per-chunk factors: fp32 CUDA cores and bf16 warp "
+                    "MMAs) + chain_kernel (KDA mode, tcgen05)",
             "roofline": {"kernel": "whole call", "bound": "hbm",
                          "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "traffic": None, "algorithmic_bytes": byts,
@@ -624,6 +624,9 @@ def main():
     ap.add_argument("--path", choices=["chunk", "recurrent"], default="chunk")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffers) measurement, e.g. for a "
+                         "profiler's launch list of the prefill alone")
     ap.add_argument("--no-kda", action="store_true",
                     help="skip the per-channel-gate (KDA form) prefill measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
