@@ -36,6 +36,22 @@
  * h-form, per token:  h <- Diag(a) h  (row i scaled by a_i);  r = h^T k;
  *                     u = beta (v - r);  h <- h + k u^T;  o = h^T q.
  *
+ * Gradients (reverse mode through the token loop of the GDN form, for a
+ * loss L with dL/do = do and dL/dh_T = dhT; the pages print no backward
+ * algorithm, so this is the chain rule applied to the lines above, each
+ * step of it named where it is taken).  The states h_t are kept for every
+ * token; walking t down from T - 1 with H = dL/dh_t:
+ *   H += q_t do_t^T;  dq_t = h_t do_t                      (o_t = h_t^T q_t)
+ *   du = H^T k_t;  dk_t += H u_t;  da = <H, h_{t-1}>;  H' = alpha H
+ *                                                      (h_t = alpha h_{t-1} + k u^T)
+ *   dv_t = beta du;  dbeta = du . (v - alpha r);  da -= beta du . r;
+ *   dr = -alpha beta du                              (u = beta (v - alpha r))
+ *   H' += k dr^T;  dk_t += h_{t-1} dr                (r = h_{t-1}^T k)
+ *   dg_t = da alpha                                  (alpha = exp(g))
+ * and H <- H'; dh0 = H at the end.  KLA adds the step size
+ * beta = eta / (n2 + eps), n2 = ||k||^2: deta = dbeta / (n2 + eps) and
+ * dk += -2 dbeta eta / (n2 + eps)^2 k.
+ *
  * Layouts (row-major, contiguous):
  *   q, k : [B][T][H][dk]     v, o : [B][T][H][dv]
  *   g, eta, beta : [B][T][H]  (per-channel gate: g is [B][T][H][dk])
@@ -180,6 +196,141 @@ void kla_oracle_kda(const double *q, const double *k, const double *v,
         free(S);
         free(u);
     }
+}
+
+/* Gradients of the GDN form (beta given) for dL/do = dout and dL/dh_T =
+ * dhT (NULL = 0): writes dq, dk [B][T][H][dk], dv [B][T][H][dv],
+ * dg, dbeta [B][T][H] and dh0 [B][H][dk][dv] (NULL = not returned). */
+void kla_oracle_gated_delta_backward(const double *q, const double *k, const double *v,
+                                     const double *g, const double *beta, const double *h0,
+                                     const double *dout, const double *dhT,
+                                     double *dq, double *dk, double *dv, double *dg,
+                                     double *dbeta, double *dh0,
+                                     int B, int T, int H, int dk_, int dv_)
+{
+    const int dK = dk_, dV = dv_;
+    int nheads = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < nheads; ++bh) {
+        int b = bh / H, hh = bh % H;
+        size_t SZ = (size_t)dK * dV;
+        /* hs[t + 1] = h_t, hs[0] = h0 */
+        double *hs = (double *)malloc(sizeof(double) * SZ * (size_t)(T + 1));
+        double *Hm = (double *)malloc(sizeof(double) * SZ);
+        double *Hn = (double *)malloc(sizeof(double) * SZ);
+        double *r = (double *)malloc(sizeof(double) * (size_t)dV);
+        double *u = (double *)malloc(sizeof(double) * (size_t)dV);
+        double *du = (double *)malloc(sizeof(double) * (size_t)dV);
+        double *dr = (double *)malloc(sizeof(double) * (size_t)dV);
+        if (h0)
+            memcpy(hs, h0 + (size_t)bh * SZ, sizeof(double) * SZ);
+        else
+            memset(hs, 0, sizeof(double) * SZ);
+        /* forward, keeping every state */
+        for (int t = 0; t < T; ++t) {
+            size_t tok = ((size_t)b * T + t) * H + hh;
+            const double *kt = k + tok * dK, *vt = v + tok * dV;
+            const double *hp = hs + (size_t)t * SZ;
+            double *hc = hs + (size_t)(t + 1) * SZ;
+            double alpha = exp(g[tok]), bt = beta[tok];
+            for (int j = 0; j < dV; ++j) r[j] = 0.0;
+            for (int i = 0; i < dK; ++i)
+                for (int j = 0; j < dV; ++j) r[j] += hp[(size_t)i * dV + j] * kt[i];
+            for (int j = 0; j < dV; ++j) u[j] = bt * (vt[j] - alpha * r[j]);
+            for (int i = 0; i < dK; ++i)
+                for (int j = 0; j < dV; ++j)
+                    hc[(size_t)i * dV + j] = alpha * hp[(size_t)i * dV + j] + kt[i] * u[j];
+        }
+        /* reverse */
+        if (dhT)
+            memcpy(Hm, dhT + (size_t)bh * SZ, sizeof(double) * SZ);
+        else
+            memset(Hm, 0, sizeof(double) * SZ);
+        for (int t = T - 1; t >= 0; --t) {
+            size_t tok = ((size_t)b * T + t) * H + hh;
+            const double *qt = q + tok * dK, *kt = k + tok * dK, *vt = v + tok * dV;
+            const double *dot = dout + tok * dV;
+            const double *hp = hs + (size_t)t * SZ, *hc = hs + (size_t)(t + 1) * SZ;
+            double *dqt = dq + tok * dK, *dkt = dk + tok * dK, *dvt = dv + tok * dV;
+            double alpha = exp(g[tok]), bt = beta[tok];
+            /* o_t = h_t^T q_t */
+            for (int i = 0; i < dK; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dV; ++j) {
+                    Hm[(size_t)i * dV + j] += qt[i] * dot[j];
+                    acc += hc[(size_t)i * dV + j] * dot[j];
+                }
+                dqt[i] = acc;
+            }
+            /* recompute r, u of this step */
+            for (int j = 0; j < dV; ++j) r[j] = 0.0;
+            for (int i = 0; i < dK; ++i)
+                for (int j = 0; j < dV; ++j) r[j] += hp[(size_t)i * dV + j] * kt[i];
+            for (int j = 0; j < dV; ++j) u[j] = bt * (vt[j] - alpha * r[j]);
+            /* h_t = alpha h_{t-1} + k u^T */
+            double da = 0.0;
+            for (int j = 0; j < dV; ++j) du[j] = 0.0;
+            for (int i = 0; i < dK; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dV; ++j) {
+                    du[j] += Hm[(size_t)i * dV + j] * kt[i];
+                    acc += Hm[(size_t)i * dV + j] * u[j];
+                    da += Hm[(size_t)i * dV + j] * hp[(size_t)i * dV + j];
+                    Hn[(size_t)i * dV + j] = alpha * Hm[(size_t)i * dV + j];
+                }
+                dkt[i] = acc;
+            }
+            /* u = beta (v - alpha r) */
+            double db = 0.0;
+            for (int j = 0; j < dV; ++j) {
+                dvt[j] = bt * du[j];
+                db += du[j] * (vt[j] - alpha * r[j]);
+                da -= bt * du[j] * r[j];
+                dr[j] = -alpha * bt * du[j];
+            }
+            /* r = h_{t-1}^T k */
+            for (int i = 0; i < dK; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dV; ++j) {
+                    Hn[(size_t)i * dV + j] += kt[i] * dr[j];
+                    acc += hp[(size_t)i * dV + j] * dr[j];
+                }
+                dkt[i] += acc;
+            }
+            dg[tok] = da * alpha;
+            dbeta[tok] = db;
+            double *tmp = Hm; Hm = Hn; Hn = tmp;
+        }
+        if (dh0) memcpy(dh0 + (size_t)bh * SZ, Hm, sizeof(double) * SZ);
+        free(hs); free(Hm); free(Hn); free(r); free(u); free(du); free(dr);
+    }
+}
+
+/* Gradients of KLA (beta = eta / (||k||^2 + eps)): the GDN gradients, then
+ * the step size's chain rule into deta and dk. */
+void kla_oracle_backward(const double *q, const double *k, const double *v, const double *g,
+                         const double *eta, double eps, const double *h0,
+                         const double *dout, const double *dhT,
+                         double *dq, double *dk, double *dv, double *dg, double *deta,
+                         double *dh0, int B, int T, int H, int dk_, int dv_)
+{
+    size_t n = (size_t)B * T * H;
+    double *beta = (double *)malloc(sizeof(double) * (n ? n : 1));
+    double *dbeta = (double *)malloc(sizeof(double) * (n ? n : 1));
+    kla_oracle_beta(k, eta, eps, beta, B, T, H, dk_);
+    kla_oracle_gated_delta_backward(q, k, v, g, beta, h0, dout, dhT, dq, dk, dv, dg, dbeta,
+                                    dh0, B, T, H, dk_, dv_);
+    for (size_t p = 0; p < n; ++p) {
+        const double *kp = k + p * dk_;
+        double n2 = 0.0;
+        for (int i = 0; i < dk_; ++i) n2 += kp[i] * kp[i];
+        double den = n2 + eps;
+        deta[p] = dbeta[p] / den;
+        double c = -2.0 * dbeta[p] * eta[p] / (den * den);
+        for (int i = 0; i < dk_; ++i) dk[p * dk_ + i] += c * kp[i];
+    }
+    free(beta);
+    free(dbeta);
 }
 
 /* Number of OpenMP threads a parallel region would use (for reporting). */

@@ -1,0 +1,70 @@
+"""Pins for the oracle's gradients of KLA (reverse mode through the token
+loop; the pages print no backward algorithm): central finite differences
+of the separately pinned forward oracle, the Euler identities of the two
+linear dependences (o is linear in q; (o, h_T) jointly linear in (v, h0)),
+and a one-token closed form."""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _problem(seed, B=1, T=7, H=2, dk=5, dv=4, gate=True):
+    r = np.random.Generator(np.random.PCG64(seed))
+    q = r.standard_normal((B, T, H, dk))
+    k = r.standard_normal((B, T, H, dk)) * np.exp(r.uniform(-0.7, 0.7, (B, T, H, 1)))
+    v = r.standard_normal((B, T, H, dv))
+    g = -np.log1p(np.exp(r.normal(0.5, 1.0, (B, T, H)))) if gate else np.zeros((B, T, H))
+    eta = r.uniform(0.2, 1.8, (B, T, H))
+    h0 = r.standard_normal((B, H, dk, dv)) * 0.3
+    dout = r.standard_normal((B, T, H, dv))
+    dhT = r.standard_normal((B, H, dk, dv))
+    return dict(q=q, k=k, v=v, g=g, eta=eta, h0=h0), dout, dhT
+
+
+def _loss(x, eps, dout, dhT):
+    o, hT = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["eta"], eps, x["h0"])
+    return float((o * dout).sum() + (hT * dhT).sum())
+
+
+@pytest.mark.parametrize("eps", [1e-6, 0.5])
+def test_gradients_match_finite_differences(eps):
+    x, dout, dhT = _problem(31)
+    gr = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["eta"], eps, x["h0"], dout, dhT)
+    r = np.random.Generator(np.random.PCG64(32))
+    names = dict(q="dq", k="dk", v="dv", g="dg", eta="deta", h0="dh0")
+    for name, gname in names.items():
+        for trial in range(2):
+            d = r.standard_normal(x[name].shape)
+            h = 1e-6
+            xp = dict(x); xp[name] = x[name] + h * d
+            xm = dict(x); xm[name] = x[name] - h * d
+            fd = (_loss(xp, eps, dout, dhT) - _loss(xm, eps, dout, dhT)) / (2 * h)
+            an = float((gr[gname] * d).sum())
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_euler_identities():
+    x, dout, dhT = _problem(33, T=9)
+    eps = 1e-6
+    gr = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["eta"], eps, x["h0"], dout, dhT)
+    o, hT = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["eta"], eps, x["h0"])
+    lo = float((o * dout).sum())
+    lh = float((hT * dhT).sum())
+    assert abs(float((gr["dq"] * x["q"]).sum()) - lo) < 1e-10 * max(1.0, abs(lo))
+    lin = float((gr["dv"] * x["v"]).sum() + (gr["dh0"] * x["h0"]).sum())
+    assert abs(lin - (lo + lh)) < 1e-10 * max(1.0, abs(lo + lh))
+
+
+def test_one_token_closed_form():
+    """T = 1, h0 = 0: o = beta (k . q) v, so dv = beta (k . q) dout and
+    dq = beta (v . dout) k."""
+    x, dout, _ = _problem(34, T=1, H=1)
+    x["h0"] = np.zeros_like(x["h0"])
+    eps = 0.25
+    gr = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["eta"], eps, None, dout, None)
+    k = x["k"][0, 0, 0]; q = x["q"][0, 0, 0]; v = x["v"][0, 0, 0]; do = dout[0, 0, 0]
+    beta = x["eta"][0, 0, 0] / (k @ k + eps)
+    np.testing.assert_allclose(gr["dv"][0, 0, 0], beta * (k @ q) * do, rtol=1e-12)
+    np.testing.assert_allclose(gr["dq"][0, 0, 0], beta * (v @ do) * k, rtol=1e-12)
+    assert abs(gr["dg"][0, 0, 0]) < 1e-12  # alpha multiplies the zero state only
