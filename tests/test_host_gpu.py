@@ -52,3 +52,24 @@ def test_host_prefill_repeated_calls_share_staging():
         o_ref, h_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"],
                                       x["h0"])
         assert rel(o, o_ref) < TOL["bf16"] and rel(hT, h_ref) < TOL["bf16"]
+
+
+def test_host_prefill_many_pieces_reuse_slots():
+    """Large enough to be cut into four pieces of two sequences (slots are
+    reused): equal to the device-buffer call to rounding, and to the oracle
+    on a sampled head of the last piece."""
+    w = inputs.WORKLOADS["prefill_4k"].scaled(B=8, T=8192, H=8, seed=63)
+    x = _pinned(inputs.make_prefill(w, with_h0=True))
+    o, hT = api.chunk_fwd_host(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"])
+    torch.cuda.synchronize()
+    api.check_device_error()
+    xc = cuda(x)
+    o2, h2 = api.chunk_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"], xc["h0"])
+    torch.cuda.synchronize()
+    assert rel(o, o2.cpu()) < 2e-3 and rel(hT, h2.cpu()) < 2e-3
+    b, h = 7, 5
+    sl = lambda t: t[b:b + 1, :, h:h + 1]
+    o_ref, h_ref = oracle.forward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["eta"]),
+                                  x["eps"], x["h0"][b:b + 1, h:h + 1])
+    assert rel(o[b:b + 1, :, h:h + 1], o_ref) < TOL["bf16"]
+    assert rel(hT[b:b + 1, h:h + 1], h_ref) < TOL["bf16"]
