@@ -52,6 +52,14 @@ constexpr int SB = 16;  // sub-block of rows sharing one decay reference
 // operands, never A, which other warps may still be reading while T is
 // written).
 template <int DK>
+struct KdaPrepHead {  // the operands that live before A in the first phase
+  __nv_bfloat16 q[C][DK + 2];
+  __nv_bfloat16 x[2 * SB][DK + 8];
+  __nv_bfloat16 y[3 * SB][DK + 8];
+};
+constexpr size_t kInvBytes = 3 * C * (C + 8) * 2;  // the inverse's first operands
+
+template <int DK>
 struct KdaPrepSmem {
   __nv_bfloat16 k[C][DK + 2];  // keys, token-major (the bf16 inputs, exact)
   float g[C][DK + 1];          // G, the in-chunk cumsum of the gate, token-major
@@ -61,8 +69,17 @@ struct KdaPrepSmem {
       __nv_bfloat16 x[2 * SB][DK + 8];  // rows of one sub-block: k_ri e^{G_ri - G_ref,i},
                                         // then q_ri e^{G_ri - G_ref,i}
       __nv_bfloat16 y[3 * SB][DK + 8];  // k_si e^{G_ref,i - G_si}, s before the sub-block
-      float a[C][C + 1];                // A, row r column s
+      // A comes after the inverse's first operands, which are formed from it
+      uint8_t pad[sizeof(KdaPrepHead<DK>) >= kInvBytes
+                      ? 16
+                      : kInvBytes - sizeof(KdaPrepHead<DK>) + 16];
+      float a[C][C + 1];  // A, row r column s
     } p1;
+    struct {  // the inverse: N = D A_O, X_{i+1} = D - N X_i (bf16 operands)
+      __nv_bfloat16 d[C][C + 8];   // D = block-diagonal (I + A_D)^{-1}, row-major; then X_1^T
+      __nv_bfloat16 xt[C][C + 8];  // X_0^T = D^T, then X_2^T
+      __nv_bfloat16 aot[C][C + 8];  // A_O^T (A outside the diagonal blocks, transposed)
+    } p3;
     struct {
       float t[C][C + 1];            // T = (I + A)^{-1}, then T' = T diag(beta)
       __nv_bfloat16 tb[C][C + 8];   // T', bf16
@@ -252,32 +269,105 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   }
   __syncthreads();
 
-  // ---- T = (I + A)^{-1} by forward substitution, four threads per column
-  // c: thread j keeps T[m][c] for m = j, j + 4, ... in registers; the four
-  // split the sum over m and combine it with two shuffles
-  {
-    constexpr int TPC = NT / C;  // threads per column
-    const int c = tid / TPC, j = tid % TPC;
-    float tc[C / TPC];
+  // ---- T = (I + A)^{-1} by 16-blocks: with A_D the diagonal 16 x 16
+  // blocks of A, A_O the rest and D = (I + A_D)^{-1}, I + A = (I + A_D)(I + N)
+  // with N = D A_O strictly block-lower (N^4 = 0), so
+  // T = (I - N + N^2 - N^3) D:  X_0 = D, X_{i+1} = D - N X_i, T = X_3.
+  // The blocks of D by forward substitution (fp32), N and the three Horner
+  // products as bf16 warp-level tensor-core products with fp32 sums.
+  static_assert(offsetof(Smem, u.p1.a) - offsetof(Smem, u) >= kInvBytes, "A after D, D^T, A_O^T");
+  __nv_bfloat16 (*nbuf)[C + 8] = reinterpret_cast<__nv_bfloat16 (*)[C + 8]>(&s.u.p1.a[0][0]);
+  if (tid < C) {  // thread (block R, column c): column c of (I + A_RR)^{-1}
+    const int R = tid / SB, c = tid % SB, o0 = R * SB;
+    float xcol[SB];
 #pragma unroll
-    for (int u = 0; u < C / TPC; ++u) tc[u] = (TPC * u + j == c) ? 1.f : 0.f;
-    for (int r = 1; r < C; ++r) {  // uniform over the warp (eight columns)
-      float part = 0.f;
+    for (int i = 0; i < SB; ++i) {
+      float acc = 0.f;
 #pragma unroll
-      for (int u = 0; u < C / TPC; ++u) {
-        const int m = TPC * u + j;
-        if (m >= c && m < r) part = fmaf(s.u.p1.a[r][m], tc[u], part);
-      }
-#pragma unroll
-      for (int w = 1; w < TPC; w <<= 1) part += __shfl_xor_sync(0xffffffffu, part, w, TPC);
-#pragma unroll
-      for (int u = 0; u < C / TPC; ++u)
-        if (r > c && TPC * u + j == r) tc[u] = -part;
+      for (int m = 0; m < i; ++m) acc = fmaf(s.u.p1.a[o0 + i][o0 + m], xcol[m], acc);
+      xcol[i] = i == c ? 1.f : (i < c ? 0.f : -acc);
     }
-    __syncthreads();  // every thread is done reading A: T may go over q
 #pragma unroll
-    for (int u = 0; u < C / TPC; ++u) s.u.p2.t[TPC * u + j][c] = tc[u] * s.beta[c];
+    for (int i = 0; i < SB; ++i) {
+      s.u.p3.d[o0 + i][o0 + c] = __float2bfloat16_rn(xcol[i]);   // D, row-major
+      s.u.p3.xt[o0 + c][o0 + i] = __float2bfloat16_rn(xcol[i]);  // D^T
+    }
   }
+  for (int p = tid; p < C * C; p += NT) {
+    const int r = p / C, c = p % C;
+    if (r / SB != c / SB) {  // zeros of D and D^T outside the diagonal blocks
+      s.u.p3.d[r][c] = __float2bfloat16_rn(0.f);
+      s.u.p3.xt[r][c] = __float2bfloat16_rn(0.f);
+    }
+    // A_O^T (threads on consecutive c read row r of A)
+    s.u.p3.aot[c][r] = __float2bfloat16_rn(r / SB > c / SB ? s.u.p1.a[r][c] : 0.f);
+  }
+  __syncthreads();  // A is consumed: N may take its place
+  // warp w: output rows 16 (w % 4), column tiles 2 (w / 4) .. + 1 of 8
+  const int mt = warp & 3, nt0 = (warp >> 2) * 4;
+  const int gq = lane >> 2, tq = lane & 3;
+  {  // N = D A_O
+    float dn[4][4] = {};
+#pragma unroll
+    for (int k0 = 0; k0 < C; k0 += 16)
+#pragma unroll
+      for (int q2 = 0; q2 < 4; ++q2)
+        mma_16x8x16(dn[q2], &s.u.p3.d[0][0], C + 8, 16 * mt, &s.u.p3.aot[0][0], C + 8,
+                    8 * (nt0 + q2), k0, lane);
+#pragma unroll
+    for (int q2 = 0; q2 < 4; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        nbuf[16 * mt + gq + 8 * (e >> 1)][8 * (nt0 + q2) + 2 * tq + (e & 1)] =
+            __float2bfloat16_rn(dn[q2][e]);
+  }
+  // D at this thread's output positions, for the Horner combination
+  float dloc[4][4];
+#pragma unroll
+  for (int q2 = 0; q2 < 4; ++q2)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      dloc[q2][e] = __bfloat162float(
+          s.u.p3.xt[8 * (nt0 + q2) + 2 * tq + (e & 1)][16 * mt + gq + 8 * (e >> 1)]);
+  __syncthreads();  // N complete; D (row-major) is free for X_1^T
+  float xr[4][4];
+#pragma unroll
+  for (int step = 0; step < 3; ++step) {
+    // X_{step+1} = D - N X_step; X_step^T in xt (step 0, 2) or d (step 1)
+    const __nv_bfloat16* xin = step == 1 ? &s.u.p3.d[0][0] : &s.u.p3.xt[0][0];
+    __nv_bfloat16(*xout)[C + 8] = step == 0 ? s.u.p3.d : s.u.p3.xt;
+#pragma unroll
+    for (int q2 = 0; q2 < 4; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) xr[q2][e] = 0.f;
+#pragma unroll
+    for (int k0 = 0; k0 < C; k0 += 16)
+#pragma unroll
+      for (int q2 = 0; q2 < 4; ++q2)
+        mma_16x8x16(xr[q2], &nbuf[0][0], C + 8, 16 * mt, xin, C + 8, 8 * (nt0 + q2), k0, lane);
+#pragma unroll
+    for (int q2 = 0; q2 < 4; ++q2)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) xr[q2][e] = dloc[q2][e] - xr[q2][e];
+    __syncthreads();  // every warp has read X_step
+    if (step < 2) {
+#pragma unroll
+      for (int q2 = 0; q2 < 4; ++q2)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          xout[8 * (nt0 + q2) + 2 * tq + (e & 1)][16 * mt + gq + 8 * (e >> 1)] =
+              __float2bfloat16_rn(xr[q2][e]);
+      __syncthreads();
+    }
+  }
+  // T' = T diag(beta) in fp32 (T = X_3, still in registers)
+#pragma unroll
+  for (int q2 = 0; q2 < 4; ++q2)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = 16 * mt + gq + 8 * (e >> 1), c = 8 * (nt0 + q2) + 2 * tq + (e & 1);
+      s.u.p2.t[r][c] = xr[q2][e] * s.beta[c];
+    }
   __syncthreads();
 
   // ---- T'^T rows (row c = column c of T'), K o e^{G_last - G}, e^{G_last},
