@@ -330,6 +330,8 @@ def run_ours(args, rank, world, dev):
         res["decode"] = run_decode(args, rank, dev, stream, flush, peaks, peak_src, fn, clk)
     if not args.no_kda and w.dtype == "bf16":
         res["kda_prefill"] = run_kda_prefill(w, dev, stream, flush, peaks, peak_src)
+    if not args.no_bwd:
+        res["backward"] = run_backward(w, dev, stream, flush, peaks, peak_src)
     time.sleep(0.25)
     clk.__exit__()
     res["clocks"] = clk.summary(t_load, t1 + 0.15)
@@ -507,6 +509,54 @@ def run_kda_prefill(w, dev, stream, flush, peaks, peak_src, steps=3):
                          "peak_source": peak_src}}
 
 
+def run_backward(w, dev, stream, flush, peaks, peak_src, steps=2):
+    """Gradients of the prefill (token-serial fp32 backward) on the same
+    workload for a seeded dL/do and dL/dh_T: time per call and achieved GB/s
+    of its algorithmic bytes (reads q, k, v, dL/do, g, eta, dL/dh_T; writes
+    the fp32 gradients of q, k, v, g, eta, h0)."""
+    from delta_rule_linear_kla_b200 import api, inputs
+
+    x = inputs.make_prefill(w)
+    xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    gen = torch.Generator(device="cpu").manual_seed(w.seed + 21)
+    do = torch.randn((w.B, w.T, w.H, w.dv), generator=gen).to(w.torch_dtype).to(dev)
+    dhT = torch.randn((w.B, w.H, w.dk, w.dv), generator=gen).to(dev)
+    ws = torch.empty(max(1, api.recurrent_bwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv)),
+                     dtype=torch.uint8, device=dev)
+    run = lambda: api.recurrent_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["eta"], do,
+                                    x["eps"], xd["h0"], dhT, workspace=ws, stream=stream)
+    run()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for e0, e1 in evs:
+        flush()
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    api.check_device_error()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    es = 2 if w.dtype == "bf16" else 4
+    ntok = w.B * w.T * w.H
+    sb = w.B * w.H * w.dk * w.dv * 4
+    byts = (ntok * (2 * w.dk + 2 * w.dv) * es + ntok * 2 * 4 + sb
+            + ntok * (2 * w.dk + w.dv + 2) * 4 + sb)
+    gbs = byts / (ms / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    return {"metric": "backward tokens/s (%s)" % w.name,
+            "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
+            "calls": steps, "dtype": "f32",
+            "path": "bwd_checkpoint_kernel + bwd_kernel (token-serial fp32, states "
+                    "recomputed from 64-token checkpoints) + bwd_finish_kernel",
+            "roofline": {"kernel": "whole call", "bound": "hbm",
+                         "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "algorithmic_bytes": byts,
+                         "peak_source": peak_src,
+                         "note": "token-serial: bounded by the per-token dependency "
+                                 "chain, not by HBM"}}
+
+
 # ------------------------------------------------------------ reference
 def oracle_sample(w, budget_s):
     """Size a sample of workload ``w`` that costs the oracle about
@@ -629,6 +679,8 @@ def main():
                          "profiler's launch list of the prefill alone")
     ap.add_argument("--no-kda", action="store_true",
                     help="skip the per-channel-gate (KDA form) prefill measurement")
+    ap.add_argument("--no-bwd", action="store_true",
+                    help="skip the backward (gradients) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -153,6 +153,63 @@ def recurrent_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=Non
     return o, hT
 
 
+def recurrent_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int) -> int:
+    return int(_native.lib().kla_recurrent_bwd_workspace_size(B, T, H, dk, dv))
+
+
+def _bwd(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0, workspace, stream):
+    _need(q, "q")
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v must be bfloat16 or float32")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", q.dtype, (B, T, H, dk))
+    _need(v, "v", q.dtype, (B, T, H, dv))
+    _need(g, "g", torch.float32, (B, T, H))
+    _need(step, "eta/beta", torch.float32, (B, T, H))
+    _need(h0, "h0", torch.float32, (B, H, dk, dv))
+    _need(grad_o, "grad_o", q.dtype, (B, T, H, dv))
+    _need(grad_hT, "grad_hT", torch.float32, (B, H, dk, dv))
+    f32 = dict(dtype=torch.float32, device=q.device)
+    out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+               dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty((B, T, H), **f32),
+               dstep=torch.empty((B, T, H), **f32),
+               dh0=torch.empty((B, H, dk, dv), **f32) if need_h0 else None)
+    need = recurrent_bwd_workspace_size(B, T, H, dk, dv)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
+    if eps is not None:
+        args.append(float(eps))
+    args += [_ptr(h0), _ptr(grad_o), _ptr(grad_hT), _ptr(out["dq"]), _ptr(out["dk"]),
+             _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dstep"]), _ptr(out["dh0"]),
+             B, T, H, dk, dv, _DT[q.dtype], _ptr(workspace), ws_bytes, _stream(stream)]
+    _check(fn(*args), name)
+    return out
+
+
+def recurrent_bwd(q, k, v, g, eta, grad_o, eps: float = 1e-6, h0=None, grad_hT=None, *,
+                  need_h0: bool = True, workspace=None, stream=None):
+    """Gradients of the KLA prefill for dL/do = grad_o and dL/dh_T = grad_hT
+    (None = 0), token-serial fp32 (kla_recurrent_bwd).  Returns a dict of
+    fp32 tensors dq, dk, dv, dg, deta, dh0 (None unless need_h0)."""
+    out = _bwd(_native.lib().kla_recurrent_bwd, "kla_recurrent_bwd", q, k, v, g, eta, eps, h0,
+               grad_o, grad_hT, need_h0, workspace, stream)
+    out["deta"] = out.pop("dstep")
+    return out
+
+
+def gdn_recurrent_bwd(q, k, v, g, beta, grad_o, h0=None, grad_hT=None, *, need_h0: bool = True,
+                      workspace=None, stream=None):
+    """Gradients of the gated delta rule prefill (beta given per token):
+    dq, dk, dv, dg, dbeta, dh0 (kla_gdn_recurrent_bwd)."""
+    out = _bwd(_native.lib().kla_gdn_recurrent_bwd, "kla_gdn_recurrent_bwd", q, k, v, g, beta,
+               None, h0, grad_o, grad_hT, need_h0, workspace, stream)
+    out["dbeta"] = out.pop("dstep")
+    return out
+
+
 def decode_step(q, k, v, g, eta, S, eps: float = 1e-6, *, o=None, stream=None):
     """One decode token per sequence; S [B,H,dk,dv] fp32 is updated in place.
     Returns o [B,H,dv]."""

@@ -338,6 +338,90 @@ kla_status kla_kda_fwd_beta(const void* q, const void* k, const void* v, const f
 
 }  // extern "C"
 
+// Gradients of the prefill (token-serial backward), KLA step size or
+// (eps == kBetaGiven) beta given.
+static kla_status bwd_impl(const void* q, const void* k, const void* v, const float* g,
+                           const float* eta, float eps, const float* h0, const void* grad_o,
+                           const float* grad_hT, float* grad_q, float* grad_k, float* grad_v,
+                           float* grad_g, float* grad_eta, float* grad_h0, int B, int T, int H,
+                           int dk, int dv, int dtype, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  if (B < 1 || H < 1 || T < 0) return KLA_ERR_INVALID_ARG;
+  if (dtype != KLA_BF16 && dtype != KLA_FP32) return KLA_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) && eps != kBetaGiven) return KLA_ERR_INVALID_ARG;
+  if ((long long)B * T * H * (dk > dv ? dk : dv) >= (1LL << 40)) return KLA_ERR_INVALID_ARG;
+  if (T > 0 && (!q || !k || !v || !g || !eta || !grad_o || !grad_q || !grad_k || !grad_v ||
+                !grad_g || !grad_eta))
+    return KLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q,      k,      v,      g,      eta,      h0,      grad_o, grad_hT,
+                        grad_q, grad_k, grad_v, grad_g, grad_eta, grad_h0, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KLA_ERR_INVALID_ARG;
+  if (!head_dims_ok(dk, dv)) return KLA_ERR_UNSUPPORTED;
+  const size_t es = dtype == KLA_BF16 ? 2 : 4;
+  const size_t ntok = (size_t)B * T * H, sb = (size_t)B * H * dk * dv * 4;
+  const size_t need = recurrent_bwd_workspace_bytes(B, T, H, dk, dv);
+  if (T > 0 && (!workspace || ws_bytes < need)) return KLA_ERR_INVALID_ARG;
+  // every written range (gradients, workspace) is disjoint from every input
+  // and from the other written ranges
+  const Range ins[] = {rng(q, ntok * dk * es),         rng(k, ntok * dk * es),
+                       rng(v, ntok * dv * es),         rng(g, ntok * 4),
+                       rng(eta, ntok * 4),             rng(h0, h0 ? sb : 0),
+                       rng(grad_o, ntok * dv * es),    rng(grad_hT, grad_hT ? sb : 0)};
+  const Range outs[] = {rng(grad_q, ntok * dk * 4), rng(grad_k, ntok * dk * 4),
+                        rng(grad_v, ntok * dv * 4), rng(grad_g, ntok * 4),
+                        rng(grad_eta, ntok * 4),    rng(grad_h0, grad_h0 ? sb : 0),
+                        rng(workspace, T > 0 ? need : 0)};
+  for (size_t a = 0; a < sizeof(outs) / sizeof(outs[0]); ++a) {
+    for (const Range& r : ins)
+      if (overlap(outs[a], r)) return KLA_ERR_INVALID_ARG;
+    for (size_t b2 = a + 1; b2 < sizeof(outs) / sizeof(outs[0]); ++b2)
+      if (overlap(outs[a], outs[b2])) return KLA_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  if (T == 0) {  // no tokens: dL/dh0 = dL/dh_T
+    if (!grad_h0) return KLA_OK;
+    cudaError_t e = grad_hT ? cudaMemcpyAsync(grad_h0, grad_hT, sb, cudaMemcpyDeviceToDevice, st)
+                            : cudaMemsetAsync(grad_h0, 0, sb, st);
+    return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+  }
+  cudaError_t e = launch_recurrent_bwd(q, k, v, g, eta, eps, h0, grad_o, grad_hT, grad_q, grad_k,
+                                       grad_v, grad_g, grad_eta, grad_h0, B, T, H, dk, dv, dtype,
+                                       workspace, st);
+  return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+extern "C" {
+
+size_t kla_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
+  if (!head_dims_ok(dk, dv)) return 0;
+  return recurrent_bwd_workspace_bytes(B, T, H, dk, dv);
+}
+
+kla_status kla_recurrent_bwd(const void* q, const void* k, const void* v, const float* g,
+                             const float* eta, float eps, const float* h0, const void* grad_o,
+                             const float* grad_hT, float* grad_q, float* grad_k, float* grad_v,
+                             float* grad_g, float* grad_eta, float* grad_h0, int B, int T,
+                             int H, int dk, int dv, int dtype, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, g, eta, eps, h0, grad_o, grad_hT, grad_q, grad_k, grad_v, grad_g,
+                  grad_eta, grad_h0, B, T, H, dk, dv, dtype, workspace, ws_bytes, stream);
+}
+
+kla_status kla_gdn_recurrent_bwd(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, const float* h0, const void* grad_o,
+                                 const float* grad_hT, float* grad_q, float* grad_k,
+                                 float* grad_v, float* grad_g, float* grad_beta, float* grad_h0,
+                                 int B, int T, int H, int dk, int dv, int dtype, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  return bwd_impl(q, k, v, g, beta, kBetaGiven, h0, grad_o, grad_hT, grad_q, grad_k, grad_v,
+                  grad_g, grad_beta, grad_h0, B, T, H, dk, dv, dtype, workspace, ws_bytes,
+                  stream);
+}
+
+}  // extern "C"
+
 // One decode step with the KLA step size, or (eps == kBetaGiven) beta given;
 // a per-channel gate when vector_gate (g [B][H][dk]).
 static kla_status decode_impl(const void* q, const void* k, const void* v,

@@ -252,6 +252,54 @@ KLA_API kla_status kla_kda_decode_step_beta(const void *q, const void *k, const 
                                             int dtype, void *stream);
 
 /*
+ * Backward of the prefill (kla_recurrent_fwd / kla_chunk_fwd), for training:
+ * given dL/do (grad_o) and dL/dh_T (grad_hT, nullable = 0), the gradients of
+ * a loss L with respect to q, k, v, g, eta (the _gdn variant: beta) and h0.
+ * The pages print no backward; these are the exact adjoints of the token
+ * recurrence above ("Kaczmarz Linear Attention", Abstract, for the step
+ * size; "Deep Dive into KDA", section 2.2, for the gated delta rule), taken
+ * token by token in reverse order:
+ *   dH += q do^T;  dq = h_t do;  du = dH^T k;  dr = -alpha beta du;
+ *   dk = dH u + h_{t-1} dr;  dv = beta du;  dbeta = du . (v - alpha r);
+ *   dalpha = <dH, h_{t-1}> - beta du . r;  dH <- alpha dH + k dr^T;
+ *   dg = alpha dalpha;  deta = dbeta / (||k||^2 + eps) and
+ *   dk += -2 dbeta eta k / (||k||^2 + eps)^2 (KLA only).
+ * Arithmetic in fp32 on CUDA cores (token-serial; states recomputed from
+ * checkpoints every 64 tokens kept in the workspace).
+ *
+ *   q, k   [B][T][H][dk] dtype;  v, grad_o [B][T][H][dv] dtype
+ *   g, eta (beta) [B][T][H] fp32;  h0, grad_hT [B][H][dk][dv] fp32, nullable
+ *   grad_q, grad_k [B][T][H][dk] fp32;  grad_v [B][T][H][dv] fp32
+ *   grad_g, grad_eta (grad_beta) [B][T][H] fp32;  grad_h0 [B][H][dk][dv]
+ *   fp32, nullable (not computed)
+ *   workspace: device memory of kla_recurrent_bwd_workspace_size(...) bytes
+ *   (16-byte aligned; contents need no initialisation; about
+ *   B*H*ceil(T/64)*dk*dv*4 + 2*(dv/32)*B*T*H*(dk+1)*4 bytes), NULL allowed
+ *   when T == 0.
+ * dk = dv in {64, 128} (else KLA_ERR_UNSUPPORTED); T >= 0 (T == 0: grad_h0 =
+ * grad_hT).  Every gradient buffer and the workspace must be disjoint from
+ * each other and from every input, else KLA_ERR_INVALID_ARG.  Deterministic:
+ * no atomics.  Asynchronous on `stream`, no allocation.
+ */
+KLA_API size_t kla_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv);
+KLA_API kla_status kla_recurrent_bwd(const void *q, const void *k, const void *v,
+                                     const float *g, const float *eta, float eps,
+                                     const float *h0, const void *grad_o,
+                                     const float *grad_hT, float *grad_q, float *grad_k,
+                                     float *grad_v, float *grad_g, float *grad_eta,
+                                     float *grad_h0, int B, int T, int H, int dk, int dv,
+                                     int dtype, void *workspace, size_t ws_bytes,
+                                     void *stream);
+KLA_API kla_status kla_gdn_recurrent_bwd(const void *q, const void *k, const void *v,
+                                         const float *g, const float *beta,
+                                         const float *h0, const void *grad_o,
+                                         const float *grad_hT, float *grad_q, float *grad_k,
+                                         float *grad_v, float *grad_g, float *grad_beta,
+                                         float *grad_h0, int B, int T, int H, int dk, int dv,
+                                         int dtype, void *workspace, size_t ws_bytes,
+                                         void *stream);
+
+/*
  * Prefill from HOST buffers, end to end: the same computation as
  * kla_chunk_fwd with q, k, v, g, eta, h0 (nullable), o and hT (nullable) in
  * host memory (same layouts; page-locked memory is needed for the copies to

@@ -70,6 +70,9 @@ def _load():
     lib.kla_oracle_backward.argtypes = [dp, dp, dp, dp, dp, ctypes.c_double, dp, dp, dp,
                                         dp, dp, dp, dp, dp, dp, i, i, i, i, i]
     lib.kla_oracle_backward.restype = None
+    lib.kla_oracle_gated_delta_backward.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp,
+                                                    dp, dp, dp, dp, dp, dp, i, i, i, i, i]
+    lib.kla_oracle_gated_delta_backward.restype = None
     lib.kla_oracle_num_threads.argtypes = []
     lib.kla_oracle_num_threads.restype = i
     _lib = lib
@@ -151,6 +154,24 @@ def backward(q, k, v, g, eta, eps: float, h0, dout, dhT=None):
                                 _ptr(h0), _ptr(dout), _ptr(dhT), _ptr(out["dq"]),
                                 _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
                                 _ptr(out["deta"]), _ptr(out["dh0"]), B, T, H, dk, dv)
+    return out
+
+
+def gated_delta_backward(q, k, v, g, beta_, h0, dout, dhT=None):
+    """Gradients of the gated delta rule (beta given per token) for
+    dL/do = dout and dL/dh_T = dhT (None = 0).  Returns dq, dk, dv, dg,
+    dbeta, dh0 (fp64)."""
+    q, k, v, g, beta_, h0, dout, dhT = map(f64, (q, k, v, g, beta_, h0, dout, dhT))
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    assert q.shape == k.shape and v.shape[:3] == (B, T, H) and dout.shape == v.shape
+    out = dict(dq=np.empty_like(q), dk=np.empty_like(k), dv=np.empty_like(v),
+               dg=np.empty((B, T, H)), dbeta=np.empty((B, T, H)),
+               dh0=np.empty((B, H, dk, dv)))
+    _load().kla_oracle_gated_delta_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta_), _ptr(h0), _ptr(dout), _ptr(dhT),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+        _ptr(out["dh0"]), B, T, H, dk, dv)
     return out
 
 

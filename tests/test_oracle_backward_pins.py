@@ -68,3 +68,27 @@ def test_one_token_closed_form():
     np.testing.assert_allclose(gr["dv"][0, 0, 0], beta * (k @ q) * do, rtol=1e-12)
     np.testing.assert_allclose(gr["dq"][0, 0, 0], beta * (v @ do) * k, rtol=1e-12)
     assert abs(gr["dg"][0, 0, 0]) < 1e-12  # alpha multiplies the zero state only
+
+
+def test_gated_delta_gradients_match_finite_differences():
+    """The gated delta form (beta given): its gradients against central
+    differences of the separately pinned gated_delta forward."""
+    x, dout, dhT = _problem(35, T=6)
+    r = np.random.Generator(np.random.PCG64(36))
+    x["beta"] = r.uniform(0.1, 1.9, x["eta"].shape)
+    gr = oracle.gated_delta_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], dout,
+                                     dhT)
+
+    def loss(y):
+        o, hT = oracle.gated_delta(y["q"], y["k"], y["v"], y["g"], y["beta"], y["h0"])
+        return float((o * dout).sum() + (hT * dhT).sum())
+
+    names = dict(q="dq", k="dk", v="dv", g="dg", beta="dbeta", h0="dh0")
+    for name, gname in names.items():
+        d = r.standard_normal(x[name].shape)
+        h = 1e-6
+        xp = dict(x); xp[name] = x[name] + h * d
+        xm = dict(x); xm[name] = x[name] - h * d
+        fd = (loss(xp) - loss(xm)) / (2 * h)
+        an = float((gr[gname] * d).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
