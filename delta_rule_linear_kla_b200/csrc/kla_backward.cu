@@ -17,14 +17,17 @@
 // The reverse sweep needs h_{t-1} at every token.  The step is not inverted
 // (with beta ||k||^2 = 1 it is singular); states are recomputed instead:
 //  * bwd_checkpoint_kernel runs the forward and stores h at the start of every
-//    64-token block, fp32 [B][H][nblk][dk][dv];
+//    64-token block, fp32 [B][H][nblk][dk][dv], and every token's beta and
+//    alpha;
 //  * bwd_kernel walks the blocks in reverse; per block it reruns the forward
-//    from the checkpoint keeping the state at every 8th token (thread-private
-//    scratch in global memory, a few MB in all, so it stays in L2), then for
-//    each 8-token sub-block in reverse reruns those 8 tokens keeping their
-//    states in shared memory and takes the 8 reverse steps.
-// Every rerun uses the same step function, so the recomputed states are
-// bitwise those of the first forward.
+//    from the checkpoint keeping the state at every 4th token (thread-private
+//    scratch in global memory, 256 KB per CTA, so it stays in L2), then for
+//    each 4-token sub-block in reverse reruns those tokens keeping their
+//    states in shared memory and takes the reverse steps.
+// Both kernels first copy a block's operands (k, q, the CTA's columns of v and
+// dL/do, beta, alpha) into shared memory, so no token step waits on a global
+// load.  Every rerun uses the same step function on the same beta and alpha,
+// so the recomputed states are bitwise those of the first forward.
 //
 // Layout: a CTA of 256 threads owns a 32-column slab of one head's state and
 // of its adjoint.  Warp w has columns 4w .. 4w+3; lane 4 rg + c owns column
@@ -41,8 +44,8 @@ namespace bwd {
 
 constexpr int NT = 256;    // threads per CTA
 constexpr int BV = 32;     // state columns per CTA
-constexpr int BLK = 64;    // tokens per checkpoint
-constexpr int SUB = 8;     // tokens per sub-block (states kept in shared memory)
+constexpr int BLK = 64;    // tokens per checkpoint (and per operand stage)
+constexpr int SUB = 4;     // tokens per sub-block (states kept in shared memory)
 constexpr int NSUB = BLK / SUB;
 constexpr unsigned FULL = 0xffffffffu;
 
@@ -54,55 +57,98 @@ __device__ __forceinline__ float rows_sum(float x) {
   return x;
 }
 
-// Operands of one token as one lane needs them.
-template <int R>
-struct Tok {
-  float k[R], q[R];
-  float v, d, g, e;  // v_j, do_j, log-gate, eta (or beta)
+// Key and query rows in shared memory get 4 floats of padding after every 32:
+// a lane reads 4-float pieces of its row group's R rows, and without the pad
+// the row groups 2 apart (64 or 32 bytes) fall on the same banks.
+__host__ __device__ constexpr int kpad(int i) { return i + ((i >> 5) << 2); }
+
+// One 64-token block's operands, staged in shared memory widened to fp32: the
+// full key and query rows, the CTA's 32 columns of v and dL/do, and per token
+// the step size beta and the decay alpha = e^g.
+template <int DK>
+struct alignas(16) Ops {
+  float k[BLK][kpad(DK)];
+  float q[BLK][kpad(DK)];
+  float v[BLK][BV];
+  float d[BLK][BV];
+  float beta[BLK];
+  float alpha[BLK];
 };
 
-template <typename T, int DK, int DV, bool WITH_Q>
-__device__ __forceinline__ void load_tok(Tok<DK / 8>& x, const T* __restrict__ q,
-                                         const T* __restrict__ k, const T* __restrict__ v,
-                                         const T* __restrict__ dout, const float* __restrict__ g,
-                                         const float* __restrict__ eta, size_t tok, int row0,
-                                         int j) {
-  constexpr int R = DK / 8;
-  const T* kt = k + tok * DK + row0;
+// Elements row0 .. row0 + R - 1 of a padded shared-memory row.
+template <int R>
+__device__ __forceinline__ void row_ld(const float* row, int row0, float (&x)[R]) {
 #pragma unroll
   for (int m = 0; m < R; m += 4) {
-    const float4 a = IO<T>::ld4(kt + m);
-    x.k[m] = a.x; x.k[m + 1] = a.y; x.k[m + 2] = a.z; x.k[m + 3] = a.w;
+    const float4 a = *reinterpret_cast<const float4*>(row + kpad(row0 + m));
+    x[m] = a.x; x[m + 1] = a.y; x[m + 2] = a.z; x[m + 3] = a.w;
   }
-  if constexpr (WITH_Q) {
-    const T* qt = q + tok * DK + row0;
-#pragma unroll
-    for (int m = 0; m < R; m += 4) {
-      const float4 a = IO<T>::ld4(qt + m);
-      x.q[m] = a.x; x.q[m + 1] = a.y; x.q[m + 2] = a.z; x.q[m + 3] = a.w;
-    }
-    x.d = IO<T>::ld(dout + tok * DV + j);
-  }
-  x.v = IO<T>::ld(v + tok * DV + j);
-  x.g = g[tok];
-  x.e = eta[tok];
 }
 
-// One forward token step of the lane's part of the state.
+// A thread's R state values to / from a [R/4][NT][4] scratch slot: 4-float
+// pieces interleaved by thread, so one vector access of a warp is 512
+// contiguous bytes (p = slot + 4 * tid).
 template <int R>
-__device__ __forceinline__ void fwd_step(float (&hs)[R], const Tok<R>& x, float eps) {
-  float n2 = 0.f, r = 0.f;
+__device__ __forceinline__ void vec_st(float* p, const float (&x)[R]) {
 #pragma unroll
-  for (int m = 0; m < R; ++m) {
-    n2 = fmaf(x.k[m], x.k[m], n2);
-    r = fmaf(hs[m], x.k[m], r);
+  for (int m = 0; m < R; m += 4)
+    *reinterpret_cast<float4*>(p + m * NT) = make_float4(x[m], x[m + 1], x[m + 2], x[m + 3]);
+}
+template <int R>
+__device__ __forceinline__ void vec_ld(const float* p, float (&x)[R]) {
+#pragma unroll
+  for (int m = 0; m < R; m += 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p + m * NT);
+    x[m] = a.x; x[m + 1] = a.y; x[m + 2] = a.z; x[m + 3] = a.w;
   }
-  n2 = rows_sum(n2);
-  r = rows_sum(r);
-  const float beta = step_size(x.e, n2, eps), alpha = expf(x.g);
-  const float u = beta * (x.v - alpha * r);
+}
+
+// 4 consecutive elements from global memory -> 4 floats in shared memory.
+template <typename T>
+__device__ __forceinline__ void copy4(float* dst, const T* src) {
+  *reinterpret_cast<float4*>(dst) = IO<T>::ld4(src);
+}
+
+// Cooperative copy of tokens t0 .. t0 + n - 1 into the stage, widened.
+template <typename T, int DK, int DV, bool WITH_QD>
+__device__ __forceinline__ void stage_block(Ops<DK>& s, const T* __restrict__ q,
+                                            const T* __restrict__ k, const T* __restrict__ v,
+                                            const T* __restrict__ dout, int b, int hh,
+                                            int Tlen, int H, int t0, int n, int j0) {
+  constexpr int RK = DK / 4, RV = BV / 4;  // 4-element pieces per row
+  for (int p = threadIdx.x; p < n * RK; p += NT) {
+    const int t = p / RK, ch = p % RK;
+    const size_t tok = ((size_t)b * Tlen + t0 + t) * H + hh;
+    copy4(&s.k[t][kpad(ch * 4)], k + tok * DK + ch * 4);
+    if constexpr (WITH_QD) copy4(&s.q[t][kpad(ch * 4)], q + tok * DK + ch * 4);
+  }
+  for (int p = threadIdx.x; p < n * RV; p += NT) {
+    const int t = p / RV, ch = p % RV;
+    const size_t tok = ((size_t)b * Tlen + t0 + t) * H + hh;
+    copy4(&s.v[t][ch * 4], v + tok * DV + j0 + ch * 4);
+    if constexpr (WITH_QD) copy4(&s.d[t][ch * 4], dout + tok * DV + j0 + ch * 4);
+  }
+}
+
+// One forward token step of the lane's part of the state, operands from the
+// stage (token t of the block).
+template <int DK>
+__device__ __forceinline__ void fwd_step(float (&hs)[DK / 8], const Ops<DK>& s, int t,
+                                         int row0, int col) {
+  constexpr int R = DK / 8;
+  float kk[R];
+  row_ld<R>(s.k[t], row0, kk);
+  float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-  for (int m = 0; m < R; ++m) hs[m] = fmaf(x.k[m], u, alpha * hs[m]);
+  for (int m = 0; m < R; m += 2) {
+    r0 = fmaf(hs[m], kk[m], r0);
+    r1 = fmaf(hs[m + 1], kk[m + 1], r1);
+  }
+  const float r = rows_sum(r0 + r1);
+  const float beta = s.beta[t], alpha = s.alpha[t];
+  const float u = beta * (s.v[t][col] - alpha * r);
+#pragma unroll
+  for (int m = 0; m < R; ++m) hs[m] = fmaf(kk[m], u, alpha * hs[m]);
 }
 
 // Sum the lane's R row values over the 4 column lanes of its row group; the
@@ -126,28 +172,34 @@ __device__ __forceinline__ void cols_sum_store(const float (&x)[R], float* dst, 
   }
   const int base = (b1 ? H1 : 0) + (b0 ? H2 : 0);
 #pragma unroll
-  for (int i = 0; i < H2; ++i) dst[base + i] = z[i];
+  for (int i = 0; i < H2; i += 2)
+    *reinterpret_cast<float2*>(dst + base + i) = make_float2(z[i], z[i + 1]);
 }
 
 template <int DK>
 constexpr size_t smem_bytes() {
-  return sizeof(float) * ((size_t)SUB * (DK / 8) * NT + (size_t)SUB * 2 * 8 * DK + SUB * 2 * 8);
+  return sizeof(Ops<DK>) +
+         sizeof(float) * ((size_t)SUB * (DK / 8) * NT + (size_t)SUB * 2 * 8 * DK + SUB * 2 * NT);
 }
 
 }  // namespace bwd
 
-// Forward with a checkpoint of h at the start of each 64-token block.
+// Forward with a checkpoint of h at the start of each 64-token block; also
+// writes every token's beta and alpha = e^g (CTAs of slab 0).
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(bwd::NT)
 bwd_checkpoint_kernel(const T* __restrict__ k, const T* __restrict__ v,
                       const float* __restrict__ g, const float* __restrict__ eta, float eps,
-                      const float* __restrict__ h0, float* __restrict__ ck, int Tlen, int H,
-                      int nblk) {
+                      const float* __restrict__ h0, float* __restrict__ ck,
+                      float* __restrict__ beta_out, float* __restrict__ alpha_out, int Tlen,
+                      int H, int nblk) {
   using namespace bwd;
   constexpr int R = DK / 8;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  Ops<DK>& s = *reinterpret_cast<Ops<DK>*>(smem_raw);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int rg = lane >> 2, c = lane & 3;
-  const int j = blockIdx.x * BV + warp * 4 + c, row0 = rg * R;
+  const int col = warp * 4 + c, j = blockIdx.x * BV + col, row0 = rg * R;
   const int hh = blockIdx.y, b = blockIdx.z;
   const size_t head = (size_t)b * H + hh;
 
@@ -155,44 +207,64 @@ bwd_checkpoint_kernel(const T* __restrict__ k, const T* __restrict__ v,
 #pragma unroll
   for (int m = 0; m < R; ++m) hs[m] = h0 ? h0[(head * DK + row0 + m) * DV + j] : 0.f;
 
-  Tok<R> cur, nxt;
-  auto tok_of = [&](int t) { return ((size_t)b * Tlen + t) * H + hh; };
-  const int tlast = (nblk - 1) * BLK;  // tokens before the last checkpoint
-  if (tlast > 0) load_tok<T, DK, DV, false>(cur, nullptr, k, v, nullptr, g, eta, tok_of(0), row0, j);
-  for (int t = 0; t <= tlast; ++t) {
-    if (t % BLK == 0) {
-      float* dst = ck + ((head * nblk + t / BLK) * DK + row0) * DV + j;
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int t0 = blk * BLK, n = min(BLK, Tlen - t0);
+    {
+      float* dst = ck + ((head * nblk + blk) * DK + row0) * DV + j;
 #pragma unroll
       for (int m = 0; m < R; ++m) dst[(size_t)m * DV] = hs[m];
     }
-    if (t == tlast) break;
-    if (t + 1 < tlast)
-      load_tok<T, DK, DV, false>(nxt, nullptr, k, v, nullptr, g, eta, tok_of(t + 1), row0, j);
-    fwd_step(hs, cur, eps);
-    cur = nxt;
+    __syncthreads();  // the previous block's stage is no longer read
+    stage_block<T, DK, DV, false>(s, nullptr, k, v, nullptr, b, hh, Tlen, H, t0, n,
+                                  blockIdx.x * BV);
+    for (int t = threadIdx.x; t < n; t += NT) {  // eta and g, replaced below
+      const size_t tok = ((size_t)b * Tlen + t0 + t) * H + hh;
+      s.beta[t] = eta[tok];
+      s.alpha[t] = g[tok];
+    }
+    __syncthreads();
+    for (int t = warp; t < n; t += NT / 32) {  // ||k||^2 -> beta, and alpha
+      float a = 0.f;
+      for (int i = lane; i < DK; i += 32) a = fmaf(s.k[t][kpad(i)], s.k[t][kpad(i)], a);
+      a = warp_sum(a);
+      if (lane == 0) {
+        const size_t tok = ((size_t)b * Tlen + t0 + t) * H + hh;
+        const float be = step_size(s.beta[t], a, eps), al = expf(s.alpha[t]);
+        s.beta[t] = be;
+        s.alpha[t] = al;
+        if (blockIdx.x == 0) {
+          beta_out[tok] = be;
+          alpha_out[tok] = al;
+        }
+      }
+    }
+    __syncthreads();
+    if (blk + 1 < nblk)
+      for (int t = 0; t < n; ++t) fwd_step<DK>(hs, s, t, row0, col);
   }
 }
 
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(bwd::NT)
 bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-           const float* __restrict__ g, const float* __restrict__ eta, float eps,
            const T* __restrict__ dout, const float* __restrict__ dhT,
+           const float* __restrict__ beta_in, const float* __restrict__ alpha_in,
            const float* __restrict__ ck, float* __restrict__ sub, float* __restrict__ pq,
            float* __restrict__ pk, float* __restrict__ ps, float* __restrict__ dv_out,
            float* __restrict__ dh0, int Tlen, int H, int nblk) {
   using namespace bwd;
   constexpr int R = DK / 8;
   constexpr int NSLAB = DV / BV;
-  extern __shared__ float smem[];
-  float* st = smem;                           // [SUB][R][NT] thread-private states
-  float* red = st + SUB * R * NT;             // [SUB][2][8 warps][DK]
-  float* reds = red + SUB * 2 * 8 * DK;       // [SUB][2][8 warps]
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  Ops<DK>& s = *reinterpret_cast<Ops<DK>*>(smem_raw);
+  float* st = reinterpret_cast<float*>(smem_raw + sizeof(Ops<DK>));  // [SUB][R/4][NT][4]
+  float* red = st + SUB * R * NT;        // [SUB][2][8 warps][DK]
+  float* reds = red + SUB * 2 * 8 * DK;  // [SUB][2][NT]: dalpha, dbeta per thread
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rg = lane >> 2, c = lane & 3;
   const int slab = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
-  const int j = slab * BV + warp * 4 + c, row0 = rg * R;
+  const int col = warp * 4 + c, j = slab * BV + col, row0 = rg * R;
   const size_t head = (size_t)b * H + hh;
   const size_t ntok = (size_t)gridDim.z * Tlen * H;
   float* my_sub = sub + (head * NSLAB + slab) * (size_t)(NSUB * R * NT);
@@ -202,118 +274,121 @@ bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
 #pragma unroll
   for (int m = 0; m < R; ++m) dH[m] = dhT ? dhT[(head * DK + row0 + m) * DV + j] : 0.f;
 
-  Tok<R> cur, nxt;
   for (int blk = nblk - 1; blk >= 0; --blk) {
-    const int t0 = blk * BLK, t1 = min(t0 + BLK, Tlen);
+    const int t0 = blk * BLK, n = min(BLK, Tlen - t0);
+    stage_block<T, DK, DV, true>(s, q, k, v, dout, b, hh, Tlen, H, t0, n, slab * BV);
+    for (int t = tid; t < n; t += NT) {
+      s.beta[t] = beta_in[tok_of(t0 + t)];
+      s.alpha[t] = alpha_in[tok_of(t0 + t)];
+    }
     float hs[R];
     {
       const float* src = ck + ((head * nblk + blk) * DK + row0) * DV + j;
 #pragma unroll
       for (int m = 0; m < R; ++m) hs[m] = src[(size_t)m * DV];
     }
-    // the state at every SUB-th token of the block
-    load_tok<T, DK, DV, false>(cur, q, k, v, dout, g, eta, tok_of(t0), row0, j);
-    for (int t = t0; t < t1; ++t) {
-      if ((t - t0) % SUB == 0) {
-        float* dst = my_sub + (size_t)((t - t0) / SUB) * R * NT + tid;
-#pragma unroll
-        for (int m = 0; m < R; ++m) dst[m * NT] = hs[m];
+    __syncthreads();
+    // the state at every SUB-th token of the block (thread-private scratch)
+    for (int t = 0; t < n; ++t) {
+      if (t % SUB == 0) {
+        vec_st<R>(my_sub + (size_t)(t / SUB) * R * NT + 4 * tid, hs);
       }
-      if (t + 1 == t1) break;
-      load_tok<T, DK, DV, false>(nxt, q, k, v, dout, g, eta, tok_of(t + 1), row0, j);
-      fwd_step(hs, cur, eps);
-      cur = nxt;
+      if (t + 1 < n) fwd_step<DK>(hs, s, t, row0, col);
     }
-    const int nsb = (t1 - t0 + SUB - 1) / SUB;
+    const int nsb = (n + SUB - 1) / SUB;
+    float hn[R];  // the next sub-block's start state, loaded one sub-block ahead
+    {
+      vec_ld<R>(my_sub + (size_t)(nsb - 1) * R * NT + 4 * tid, hn);
+    }
     for (int sb = nsb - 1; sb >= 0; --sb) {
-      const int s0 = t0 + sb * SUB, s1 = min(s0 + SUB, t1);
-      {
-        const float* src = my_sub + (size_t)sb * R * NT + tid;
+      const int s0 = sb * SUB, s1 = min(s0 + SUB, n);  // block-local tokens
 #pragma unroll
-        for (int m = 0; m < R; ++m) hs[m] = src[m * NT];
+      for (int m = 0; m < R; ++m) hs[m] = hn[m];
+      if (sb > 0) {
+        vec_ld<R>(my_sub + (size_t)(sb - 1) * R * NT + 4 * tid, hn);
       }
       // states before each token of the sub-block
-      load_tok<T, DK, DV, false>(cur, q, k, v, dout, g, eta, tok_of(s0), row0, j);
       for (int t = s0; t < s1; ++t) {
-        float* dst = st + (size_t)(t - s0) * R * NT + tid;
-#pragma unroll
-        for (int m = 0; m < R; ++m) dst[m * NT] = hs[m];
-        if (t + 1 == s1) break;
-        load_tok<T, DK, DV, false>(nxt, q, k, v, dout, g, eta, tok_of(t + 1), row0, j);
-        fwd_step(hs, cur, eps);
-        cur = nxt;
+        vec_st<R>(st + (size_t)(t - s0) * R * NT + 4 * tid, hs);
+        if (t + 1 < s1) fwd_step<DK>(hs, s, t, row0, col);
       }
       // reverse steps
-      load_tok<T, DK, DV, true>(cur, q, k, v, dout, g, eta, tok_of(s1 - 1), row0, j);
       for (int t = s1 - 1; t >= s0; --t) {
-        const int s = t - s0;
-        if (t > s0) load_tok<T, DK, DV, true>(nxt, q, k, v, dout, g, eta, tok_of(t - 1), row0, j);
-        float hp[R];
+        const int si = t - s0;
+        float hp[R], kk[R];
         {
-          const float* src = st + (size_t)s * R * NT + tid;
+          vec_ld<R>(st + (size_t)si * R * NT + 4 * tid, hp);
+        }
+        row_ld<R>(s.k[t], row0, kk);
+        float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-          for (int m = 0; m < R; ++m) hp[m] = src[m * NT];
+        for (int m = 0; m < R; m += 2) {
+          r0 = fmaf(hp[m], kk[m], r0);
+          r1 = fmaf(hp[m + 1], kk[m + 1], r1);
         }
-        float n2 = 0.f, r = 0.f;
+        const float r = rows_sum(r0 + r1);
+        const float beta = s.beta[t], alpha = s.alpha[t];
+        const float vj = s.v[t][col], dj = s.d[t][col];
+        const float u = beta * (vj - alpha * r);
+        float x[R];
+        {
+          float qq[R];
+          row_ld<R>(s.q[t], row0, qq);
+          float du0 = 0.f, du1 = 0.f;
 #pragma unroll
-        for (int m = 0; m < R; ++m) {
-          n2 = fmaf(cur.k[m], cur.k[m], n2);
-          r = fmaf(hp[m], cur.k[m], r);
-        }
-        n2 = rows_sum(n2);
-        r = rows_sum(r);
-        const float beta = step_size(cur.e, n2, eps), alpha = expf(cur.g);
-        const float u = beta * (cur.v - alpha * r);
-        float xq[R], xk[R];
-        float du = 0.f;
+          for (int m = 0; m < R; ++m) {
+            x[m] = fmaf(kk[m], u, alpha * hp[m]) * dj;  // h_t[i][j] do_j
+            dH[m] = fmaf(qq[m], dj, dH[m]);
+            if (m & 1)
+              du1 = fmaf(dH[m], kk[m], du1);
+            else
+              du0 = fmaf(dH[m], kk[m], du0);
+          }
+          cols_sum_store(x, red + ((size_t)(si * 2 + 0) * 8 + warp) * DK + row0, c);
+          const float du = rows_sum(du0 + du1);
+          const float dr = -alpha * beta * du;
+          float da0 = 0.f, da1 = 0.f, db = 0.f;
 #pragma unroll
-        for (int m = 0; m < R; ++m) {
-          xq[m] = fmaf(cur.k[m], u, alpha * hp[m]) * cur.d;  // h_t[i][j] do_j
-          dH[m] = fmaf(cur.q[m], cur.d, dH[m]);
-          du = fmaf(dH[m], cur.k[m], du);
+          for (int m = 0; m < R; ++m) {
+            x[m] = fmaf(dH[m], u, hp[m] * dr);
+            if (m & 1)
+              da1 = fmaf(dH[m], hp[m], da1);
+            else
+              da0 = fmaf(dH[m], hp[m], da0);
+            dH[m] = fmaf(kk[m], dr, alpha * dH[m]);
+          }
+          float da = da0 + da1;
+          if (rg == 0) {  // per-column terms, once per column
+            da -= beta * du * r;
+            db = du * (vj - alpha * r);
+            dv_out[tok_of(t0 + t) * DV + j] = beta * du;
+          }
+          cols_sum_store(x, red + ((size_t)(si * 2 + 1) * 8 + warp) * DK + row0, c);
+          // per-thread terms, summed over the CTA after the sub-block
+          reds[(si * 2 + 0) * NT + tid] = da;
+          reds[(si * 2 + 1) * NT + tid] = db;
         }
-        du = rows_sum(du);
-        const float dr = -alpha * beta * du;
-        float da = 0.f, db = 0.f;
-#pragma unroll
-        for (int m = 0; m < R; ++m) {
-          xk[m] = fmaf(dH[m], u, hp[m] * dr);
-          da = fmaf(dH[m], hp[m], da);
-          dH[m] = fmaf(cur.k[m], dr, alpha * dH[m]);
-        }
-        if (rg == 0) {  // per-column terms, once per column
-          da -= beta * du * r;
-          db = du * (cur.v - alpha * r);
-          dv_out[tok_of(t) * DV + j] = beta * du;
-        }
-        cols_sum_store(xq, red + ((size_t)(s * 2 + 0) * 8 + warp) * DK + row0, c);
-        cols_sum_store(xk, red + ((size_t)(s * 2 + 1) * 8 + warp) * DK + row0, c);
-        da = warp_sum(da);
-        db = warp_sum(db);
-        if (lane == 0) {
-          reds[(s * 2 + 0) * 8 + warp] = da;
-          reds[(s * 2 + 1) * 8 + warp] = db;
-        }
-        cur = nxt;
       }
       __syncthreads();
       // sums over the 8 warps -> this slab's partials
-      const int n = s1 - s0;
-      for (int p = tid; p < n * 2 * DK; p += NT) {
-        const int s = p / (2 * DK), qi = (p / DK) & 1, i = p % DK;
-        const float* src = red + ((size_t)(s * 2 + qi) * 8) * DK + i;
+      const int ns = s1 - s0;
+      for (int p = tid; p < ns * 2 * DK; p += NT) {
+        const int si = p / (2 * DK), qi = (p / DK) & 1, i = p % DK;
+        const float* src = red + ((size_t)(si * 2 + qi) * 8) * DK + i;
         float a = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; ++w) a += src[w * DK];
         float* dst = qi == 0 ? pq : pk;
-        dst[((size_t)slab * ntok + tok_of(s0 + s)) * DK + i] = a;
+        dst[((size_t)slab * ntok + tok_of(t0 + s0 + si)) * DK + i] = a;
       }
-      if (tid < n * 2) {
-        const int s = tid >> 1, qi = tid & 1;
+      if (warp < ns * 2) {  // warp (si, qi) sums its token's NT terms
+        const int si = warp >> 1, qi = warp & 1;
+        const float* src = reds + (si * 2 + qi) * NT;
         float a = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) a += reds[(s * 2 + qi) * 8 + w];
-        ps[((size_t)slab * ntok + tok_of(s0 + s)) * 2 + qi] = a;
+        for (int w = 0; w < NT / 32; ++w) a += src[w * 32 + lane];
+        a = warp_sum(a);
+        if (lane == 0) ps[((size_t)slab * ntok + tok_of(t0 + s0 + si)) * 2 + qi] = a;
       }
       __syncthreads();
     }
@@ -328,8 +403,8 @@ bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
 // step size's chain rule into deta and dk (KLA), or dbeta as is (eps < 0).
 template <typename T, int DK>
 __global__ void __launch_bounds__(256)
-bwd_finish_kernel(const T* __restrict__ k, const float* __restrict__ g,
-                  const float* __restrict__ eta, float eps, const float* __restrict__ pq,
+bwd_finish_kernel(const T* __restrict__ k, const float* __restrict__ eta,
+                  const float* __restrict__ alpha_in, float eps, const float* __restrict__ pq,
                   const float* __restrict__ pk, const float* __restrict__ ps, int nslab,
                   size_t ntok, float* __restrict__ dq, float* __restrict__ dk,
                   float* __restrict__ dg, float* __restrict__ deta) {
@@ -367,7 +442,7 @@ bwd_finish_kernel(const T* __restrict__ k, const float* __restrict__ g,
   } else if (lane == 0) {
     deta[tok] = sb;  // dbeta
   }
-  if (lane == 0) dg[tok] = expf(g[tok]) * sa;
+  if (lane == 0) dg[tok] = alpha_in[tok] * sa;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const int i = lane * E + e;
@@ -381,7 +456,7 @@ bwd_finish_kernel(const T* __restrict__ k, const float* __restrict__ g,
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdWs {
-  size_t ck, sub, pq, pk, ps, total;
+  size_t ck, sub, pq, pk, ps, beta, alpha, total;
 };
 
 static BwdWs bwd_layout(int B, int T, int H, int dk, int dv) {
@@ -393,7 +468,9 @@ static BwdWs bwd_layout(int B, int T, int H, int dk, int dv) {
   w.pq = w.sub + align256(heads * nslab * (size_t)bwd::NSUB * (dk / 8) * bwd::NT * 4);
   w.pk = w.pq + align256(nslab * ntok * dk * 4);
   w.ps = w.pk + align256(nslab * ntok * dk * 4);
-  w.total = w.ps + align256(nslab * ntok * 2 * 4);
+  w.beta = w.ps + align256(nslab * ntok * 2 * 4);
+  w.alpha = w.beta + align256(ntok * 4);
+  w.total = w.alpha + align256(ntok * 4);
   return w;
 }
 
@@ -415,20 +492,26 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
   float* pq = (float*)(base + w.pq);
   float* pk = (float*)(base + w.pk);
   float* ps = (float*)(base + w.ps);
+  float* wbeta = (float*)(base + w.beta);
+  float* walpha = (float*)(base + w.alpha);
   const int nblk = (Tlen + bwd::BLK - 1) / bwd::BLK;
   const dim3 grid(DV / bwd::BV, H, B);
-  bwd_checkpoint_kernel<T, DK, DV><<<grid, bwd::NT, 0, st>>>(
-      (const T*)k, (const T*)v, g, eta, eps, h0, ck, Tlen, H, nblk);
+  constexpr size_t smem_ck = sizeof(bwd::Ops<DK>);
+  cudaError_t e = cudaFuncSetAttribute(bwd_checkpoint_kernel<T, DK, DV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_ck);
+  if (e != cudaSuccess) return e;
+  bwd_checkpoint_kernel<T, DK, DV><<<grid, bwd::NT, smem_ck, st>>>(
+      (const T*)k, (const T*)v, g, eta, eps, h0, ck, wbeta, walpha, Tlen, H, nblk);
   constexpr size_t smem = bwd::smem_bytes<DK>();
-  cudaError_t e = cudaFuncSetAttribute(bwd_kernel<T, DK, DV>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(bwd_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
   if (e != cudaSuccess) return e;
   bwd_kernel<T, DK, DV><<<grid, bwd::NT, smem, st>>>(
-      (const T*)q, (const T*)k, (const T*)v, g, eta, eps, (const T*)dout, dhT, ck, sub, pq, pk,
-      ps, dv, dh0, Tlen, H, nblk);
+      (const T*)q, (const T*)k, (const T*)v, (const T*)dout, dhT, wbeta, walpha, ck, sub, pq,
+      pk, ps, dv, dh0, Tlen, H, nblk);
   const size_t ntok = (size_t)B * Tlen * H;
   const unsigned nb = (unsigned)((ntok + 7) / 8);
-  bwd_finish_kernel<T, DK><<<nb, 256, 0, st>>>((const T*)k, g, eta, eps, pq, pk, ps,
+  bwd_finish_kernel<T, DK><<<nb, 256, 0, st>>>((const T*)k, eta, walpha, eps, pq, pk, ps,
                                               DV / bwd::BV, ntok, dq, dk, dg, deta);
   return cudaGetLastError();
 }
