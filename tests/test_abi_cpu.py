@@ -201,3 +201,38 @@ def test_prefill_workspace_checks(lib):
     ut = _ut_bytes(1, T, 1)
     assert full > ut
     assert _fwd(lib, ws=6 * A - ut, wsb=full, T=T, H=1, dk=d, dv=d) == INVALID
+
+
+def _bwd(lib, q=A, k=2 * A, v=3 * A, g=4 * A, eta=5 * A, eps=1e-6, h0=None, go=6 * A,
+         ghT=None, gq=7 * A, gk=8 * A, gv=9 * A, gg=10 * A, geta=11 * A, gh0=None, B=1, T=128,
+         H=2, dk=128, dv=128, dtype=0, ws=64 * A, wsb=None):
+    if wsb is None:
+        wsb = lib.kla_recurrent_bwd_workspace_size(B, T, H, dk, dv)
+    return lib.kla_recurrent_bwd(q, k, v, g, eta, eps, h0, go, ghT, gq, gk, gv, gg, geta, gh0,
+                                 B, T, H, dk, dv, dtype, ws, wsb, None)
+
+
+def test_backward_rejects_bad_arguments(lib):
+    # the fake buffers above are 1 MiB apart: big enough for these sizes
+    need = lib.kla_recurrent_bwd_workspace_size(1, 128, 2, 128, 128)
+    assert need > 2 * 2 * 128 * 128 * 4  # two checkpoints for each of the two heads
+    assert lib.kla_recurrent_bwd_workspace_size(1, 128, 2, 96, 96) == 0
+    assert _bwd(lib, dk=96, dv=96) == UNSUPPORTED
+    assert _bwd(lib, wsb=need - 1) == INVALID
+    assert _bwd(lib, ws=None) == INVALID
+    assert _bwd(lib, eps=-1.0) == INVALID
+    assert _bwd(lib, B=0) == INVALID
+    assert _bwd(lib, dtype=7) == INVALID
+    assert _bwd(lib, gq=None) == INVALID
+    assert _bwd(lib, go=None) == INVALID
+    assert _bwd(lib, q=A + 4) == INVALID          # misaligned
+    assert _bwd(lib, gk=7 * A) == INVALID         # two gradients in one buffer
+    assert _bwd(lib, gv=3 * A) == INVALID         # a gradient over an input
+    assert _bwd(lib, ws=2 * A) == INVALID         # workspace over an input
+    assert _bwd(lib, gh0=64 * A + 4096) == INVALID  # dh0 inside the workspace
+    # T == 0 with nothing to write: valid, no CUDA call
+    assert _bwd(lib, T=0, ws=None, wsb=0) == OK
+    # the gated delta variant takes the same checks (beta for eta, no eps)
+    assert lib.kla_gdn_recurrent_bwd(A, 2 * A, 3 * A, 4 * A, 5 * A, None, 6 * A, None, 7 * A,
+                                     7 * A, 9 * A, 10 * A, 11 * A, None, 1, 128, 2, 128, 128,
+                                     0, 64 * A, need, None) == INVALID
