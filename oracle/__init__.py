@@ -73,6 +73,9 @@ def _load():
     lib.kla_oracle_gated_delta_backward.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp,
                                                     dp, dp, dp, dp, dp, dp, i, i, i, i, i]
     lib.kla_oracle_gated_delta_backward.restype = None
+    lib.kla_oracle_kda_backward.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp,
+                                            dp, dp, dp, dp, dp, dp, i, i, i, i, i]
+    lib.kla_oracle_kda_backward.restype = None
     lib.kla_oracle_num_threads.argtypes = []
     lib.kla_oracle_num_threads.restype = i
     _lib = lib
@@ -172,6 +175,38 @@ def gated_delta_backward(q, k, v, g, beta_, h0, dout, dhT=None):
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta_), _ptr(h0), _ptr(dout), _ptr(dhT),
         _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
         _ptr(out["dh0"]), B, T, H, dk, dv)
+    return out
+
+
+def kda_backward_beta(q, k, v, g, beta_, h0, dout, dhT=None):
+    """Gradients of the per-channel-gate form with beta given (g [B,T,H,dk])
+    for dL/do = dout and dL/dh_T = dhT (None = 0).  Returns dq, dk, dv, dg
+    ([B,T,H,dk]), dbeta, dh0 (fp64)."""
+    q, k, v, g, beta_, h0, dout, dhT = map(f64, (q, k, v, g, beta_, h0, dout, dhT))
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    assert q.shape == k.shape and g.shape == k.shape and dout.shape == v.shape
+    out = dict(dq=np.empty_like(q), dk=np.empty_like(k), dv=np.empty_like(v),
+               dg=np.empty_like(g), dbeta=np.empty((B, T, H)), dh0=np.empty((B, H, dk, dv)))
+    _load().kla_oracle_kda_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta_), _ptr(h0), _ptr(dout), _ptr(dhT),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+        _ptr(out["dh0"]), B, T, H, dk, dv)
+    return out
+
+
+def kda_backward(q, k, v, g, eta, eps: float, h0, dout, dhT=None):
+    """Gradients of KLA with the per-channel gate (beta = eta / (||k||^2 +
+    eps)): the beta-given gradients, then the step size's chain rule into
+    deta and dk.  Returns dq, dk, dv, dg, deta, dh0 (fp64)."""
+    kf = f64(k)
+    n2 = (kf * kf).sum(-1)
+    den = n2 + eps
+    b = f64(eta) / den
+    out = kda_backward_beta(q, k, v, g, b, h0, dout, dhT)
+    db = out.pop("dbeta")
+    out["deta"] = db / den
+    out["dk"] = out["dk"] - (2.0 * db * f64(eta) / den ** 2)[..., None] * kf
     return out
 
 

@@ -306,6 +306,124 @@ void kla_oracle_gated_delta_backward(const double *q, const double *k, const dou
     }
 }
 
+/* Gradients of the per-channel-gate form (beta given) for dL/do = dout and
+ * dL/dh_T = dhT (NULL = 0): dq, dk, dg [B][T][H][dk], dv [B][T][H][dv],
+ * dbeta [B][T][H], dh0 [B][H][dk][dv] (NULL = not returned).  Reverse mode
+ * through the token loop of kla_oracle_kda, with H = dL/dh_t and
+ * hd = Diag(a_t) h_{t-1} the decayed state:
+ *   H += q_t do_t^T;  dq_t = h_t do_t                      (o_t = h_t^T q_t)
+ *   du = H^T k;  dk_t += H u;  Hd = H                       (h_t = hd + k u^T)
+ *   dv_t = beta du;  dbeta = du . (v - r);  dr = -beta du   (u = beta (v - r))
+ *   Hd += k dr^T;  dk_t += hd dr                            (r = hd^T k)
+ *   dg_{t,i} = sum_j Hd_ij hd_ij;  H' = Diag(a_t) Hd          (hd = Diag(a) h)
+ */
+void kla_oracle_kda_backward(const double *q, const double *k, const double *v,
+                             const double *g, const double *beta, const double *h0,
+                             const double *dout, const double *dhT, double *dq, double *dk,
+                             double *dv, double *dg, double *dbeta, double *dh0, int B, int T,
+                             int H, int dk_, int dv_)
+{
+    const int dK = dk_, dV = dv_;
+    int nheads = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < nheads; ++bh) {
+        int b = bh / H, hh = bh % H;
+        size_t SZ = (size_t)dK * dV;
+        /* hs[t + 1] = h_t, hs[0] = h0 */
+        double *hs = (double *)malloc(sizeof(double) * SZ * (size_t)(T + 1));
+        double *Hm = (double *)malloc(sizeof(double) * SZ);
+        double *hd = (double *)malloc(sizeof(double) * SZ);
+        double *r = (double *)malloc(sizeof(double) * (size_t)dV);
+        double *u = (double *)malloc(sizeof(double) * (size_t)dV);
+        double *du = (double *)malloc(sizeof(double) * (size_t)dV);
+        if (h0)
+            memcpy(hs, h0 + (size_t)bh * SZ, sizeof(double) * SZ);
+        else
+            memset(hs, 0, sizeof(double) * SZ);
+        /* forward, keeping every state (the steps of kla_oracle_kda) */
+        for (int t = 0; t < T; ++t) {
+            size_t tok = ((size_t)b * T + t) * H + hh;
+            const double *kt = k + tok * dK, *vt = v + tok * dV, *gt = g + tok * dK;
+            const double *hp = hs + (size_t)t * SZ;
+            double *hc = hs + (size_t)(t + 1) * SZ;
+            for (int i = 0; i < dK; ++i) {
+                double a = exp(gt[i]);
+                for (int j = 0; j < dV; ++j) hc[(size_t)i * dV + j] = a * hp[(size_t)i * dV + j];
+            }
+            for (int j = 0; j < dV; ++j) r[j] = 0.0;
+            for (int i = 0; i < dK; ++i)
+                for (int j = 0; j < dV; ++j) r[j] += hc[(size_t)i * dV + j] * kt[i];
+            for (int j = 0; j < dV; ++j) u[j] = beta[tok] * (vt[j] - r[j]);
+            for (int i = 0; i < dK; ++i)
+                for (int j = 0; j < dV; ++j) hc[(size_t)i * dV + j] += kt[i] * u[j];
+        }
+        /* reverse */
+        if (dhT)
+            memcpy(Hm, dhT + (size_t)bh * SZ, sizeof(double) * SZ);
+        else
+            memset(Hm, 0, sizeof(double) * SZ);
+        for (int t = T - 1; t >= 0; --t) {
+            size_t tok = ((size_t)b * T + t) * H + hh;
+            const double *qt = q + tok * dK, *kt = k + tok * dK, *vt = v + tok * dV;
+            const double *gt = g + tok * dK, *dot = dout + tok * dV;
+            const double *hp = hs + (size_t)t * SZ, *hc = hs + (size_t)(t + 1) * SZ;
+            double *dqt = dq + tok * dK, *dkt = dk + tok * dK, *dvt = dv + tok * dV;
+            double *dgt = dg + tok * dK;
+            double bt = beta[tok];
+            /* o_t = h_t^T q_t */
+            for (int i = 0; i < dK; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dV; ++j) {
+                    Hm[(size_t)i * dV + j] += qt[i] * dot[j];
+                    acc += hc[(size_t)i * dV + j] * dot[j];
+                }
+                dqt[i] = acc;
+            }
+            /* recompute hd = Diag(a) h_{t-1}, r, u of this step */
+            for (int i = 0; i < dK; ++i) {
+                double a = exp(gt[i]);
+                for (int j = 0; j < dV; ++j) hd[(size_t)i * dV + j] = a * hp[(size_t)i * dV + j];
+            }
+            for (int j = 0; j < dV; ++j) r[j] = 0.0;
+            for (int i = 0; i < dK; ++i)
+                for (int j = 0; j < dV; ++j) r[j] += hd[(size_t)i * dV + j] * kt[i];
+            for (int j = 0; j < dV; ++j) u[j] = bt * (vt[j] - r[j]);
+            /* h_t = hd + k u^T */
+            for (int j = 0; j < dV; ++j) du[j] = 0.0;
+            for (int i = 0; i < dK; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dV; ++j) {
+                    du[j] += Hm[(size_t)i * dV + j] * kt[i];
+                    acc += Hm[(size_t)i * dV + j] * u[j];
+                }
+                dkt[i] = acc;
+            }
+            /* u = beta (v - r) */
+            double db = 0.0;
+            for (int j = 0; j < dV; ++j) {
+                dvt[j] = bt * du[j];
+                db += du[j] * (vt[j] - r[j]);
+            }
+            dbeta[tok] = db;
+            /* r = hd^T k:  Hd = H + k dr^T,  dk += hd dr;  then hd = Diag(a) h */
+            for (int i = 0; i < dK; ++i) {
+                double acc = 0.0, ga = 0.0, a = exp(gt[i]);
+                for (int j = 0; j < dV; ++j) {
+                    double drj = -bt * du[j];
+                    double Hd = Hm[(size_t)i * dV + j] + kt[i] * drj;
+                    acc += hd[(size_t)i * dV + j] * drj;
+                    ga += Hd * hd[(size_t)i * dV + j];
+                    Hm[(size_t)i * dV + j] = a * Hd;
+                }
+                dkt[i] += acc;
+                dgt[i] = ga;
+            }
+        }
+        if (dh0) memcpy(dh0 + (size_t)bh * SZ, Hm, sizeof(double) * SZ);
+        free(hs); free(Hm); free(hd); free(r); free(u); free(du);
+    }
+}
+
 /* Gradients of KLA (beta = eta / (||k||^2 + eps)): the GDN gradients, then
  * the step size's chain rule into deta and dk. */
 void kla_oracle_backward(const double *q, const double *k, const double *v, const double *g,

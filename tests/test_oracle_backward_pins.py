@@ -92,3 +92,59 @@ def test_gated_delta_gradients_match_finite_differences():
         fd = (loss(xp) - loss(xm)) / (2 * h)
         an = float((gr[gname] * d).sum())
         assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def _kda_problem(seed, T=6, H=2, dk=5, dv=4):
+    x, dout, dhT = _problem(seed, T=T, H=H, dk=dk, dv=dv)
+    r = np.random.Generator(np.random.PCG64(seed + 100))
+    x["gv"] = -np.log1p(np.exp(r.normal(0.5, 1.5, x["k"].shape)))  # per key channel
+    x["beta"] = r.uniform(0.1, 1.9, x["eta"].shape)
+    return x, dout, dhT
+
+
+@pytest.mark.parametrize("form", ["beta", "kla"])
+def test_kda_gradients_match_finite_differences(form):
+    """Per-channel gate: gradients against central differences of the pinned
+    per-channel-gate forward, for beta given and for the KLA step size."""
+    x, dout, dhT = _kda_problem(37)
+    eps = 1e-6
+    step = "beta" if form == "beta" else "eta"
+    if form == "beta":
+        gr = oracle.kda_backward_beta(x["q"], x["k"], x["v"], x["gv"], x["beta"], x["h0"], dout,
+                                      dhT)
+    else:
+        gr = oracle.kda_backward(x["q"], x["k"], x["v"], x["gv"], x["eta"], eps, x["h0"], dout,
+                                 dhT)
+
+    def loss(y):
+        if form == "beta":
+            o, hT = oracle.kda(y["q"], y["k"], y["v"], y["gv"], y["beta"], y["h0"])
+        else:
+            o, hT = oracle.kda_forward(y["q"], y["k"], y["v"], y["gv"], y["eta"], eps, y["h0"])
+        return float((o * dout).sum() + (hT * dhT).sum())
+
+    r = np.random.Generator(np.random.PCG64(38))
+    names = dict(q="dq", k="dk", v="dv", gv="dg", h0="dh0")
+    names[step] = "dbeta" if form == "beta" else "deta"
+    for name, gname in names.items():
+        d = r.standard_normal(x[name].shape)
+        h = 1e-6
+        xp = dict(x); xp[name] = x[name] + h * d
+        xm = dict(x); xm[name] = x[name] - h * d
+        fd = (loss(xp) - loss(xm)) / (2 * h)
+        an = float((gr[gname] * d).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_kda_gradients_reduce_to_scalar_gate():
+    """A per-channel gate equal on every channel is the scalar gate: the
+    per-channel gradients equal the gated delta ones, and the channel sum of
+    dg is the scalar dg."""
+    x, dout, dhT = _kda_problem(39)
+    gv = np.repeat(x["g"][..., None], x["k"].shape[-1], axis=-1)
+    a = oracle.kda_backward_beta(x["q"], x["k"], x["v"], gv, x["beta"], x["h0"], dout, dhT)
+    b = oracle.gated_delta_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], dout,
+                                    dhT)
+    for n in ("dq", "dk", "dv", "dbeta", "dh0"):
+        np.testing.assert_allclose(a[n], b[n], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(a["dg"].sum(-1), b["dg"], rtol=1e-10, atol=1e-12)
