@@ -55,6 +55,13 @@ SIGNATURES = {
     "kla_gdn_recurrent_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _vp, _vp, _vp,
                                    _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_kda_recurrent_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "kla_kda_recurrent_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
+                                   _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_kda_recurrent_bwd_beta": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_check_device_error": (_i, [_vp]),
     "kla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "kla_status_string": (ctypes.c_char_p, [_i]),

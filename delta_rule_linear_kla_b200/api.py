@@ -157,7 +157,12 @@ def recurrent_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int) -> in
     return int(_native.lib().kla_recurrent_bwd_workspace_size(B, T, H, dk, dv))
 
 
-def _bwd(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0, workspace, stream):
+def kda_recurrent_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int) -> int:
+    return int(_native.lib().kla_kda_recurrent_bwd_workspace_size(B, T, H, dk, dv))
+
+
+def _bwd(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0, workspace, stream,
+         vector_gate=False):
     _need(q, "q")
     if q.dtype not in _DT:
         raise ValueError("q, k, v must be bfloat16 or float32")
@@ -165,17 +170,19 @@ def _bwd(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0, workspac
     dv = v.shape[-1]
     _need(k, "k", q.dtype, (B, T, H, dk))
     _need(v, "v", q.dtype, (B, T, H, dv))
-    _need(g, "g", torch.float32, (B, T, H))
+    gshape = (B, T, H, dk) if vector_gate else (B, T, H)
+    _need(g, "g", torch.float32, gshape)
     _need(step, "eta/beta", torch.float32, (B, T, H))
     _need(h0, "h0", torch.float32, (B, H, dk, dv))
     _need(grad_o, "grad_o", q.dtype, (B, T, H, dv))
     _need(grad_hT, "grad_hT", torch.float32, (B, H, dk, dv))
     f32 = dict(dtype=torch.float32, device=q.device)
     out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
-               dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty((B, T, H), **f32),
+               dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty(gshape, **f32),
                dstep=torch.empty((B, T, H), **f32),
                dh0=torch.empty((B, H, dk, dv), **f32) if need_h0 else None)
-    need = recurrent_bwd_workspace_size(B, T, H, dk, dv)
+    need = (kda_recurrent_bwd_workspace_size if vector_gate
+            else recurrent_bwd_workspace_size)(B, T, H, dk, dv)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -197,6 +204,26 @@ def recurrent_bwd(q, k, v, g, eta, grad_o, eps: float = 1e-6, h0=None, grad_hT=N
     out = _bwd(_native.lib().kla_recurrent_bwd, "kla_recurrent_bwd", q, k, v, g, eta, eps, h0,
                grad_o, grad_hT, need_h0, workspace, stream)
     out["deta"] = out.pop("dstep")
+    return out
+
+
+def kda_recurrent_bwd(q, k, v, g, eta, grad_o, eps: float = 1e-6, h0=None, grad_hT=None, *,
+                      need_h0: bool = True, workspace=None, stream=None):
+    """Gradients of the per-channel-gate prefill (g [B,T,H,dk]), KLA step
+    size (kla_kda_recurrent_bwd): dq, dk, dv, dg [B,T,H,dk], deta, dh0."""
+    out = _bwd(_native.lib().kla_kda_recurrent_bwd, "kla_kda_recurrent_bwd", q, k, v, g, eta,
+               eps, h0, grad_o, grad_hT, need_h0, workspace, stream, vector_gate=True)
+    out["deta"] = out.pop("dstep")
+    return out
+
+
+def kda_recurrent_bwd_beta(q, k, v, g, beta, grad_o, h0=None, grad_hT=None, *,
+                           need_h0: bool = True, workspace=None, stream=None):
+    """The same with beta given per token (kla_kda_recurrent_bwd_beta):
+    dq, dk, dv, dg, dbeta, dh0."""
+    out = _bwd(_native.lib().kla_kda_recurrent_bwd_beta, "kla_kda_recurrent_bwd_beta", q, k, v,
+               g, beta, None, h0, grad_o, grad_hT, need_h0, workspace, stream, vector_gate=True)
+    out["dbeta"] = out.pop("dstep")
     return out
 
 

@@ -339,13 +339,14 @@ kla_status kla_kda_fwd_beta(const void* q, const void* k, const void* v, const f
 }  // extern "C"
 
 // Gradients of the prefill (token-serial backward), KLA step size or
-// (eps == kBetaGiven) beta given.
+// (eps == kBetaGiven) beta given; per-channel gate (g, grad_g [B][T][H][dk])
+// when vector_gate.
 static kla_status bwd_impl(const void* q, const void* k, const void* v, const float* g,
                            const float* eta, float eps, const float* h0, const void* grad_o,
                            const float* grad_hT, float* grad_q, float* grad_k, float* grad_v,
                            float* grad_g, float* grad_eta, float* grad_h0, int B, int T, int H,
                            int dk, int dv, int dtype, void* workspace, size_t ws_bytes,
-                           void* stream) {
+                           void* stream, bool vector_gate = false) {
   if (B < 1 || H < 1 || T < 0) return KLA_ERR_INVALID_ARG;
   if (dtype != KLA_BF16 && dtype != KLA_FP32) return KLA_ERR_INVALID_ARG;
   if (!(eps >= 0.0f) && eps != kBetaGiven) return KLA_ERR_INVALID_ARG;
@@ -360,16 +361,17 @@ static kla_status bwd_impl(const void* q, const void* k, const void* v, const fl
   if (!head_dims_ok(dk, dv)) return KLA_ERR_UNSUPPORTED;
   const size_t es = dtype == KLA_BF16 ? 2 : 4;
   const size_t ntok = (size_t)B * T * H, sb = (size_t)B * H * dk * dv * 4;
-  const size_t need = recurrent_bwd_workspace_bytes(B, T, H, dk, dv);
+  const size_t gdim = vector_gate ? dk : 1;
+  const size_t need = recurrent_bwd_workspace_bytes(B, T, H, dk, dv, vector_gate);
   if (T > 0 && (!workspace || ws_bytes < need)) return KLA_ERR_INVALID_ARG;
   // every written range (gradients, workspace) is disjoint from every input
   // and from the other written ranges
   const Range ins[] = {rng(q, ntok * dk * es),         rng(k, ntok * dk * es),
-                       rng(v, ntok * dv * es),         rng(g, ntok * 4),
+                       rng(v, ntok * dv * es),         rng(g, ntok * gdim * 4),
                        rng(eta, ntok * 4),             rng(h0, h0 ? sb : 0),
                        rng(grad_o, ntok * dv * es),    rng(grad_hT, grad_hT ? sb : 0)};
   const Range outs[] = {rng(grad_q, ntok * dk * 4), rng(grad_k, ntok * dk * 4),
-                        rng(grad_v, ntok * dv * 4), rng(grad_g, ntok * 4),
+                        rng(grad_v, ntok * dv * 4), rng(grad_g, ntok * gdim * 4),
                         rng(grad_eta, ntok * 4),    rng(grad_h0, grad_h0 ? sb : 0),
                         rng(workspace, T > 0 ? need : 0)};
   for (size_t a = 0; a < sizeof(outs) / sizeof(outs[0]); ++a) {
@@ -385,9 +387,9 @@ static kla_status bwd_impl(const void* q, const void* k, const void* v, const fl
                             : cudaMemsetAsync(grad_h0, 0, sb, st);
     return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
   }
-  cudaError_t e = launch_recurrent_bwd(q, k, v, g, eta, eps, h0, grad_o, grad_hT, grad_q, grad_k,
-                                       grad_v, grad_g, grad_eta, grad_h0, B, T, H, dk, dv, dtype,
-                                       workspace, st);
+  cudaError_t e = launch_recurrent_bwd(q, k, v, g, vector_gate, eta, eps, h0, grad_o, grad_hT,
+                                       grad_q, grad_k, grad_v, grad_g, grad_eta, grad_h0, B, T, H,
+                                       dk, dv, dtype, workspace, st);
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
 
@@ -395,7 +397,35 @@ extern "C" {
 
 size_t kla_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
   if (!head_dims_ok(dk, dv)) return 0;
-  return recurrent_bwd_workspace_bytes(B, T, H, dk, dv);
+  return recurrent_bwd_workspace_bytes(B, T, H, dk, dv, false);
+}
+
+size_t kla_kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
+  if (!head_dims_ok(dk, dv)) return 0;
+  return recurrent_bwd_workspace_bytes(B, T, H, dk, dv, true);
+}
+
+kla_status kla_kda_recurrent_bwd(const void* q, const void* k, const void* v, const float* g,
+                                 const float* eta, float eps, const float* h0,
+                                 const void* grad_o, const float* grad_hT, float* grad_q,
+                                 float* grad_k, float* grad_v, float* grad_g, float* grad_eta,
+                                 float* grad_h0, int B, int T, int H, int dk, int dv, int dtype,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, g, eta, eps, h0, grad_o, grad_hT, grad_q, grad_k, grad_v, grad_g,
+                  grad_eta, grad_h0, B, T, H, dk, dv, dtype, workspace, ws_bytes, stream, true);
+}
+
+kla_status kla_kda_recurrent_bwd_beta(const void* q, const void* k, const void* v,
+                                      const float* g, const float* beta, const float* h0,
+                                      const void* grad_o, const float* grad_hT, float* grad_q,
+                                      float* grad_k, float* grad_v, float* grad_g,
+                                      float* grad_beta, float* grad_h0, int B, int T, int H,
+                                      int dk, int dv, int dtype, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+  return bwd_impl(q, k, v, g, beta, kBetaGiven, h0, grad_o, grad_hT, grad_q, grad_k, grad_v,
+                  grad_g, grad_beta, grad_h0, B, T, H, dk, dv, dtype, workspace, ws_bytes,
+                  stream, true);
 }
 
 kla_status kla_recurrent_bwd(const void* q, const void* k, const void* v, const float* g,

@@ -40,13 +40,14 @@ cudaError_t launch_recurrent(const void* q, const void* k, const void* v,
                              int H, int dk, int dv, int dtype, cudaStream_t st);
 
 // Token-serial backward (kla_backward.cu): gradients of q, k, v (fp32), of
-// the log-gate, of eta (or of beta when eps == kBetaGiven) and of h0.
-size_t recurrent_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+// the log-gate(s), of eta (or of beta when eps == kBetaGiven) and of h0.
+size_t recurrent_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, bool vector_gate);
 cudaError_t launch_recurrent_bwd(const void* q, const void* k, const void* v, const float* g,
-                                 const float* eta, float eps, const float* h0,
-                                 const void* dout, const float* dhT, float* dq, float* dk,
-                                 float* dv, float* dg, float* deta, float* dh0, int B, int T,
-                                 int H, int dkd, int dvd, int dtype, void* ws, cudaStream_t st);
+                                 bool vector_gate, const float* eta, float eps,
+                                 const float* h0, const void* dout, const float* dhT,
+                                 float* dq, float* dk, float* dv, float* dg, float* deta,
+                                 float* dh0, int B, int T, int H, int dkd, int dvd, int dtype,
+                                 void* ws, cudaStream_t st);
 
 template <typename T> struct IO;
 

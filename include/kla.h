@@ -290,6 +290,36 @@ KLA_API kla_status kla_recurrent_bwd(const void *q, const void *k, const void *v
                                      float *grad_h0, int B, int T, int H, int dk, int dv,
                                      int dtype, void *workspace, size_t ws_bytes,
                                      void *stream);
+/*
+ * The same backward for the per-channel-gate form (kla_kda_fwd; "Deep Dive
+ * into KDA", section 2.3): g and grad_g are [B][T][H][dk] (one log-gate per
+ * key channel), the forward being hd = Diag(e^{g_t}) h_{t-1}; r = hd^T k;
+ * u = beta (v - r); h_t = hd + k u^T.  Reverse per token: dH += q do^T;
+ * dq = h_t do; du = dH^T k; dr = -beta du; dv = beta du;
+ * dbeta = du . (v - r); dk = dH u + hd dr; Hd = dH + k dr^T;
+ * dg_i = sum_j Hd_ij hd_ij; dH <- Diag(e^{g_t}) Hd; then the step size's
+ * chain rule as above (the _beta form returns dbeta).  Workspace:
+ * kla_kda_recurrent_bwd_workspace_size(...) bytes (about (dv/32)*dk*4 more
+ * per head-token than the scalar gate's).  Everything else as
+ * kla_recurrent_bwd.
+ */
+KLA_API size_t kla_kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv);
+KLA_API kla_status kla_kda_recurrent_bwd(const void *q, const void *k, const void *v,
+                                         const float *g, const float *eta, float eps,
+                                         const float *h0, const void *grad_o,
+                                         const float *grad_hT, float *grad_q, float *grad_k,
+                                         float *grad_v, float *grad_g, float *grad_eta,
+                                         float *grad_h0, int B, int T, int H, int dk, int dv,
+                                         int dtype, void *workspace, size_t ws_bytes,
+                                         void *stream);
+KLA_API kla_status kla_kda_recurrent_bwd_beta(const void *q, const void *k, const void *v,
+                                              const float *g, const float *beta,
+                                              const float *h0, const void *grad_o,
+                                              const float *grad_hT, float *grad_q,
+                                              float *grad_k, float *grad_v, float *grad_g,
+                                              float *grad_beta, float *grad_h0, int B, int T,
+                                              int H, int dk, int dv, int dtype,
+                                              void *workspace, size_t ws_bytes, void *stream);
 KLA_API kla_status kla_gdn_recurrent_bwd(const void *q, const void *k, const void *v,
                                          const float *g, const float *beta,
                                          const float *h0, const void *grad_o,

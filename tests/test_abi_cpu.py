@@ -236,3 +236,17 @@ def test_backward_rejects_bad_arguments(lib):
     assert lib.kla_gdn_recurrent_bwd(A, 2 * A, 3 * A, 4 * A, 5 * A, None, 6 * A, None, 7 * A,
                                      7 * A, 9 * A, 10 * A, 11 * A, None, 1, 128, 2, 128, 128,
                                      0, 64 * A, need, None) == INVALID
+
+
+def test_kda_backward_rejects_bad_arguments(lib):
+    need = lib.kla_kda_recurrent_bwd_workspace_size(1, 128, 2, 128, 128)
+    assert need > lib.kla_recurrent_bwd_workspace_size(1, 128, 2, 128, 128)
+    args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, None, 6 * A, None, 7 * A, 8 * A, 9 * A,
+            10 * A, 11 * A, None, 1, 128, 2, 128, 128, 0, 64 * A, need, None]
+    bad = list(args); bad[22] = need - 1
+    assert lib.kla_kda_recurrent_bwd(*bad) == INVALID
+    bad = list(args); bad[12] = 4 * A + 64  # grad_g ([B,T,H,dk] fp32) over g
+    assert lib.kla_kda_recurrent_bwd(*bad) == INVALID
+    beta_args = args[:5] + args[6:]
+    bad = list(beta_args); bad[17] = 96; bad[18] = 96
+    assert lib.kla_kda_recurrent_bwd_beta(*bad) == UNSUPPORTED

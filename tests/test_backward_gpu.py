@@ -123,3 +123,59 @@ def test_backward_full_size_sampled_heads():
         got = {n: sl(out[n].cpu()) for n in ("dq", "dk", "dv", "dg", "deta")}
         got["dh0"] = out["dh0"][b:b + 1, h:h + 1].cpu()
         _check(got, ref)
+
+
+@pytest.mark.parametrize("name,B,T,H,dt,with_h0,strong", [
+    ("prefill_4k", 1, 200, 2, "bf16", False, False),
+    ("tiny", 2, 130, 2, "fp32", True, False),
+    ("prefill_4k", 1, 65, 2, "bf16", True, True),   # some channels wiped (g = -60)
+    ("stress", 1, 100, 2, "bf16", True, False),
+])
+def test_kda_backward(name, B, T, H, dt, with_h0, strong):
+    """Per-channel gate, KLA step size: against the oracle's per-channel-gate
+    gradients (pinned by finite differences and by the equal-channel
+    reduction to the scalar gate)."""
+    w = inputs.WORKLOADS[name].scaled(B=B, T=T, H=H, dtype=dt)
+    x = inputs.make_prefill(w, with_h0=with_h0)
+    gv = inputs.channel_gates((B, T, H, w.dk), 83)
+    if strong:
+        gv[:, ::7, :, ::5] = -60.0
+    do, dhT = _upstream(w, 84)
+    xc = cuda(x)
+    out = api.kda_recurrent_bwd(xc["q"], xc["k"], xc["v"], cuda(gv), xc["eta"], cuda(do),
+                                x["eps"], xc["h0"], cuda(dhT))
+    api.check_device_error()
+    ref = oracle.kda_backward(x["q"], x["k"], x["v"], gv, x["eta"], x["eps"], x["h0"], do, dhT)
+    _check(out, ref)
+
+
+def test_kda_backward_beta():
+    w = inputs.WORKLOADS["prefill_4k"].scaled(B=2, T=140, H=2, dk=64, dv=64)
+    x = inputs.make_prefill(w, with_h0=True)
+    kf = x["k"].float()
+    k = (kf / kf.norm(dim=-1, keepdim=True)).to(x["k"].dtype)
+    gv = inputs.channel_gates((2, 140, 2, 64), 85)
+    rng = np.random.Generator(np.random.PCG64(86))
+    beta = torch.from_numpy(rng.uniform(0.05, 1.95, x["g"].shape).astype(np.float32))
+    do, dhT = _upstream(w, 87)
+    xc = cuda(x)
+    out = api.kda_recurrent_bwd_beta(xc["q"], cuda(k), xc["v"], cuda(gv), cuda(beta), cuda(do),
+                                     xc["h0"], cuda(dhT))
+    ref = oracle.kda_backward_beta(x["q"], k, x["v"], gv, beta, x["h0"], do, dhT)
+    _check(out, ref, names=("dq", "dk", "dv", "dg", "dbeta", "dh0"))
+
+
+def test_kda_backward_equal_channels_is_scalar_gate():
+    """The same per-token gate on every channel: the per-channel kernels give
+    the scalar-gate gradients (dg summed over channels)."""
+    w = inputs.WORKLOADS["prefill_4k"].scaled(B=1, T=150, H=2)
+    x = cuda(inputs.make_prefill(w))
+    do, _ = _upstream(w, 88, False)
+    do = cuda(do)
+    gv = x["g"][..., None].expand(-1, -1, -1, w.dk).contiguous()
+    a = api.kda_recurrent_bwd(x["q"], x["k"], x["v"], gv, x["eta"], do, x["eps"])
+    b = api.recurrent_bwd(x["q"], x["k"], x["v"], x["g"], x["eta"], do, x["eps"])
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "deta", "dh0"):
+        assert rel(a[n].cpu(), b[n].cpu()) < 1e-5, n
+    assert rel(a["dg"].sum(-1).cpu(), b["dg"].cpu()) < 1e-5
