@@ -9,7 +9,8 @@ from .api import (KLAError, check_device_error, chunk_fwd, chunk_fwd_host,  # no
                   chunk_ut_transform, decode_step, gdn_chunk_fwd, gdn_decode_step,
                   kda_chunk_fwd, kda_chunk_fwd_beta, kda_decode_step, kda_decode_step_beta,
                   kda_fwd, kda_fwd_beta, kda_recurrent_bwd, kda_recurrent_bwd_beta,
-                  kda_recurrent_bwd_workspace_size, gdn_recurrent_bwd,
+                  kda_recurrent_bwd_workspace_size, gdn_recurrent_bwd, chunk_bwd,
+                  gdn_chunk_bwd, chunk_bwd_workspace_size,
                   recurrent_bwd, recurrent_bwd_workspace_size, recurrent_fwd)
 
 __all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_ut_transform", "chunk_state_fwd", "recurrent_fwd",
@@ -18,4 +19,5 @@ __all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_ut_transform", "chunk_state_fwd
            "kda_decode_step",
            "kda_decode_step_beta", "recurrent_bwd", "gdn_recurrent_bwd",
            "recurrent_bwd_workspace_size", "kda_recurrent_bwd", "kda_recurrent_bwd_beta",
-           "kda_recurrent_bwd_workspace_size", "check_device_error", "KLAError"]
+           "kda_recurrent_bwd_workspace_size", "chunk_bwd", "gdn_chunk_bwd",
+           "chunk_bwd_workspace_size", "check_device_error", "KLAError"]

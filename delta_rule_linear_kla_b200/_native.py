@@ -62,6 +62,13 @@ SIGNATURES = {
     "kla_kda_recurrent_bwd_beta": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                         _vp, _vp, _vp, _vp, _vp, _vp,
                                         _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_chunk_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "kla_chunk_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
+                           _vp, _vp, _vp, _vp, _vp, _vp,
+                           _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_gdn_chunk_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                               _vp, _vp, _vp, _vp, _vp, _vp,
+                               _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_check_device_error": (_i, [_vp]),
     "kla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "kla_status_string": (ctypes.c_char_p, [_i]),

@@ -161,8 +161,13 @@ def kda_recurrent_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int) -
     return int(_native.lib().kla_kda_recurrent_bwd_workspace_size(B, T, H, dk, dv))
 
 
+def chunk_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
+                             dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(_native.lib().kla_chunk_bwd_workspace_size(B, T, H, dk, dv, _DT[dtype]))
+
+
 def _bwd(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0, workspace, stream,
-         vector_gate=False):
+         vector_gate=False, chunked=False):
     _need(q, "q")
     if q.dtype not in _DT:
         raise ValueError("q, k, v must be bfloat16 or float32")
@@ -181,8 +186,11 @@ def _bwd(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0, workspac
                dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty(gshape, **f32),
                dstep=torch.empty((B, T, H), **f32),
                dh0=torch.empty((B, H, dk, dv), **f32) if need_h0 else None)
-    need = (kda_recurrent_bwd_workspace_size if vector_gate
-            else recurrent_bwd_workspace_size)(B, T, H, dk, dv)
+    if chunked:
+        need = chunk_bwd_workspace_size(B, T, H, dk, dv, q.dtype)
+    else:
+        need = (kda_recurrent_bwd_workspace_size if vector_gate
+                else recurrent_bwd_workspace_size)(B, T, H, dk, dv)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -204,6 +212,26 @@ def recurrent_bwd(q, k, v, g, eta, grad_o, eps: float = 1e-6, h0=None, grad_hT=N
     out = _bwd(_native.lib().kla_recurrent_bwd, "kla_recurrent_bwd", q, k, v, g, eta, eps, h0,
                grad_o, grad_hT, need_h0, workspace, stream)
     out["deta"] = out.pop("dstep")
+    return out
+
+
+def chunk_bwd(q, k, v, g, eta, grad_o, eps: float = 1e-6, h0=None, grad_hT=None, *,
+              need_h0: bool = True, workspace=None, stream=None):
+    """Gradients of the KLA prefill from the chunk form (kla_chunk_bwd):
+    dq, dk, dv, dg, deta, dh0 (fp32).  bf16 with d = 128 runs the chunkwise
+    tensor-core kernels, everything else the token-serial ones."""
+    out = _bwd(_native.lib().kla_chunk_bwd, "kla_chunk_bwd", q, k, v, g, eta, eps, h0, grad_o,
+               grad_hT, need_h0, workspace, stream, chunked=True)
+    out["deta"] = out.pop("dstep")
+    return out
+
+
+def gdn_chunk_bwd(q, k, v, g, beta, grad_o, h0=None, grad_hT=None, *, need_h0: bool = True,
+                  workspace=None, stream=None):
+    """The same with beta given per token (kla_gdn_chunk_bwd)."""
+    out = _bwd(_native.lib().kla_gdn_chunk_bwd, "kla_gdn_chunk_bwd", q, k, v, g, beta, None, h0,
+               grad_o, grad_hT, need_h0, workspace, stream, chunked=True)
+    out["dbeta"] = out.pop("dstep")
     return out
 
 

@@ -346,7 +346,7 @@ static kla_status bwd_impl(const void* q, const void* k, const void* v, const fl
                            const float* grad_hT, float* grad_q, float* grad_k, float* grad_v,
                            float* grad_g, float* grad_eta, float* grad_h0, int B, int T, int H,
                            int dk, int dv, int dtype, void* workspace, size_t ws_bytes,
-                           void* stream, bool vector_gate = false) {
+                           void* stream, bool vector_gate = false, bool chunked = false) {
   if (B < 1 || H < 1 || T < 0) return KLA_ERR_INVALID_ARG;
   if (dtype != KLA_BF16 && dtype != KLA_FP32) return KLA_ERR_INVALID_ARG;
   if (!(eps >= 0.0f) && eps != kBetaGiven) return KLA_ERR_INVALID_ARG;
@@ -362,7 +362,11 @@ static kla_status bwd_impl(const void* q, const void* k, const void* v, const fl
   const size_t es = dtype == KLA_BF16 ? 2 : 4;
   const size_t ntok = (size_t)B * T * H, sb = (size_t)B * H * dk * dv * 4;
   const size_t gdim = vector_gate ? dk : 1;
-  const size_t need = recurrent_bwd_workspace_bytes(B, T, H, dk, dv, vector_gate);
+  // the chunkwise kernels cover bf16 with d = 128 and the scalar gate; the
+  // rest runs the token-serial kernels
+  const bool use_chunks = chunked && !vector_gate && dtype == KLA_BF16 && dk == 128 && dv == 128;
+  const size_t need = use_chunks ? chunk_bwd_workspace_bytes(B, T, H, dk, dv)
+                                 : recurrent_bwd_workspace_bytes(B, T, H, dk, dv, vector_gate);
   if (T > 0 && (!workspace || ws_bytes < need)) return KLA_ERR_INVALID_ARG;
   // every written range (gradients, workspace) is disjoint from every input
   // and from the other written ranges
@@ -387,9 +391,13 @@ static kla_status bwd_impl(const void* q, const void* k, const void* v, const fl
                             : cudaMemsetAsync(grad_h0, 0, sb, st);
     return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
   }
-  cudaError_t e = launch_recurrent_bwd(q, k, v, g, vector_gate, eta, eps, h0, grad_o, grad_hT,
-                                       grad_q, grad_k, grad_v, grad_g, grad_eta, grad_h0, B, T, H,
-                                       dk, dv, dtype, workspace, st);
+  cudaError_t e =
+      use_chunks
+          ? launch_chunk_bwd(q, k, v, g, eta, eps, h0, grad_o, grad_hT, grad_q, grad_k, grad_v,
+                             grad_g, grad_eta, grad_h0, B, T, H, dk, dv, workspace, st)
+          : launch_recurrent_bwd(q, k, v, g, vector_gate, eta, eps, h0, grad_o, grad_hT, grad_q,
+                                 grad_k, grad_v, grad_g, grad_eta, grad_h0, B, T, H, dk, dv,
+                                 dtype, workspace, st);
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
 
@@ -398,6 +406,35 @@ extern "C" {
 size_t kla_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
   if (!head_dims_ok(dk, dv)) return 0;
   return recurrent_bwd_workspace_bytes(B, T, H, dk, dv, false);
+}
+
+size_t kla_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int dtype) {
+  if (!head_dims_ok(dk, dv)) return 0;
+  if (dtype == KLA_BF16 && dk == 128 && dv == 128) return chunk_bwd_workspace_bytes(B, T, H, dk, dv);
+  return recurrent_bwd_workspace_bytes(B, T, H, dk, dv, false);
+}
+
+kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                         const float* eta, float eps, const float* h0, const void* grad_o,
+                         const float* grad_hT, float* grad_q, float* grad_k, float* grad_v,
+                         float* grad_g, float* grad_eta, float* grad_h0, int B, int T, int H,
+                         int dk, int dv, int dtype, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, g, eta, eps, h0, grad_o, grad_hT, grad_q, grad_k, grad_v, grad_g,
+                  grad_eta, grad_h0, B, T, H, dk, dv, dtype, workspace, ws_bytes, stream, false,
+                  true);
+}
+
+kla_status kla_gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, const float* h0, const void* grad_o,
+                             const float* grad_hT, float* grad_q, float* grad_k, float* grad_v,
+                             float* grad_g, float* grad_beta, float* grad_h0, int B, int T,
+                             int H, int dk, int dv, int dtype, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  return bwd_impl(q, k, v, g, beta, kBetaGiven, h0, grad_o, grad_hT, grad_q, grad_k, grad_v,
+                  grad_g, grad_beta, grad_h0, B, T, H, dk, dv, dtype, workspace, ws_bytes,
+                  stream, false, true);
 }
 
 size_t kla_kda_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv) {

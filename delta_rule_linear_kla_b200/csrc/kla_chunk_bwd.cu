@@ -1,0 +1,864 @@
+// Chunkwise backward of the KLA / gated delta rule prefill (bf16 I/O,
+// scalar gate): the gradients of a loss L given dL/do and dL/dh_T, from the
+// chunk form of the forward ("Deep Dive into KDA", section 3, with the KLA
+// step size of "Kaczmarz Linear Attention", Abstract).  Per chunk n of C = 64
+// tokens with start state h_n (G = in-chunk cumsum of g, gamma = e^G,
+// gamma_C = e^{G_last}, Gamma_rs = e^{G_r - G_s}):
+//   A = strict_lower(diag(beta) K K^T (*) Gamma),  T = (I + A)^{-1}
+//   W = T diag(beta gamma) K,  U = T diag(beta) V,  V' = U - W h_n
+//   P = lower_incl(Q K^T (*) Gamma),  O = diag(gamma) Q h_n + P V'
+//   h_{n+1} = gamma_C h_n + Kt^T V',  Kt = diag(gamma_C / gamma) K.
+// The pages print no backward.  Its adjoint, derived here, splits into one
+// reverse chain over the chunks and independent per-chunk work:
+//   dV'_n = P^T dO + Kt dH_{n+1}
+//   dH_n  = gamma_C dH_{n+1} + (diag(gamma) Q)^T dO - W^T dV'_n      (chain)
+//   dP = dO V'^T (*) incl;  dQ = diag(gamma) dO h_n^T + (dP (*) Gamma) K
+//   dW = -dV' h_n^T;  dT = dW (diag(beta gamma) K)^T + dV' (diag(beta) V)^T
+//   dA = -strict_lower(T^T dT T^T);  E = dA (*) Gamma
+//   dV = diag(beta) T^T dV'
+//   dK = (dP (*) Gamma)^T Q + diag(gamma_C / gamma) V' dH_{n+1}^T
+//        + diag(beta gamma) T^T dW + diag(beta) E K + (diag(beta) E)^T K
+//   dbeta = gamma (*) rowdot(T^T dW, K) + rowdot(T^T dV', V) + rowsum(E (*) K K^T)
+//   dG = rowsum(F) - colsum(F) for F = dA (*) A and F = dP (*) P,
+//        + rowdot(dO, diag(gamma) Q h_n) + beta gamma rowdot(T^T dW, K)
+//        - rowdot(dKt, Kt);  dG_last += sum rowdot(dKt, Kt) + gamma_C <dH_{n+1}, h_n>
+//   dg = reverse in-chunk cumsum of dG;  KLA: deta = dbeta / (||k||^2 + eps),
+//   dk += -2 dbeta eta k / (||k||^2 + eps)^2.
+//
+// Kernels (after the checkpoint kernel of kla_backward.cu, which leaves every
+// h_n in fp32 and each token's beta and alpha):
+//   cbwd_prep_kernel     per chunk: T and V' into the workspace (fp32)
+//   cbwd_adjoint_kernel  per head and 64-column slab, chunks in reverse: the
+//                        chain above, dH in registers; writes dV'_n and dH_{n+1}
+//   cbwd_grad_kernel     per chunk: every gradient of the chunk's tokens
+// Products are warp-level tensor-core MMAs (mma.sync m16n8k8, tf32 operands,
+// fp32 sums); operands are read from shared memory through small accessors,
+// so transposed or row-scaled operands need no extra copies.  Ragged tails
+// are zero rows with g = 0 and beta = 0 (identity steps).
+#include "kla_common.cuh"
+
+namespace kla {
+namespace cbwd {
+
+constexpr int C = 64;
+constexpr int NT = 256;
+constexpr int BVA = 64;  // state columns per adjoint-chain CTA
+
+__device__ __forceinline__ uint32_t tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// d[nt] (16 x 8 tiles at rows m0.., columns n0 + 8 nt ..) += A (16 x K) B (K x 8):
+// A(m, k) and B(k, n) are callables returning fp32.  Fragment element e of a
+// tile: row m0 + g + 8 (e >> 1), column n0 + 8 nt + 2 t + (e & 1), with
+// g = lane / 4, t = lane % 4.
+template <int NTL, class FA, class FB>
+__device__ __forceinline__ void mma_rows(float (&d)[NTL][4], const FA& A, const FB& B, int m0,
+                                         int n0, int K, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll 2
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    const uint32_t a0 = tf32(A(m0 + g, k0 + t)), a1 = tf32(A(m0 + g + 8, k0 + t));
+    const uint32_t a2 = tf32(A(m0 + g, k0 + t + 4)), a3 = tf32(A(m0 + g + 8, k0 + t + 4));
+#pragma unroll
+    for (int nt = 0; nt < NTL; ++nt) {
+      const uint32_t b0 = tf32(B(k0 + t, n0 + 8 * nt + g));
+      const uint32_t b1 = tf32(B(k0 + t + 4, n0 + 8 * nt + g));
+      asm volatile(
+          "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+          "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+          : "+f"(d[nt][0]), "+f"(d[nt][1]), "+f"(d[nt][2]), "+f"(d[nt][3])
+          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+  }
+}
+
+template <int NTL>
+__device__ __forceinline__ void zero(float (&d)[NTL][4]) {
+#pragma unroll
+  for (int i = 0; i < NTL; ++i) d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.f;
+}
+
+// Row / column of fragment element e.
+__device__ __forceinline__ int frow(int m0, int lane, int e) { return m0 + (lane >> 2) + 8 * (e >> 1); }
+__device__ __forceinline__ int fcol(int n0, int nt, int lane, int e) {
+  return n0 + 8 * nt + 2 * (lane & 3) + (e & 1);
+}
+
+__device__ __forceinline__ float bf(const __nv_bfloat16& x) { return __bfloat162float(x); }
+
+// Strides (elements) of the shared-memory tiles: fp32 rows padded by 4, bf16
+// rows by 8, against bank conflicts of the fragment reads.
+template <int D> constexpr int LF() { return D + 4; }
+template <int D> constexpr int LB() { return D + 8; }
+
+// Copy n rows of a [rows][D] bf16 matrix with row stride rs (elements) into
+// a padded tile (rows >= n zero-filled up to C).
+template <int D>
+__device__ __forceinline__ void load_rows_bf16(__nv_bfloat16* dst, const __nv_bfloat16* src,
+                                               size_t rs, int n) {
+  constexpr int PR = D / 8;  // 16-byte pieces per row
+  for (int p = threadIdx.x; p < C * PR; p += NT) {
+    const int r = p / PR, ch = p % PR;
+    uint4 x = make_uint4(0, 0, 0, 0);
+    if (r < n) x = *reinterpret_cast<const uint4*>(src + r * rs + ch * 8);
+    *reinterpret_cast<uint4*>(dst + r * LB<D>() + ch * 8) = x;
+  }
+}
+
+// Copy a [R][D] fp32 block (row stride rs) into a padded tile.
+template <int R, int D>
+__device__ __forceinline__ void load_f32(float* dst, const float* src, size_t rs) {
+  constexpr int PR = D / 4;
+  for (int p = threadIdx.x; p < R * PR; p += NT) {
+    const int r = p / PR, ch = p % PR;
+    *reinterpret_cast<float4*>(dst + r * LF<D>() + ch * 4) =
+        *reinterpret_cast<const float4*>(src + r * rs + ch * 4);
+  }
+}
+
+// Per-chunk scalars: G (in-chunk cumsum of g), gamma = e^G, beta, ||k||^2,
+// from the staged keys (rows >= n: g = 0, beta = 0).  Decay ratios are only
+// ever formed as e^{difference} (gamma_C / gamma_r as e^{G_last - G_r}): with
+// strong gates e^G itself underflows to 0 inside a chunk.
+template <int DK>
+__device__ __forceinline__ void chunk_scalars(float* G, float* gam, float* beta, float* n2,
+                                              const __nv_bfloat16* kb, const float* g,
+                                              const float* eta, float eps, size_t tok0,
+                                              size_t tstride, int n) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int r = warp; r < C; r += NT / 32) {
+    float a = 0.f;
+    for (int i = lane; i < DK; i += 32) {
+      const float x = bf(kb[r * LB<DK>() + i]);
+      a = fmaf(x, x, a);
+    }
+    a = warp_sum(a);
+    if (lane == 0) {
+      n2[r] = a;
+      beta[r] = r < n ? step_size(eta[tok0 + r * tstride], a, eps) : 0.f;
+    }
+  }
+  if (warp == 0) {  // inclusive cumsum of the 64 gates: two per lane
+    float x0 = 2 * lane < n ? g[tok0 + (2 * lane) * tstride] : 0.f;
+    float x1 = 2 * lane + 1 < n ? g[tok0 + (2 * lane + 1) * tstride] : 0.f;
+    float s = x0 + x1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    const float base = s - (x0 + x1);
+    G[2 * lane] = base + x0;
+    G[2 * lane + 1] = s;
+    gam[2 * lane] = __expf(base + x0);
+    gam[2 * lane + 1] = __expf(s);
+  }
+}
+
+// T = (I + A)^{-1} for the strictly lower A (fp32 [C][LF<C>]) by forward
+// substitution, four threads per column (column tid / 4); writes Tm.
+__device__ __forceinline__ void unit_lower_inverse(float* Tm, const float* A) {
+  const int c = threadIdx.x >> 2, l = threadIdx.x & 3;
+  float tc[C / 4];  // T[4 j + l][c]
+#pragma unroll
+  for (int j = 0; j < C / 4; ++j) tc[j] = 0.f;
+#pragma unroll
+  for (int r = 0; r < C; ++r) {
+    float p = 0.f;
+#pragma unroll
+    for (int j = 0; j < C / 4; ++j) p = fmaf(A[r * LF<C>() + 4 * j + l], tc[j], p);
+    p += __shfl_xor_sync(0xffffffffu, p, 1);
+    p += __shfl_xor_sync(0xffffffffu, p, 2);
+    const float val = r < c ? 0.f : (r == c ? 1.f : -p);
+    if (l == (r & 3)) tc[r >> 2] = val;
+  }
+#pragma unroll
+  for (int j = 0; j < C / 4; ++j) Tm[(4 * j + l) * LF<C>() + c] = tc[j];
+}
+
+}  // namespace cbwd
+
+using namespace cbwd;
+
+// ---------------------------------------------------------------- prep
+template <int DK, int DV>
+struct PrepSmem {
+  __nv_bfloat16 kb[C][LB<DK>()];
+  __nv_bfloat16 vb[C][LB<DV>()];
+  float A[C][LF<C>()];
+  float Tm[C][LF<C>()];
+  float W[C][LF<DK>()];
+  float h[DK][LF<DV>()];
+  float G[C], gam[C], beta[C], n2[C];
+};
+
+// Per chunk: T and V' = T diag(beta) V - W h_n into the workspace.
+template <int DK, int DV>
+__global__ void __launch_bounds__(NT)
+cbwd_prep_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                 const float* __restrict__ g, const float* __restrict__ eta, float eps,
+                 const float* __restrict__ ck, float* __restrict__ Tws, float* __restrict__ Vws,
+                 int Tlen, int H, int nblk) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  auto& s = *reinterpret_cast<PrepSmem<DK, DV>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
+  const size_t head = (size_t)b * H + hh, chunk = head * nblk + n;
+  const int t0 = n * C, len = min(C, Tlen - t0);
+  const size_t tok0 = ((size_t)b * Tlen + t0) * H + hh;
+
+  load_rows_bf16<DK>(&s.kb[0][0], k + tok0 * DK, (size_t)H * DK, len);
+  load_rows_bf16<DV>(&s.vb[0][0], v + tok0 * DV, (size_t)H * DV, len);
+  load_f32<DK, DV>(&s.h[0][0], ck + chunk * DK * DV, DV);
+  __syncthreads();
+  chunk_scalars<DK>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
+  __syncthreads();
+
+  const int mt = warp & 3, nh = warp >> 2;  // m-tile of 16 rows; column half
+  {  // A = beta_r (k_r . k_s) Gamma_rs, s < r
+    float d[4][4];
+    zero(d);
+    auto Ka = [&](int r, int i) { return bf(s.kb[r][i]); };
+    auto Kb = [&](int i, int c) { return bf(s.kb[c][i]); };
+    mma_rows<4>(d, Ka, Kb, 16 * mt, 32 * nh, DK, lane);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
+        s.A[r][c] = c < r ? s.beta[r] * d[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;
+      }
+  }
+  __syncthreads();
+  unit_lower_inverse(&s.Tm[0][0], &s.A[0][0]);
+  __syncthreads();
+  {  // W = T diag(beta gamma) K
+    float d[DK / 16][4];
+    zero(d);
+    auto Ta = [&](int r, int c) { return s.Tm[r][c]; };
+    auto Kb = [&](int c, int i) { return s.beta[c] * s.gam[c] * bf(s.kb[c][i]); };
+    mma_rows<DK / 16>(d, Ta, Kb, 16 * mt, (DK / 2) * nh, C, lane);
+#pragma unroll
+    for (int nt = 0; nt < DK / 16; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        s.W[frow(16 * mt, lane, e)][fcol((DK / 2) * nh, nt, lane, e)] = d[nt][e];
+  }
+  __syncthreads();
+  {  // V' = T diag(beta) V - W h_n
+    float d[DV / 16][4];
+    zero(d);
+    auto Ta = [&](int r, int c) { return s.Tm[r][c]; };
+    auto Vb = [&](int c, int j) { return s.beta[c] * bf(s.vb[c][j]); };
+    mma_rows<DV / 16>(d, Ta, Vb, 16 * mt, (DV / 2) * nh, C, lane);
+    auto Wa = [&](int r, int i) { return -s.W[r][i]; };
+    auto Hb = [&](int i, int j) { return s.h[i][j]; };
+    mma_rows<DV / 16>(d, Wa, Hb, 16 * mt, (DV / 2) * nh, DK, lane);
+    float* dst = Vws + chunk * C * DV;
+#pragma unroll
+    for (int nt = 0; nt < DV / 16; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; e += 2) {
+        const int r = frow(16 * mt, lane, e), j = fcol((DV / 2) * nh, nt, lane, e);
+        *reinterpret_cast<float2*>(dst + r * DV + j) = make_float2(d[nt][e], d[nt][e + 1]);
+      }
+  }
+  {
+    float* dst = Tws + chunk * C * C;
+    for (int p = tid; p < C * C; p += NT) dst[p] = s.Tm[p / C][p % C];
+  }
+}
+
+// ---------------------------------------------------------------- adjoint chain
+template <int DK>
+struct AdjSmem {
+  __nv_bfloat16 kb[C][LB<DK>()];
+  __nv_bfloat16 qb[C][LB<DK>()];
+  __nv_bfloat16 ob[C][LB<BVA>()];
+  float Tm[C][LF<C>()];
+  float W[C][LF<DK>()];
+  float P[C][LF<C>()];
+  float dH[DK][LF<BVA>()];
+  float dV[C][LF<BVA>()];
+  float G[C], gam[C], beta[C], n2[C], kts[C];
+};
+
+// One CTA per (head, 64-column slab); chunks in reverse.  dH (the adjoint of
+// h_{n+1}) lives in registers: warp w holds rows 16 w .. 16 w + 15.
+template <int DK, int DV>
+__global__ void __launch_bounds__(NT)
+cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                    const __nv_bfloat16* __restrict__ dout, const float* __restrict__ g,
+                    const float* __restrict__ eta, float eps, const float* __restrict__ dhT,
+                    const float* __restrict__ Tws, float* __restrict__ dVws,
+                    float* __restrict__ dHws, float* __restrict__ dh0, int Tlen, int H,
+                    int nblk) {
+  static_assert(DK == 128, "one 16-row tile of the state per warp");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  auto& s = *reinterpret_cast<AdjSmem<DK>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int slab = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
+  const int j0 = slab * BVA;
+  const size_t head = (size_t)b * H + hh;
+
+  float acc[BVA / 8][4];  // dH rows 16 warp .., columns j0 ..
+#pragma unroll
+  for (int nt = 0; nt < BVA / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      acc[nt][e] = dhT ? dhT[(head * DK + frow(16 * warp, lane, e)) * DV + j0 +
+                             fcol(0, nt, lane, e)]
+                       : 0.f;
+
+  for (int n = nblk - 1; n >= 0; --n) {
+    const size_t chunk = head * nblk + n;
+    const int t0 = n * C, len = min(C, Tlen - t0);
+    const size_t tok0 = ((size_t)b * Tlen + t0) * H + hh;
+    __syncthreads();  // the previous chunk's tiles are no longer read
+    load_rows_bf16<DK>(&s.kb[0][0], k + tok0 * DK, (size_t)H * DK, len);
+    load_rows_bf16<DK>(&s.qb[0][0], q + tok0 * DK, (size_t)H * DK, len);
+    load_rows_bf16<BVA>(&s.ob[0][0], dout + tok0 * DV + j0, (size_t)H * DV, len);
+    load_f32<C, C>(&s.Tm[0][0], Tws + chunk * C * C, C);
+    // dH_{n+1}: to shared memory (operand) and to the workspace (for the
+    // gradient kernel)
+#pragma unroll
+    for (int nt = 0; nt < BVA / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; e += 2) {
+        const int r = frow(16 * warp, lane, e), c = fcol(0, nt, lane, e);
+        s.dH[r][c] = acc[nt][e];
+        s.dH[r][c + 1] = acc[nt][e + 1];
+        *reinterpret_cast<float2*>(dHws + (chunk * DK + r) * DV + j0 + c) =
+            make_float2(acc[nt][e], acc[nt][e + 1]);
+      }
+    __syncthreads();
+    chunk_scalars<DK>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
+    __syncthreads();
+    if (tid < C) s.kts[tid] = __expf(s.G[C - 1] - s.G[tid]);
+    const int mt = warp & 3, nh = warp >> 2;
+    {  // W = T diag(beta gamma) K;  P = lower_incl(Q K^T (*) Gamma)
+      float d[DK / 16][4];
+      zero(d);
+      auto Ta = [&](int r, int c) { return s.Tm[r][c]; };
+      auto Kb = [&](int c, int i) { return s.beta[c] * s.gam[c] * bf(s.kb[c][i]); };
+      mma_rows<DK / 16>(d, Ta, Kb, 16 * mt, (DK / 2) * nh, C, lane);
+#pragma unroll
+      for (int nt = 0; nt < DK / 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          s.W[frow(16 * mt, lane, e)][fcol((DK / 2) * nh, nt, lane, e)] = d[nt][e];
+      float p[4][4];
+      zero(p);
+      auto Qa = [&](int r, int i) { return bf(s.qb[r][i]); };
+      auto Kt = [&](int i, int c) { return bf(s.kb[c][i]); };
+      mma_rows<4>(p, Qa, Kt, 16 * mt, 32 * nh, DK, lane);
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
+          s.P[r][c] = c <= r ? p[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;
+        }
+    }
+    __syncthreads();
+    const float gC = s.gam[C - 1];
+    {  // dV' = P^T dO + Kt dH_{n+1}   [C x 64]
+      float d[4][4];
+      zero(d);
+      auto PTa = [&](int r, int c) { return s.P[c][r]; };
+      auto Ob = [&](int c, int j) { return bf(s.ob[c][j]); };
+      mma_rows<4>(d, PTa, Ob, 16 * mt, 32 * nh, C, lane);
+      auto Kta = [&](int r, int i) { return s.kts[r] * bf(s.kb[r][i]); };
+      auto Hb = [&](int i, int j) { return s.dH[i][j]; };
+      mma_rows<4>(d, Kta, Hb, 16 * mt, 32 * nh, DK, lane);
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+          const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
+          s.dV[r][c] = d[nt][e];
+          s.dV[r][c + 1] = d[nt][e + 1];
+          *reinterpret_cast<float2*>(dVws + (chunk * C + r) * DV + j0 + c) =
+              make_float2(d[nt][e], d[nt][e + 1]);
+        }
+    }
+    __syncthreads();
+    {  // dH_n = gamma_C dH_{n+1} + (diag(gamma) Q)^T dO - W^T dV'
+#pragma unroll
+      for (int nt = 0; nt < BVA / 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] *= gC;
+      auto QTa = [&](int i, int c) { return s.gam[c] * bf(s.qb[c][i]); };
+      auto Ob = [&](int c, int j) { return bf(s.ob[c][j]); };
+      mma_rows<BVA / 8>(acc, QTa, Ob, 16 * warp, 0, C, lane);
+      auto WTa = [&](int i, int c) { return -s.W[c][i]; };
+      auto dVb = [&](int c, int j) { return s.dV[c][j]; };
+      mma_rows<BVA / 8>(acc, WTa, dVb, 16 * warp, 0, C, lane);
+    }
+  }
+  if (dh0) {
+#pragma unroll
+    for (int nt = 0; nt < BVA / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        dh0[(head * DK + frow(16 * warp, lane, e)) * DV + j0 + fcol(0, nt, lane, e)] =
+            acc[nt][e];
+  }
+}
+
+// ---------------------------------------------------------------- gradients
+template <int DK, int DV>
+struct GradSmem {
+  __nv_bfloat16 qb[C][LB<DK>()];
+  __nv_bfloat16 kb[C][LB<DK>()];
+  __nv_bfloat16 vb[C][LB<DV>()];
+  __nv_bfloat16 ob[C][LB<DV>()];
+  float Tm[C][LF<C>()];
+  float Vp[C][LF<DV>()];   // V'
+  float dVp[C][LF<DV>()];  // dV'
+  float big[DK][LF<DV / 2>()];  // a 64-column half of h_n or dH, or dW [C][DK]
+  float X1[C][LF<C>()];
+  float X2[C][LF<C>()];
+  float G[C], gam[C], beta[C], n2[C], kts[C];
+  float dG[C], dB[C];
+  float part[2][C];  // per-row partial sums of the two warps sharing a row tile
+  float red[NT / 32];
+};
+
+// Sum a per-row value over the 4 lanes holding one fragment row (t), then the
+// two warps (nh) sharing the row tile, into dst[row] in a fixed order.
+__device__ __forceinline__ float quad_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  return x;
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(NT)
+cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                 const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
+                 const float* __restrict__ g, const float* __restrict__ eta, float eps,
+                 const float* __restrict__ ck, const float* __restrict__ Tws,
+                 const float* __restrict__ Vws, const float* __restrict__ dVws,
+                 const float* __restrict__ dHws, float* __restrict__ dq, float* __restrict__ dk,
+                 float* __restrict__ dv, float* __restrict__ dg, float* __restrict__ deta,
+                 int Tlen, int H, int nblk) {
+  static_assert(DK == DV, "square heads");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  auto& s = *reinterpret_cast<GradSmem<DK, DV>*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
+  const size_t head = (size_t)b * H + hh, chunk = head * nblk + n;
+  const int t0 = n * C, len = min(C, Tlen - t0);
+  const size_t tok0 = ((size_t)b * Tlen + t0) * H + hh;
+  const int mt = warp & 3, nh = warp >> 2;
+  constexpr int HALF = DV / 2;
+  const float* hn = ck + chunk * DK * DV;
+  const float* dHn = dHws + chunk * DK * DV;
+
+  load_rows_bf16<DK>(&s.qb[0][0], q + tok0 * DK, (size_t)H * DK, len);
+  load_rows_bf16<DK>(&s.kb[0][0], k + tok0 * DK, (size_t)H * DK, len);
+  load_rows_bf16<DV>(&s.vb[0][0], v + tok0 * DV, (size_t)H * DV, len);
+  load_rows_bf16<DV>(&s.ob[0][0], dout + tok0 * DV, (size_t)H * DV, len);
+  load_f32<C, C>(&s.Tm[0][0], Tws + chunk * C * C, C);
+  load_f32<C, DV>(&s.Vp[0][0], Vws + chunk * C * DV, DV);
+  load_f32<C, DV>(&s.dVp[0][0], dVws + chunk * C * DV, DV);
+  if (tid < C) s.dG[tid] = s.dB[tid] = 0.f;
+  __syncthreads();
+  chunk_scalars<DK>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
+  __syncthreads();
+  if (tid < C) s.kts[tid] = __expf(s.G[C - 1] - s.G[tid]);
+  const float gC = s.gam[C - 1];
+
+  // ---- phase 1: products with h_n, one 64-column half of it at a time
+  float accQ[DK / 16][4], accW[DK / 16][4];  // rows 16 mt .., columns (DK/2) nh ..
+  zero(accQ);
+  zero(accW);
+  float rowO[2] = {0.f, 0.f};  // rowdot(dO, diag(gamma) Q h_n) for rows g, g + 8
+  for (int half = 0; half < 2; ++half) {
+    __syncthreads();
+    load_f32<DK, HALF>(&s.big[0][0], hn + half * HALF, DV);
+    __syncthreads();
+    // dO h_n^T and -dV' h_n^T over this half of the dv index
+    auto Oa = [&](int r, int j) { return bf(s.ob[r][half * HALF + j]); };
+    auto dVa = [&](int r, int j) { return -s.dVp[r][half * HALF + j]; };
+    auto HTb = [&](int j, int i) { return s.big[i][j]; };
+    mma_rows<DK / 16>(accQ, Oa, HTb, 16 * mt, (DK / 2) * nh, HALF, lane);
+    mma_rows<DK / 16>(accW, dVa, HTb, 16 * mt, (DK / 2) * nh, HALF, lane);
+    // diag(gamma) Q h_n on this half's columns: 64 x 64, 4 tiles per warp
+    float o[4][4];
+    zero(o);
+    auto Qa = [&](int r, int i) { return s.gam[r] * bf(s.qb[r][i]); };
+    auto Hb = [&](int i, int j) { return s.big[i][j]; };
+    mma_rows<4>(o, Qa, Hb, 16 * mt, 32 * nh, DK, lane);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        rowO[e >> 1] += o[nt][e] * bf(s.ob[frow(16 * mt, lane, e)]
+                                          [half * HALF + fcol(32 * nh, nt, lane, e)]);
+  }
+  // <dH_{n+1}, h_n> (block sum, fixed order)
+  float hd = 0.f;
+  for (int p = tid; p < DK * DV; p += NT) hd = fmaf(hn[p], dHn[p], hd);
+  hd = warp_sum(hd);
+  if (lane == 0) s.red[warp] = hd;
+  // rowO -> dG (two warps per row tile: nh = 0 writes part[0], nh = 1 part[1])
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const float x = quad_sum(rowO[hr]);
+    if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+  }
+  __syncthreads();
+  if (tid < C) s.dG[tid] += s.part[0][tid] + s.part[1][tid];
+  // dq (first part) stays in accQ; dW -> big as [C][DK]
+  float* dW = &s.big[0][0];  // [C][LF<DK>] fits in [DK][LF<DV/2>]
+  static_assert(C * LF<DK>() <= DK * LF<DV / 2>(), "dW in big");
+#pragma unroll
+  for (int nt = 0; nt < DK / 16; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      dW[frow(16 * mt, lane, e) * LF<DK>() + fcol((DK / 2) * nh, nt, lane, e)] = accW[nt][e];
+
+  // ---- phase 2: the C x C quantities
+  {  // dP = dO V'^T (*) incl -> X1;  Q K^T -> X2
+    float d[4][4], p[4][4];
+    zero(d);
+    zero(p);
+    auto Oa = [&](int r, int j) { return bf(s.ob[r][j]); };
+    auto VTb = [&](int j, int c) { return s.Vp[c][j]; };
+    mma_rows<4>(d, Oa, VTb, 16 * mt, 32 * nh, DV, lane);
+    auto Qa = [&](int r, int i) { return bf(s.qb[r][i]); };
+    auto KTb = [&](int i, int c) { return bf(s.kb[c][i]); };
+    mma_rows<4>(p, Qa, KTb, 16 * mt, 32 * nh, DK, lane);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
+        const bool in = c <= r;
+        s.X1[r][c] = in ? d[nt][e] : 0.f;
+        s.X2[r][c] = in ? p[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;  // P
+      }
+  }
+  __syncthreads();
+  // F = dP (*) P: dG_r += rowsum, dG_s -= colsum;  X1 <- dP (*) Gamma
+  if (tid < C) {
+    float rs = 0.f, cs = 0.f;
+    for (int c = 0; c < C; ++c) {
+      rs = fmaf(s.X1[tid][c], s.X2[tid][c], rs);
+      cs = fmaf(s.X1[c][tid], s.X2[c][tid], cs);
+    }
+    s.dG[tid] += rs - cs;
+  }
+  __syncthreads();
+  for (int p = tid; p < C * C; p += NT) {
+    const int r = p / C, c = p % C;
+    if (c <= r) s.X1[r][c] *= __expf(s.G[r] - s.G[c]);
+  }
+  __syncthreads();
+  float accK[DK / 16][4];
+  zero(accK);
+  {  // dQ += (dP (*) Gamma) K -> dq;  dK = (dP (*) Gamma)^T Q
+    auto Xa = [&](int r, int c) { return s.X1[r][c]; };
+    auto Kb = [&](int c, int i) { return bf(s.kb[c][i]); };
+#pragma unroll
+    for (int nt = 0; nt < DK / 16; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) accQ[nt][e] *= s.gam[frow(16 * mt, lane, e)];
+    mma_rows<DK / 16>(accQ, Xa, Kb, 16 * mt, (DK / 2) * nh, C, lane);
+    auto XTa = [&](int r, int c) { return s.X1[c][r]; };
+    auto Qb = [&](int c, int i) { return bf(s.qb[c][i]); };
+    mma_rows<DK / 16>(accK, XTa, Qb, 16 * mt, (DK / 2) * nh, C, lane);
+#pragma unroll
+    for (int nt = 0; nt < DK / 16; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; e += 2) {
+        const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
+        if (r < len)
+          *reinterpret_cast<float2*>(dq + (tok0 + (size_t)r * H) * DK + i) =
+              make_float2(accQ[nt][e], accQ[nt][e + 1]);
+      }
+  }
+  {  // T^T dW: dK += diag(beta gamma) T^T dW;  dbeta, dG += rowdot(T^T dW, K) terms
+    float d[DK / 16][4];
+    zero(d);
+    auto TTa = [&](int r, int c) { return s.Tm[c][r]; };
+    auto dWb = [&](int c, int i) { return dW[c * LF<DK>() + i]; };
+    mma_rows<DK / 16>(d, TTa, dWb, 16 * mt, (DK / 2) * nh, C, lane);
+    float rk[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < DK / 16; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
+        accK[nt][e] = fmaf(s.beta[r] * s.gam[r], d[nt][e], accK[nt][e]);
+        rk[e >> 1] = fmaf(d[nt][e], bf(s.kb[r][i]), rk[e >> 1]);
+      }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const float x = quad_sum(rk[hr]);
+      if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+    }
+  }
+  __syncthreads();
+  if (tid < C) {
+    const float x = s.part[0][tid] + s.part[1][tid];
+    s.dB[tid] += s.gam[tid] * x;
+    s.dG[tid] += s.beta[tid] * s.gam[tid] * x;
+  }
+  __syncthreads();
+  {  // T^T dV': dv = diag(beta) T^T dV';  dbeta += rowdot(T^T dV', V)
+    float d[DV / 16][4];
+    zero(d);
+    auto TTa = [&](int r, int c) { return s.Tm[c][r]; };
+    auto dVb = [&](int c, int j) { return s.dVp[c][j]; };
+    mma_rows<DV / 16>(d, TTa, dVb, 16 * mt, (DV / 2) * nh, C, lane);
+    float rv[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < DV / 16; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; e += 2) {
+        const int r = frow(16 * mt, lane, e), j = fcol((DV / 2) * nh, nt, lane, e);
+        rv[e >> 1] = fmaf(d[nt][e], bf(s.vb[r][j]), rv[e >> 1]);
+        rv[e >> 1] = fmaf(d[nt][e + 1], bf(s.vb[r][j + 1]), rv[e >> 1]);
+        if (r < len)
+          *reinterpret_cast<float2*>(dv + (tok0 + (size_t)r * H) * DV + j) =
+              make_float2(s.beta[r] * d[nt][e], s.beta[r] * d[nt][e + 1]);
+      }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const float x = quad_sum(rv[hr]);
+      if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+    }
+  }
+  __syncthreads();
+  if (tid < C) s.dB[tid] += s.part[0][tid] + s.part[1][tid];
+  {  // dT = dW (diag(beta gamma) K)^T + dV' (diag(beta) V)^T -> X2 (P is done)
+    float d[4][4];
+    zero(d);
+    auto dWa = [&](int r, int i) { return dW[r * LF<DK>() + i]; };
+    auto KTb = [&](int i, int c) { return s.beta[c] * s.gam[c] * bf(s.kb[c][i]); };
+    mma_rows<4>(d, dWa, KTb, 16 * mt, 32 * nh, DK, lane);
+    auto dVa = [&](int r, int j) { return s.dVp[r][j]; };
+    auto VTb = [&](int j, int c) { return s.beta[c] * bf(s.vb[c][j]); };
+    mma_rows<4>(d, dVa, VTb, 16 * mt, 32 * nh, DV, lane);
+    __syncthreads();  // every warp is done reading X2 (P) and X1 (dP Gamma)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s.X2[frow(16 * mt, lane, e)][fcol(32 * nh, nt, lane, e)] = d[nt][e];
+  }
+  __syncthreads();
+  {  // Y = T^T dT -> X1
+    float d[4][4];
+    zero(d);
+    auto TTa = [&](int r, int c) { return s.Tm[c][r]; };
+    auto Xb = [&](int c, int j) { return s.X2[c][j]; };
+    mma_rows<4>(d, TTa, Xb, 16 * mt, 32 * nh, C, lane);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s.X1[frow(16 * mt, lane, e)][fcol(32 * nh, nt, lane, e)] = d[nt][e];
+  }
+  __syncthreads();
+  {  // dA = -strict_lower(Y T^T) -> X2;  K K^T kept in registers
+    float d[4][4], kk[4][4];
+    zero(d);
+    zero(kk);
+    auto Ya = [&](int r, int c) { return s.X1[r][c]; };
+    auto TTb = [&](int c, int j) { return s.Tm[j][c]; };
+    mma_rows<4>(d, Ya, TTb, 16 * mt, 32 * nh, C, lane);
+    auto Ka = [&](int r, int i) { return bf(s.kb[r][i]); };
+    auto KTb = [&](int i, int c) { return bf(s.kb[c][i]); };
+    mma_rows<4>(kk, Ka, KTb, 16 * mt, 32 * nh, DK, lane);
+    __syncthreads();  // X2 (dT) fully read
+    // E = dA (*) Gamma -> X2;  F = dA (*) A -> X1 (A = beta_r KK Gamma);
+    // dbeta_r += sum_s E_rs KK_rs
+    float rb[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
+        const float E = c < r ? -d[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;  // dA (*) Gamma
+        s.X2[r][c] = E;
+        s.X1[r][c] = E * s.beta[r] * kk[nt][e];  // dA (*) A
+        rb[e >> 1] = fmaf(E, kk[nt][e], rb[e >> 1]);
+      }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const float x = quad_sum(rb[hr]);
+      if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+    }
+  }
+  __syncthreads();
+  if (tid < C) {
+    float rs = 0.f, cs = 0.f;
+    for (int c = 0; c < C; ++c) {
+      rs += s.X1[tid][c];
+      cs += s.X1[c][tid];
+    }
+    s.dG[tid] += rs - cs;
+    s.dB[tid] += s.part[0][tid] + s.part[1][tid];
+  }
+  {  // dK += diag(beta) E K + (diag(beta) E)^T K
+    auto Ea = [&](int r, int c) { return s.beta[r] * s.X2[r][c]; };
+    auto ETa = [&](int r, int c) { return s.beta[c] * s.X2[c][r]; };
+    auto Kb = [&](int c, int i) { return bf(s.kb[c][i]); };
+    mma_rows<DK / 16>(accK, Ea, Kb, 16 * mt, (DK / 2) * nh, C, lane);
+    mma_rows<DK / 16>(accK, ETa, Kb, 16 * mt, (DK / 2) * nh, C, lane);
+  }
+
+  // ---- phase 3: dKt = V' dH_{n+1}^T, a 64-column half of dH at a time
+  float dKt[DK / 16][4];
+  zero(dKt);
+  for (int half = 0; half < 2; ++half) {
+    __syncthreads();  // big (dW, or the other half of dH) is no longer read
+    load_f32<DK, HALF>(&s.big[0][0], dHn + half * HALF, DV);
+    __syncthreads();
+    auto Va = [&](int r, int j) { return s.Vp[r][half * HALF + j]; };
+    auto HTb = [&](int j, int i) { return s.big[i][j]; };
+    mma_rows<DK / 16>(dKt, Va, HTb, 16 * mt, (DK / 2) * nh, HALF, lane);
+  }
+  float rt[2] = {0.f, 0.f};
+#pragma unroll
+  for (int nt = 0; nt < DK / 16; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
+      const float sc = s.kts[r];
+      accK[nt][e] = fmaf(sc, dKt[nt][e], accK[nt][e]);
+      rt[e >> 1] = fmaf(dKt[nt][e], sc * bf(s.kb[r][i]), rt[e >> 1]);
+    }
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const float x = quad_sum(rt[hr]);
+    if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+  }
+  __syncthreads();
+  if (tid < C) s.dG[tid] -= s.part[0][tid] + s.part[1][tid];
+  __syncthreads();
+  if (tid == 0) {
+    float tot = 0.f, hdt = 0.f;
+    for (int r = 0; r < C; ++r) tot += s.part[0][r] + s.part[1][r];
+    for (int w = 0; w < NT / 32; ++w) hdt += s.red[w];
+    s.dG[C - 1] += tot + gC * hdt;
+    // dg = reverse in-chunk cumsum of dG (rows >= len carry no gradient)
+    float acc = 0.f;
+    for (int r = C - 1; r >= 0; --r) {
+      acc += s.dG[r];
+      s.dG[r] = acc;
+    }
+  }
+  __syncthreads();
+  // step size: KLA beta = eta / (||k||^2 + eps)
+  if (tid < len) {
+    const size_t tok = tok0 + (size_t)tid * H;
+    dg[tok] = s.dG[tid];
+    if (eps >= 0.f) {
+      const float den = s.n2[tid] + eps;
+      deta[tok] = s.dB[tid] / den;
+      s.part[0][tid] = -2.f * s.dB[tid] * eta[tok] / (den * den);
+    } else {
+      deta[tok] = s.dB[tid];
+      s.part[0][tid] = 0.f;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int nt = 0; nt < DK / 16; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
+      if (r < len) {
+        const float cf = s.part[0][r];
+        *reinterpret_cast<float2*>(dk + (tok0 + (size_t)r * H) * DK + i) =
+            make_float2(fmaf(cf, bf(s.kb[r][i]), accK[nt][e]),
+                        fmaf(cf, bf(s.kb[r][i + 1]), accK[nt][e + 1]));
+      }
+    }
+}
+
+// ---------------------------------------------------------------- launch
+
+static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct CbwdWs {
+  size_t ck, Tm, Vp, dVp, dH, beta, alpha, total;
+};
+
+static CbwdWs cbwd_layout(int B, int T, int H, int dk, int dv) {
+  const size_t nblk = ((size_t)T + C - 1) / C, chunks = (size_t)B * H * nblk;
+  const size_t ntok = (size_t)B * T * H;
+  CbwdWs w;
+  w.ck = 0;
+  w.Tm = w.ck + al256(chunks * dk * dv * 4);
+  w.Vp = w.Tm + al256(chunks * C * C * 4);
+  w.dVp = w.Vp + al256(chunks * C * dv * 4);
+  w.dH = w.dVp + al256(chunks * C * dv * 4);
+  w.beta = w.dH + al256(chunks * dk * dv * 4);
+  w.alpha = w.beta + al256(ntok * 4);
+  w.total = w.alpha + al256(ntok * 4);
+  return w;
+}
+
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
+  if (B < 1 || H < 1 || T < 1 || dk != 128 || dv != 128) return 0;
+  return cbwd_layout(B, T, H, dk, dv).total;
+}
+
+// The checkpoint kernel of kla_backward.cu (h at every 64-token block start,
+// every token's beta and alpha).
+cudaError_t launch_bwd_checkpoints(const void* k, const void* v, const float* g,
+                                   const float* eta, float eps, const float* h0, float* ck,
+                                   float* beta_out, float* alpha_out, int B, int T, int H,
+                                   int dk, int dv, int dtype, cudaStream_t st);
+
+cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                             const float* eta, float eps, const float* h0, const void* dout,
+                             const float* dhT, float* dq, float* dk, float* dv, float* dg,
+                             float* deta, float* dh0, int B, int Tlen, int H, int dkd, int dvd,
+                             void* ws, cudaStream_t st) {
+  constexpr int DK = 128, DV = 128;
+  if (dkd != DK || dvd != DV) return cudaErrorInvalidValue;
+  const CbwdWs w = cbwd_layout(B, Tlen, H, DK, DV);
+  char* base = (char*)ws;
+  float* ck = (float*)(base + w.ck);
+  float* Tws = (float*)(base + w.Tm);
+  float* Vws = (float*)(base + w.Vp);
+  float* dVws = (float*)(base + w.dVp);
+  float* dHws = (float*)(base + w.dH);
+  const int nblk = (Tlen + C - 1) / C;
+  cudaError_t e = launch_bwd_checkpoints(k, v, g, eta, eps, h0, ck, (float*)(base + w.beta),
+                                         (float*)(base + w.alpha), B, Tlen, H, DK, DV,
+                                         KLA_BF16, st);
+  if (e != cudaSuccess) return e;
+  const auto* qb = (const __nv_bfloat16*)q;
+  const auto* kb = (const __nv_bfloat16*)k;
+  const auto* vb = (const __nv_bfloat16*)v;
+  const auto* ob = (const __nv_bfloat16*)dout;
+  constexpr size_t sp = sizeof(PrepSmem<DK, DV>), sa = sizeof(AdjSmem<DK>),
+                   sg = sizeof(GradSmem<DK, DV>);
+  static_assert(sp <= 227 * 1024 && sa <= 227 * 1024 && sg <= 227 * 1024, "shared memory");
+  if ((e = cudaFuncSetAttribute(cbwd_prep_kernel<DK, DV>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp)) ||
+      (e = cudaFuncSetAttribute(cbwd_adjoint_kernel<DK, DV>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa)) ||
+      (e = cudaFuncSetAttribute(cbwd_grad_kernel<DK, DV>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg)))
+    return e;
+  cbwd_prep_kernel<DK, DV><<<dim3(nblk, H, B), NT, sp, st>>>(kb, vb, g, eta, eps, ck, Tws, Vws,
+                                                             Tlen, H, nblk);
+  cbwd_adjoint_kernel<DK, DV><<<dim3(DV / BVA, H, B), NT, sa, st>>>(
+      qb, kb, ob, g, eta, eps, dhT, Tws, dVws, dHws, dh0, Tlen, H, nblk);
+  cbwd_grad_kernel<DK, DV><<<dim3(nblk, H, B), NT, sg, st>>>(
+      qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, dVws, dHws, dq, dk, dv, dg, deta, Tlen, H,
+      nblk);
+  return cudaGetLastError();
+}
+
+}  // namespace kla

@@ -291,6 +291,39 @@ KLA_API kla_status kla_recurrent_bwd(const void *q, const void *k, const void *v
                                      int dtype, void *workspace, size_t ws_bytes,
                                      void *stream);
 /*
+ * Chunkwise backward: the same gradients, arguments, layouts and errors as
+ * kla_recurrent_bwd / kla_gdn_recurrent_bwd, computed from the chunk form
+ * of the forward (chunk C = 64; "Deep Dive into KDA", section 3).  Per chunk
+ * n with start state h_n: dV'_n = P^T dO + Kt dH_{n+1} and
+ * dH_n = gamma_C dH_{n+1} + (diag(gamma) Q)^T dO - W^T dV'_n form one
+ * reverse chain over the chunks (per head and 64-column slab); every other
+ * gradient is per-chunk work on warp-level tensor-core products (tf32
+ * operands, fp32 sums): dQ, dK from P, W, U = T diag(beta) V and
+ * T = (I + A)^{-1} (dA = -strict_lower(T^T dT T^T)), dg as the reverse
+ * in-chunk cumsum of dG.  The states h_n come from a token-serial fp32
+ * forward.  bf16 with dk = dv = 128 runs these kernels (accuracy of tf32
+ * products: relative L2 about 1e-3); fp32 I/O and d = 64 run the
+ * token-serial kernels of kla_recurrent_bwd.  Workspace:
+ * kla_chunk_bwd_workspace_size(...) bytes (for the chunk kernels about
+ * B*H*ceil(T/64) * 208 KiB).
+ */
+KLA_API size_t kla_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int dtype);
+KLA_API kla_status kla_chunk_bwd(const void *q, const void *k, const void *v,
+                                 const float *g, const float *eta, float eps,
+                                 const float *h0, const void *grad_o, const float *grad_hT,
+                                 float *grad_q, float *grad_k, float *grad_v, float *grad_g,
+                                 float *grad_eta, float *grad_h0, int B, int T, int H,
+                                 int dk, int dv, int dtype, void *workspace, size_t ws_bytes,
+                                 void *stream);
+KLA_API kla_status kla_gdn_chunk_bwd(const void *q, const void *k, const void *v,
+                                     const float *g, const float *beta, const float *h0,
+                                     const void *grad_o, const float *grad_hT, float *grad_q,
+                                     float *grad_k, float *grad_v, float *grad_g,
+                                     float *grad_beta, float *grad_h0, int B, int T, int H,
+                                     int dk, int dv, int dtype, void *workspace,
+                                     size_t ws_bytes, void *stream);
+
+/*
  * The same backward for the per-channel-gate form (kla_kda_fwd; "Deep Dive
  * into KDA", section 2.3): g and grad_g are [B][T][H][dk] (one log-gate per
  * key channel), the forward being hd = Diag(e^{g_t}) h_{t-1}; r = hd^T k;

@@ -179,3 +179,74 @@ def test_kda_backward_equal_channels_is_scalar_gate():
     for n in ("dq", "dk", "dv", "deta", "dh0"):
         assert rel(a[n].cpu(), b[n].cpu()) < 1e-5, n
     assert rel(a["dg"].sum(-1).cpu(), b["dg"].cpu()) < 1e-5
+
+
+# ---- chunkwise backward (kla_chunk_bwd): bf16, d = 128 on the chunk kernels
+# (tf32 tensor-core products), so the bf16 bar applies
+TOL_CHUNK = 1e-2
+
+
+@pytest.mark.parametrize("name,B,T,H,with_h0,with_dhT", [
+    ("prefill_4k", 1, 150, 2, True, True),     # 3 chunks, ragged last one
+    ("prefill_4k", 2, 64, 3, False, True),     # exactly one chunk
+    ("prefill_4k", 1, 1, 2, True, True),       # one token
+    ("prefill_4k", 1, 257, 1, False, False),   # one token past 4 chunks
+    ("prefill_65k", 1, 700, 2, False, True),   # strong forgets
+])
+def test_chunk_backward(name, B, T, H, with_h0, with_dhT):
+    w = inputs.WORKLOADS[name].scaled(B=B, T=T, H=H)
+    x = inputs.make_prefill(w, with_h0=with_h0)
+    do, dhT = _upstream(w, 90, with_dhT)
+    xc = cuda(x)
+    out = api.chunk_bwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], cuda(do), x["eps"],
+                        xc["h0"], cuda(dhT))
+    api.check_device_error()
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"], do, dhT)
+    _check(out, ref, tol=TOL_CHUNK)
+
+
+def test_gdn_chunk_backward():
+    w = inputs.WORKLOADS["prefill_4k"].scaled(B=2, T=130, H=2)
+    x = inputs.make_prefill(w, with_h0=True)
+    kf = x["k"].float()
+    k = (kf / kf.norm(dim=-1, keepdim=True)).to(x["k"].dtype)
+    rng = np.random.Generator(np.random.PCG64(91))
+    beta = torch.from_numpy(rng.uniform(0.05, 1.95, x["g"].shape).astype(np.float32))
+    do, dhT = _upstream(w, 92)
+    xc = cuda(x)
+    out = api.gdn_chunk_bwd(xc["q"], cuda(k), xc["v"], xc["g"], cuda(beta), cuda(do), xc["h0"],
+                            cuda(dhT))
+    ref = oracle.gated_delta_backward(x["q"], k, x["v"], x["g"], beta, x["h0"], do, dhT)
+    _check(out, ref, names=("dq", "dk", "dv", "dg", "dbeta", "dh0"), tol=TOL_CHUNK)
+
+
+def test_chunk_backward_other_shapes_run_token_serial():
+    """fp32 I/O and d = 64 take the token-serial kernels through the same
+    entry point (the fp32 bar then holds)."""
+    w = inputs.WORKLOADS["tiny"].scaled(B=1, T=100, H=2)
+    x = inputs.make_prefill(w, with_h0=True)
+    do, dhT = _upstream(w, 93)
+    xc = cuda(x)
+    out = api.chunk_bwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], cuda(do), x["eps"],
+                        xc["h0"], cuda(dhT))
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"], do, dhT)
+    _check(out, ref)
+
+
+def test_chunk_backward_full_size_sampled_heads():
+    """The 4K layer (B=8 T=4096 H=8 d=128, bf16) in one call on the chunk
+    kernels; the oracle's gradients of two sampled heads."""
+    w = inputs.WORKLOADS["prefill_4k"]
+    x = inputs.make_prefill(w)
+    do, dhT = _upstream(w, 94)
+    xc = cuda(x)
+    out = api.chunk_bwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], cuda(do), x["eps"],
+                        None, cuda(dhT))
+    api.check_device_error()
+    for b, h in ((2, 6), (5, 1)):
+        sl = lambda t: t[b:b + 1, :, h:h + 1]
+        ref = oracle.backward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["eta"]),
+                              x["eps"], None, sl(do), dhT[b:b + 1, h:h + 1])
+        got = {n: sl(out[n].cpu()) for n in ("dq", "dk", "dv", "dg", "deta")}
+        got["dh0"] = out["dh0"][b:b + 1, h:h + 1].cpu()
+        _check(got, ref, tol=TOL_CHUNK)
