@@ -510,10 +510,11 @@ def run_kda_prefill(w, dev, stream, flush, peaks, peak_src, steps=3):
 
 
 def run_backward(w, dev, stream, flush, peaks, peak_src, steps=2):
-    """Gradients of the prefill (token-serial fp32 backward) on the same
-    workload for a seeded dL/do and dL/dh_T: time per call and achieved GB/s
-    of its algorithmic bytes (reads q, k, v, dL/do, g, eta, dL/dh_T; writes
-    the fp32 gradients of q, k, v, g, eta, h0)."""
+    """Gradients of the prefill (chunkwise backward; the token-serial one
+    timed beside it) on the same workload for a seeded dL/do and dL/dh_T:
+    time per call and achieved GB/s of its algorithmic bytes (reads q, k, v,
+    dL/do, g, eta, dL/dh_T; writes the fp32 gradients of q, k, v, g, eta,
+    h0)."""
     from delta_rule_linear_kla_b200 import api, inputs
 
     x = inputs.make_prefill(w)
@@ -521,22 +522,28 @@ def run_backward(w, dev, stream, flush, peaks, peak_src, steps=2):
     gen = torch.Generator(device="cpu").manual_seed(w.seed + 21)
     do = torch.randn((w.B, w.T, w.H, w.dv), generator=gen).to(w.torch_dtype).to(dev)
     dhT = torch.randn((w.B, w.H, w.dk, w.dv), generator=gen).to(dev)
-    ws = torch.empty(max(1, api.recurrent_bwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv)),
-                     dtype=torch.uint8, device=dev)
-    run = lambda: api.recurrent_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["eta"], do,
-                                    x["eps"], xd["h0"], dhT, workspace=ws, stream=stream)
-    run()
-    torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(steps)]
-    for e0, e1 in evs:
-        flush()
-        e0.record(stream)
+    def timed(fn, wsize):
+        ws = torch.empty(max(1, wsize), dtype=torch.uint8, device=dev)
+        run = lambda: fn(xd["q"], xd["k"], xd["v"], xd["g"], xd["eta"], do, x["eps"],
+                         xd["h0"], dhT, workspace=ws, stream=stream)
         run()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    api.check_device_error()
-    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for e0, e1 in evs:
+            flush()
+            e0.record(stream)
+            run()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        api.check_device_error()
+        del ws
+        return sum(a.elapsed_time(b) for a, b in evs) / steps
+
+    ms = timed(api.chunk_bwd, api.chunk_bwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv,
+                                                           w.torch_dtype))
+    ms_serial = timed(api.recurrent_bwd, api.recurrent_bwd_workspace_size(w.B, w.T, w.H, w.dk,
+                                                                          w.dv))
     es = 2 if w.dtype == "bf16" else 4
     ntok = w.B * w.T * w.H
     sb = w.B * w.H * w.dk * w.dv * 4
@@ -547,14 +554,16 @@ def run_backward(w, dev, stream, flush, peaks, peak_src, steps=2):
     return {"metric": "backward tokens/s (%s)" % w.name,
             "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
             "calls": steps, "dtype": "f32",
-            "path": "bwd_checkpoint_kernel + bwd_kernel (token-serial fp32, states "
-                    "recomputed from 64-token checkpoints) + bwd_finish_kernel",
+            "path": "kla_chunk_bwd: forward chunk prefill writing every chunk-start state, "
+                    "cbwd_prep_kernel, cbwd_adjoint_kernel (reverse state-adjoint chain), "
+                    "cbwd_grad_kernel (warp-level tf32 tensor-core products)",
+            "token_serial_ms_per_call": ms_serial,
             "roofline": {"kernel": "whole call", "bound": "hbm",
                          "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "traffic": None, "algorithmic_bytes": byts,
                          "peak_source": peak_src,
-                         "note": "token-serial: bounded by the per-token dependency "
-                                 "chain, not by HBM"}}
+                         "note": "the per-chunk kernels are bound by issuing their "
+                                 "warp-level products' operand loads, not by HBM"}}
 
 
 # ------------------------------------------------------------ reference

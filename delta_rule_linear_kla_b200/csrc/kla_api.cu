@@ -391,10 +391,12 @@ static kla_status bwd_impl(const void* q, const void* k, const void* v, const fl
                             : cudaMemsetAsync(grad_h0, 0, sb, st);
     return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
   }
+  unsigned int* err = use_chunks ? device_error_ptr() : nullptr;
+  if (use_chunks && !err) return KLA_ERR_CUDA;
   cudaError_t e =
       use_chunks
           ? launch_chunk_bwd(q, k, v, g, eta, eps, h0, grad_o, grad_hT, grad_q, grad_k, grad_v,
-                             grad_g, grad_eta, grad_h0, B, T, H, dk, dv, workspace, st)
+                             grad_g, grad_eta, grad_h0, B, T, H, dk, dv, workspace, err, st)
           : launch_recurrent_bwd(q, k, v, g, vector_gate, eta, eps, h0, grad_o, grad_hT, grad_q,
                                  grad_k, grad_v, grad_g, grad_eta, grad_h0, B, T, H, dk, dv,
                                  dtype, workspace, st);

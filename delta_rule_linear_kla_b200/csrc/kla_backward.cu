@@ -568,25 +568,6 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
   return cudaGetLastError();
 }
 
-// The checkpoint kernel alone (bf16, d = 128, scalar gate): every h_n and
-// each token's beta and alpha, for the chunkwise backward (kla_chunk_bwd.cu).
-cudaError_t launch_bwd_checkpoints(const void* k, const void* v, const float* g,
-                                   const float* eta, float eps, const float* h0, float* ck,
-                                   float* beta_out, float* alpha_out, int B, int T, int H,
-                                   int dk, int dv, int dtype, cudaStream_t st) {
-  if (dtype != KLA_BF16 || dk != 128 || dv != 128) return cudaErrorInvalidValue;
-  using TT = __nv_bfloat16;
-  constexpr int DK = 128, DV = 128;
-  const int nblk = (T + bwd::BLK - 1) / bwd::BLK;
-  constexpr size_t smem = sizeof(bwd::Ops<DK, false>);
-  cudaError_t e = cudaFuncSetAttribute(bwd_checkpoint_kernel<TT, DK, DV, false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  bwd_checkpoint_kernel<TT, DK, DV, false><<<dim3(DV / bwd::BV, H, B), bwd::NT, smem, st>>>(
-      (const TT*)k, (const TT*)v, g, eta, eps, h0, ck, beta_out, alpha_out, T, H, nblk);
-  return cudaGetLastError();
-}
-
 template <bool VG>
 static cudaError_t launch_bwd_vg(const void* q, const void* k, const void* v, const float* g,
                                  const float* eta, float eps, const float* h0,

@@ -31,7 +31,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v,
                             const float* g, const float* eta, float eps,
                             const float* h0, void* o, float* hT, int B, int T,
                             int H, int dk, int dv, void* workspace, size_t ws_bytes,
-                            unsigned int* err, cudaStream_t st);
+                            unsigned int* err, cudaStream_t st, float* hs = nullptr);
 
 // The two stages of launch_chunk_tc on their own: the UT transform of every
 // chunk into the workspace, then the chain kernel that reads it.
@@ -43,7 +43,8 @@ cudaError_t launch_chunk_ut(const void* k, const float* g, const float* eta, flo
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, const float* g,
                                const float* h0, void* o, float* hT, int B, int T, int H,
                                int dk, int dv, void* workspace, size_t ws_bytes,
-                               unsigned int* err, cudaStream_t st);
+                               unsigned int* err, cudaStream_t st,
+                               float* hs = nullptr);
 
 // Per-chunk factors of the per-channel-gate (KDA form) path, one tile per
 // chunk in chunk-major order: byte offsets of T'^T, P, W, Q o e^G,

@@ -25,16 +25,22 @@
 //   dg = reverse in-chunk cumsum of dG;  KLA: deta = dbeta / (||k||^2 + eps),
 //   dk += -2 dbeta eta k / (||k||^2 + eps)^2.
 //
-// Kernels (after the checkpoint kernel of kla_backward.cu, which leaves every
-// h_n in fp32 and each token's beta and alpha):
-//   cbwd_prep_kernel     per chunk: T and V' into the workspace (fp32)
-//   cbwd_adjoint_kernel  per head and 64-column slab, chunks in reverse: the
-//                        chain above, dH in registers; writes dV'_n and dH_{n+1}
+// Kernels (after the forward chunk prefill of kla_ut.cu / kla_chunk_tc.cu run
+// with its outputs off and its chain writing every h_n, fp32):
+//   cbwd_prep_kernel     per chunk: T, V', W and the two dH-independent terms
+//                        of the chain, X = P^T dO and Y = (diag(gamma) Q)^T dO,
+//                        into the workspace (fp32)
+//   cbwd_adjoint_kernel  per head and 32-column slab, chunks in reverse:
+//                        dV' = X + Kt dH, dH <- gamma_C dH + Y - W^T dV' (two
+//                        products per chunk), dH in registers, the next
+//                        chunk's operands copied in asynchronously meanwhile;
+//                        writes dV'_n and dH_{n+1}
 //   cbwd_grad_kernel     per chunk: every gradient of the chunk's tokens
 // Products are warp-level tensor-core MMAs (mma.sync m16n8k8, tf32 operands,
 // fp32 sums); operands are read from shared memory through small accessors,
 // so transposed or row-scaled operands need no extra copies.  Ragged tails
 // are zero rows with g = 0 and beta = 0 (identity steps).
+#include "kla_chunk.h"
 #include "kla_common.cuh"
 
 namespace kla {
@@ -42,8 +48,10 @@ namespace cbwd {
 
 constexpr int C = 64;
 constexpr int NT = 256;
-constexpr int BVA = 64;  // state columns per adjoint-chain CTA
+constexpr int BVA = 32;  // state columns per adjoint-chain CTA
 
+// An fp32 value rounded to a tf32 operand (to nearest; the tensor core would
+// otherwise truncate, which measured three times the gradient error).
 __device__ __forceinline__ uint32_t tf32(float x) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -58,7 +66,7 @@ template <int NTL, class FA, class FB>
 __device__ __forceinline__ void mma_rows(float (&d)[NTL][4], const FA& A, const FB& B, int m0,
                                          int n0, int K, int lane) {
   const int g = lane >> 2, t = lane & 3;
-#pragma unroll 2
+#pragma unroll 4
   for (int k0 = 0; k0 < K; k0 += 8) {
     const uint32_t a0 = tf32(A(m0 + g, k0 + t)), a1 = tf32(A(m0 + g + 8, k0 + t));
     const uint32_t a2 = tf32(A(m0 + g, k0 + t + 4)), a3 = tf32(A(m0 + g + 8, k0 + t + 4));
@@ -188,19 +196,24 @@ template <int DK, int DV>
 struct PrepSmem {
   __nv_bfloat16 kb[C][LB<DK>()];
   __nv_bfloat16 vb[C][LB<DV>()];
-  float A[C][LF<C>()];
+  __nv_bfloat16 qb[C][LB<DK>()];
+  __nv_bfloat16 ob[C][LB<DV>()];
+  float A[C][LF<C>()];  // A, then P
   float Tm[C][LF<C>()];
   float W[C][LF<DK>()];
   float h[DK][LF<DV>()];
   float G[C], gam[C], beta[C], n2[C];
 };
 
-// Per chunk: T and V' = T diag(beta) V - W h_n into the workspace.
+// Per chunk: T, V' = T diag(beta) V - W h_n, W, X = P^T dO and
+// Y = (diag(gamma) Q)^T dO into the workspace.
 template <int DK, int DV>
 __global__ void __launch_bounds__(NT)
-cbwd_prep_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                 const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
                  const float* __restrict__ g, const float* __restrict__ eta, float eps,
                  const float* __restrict__ ck, float* __restrict__ Tws, float* __restrict__ Vws,
+                 float* __restrict__ Wws, float* __restrict__ Xws, float* __restrict__ Yws,
                  int Tlen, int H, int nblk) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   auto& s = *reinterpret_cast<PrepSmem<DK, DV>*>(smem_raw);
@@ -212,6 +225,8 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __res
 
   load_rows_bf16<DK>(&s.kb[0][0], k + tok0 * DK, (size_t)H * DK, len);
   load_rows_bf16<DV>(&s.vb[0][0], v + tok0 * DV, (size_t)H * DV, len);
+  load_rows_bf16<DK>(&s.qb[0][0], q + tok0 * DK, (size_t)H * DK, len);
+  load_rows_bf16<DV>(&s.ob[0][0], dout + tok0 * DV, (size_t)H * DV, len);
   load_f32<DK, DV>(&s.h[0][0], ck + chunk * DK * DV, DV);
   __syncthreads();
   chunk_scalars<DK>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
@@ -241,13 +256,64 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __res
     auto Ta = [&](int r, int c) { return s.Tm[r][c]; };
     auto Kb = [&](int c, int i) { return s.beta[c] * s.gam[c] * bf(s.kb[c][i]); };
     mma_rows<DK / 16>(d, Ta, Kb, 16 * mt, (DK / 2) * nh, C, lane);
+    float* wdst = Wws + chunk * C * DK;
 #pragma unroll
     for (int nt = 0; nt < DK / 16; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        s.W[frow(16 * mt, lane, e)][fcol((DK / 2) * nh, nt, lane, e)] = d[nt][e];
+      for (int e = 0; e < 4; e += 2) {
+        const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
+        s.W[r][i] = d[nt][e];
+        s.W[r][i + 1] = d[nt][e + 1];
+        *reinterpret_cast<float2*>(wdst + r * DK + i) = make_float2(d[nt][e], d[nt][e + 1]);
+      }
+  }
+  {  // P = lower_incl(Q K^T (*) Gamma) over A (no longer read after the inverse)
+    float p[4][4];
+    zero(p);
+    auto Qa = [&](int r, int i) { return bf(s.qb[r][i]); };
+    auto Kb = [&](int i, int c) { return bf(s.kb[c][i]); };
+    mma_rows<4>(p, Qa, Kb, 16 * mt, 32 * nh, DK, lane);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
+        s.A[r][c] = c <= r ? p[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;
+      }
   }
   __syncthreads();
+  {  // Y = (diag(gamma) Q)^T dO  [DK x DV]: warp w has rows 16 w .., two column halves
+    auto QTa = [&](int i, int c) { return s.gam[c] * bf(s.qb[c][i]); };
+    auto Ob = [&](int c, int j) { return bf(s.ob[c][j]); };
+    float* ydst = Yws + chunk * DK * DV;
+    for (int half = 0; half < 2; ++half) {
+      float d[DV / 16][4];
+      zero(d);
+      mma_rows<DV / 16>(d, QTa, Ob, 16 * warp, half * (DV / 2), C, lane);
+#pragma unroll
+      for (int nt = 0; nt < DV / 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+          const int i = frow(16 * warp, lane, e), j = fcol(half * (DV / 2), nt, lane, e);
+          *reinterpret_cast<float2*>(ydst + i * DV + j) = make_float2(d[nt][e], d[nt][e + 1]);
+        }
+    }
+  }
+  {  // X = P^T dO  [C x DV]
+    float d[DV / 16][4];
+    zero(d);
+    auto PTa = [&](int r, int c) { return s.A[c][r]; };
+    auto Ob = [&](int c, int j) { return bf(s.ob[c][j]); };
+    mma_rows<DV / 16>(d, PTa, Ob, 16 * mt, (DV / 2) * nh, C, lane);
+    float* xdst = Xws + chunk * C * DV;
+#pragma unroll
+    for (int nt = 0; nt < DV / 16; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; e += 2) {
+        const int r = frow(16 * mt, lane, e), j = fcol((DV / 2) * nh, nt, lane, e);
+        *reinterpret_cast<float2*>(xdst + r * DV + j) = make_float2(d[nt][e], d[nt][e + 1]);
+      }
+  }
   {  // V' = T diag(beta) V - W h_n
     float d[DV / 16][4];
     zero(d);
@@ -273,29 +339,86 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __res
 }
 
 // ---------------------------------------------------------------- adjoint chain
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// One chunk's operands of the adjoint chain (the CTA's 32 columns of X, Y).
 template <int DK>
-struct AdjSmem {
+struct AdjBuf {
   __nv_bfloat16 kb[C][LB<DK>()];
-  __nv_bfloat16 qb[C][LB<DK>()];
-  __nv_bfloat16 ob[C][LB<BVA>()];
-  float Tm[C][LF<C>()];
   float W[C][LF<DK>()];
-  float P[C][LF<C>()];
-  float dH[DK][LF<BVA>()];
-  float dV[C][LF<BVA>()];
-  float G[C], gam[C], beta[C], n2[C], kts[C];
+  float X[C][LF<BVA>()];
+  float Y[DK][LF<BVA>()];
+  float g[C];
 };
 
-// One CTA per (head, 64-column slab); chunks in reverse.  dH (the adjoint of
+template <int DK>
+struct AdjSmem {
+  AdjBuf<DK> buf[2];
+  float dH[DK][LF<BVA>()];
+  float dV[C][LF<BVA>()];
+  float kts[C];
+  float gC;
+};
+
+// Copies of chunk n's operands into a buffer (zero rows past the sequence).
+template <int DK, int DV>
+__device__ __forceinline__ void adj_fetch(AdjBuf<DK>& d, const __nv_bfloat16* k,
+                                          const float* g, const float* Wws, const float* Xws,
+                                          const float* Yws, size_t head, int n, int nblk,
+                                          int j0, int b, int hh, int Tlen, int H) {
+  const size_t chunk = head * nblk + n;
+  const int t0 = n * C, len = min(C, Tlen - t0);
+  const size_t tok0 = ((size_t)b * Tlen + t0) * H + hh;
+  for (int p = threadIdx.x; p < C * (DK / 8); p += NT) {  // keys, bf16
+    const int r = p / (DK / 8), ch = p % (DK / 8);
+    const bool ok = r < len;
+    cp_async16(&d.kb[r][ch * 8], k + (ok ? (tok0 + (size_t)r * H) * DK + ch * 8 : 0), ok);
+  }
+  for (int p = threadIdx.x; p < C * (DK / 4); p += NT) {  // W
+    const int r = p / (DK / 4), ch = p % (DK / 4);
+    cp_async16(&d.W[r][ch * 4], Wws + (chunk * C + r) * DK + ch * 4, true);
+  }
+  for (int p = threadIdx.x; p < C * (BVA / 4); p += NT) {  // X columns j0 ..
+    const int r = p / (BVA / 4), ch = p % (BVA / 4);
+    cp_async16(&d.X[r][ch * 4], Xws + (chunk * C + r) * DV + j0 + ch * 4, true);
+  }
+  for (int p = threadIdx.x; p < DK * (BVA / 4); p += NT) {  // Y columns j0 ..
+    const int r = p / (BVA / 4), ch = p % (BVA / 4);
+    cp_async16(&d.Y[r][ch * 4], Yws + (chunk * DK + r) * DV + j0 + ch * 4, true);
+  }
+  if (threadIdx.x < C) {
+    const bool ok = (int)threadIdx.x < len;
+    cp_async4(&d.g[threadIdx.x], g + (ok ? tok0 + (size_t)threadIdx.x * H : 0), ok);
+  }
+  cp_async_commit();
+}
+
+// One CTA per (head, 32-column slab); chunks in reverse.  dH (the adjoint of
 // h_{n+1}) lives in registers: warp w holds rows 16 w .. 16 w + 15.
 template <int DK, int DV>
 __global__ void __launch_bounds__(NT)
-cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                    const __nv_bfloat16* __restrict__ dout, const float* __restrict__ g,
-                    const float* __restrict__ eta, float eps, const float* __restrict__ dhT,
-                    const float* __restrict__ Tws, float* __restrict__ dVws,
-                    float* __restrict__ dHws, float* __restrict__ dh0, int Tlen, int H,
-                    int nblk) {
+cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict__ g,
+                    const float* __restrict__ dhT, const float* __restrict__ Wws,
+                    const float* __restrict__ Xws, const float* __restrict__ Yws,
+                    float* __restrict__ dVws, float* __restrict__ dHws, float* __restrict__ dh0,
+                    int Tlen, int H, int nblk) {
   static_assert(DK == 128, "one 16-row tile of the state per warp");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   auto& s = *reinterpret_cast<AdjSmem<DK>*>(smem_raw);
@@ -312,18 +435,18 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
       acc[nt][e] = dhT ? dhT[(head * DK + frow(16 * warp, lane, e)) * DV + j0 +
                              fcol(0, nt, lane, e)]
                        : 0.f;
+  adj_fetch<DK, DV>(s.buf[(nblk - 1) & 1], k, g, Wws, Xws, Yws, head, nblk - 1, nblk, j0, b,
+                    hh, Tlen, H);
 
   for (int n = nblk - 1; n >= 0; --n) {
     const size_t chunk = head * nblk + n;
-    const int t0 = n * C, len = min(C, Tlen - t0);
-    const size_t tok0 = ((size_t)b * Tlen + t0) * H + hh;
-    __syncthreads();  // the previous chunk's tiles are no longer read
-    load_rows_bf16<DK>(&s.kb[0][0], k + tok0 * DK, (size_t)H * DK, len);
-    load_rows_bf16<DK>(&s.qb[0][0], q + tok0 * DK, (size_t)H * DK, len);
-    load_rows_bf16<BVA>(&s.ob[0][0], dout + tok0 * DV + j0, (size_t)H * DV, len);
-    load_f32<C, C>(&s.Tm[0][0], Tws + chunk * C * C, C);
-    // dH_{n+1}: to shared memory (operand) and to the workspace (for the
-    // gradient kernel)
+    AdjBuf<DK>& cur = s.buf[n & 1];
+    cp_async_wait_all();
+    __syncthreads();  // chunk n's operands are in; the previous chunk is done
+    if (n > 0)
+      adj_fetch<DK, DV>(s.buf[(n - 1) & 1], k, g, Wws, Xws, Yws, head, n - 1, nblk, j0, b, hh,
+                        Tlen, H);
+    // dH_{n+1}: to shared memory (operand) and to the workspace
 #pragma unroll
     for (int nt = 0; nt < BVA / 8; ++nt)
 #pragma unroll
@@ -334,51 +457,36 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
         *reinterpret_cast<float2*>(dHws + (chunk * DK + r) * DV + j0 + c) =
             make_float2(acc[nt][e], acc[nt][e + 1]);
       }
-    __syncthreads();
-    chunk_scalars<DK>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
-    __syncthreads();
-    if (tid < C) s.kts[tid] = __expf(s.G[C - 1] - s.G[tid]);
-    const int mt = warp & 3, nh = warp >> 2;
-    {  // W = T diag(beta gamma) K;  P = lower_incl(Q K^T (*) Gamma)
-      float d[DK / 16][4];
-      zero(d);
-      auto Ta = [&](int r, int c) { return s.Tm[r][c]; };
-      auto Kb = [&](int c, int i) { return s.beta[c] * s.gam[c] * bf(s.kb[c][i]); };
-      mma_rows<DK / 16>(d, Ta, Kb, 16 * mt, (DK / 2) * nh, C, lane);
+    if (warp == 0) {  // G (in-chunk cumsum) -> e^{G_last - G_r}, e^{G_last}
+      const float x0 = cur.g[2 * lane], x1 = cur.g[2 * lane + 1];
+      float sum = x0 + x1;
 #pragma unroll
-      for (int nt = 0; nt < DK / 16; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          s.W[frow(16 * mt, lane, e)][fcol((DK / 2) * nh, nt, lane, e)] = d[nt][e];
-      float p[4][4];
-      zero(p);
-      auto Qa = [&](int r, int i) { return bf(s.qb[r][i]); };
-      auto Kt = [&](int i, int c) { return bf(s.kb[c][i]); };
-      mma_rows<4>(p, Qa, Kt, 16 * mt, 32 * nh, DK, lane);
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
-          s.P[r][c] = c <= r ? p[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;
-        }
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, sum, o);
+        if (lane >= o) sum += y;
+      }
+      const float last = __shfl_sync(0xffffffffu, sum, 31);
+      s.kts[2 * lane] = __expf(last - (sum - x1));
+      s.kts[2 * lane + 1] = __expf(last - sum);
+      if (lane == 0) s.gC = __expf(last);
     }
     __syncthreads();
-    const float gC = s.gam[C - 1];
-    {  // dV' = P^T dO + Kt dH_{n+1}   [C x 64]
-      float d[4][4];
-      zero(d);
-      auto PTa = [&](int r, int c) { return s.P[c][r]; };
-      auto Ob = [&](int c, int j) { return bf(s.ob[c][j]); };
-      mma_rows<4>(d, PTa, Ob, 16 * mt, 32 * nh, C, lane);
-      auto Kta = [&](int r, int i) { return s.kts[r] * bf(s.kb[r][i]); };
-      auto Hb = [&](int i, int j) { return s.dH[i][j]; };
-      mma_rows<4>(d, Kta, Hb, 16 * mt, 32 * nh, DK, lane);
+    const int mt = warp & 3, nq = warp >> 2;
+    {  // dV' = X + Kt dH_{n+1}   [C x 32]: warp (mt, nq) has 2 column tiles
+      float d[2][4];
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          d[nt][e] = cur.X[frow(16 * mt, lane, e)][fcol(16 * nq, nt, lane, e)];
+      auto Kta = [&](int r, int i) { return s.kts[r] * bf(cur.kb[r][i]); };
+      auto Hb = [&](int i, int j) { return s.dH[i][j]; };
+      mma_rows<2>(d, Kta, Hb, 16 * mt, 16 * nq, DK, lane);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; e += 2) {
-          const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
+          const int r = frow(16 * mt, lane, e), c = fcol(16 * nq, nt, lane, e);
           s.dV[r][c] = d[nt][e];
           s.dV[r][c + 1] = d[nt][e + 1];
           *reinterpret_cast<float2*>(dVws + (chunk * C + r) * DV + j0 + c) =
@@ -386,15 +494,15 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
         }
     }
     __syncthreads();
-    {  // dH_n = gamma_C dH_{n+1} + (diag(gamma) Q)^T dO - W^T dV'
+    {  // dH_n = gamma_C dH_{n+1} + Y - W^T dV'
+      const float gC = s.gC;
 #pragma unroll
       for (int nt = 0; nt < BVA / 8; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][e] *= gC;
-      auto QTa = [&](int i, int c) { return s.gam[c] * bf(s.qb[c][i]); };
-      auto Ob = [&](int c, int j) { return bf(s.ob[c][j]); };
-      mma_rows<BVA / 8>(acc, QTa, Ob, 16 * warp, 0, C, lane);
-      auto WTa = [&](int i, int c) { return -s.W[c][i]; };
+        for (int e = 0; e < 4; ++e)
+          acc[nt][e] = fmaf(gC, acc[nt][e],
+                            cur.Y[frow(16 * warp, lane, e)][fcol(0, nt, lane, e)]);
+      auto WTa = [&](int i, int c) { return -cur.W[c][i]; };
       auto dVb = [&](int c, int j) { return s.dV[c][j]; };
       mma_rows<BVA / 8>(acc, WTa, dVb, 16 * warp, 0, C, lane);
     }
@@ -788,21 +896,26 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct CbwdWs {
-  size_t ck, Tm, Vp, dVp, dH, beta, alpha, total;
+  size_t ck, Tm, Vp, dVp, dH, W, X, Y, fwd, fwd_bytes, total;
 };
 
+// h_n, T, V', dV', dH_{n+1}, W, X, Y per chunk (fp32), then the forward
+// prefill's own workspace (UT factors and, where the chain is cut, segment
+// states).
 static CbwdWs cbwd_layout(int B, int T, int H, int dk, int dv) {
   const size_t nblk = ((size_t)T + C - 1) / C, chunks = (size_t)B * H * nblk;
-  const size_t ntok = (size_t)B * T * H;
   CbwdWs w;
   w.ck = 0;
   w.Tm = w.ck + al256(chunks * dk * dv * 4);
   w.Vp = w.Tm + al256(chunks * C * C * 4);
   w.dVp = w.Vp + al256(chunks * C * dv * 4);
   w.dH = w.dVp + al256(chunks * C * dv * 4);
-  w.beta = w.dH + al256(chunks * dk * dv * 4);
-  w.alpha = w.beta + al256(ntok * 4);
-  w.total = w.alpha + al256(ntok * 4);
+  w.W = w.dH + al256(chunks * dk * dv * 4);
+  w.X = w.W + al256(chunks * C * dk * 4);
+  w.Y = w.X + al256(chunks * C * dv * 4);
+  w.fwd = w.Y + al256(chunks * dk * dv * 4);
+  w.fwd_bytes = chunk_workspace_bytes(B, T, H, dk, dv, KLA_BF16);
+  w.total = w.fwd + al256(w.fwd_bytes);
   return w;
 }
 
@@ -811,18 +924,11 @@ size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
   return cbwd_layout(B, T, H, dk, dv).total;
 }
 
-// The checkpoint kernel of kla_backward.cu (h at every 64-token block start,
-// every token's beta and alpha).
-cudaError_t launch_bwd_checkpoints(const void* k, const void* v, const float* g,
-                                   const float* eta, float eps, const float* h0, float* ck,
-                                   float* beta_out, float* alpha_out, int B, int T, int H,
-                                   int dk, int dv, int dtype, cudaStream_t st);
-
 cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
                              const float* eta, float eps, const float* h0, const void* dout,
                              const float* dhT, float* dq, float* dk, float* dv, float* dg,
                              float* deta, float* dh0, int B, int Tlen, int H, int dkd, int dvd,
-                             void* ws, cudaStream_t st) {
+                             void* ws, unsigned int* err, cudaStream_t st) {
   constexpr int DK = 128, DV = 128;
   if (dkd != DK || dvd != DV) return cudaErrorInvalidValue;
   const CbwdWs w = cbwd_layout(B, Tlen, H, DK, DV);
@@ -832,10 +938,13 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
   float* Vws = (float*)(base + w.Vp);
   float* dVws = (float*)(base + w.dVp);
   float* dHws = (float*)(base + w.dH);
+  float* Wws = (float*)(base + w.W);
+  float* Xws = (float*)(base + w.X);
+  float* Yws = (float*)(base + w.Y);
   const int nblk = (Tlen + C - 1) / C;
-  cudaError_t e = launch_bwd_checkpoints(k, v, g, eta, eps, h0, ck, (float*)(base + w.beta),
-                                         (float*)(base + w.alpha), B, Tlen, H, DK, DV,
-                                         KLA_BF16, st);
+  // the forward chunk prefill, outputs off, leaves every h_n in ck
+  cudaError_t e = launch_chunk_tc(q, k, v, g, eta, eps, h0, nullptr, nullptr, B, Tlen, H, DK,
+                                  DV, base + w.fwd, w.fwd_bytes, err, st, ck);
   if (e != cudaSuccess) return e;
   const auto* qb = (const __nv_bfloat16*)q;
   const auto* kb = (const __nv_bfloat16*)k;
@@ -851,10 +960,10 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
       (e = cudaFuncSetAttribute(cbwd_grad_kernel<DK, DV>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg)))
     return e;
-  cbwd_prep_kernel<DK, DV><<<dim3(nblk, H, B), NT, sp, st>>>(kb, vb, g, eta, eps, ck, Tws, Vws,
-                                                             Tlen, H, nblk);
+  cbwd_prep_kernel<DK, DV><<<dim3(nblk, H, B), NT, sp, st>>>(
+      qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, Wws, Xws, Yws, Tlen, H, nblk);
   cbwd_adjoint_kernel<DK, DV><<<dim3(DV / BVA, H, B), NT, sa, st>>>(
-      qb, kb, ob, g, eta, eps, dhT, Tws, dVws, dHws, dh0, Tlen, H, nblk);
+      kb, g, dhT, Wws, Xws, Yws, dVws, dHws, dh0, Tlen, H, nblk);
   cbwd_grad_kernel<DK, DV><<<dim3(nblk, H, B), NT, sg, st>>>(
       qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, dVws, dHws, dq, dk, dv, dg, deta, Tlen, H,
       nblk);

@@ -145,9 +145,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
              const float* __restrict__ h0, __nv_bfloat16* __restrict__ o,
-             float* __restrict__ hT, float* __restrict__ phi, int T, int H, int DV,
-             int nseg, int seg_chunks, int mode, const uint8_t* __restrict__ ws,
-             unsigned int* err) {
+             float* __restrict__ hT, float* __restrict__ phi, float* __restrict__ hs, int T,
+             int H, int DV, int nseg, int seg_chunks, int mode,
+             const uint8_t* __restrict__ ws, unsigned int* err) {
   using Smem = ChainSmem<DK>;
   constexpr int NP = Stage<DK>::NP;
   constexpr uint32_t PANEL = 3 * 8192;  // byte stride between key panels
@@ -168,7 +168,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   // last segment writes h_T to hT[head].  mode 1 (segment transitions, no
   // outputs): slabs below DV / BV run from a zero state and leave the end
   // state E in hT[sidx]; the others propagate the identity with V = 0 and
-  // leave Phi (the segment's transition, [DK][DK]) in phi[sidx].
+  // leave Phi (the segment's transition, [DK][DK]) in phi[sidx].  hs (mode 0,
+  // nullable): the fp32 state at the start of every chunk,
+  // [B][H][nchunks][DK][DV].  o may be NULL (no outputs written).
   const int nvs = DV / BV;
   const bool phi_slab = mode == 1 && (int)blockIdx.x >= nvs;
   const int slab = phi_slab ? (int)blockIdx.x - nvs : (int)blockIdx.x;
@@ -548,6 +550,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const bool v_rows = row < 64;
     bool ok = true;
     for (int n = 0; n < nchunks && ok; ++n) {
+      if (hs && mode == 0 && has_h) {  // h at the start of chunk n0 + n
+        float4* dst = reinterpret_cast<float4*>(
+            hs + ((head * nchunks_all + n0 + n) * DK + row) * DV + slab * BV + cg);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
+      }
       const float* Gn = s.G[n % 3];
       const uint32_t par = (uint32_t)(n & 1);
       const uint32_t col_u = COL_U + 64 * (n & 1);
@@ -624,7 +633,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           mbar_arrive(&s.u_free[n & 1]);
           mbar_arrive(&s.pv_free);
         }
-        if (t < T && mode == 0) {
+        if (t < T && mode == 0 && o) {
           uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * T + t) * H + hh) * DV +
                                                 slab * BV + cg);
 #pragma unroll
@@ -743,7 +752,8 @@ template <int DK, bool KDA>
 cudaError_t launch_chain_dk(const void* q, const void* k, const void* v, const float* g,
                             const float* h0, void* o, float* hT, float* phi, int B, int T,
                             int H, int DV, int nseg, int seg_chunks, int mode,
-                            const uint8_t* ws, unsigned int* err, cudaStream_t st) {
+                            const uint8_t* ws, unsigned int* err, cudaStream_t st,
+                            float* hs = nullptr) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, DK, H, T, B) || !make_map(&mk, k, DK, H, T, B) ||
       !make_map(&mv, v, DV, H, T, B))
@@ -761,8 +771,8 @@ cudaError_t launch_chain_dk(const void* q, const void* k, const void* v, const f
   }
   dim3 grid((mode == 1 ? DV + DK : DV) / BV, H, B * nseg);
   chain_kernel<DK, KDA><<<grid, NTHREADS, smem, st>>>(mq, mk, mv, g, h0, (__nv_bfloat16*)o, hT,
-                                                      phi, T, H, DV, nseg, seg_chunks, mode, ws,
-                                                      err);
+                                                      phi, hs, T, H, DV, nseg, seg_chunks, mode,
+                                                      ws, err);
   return cudaGetLastError();
 }
 
@@ -846,12 +856,12 @@ template <int DK, bool KDA>
 static cudaError_t launch_segmented(const void* q, const void* k, const void* v, const float* g,
                                     const float* h0, void* o, float* hT, int B, int T, int H,
                                     int sg, uint8_t* ws, size_t tiles, unsigned int* err,
-                                    cudaStream_t st);
+                                    cudaStream_t st, float* hs = nullptr);
 
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, const float* g,
                                const float* h0, void* o, float* hT, int B, int T, int H,
                                int dk, int dv, void* workspace, size_t ws_bytes,
-                               unsigned int* err, cudaStream_t st) {
+                               unsigned int* err, cudaStream_t st, float* hs) {
   if (dk != dv) return cudaErrorNotSupported;
   const int sg = chunk_chain_segments(B, T, H, dk, dv, ws_bytes);
   if (sg > 1) {
@@ -859,17 +869,18 @@ cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, cons
     const size_t tiles = ut_workspace_bytes(B, T, H);
     if (dk == 128)
       return launch_segmented<128, false>(q, k, v, g, h0, o, hT, B, T, H, sg, wsm, tiles, err,
-                                          st);
-    return launch_segmented<64, false>(q, k, v, g, h0, o, hT, B, T, H, sg, wsm, tiles, err, st);
+                                          st, hs);
+    return launch_segmented<64, false>(q, k, v, g, h0, o, hT, B, T, H, sg, wsm, tiles, err, st,
+                                       hs);
   }
   const uint8_t* ws = (const uint8_t*)workspace;
   const int nchunks = (T + C - 1) / C;
   if (dk == 128)
     return launch_chain_dk<128, false>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks,
-                                       0, ws, err, st);
+                                       0, ws, err, st, hs);
   if (dk == 64)
     return launch_chain_dk<64, false>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks,
-                                      0, ws, err, st);
+                                      0, ws, err, st, hs);
   return cudaErrorNotSupported;
 }
 
@@ -877,7 +888,7 @@ template <int DK, bool KDA>
 static cudaError_t launch_segmented(const void* q, const void* k, const void* v, const float* g,
                                     const float* h0, void* o, float* hT, int B, int T, int H,
                                     int sg, uint8_t* ws, size_t tiles, unsigned int* err,
-                                    cudaStream_t st) {
+                                    cudaStream_t st, float* hs) {
   constexpr int DV = DK;
   const int nchunks = (T + C - 1) / C;
   const int len = (nchunks + sg - 1) / sg;
@@ -894,18 +905,18 @@ static cudaError_t launch_segmented(const void* q, const void* k, const void* v,
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_chain_dk<DK, KDA>(q, k, v, g, hstart, o, hT, nullptr, B, T, H, DV, sg, len, 0,
-                                  ws, err, st);
+                                  ws, err, st, hs);
 }
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                             const float* eta, float eps, const float* h0, void* o, float* hT,
                             int B, int T, int H, int dk, int dv, void* workspace,
-                            size_t ws_bytes, unsigned int* err, cudaStream_t st) {
+                            size_t ws_bytes, unsigned int* err, cudaStream_t st, float* hs) {
   if (dk != dv || (dk != 64 && dk != 128)) return cudaErrorNotSupported;
   cudaError_t e = launch_chunk_ut(k, g, eta, eps, B, T, H, dk, workspace, err, st);
   if (e != cudaSuccess) return e;
   return launch_chunk_chain(q, k, v, g, h0, o, hT, B, T, H, dk, dv, workspace, ws_bytes, err,
-                            st);
+                            st, hs);
 }
 
 // ---------------------------------------------------- per-channel gate

@@ -55,7 +55,7 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
                              const float* eta, float eps, const float* h0, const void* dout,
                              const float* dhT, float* dq, float* dk, float* dv, float* dg,
                              float* deta, float* dh0, int B, int T, int H, int dkd, int dvd,
-                             void* ws, cudaStream_t st);
+                             void* ws, unsigned int* err, cudaStream_t st);
 
 template <typename T> struct IO;
 

@@ -300,12 +300,13 @@ KLA_API kla_status kla_recurrent_bwd(const void *q, const void *k, const void *v
  * gradient is per-chunk work on warp-level tensor-core products (tf32
  * operands, fp32 sums): dQ, dK from P, W, U = T diag(beta) V and
  * T = (I + A)^{-1} (dA = -strict_lower(T^T dT T^T)), dg as the reverse
- * in-chunk cumsum of dG.  The states h_n come from a token-serial fp32
- * forward.  bf16 with dk = dv = 128 runs these kernels (accuracy of tf32
- * products: relative L2 about 1e-3); fp32 I/O and d = 64 run the
- * token-serial kernels of kla_recurrent_bwd.  Workspace:
- * kla_chunk_bwd_workspace_size(...) bytes (for the chunk kernels about
- * B*H*ceil(T/64) * 208 KiB).
+ * in-chunk cumsum of dG.  The states h_n come from the forward chunk
+ * prefill (the kernels of kla_chunk_fwd, outputs off, its state chain
+ * writing every h_n).  bf16 with dk = dv = 128 runs these kernels (relative
+ * L2 of the gradients about 1e-3: bf16 state chain, tf32 products); fp32
+ * I/O and d = 64 run the token-serial kernels of kla_recurrent_bwd.
+ * Workspace: kla_chunk_bwd_workspace_size(...) bytes (for the chunk kernels
+ * about B*H*ceil(T/64) * 224 KiB).
  */
 KLA_API size_t kla_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int dtype);
 KLA_API kla_status kla_chunk_bwd(const void *q, const void *k, const void *v,
