@@ -102,29 +102,54 @@ __device__ __forceinline__ float bf(const __nv_bfloat16& x) { return __bfloat162
 template <int D> constexpr int LF() { return D + 4; }
 template <int D> constexpr int LB() { return D + 8; }
 
-// Copy n rows of a [rows][D] bf16 matrix with row stride rs (elements) into
-// a padded tile (rows >= n zero-filled up to C).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Asynchronous copy of n rows of a [rows][D] bf16 matrix with row stride rs
+// (elements) into a padded tile (rows >= n zero-filled up to C); complete
+// after cp_async_commit + cp_async_wait_all.
 template <int D>
 __device__ __forceinline__ void load_rows_bf16(__nv_bfloat16* dst, const __nv_bfloat16* src,
                                                size_t rs, int n) {
   constexpr int PR = D / 8;  // 16-byte pieces per row
   for (int p = threadIdx.x; p < C * PR; p += NT) {
     const int r = p / PR, ch = p % PR;
-    uint4 x = make_uint4(0, 0, 0, 0);
-    if (r < n) x = *reinterpret_cast<const uint4*>(src + r * rs + ch * 8);
-    *reinterpret_cast<uint4*>(dst + r * LB<D>() + ch * 8) = x;
+    const bool ok = r < n;
+    cp_async16(dst + r * LB<D>() + ch * 8, ok ? src + r * rs + ch * 8 : src, ok);
   }
 }
 
-// Copy a [R][D] fp32 block (row stride rs) into a padded tile.
+// Asynchronous copy of a [R][D] fp32 block (row stride rs) into a padded tile.
 template <int R, int D>
 __device__ __forceinline__ void load_f32(float* dst, const float* src, size_t rs) {
   constexpr int PR = D / 4;
   for (int p = threadIdx.x; p < R * PR; p += NT) {
     const int r = p / PR, ch = p % PR;
-    *reinterpret_cast<float4*>(dst + r * LF<D>() + ch * 4) =
-        *reinterpret_cast<const float4*>(src + r * rs + ch * 4);
+    cp_async16(dst + r * LF<D>() + ch * 4, src + r * rs + ch * 4, true);
   }
+}
+
+// Wait for this thread's copies, then for the whole CTA's.
+__device__ __forceinline__ void copies_landed() {
+  cp_async_commit();
+  cp_async_wait_all();
+  __syncthreads();
 }
 
 // Per-chunk scalars: G (in-chunk cumsum of g), gamma = e^G, beta, ||k||^2,
@@ -228,7 +253,7 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   load_rows_bf16<DK>(&s.qb[0][0], q + tok0 * DK, (size_t)H * DK, len);
   load_rows_bf16<DV>(&s.ob[0][0], dout + tok0 * DV, (size_t)H * DV, len);
   load_f32<DK, DV>(&s.h[0][0], ck + chunk * DK * DV, DV);
-  __syncthreads();
+  copies_landed();
   chunk_scalars<DK>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
   __syncthreads();
 
@@ -339,25 +364,6 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 }
 
 // ---------------------------------------------------------------- adjoint chain
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src),
-               "r"(valid ? 4 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
-
 // One chunk's operands of the adjoint chain (the CTA's 32 columns of X, Y).
 template <int DK>
 struct AdjBuf {
@@ -575,7 +581,7 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   load_f32<C, DV>(&s.Vp[0][0], Vws + chunk * C * DV, DV);
   load_f32<C, DV>(&s.dVp[0][0], dVws + chunk * C * DV, DV);
   if (tid < C) s.dG[tid] = s.dB[tid] = 0.f;
-  __syncthreads();
+  copies_landed();
   chunk_scalars<DK>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
   __syncthreads();
   if (tid < C) s.kts[tid] = __expf(s.G[C - 1] - s.G[tid]);
@@ -589,7 +595,7 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   for (int half = 0; half < 2; ++half) {
     __syncthreads();
     load_f32<DK, HALF>(&s.big[0][0], hn + half * HALF, DV);
-    __syncthreads();
+    copies_landed();
     // dO h_n^T and -dV' h_n^T over this half of the dv index
     auto Oa = [&](int r, int j) { return bf(s.ob[r][half * HALF + j]); };
     auto dVa = [&](int r, int j) { return -s.dVp[r][half * HALF + j]; };
@@ -609,9 +615,20 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         rowO[e >> 1] += o[nt][e] * bf(s.ob[frow(16 * mt, lane, e)]
                                           [half * HALF + fcol(32 * nh, nt, lane, e)]);
   }
-  // <dH_{n+1}, h_n> (block sum, fixed order)
+  // <dH_{n+1}, h_n> (block sum, fixed order; every load issued up front)
   float hd = 0.f;
-  for (int p = tid; p < DK * DV; p += NT) hd = fmaf(hn[p], dHn[p], hd);
+  {
+    constexpr int NV = DK * DV / 4 / NT;  // float4 pieces per thread
+    float4 a[NV], c[NV];
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+      a[u] = reinterpret_cast<const float4*>(hn)[tid + u * NT];
+      c[u] = reinterpret_cast<const float4*>(dHn)[tid + u * NT];
+    }
+#pragma unroll
+    for (int u = 0; u < NV; ++u)
+      hd = fmaf(a[u].x, c[u].x, fmaf(a[u].y, c[u].y, fmaf(a[u].z, c[u].z, fmaf(a[u].w, c[u].w, hd))));
+  }
   hd = warp_sum(hd);
   if (lane == 0) s.red[warp] = hd;
   // rowO -> dG (two warps per row tile: nh = 0 writes part[0], nh = 1 part[1])
@@ -827,7 +844,7 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   for (int half = 0; half < 2; ++half) {
     __syncthreads();  // big (dW, or the other half of dH) is no longer read
     load_f32<DK, HALF>(&s.big[0][0], dHn + half * HALF, DV);
-    __syncthreads();
+    copies_landed();
     auto Va = [&](int r, int j) { return s.Vp[r][half * HALF + j]; };
     auto HTb = [&](int j, int i) { return s.big[i][j]; };
     mma_rows<DK / 16>(dKt, Va, HTb, 16 * mt, (DK / 2) * nh, HALF, lane);
