@@ -124,11 +124,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // Asynchronous copy of n rows of a [rows][D] bf16 matrix with row stride rs
 // (elements) into a padded tile (rows >= n zero-filled up to C); complete
 // after cp_async_commit + cp_async_wait_all.
-template <int D>
+template <int D, int NTH = NT>
 __device__ __forceinline__ void load_rows_bf16(__nv_bfloat16* dst, const __nv_bfloat16* src,
                                                size_t rs, int n) {
   constexpr int PR = D / 8;  // 16-byte pieces per row
-  for (int p = threadIdx.x; p < C * PR; p += NT) {
+  for (int p = threadIdx.x; p < C * PR; p += NTH) {
     const int r = p / PR, ch = p % PR;
     const bool ok = r < n;
     cp_async16(dst + r * LB<D>() + ch * 8, ok ? src + r * rs + ch * 8 : src, ok);
@@ -136,10 +136,10 @@ __device__ __forceinline__ void load_rows_bf16(__nv_bfloat16* dst, const __nv_bf
 }
 
 // Asynchronous copy of a [R][D] fp32 block (row stride rs) into a padded tile.
-template <int R, int D>
+template <int R, int D, int NTH = NT>
 __device__ __forceinline__ void load_f32(float* dst, const float* src, size_t rs) {
   constexpr int PR = D / 4;
-  for (int p = threadIdx.x; p < R * PR; p += NT) {
+  for (int p = threadIdx.x; p < R * PR; p += NTH) {
     const int r = p / PR, ch = p % PR;
     cp_async16(dst + r * LF<D>() + ch * 4, src + r * rs + ch * 4, true);
   }
@@ -156,13 +156,13 @@ __device__ __forceinline__ void copies_landed() {
 // from the staged keys (rows >= n: g = 0, beta = 0).  Decay ratios are only
 // ever formed as e^{difference} (gamma_C / gamma_r as e^{G_last - G_r}): with
 // strong gates e^G itself underflows to 0 inside a chunk.
-template <int DK>
+template <int DK, int NTH = NT>
 __device__ __forceinline__ void chunk_scalars(float* G, float* gam, float* beta, float* n2,
                                               const __nv_bfloat16* kb, const float* g,
                                               const float* eta, float eps, size_t tok0,
                                               size_t tstride, int n) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int r = warp; r < C; r += NT / 32) {
+  for (int r = warp; r < C; r += NTH / 32) {
     float a = 0.f;
     for (int i = lane; i < DK; i += 32) {
       const float x = bf(kb[r * LB<DK>() + i]);
@@ -538,8 +538,8 @@ struct GradSmem {
   float X2[C][LF<C>()];
   float G[C], gam[C], beta[C], n2[C], kts[C];
   float dG[C], dB[C];
-  float part[2][C];  // per-row partial sums of the two warps sharing a row tile
-  float red[NT / 32];
+  float part[4][C];  // per-row partial sums of the four warps sharing a row tile
+  float red[16];
 };
 
 // Sum a per-row value over the 4 lanes holding one fragment row (t), then the
@@ -550,8 +550,10 @@ __device__ __forceinline__ float quad_sum(float x) {
   return x;
 }
 
+constexpr int GT = 512;  // threads of the gradient kernel: 16 warps, 4 per row tile
+
 template <int DK, int DV>
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(GT)
 cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                  const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
                  const float* __restrict__ g, const float* __restrict__ eta, float eps,
@@ -568,62 +570,62 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   const size_t head = (size_t)b * H + hh, chunk = head * nblk + n;
   const int t0 = n * C, len = min(C, Tlen - t0);
   const size_t tok0 = ((size_t)b * Tlen + t0) * H + hh;
-  const int mt = warp & 3, nh = warp >> 2;
+  const int mt = warp & 3, nq = warp >> 2;  // row tile; column quarter
   constexpr int HALF = DV / 2;
   const float* hn = ck + chunk * DK * DV;
   const float* dHn = dHws + chunk * DK * DV;
 
-  load_rows_bf16<DK>(&s.qb[0][0], q + tok0 * DK, (size_t)H * DK, len);
-  load_rows_bf16<DK>(&s.kb[0][0], k + tok0 * DK, (size_t)H * DK, len);
-  load_rows_bf16<DV>(&s.vb[0][0], v + tok0 * DV, (size_t)H * DV, len);
-  load_rows_bf16<DV>(&s.ob[0][0], dout + tok0 * DV, (size_t)H * DV, len);
-  load_f32<C, C>(&s.Tm[0][0], Tws + chunk * C * C, C);
-  load_f32<C, DV>(&s.Vp[0][0], Vws + chunk * C * DV, DV);
-  load_f32<C, DV>(&s.dVp[0][0], dVws + chunk * C * DV, DV);
+  load_rows_bf16<DK, GT>(&s.qb[0][0], q + tok0 * DK, (size_t)H * DK, len);
+  load_rows_bf16<DK, GT>(&s.kb[0][0], k + tok0 * DK, (size_t)H * DK, len);
+  load_rows_bf16<DV, GT>(&s.vb[0][0], v + tok0 * DV, (size_t)H * DV, len);
+  load_rows_bf16<DV, GT>(&s.ob[0][0], dout + tok0 * DV, (size_t)H * DV, len);
+  load_f32<C, C, GT>(&s.Tm[0][0], Tws + chunk * C * C, C);
+  load_f32<C, DV, GT>(&s.Vp[0][0], Vws + chunk * C * DV, DV);
+  load_f32<C, DV, GT>(&s.dVp[0][0], dVws + chunk * C * DV, DV);
   if (tid < C) s.dG[tid] = s.dB[tid] = 0.f;
   copies_landed();
-  chunk_scalars<DK>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
+  chunk_scalars<DK, GT>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
   __syncthreads();
   if (tid < C) s.kts[tid] = __expf(s.G[C - 1] - s.G[tid]);
   const float gC = s.gam[C - 1];
 
   // ---- phase 1: products with h_n, one 64-column half of it at a time
-  float accQ[DK / 16][4], accW[DK / 16][4];  // rows 16 mt .., columns (DK/2) nh ..
+  float accQ[DK / 32][4], accW[DK / 32][4];  // rows 16 mt .., columns (DK/4) nq ..
   zero(accQ);
   zero(accW);
   float rowO[2] = {0.f, 0.f};  // rowdot(dO, diag(gamma) Q h_n) for rows g, g + 8
   for (int half = 0; half < 2; ++half) {
     __syncthreads();
-    load_f32<DK, HALF>(&s.big[0][0], hn + half * HALF, DV);
+    load_f32<DK, HALF, GT>(&s.big[0][0], hn + half * HALF, DV);
     copies_landed();
     // dO h_n^T and -dV' h_n^T over this half of the dv index
     auto Oa = [&](int r, int j) { return bf(s.ob[r][half * HALF + j]); };
     auto dVa = [&](int r, int j) { return -s.dVp[r][half * HALF + j]; };
     auto HTb = [&](int j, int i) { return s.big[i][j]; };
-    mma_rows<DK / 16>(accQ, Oa, HTb, 16 * mt, (DK / 2) * nh, HALF, lane);
-    mma_rows<DK / 16>(accW, dVa, HTb, 16 * mt, (DK / 2) * nh, HALF, lane);
+    mma_rows<DK / 32>(accQ, Oa, HTb, 16 * mt, (DK / 4) * nq, HALF, lane);
+    mma_rows<DK / 32>(accW, dVa, HTb, 16 * mt, (DK / 4) * nq, HALF, lane);
     // diag(gamma) Q h_n on this half's columns: 64 x 64, 4 tiles per warp
-    float o[4][4];
+    float o[2][4];
     zero(o);
     auto Qa = [&](int r, int i) { return s.gam[r] * bf(s.qb[r][i]); };
     auto Hb = [&](int i, int j) { return s.big[i][j]; };
-    mma_rows<4>(o, Qa, Hb, 16 * mt, 32 * nh, DK, lane);
+    mma_rows<2>(o, Qa, Hb, 16 * mt, 16 * nq, DK, lane);
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         rowO[e >> 1] += o[nt][e] * bf(s.ob[frow(16 * mt, lane, e)]
-                                          [half * HALF + fcol(32 * nh, nt, lane, e)]);
+                                          [half * HALF + fcol(16 * nq, nt, lane, e)]);
   }
   // <dH_{n+1}, h_n> (block sum, fixed order; every load issued up front)
   float hd = 0.f;
   {
-    constexpr int NV = DK * DV / 4 / NT;  // float4 pieces per thread
+    constexpr int NV = DK * DV / 4 / GT;  // float4 pieces per thread
     float4 a[NV], c[NV];
 #pragma unroll
     for (int u = 0; u < NV; ++u) {
-      a[u] = reinterpret_cast<const float4*>(hn)[tid + u * NT];
-      c[u] = reinterpret_cast<const float4*>(dHn)[tid + u * NT];
+      a[u] = reinterpret_cast<const float4*>(hn)[tid + u * GT];
+      c[u] = reinterpret_cast<const float4*>(dHn)[tid + u * GT];
     }
 #pragma unroll
     for (int u = 0; u < NV; ++u)
@@ -631,39 +633,39 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   }
   hd = warp_sum(hd);
   if (lane == 0) s.red[warp] = hd;
-  // rowO -> dG (two warps per row tile: nh = 0 writes part[0], nh = 1 part[1])
+  // rowO -> dG (four warps per row tile, warp quarter nq writes part[nq])
 #pragma unroll
   for (int hr = 0; hr < 2; ++hr) {
     const float x = quad_sum(rowO[hr]);
-    if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+    if ((lane & 3) == 0) s.part[nq][16 * mt + (lane >> 2) + 8 * hr] = x;
   }
   __syncthreads();
-  if (tid < C) s.dG[tid] += s.part[0][tid] + s.part[1][tid];
+  if (tid < C) s.dG[tid] += s.part[0][tid] + s.part[1][tid] + s.part[2][tid] + s.part[3][tid];
   // dq (first part) stays in accQ; dW -> big as [C][DK]
   float* dW = &s.big[0][0];  // [C][LF<DK>] fits in [DK][LF<DV/2>]
   static_assert(C * LF<DK>() <= DK * LF<DV / 2>(), "dW in big");
 #pragma unroll
-  for (int nt = 0; nt < DK / 16; ++nt)
+  for (int nt = 0; nt < DK / 32; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      dW[frow(16 * mt, lane, e) * LF<DK>() + fcol((DK / 2) * nh, nt, lane, e)] = accW[nt][e];
+      dW[frow(16 * mt, lane, e) * LF<DK>() + fcol((DK / 4) * nq, nt, lane, e)] = accW[nt][e];
 
   // ---- phase 2: the C x C quantities
   {  // dP = dO V'^T (*) incl -> X1;  Q K^T -> X2
-    float d[4][4], p[4][4];
+    float d[2][4], p[2][4];
     zero(d);
     zero(p);
     auto Oa = [&](int r, int j) { return bf(s.ob[r][j]); };
     auto VTb = [&](int j, int c) { return s.Vp[c][j]; };
-    mma_rows<4>(d, Oa, VTb, 16 * mt, 32 * nh, DV, lane);
+    mma_rows<2>(d, Oa, VTb, 16 * mt, 16 * nq, DV, lane);
     auto Qa = [&](int r, int i) { return bf(s.qb[r][i]); };
     auto KTb = [&](int i, int c) { return bf(s.kb[c][i]); };
-    mma_rows<4>(p, Qa, KTb, 16 * mt, 32 * nh, DK, lane);
+    mma_rows<2>(p, Qa, KTb, 16 * mt, 16 * nq, DK, lane);
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
+        const int r = frow(16 * mt, lane, e), c = fcol(16 * nq, nt, lane, e);
         const bool in = c <= r;
         s.X1[r][c] = in ? d[nt][e] : 0.f;
         s.X2[r][c] = in ? p[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;  // P
@@ -680,74 +682,74 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     s.dG[tid] += rs - cs;
   }
   __syncthreads();
-  for (int p = tid; p < C * C; p += NT) {
+  for (int p = tid; p < C * C; p += GT) {
     const int r = p / C, c = p % C;
     if (c <= r) s.X1[r][c] *= __expf(s.G[r] - s.G[c]);
   }
   __syncthreads();
-  float accK[DK / 16][4];
+  float accK[DK / 32][4];
   zero(accK);
   {  // dQ += (dP (*) Gamma) K -> dq;  dK = (dP (*) Gamma)^T Q
     auto Xa = [&](int r, int c) { return s.X1[r][c]; };
     auto Kb = [&](int c, int i) { return bf(s.kb[c][i]); };
 #pragma unroll
-    for (int nt = 0; nt < DK / 16; ++nt)
+    for (int nt = 0; nt < DK / 32; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) accQ[nt][e] *= s.gam[frow(16 * mt, lane, e)];
-    mma_rows<DK / 16>(accQ, Xa, Kb, 16 * mt, (DK / 2) * nh, C, lane);
+    mma_rows<DK / 32>(accQ, Xa, Kb, 16 * mt, (DK / 4) * nq, C, lane);
     auto XTa = [&](int r, int c) { return s.X1[c][r]; };
     auto Qb = [&](int c, int i) { return bf(s.qb[c][i]); };
-    mma_rows<DK / 16>(accK, XTa, Qb, 16 * mt, (DK / 2) * nh, C, lane);
+    mma_rows<DK / 32>(accK, XTa, Qb, 16 * mt, (DK / 4) * nq, C, lane);
 #pragma unroll
-    for (int nt = 0; nt < DK / 16; ++nt)
+    for (int nt = 0; nt < DK / 32; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; e += 2) {
-        const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
+        const int r = frow(16 * mt, lane, e), i = fcol((DK / 4) * nq, nt, lane, e);
         if (r < len)
           *reinterpret_cast<float2*>(dq + (tok0 + (size_t)r * H) * DK + i) =
               make_float2(accQ[nt][e], accQ[nt][e + 1]);
       }
   }
   {  // T^T dW: dK += diag(beta gamma) T^T dW;  dbeta, dG += rowdot(T^T dW, K) terms
-    float d[DK / 16][4];
+    float d[DK / 32][4];
     zero(d);
     auto TTa = [&](int r, int c) { return s.Tm[c][r]; };
     auto dWb = [&](int c, int i) { return dW[c * LF<DK>() + i]; };
-    mma_rows<DK / 16>(d, TTa, dWb, 16 * mt, (DK / 2) * nh, C, lane);
+    mma_rows<DK / 32>(d, TTa, dWb, 16 * mt, (DK / 4) * nq, C, lane);
     float rk[2] = {0.f, 0.f};
 #pragma unroll
-    for (int nt = 0; nt < DK / 16; ++nt)
+    for (int nt = 0; nt < DK / 32; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
+        const int r = frow(16 * mt, lane, e), i = fcol((DK / 4) * nq, nt, lane, e);
         accK[nt][e] = fmaf(s.beta[r] * s.gam[r], d[nt][e], accK[nt][e]);
         rk[e >> 1] = fmaf(d[nt][e], bf(s.kb[r][i]), rk[e >> 1]);
       }
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
       const float x = quad_sum(rk[hr]);
-      if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+      if ((lane & 3) == 0) s.part[nq][16 * mt + (lane >> 2) + 8 * hr] = x;
     }
   }
   __syncthreads();
   if (tid < C) {
-    const float x = s.part[0][tid] + s.part[1][tid];
+    const float x = s.part[0][tid] + s.part[1][tid] + s.part[2][tid] + s.part[3][tid];
     s.dB[tid] += s.gam[tid] * x;
     s.dG[tid] += s.beta[tid] * s.gam[tid] * x;
   }
   __syncthreads();
   {  // T^T dV': dv = diag(beta) T^T dV';  dbeta += rowdot(T^T dV', V)
-    float d[DV / 16][4];
+    float d[DV / 32][4];
     zero(d);
     auto TTa = [&](int r, int c) { return s.Tm[c][r]; };
     auto dVb = [&](int c, int j) { return s.dVp[c][j]; };
-    mma_rows<DV / 16>(d, TTa, dVb, 16 * mt, (DV / 2) * nh, C, lane);
+    mma_rows<DV / 32>(d, TTa, dVb, 16 * mt, (DV / 4) * nq, C, lane);
     float rv[2] = {0.f, 0.f};
 #pragma unroll
-    for (int nt = 0; nt < DV / 16; ++nt)
+    for (int nt = 0; nt < DV / 32; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; e += 2) {
-        const int r = frow(16 * mt, lane, e), j = fcol((DV / 2) * nh, nt, lane, e);
+        const int r = frow(16 * mt, lane, e), j = fcol((DV / 4) * nq, nt, lane, e);
         rv[e >> 1] = fmaf(d[nt][e], bf(s.vb[r][j]), rv[e >> 1]);
         rv[e >> 1] = fmaf(d[nt][e + 1], bf(s.vb[r][j + 1]), rv[e >> 1]);
         if (r < len)
@@ -757,58 +759,58 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
       const float x = quad_sum(rv[hr]);
-      if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+      if ((lane & 3) == 0) s.part[nq][16 * mt + (lane >> 2) + 8 * hr] = x;
     }
   }
   __syncthreads();
-  if (tid < C) s.dB[tid] += s.part[0][tid] + s.part[1][tid];
+  if (tid < C) s.dB[tid] += s.part[0][tid] + s.part[1][tid] + s.part[2][tid] + s.part[3][tid];
   {  // dT = dW (diag(beta gamma) K)^T + dV' (diag(beta) V)^T -> X2 (P is done)
-    float d[4][4];
+    float d[2][4];
     zero(d);
     auto dWa = [&](int r, int i) { return dW[r * LF<DK>() + i]; };
     auto KTb = [&](int i, int c) { return s.beta[c] * s.gam[c] * bf(s.kb[c][i]); };
-    mma_rows<4>(d, dWa, KTb, 16 * mt, 32 * nh, DK, lane);
+    mma_rows<2>(d, dWa, KTb, 16 * mt, 16 * nq, DK, lane);
     auto dVa = [&](int r, int j) { return s.dVp[r][j]; };
     auto VTb = [&](int j, int c) { return s.beta[c] * bf(s.vb[c][j]); };
-    mma_rows<4>(d, dVa, VTb, 16 * mt, 32 * nh, DV, lane);
+    mma_rows<2>(d, dVa, VTb, 16 * mt, 16 * nq, DV, lane);
     __syncthreads();  // every warp is done reading X2 (P) and X1 (dP Gamma)
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s.X2[frow(16 * mt, lane, e)][fcol(32 * nh, nt, lane, e)] = d[nt][e];
+      for (int e = 0; e < 4; ++e) s.X2[frow(16 * mt, lane, e)][fcol(16 * nq, nt, lane, e)] = d[nt][e];
   }
   __syncthreads();
   {  // Y = T^T dT -> X1
-    float d[4][4];
+    float d[2][4];
     zero(d);
     auto TTa = [&](int r, int c) { return s.Tm[c][r]; };
     auto Xb = [&](int c, int j) { return s.X2[c][j]; };
-    mma_rows<4>(d, TTa, Xb, 16 * mt, 32 * nh, C, lane);
+    mma_rows<2>(d, TTa, Xb, 16 * mt, 16 * nq, C, lane);
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s.X1[frow(16 * mt, lane, e)][fcol(32 * nh, nt, lane, e)] = d[nt][e];
+      for (int e = 0; e < 4; ++e) s.X1[frow(16 * mt, lane, e)][fcol(16 * nq, nt, lane, e)] = d[nt][e];
   }
   __syncthreads();
   {  // dA = -strict_lower(Y T^T) -> X2;  K K^T kept in registers
-    float d[4][4], kk[4][4];
+    float d[2][4], kk[2][4];
     zero(d);
     zero(kk);
     auto Ya = [&](int r, int c) { return s.X1[r][c]; };
     auto TTb = [&](int c, int j) { return s.Tm[j][c]; };
-    mma_rows<4>(d, Ya, TTb, 16 * mt, 32 * nh, C, lane);
+    mma_rows<2>(d, Ya, TTb, 16 * mt, 16 * nq, C, lane);
     auto Ka = [&](int r, int i) { return bf(s.kb[r][i]); };
     auto KTb = [&](int i, int c) { return bf(s.kb[c][i]); };
-    mma_rows<4>(kk, Ka, KTb, 16 * mt, 32 * nh, DK, lane);
+    mma_rows<2>(kk, Ka, KTb, 16 * mt, 16 * nq, DK, lane);
     __syncthreads();  // X2 (dT) fully read
     // E = dA (*) Gamma -> X2;  F = dA (*) A -> X1 (A = beta_r KK Gamma);
     // dbeta_r += sum_s E_rs KK_rs
     float rb[2] = {0.f, 0.f};
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
+        const int r = frow(16 * mt, lane, e), c = fcol(16 * nq, nt, lane, e);
         const float E = c < r ? -d[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;  // dA (*) Gamma
         s.X2[r][c] = E;
         s.X1[r][c] = E * s.beta[r] * kk[nt][e];  // dA (*) A
@@ -817,7 +819,7 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
       const float x = quad_sum(rb[hr]);
-      if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+      if ((lane & 3) == 0) s.part[nq][16 * mt + (lane >> 2) + 8 * hr] = x;
     }
   }
   __syncthreads();
@@ -828,33 +830,33 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
       cs += s.X1[c][tid];
     }
     s.dG[tid] += rs - cs;
-    s.dB[tid] += s.part[0][tid] + s.part[1][tid];
+    s.dB[tid] += s.part[0][tid] + s.part[1][tid] + s.part[2][tid] + s.part[3][tid];
   }
   {  // dK += diag(beta) E K + (diag(beta) E)^T K
     auto Ea = [&](int r, int c) { return s.beta[r] * s.X2[r][c]; };
     auto ETa = [&](int r, int c) { return s.beta[c] * s.X2[c][r]; };
     auto Kb = [&](int c, int i) { return bf(s.kb[c][i]); };
-    mma_rows<DK / 16>(accK, Ea, Kb, 16 * mt, (DK / 2) * nh, C, lane);
-    mma_rows<DK / 16>(accK, ETa, Kb, 16 * mt, (DK / 2) * nh, C, lane);
+    mma_rows<DK / 32>(accK, Ea, Kb, 16 * mt, (DK / 4) * nq, C, lane);
+    mma_rows<DK / 32>(accK, ETa, Kb, 16 * mt, (DK / 4) * nq, C, lane);
   }
 
   // ---- phase 3: dKt = V' dH_{n+1}^T, a 64-column half of dH at a time
-  float dKt[DK / 16][4];
+  float dKt[DK / 32][4];
   zero(dKt);
   for (int half = 0; half < 2; ++half) {
     __syncthreads();  // big (dW, or the other half of dH) is no longer read
-    load_f32<DK, HALF>(&s.big[0][0], dHn + half * HALF, DV);
+    load_f32<DK, HALF, GT>(&s.big[0][0], dHn + half * HALF, DV);
     copies_landed();
     auto Va = [&](int r, int j) { return s.Vp[r][half * HALF + j]; };
     auto HTb = [&](int j, int i) { return s.big[i][j]; };
-    mma_rows<DK / 16>(dKt, Va, HTb, 16 * mt, (DK / 2) * nh, HALF, lane);
+    mma_rows<DK / 32>(dKt, Va, HTb, 16 * mt, (DK / 4) * nq, HALF, lane);
   }
   float rt[2] = {0.f, 0.f};
 #pragma unroll
-  for (int nt = 0; nt < DK / 16; ++nt)
+  for (int nt = 0; nt < DK / 32; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
+      const int r = frow(16 * mt, lane, e), i = fcol((DK / 4) * nq, nt, lane, e);
       const float sc = s.kts[r];
       accK[nt][e] = fmaf(sc, dKt[nt][e], accK[nt][e]);
       rt[e >> 1] = fmaf(dKt[nt][e], sc * bf(s.kb[r][i]), rt[e >> 1]);
@@ -862,15 +864,15 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll
   for (int hr = 0; hr < 2; ++hr) {
     const float x = quad_sum(rt[hr]);
-    if ((lane & 3) == 0) s.part[nh][16 * mt + (lane >> 2) + 8 * hr] = x;
+    if ((lane & 3) == 0) s.part[nq][16 * mt + (lane >> 2) + 8 * hr] = x;
   }
   __syncthreads();
-  if (tid < C) s.dG[tid] -= s.part[0][tid] + s.part[1][tid];
+  if (tid < C) s.dG[tid] -= s.part[0][tid] + s.part[1][tid] + s.part[2][tid] + s.part[3][tid];
   __syncthreads();
   if (tid == 0) {
     float tot = 0.f, hdt = 0.f;
-    for (int r = 0; r < C; ++r) tot += s.part[0][r] + s.part[1][r];
-    for (int w = 0; w < NT / 32; ++w) hdt += s.red[w];
+    for (int r = 0; r < C; ++r) tot += s.part[0][r] + s.part[1][r] + s.part[2][r] + s.part[3][r];
+    for (int w = 0; w < GT / 32; ++w) hdt += s.red[w];
     s.dG[C - 1] += tot + gC * hdt;
     // dg = reverse in-chunk cumsum of dG (rows >= len carry no gradient)
     float acc = 0.f;
@@ -895,10 +897,10 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   }
   __syncthreads();
 #pragma unroll
-  for (int nt = 0; nt < DK / 16; ++nt)
+  for (int nt = 0; nt < DK / 32; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; e += 2) {
-      const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
+      const int r = frow(16 * mt, lane, e), i = fcol((DK / 4) * nq, nt, lane, e);
       if (r < len) {
         const float cf = s.part[0][r];
         *reinterpret_cast<float2*>(dk + (tok0 + (size_t)r * H) * DK + i) =
@@ -981,7 +983,7 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
       qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, Wws, Xws, Yws, Tlen, H, nblk);
   cbwd_adjoint_kernel<DK, DV><<<dim3(DV / BVA, H, B), NT, sa, st>>>(
       kb, g, dhT, Wws, Xws, Yws, dVws, dHws, dh0, Tlen, H, nblk);
-  cbwd_grad_kernel<DK, DV><<<dim3(nblk, H, B), NT, sg, st>>>(
+  cbwd_grad_kernel<DK, DV><<<dim3(nblk, H, B), GT, sg, st>>>(
       qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, dVws, dHws, dq, dk, dv, dg, deta, Tlen, H,
       nblk);
   return cudaGetLastError();
