@@ -548,16 +548,22 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
   const int nblk = (Tlen + bwd::BLK - 1) / bwd::BLK;
   const dim3 grid(DV / bwd::BV, H, B);
   constexpr size_t smem_ck = sizeof(bwd::Ops<DK, VG>);
-  cudaError_t e = cudaFuncSetAttribute(bwd_checkpoint_kernel<T, DK, DV, VG>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_ck);
-  if (e != cudaSuccess) return e;
-  bwd_checkpoint_kernel<T, DK, DV, VG><<<grid, bwd::NT, smem_ck, st>>>(
-      (const T*)k, (const T*)v, g, eta, eps, h0, ck, wbeta, walpha, Tlen, H, nblk);
   constexpr size_t smem = bwd::smem_bytes<DK, VG>();
   static_assert(smem <= 227 * 1024, "shared memory");
-  e = cudaFuncSetAttribute(bwd_kernel<T, DK, DV, VG>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};  // the kernels' shared-memory limits, once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  cudaError_t e = cudaSuccess;
+  if (!attr_set[dev]) {
+    if ((e = cudaFuncSetAttribute(bwd_checkpoint_kernel<T, DK, DV, VG>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_ck)) ||
+        (e = cudaFuncSetAttribute(bwd_kernel<T, DK, DV, VG>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+      return e;
+    attr_set[dev] = true;
+  }
+  bwd_checkpoint_kernel<T, DK, DV, VG><<<grid, bwd::NT, smem_ck, st>>>(
+      (const T*)k, (const T*)v, g, eta, eps, h0, ck, wbeta, walpha, Tlen, H, nblk);
   bwd_kernel<T, DK, DV, VG><<<grid, bwd::NT, smem, st>>>(
       (const T*)q, (const T*)k, (const T*)v, g, (const T*)dout, dhT, wbeta, walpha, ck, sub,
       part, ps, dv, dh0, Tlen, H, nblk);

@@ -972,13 +972,19 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
   constexpr size_t sp = sizeof(PrepSmem<DK, DV>), sa = sizeof(AdjSmem<DK>),
                    sg = sizeof(GradSmem<DK, DV>);
   static_assert(sp <= 227 * 1024 && sa <= 227 * 1024 && sg <= 227 * 1024, "shared memory");
-  if ((e = cudaFuncSetAttribute(cbwd_prep_kernel<DK, DV>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp)) ||
-      (e = cudaFuncSetAttribute(cbwd_adjoint_kernel<DK, DV>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa)) ||
-      (e = cudaFuncSetAttribute(cbwd_grad_kernel<DK, DV>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg)))
-    return e;
+  static bool attr_set[64] = {};  // the kernels' shared-memory limits, once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    if ((e = cudaFuncSetAttribute(cbwd_prep_kernel<DK, DV>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp)) ||
+        (e = cudaFuncSetAttribute(cbwd_adjoint_kernel<DK, DV>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa)) ||
+        (e = cudaFuncSetAttribute(cbwd_grad_kernel<DK, DV>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg)))
+      return e;
+    attr_set[dev] = true;
+  }
   cbwd_prep_kernel<DK, DV><<<dim3(nblk, H, B), NT, sp, st>>>(
       qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, Wws, Xws, Yws, Tlen, H, nblk);
   cbwd_adjoint_kernel<DK, DV><<<dim3(DV / BVA, H, B), NT, sa, st>>>(
