@@ -250,3 +250,29 @@ def test_kda_backward_rejects_bad_arguments(lib):
     beta_args = args[:5] + args[6:]
     bad = list(beta_args); bad[17] = 96; bad[18] = 96
     assert lib.kla_kda_recurrent_bwd_beta(*bad) == UNSUPPORTED
+
+
+def test_chunk_backward_rejects_bad_arguments(lib):
+    """kla_chunk_bwd: the chunk kernels' workspace for bf16 d = 128, the
+    token-serial one otherwise; the same argument checks as the token-serial
+    entry points (no CUDA call is made for these)."""
+    need = lib.kla_chunk_bwd_workspace_size(1, 128, 2, 128, 128, 0)
+    assert need > lib.kla_recurrent_bwd_workspace_size(1, 128, 2, 128, 128) // 8
+    assert lib.kla_chunk_bwd_workspace_size(1, 128, 2, 64, 64, 0) == \
+        lib.kla_recurrent_bwd_workspace_size(1, 128, 2, 64, 64)
+    assert lib.kla_chunk_bwd_workspace_size(1, 128, 2, 128, 128, 1) == \
+        lib.kla_recurrent_bwd_workspace_size(1, 128, 2, 128, 128)
+    args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, None, 6 * A, None, 7 * A, 8 * A, 9 * A,
+            10 * A, 11 * A, None, 1, 128, 2, 128, 128, 0, 64 * A, need, None]
+    bad = list(args); bad[22] = need - 1
+    assert lib.kla_chunk_bwd(*bad) == INVALID
+    bad = list(args); bad[5] = -1.0
+    assert lib.kla_chunk_bwd(*bad) == INVALID
+    bad = list(args); bad[9] = 3 * A  # grad_q over v
+    assert lib.kla_chunk_bwd(*bad) == INVALID
+    bad = list(args); bad[18] = 96; bad[19] = 96
+    assert lib.kla_chunk_bwd(*bad) == UNSUPPORTED
+    gdn = args[:5] + args[6:]
+    bad = list(gdn); bad[20] = None  # no workspace
+    assert lib.kla_gdn_chunk_bwd(*bad) == INVALID
+    assert lib.kla_gdn_chunk_bwd(*(gdn[:14] + [0] + gdn[15:])) == INVALID  # B = 0
