@@ -364,7 +364,7 @@ static kla_status bwd_impl(const void* q, const void* k, const void* v, const fl
   const size_t gdim = vector_gate ? dk : 1;
   // the chunkwise kernels cover bf16 with d = 128 and the scalar gate; the
   // rest runs the token-serial kernels
-  const bool use_chunks = chunked && !vector_gate && dtype == KLA_BF16 && dk == 128 && dv == 128;
+  const bool use_chunks = chunked && !vector_gate && dtype == KLA_BF16 && dk == dv;
   const size_t need = use_chunks ? chunk_bwd_workspace_bytes(B, T, H, dk, dv)
                                  : recurrent_bwd_workspace_bytes(B, T, H, dk, dv, vector_gate);
   if (T > 0 && (!workspace || ws_bytes < need)) return KLA_ERR_INVALID_ARG;
@@ -412,7 +412,7 @@ size_t kla_recurrent_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
 
 size_t kla_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int dtype) {
   if (!head_dims_ok(dk, dv)) return 0;
-  if (dtype == KLA_BF16 && dk == 128 && dv == 128) return chunk_bwd_workspace_bytes(B, T, H, dk, dv);
+  if (dtype == KLA_BF16 && dk == dv) return chunk_bwd_workspace_bytes(B, T, H, dk, dv);
   return recurrent_bwd_workspace_bytes(B, T, H, dk, dv, false);
 }
 

@@ -1,5 +1,5 @@
 // Chunkwise backward of the KLA / gated delta rule prefill (bf16 I/O,
-// scalar gate): the gradients of a loss L given dL/do and dL/dh_T, from the
+// scalar gate, d_k = d_v = 64 or 128): the gradients of a loss L given dL/do and dL/dh_T, from the
 // chunk form of the forward ("Deep Dive into KDA", section 3, with the KLA
 // step size of "Kaczmarz Linear Attention", Abstract).  Per chunk n of C = 64
 // tokens with start state h_n (G = in-chunk cumsum of g, gamma = e^G,
@@ -307,19 +307,23 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
       }
   }
   __syncthreads();
-  {  // Y = (diag(gamma) Q)^T dO  [DK x DV]: warp w has rows 16 w .., two column halves
+  {  // Y = (diag(gamma) Q)^T dO  [DK x DV]: DK / 16 row tiles; with 8 row tiles
+     // warp w takes row tile w and both column halves, with 4 it takes row
+     // tile w % 4 and column half w / 4
+    constexpr int RT = DK / 16;
     auto QTa = [&](int i, int c) { return s.gam[c] * bf(s.qb[c][i]); };
     auto Ob = [&](int c, int j) { return bf(s.ob[c][j]); };
     float* ydst = Yws + chunk * DK * DV;
-    for (int half = 0; half < 2; ++half) {
+    const int ym = warp % RT;
+    for (int half = RT == 8 ? 0 : warp / RT; half < 2; half += RT == 8 ? 1 : 2) {
       float d[DV / 16][4];
       zero(d);
-      mma_rows<DV / 16>(d, QTa, Ob, 16 * warp, half * (DV / 2), C, lane);
+      mma_rows<DV / 16>(d, QTa, Ob, 16 * ym, half * (DV / 2), C, lane);
 #pragma unroll
       for (int nt = 0; nt < DV / 16; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; e += 2) {
-          const int i = frow(16 * warp, lane, e), j = fcol(half * (DV / 2), nt, lane, e);
+          const int i = frow(16 * ym, lane, e), j = fcol(half * (DV / 2), nt, lane, e);
           *reinterpret_cast<float2*>(ydst + i * DV + j) = make_float2(d[nt][e], d[nt][e + 1]);
         }
     }
@@ -425,21 +429,25 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict
                     const float* __restrict__ Xws, const float* __restrict__ Yws,
                     float* __restrict__ dVws, float* __restrict__ dHws, float* __restrict__ dh0,
                     int Tlen, int H, int nblk) {
-  static_assert(DK == 128, "one 16-row tile of the state per warp");
+  // the dH slab [DK x 32] in 16-row tiles: DK / 16 of them, NT / 32 / (DK / 16)
+  // warps per tile splitting its columns
+  constexpr int RT = DK / 16, WPT = (NT / 32) / RT, NTH = (BVA / 8) / WPT;
+  static_assert(RT * WPT == NT / 32 && NTH >= 1, "state tiling");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   auto& s = *reinterpret_cast<AdjSmem<DK>*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int slab = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
   const int j0 = slab * BVA;
   const size_t head = (size_t)b * H + hh;
+  const int hm0 = 16 * (warp % RT), hn0 = (BVA / WPT) * (warp / RT);  // this warp's dH tile
 
-  float acc[BVA / 8][4];  // dH rows 16 warp .., columns j0 ..
+  float acc[NTH][4];  // dH rows hm0 .., columns j0 + hn0 ..
 #pragma unroll
-  for (int nt = 0; nt < BVA / 8; ++nt)
+  for (int nt = 0; nt < NTH; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      acc[nt][e] = dhT ? dhT[(head * DK + frow(16 * warp, lane, e)) * DV + j0 +
-                             fcol(0, nt, lane, e)]
+      acc[nt][e] = dhT ? dhT[(head * DK + frow(hm0, lane, e)) * DV + j0 +
+                             fcol(hn0, nt, lane, e)]
                        : 0.f;
   adj_fetch<DK, DV>(s.buf[(nblk - 1) & 1], k, g, Wws, Xws, Yws, head, nblk - 1, nblk, j0, b,
                     hh, Tlen, H);
@@ -454,10 +462,10 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict
                         Tlen, H);
     // dH_{n+1}: to shared memory (operand) and to the workspace
 #pragma unroll
-    for (int nt = 0; nt < BVA / 8; ++nt)
+    for (int nt = 0; nt < NTH; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; e += 2) {
-        const int r = frow(16 * warp, lane, e), c = fcol(0, nt, lane, e);
+        const int r = frow(hm0, lane, e), c = fcol(hn0, nt, lane, e);
         s.dH[r][c] = acc[nt][e];
         s.dH[r][c + 1] = acc[nt][e + 1];
         *reinterpret_cast<float2*>(dHws + (chunk * DK + r) * DV + j0 + c) =
@@ -503,23 +511,21 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict
     {  // dH_n = gamma_C dH_{n+1} + Y - W^T dV'
       const float gC = s.gC;
 #pragma unroll
-      for (int nt = 0; nt < BVA / 8; ++nt)
+      for (int nt = 0; nt < NTH; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          acc[nt][e] = fmaf(gC, acc[nt][e],
-                            cur.Y[frow(16 * warp, lane, e)][fcol(0, nt, lane, e)]);
+          acc[nt][e] = fmaf(gC, acc[nt][e], cur.Y[frow(hm0, lane, e)][fcol(hn0, nt, lane, e)]);
       auto WTa = [&](int i, int c) { return -cur.W[c][i]; };
       auto dVb = [&](int c, int j) { return s.dV[c][j]; };
-      mma_rows<BVA / 8>(acc, WTa, dVb, 16 * warp, 0, C, lane);
+      mma_rows<NTH>(acc, WTa, dVb, hm0, hn0, C, lane);
     }
   }
   if (dh0) {
 #pragma unroll
-    for (int nt = 0; nt < BVA / 8; ++nt)
+    for (int nt = 0; nt < NTH; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        dh0[(head * DK + frow(16 * warp, lane, e)) * DV + j0 + fcol(0, nt, lane, e)] =
-            acc[nt][e];
+        dh0[(head * DK + frow(hm0, lane, e)) * DV + j0 + fcol(hn0, nt, lane, e)] = acc[nt][e];
   }
 }
 
@@ -533,7 +539,8 @@ struct GradSmem {
   float Tm[C][LF<C>()];
   float Vp[C][LF<DV>()];   // V'
   float dVp[C][LF<DV>()];  // dV'
-  float big[DK][LF<DV / 2>()];  // a 64-column half of h_n or dH, or dW [C][DK]
+  // a column half of h_n or dH ([DK][LF<DV/2>]), or dW ([C][LF<DK>])
+  float big[(DK * LF<DV / 2>() > C * LF<DK>()) ? DK * LF<DV / 2>() : C * LF<DK>()];
   float X1[C][LF<C>()];
   float X2[C][LF<C>()];
   float G[C], gam[C], beta[C], n2[C], kts[C];
@@ -596,26 +603,27 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   float rowO[2] = {0.f, 0.f};  // rowdot(dO, diag(gamma) Q h_n) for rows g, g + 8
   for (int half = 0; half < 2; ++half) {
     __syncthreads();
-    load_f32<DK, HALF, GT>(&s.big[0][0], hn + half * HALF, DV);
+    load_f32<DK, HALF, GT>(s.big, hn + half * HALF, DV);
     copies_landed();
     // dO h_n^T and -dV' h_n^T over this half of the dv index
     auto Oa = [&](int r, int j) { return bf(s.ob[r][half * HALF + j]); };
     auto dVa = [&](int r, int j) { return -s.dVp[r][half * HALF + j]; };
-    auto HTb = [&](int j, int i) { return s.big[i][j]; };
+    auto HTb = [&](int j, int i) { return s.big[i * LF<HALF>() + j]; };
     mma_rows<DK / 32>(accQ, Oa, HTb, 16 * mt, (DK / 4) * nq, HALF, lane);
     mma_rows<DK / 32>(accW, dVa, HTb, 16 * mt, (DK / 4) * nq, HALF, lane);
-    // diag(gamma) Q h_n on this half's columns: 64 x 64, 4 tiles per warp
-    float o[2][4];
+    // diag(gamma) Q h_n on this half's columns: [C x HALF], a quarter per warp
+    constexpr int OQ = HALF / 4, NTO = OQ / 8;
+    float o[NTO][4];
     zero(o);
     auto Qa = [&](int r, int i) { return s.gam[r] * bf(s.qb[r][i]); };
-    auto Hb = [&](int i, int j) { return s.big[i][j]; };
-    mma_rows<2>(o, Qa, Hb, 16 * mt, 16 * nq, DK, lane);
+    auto Hb = [&](int i, int j) { return s.big[i * LF<HALF>() + j]; };
+    mma_rows<NTO>(o, Qa, Hb, 16 * mt, OQ * nq, DK, lane);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NTO; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         rowO[e >> 1] += o[nt][e] * bf(s.ob[frow(16 * mt, lane, e)]
-                                          [half * HALF + fcol(16 * nq, nt, lane, e)]);
+                                          [half * HALF + fcol(OQ * nq, nt, lane, e)]);
   }
   // <dH_{n+1}, h_n> (block sum, fixed order; every load issued up front)
   float hd = 0.f;
@@ -642,8 +650,7 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   __syncthreads();
   if (tid < C) s.dG[tid] += s.part[0][tid] + s.part[1][tid] + s.part[2][tid] + s.part[3][tid];
   // dq (first part) stays in accQ; dW -> big as [C][DK]
-  float* dW = &s.big[0][0];  // [C][LF<DK>] fits in [DK][LF<DV/2>]
-  static_assert(C * LF<DK>() <= DK * LF<DV / 2>(), "dW in big");
+  float* dW = s.big;  // [C][LF<DK>]
 #pragma unroll
   for (int nt = 0; nt < DK / 32; ++nt)
 #pragma unroll
@@ -845,10 +852,10 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   zero(dKt);
   for (int half = 0; half < 2; ++half) {
     __syncthreads();  // big (dW, or the other half of dH) is no longer read
-    load_f32<DK, HALF, GT>(&s.big[0][0], dHn + half * HALF, DV);
+    load_f32<DK, HALF, GT>(s.big, dHn + half * HALF, DV);
     copies_landed();
     auto Va = [&](int r, int j) { return s.Vp[r][half * HALF + j]; };
-    auto HTb = [&](int j, int i) { return s.big[i][j]; };
+    auto HTb = [&](int j, int i) { return s.big[i * LF<HALF>() + j]; };
     mma_rows<DK / 32>(dKt, Va, HTb, 16 * mt, (DK / 4) * nq, HALF, lane);
   }
   float rt[2] = {0.f, 0.f};
@@ -939,17 +946,18 @@ static CbwdWs cbwd_layout(int B, int T, int H, int dk, int dv) {
 }
 
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
-  if (B < 1 || H < 1 || T < 1 || dk != 128 || dv != 128) return 0;
+  if (B < 1 || H < 1 || T < 1 || dk != dv || (dk != 64 && dk != 128)) return 0;
   return cbwd_layout(B, T, H, dk, dv).total;
 }
 
-cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
-                             const float* eta, float eps, const float* h0, const void* dout,
-                             const float* dhT, float* dq, float* dk, float* dv, float* dg,
-                             float* deta, float* dh0, int B, int Tlen, int H, int dkd, int dvd,
-                             void* ws, unsigned int* err, cudaStream_t st) {
-  constexpr int DK = 128, DV = 128;
-  if (dkd != DK || dvd != DV) return cudaErrorInvalidValue;
+template <int D>
+static cudaError_t launch_chunk_bwd_d(const void* q, const void* k, const void* v,
+                                      const float* g, const float* eta, float eps,
+                                      const float* h0, const void* dout, const float* dhT,
+                                      float* dq, float* dk, float* dv, float* dg, float* deta,
+                                      float* dh0, int B, int Tlen, int H, void* ws,
+                                      unsigned int* err, cudaStream_t st) {
+  constexpr int DK = D, DV = D;
   const CbwdWs w = cbwd_layout(B, Tlen, H, DK, DV);
   char* base = (char*)ws;
   float* ck = (float*)(base + w.ck);
@@ -993,6 +1001,20 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
       qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, dVws, dHws, dq, dk, dv, dg, deta, Tlen, H,
       nblk);
   return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                             const float* eta, float eps, const float* h0, const void* dout,
+                             const float* dhT, float* dq, float* dk, float* dv, float* dg,
+                             float* deta, float* dh0, int B, int Tlen, int H, int dkd, int dvd,
+                             void* ws, unsigned int* err, cudaStream_t st) {
+  if (dkd == 128 && dvd == 128)
+    return launch_chunk_bwd_d<128>(q, k, v, g, eta, eps, h0, dout, dhT, dq, dk, dv, dg, deta,
+                                   dh0, B, Tlen, H, ws, err, st);
+  if (dkd == 64 && dvd == 64)
+    return launch_chunk_bwd_d<64>(q, k, v, g, eta, eps, h0, dout, dhT, dq, dk, dv, dg, deta,
+                                  dh0, B, Tlen, H, ws, err, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kla

@@ -49,7 +49,7 @@ cudaError_t launch_recurrent_bwd(const void* q, const void* k, const void* v, co
                                  float* dh0, int B, int T, int H, int dkd, int dvd, int dtype,
                                  void* ws, cudaStream_t st);
 
-// Chunkwise backward (kla_chunk_bwd.cu; bf16, d_k = d_v = 128, scalar gate).
+// Chunkwise backward (kla_chunk_bwd.cu; bf16, d_k = d_v in {64, 128}, scalar gate).
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
                              const float* eta, float eps, const float* h0, const void* dout,

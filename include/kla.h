@@ -302,9 +302,9 @@ KLA_API kla_status kla_recurrent_bwd(const void *q, const void *k, const void *v
  * T = (I + A)^{-1} (dA = -strict_lower(T^T dT T^T)), dg as the reverse
  * in-chunk cumsum of dG.  The states h_n come from the forward chunk
  * prefill (the kernels of kla_chunk_fwd, outputs off, its state chain
- * writing every h_n).  bf16 with dk = dv = 128 runs these kernels (relative
- * L2 of the gradients about 1e-3: bf16 state chain, tf32 products); fp32
- * I/O and d = 64 run the token-serial kernels of kla_recurrent_bwd.
+ * writing every h_n).  bf16 I/O runs these kernels (relative L2 of the
+ * gradients about 1e-3: bf16 state chain, tf32 products); fp32 I/O runs the
+ * token-serial kernels of kla_recurrent_bwd (fp32 accuracy).
  * Workspace: kla_chunk_bwd_workspace_size(...) bytes (for the chunk kernels
  * about B*H*ceil(T/64) * 224 KiB).
  */

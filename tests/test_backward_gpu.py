@@ -192,6 +192,8 @@ TOL_CHUNK = 1e-2
     ("prefill_4k", 1, 1, 2, True, True),       # one token
     ("prefill_4k", 1, 257, 1, False, False),   # one token past 4 chunks
     ("prefill_65k", 1, 700, 2, False, True),   # strong forgets
+    ("stress", 1, 200, 3, True, True),         # d = 64: key norms 1e-2 .. 1e2, eta up to 2
+    ("stress", 2, 64, 2, True, False),
 ])
 def test_chunk_backward(name, B, T, H, with_h0, with_dhT):
     w = inputs.WORKLOADS[name].scaled(B=B, T=T, H=H)
