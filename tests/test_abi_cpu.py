@@ -253,15 +253,16 @@ def test_kda_backward_rejects_bad_arguments(lib):
 
 
 def test_chunk_backward_rejects_bad_arguments(lib):
-    """kla_chunk_bwd: the chunk kernels' workspace for bf16 d = 128, the
-    token-serial one otherwise; the same argument checks as the token-serial
-    entry points (no CUDA call is made for these)."""
+    """kla_chunk_bwd: the chunk kernels' workspace for bf16 (d = 64, 128),
+    the token-serial one for fp32 I/O; the same argument checks as the
+    token-serial entry points (no CUDA call is made for these)."""
     need = lib.kla_chunk_bwd_workspace_size(1, 128, 2, 128, 128, 0)
-    assert need > lib.kla_recurrent_bwd_workspace_size(1, 128, 2, 128, 128) // 8
-    assert lib.kla_chunk_bwd_workspace_size(1, 128, 2, 64, 64, 0) == \
-        lib.kla_recurrent_bwd_workspace_size(1, 128, 2, 64, 64)
+    # per chunk: h_n, dH (64 KiB each), T (16 KiB), V', dV', W, X (32 KiB each), Y (64 KiB)
+    assert need >= 4 * (2 * 65536 + 16384 + 4 * 32768 + 65536)
+    assert lib.kla_chunk_bwd_workspace_size(1, 128, 2, 64, 64, 0) < need
     assert lib.kla_chunk_bwd_workspace_size(1, 128, 2, 128, 128, 1) == \
         lib.kla_recurrent_bwd_workspace_size(1, 128, 2, 128, 128)
+    assert lib.kla_chunk_bwd_workspace_size(1, 128, 2, 96, 96, 0) == 0
     args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, None, 6 * A, None, 7 * A, 8 * A, 9 * A,
             10 * A, 11 * A, None, 1, 128, 2, 128, 128, 0, 64 * A, need, None]
     bad = list(args); bad[22] = need - 1
