@@ -679,14 +679,19 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
       }
   }
   __syncthreads();
-  // F = dP (*) P: dG_r += rowsum, dG_s -= colsum;  X1 <- dP (*) Gamma
-  if (tid < C) {
+  // F = dP (*) P: dG_r += rowsum, dG_s -= colsum (four threads per row);
+  // X1 <- dP (*) Gamma
+  if (tid < 4 * C) {
+    const int r = tid >> 2, c0 = 16 * (tid & 3);
     float rs = 0.f, cs = 0.f;
-    for (int c = 0; c < C; ++c) {
-      rs = fmaf(s.X1[tid][c], s.X2[tid][c], rs);
-      cs = fmaf(s.X1[c][tid], s.X2[c][tid], cs);
+#pragma unroll 4
+    for (int c = c0; c < c0 + 16; ++c) {
+      rs = fmaf(s.X1[r][c], s.X2[r][c], rs);
+      cs = fmaf(s.X1[c][r], s.X2[c][r], cs);
     }
-    s.dG[tid] += rs - cs;
+    rs = quad_sum(rs);
+    cs = quad_sum(cs);
+    if ((tid & 3) == 0) s.dG[r] += rs - cs;
   }
   __syncthreads();
   for (int p = tid; p < C * C; p += GT) {
@@ -830,15 +835,20 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     }
   }
   __syncthreads();
-  if (tid < C) {
+  if (tid < 4 * C) {  // F = dA (*) A: row and column sums, four threads per row
+    const int r = tid >> 2, c0 = 16 * (tid & 3);
     float rs = 0.f, cs = 0.f;
-    for (int c = 0; c < C; ++c) {
-      rs += s.X1[tid][c];
-      cs += s.X1[c][tid];
+#pragma unroll 4
+    for (int c = c0; c < c0 + 16; ++c) {
+      rs += s.X1[r][c];
+      cs += s.X1[c][r];
     }
-    s.dG[tid] += rs - cs;
-    s.dB[tid] += s.part[0][tid] + s.part[1][tid] + s.part[2][tid] + s.part[3][tid];
+    rs = quad_sum(rs);
+    cs = quad_sum(cs);
+    if ((tid & 3) == 0)
+      s.dG[r] += rs - cs;
   }
+  if (tid < C) s.dB[tid] += s.part[0][tid] + s.part[1][tid] + s.part[2][tid] + s.part[3][tid];
   {  // dK += diag(beta) E K + (diag(beta) E)^T K
     auto Ea = [&](int r, int c) { return s.beta[r] * s.X2[r][c]; };
     auto ETa = [&](int r, int c) { return s.beta[c] * s.X2[c][r]; };
@@ -876,17 +886,25 @@ cbwd_grad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   __syncthreads();
   if (tid < C) s.dG[tid] -= s.part[0][tid] + s.part[1][tid] + s.part[2][tid] + s.part[3][tid];
   __syncthreads();
-  if (tid == 0) {
-    float tot = 0.f, hdt = 0.f;
-    for (int r = 0; r < C; ++r) tot += s.part[0][r] + s.part[1][r] + s.part[2][r] + s.part[3][r];
-    for (int w = 0; w < GT / 32; ++w) hdt += s.red[w];
-    s.dG[C - 1] += tot + gC * hdt;
-    // dg = reverse in-chunk cumsum of dG (rows >= len carry no gradient)
-    float acc = 0.f;
-    for (int r = C - 1; r >= 0; --r) {
-      acc += s.dG[r];
-      s.dG[r] = acc;
+  if (warp == 0) {
+    float tot = 0.f;
+    for (int r = lane; r < C; r += 32)
+      tot += s.part[0][r] + s.part[1][r] + s.part[2][r] + s.part[3][r];
+    tot = warp_sum(tot);
+    const float hdt = warp_sum(lane < GT / 32 ? s.red[lane] : 0.f);
+    if (lane == 0) s.dG[C - 1] += tot + gC * hdt;
+    __syncwarp();
+    // dg = reverse in-chunk cumsum of dG (rows >= len carry no gradient):
+    // lane l holds rows 2l, 2l + 1; suffix sums of the pairs across lanes
+    const float a0 = s.dG[2 * lane], a1 = s.dG[2 * lane + 1];
+    float suf = a0 + a1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_down_sync(0xffffffffu, suf, o);
+      if (lane + o < 32) suf += y;
     }
+    s.dG[2 * lane] = suf;
+    s.dG[2 * lane + 1] = suf - a0;
   }
   __syncthreads();
   // step size: KLA beta = eta / (||k||^2 + eps)
