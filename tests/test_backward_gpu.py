@@ -252,3 +252,25 @@ def test_chunk_backward_full_size_sampled_heads():
         got = {n: sl(out[n].cpu()) for n in ("dq", "dk", "dv", "dg", "deta")}
         got["dh0"] = out["dh0"][b:b + 1, h:h + 1].cpu()
         _check(got, ref, tol=TOL_CHUNK)
+
+
+def test_autograd_binding_matches_oracle_gradients():
+    """kla_prefill under torch.autograd: a loss <o, do> + <hT, dhT> gives the
+    oracle's gradients (bf16 inputs receive their gradients in bf16)."""
+    from delta_rule_linear_kla_b200 import kla_prefill
+    w = inputs.WORKLOADS["prefill_4k"].scaled(B=1, T=160, H=2)
+    x = inputs.make_prefill(w, with_h0=True)
+    do, dhT = _upstream(w, 95)
+    leaves = {n: cuda(x[n]).requires_grad_(True) for n in ("q", "k", "v", "g", "eta", "h0")}
+    o, hT = kla_prefill(leaves["q"], leaves["k"], leaves["v"], leaves["g"], leaves["eta"],
+                        x["eps"], leaves["h0"])
+    loss = (o.float() * cuda(do).float()).sum() + (hT * cuda(dhT)).sum()
+    loss.backward()
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"], do, dhT)
+    names = dict(q="dq", k="dk", v="dv", g="dg", eta="deta", h0="dh0")
+    for n, rn in names.items():
+        got = leaves[n].grad
+        assert got.dtype == leaves[n].dtype
+        err = rel(got.float().cpu(), ref[rn])
+        # bf16 gradients add their own rounding (2^-9) to the kernels' error
+        assert err < TOL_CHUNK, (n, err)
