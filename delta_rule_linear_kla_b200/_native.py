@@ -19,6 +19,8 @@ SIGNATURES = {
     "kla_chunk_fwd_segments": (_i, [_i, _i, _i, _i, _i, _i, _sz]),
     "kla_chunk_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
                            _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_chunk_fwd_states": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp,
+                                  _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_chunk_ut_transform": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_chunk_state_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),

@@ -104,6 +104,27 @@ def chunk_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
     return o, hT
 
 
+def chunk_fwd_states(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, outputs: bool = True,
+                     workspace=None, stream=None):
+    """bf16 chunk prefill that also returns the state at the start of every
+    chunk (kla_chunk_fwd_states).  Returns (o, hT, hs) with hs
+    [B, H, ceil(T / 64), dk, dv] fp32; o and hT are None if not outputs."""
+    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, eta, h0, None, None, outputs)
+    if not outputs:
+        o = None
+    hs = torch.empty((B, H, (T + CHUNK - 1) // CHUNK, dk, dv), dtype=torch.float32,
+                     device=q.device)
+    need = chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _native.lib().kla_chunk_fwd_states(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0), _ptr(o), _ptr(hT),
+        _ptr(hs), B, T, H, dk, dv, _DT[q.dtype], _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "kla_chunk_fwd_states")
+    return o, hT, hs
+
+
 def _workspace(workspace, B, T, H, dk, dv, dtype, device):
     need = chunk_fwd_workspace_size(B, T, H, dk, dv, dtype)
     if workspace is None:

@@ -49,12 +49,12 @@ static kla_status check_prefill(const void* q, const void* k, const void* v,
                                 const float* g, const float* eta, float eps,
                                 const float* h0, const void* o, const float* hT,
                                 int B, int T, int H, int dk, int dv, int dtype,
-                                int gdim = 1) {
+                                int gdim = 1, bool o_optional = false) {
   if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return KLA_ERR_INVALID_ARG;
   if (dtype != KLA_BF16 && dtype != KLA_FP32) return KLA_ERR_INVALID_ARG;
   if (!(eps >= 0.0f) || eps != eps) return KLA_ERR_INVALID_ARG;
   if ((long long)B * T * H * (dk > dv ? dk : dv) >= (1LL << 40)) return KLA_ERR_INVALID_ARG;
-  if (T > 0 && (!q || !k || !v || !g || !eta || !o)) return KLA_ERR_INVALID_ARG;
+  if (T > 0 && (!q || !k || !v || !g || !eta || (!o && !o_optional))) return KLA_ERR_INVALID_ARG;
   if (T == 0 && hT == nullptr) return KLA_OK;
   const void* ptrs[] = {q, k, v, g, eta, h0, o, hT};
   for (const void* p : ptrs)
@@ -158,6 +158,37 @@ static kla_status chunk_fwd_impl(const void* q, const void* k, const void* v,
 }
 
 extern "C" {
+
+kla_status kla_chunk_fwd_states(const void* q, const void* k, const void* v, const float* g,
+                                const float* eta, float eps, const float* h0, void* o,
+                                float* hT, float* hs, int B, int T, int H, int dk, int dv,
+                                int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  kla_status s = check_prefill(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, dtype, 1, true);
+  if (s != KLA_OK) return s;
+  if (dtype != KLA_BF16) return KLA_ERR_UNSUPPORTED;
+  if (T < 1 || !hs || !aligned16(hs)) return KLA_ERR_INVALID_ARG;
+  const size_t need = chunk_ut_workspace_bytes(B, T, H, dk, dv, dtype);
+  if (ws_bytes < need || !workspace || !aligned16(workspace)) return KLA_ERR_INVALID_ARG;
+  const size_t used = chunk_workspace_used(B, T, H, dk, dv, dtype, ws_bytes);
+  if (workspace_overlaps(workspace, used, q, k, v, g, eta, h0, o, hT, B, T, H, dk, dv, dtype))
+    return KLA_ERR_INVALID_ARG;
+  // hs is written: disjoint from every other argument
+  const size_t ntok = (size_t)B * T * H, sb = (size_t)B * H * dk * dv * 4;
+  const Range rs = rng(hs, (size_t)B * H * ((T + KLA_CHUNK - 1) / KLA_CHUNK) * dk * dv * 4);
+  const Range others[] = {rng(q, ntok * dk * 2), rng(k, ntok * dk * 2), rng(v, ntok * dv * 2),
+                          rng(g, ntok * 4),      rng(eta, ntok * 4),    rng(h0, h0 ? sb : 0),
+                          rng(o, o ? ntok * dv * 2 : 0), rng(hT, hT ? sb : 0),
+                          rng(workspace, used)};
+  for (const Range& r : others)
+    if (overlap(rs, r)) return KLA_ERR_INVALID_ARG;
+  unsigned int* err = device_error_ptr();
+  if (!err) return KLA_ERR_CUDA;
+  cudaError_t e = launch_chunk_tc(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, workspace,
+                                  ws_bytes, err, (cudaStream_t)stream, hs);
+  if (e == cudaErrorNotSupported) return KLA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
 
 kla_status kla_chunk_fwd(const void* q, const void* k, const void* v,
                          const float* g, const float* eta, float eps,

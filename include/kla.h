@@ -109,6 +109,21 @@ KLA_API kla_status kla_chunk_fwd(const void *q, const void *k, const void *v,
                          void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * kla_chunk_fwd (bf16, same arguments, layouts and workspace) that also
+ * writes the state at the start of every chunk: hs [B][H][ceil(T/64)]
+ * [dk][dv] fp32, hs[b][h][n] = h after the first 64 n tokens (n = 0: h0, or
+ * zeros), as the state kernel carries it (fp32 sums of bf16 products) -- the
+ * checkpoints a training framework needs for its own backward.  o and hT
+ * may be NULL (not written).  hs must be 16-byte aligned and disjoint from
+ * every other argument; dtype KLA_FP32 -> KLA_ERR_UNSUPPORTED; T >= 1.
+ */
+KLA_API kla_status kla_chunk_fwd_states(const void *q, const void *k, const void *v,
+                                        const float *g, const float *eta, float eps,
+                                        const float *h0, void *o, float *hT, float *hs,
+                                        int B, int T, int H, int dk, int dv, int dtype,
+                                        void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * The two stages of the bf16 kla_chunk_fwd, callable on their own (same
  * layouts and conventions; kla_chunk_fwd is exactly the first call followed
  * by the second on the same stream).  dtype must be KLA_BF16 (KLA_FP32 ->

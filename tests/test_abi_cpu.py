@@ -277,3 +277,19 @@ def test_chunk_backward_rejects_bad_arguments(lib):
     bad = list(gdn); bad[20] = None  # no workspace
     assert lib.kla_gdn_chunk_bwd(*bad) == INVALID
     assert lib.kla_gdn_chunk_bwd(*(gdn[:14] + [0] + gdn[15:])) == INVALID  # B = 0
+
+
+def test_chunk_fwd_states_rejects_bad_arguments(lib):
+    ws = lib.kla_chunk_fwd_workspace_size(1, 128, 2, 128, 128, 0)
+    args = [A, 2 * A, 3 * A, 4 * A, 5 * A, 1e-6, None, None, None, 7 * A,
+            1, 128, 2, 128, 128, 0, 16 * A, ws, None]
+    bad = list(args); bad[9] = A  # states over q
+    assert lib.kla_chunk_fwd_states(*bad) == INVALID
+    bad = list(args); bad[9] = None
+    assert lib.kla_chunk_fwd_states(*bad) == INVALID
+    bad = list(args); bad[15] = 1
+    assert lib.kla_chunk_fwd_states(*bad) == UNSUPPORTED  # fp32 I/O
+    bad = list(args); bad[17] = ws - 1
+    assert lib.kla_chunk_fwd_states(*bad) == INVALID
+    bad = list(args); bad[11] = 0
+    assert lib.kla_chunk_fwd_states(*bad) == INVALID  # T = 0

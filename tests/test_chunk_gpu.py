@@ -200,3 +200,30 @@ def test_all_keys_zero_is_pure_decay():
     api.check_device_error()
     o_ref, h_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"])
     assert rel(o.cpu(), o_ref) < TOL and rel(hT.cpu(), h_ref) < TOL
+
+
+@pytest.mark.parametrize("B,T,H", [(2, 300, 2),     # uncut chain
+                                   (1, 4000, 2)])  # cut chain
+def test_chunk_start_states(B, T, H):
+    """kla_chunk_fwd_states: the state at the start of every chunk equals the
+    oracle's state after the first 64 n tokens; o and h_T are bitwise those
+    of kla_chunk_fwd."""
+    w = inputs.WORKLOADS["prefill_4k"].scaled(B=B, T=T, H=H)
+    x = inputs.make_prefill(w, with_h0=True)
+    xc = cuda(x)
+    o, hT, hs = api.chunk_fwd_states(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"],
+                                     xc["h0"])
+    o2, h2 = api.chunk_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["eta"], x["eps"], xc["h0"])
+    api.check_device_error()
+    assert torch.equal(o, o2) and torch.equal(hT, h2)
+    nck = (T + 63) // 64
+    assert hs.shape == (B, H, nck, w.dk, w.dv)
+    hs = hs.cpu()
+    for n in sorted({0, 1, nck // 2, nck - 1}):
+        if n == 0:
+            ref = oracle.f64(x["h0"])
+        else:
+            sl = lambda t: t[:, :64 * n]
+            _, ref = oracle.forward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["eta"]),
+                                    x["eps"], x["h0"])
+        assert rel(hs[:, :, n], ref) < TOL, n
