@@ -378,9 +378,9 @@ struct AdjBuf {
   float g[C];
 };
 
-template <int DK>
+template <int DK, int NBUF>
 struct AdjSmem {
-  AdjBuf<DK> buf[2];
+  AdjBuf<DK> buf[NBUF];
   float dH[DK][LF<BVA>()];
   float dV[C][LF<BVA>()];
   float kts[C];
@@ -421,8 +421,11 @@ __device__ __forceinline__ void adj_fetch(AdjBuf<DK>& d, const __nv_bfloat16* k,
 }
 
 // One CTA per (head, 32-column slab); chunks in reverse.  dH (the adjoint of
-// h_{n+1}) lives in registers: warp w holds rows 16 w .. 16 w + 15.
-template <int DK, int DV>
+// h_{n+1}) lives in registers.  NBUF = 2: the next chunk's operands are
+// copied in while the current one is worked on (for few CTAs, one per SM);
+// NBUF = 1: one buffer, small enough for two CTAs per SM, whose work hides
+// each other's copies (for many CTAs).
+template <int DK, int DV, int NBUF>
 __global__ void __launch_bounds__(NT)
 cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict__ g,
                     const float* __restrict__ dhT, const float* __restrict__ Wws,
@@ -434,7 +437,7 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict
   constexpr int RT = DK / 16, WPT = (NT / 32) / RT, NTH = (BVA / 8) / WPT;
   static_assert(RT * WPT == NT / 32 && NTH >= 1, "state tiling");
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  auto& s = *reinterpret_cast<AdjSmem<DK>*>(smem_raw);
+  auto& s = *reinterpret_cast<AdjSmem<DK, NBUF>*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int slab = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
   const int j0 = slab * BVA;
@@ -449,17 +452,23 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict
       acc[nt][e] = dhT ? dhT[(head * DK + frow(hm0, lane, e)) * DV + j0 +
                              fcol(hn0, nt, lane, e)]
                        : 0.f;
-  adj_fetch<DK, DV>(s.buf[(nblk - 1) & 1], k, g, Wws, Xws, Yws, head, nblk - 1, nblk, j0, b,
-                    hh, Tlen, H);
+  if constexpr (NBUF == 2)
+    adj_fetch<DK, DV>(s.buf[(nblk - 1) & 1], k, g, Wws, Xws, Yws, head, nblk - 1, nblk, j0, b,
+                      hh, Tlen, H);
 
   for (int n = nblk - 1; n >= 0; --n) {
     const size_t chunk = head * nblk + n;
-    AdjBuf<DK>& cur = s.buf[n & 1];
+    AdjBuf<DK>& cur = s.buf[NBUF == 2 ? (n & 1) : 0];
+    if constexpr (NBUF == 1) {
+      __syncthreads();  // the previous chunk is done with the buffer
+      adj_fetch<DK, DV>(cur, k, g, Wws, Xws, Yws, head, n, nblk, j0, b, hh, Tlen, H);
+    }
     cp_async_wait_all();
     __syncthreads();  // chunk n's operands are in; the previous chunk is done
-    if (n > 0)
-      adj_fetch<DK, DV>(s.buf[(n - 1) & 1], k, g, Wws, Xws, Yws, head, n - 1, nblk, j0, b, hh,
-                        Tlen, H);
+    if constexpr (NBUF == 2)
+      if (n > 0)
+        adj_fetch<DK, DV>(s.buf[(n - 1) & 1], k, g, Wws, Xws, Yws, head, n - 1, nblk, j0, b,
+                          hh, Tlen, H);
     // dH_{n+1}: to shared memory (operand) and to the workspace
 #pragma unroll
     for (int nt = 0; nt < NTH; ++nt)
@@ -995,17 +1004,20 @@ static cudaError_t launch_chunk_bwd_d(const void* q, const void* k, const void* 
   const auto* kb = (const __nv_bfloat16*)k;
   const auto* vb = (const __nv_bfloat16*)v;
   const auto* ob = (const __nv_bfloat16*)dout;
-  constexpr size_t sp = sizeof(PrepSmem<DK, DV>), sa = sizeof(AdjSmem<DK>),
-                   sg = sizeof(GradSmem<DK, DV>);
+  constexpr size_t sp = sizeof(PrepSmem<DK, DV>), sa = sizeof(AdjSmem<DK, 2>),
+                   sa1 = sizeof(AdjSmem<DK, 1>), sg = sizeof(GradSmem<DK, DV>);
   static_assert(sp <= 227 * 1024 && sa <= 227 * 1024 && sg <= 227 * 1024, "shared memory");
+  static_assert(2 * (sa1 + 1024) <= 228 * 1024, "two single-buffered adjoint CTAs per SM");
   static bool attr_set[64] = {};  // the kernels' shared-memory limits, once per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
     if ((e = cudaFuncSetAttribute(cbwd_prep_kernel<DK, DV>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp)) ||
-        (e = cudaFuncSetAttribute(cbwd_adjoint_kernel<DK, DV>,
+        (e = cudaFuncSetAttribute(cbwd_adjoint_kernel<DK, DV, 2>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa)) ||
+        (e = cudaFuncSetAttribute(cbwd_adjoint_kernel<DK, DV, 1>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa1)) ||
         (e = cudaFuncSetAttribute(cbwd_grad_kernel<DK, DV>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg)))
       return e;
@@ -1013,8 +1025,17 @@ static cudaError_t launch_chunk_bwd_d(const void* q, const void* k, const void* 
   }
   cbwd_prep_kernel<DK, DV><<<dim3(nblk, H, B), NT, sp, st>>>(
       qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, Wws, Xws, Yws, Tlen, H, nblk);
-  cbwd_adjoint_kernel<DK, DV><<<dim3(DV / BVA, H, B), NT, sa, st>>>(
-      kb, g, dhT, Wws, Xws, Yws, dVws, dHws, dh0, Tlen, H, nblk);
+  // one buffer and two CTAs per SM where that turns two waves into one
+  // (149 .. 296 CTAs); otherwise double buffering (measured: 4K layer 0.54 ->
+  // 0.46 ms single-buffered; 512 CTAs 0.55 double- against 0.58 single-)
+  const dim3 agrid(DV / BVA, H, B);
+  const long actas = (long)B * H * (DV / BVA);
+  if (actas > 148 && actas <= 2 * 148)
+    cbwd_adjoint_kernel<DK, DV, 1><<<agrid, NT, sa1, st>>>(kb, g, dhT, Wws, Xws, Yws, dVws,
+                                                           dHws, dh0, Tlen, H, nblk);
+  else
+    cbwd_adjoint_kernel<DK, DV, 2><<<agrid, NT, sa, st>>>(kb, g, dhT, Wws, Xws, Yws, dVws,
+                                                          dHws, dh0, Tlen, H, nblk);
   cbwd_grad_kernel<DK, DV><<<dim3(nblk, H, B), GT, sg, st>>>(
       qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, dVws, dHws, dq, dk, dv, dg, deta, Tlen, H,
       nblk);
