@@ -32,10 +32,12 @@
 //                        into the workspace (fp32)
 //   cbwd_adjoint_kernel  per head and 32-column slab, chunks in reverse:
 //                        dV' = X + Kt dH, dH <- gamma_C dH + Y - W^T dV' (two
-//                        products per chunk), dH in registers, the next
-//                        chunk's operands copied in asynchronously meanwhile;
+//                        products per chunk), dH in registers; the chunk
+//                        operands arrive by asynchronous copies (double
+//                        buffered, or single buffered at two CTAs per SM);
 //                        writes dV'_n and dH_{n+1}
-//   cbwd_grad_kernel     per chunk: every gradient of the chunk's tokens
+//   cbwd_grad_kernel     per chunk (16 warps): every gradient of the chunk's
+//                        tokens, in three phases around one shared-memory plan
 // Products are warp-level tensor-core MMAs (mma.sync m16n8k8, tf32 operands,
 // fp32 sums); operands are read from shared memory through small accessors,
 // so transposed or row-scaled operands need no extra copies.  Ragged tails
