@@ -43,10 +43,12 @@ constexpr int C = 64;
 constexpr int NT = 256;
 constexpr int SB = 16;  // sub-block of rows sharing one decay reference
 
-// Shared memory, two CTAs per SM.  fp32 rows are padded to an odd number of
-// words and bf16 operand rows by 8 elements, so that the threads of a warp
-// reading different rows at one channel (or the fragment loads of a
-// tensor-core product) hit distinct banks.  The union follows the
+// Shared memory, two CTAs per SM.  Rows are padded so that the threads of a
+// warp reading different rows at one channel (or the fragment loads of a
+// tensor-core product) hit distinct banks: the token-major bf16 rows by 2
+// elements (an odd number of words), the gate rows by 2 words (an even
+// stride, so that two channels load as one 8-byte word: 16 rows then cover
+// the 32 banks once), the bf16 operand rows by 8 elements.  The union follows the
 // lifetimes: q, the sub-block operands and A live until T is formed; T and
 // the operands of W after that (T's rows overlap only q and the sub-block
 // operands, never A, which other warps may still be reading while T is
@@ -62,7 +64,7 @@ constexpr size_t kInvBytes = 3 * C * (C + 8) * 2;  // the inverse's first operan
 template <int DK>
 struct KdaPrepSmem {
   __nv_bfloat16 k[C][DK + 2];  // keys, token-major (the bf16 inputs, exact)
-  float g[C][DK + 1];          // G, the in-chunk cumsum of the gate, token-major
+  float g[C][DK + 2];          // G, the in-chunk cumsum of the gate, token-major
   union {
     struct {
       __nv_bfloat16 q[C][DK + 2];       // queries, token-major
@@ -117,9 +119,21 @@ __device__ __forceinline__ void mma_16x8x16(float* d, const __nv_bfloat16* a, in
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Two consecutive bf16 values (4-byte aligned) as floats.
+__device__ __forceinline__ float2 bf16x2_at(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+
 __device__ __forceinline__ void store_bf16_at(uint8_t* tile, int row, int col, float x) {
   reinterpret_cast<__nv_bfloat16*>(tile)[(sw128_chunk_off(row, col >> 3) >> 1) + (col & 7)] =
       __float2bfloat16_rn(x);
+}
+
+// Columns col, col + 1 (col even: one 4-byte word of an 8-column chunk).
+__device__ __forceinline__ void store_bf16x2_at(uint8_t* tile, int row, int col, float x0,
+                                                float x1) {
+  *reinterpret_cast<uint32_t*>(tile + sw128_chunk_off(row, col >> 3) + 2 * (col & 7)) =
+      pack_bf16x2(x0, x1);
 }
 
 __device__ __forceinline__ uint4 pack8(const float* x) {
@@ -160,7 +174,8 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
       kv = *reinterpret_cast<const uint2*>(k + base);
       qv = *reinterpret_cast<const uint2*>(q + base);
     }
-    s.g[tok][i0] = gv.x; s.g[tok][i0 + 1] = gv.y; s.g[tok][i0 + 2] = gv.z; s.g[tok][i0 + 3] = gv.w;
+    *reinterpret_cast<float2*>(&s.g[tok][i0]) = make_float2(gv.x, gv.y);
+    *reinterpret_cast<float2*>(&s.g[tok][i0 + 2]) = make_float2(gv.z, gv.w);
     *reinterpret_cast<uint32_t*>(&s.k[tok][i0]) = kv.x;
     *reinterpret_cast<uint32_t*>(&s.k[tok][i0 + 2]) = kv.y;
     *reinterpret_cast<uint32_t*>(&s.u.p1.q[tok][i0]) = qv.x;
@@ -193,40 +208,65 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     const int tok = p / (DK / 8), i0 = (p % (DK / 8)) * 8;
     float x[8];
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj)
-      x[jj] = __bfloat162float(s.u.p1.q[tok][i0 + jj]) * __expf(s.g[tok][i0 + jj]);
+    for (int jj = 0; jj < 8; jj += 2) {
+      const float2 gg = *reinterpret_cast<const float2*>(&s.g[tok][i0 + jj]);
+      const float2 qq = bf16x2_at(&s.u.p1.q[tok][i0 + jj]);
+      x[jj] = qq.x * __expf(gg.x);
+      x[jj + 1] = qq.y * __expf(gg.y);
+    }
     *reinterpret_cast<uint4*>(out + off.q + (i0 / 64) * 8192 +
                               sw128_chunk_off(tok, (i0 % 64) / 8)) = pack8(x);
   }
 
   // ---- diagonal sub-blocks of A (s < r) and P (s <= r), both tokens in one
-  // sub-block: one thread per pair, one exponential per channel
-  constexpr int NPAIR = SB * (SB + 1) / 2;  // pairs per sub-block, s <= r
-  for (int pi = tid; pi < (C / SB) * NPAIR; pi += NT) {
-    const int blk = pi / NPAIR;
-    int rem = pi % NPAIR, rl = 0;
-    while (rem > rl) {  // pair index -> (row, column) inside the sub-block
-      rem -= rl + 1;
+  // sub-block: one thread per row and pair of columns (row rl of a sub-block
+  // has rl / 2 + 1 pairs; a second column past the diagonal is computed as a
+  // copy of the first and dropped: the zero fill below owns it), two
+  // channels per step (the row's key, query and gate loads serve both
+  // columns), one exponential per (pair, channel)
+  constexpr int TPB = (SB / 2) * (SB / 2 + 1);  // tasks per sub-block
+  for (int ti = tid; ti < (C / SB) * TPB; ti += NT) {
+    const int blk = ti / TPB;
+    int rem = ti % TPB, rl = 0;
+    while (rem > rl / 2) {  // task index -> (row, column pair) inside the sub-block
+      rem -= rl / 2 + 1;
       ++rl;
     }
-    const int r = blk * SB + rl, sc = blk * SB + rem;
-    float aa = 0.f, pp = 0.f;
+    const int r = blk * SB + rl, s0 = blk * SB + 2 * rem;
+    const bool two = s0 + 1 <= r;
+    const int s1 = two ? s0 + 1 : s0;
+    float a0 = 0.f, a1 = 0.f, p0 = 0.f, p1 = 0.f;
 #pragma unroll 4
-    for (int i = 0; i < DK; ++i) {
-      const float x = __bfloat162float(s.k[sc][i]) * __expf(s.g[r][i] - s.g[sc][i]);
-      aa = fmaf(__bfloat162float(s.k[r][i]), x, aa);
-      pp = fmaf(__bfloat162float(s.u.p1.q[r][i]), x, pp);
+    for (int i = 0; i < DK; i += 2) {
+      const float2 gr = *reinterpret_cast<const float2*>(&s.g[r][i]);
+      const float2 g0 = *reinterpret_cast<const float2*>(&s.g[s0][i]);
+      const float2 g1 = *reinterpret_cast<const float2*>(&s.g[s1][i]);
+      const float2 kr = bf16x2_at(&s.k[r][i]), qr = bf16x2_at(&s.u.p1.q[r][i]);
+      const float2 k0 = bf16x2_at(&s.k[s0][i]), k1 = bf16x2_at(&s.k[s1][i]);
+      const float x00 = k0.x * __expf(gr.x - g0.x), x01 = k0.y * __expf(gr.y - g0.y);
+      const float x10 = k1.x * __expf(gr.x - g1.x), x11 = k1.y * __expf(gr.y - g1.y);
+      a0 = fmaf(kr.y, x01, fmaf(kr.x, x00, a0));
+      p0 = fmaf(qr.y, x01, fmaf(qr.x, x00, p0));
+      a1 = fmaf(kr.y, x11, fmaf(kr.x, x10, a1));
+      p1 = fmaf(qr.y, x11, fmaf(qr.x, x10, p1));
     }
-    s.u.p1.a[r][sc] = sc < r ? s.beta[r] * aa : 0.f;
-    store_bf16_at(outP, r, sc, pp);
+    s.u.p1.a[r][s0] = s0 < r ? s.beta[r] * a0 : 0.f;
+    if (two) {
+      s.u.p1.a[r][s1] = s1 < r ? s.beta[r] * a1 : 0.f;
+      store_bf16x2_at(outP, r, s0, p0, p1);  // s0 even
+    } else {
+      store_bf16_at(outP, r, s0, p0);
+    }
   }
-  // zeros of A and P above the diagonal (s > r)
-  for (int p = tid; p < C * C; p += NT) {
-    const int r = p / C, sc = p % C;
-    if (sc > r) {
-      s.u.p1.a[r][sc] = 0.f;
-      store_bf16_at(outP, r, sc, 0.f);
-    }
+  // zeros of P above the diagonal (s > r), by 16-byte chunks of 8 columns
+  // where the whole chunk is above it (A above its diagonal is never read:
+  // the inverse takes only its strictly lower part)
+  for (int p = tid; p < C * (C / 8); p += NT) {
+    const int r = p / (C / 8), c8 = p % (C / 8);
+    if (8 * c8 > r)
+      *reinterpret_cast<uint4*>(outP + sw128_chunk_off(r, c8)) = make_uint4(0u, 0u, 0u, 0u);
+    else
+      for (int sc = r + 1; sc < 8 * c8 + 8; ++sc) store_bf16_at(outP, r, sc, 0.f);
   }
   // ---- off-diagonal sub-blocks: for row sub-block R and s < 16 R the decay
   // factors through the reference G_ref = G at the sub-block's first row:
@@ -235,16 +275,24 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   for (int R = 1; R < C / SB; ++R) {
     const int r0 = R * SB, ns = r0;
     __syncthreads();  // the previous sub-block's products have read x, y
-    for (int p = tid; p < SB * DK; p += NT) {
-      const int rl = p / DK, i = p % DK;
-      const float e = __expf(s.g[r0 + rl][i] - s.g[r0][i]);
-      s.u.p1.x[rl][i] = __float2bfloat16_rn(__bfloat162float(s.k[r0 + rl][i]) * e);
-      s.u.p1.x[SB + rl][i] = __float2bfloat16_rn(__bfloat162float(s.u.p1.q[r0 + rl][i]) * e);
+    for (int p = tid; p < SB * DK / 2; p += NT) {  // two channels per item
+      const int rl = p / (DK / 2), i = 2 * (p % (DK / 2));
+      const float2 gt = *reinterpret_cast<const float2*>(&s.g[r0 + rl][i]);
+      const float2 gf = *reinterpret_cast<const float2*>(&s.g[r0][i]);
+      const float2 kk = bf16x2_at(&s.k[r0 + rl][i]), qq = bf16x2_at(&s.u.p1.q[r0 + rl][i]);
+      const float e0 = __expf(gt.x - gf.x), e1 = __expf(gt.y - gf.y);
+      *reinterpret_cast<__nv_bfloat162*>(&s.u.p1.x[rl][i]) =
+          __floats2bfloat162_rn(kk.x * e0, kk.y * e1);
+      *reinterpret_cast<__nv_bfloat162*>(&s.u.p1.x[SB + rl][i]) =
+          __floats2bfloat162_rn(qq.x * e0, qq.y * e1);
     }
-    for (int p = tid; p < ns * DK; p += NT) {
-      const int sc = p / DK, i = p % DK;
-      s.u.p1.y[sc][i] =
-          __float2bfloat16_rn(__bfloat162float(s.k[sc][i]) * __expf(s.g[r0][i] - s.g[sc][i]));
+    for (int p = tid; p < ns * DK / 2; p += NT) {
+      const int sc = p / (DK / 2), i = 2 * (p % (DK / 2));
+      const float2 gf = *reinterpret_cast<const float2*>(&s.g[r0][i]);
+      const float2 gs = *reinterpret_cast<const float2*>(&s.g[sc][i]);
+      const float2 kk = bf16x2_at(&s.k[sc][i]);
+      *reinterpret_cast<__nv_bfloat162*>(&s.u.p1.y[sc][i]) =
+          __floats2bfloat162_rn(kk.x * __expf(gf.x - gs.x), kk.y * __expf(gf.y - gs.y));
     }
     __syncthreads();
     // [A rows; P rows] (32 x ns) = x (32 x DK) y^T, in 16 x 8 tiles
@@ -258,12 +306,14 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
                     lane);
       const int gq = lane >> 2, tq = lane & 3;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = r0 + gq + 8 * (e >> 1), sc = 8 * nt + 2 * tq + (e & 1);
-        if (mt == 0)
-          s.u.p1.a[r][sc] = s.beta[r] * d[e];
-        else
-          store_bf16_at(outP, r, sc, d[e]);
+      for (int h = 0; h < 2; ++h) {  // rows gq, gq + 8; columns 2 tq, 2 tq + 1
+        const int r = r0 + gq + 8 * h, sc = 8 * nt + 2 * tq;
+        if (mt == 0) {
+          s.u.p1.a[r][sc] = s.beta[r] * d[2 * h];
+          s.u.p1.a[r][sc + 1] = s.beta[r] * d[2 * h + 1];
+        } else {
+          store_bf16x2_at(outP, r, sc, d[2 * h], d[2 * h + 1]);
+        }
       }
     }
   }
@@ -382,9 +432,12 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     const int tok = p / (DK / 8), i0 = (p % (DK / 8)) * 8;
     float x[8];
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      const int i = i0 + jj;
-      x[jj] = __bfloat162float(s.k[tok][i]) * __expf(s.g[C - 1][i] - s.g[tok][i]);
+    for (int jj = 0; jj < 8; jj += 2) {
+      const float2 gl = *reinterpret_cast<const float2*>(&s.g[C - 1][i0 + jj]);
+      const float2 gt = *reinterpret_cast<const float2*>(&s.g[tok][i0 + jj]);
+      const float2 kk = bf16x2_at(&s.k[tok][i0 + jj]);
+      x[jj] = kk.x * __expf(gl.x - gt.x);
+      x[jj + 1] = kk.y * __expf(gl.y - gt.y);
     }
     *reinterpret_cast<uint4*>(out + off.k + (i0 / 64) * 8192 +
                               sw128_chunk_off(tok, (i0 % 64) / 8)) = pack8(x);
@@ -418,9 +471,10 @@ kda_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 #pragma unroll
     for (int q2 = 0; q2 < NTW; ++q2)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = 16 * mt + gq + 8 * (e >> 1), i = 8 * (nt0 + q2) + 2 * tq + (e & 1);
-        store_bf16_at(out + off.w + (i / 64) * 8192, r, i % 64, d[q2][e]);
+      for (int h = 0; h < 2; ++h) {  // rows gq, gq + 8; channels 2 tq, 2 tq + 1
+        const int r = 16 * mt + gq + 8 * h, i = 8 * (nt0 + q2) + 2 * tq;
+        store_bf16x2_at(out + off.w + (i / 64) * 8192, r, i % 64, d[q2][2 * h],
+                        d[q2][2 * h + 1]);
       }
   }
 }
