@@ -219,47 +219,82 @@ __device__ __forceinline__ void unit_lower_inverse(float* Tm, const float* A) {
 using namespace cbwd;
 
 // ---------------------------------------------------------------- prep
+// Two CTAs per SM: the shared-memory plan follows the lifetimes.  The start
+// state h_n passes through in 64-row pieces, only to form K h_n (kept in
+// registers), so V' = T (diag(beta) V - diag(beta gamma) K h_n) needs neither
+// W nor h_n as a tile (W = T diag(beta gamma) K, so W h_n is the same
+// product reassociated); the right operand Z of that last product takes the
+// place of the queries and dL/do once X and Y are formed.
+constexpr int HR = 64;  // rows of h_n staged at a time
+
 template <int DK, int DV>
 struct PrepSmem {
   __nv_bfloat16 kb[C][LB<DK>()];
   __nv_bfloat16 vb[C][LB<DV>()];
-  __nv_bfloat16 qb[C][LB<DK>()];
-  __nv_bfloat16 ob[C][LB<DV>()];
-  float A[C][LF<C>()];  // A, then P
-  float Tm[C][LF<C>()];
-  float W[C][LF<DK>()];
-  float h[DK][LF<DV>()];
+  union {
+    struct {
+      __nv_bfloat16 qb[C][LB<DK>()];
+      __nv_bfloat16 ob[C][LB<DV>()];
+    } in;
+    float Z[C][LF<DV>()];  // diag(beta) V - diag(beta gamma) K h_n
+  } qo;
+  union {
+    float h[HR][LF<DV>()];  // rows of h_n
+    struct {
+      float A[C][LF<C>()];  // A, then P
+      float Tm[C][LF<C>()];
+    } at;
+  } u;
   float G[C], gam[C], beta[C], n2[C];
 };
 
 // Per chunk: T, V' = T diag(beta) V - W h_n, W, X = P^T dO and
 // Y = (diag(gamma) Q)^T dO into the workspace.
 template <int DK, int DV>
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(NT, 2)
 cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                  const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
                  const float* __restrict__ g, const float* __restrict__ eta, float eps,
                  const float* __restrict__ ck, float* __restrict__ Tws, float* __restrict__ Vws,
                  float* __restrict__ Wws, float* __restrict__ Xws, float* __restrict__ Yws,
                  int Tlen, int H, int nblk) {
+  using Smem = PrepSmem<DK, DV>;
+  static_assert(sizeof(Smem::qo.Z) <= sizeof(Smem::qo.in), "Z over the queries and dL/do");
+  static_assert(sizeof(Smem::u.h) <= sizeof(Smem::u.at), "h_n rows over A and T");
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  auto& s = *reinterpret_cast<PrepSmem<DK, DV>*>(smem_raw);
+  auto& s = *reinterpret_cast<Smem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
   const size_t head = (size_t)b * H + hh, chunk = head * nblk + n;
   const int t0 = n * C, len = min(C, Tlen - t0);
   const size_t tok0 = ((size_t)b * Tlen + t0) * H + hh;
+  const float* hsrc = ck + chunk * DK * DV;
 
   load_rows_bf16<DK>(&s.kb[0][0], k + tok0 * DK, (size_t)H * DK, len);
   load_rows_bf16<DV>(&s.vb[0][0], v + tok0 * DV, (size_t)H * DV, len);
-  load_rows_bf16<DK>(&s.qb[0][0], q + tok0 * DK, (size_t)H * DK, len);
-  load_rows_bf16<DV>(&s.ob[0][0], dout + tok0 * DV, (size_t)H * DV, len);
-  load_f32<DK, DV>(&s.h[0][0], ck + chunk * DK * DV, DV);
+  load_rows_bf16<DK>(&s.qo.in.qb[0][0], q + tok0 * DK, (size_t)H * DK, len);
+  load_rows_bf16<DV>(&s.qo.in.ob[0][0], dout + tok0 * DV, (size_t)H * DV, len);
+  load_f32<HR, DV>(&s.u.h[0][0], hsrc, DV);
   copies_landed();
   chunk_scalars<DK>(s.G, s.gam, s.beta, s.n2, &s.kb[0][0], g, eta, eps, tok0, H, len);
-  __syncthreads();
 
   const int mt = warp & 3, nh = warp >> 2;  // m-tile of 16 rows; column half
+  // K h_n: rows 16 mt.., columns (DV / 2) nh.. of this warp, by HR-row pieces
+  float kh[DV / 16][4];
+  zero(kh);
+#pragma unroll 1
+  for (int i0 = 0; i0 < DK; i0 += HR) {
+    if (i0 > 0) {
+      __syncthreads();  // every warp is done with the previous piece
+      load_f32<HR, DV>(&s.u.h[0][0], hsrc + (size_t)i0 * DV, DV);
+      copies_landed();
+    }
+    auto Ka = [&](int r, int i) { return bf(s.kb[r][i0 + i]); };
+    auto Hb = [&](int i, int j) { return s.u.h[i][j]; };
+    mma_rows<DV / 16>(kh, Ka, Hb, 16 * mt, (DV / 2) * nh, HR, lane);
+  }
+  __syncthreads();  // h_n read (A and T take its place); the scalars are in
+
   {  // A = beta_r (k_r . k_s) Gamma_rs, s < r
     float d[4][4];
     zero(d);
@@ -271,16 +306,16 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
-        s.A[r][c] = c < r ? s.beta[r] * d[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;
+        s.u.at.A[r][c] = c < r ? s.beta[r] * d[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;
       }
   }
   __syncthreads();
-  unit_lower_inverse(&s.Tm[0][0], &s.A[0][0]);
+  unit_lower_inverse(&s.u.at.Tm[0][0], &s.u.at.A[0][0]);
   __syncthreads();
-  {  // W = T diag(beta gamma) K
+  {  // W = T diag(beta gamma) K (to the workspace only)
     float d[DK / 16][4];
     zero(d);
-    auto Ta = [&](int r, int c) { return s.Tm[r][c]; };
+    auto Ta = [&](int r, int c) { return s.u.at.Tm[r][c]; };
     auto Kb = [&](int c, int i) { return s.beta[c] * s.gam[c] * bf(s.kb[c][i]); };
     mma_rows<DK / 16>(d, Ta, Kb, 16 * mt, (DK / 2) * nh, C, lane);
     float* wdst = Wws + chunk * C * DK;
@@ -289,15 +324,13 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll
       for (int e = 0; e < 4; e += 2) {
         const int r = frow(16 * mt, lane, e), i = fcol((DK / 2) * nh, nt, lane, e);
-        s.W[r][i] = d[nt][e];
-        s.W[r][i + 1] = d[nt][e + 1];
         *reinterpret_cast<float2*>(wdst + r * DK + i) = make_float2(d[nt][e], d[nt][e + 1]);
       }
   }
   {  // P = lower_incl(Q K^T (*) Gamma) over A (no longer read after the inverse)
     float p[4][4];
     zero(p);
-    auto Qa = [&](int r, int i) { return bf(s.qb[r][i]); };
+    auto Qa = [&](int r, int i) { return bf(s.qo.in.qb[r][i]); };
     auto Kb = [&](int i, int c) { return bf(s.kb[c][i]); };
     mma_rows<4>(p, Qa, Kb, 16 * mt, 32 * nh, DK, lane);
 #pragma unroll
@@ -305,7 +338,7 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = frow(16 * mt, lane, e), c = fcol(32 * nh, nt, lane, e);
-        s.A[r][c] = c <= r ? p[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;
+        s.u.at.A[r][c] = c <= r ? p[nt][e] * __expf(s.G[r] - s.G[c]) : 0.f;
       }
   }
   __syncthreads();
@@ -313,8 +346,8 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
      // warp w takes row tile w and both column halves, with 4 it takes row
      // tile w % 4 and column half w / 4
     constexpr int RT = DK / 16;
-    auto QTa = [&](int i, int c) { return s.gam[c] * bf(s.qb[c][i]); };
-    auto Ob = [&](int c, int j) { return bf(s.ob[c][j]); };
+    auto QTa = [&](int i, int c) { return s.gam[c] * bf(s.qo.in.qb[c][i]); };
+    auto Ob = [&](int c, int j) { return bf(s.qo.in.ob[c][j]); };
     float* ydst = Yws + chunk * DK * DV;
     const int ym = warp % RT;
     for (int half = RT == 8 ? 0 : warp / RT; half < 2; half += RT == 8 ? 1 : 2) {
@@ -333,8 +366,8 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   {  // X = P^T dO  [C x DV]
     float d[DV / 16][4];
     zero(d);
-    auto PTa = [&](int r, int c) { return s.A[c][r]; };
-    auto Ob = [&](int c, int j) { return bf(s.ob[c][j]); };
+    auto PTa = [&](int r, int c) { return s.u.at.A[c][r]; };
+    auto Ob = [&](int c, int j) { return bf(s.qo.in.ob[c][j]); };
     mma_rows<DV / 16>(d, PTa, Ob, 16 * mt, (DV / 2) * nh, C, lane);
     float* xdst = Xws + chunk * C * DV;
 #pragma unroll
@@ -345,15 +378,21 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         *reinterpret_cast<float2*>(xdst + r * DV + j) = make_float2(d[nt][e], d[nt][e + 1]);
       }
   }
-  {  // V' = T diag(beta) V - W h_n
+  __syncthreads();  // the queries and dL/do are read: Z takes their place
+#pragma unroll
+  for (int nt = 0; nt < DV / 16; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = frow(16 * mt, lane, e), j = fcol((DV / 2) * nh, nt, lane, e);
+      s.qo.Z[r][j] = s.beta[r] * (bf(s.vb[r][j]) - s.gam[r] * kh[nt][e]);
+    }
+  __syncthreads();
+  {  // V' = T Z
     float d[DV / 16][4];
     zero(d);
-    auto Ta = [&](int r, int c) { return s.Tm[r][c]; };
-    auto Vb = [&](int c, int j) { return s.beta[c] * bf(s.vb[c][j]); };
-    mma_rows<DV / 16>(d, Ta, Vb, 16 * mt, (DV / 2) * nh, C, lane);
-    auto Wa = [&](int r, int i) { return -s.W[r][i]; };
-    auto Hb = [&](int i, int j) { return s.h[i][j]; };
-    mma_rows<DV / 16>(d, Wa, Hb, 16 * mt, (DV / 2) * nh, DK, lane);
+    auto Ta = [&](int r, int c) { return s.u.at.Tm[r][c]; };
+    auto Zb = [&](int c, int j) { return s.qo.Z[c][j]; };
+    mma_rows<DV / 16>(d, Ta, Zb, 16 * mt, (DV / 2) * nh, C, lane);
     float* dst = Vws + chunk * C * DV;
 #pragma unroll
     for (int nt = 0; nt < DV / 16; ++nt)
@@ -365,7 +404,7 @@ cbwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
   }
   {
     float* dst = Tws + chunk * C * C;
-    for (int p = tid; p < C * C; p += NT) dst[p] = s.Tm[p / C][p % C];
+    for (int p = tid; p < C * C; p += NT) dst[p] = s.u.at.Tm[p / C][p % C];
   }
 }
 
