@@ -27,14 +27,15 @@
 //
 // Kernels (after the forward chunk prefill of kla_ut.cu / kla_chunk_tc.cu run
 // with its outputs off and its chain writing every h_n, fp32):
-//   cbwd_prep_kernel     per chunk: T, V', W and the two dH-independent terms
-//                        of the chain, X = P^T dO and Y = (diag(gamma) Q)^T dO,
-//                        into the workspace (fp32)
+//   cbwd_prep_kernel     per chunk (two CTAs per SM): T, V', W and the two
+//                        dH-independent terms of the chain, X = P^T dO and
+//                        Y = (diag(gamma) Q)^T dO, into the workspace (fp32)
 //   cbwd_adjoint_kernel  per head and 32-column slab, chunks in reverse:
 //                        dV' = X + Kt dH, dH <- gamma_C dH + Y - W^T dV' (two
 //                        products per chunk), dH in registers; the chunk
 //                        operands arrive by asynchronous copies (double
-//                        buffered, or single buffered at two CTAs per SM);
+//                        buffered at 16 warps, or single buffered at 8 warps
+//                        and two CTAs per SM);
 //                        writes dV'_n and dH_{n+1}
 //   cbwd_grad_kernel     per chunk (16 warps): every gradient of the chunk's
 //                        tokens, in three phases around one shared-memory plan
@@ -466,9 +467,9 @@ __device__ __forceinline__ void adj_fetch(AdjBuf<DK>& d, const __nv_bfloat16* k,
 
 // One CTA per (head, 32-column slab); chunks in reverse.  dH (the adjoint of
 // h_{n+1}) lives in registers.  NBUF = 2: the next chunk's operands are
-// copied in while the current one is worked on (for few CTAs, one per SM);
-// NBUF = 1: one buffer, small enough for two CTAs per SM, whose work hides
-// each other's copies (for many CTAs).
+// copied in while the current one is worked on (for few CTAs, one per SM,
+// 16 warps); NBUF = 1: one buffer, small enough for two CTAs of 8 warps per
+// SM, whose work hides each other's copies (for many CTAs).
 template <int DK, int DV, int NBUF>
 __global__ void __launch_bounds__(adj_threads<NBUF>())
 cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict__ g,
