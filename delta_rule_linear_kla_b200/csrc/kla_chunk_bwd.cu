@@ -34,8 +34,7 @@
 //                        dV' = X + Kt dH, dH <- gamma_C dH + Y - W^T dV' (two
 //                        products per chunk), dH in registers; the chunk
 //                        operands arrive by asynchronous copies (double
-//                        buffered at 16 warps, or single buffered at 8 warps
-//                        and two CTAs per SM);
+//                        buffered, or single buffered at two CTAs per SM);
 //                        writes dV'_n and dH_{n+1}
 //   cbwd_grad_kernel     per chunk (16 warps): every gradient of the chunk's
 //                        tokens, in three phases around one shared-memory plan
@@ -52,9 +51,6 @@ namespace cbwd {
 constexpr int C = 64;
 constexpr int NT = 256;
 constexpr int BVA = 32;  // state columns per adjoint-chain CTA
-// Threads of an adjoint-chain CTA: 16 warps when it has an SM to itself
-// (double-buffered), 8 when two share one (single-buffered).
-template <int NBUF> constexpr int adj_threads() { return NBUF == 2 ? 512 : 256; }
 
 // An fp32 value rounded to a tf32 operand (to nearest; the tensor core would
 // otherwise truncate, which measured three times the gradient error).
@@ -433,7 +429,7 @@ struct AdjSmem {
 };
 
 // Copies of chunk n's operands into a buffer (zero rows past the sequence).
-template <int DK, int DV, int AT>
+template <int DK, int DV>
 __device__ __forceinline__ void adj_fetch(AdjBuf<DK>& d, const __nv_bfloat16* k,
                                           const float* g, const float* Wws, const float* Xws,
                                           const float* Yws, size_t head, int n, int nblk,
@@ -441,20 +437,20 @@ __device__ __forceinline__ void adj_fetch(AdjBuf<DK>& d, const __nv_bfloat16* k,
   const size_t chunk = head * nblk + n;
   const int t0 = n * C, len = min(C, Tlen - t0);
   const size_t tok0 = ((size_t)b * Tlen + t0) * H + hh;
-  for (int p = threadIdx.x; p < C * (DK / 8); p += AT) {  // keys, bf16
+  for (int p = threadIdx.x; p < C * (DK / 8); p += NT) {  // keys, bf16
     const int r = p / (DK / 8), ch = p % (DK / 8);
     const bool ok = r < len;
     cp_async16(&d.kb[r][ch * 8], k + (ok ? (tok0 + (size_t)r * H) * DK + ch * 8 : 0), ok);
   }
-  for (int p = threadIdx.x; p < C * (DK / 4); p += AT) {  // W
+  for (int p = threadIdx.x; p < C * (DK / 4); p += NT) {  // W
     const int r = p / (DK / 4), ch = p % (DK / 4);
     cp_async16(&d.W[r][ch * 4], Wws + (chunk * C + r) * DK + ch * 4, true);
   }
-  for (int p = threadIdx.x; p < C * (BVA / 4); p += AT) {  // X columns j0 ..
+  for (int p = threadIdx.x; p < C * (BVA / 4); p += NT) {  // X columns j0 ..
     const int r = p / (BVA / 4), ch = p % (BVA / 4);
     cp_async16(&d.X[r][ch * 4], Xws + (chunk * C + r) * DV + j0 + ch * 4, true);
   }
-  for (int p = threadIdx.x; p < DK * (BVA / 4); p += AT) {  // Y columns j0 ..
+  for (int p = threadIdx.x; p < DK * (BVA / 4); p += NT) {  // Y columns j0 ..
     const int r = p / (BVA / 4), ch = p % (BVA / 4);
     cp_async16(&d.Y[r][ch * 4], Yws + (chunk * DK + r) * DV + j0 + ch * 4, true);
   }
@@ -467,21 +463,20 @@ __device__ __forceinline__ void adj_fetch(AdjBuf<DK>& d, const __nv_bfloat16* k,
 
 // One CTA per (head, 32-column slab); chunks in reverse.  dH (the adjoint of
 // h_{n+1}) lives in registers.  NBUF = 2: the next chunk's operands are
-// copied in while the current one is worked on (for few CTAs, one per SM,
-// 16 warps); NBUF = 1: one buffer, small enough for two CTAs of 8 warps per
-// SM, whose work hides each other's copies (for many CTAs).
+// copied in while the current one is worked on (for few CTAs, one per SM);
+// NBUF = 1: one buffer, small enough for two CTAs per SM, whose work hides
+// each other's copies (for many CTAs).
 template <int DK, int DV, int NBUF>
-__global__ void __launch_bounds__(adj_threads<NBUF>())
+__global__ void __launch_bounds__(NT)
 cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict__ g,
                     const float* __restrict__ dhT, const float* __restrict__ Wws,
                     const float* __restrict__ Xws, const float* __restrict__ Yws,
                     float* __restrict__ dVws, float* __restrict__ dHws, float* __restrict__ dh0,
                     int Tlen, int H, int nblk) {
-  // the dH slab [DK x 32] in 16-row tiles: DK / 16 of them, AT / 32 / (DK / 16)
+  // the dH slab [DK x 32] in 16-row tiles: DK / 16 of them, NT / 32 / (DK / 16)
   // warps per tile splitting its columns
-  constexpr int AT = adj_threads<NBUF>();
-  constexpr int RT = DK / 16, WPT = (AT / 32) / RT, NTH = (BVA / 8) / WPT;
-  static_assert(RT * WPT == AT / 32 && NTH >= 1, "state tiling");
+  constexpr int RT = DK / 16, WPT = (NT / 32) / RT, NTH = (BVA / 8) / WPT;
+  static_assert(RT * WPT == NT / 32 && NTH >= 1, "state tiling");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   auto& s = *reinterpret_cast<AdjSmem<DK, NBUF>*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -499,7 +494,7 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict
                              fcol(hn0, nt, lane, e)]
                        : 0.f;
   if constexpr (NBUF == 2)
-    adj_fetch<DK, DV, AT>(s.buf[(nblk - 1) & 1], k, g, Wws, Xws, Yws, head, nblk - 1, nblk, j0, b,
+    adj_fetch<DK, DV>(s.buf[(nblk - 1) & 1], k, g, Wws, Xws, Yws, head, nblk - 1, nblk, j0, b,
                       hh, Tlen, H);
 
   for (int n = nblk - 1; n >= 0; --n) {
@@ -507,13 +502,13 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict
     AdjBuf<DK>& cur = s.buf[NBUF == 2 ? (n & 1) : 0];
     if constexpr (NBUF == 1) {
       __syncthreads();  // the previous chunk is done with the buffer
-      adj_fetch<DK, DV, AT>(cur, k, g, Wws, Xws, Yws, head, n, nblk, j0, b, hh, Tlen, H);
+      adj_fetch<DK, DV>(cur, k, g, Wws, Xws, Yws, head, n, nblk, j0, b, hh, Tlen, H);
     }
     cp_async_wait_all();
     __syncthreads();  // chunk n's operands are in; the previous chunk is done
     if constexpr (NBUF == 2)
       if (n > 0)
-        adj_fetch<DK, DV, AT>(s.buf[(n - 1) & 1], k, g, Wws, Xws, Yws, head, n - 1, nblk, j0, b,
+        adj_fetch<DK, DV>(s.buf[(n - 1) & 1], k, g, Wws, Xws, Yws, head, n - 1, nblk, j0, b,
                           hh, Tlen, H);
     // dH_{n+1}: to shared memory (operand) and to the workspace
 #pragma unroll
@@ -541,22 +536,21 @@ cbwd_adjoint_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict
     }
     __syncthreads();
     const int mt = warp & 3, nq = warp >> 2;
-    {  // dV' = X + Kt dH_{n+1}   [C x 32]: warp (mt, nq) has VT column tiles of 8
-      constexpr int VT = 4 / (AT / 128);
-      float d[VT][4];
+    {  // dV' = X + Kt dH_{n+1}   [C x 32]: warp (mt, nq) has 2 column tiles
+      float d[2][4];
 #pragma unroll
-      for (int nt = 0; nt < VT; ++nt)
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          d[nt][e] = cur.X[frow(16 * mt, lane, e)][fcol(8 * VT * nq, nt, lane, e)];
+          d[nt][e] = cur.X[frow(16 * mt, lane, e)][fcol(16 * nq, nt, lane, e)];
       auto Kta = [&](int r, int i) { return s.kts[r] * bf(cur.kb[r][i]); };
       auto Hb = [&](int i, int j) { return s.dH[i][j]; };
-      mma_rows<VT>(d, Kta, Hb, 16 * mt, 8 * VT * nq, DK, lane);
+      mma_rows<2>(d, Kta, Hb, 16 * mt, 16 * nq, DK, lane);
 #pragma unroll
-      for (int nt = 0; nt < VT; ++nt)
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; e += 2) {
-          const int r = frow(16 * mt, lane, e), c = fcol(8 * VT * nq, nt, lane, e);
+          const int r = frow(16 * mt, lane, e), c = fcol(16 * nq, nt, lane, e);
           s.dV[r][c] = d[nt][e];
           s.dV[r][c + 1] = d[nt][e + 1];
           *reinterpret_cast<float2*>(dVws + (chunk * C + r) * DV + j0 + c) =
@@ -1078,10 +1072,10 @@ static cudaError_t launch_chunk_bwd_d(const void* q, const void* k, const void* 
   const dim3 agrid(DV / BVA, H, B);
   const long actas = (long)B * H * (DV / BVA);
   if (actas > 148 && actas <= 2 * 148)
-    cbwd_adjoint_kernel<DK, DV, 1><<<agrid, adj_threads<1>(), sa1, st>>>(kb, g, dhT, Wws, Xws, Yws, dVws,
+    cbwd_adjoint_kernel<DK, DV, 1><<<agrid, NT, sa1, st>>>(kb, g, dhT, Wws, Xws, Yws, dVws,
                                                            dHws, dh0, Tlen, H, nblk);
   else
-    cbwd_adjoint_kernel<DK, DV, 2><<<agrid, adj_threads<2>(), sa, st>>>(kb, g, dhT, Wws, Xws, Yws, dVws,
+    cbwd_adjoint_kernel<DK, DV, 2><<<agrid, NT, sa, st>>>(kb, g, dhT, Wws, Xws, Yws, dVws,
                                                           dHws, dh0, Tlen, H, nblk);
   cbwd_grad_kernel<DK, DV><<<dim3(nblk, H, B), GT, sg, st>>>(
       qb, kb, vb, ob, g, eta, eps, ck, Tws, Vws, dVws, dHws, dq, dk, dv, dg, deta, Tlen, H,
