@@ -28,6 +28,10 @@ A ragged tail is padded with g = 0, beta = 0 and zero vectors, which is an
 exact identity step.  It is pinned against the token recurrence in the tests
 for C in {1, 2, 4, 8, 64}; it exposes T, W, U, V' and the per-chunk states so
 GPU stages can be checked one by one.
+
+The module also holds the reverse mode of the same chunk form (the
+chunkwise adjoint, derived below since the pages print no backward), pinned
+against the oracle's token-loop gradients for C in {1, 3, 8, 64}.
 """
 from __future__ import annotations
 
@@ -97,3 +101,129 @@ def forward(q, k, v, g, beta, h0=None, C: int = 64, keep: bool = False):
     if keep:
         return o, hT, inters
     return o, hT
+
+
+# ---------------------------------------------------------------- reverse mode
+#
+# The pages print no backward.  Differentiating the chunk form above by hand
+# (loss L with dL/do and dL/dh_T given) splits it into one reverse chain over
+# the chunks and independent per-chunk terms.  With Gam_rs = e^{G_r - G_s},
+# gam = e^G, gC = e^{G_{C-1}}, Qt = diag(gam) Q, Kt = diag(gC / gam) K, the
+# strict (s < r) and inclusive (s <= r) masks, and dH the adjoint of the
+# state after the chunk:
+#
+#   dV' = P^T dO + Kt dH                     (V' enters O and h_{n+1})
+#   dh_n = gC dH + Qt^T dO - W^T dV'         (the chain, chunk by chunk)
+#   dP = (dO V'^T) masked inclusive;  dQ = diag(gam) dO h_n^T + (dP * Gam) K
+#   dW = -dV' h_n^T;  dU = dV';  dT = dW (diag(beta gam) K)^T + dU (diag(beta) V)^T
+#   dA = -strict(T^T dT T^T)                 (T = (I + A)^{-1})
+#   dK = (dP * Gam)^T Q + diag(gC / gam) V' dH^T + diag(beta gam) T^T dW
+#        + diag(beta) (dA * Gam) K + (diag(beta) (dA * Gam))^T K
+#   dV = diag(beta) T^T dU
+#   dbeta = gam * rowdot(T^T dW, K) + rowdot(T^T dU, V) + rowsum(dA * Gam * K K^T)
+#   dG = rowsum - colsum of (dA * A) and of (dP * P) + rowdot(dO, Qt h_n)
+#        + beta gam rowdot(T^T dW, K) - rowdot(V' dH^T, Kt),
+#   dG_{C-1} += sum rowdot(V' dH^T, Kt) + gC <dH, h_n>,
+#   dg = reverse in-chunk cumsum of dG (G_r = sum_{j <= r} g_j).
+#
+# It is pinned in the tests against the token-loop gradients of the oracle
+# (themselves pinned by finite differences) for several chunk lengths.
+
+def _chunk_head_backward(q, k, v, g, beta, h, do, dh, C):
+    """One head, beta given.  Returns dq, dk, dv, dg, dbeta, dh0."""
+    T, dk = k.shape
+    dv = v.shape[1]
+    nchunks = (T + C - 1) // C
+    pad = nchunks * C - T
+    if pad:  # identity steps, as in the forward; their gradients are dropped
+        z = lambda a, w: np.concatenate([a, np.zeros((pad, w))])
+        q, k, v, do = z(q, dk), z(k, dk), z(v, dv), z(do, dv)
+        g = np.concatenate([g, np.zeros(pad)])
+        beta = np.concatenate([beta, np.zeros(pad)])
+    r_idx = np.arange(C)[:, None]
+    s_idx = np.arange(C)[None, :]
+    strict = s_idx < r_idx
+    incl = s_idx <= r_idx
+    # forward, keeping what the reverse pass reads
+    saved = []
+    h = h.copy()
+    for n in range(nchunks):
+        sl = slice(n * C, (n + 1) * C)
+        Q, K, V, bb = q[sl], k[sl], v[sl], beta[sl]
+        G = np.cumsum(g[sl])
+        D = G[:, None] - G[None, :]
+        Gam = np.exp(np.where(incl, D, 0.0)) * incl
+        A = bb[:, None] * (K @ K.T) * Gam * strict
+        Tm = np.linalg.inv(np.eye(C) + A)
+        gam = np.exp(G)
+        W = Tm @ ((bb * gam)[:, None] * K)
+        Vp = Tm @ (bb[:, None] * V) - W @ h
+        P = (Q @ K.T) * Gam
+        Kt = np.exp(G[-1] - G)[:, None] * K
+        saved.append((h.copy(), G, Gam, A, Tm, gam, W, Vp, P, Kt))
+        h = np.exp(G[-1]) * h + Kt.T @ Vp
+    out_q, out_k, out_v = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    out_g, out_b = np.zeros(len(g)), np.zeros(len(g))
+    dH = dh.copy()
+    for n in range(nchunks - 1, -1, -1):
+        sl = slice(n * C, (n + 1) * C)
+        Q, K, V, bb, dO = q[sl], k[sl], v[sl], beta[sl], do[sl]
+        hn, G, Gam, A, Tm, gam, W, Vp, P, Kt = saved[n]
+        gC = np.exp(G[-1])
+        Qt = gam[:, None] * Q
+        dVp = P.T @ dO + Kt @ dH
+        dP = (dO @ Vp.T) * incl
+        dPG = dP * Gam
+        dKt = Vp @ dH.T
+        TdW = Tm.T @ (-dVp @ hn.T)
+        TdU = Tm.T @ dVp
+        dT = (-dVp @ hn.T) @ ((bb * gam)[:, None] * K).T + dVp @ (bb[:, None] * V).T
+        dA = -(Tm.T @ dT @ Tm.T) * strict
+        E = dA * Gam
+        out_q[sl] = gam[:, None] * (dO @ hn.T) + dPG @ K
+        out_k[sl] = (dPG.T @ Q + np.exp(G[-1] - G)[:, None] * dKt + (bb * gam)[:, None] * TdW
+                     + bb[:, None] * (E @ K) + (bb[:, None] * E).T @ K)
+        out_v[sl] = bb[:, None] * TdU
+        out_b[sl] = (gam * (TdW * K).sum(1) + (TdU * V).sum(1) + (E * (K @ K.T)).sum(1))
+        FA, FP = dA * A, dP * P
+        dG = (FA.sum(1) - FA.sum(0) + FP.sum(1) - FP.sum(0) + (dO * (Qt @ hn)).sum(1)
+              + bb * gam * (TdW * K).sum(1) - (dKt * Kt).sum(1))
+        dG[-1] += (dKt * Kt).sum() + gC * (dH * hn).sum()
+        out_g[sl] = np.cumsum(dG[::-1])[::-1]
+        dH = gC * dH + Qt.T @ dO - W.T @ dVp
+    return out_q[:T], out_k[:T], out_v[:T], out_g[:T], out_b[:T], dH
+
+
+def gated_delta_backward(q, k, v, g, beta, h0, do, dhT, C: int = 64):
+    """Chunk-form gradients of the gated delta rule (beta given) for
+    dL/do = do and dL/dh_T = dhT.  Returns dq, dk, dv, dg, dbeta, dh0 (fp64)."""
+    q, k, v, g, beta, do = map(f64, (q, k, v, g, beta, do))
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    h0 = np.zeros((B, H, dk, dv)) if h0 is None else f64(h0)
+    dhT = np.zeros((B, H, dk, dv)) if dhT is None else f64(dhT)
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v),
+               dg=np.zeros((B, T, H)), dbeta=np.zeros((B, T, H)), dh0=np.zeros((B, H, dk, dv)))
+    for b in range(B):
+        for hh in range(H):
+            r = _chunk_head_backward(q[b, :, hh], k[b, :, hh], v[b, :, hh], g[b, :, hh],
+                                     beta[b, :, hh], h0[b, hh], do[b, :, hh], dhT[b, hh], C)
+            for name, x in zip(("dq", "dk", "dv", "dg", "dbeta"), r[:5]):
+                out[name][b, :, hh] = x
+            out["dh0"][b, hh] = r[5]
+    return out
+
+
+def backward(q, k, v, g, eta, eps: float, h0, do, dhT, C: int = 64):
+    """Chunk-form gradients of KLA (beta = eta / (||k||^2 + eps), "Kaczmarz
+    Linear Attention", Abstract): the gated-delta gradients above, then the
+    step size's chain rule, deta = dbeta / (||k||^2 + eps) and
+    dk -= 2 dbeta eta k / (||k||^2 + eps)^2.  Returns dq, dk, dv, dg, deta,
+    dh0 (fp64)."""
+    k64, eta64 = f64(k), f64(eta)
+    den = (k64 * k64).sum(-1) + eps
+    out = gated_delta_backward(q, k64, v, g, eta64 / den, h0, do, dhT, C)
+    dbeta = out.pop("dbeta")
+    out["deta"] = dbeta / den
+    out["dk"] = out["dk"] - (2.0 * dbeta * eta64 / den ** 2)[..., None] * k64
+    return out

@@ -148,3 +148,36 @@ def test_kda_gradients_reduce_to_scalar_gate():
     for n in ("dq", "dk", "dv", "dbeta", "dh0"):
         np.testing.assert_allclose(a[n], b[n], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(a["dg"].sum(-1), b["dg"], rtol=1e-10, atol=1e-12)
+
+
+# ---- the chunkwise adjoint (the algebra the GPU backward kernels follow),
+# evaluated in fp64 by oracle.chunk_form and held to the token-loop gradients
+# above: chunk lengths 1 (no intra-chunk coupling), 3 and 8 (ragged chunks)
+# and 64 (the GPU's), a sequence that ends inside a chunk, and gates strong
+# enough that e^G underflows inside a chunk.
+
+from oracle import chunk_form  # noqa: E402
+
+
+@pytest.mark.parametrize("C", [1, 3, 8, 64])
+def test_chunk_form_backward_matches_token_loop(C):
+    x, dout, dhT = _problem(41, B=2, T=150, H=2, dk=6, dv=5)
+    eps = 1e-6
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["eta"], eps, x["h0"], dout, dhT)
+    got = chunk_form.backward(x["q"], x["k"], x["v"], x["g"], x["eta"], eps, x["h0"], dout, dhT,
+                              C=C)
+    for n in ("dq", "dk", "dv", "dg", "deta", "dh0"):
+        assert oracle.rel_l2(got[n], ref[n]) < 1e-12, (C, n)
+
+
+def test_chunk_form_backward_gated_delta_and_strong_gates():
+    x, dout, dhT = _problem(42, T=130, dk=6, dv=5)
+    r = np.random.Generator(np.random.PCG64(43))
+    x["g"] = np.where(r.uniform(size=x["g"].shape) < 0.3, -40.0, x["g"])  # e^G underflows
+    beta = r.uniform(0.05, 1.5, x["g"].shape)
+    ref = oracle.gated_delta_backward(x["q"], x["k"], x["v"], x["g"], beta, x["h0"], dout, dhT)
+    got = chunk_form.gated_delta_backward(x["q"], x["k"], x["v"], x["g"], beta, x["h0"], dout,
+                                          dhT, C=64)
+    for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
+        assert np.all(np.isfinite(got[n])), n
+        assert oracle.rel_l2(got[n], ref[n]) < 1e-11, n
