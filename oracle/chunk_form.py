@@ -30,8 +30,9 @@ for C in {1, 2, 4, 8, 64}; it exposes T, W, U, V' and the per-chunk states so
 GPU stages can be checked one by one.
 
 The module also holds the reverse mode of the same chunk form (the
-chunkwise adjoint, derived below since the pages print no backward), pinned
-against the oracle's token-loop gradients for C in {1, 3, 8, 64}.
+chunkwise adjoint, derived below since the pages print no backward), and
+the chunk form of the per-channel-gate rule with its reverse mode, all
+pinned against the oracle's token loops for C in {1, 3, 8, 64}.
 """
 from __future__ import annotations
 
@@ -226,4 +227,143 @@ def backward(q, k, v, g, eta, eps: float, h0, do, dhT, C: int = 64):
     dbeta = out.pop("dbeta")
     out["deta"] = dbeta / den
     out["dk"] = out["dk"] - (2.0 * dbeta * eta64 / den ** 2)[..., None] * k64
+    return out
+
+
+# ---------------------------------------------------------------- per-channel gate
+#
+# The chunk form of the per-channel-gate rule ("Deep Dive into KDA", section
+# 2.3, decay before the erase): one log-gate per key channel, G [C, dk] its
+# in-chunk cumsum, and E[r, s, i] = e^{G_ri - G_si} for s <= r (never above
+# 1).  Unrolling the recurrence over a chunk from h_n gives
+#
+#   A_rs = beta_r sum_i k_ri k_si E_rsi  (s < r),   T = (I + A)^{-1}
+#   W = T diag(beta) (K o e^G),  U = T diag(beta) V,  V' = U - W h_n
+#   O = (Q o e^G) h_n + P V',   P_rs = sum_i q_ri k_si E_rsi  (s <= r)
+#   h_{n+1} = Diag(e^{G_last}) h_n + (K o e^{G_last - G})^T V'
+#
+# and its reverse mode (dH the adjoint of h_{n+1}; every per-channel decay
+# passes its gradient to G channel by channel, dg being the reverse
+# in-chunk cumsum of dG per channel):
+#
+#   dV' = P^T dO + Kt dH,  dh_n = Diag(e^{G_last}) dH + Qg^T dO - W^T dV'
+#   dP = (dO V'^T) masked inclusive,  dW = -dV' h_n^T,  dU = dV'
+#   dKg = diag(beta) T^T dW,  dV = diag(beta) T^T dU
+#   dT = dW (diag(beta) Kg)^T + dU (diag(beta) V)^T,  dA = -strict(T^T dT T^T)
+#   dbeta = rowdot(T^T dW, Kg) + rowdot(T^T dU, V) + rowsum(dA * KKE)
+#   through KKE_rs = sum_i k_ri k_si E_rsi (weight beta_r dA_rs) and
+#   QKE_rs = sum_i q_ri k_si E_rsi (weight dP_rs): the products' gradients
+#   to the rows, + to G_ri and - to G_si of each term;
+#   Qg = Q o e^G, Kg = K o e^G, Kt = K o e^{G_last - G} and the state decay:
+#   elementwise, with Kt's and the decay's share of G_last on row C - 1.
+
+def _kda_chunk_head(q, k, v, g, beta, h, do, dh, C):
+    """One head, beta given, per-channel gate g [T, dk]: the outputs, the
+    final state and (with do, dh given) the gradients."""
+    T, dk = k.shape
+    dv = v.shape[1]
+    nchunks = (T + C - 1) // C
+    pad = nchunks * C - T
+    if pad:
+        z = lambda a, w: np.concatenate([a, np.zeros((pad, w))])
+        q, k, v, g = z(q, dk), z(k, dk), z(v, dv), z(g, dk)
+        do = z(do, dv) if do is not None else None
+        beta = np.concatenate([beta, np.zeros(pad)])
+    incl = np.tril(np.ones((C, C), dtype=bool))
+    strict = np.tril(np.ones((C, C), dtype=bool), -1)
+    o = np.zeros((nchunks * C, dv))
+    saved = []
+    h = h.copy()
+    for n in range(nchunks):
+        sl = slice(n * C, (n + 1) * C)
+        Q, K, V, bb = q[sl], k[sl], v[sl], beta[sl]
+        G = np.cumsum(g[sl], axis=0)
+        D = G[:, None, :] - G[None, :, :]                      # [r, s, i]
+        E = np.exp(np.where(incl[:, :, None], D, 0.0)) * incl[:, :, None]
+        KKE = np.einsum("ri,si,rsi->rs", K, K, E)
+        QKE = np.einsum("ri,si,rsi->rs", Q, K, E)
+        A = bb[:, None] * KKE * strict
+        Tm = np.linalg.inv(np.eye(C) + A)
+        eG, eL = np.exp(G), np.exp(G[-1])
+        Kg, Qg, Kt = K * eG, Q * eG, K * np.exp(G[-1][None, :] - G)
+        W = Tm @ (bb[:, None] * Kg)
+        Vp = Tm @ (bb[:, None] * V) - W @ h
+        o[sl] = Qg @ h + QKE @ Vp
+        saved.append((h.copy(), G, E, KKE, QKE, Tm, Kg, Qg, Kt, W, Vp))
+        h = eL[:, None] * h + Kt.T @ Vp
+    if do is None:
+        return o[:T], h
+    dq_, dk_, dv_ = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dg_, db_ = np.zeros_like(g), np.zeros(len(beta))
+    dH = dh.copy()
+    for n in range(nchunks - 1, -1, -1):
+        sl = slice(n * C, (n + 1) * C)
+        Q, K, V, bb, dO = q[sl], k[sl], v[sl], beta[sl], do[sl]
+        hn, G, E, KKE, QKE, Tm, Kg, Qg, Kt, W, Vp = saved[n]
+        eG, eL = np.exp(G), np.exp(G[-1])
+        P = QKE * incl
+        dVp = P.T @ dO + Kt @ dH
+        dP = (dO @ Vp.T) * incl
+        dW = -dVp @ hn.T
+        TdW, TdU = Tm.T @ dW, Tm.T @ dVp
+        dT = dW @ (bb[:, None] * Kg).T + dVp @ (bb[:, None] * V).T
+        dA = -(Tm.T @ dT @ Tm.T) * strict
+        dKKE = bb[:, None] * dA
+        dQ = np.einsum("rs,si,rsi->ri", dP, K, E) + (dO @ hn.T) * eG
+        dK = (np.einsum("rs,si,rsi->ri", dKKE, K, E) + np.einsum("rs,ri,rsi->si", dKKE, K, E)
+              + np.einsum("rs,ri,rsi->si", dP, Q, E))
+        dKg = bb[:, None] * TdW
+        dKt = Vp @ dH.T
+        dK += dKg * eG + dKt * np.exp(G[-1][None, :] - G)
+        # G: the per-channel decays inside KKE and QKE, then the elementwise ones
+        FK = np.einsum("rs,ri,si,rsi->rsi", dKKE, K, K, E)
+        FQ = np.einsum("rs,ri,si,rsi->rsi", dP, Q, K, E)
+        dG = FK.sum(1) - FK.sum(0) + FQ.sum(1) - FQ.sum(0)
+        dG += (dO @ hn.T) * Qg + dKg * Kg - dKt * Kt
+        dG[-1] += (dKt * Kt).sum(0) + eL * (dH * hn).sum(1)
+        dq_[sl], dk_[sl] = dQ, dK
+        dv_[sl] = bb[:, None] * TdU
+        db_[sl] = (TdW * Kg).sum(1) + (TdU * V).sum(1) + (dA * KKE).sum(1)
+        dg_[sl] = np.cumsum(dG[::-1], axis=0)[::-1]
+        dH = eL[:, None] * dH + Qg.T @ dO - W.T @ dVp
+    return dq_[:T], dk_[:T], dv_[:T], dg_[:T], db_[:T], dH
+
+
+def _kda_args(q, k, v, g, beta, h0):
+    q, k, v, g, beta = map(f64, (q, k, v, g, beta))
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    h0 = np.zeros((B, H, dk, dv)) if h0 is None else f64(h0)
+    return q, k, v, g, beta, h0, B, T, H, dk, dv
+
+
+def kda_forward(q, k, v, g, beta, h0=None, C: int = 64):
+    """Chunk-form per-channel-gate rule (beta given, g [B,T,H,dk]).
+    Returns (o, hT) in fp64."""
+    q, k, v, g, beta, h0, B, T, H, dk, dv = _kda_args(q, k, v, g, beta, h0)
+    o, hT = np.zeros((B, T, H, dv)), np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for hh in range(H):
+            o[b, :, hh], hT[b, hh] = _kda_chunk_head(
+                q[b, :, hh], k[b, :, hh], v[b, :, hh], g[b, :, hh], beta[b, :, hh], h0[b, hh],
+                None, None, C)
+    return o, hT
+
+
+def kda_backward_beta(q, k, v, g, beta, h0, do, dhT, C: int = 64):
+    """Chunk-form gradients of the per-channel-gate rule (beta given) for
+    dL/do = do and dL/dh_T = dhT.  Returns dq, dk, dv, dg [B,T,H,dk], dbeta,
+    dh0 (fp64)."""
+    q, k, v, g, beta, h0, B, T, H, dk, dv = _kda_args(q, k, v, g, beta, h0)
+    do = f64(do)
+    dhT = np.zeros((B, H, dk, dv)) if dhT is None else f64(dhT)
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v),
+               dg=np.zeros_like(g), dbeta=np.zeros((B, T, H)), dh0=np.zeros((B, H, dk, dv)))
+    for b in range(B):
+        for hh in range(H):
+            r = _kda_chunk_head(q[b, :, hh], k[b, :, hh], v[b, :, hh], g[b, :, hh],
+                                beta[b, :, hh], h0[b, hh], do[b, :, hh], dhT[b, hh], C)
+            for name, x in zip(("dq", "dk", "dv", "dg", "dbeta"), r[:5]):
+                out[name][b, :, hh] = x
+            out["dh0"][b, hh] = r[5]
     return out

@@ -181,3 +181,40 @@ def test_chunk_form_backward_gated_delta_and_strong_gates():
     for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
         assert np.all(np.isfinite(got[n])), n
         assert oracle.rel_l2(got[n], ref[n]) < 1e-11, n
+
+
+def _kda_chunk_problem(seed, T=150, dk=6, dv=5, strong=False):
+    r = np.random.Generator(np.random.PCG64(seed))
+    B, H = 1, 2
+    q = r.standard_normal((B, T, H, dk))
+    k = r.standard_normal((B, T, H, dk)) * 0.6
+    v = r.standard_normal((B, T, H, dv))
+    g = -np.log1p(np.exp(r.normal(1.0, 1.5, (B, T, H, dk))))
+    if strong:  # some channels wiped: e^G underflows inside a chunk
+        g = np.where(r.uniform(size=g.shape) < 0.3, -40.0, g)
+    beta = r.uniform(0.1, 1.2, (B, T, H))
+    h0 = r.standard_normal((B, H, dk, dv)) * 0.3
+    return q, k, v, g, beta, h0, r.standard_normal((B, T, H, dv)), r.standard_normal(h0.shape)
+
+
+@pytest.mark.parametrize("C", [1, 3, 8, 64])
+def test_kda_chunk_form_matches_token_loop(C):
+    """The per-channel-gate chunk form (the algebra of the per-channel prep
+    kernel) and its reverse mode, against the token-loop oracle."""
+    q, k, v, g, beta, h0, do, dhT = _kda_chunk_problem(51)
+    o_ref, h_ref = oracle.kda(q, k, v, g, beta, h0)
+    o, hT = chunk_form.kda_forward(q, k, v, g, beta, h0, C=C)
+    assert oracle.rel_l2(o, o_ref) < 1e-12 and oracle.rel_l2(hT, h_ref) < 1e-12
+    ref = oracle.kda_backward_beta(q, k, v, g, beta, h0, do, dhT)
+    got = chunk_form.kda_backward_beta(q, k, v, g, beta, h0, do, dhT, C=C)
+    for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
+        assert oracle.rel_l2(got[n], ref[n]) < 1e-12, (C, n)
+
+
+def test_kda_chunk_form_strong_channel_gates():
+    q, k, v, g, beta, h0, do, dhT = _kda_chunk_problem(52, T=130, strong=True)
+    ref = oracle.kda_backward_beta(q, k, v, g, beta, h0, do, dhT)
+    got = chunk_form.kda_backward_beta(q, k, v, g, beta, h0, do, dhT, C=64)
+    for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
+        assert np.all(np.isfinite(got[n])), n
+        assert oracle.rel_l2(got[n], ref[n]) < 1e-11, n
