@@ -33,3 +33,26 @@ def oracle_decode_state(dec_inputs):
     p = dec_inputs["prefix"]
     _, hT = oracle.forward(p["q"], p["k"], p["v"], p["g"], p["eta"], dec_inputs["eps"])
     return torch.from_numpy(hT.astype(np.float32))
+
+
+class Padded:
+    """A contiguous tensor view in the middle of a larger allocation whose
+    borders hold a byte pattern (the canaries of an out-of-bounds write):
+    ``t`` is the view, ``intact()`` says whether both borders are unchanged.
+    The view starts ``pad_bytes`` into the allocation (a multiple of 256, so
+    its alignment is that of a fresh allocation)."""
+
+    PATTERN = 0x5B
+
+    def __init__(self, shape, dtype, device, pad_bytes=4096):
+        es = torch.empty((), dtype=dtype).element_size()
+        n = int(np.prod(shape)) if len(shape) else 1
+        assert pad_bytes % 256 == 0 and pad_bytes % es == 0
+        self.lo, self.hi = pad_bytes, pad_bytes + n * es
+        self.raw = torch.full((self.hi + pad_bytes,), self.PATTERN, dtype=torch.uint8,
+                              device=device)
+        self.t = self.raw[self.lo:self.hi].view(dtype).view(shape)
+
+    def intact(self):
+        b = self.raw.cpu()
+        return bool((b[:self.lo] == self.PATTERN).all() and (b[self.hi:] == self.PATTERN).all())
