@@ -63,3 +63,13 @@ def test_workspace_queries_need_no_gpu():
     assert api.recurrent_bwd_workspace_size(**d) > 0
     assert api.kda_chunk_fwd_workspace_size(**d) > 0
     assert api.chunk_bwd_workspace_size(2, 300, 3, 128, 64) == 0  # d_k != d_v: unsupported
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without libkla.so there is no other path: the first call that needs
+    the library raises."""
+    from delta_rule_linear_kla_b200 import _native
+    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "libkla.so"))
+    monkeypatch.setattr(_native, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        api.chunk_fwd_workspace_size(1, 64, 1, 128, 128)
