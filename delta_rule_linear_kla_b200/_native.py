@@ -17,11 +17,14 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 SIGNATURES = {
     "kla_chunk_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "kla_chunk_fwd_segments": (_i, [_i, _i, _i, _i, _i, _i, _sz]),
+    "kla_chunk_fwd_single_launch": (_i, [_i, _i, _i, _i, _i, _i, _sz]),
     "kla_chunk_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,
                            _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_chunk_fwd_states": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp,
                                   _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_chunk_ut_transform": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kla_chunk_ut_bound_check": (_i, [_vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _vp, _sz, _vp,
+                                      _vp]),
     "kla_chunk_state_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "kla_recurrent_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp,

@@ -121,6 +121,12 @@ int kla_chunk_fwd_segments(int B, int T, int H, int dk, int dv, int dtype, size_
   return chunk_chain_segments(B, T, H, dk, dv, ws_bytes);
 }
 
+int kla_chunk_fwd_single_launch(int B, int T, int H, int dk, int dv, int dtype,
+                                size_t ws_bytes) {
+  if (!head_dims_ok(dk, dv) || chunk_ut_workspace_bytes(B, T, H, dk, dv, dtype) == 0) return 0;
+  return chunk_single_launch(B, T, H, dk, dv, ws_bytes) ? 1 : 0;
+}
+
 }  // extern "C"
 
 // Prefill with the KLA step size, or (eps == kBetaGiven) with beta given.
@@ -240,6 +246,36 @@ kla_status kla_chunk_ut_transform(const void* k, const float* g, const float* et
   if (!err) return KLA_ERR_CUDA;
   cudaError_t e = launch_chunk_ut(k, g, eta, eps, B, T, H, dk, workspace, err,
                                   (cudaStream_t)stream);
+  if (e == cudaErrorNotSupported) return KLA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
+}
+
+kla_status kla_chunk_ut_bound_check(const void* k, const float* g, const float* eta, float eps,
+                                    int B, int T, int H, int dk, int dtype, void* workspace,
+                                    size_t ws_bytes, float* ratio_max, void* stream) {
+  if (!ratio_max || !aligned16(ratio_max)) return KLA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || T < 1 || !k || !g || !eta) return KLA_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f)) return KLA_ERR_INVALID_ARG;
+  if ((long long)B * T * H * dk >= (1LL << 40)) return KLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {k, g, eta};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return KLA_ERR_INVALID_ARG;
+  if (!head_dims_ok(dk, dk)) return KLA_ERR_UNSUPPORTED;
+  kla_status s = check_stage(T, dtype, workspace, ws_bytes, B, H, dk, dk);
+  if (s != KLA_OK) return s;
+  const size_t ntok = (size_t)B * T * H;
+  Range rw = rng(workspace, chunk_ut_workspace_bytes(B, T, H, dk, dk, dtype));
+  const Range rr = rng(ratio_max, sizeof(float));
+  if (overlap(rw, rng(k, ntok * dk * 2)) || overlap(rw, rng(g, ntok * 4)) ||
+      overlap(rw, rng(eta, ntok * 4)) || overlap(rr, rw) || overlap(rr, rng(k, ntok * dk * 2)) ||
+      overlap(rr, rng(g, ntok * 4)) || overlap(rr, rng(eta, ntok * 4)))
+    return KLA_ERR_INVALID_ARG;
+  unsigned int* err = device_error_ptr();
+  if (!err) return KLA_ERR_CUDA;
+  if (cudaMemsetAsync(ratio_max, 0, sizeof(float), (cudaStream_t)stream) != cudaSuccess)
+    return KLA_ERR_CUDA;
+  cudaError_t e = launch_chunk_ut(k, g, eta, eps, B, T, H, dk, workspace, err,
+                                  (cudaStream_t)stream, ratio_max);
   if (e == cudaErrorNotSupported) return KLA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
@@ -543,8 +579,10 @@ static kla_status decode_impl(const void* q, const void* k, const void* v,
   if (overlap(ro, rs)) return KLA_ERR_INVALID_ARG;
   for (Range r : ins)
     if (overlap(ro, r) || overlap(rs, r)) return KLA_ERR_INVALID_ARG;
+  unsigned int* err = device_error_ptr();
+  if (!err) return KLA_ERR_CUDA;
   cudaError_t e = launch_decode(q, k, v, g, vector_gate, eta, eps, S, o, B, H, dk, dv, dtype,
-                                (cudaStream_t)stream);
+                                err, (cudaStream_t)stream);
   return e == cudaSuccess ? KLA_OK : KLA_ERR_CUDA;
 }
 
@@ -608,7 +646,8 @@ kla_status kla_check_device_error(void* stream) {
   if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return KLA_ERR_CUDA;
   if (v && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
     return KLA_ERR_CUDA;
-  return v ? KLA_ERR_TIMEOUT : KLA_OK;
+  if (v & KLA_DEVERR_TIMEOUT) return KLA_ERR_TIMEOUT;
+  return v ? KLA_ERR_BOUND : KLA_OK;
 }
 
 const char* kla_status_string(int status) {
@@ -618,6 +657,7 @@ const char* kla_status_string(int status) {
     case KLA_ERR_UNSUPPORTED: return "unsupported configuration";
     case KLA_ERR_CUDA: return "CUDA error";
     case KLA_ERR_TIMEOUT: return "device-side wait timed out";
+    case KLA_ERR_BOUND: return "a debug bound check found a value above its bound";
     default: return "unknown status";
   }
 }

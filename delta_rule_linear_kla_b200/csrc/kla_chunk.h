@@ -23,6 +23,9 @@ size_t chunk_ut_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
 size_t chunk_workspace_used(int B, int T, int H, int dk, int dv, int dtype, size_t ws_bytes);
 // Segments the state chain runs in for a workspace of ws_bytes (1 = uncut).
 int chunk_chain_segments(int B, int T, int H, int dk, int dv, size_t ws_bytes);
+// Whether the bf16 prefill of this shape runs as one launch (UT lanes and
+// state CTAs together) with a workspace of ws_bytes, on a B200's 148 SMs.
+bool chunk_single_launch(int B, int T, int H, int dk, int dv, size_t ws_bytes);
 
 // bf16 I/O chunkwise prefill (UT kernel, then the chain kernel).  Returns
 // cudaErrorNotSupported for shapes it does not handle; `err` is this
@@ -35,9 +38,11 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v,
 
 // The two stages of launch_chunk_tc on their own: the UT transform of every
 // chunk into the workspace, then the chain kernel that reads it.
+// ratio_max (device float, nullable): run the UT kernel's debug bound check
+// and record the largest bound ratio there.
 cudaError_t launch_chunk_ut(const void* k, const float* g, const float* eta, float eps,
                             int B, int T, int H, int dk, void* workspace, unsigned int* err,
-                            cudaStream_t st);
+                            cudaStream_t st, float* ratio_max = nullptr);
 // The chain is cut into segments (a sequence-parallel schedule for few heads
 // and long sequences) when ws_bytes also covers the segment states.
 cudaError_t launch_chunk_chain(const void* q, const void* k, const void* v, const float* g,
@@ -79,6 +84,6 @@ size_t kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype)
 // 64 x 64 boxes and 128-byte swizzle.
 cudaError_t launch_ut(const CUtensorMap& tm_k, const float* g, const float* eta, float eps,
                       uint8_t* ws, int B, int T, int H, int dk, unsigned int* err,
-                      cudaStream_t st);
+                      cudaStream_t st, float* ratio_max = nullptr);
 
 }  // namespace kla

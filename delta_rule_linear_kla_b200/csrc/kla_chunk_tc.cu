@@ -62,6 +62,7 @@
 #include "kla_chunk.h"
 #include "kla_common.cuh"
 #include "kla_sync.cuh"
+#include "kla_ut_body.cuh"
 #include "ptx_sm100.cuh"
 #include "tile_sw128.cuh"
 
@@ -140,14 +141,42 @@ constexpr uint64_t KSTEP_K = 2, KSTEP_MN = 128;
 // K o e^{G_last - G} as made per chunk by kda_prep_kernel (bulk copies; no
 // Q K^T or W products, no W or P epilogues), the state decays row by row with
 // e^{G_last}, and the outputs take no e^{G} factor (it is in Q o e^G).
+// Waits until the UT lane that makes chunk `idx`'s factors has raised its
+// flag (single-launch prefill), then orders this thread's later bulk copies
+// (async proxy) after that acquire.  Bounded like every other wait.
+__device__ __forceinline__ bool wait_flag(const unsigned int* flag, volatile int* abort_flag) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v != 0u) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      return true;
+    }
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
+// The state/output CTA for block coordinates (bx, by, bz) of the chain grid
+// (slab, head, batch x segment).  flags (nullable): the factors of chunk
+// (head, n) may be read only after flags[head * nchunks + n] is set (they
+// are made by UT lanes of the same launch).
 template <int DK, bool KDA>
-__global__ void __launch_bounds__(NTHREADS, 1)
-chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-             const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
-             const float* __restrict__ h0, __nv_bfloat16* __restrict__ o,
-             float* __restrict__ hT, float* __restrict__ phi, float* __restrict__ hs, int T,
-             int H, int DV, int nseg, int seg_chunks, int mode,
-             const uint8_t* __restrict__ ws, unsigned int* err) {
+__device__ __forceinline__ void chain_body(
+    const CUtensorMap* tm_q_p, const CUtensorMap* tm_k_p, const CUtensorMap* tm_v_p,
+    const float* __restrict__ g, const float* __restrict__ h0, __nv_bfloat16* __restrict__ o,
+    float* __restrict__ hT, float* __restrict__ phi, float* __restrict__ hs, int T, int H,
+    int DV, int nseg, int seg_chunks, int mode, const uint8_t* __restrict__ ws,
+    unsigned int* err, const int bx, const int by, const int bz,
+    const unsigned int* __restrict__ flags) {
+  const CUtensorMap& tm_q = *tm_q_p;
+  const CUtensorMap& tm_k = *tm_k_p;
+  const CUtensorMap& tm_v = *tm_v_p;
   using Smem = ChainSmem<DK>;
   constexpr int NP = Stage<DK>::NP;
   constexpr uint32_t PANEL = 3 * 8192;  // byte stride between key panels
@@ -156,7 +185,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                                      ~uintptr_t(1023));
   volatile int* abort_flag = &s.abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int hh = blockIdx.y, b = blockIdx.z / nseg, seg = blockIdx.z % nseg;
+  const int hh = by, b = bz / nseg, seg = bz % nseg;
   // Segment `seg` of the sequence: chunks n0 .. n0 + nchunks - 1 (the loop
   // index n below counts chunks within the segment; n0 + n addresses data).
   const int nchunks_all = (T + C - 1) / C;
@@ -172,8 +201,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   // nullable): the fp32 state at the start of every chunk,
   // [B][H][nchunks][DK][DV].  o may be NULL (no outputs written).
   const int nvs = DV / BV;
-  const bool phi_slab = mode == 1 && (int)blockIdx.x >= nvs;
-  const int slab = phi_slab ? (int)blockIdx.x - nvs : (int)blockIdx.x;
+  const bool phi_slab = mode == 1 && bx >= nvs;
+  const int slab = phi_slab ? bx - nvs : bx;
   // TMEM lane group this warp may access, and the row it stands for
   const int row = 32 * (warp & 3) + lane;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
@@ -236,6 +265,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
         Stage<DK>& S = s.st[st];
         const uint8_t* src = ws_head + (size_t)n * TILE;
+        // single-launch prefill: this chunk's factors exist once their flag
+        // is up (nothing of the stage is armed before that)
+        if (!KDA && flags && !wait_flag(flags + head * (size_t)nchunks_all + n0 + n, abort_flag))
+          break;
         ptx::mbar_arrive_expect_tx(&s.full[st], BYTES);
         if constexpr (KDA) {
           ptx::bulk_load(S.tp[TP1], src + KO.tp, 8192, &s.full[st]);
@@ -261,7 +294,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         issued = n + 1;
         if (n + 2 < nchunks) {  // warm L2 two chunks ahead of the loads
           const int m = n + 2;
-          ptx::bulk_prefetch_l2(ws_head + (size_t)m * TILE, TILE);
+          if (!flags) ptx::bulk_prefetch_l2(ws_head + (size_t)m * TILE, TILE);
           if constexpr (!KDA) {
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
@@ -677,6 +710,70 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   }
 }
 
+template <int DK, bool KDA>
+__global__ void __launch_bounds__(NTHREADS, 1)
+chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+             const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+             const float* __restrict__ h0, __nv_bfloat16* __restrict__ o,
+             float* __restrict__ hT, float* __restrict__ phi, float* __restrict__ hs, int T,
+             int H, int DV, int nseg, int seg_chunks, int mode,
+             const uint8_t* __restrict__ ws, unsigned int* err) {
+  chain_body<DK, KDA>(&tm_q, &tm_k, &tm_v, g, h0, o, hT, phi, hs, T, H, DV, nseg, seg_chunks,
+                      mode, ws, err, blockIdx.x, blockIdx.y, blockIdx.z, nullptr);
+}
+
+// UT lanes (128 threads each) per CTA of the single-launch prefill: as many
+// as the state CTA's shared memory holds.
+template <int DK>
+constexpr int fused_ut_lanes() {
+  return DK == 128 ? 3 : 4;
+}
+template <int DK>
+constexpr size_t fused_smem_bytes() {
+  return (sizeof(ChainSmem<DK>) > fused_ut_lanes<DK>() * sizeof(utb::UtSmem<DK>)
+              ? sizeof(ChainSmem<DK>)
+              : fused_ut_lanes<DK>() * sizeof(utb::UtSmem<DK>)) +
+         1024;
+}
+
+// The whole uncut prefill as one launch: CTAs 0 .. n_chain - 1 are the
+// state/output CTAs of the chain grid (slab fastest, then head, then batch);
+// every other CTA holds fused_ut_lanes UT lanes that make the per-chunk
+// factors in chunk order n = 0, 1, ... over all heads and raise one flag per
+// chunk, which the state CTAs wait for before they fetch that chunk's
+// factors.  The launch is cooperative (all CTAs resident at once, one per
+// SM), so those waits always end; they are bounded all the same.
+template <int DK>
+__global__ void __launch_bounds__(NTHREADS, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+               const float* __restrict__ eta, float eps, const float* __restrict__ h0,
+               __nv_bfloat16* __restrict__ o, float* __restrict__ hT, float* __restrict__ hs,
+               int T, int H, int DV, uint8_t* __restrict__ ws, unsigned int* flags, int n_chain,
+               unsigned int* err) {
+  const int nchunks = (T + C - 1) / C;
+  if ((int)blockIdx.x < n_chain) {
+    const int nvs = DV / BV;
+    const int bx = (int)blockIdx.x % nvs, by = ((int)blockIdx.x / nvs) % H,
+              bz = (int)blockIdx.x / (nvs * H);
+    chain_body<DK, false>(&tm_q, &tm_k, &tm_v, g, h0, o, hT, nullptr, hs, T, H, DV, 1, nchunks,
+                          0, ws, err, bx, by, bz, flags);
+    return;
+  }
+  constexpr int LANES = fused_ut_lanes<DK>();
+  const int lane_id = (int)threadIdx.x >> 7;
+  if (lane_id >= LANES) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  auto& us = *reinterpret_cast<utb::UtSmem<DK>*>(base + lane_id * sizeof(utb::UtSmem<DK>));
+  const int total = (n_chain / (DV / BV)) * nchunks;  // chain CTAs cover every head once
+  const int nlanes = ((int)gridDim.x - n_chain) * LANES;
+  utb::ut_run<DK, false>(&tm_k, g, eta, eps, ws, T, H, nchunks, total, err, nullptr, flags, us,
+                         (int)threadIdx.x & 127, 1 + lane_id,
+                         ((int)blockIdx.x - n_chain) * LANES + lane_id, nlanes, false);
+}
+
 // ------------------------------------------------------------------ host
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -816,11 +913,35 @@ size_t segment_bytes(int B, int T, int H, int dk, int dv) {
   return n * ((size_t)2 * dk * dv + (size_t)dk * dk) * sizeof(float);
 }
 
+// The single-launch prefill keeps at least this many CTAs of UT lanes beside
+// the state CTAs.
+constexpr int kMinUtCtas = 8;
+
+// Whether a shape runs as one launch: an uncut chain whose state CTAs leave
+// room for UT CTAs on the 148 SMs of a B200 (the launcher checks the actual
+// device again and otherwise runs the two kernels one after the other).
+bool fused_shape(int B, int T, int H, int dk, int dv) {
+  return chain_segments(B, T, H, dk, dv) == 1 &&
+         (long)B * H * (dv / BV) + kMinUtCtas <= kSmTarget;
+}
+
+// One ready flag per chunk after the factors (single launch only).
+size_t flag_bytes(int B, int T, int H) {
+  return ((size_t)B * H * ((T + C - 1) / C) * sizeof(unsigned int) + 255) & ~size_t(255);
+}
+
 }  // namespace
 
 size_t chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
   if (dtype != KLA_BF16 || B < 1 || H < 1 || T < 1 || dk != dv) return 0;
-  return ut_workspace_bytes(B, T, H) + segment_bytes(B, T, H, dk, dv);
+  return ut_workspace_bytes(B, T, H) + segment_bytes(B, T, H, dk, dv) +
+         (fused_shape(B, T, H, dk, dv) ? flag_bytes(B, T, H) : 0);
+}
+
+bool chunk_single_launch(int B, int T, int H, int dk, int dv, size_t ws_bytes) {
+  if (B < 1 || H < 1 || T < 1 || dk != dv || (dk != 64 && dk != 128)) return false;
+  return fused_shape(B, T, H, dk, dv) &&
+         ws_bytes >= ut_workspace_bytes(B, T, H) + flag_bytes(B, T, H);
 }
 
 size_t chunk_ut_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
@@ -842,11 +963,11 @@ size_t chunk_workspace_used(int B, int T, int H, int dk, int dv, int dtype, size
 
 cudaError_t launch_chunk_ut(const void* k, const float* g, const float* eta, float eps,
                             int B, int T, int H, int dk, void* workspace, unsigned int* err,
-                            cudaStream_t st) {
+                            cudaStream_t st, float* ratio_max) {
   if (dk != 64 && dk != 128) return cudaErrorNotSupported;
   CUtensorMap mk;
   if (!make_map(&mk, k, dk, H, T, B)) return cudaErrorInvalidValue;
-  return launch_ut(mk, g, eta, eps, (uint8_t*)workspace, B, T, H, dk, err, st);
+  return launch_ut(mk, g, eta, eps, (uint8_t*)workspace, B, T, H, dk, err, st, ratio_max);
 }
 
 // The chain in S segments: pass 1 (E, Phi of segments 0 .. S-2), the start
@@ -908,11 +1029,68 @@ static cudaError_t launch_segmented(const void* q, const void* k, const void* v,
                                   ws, err, st, hs);
 }
 
+// The single-launch prefill (see prefill_kernel).  cudaErrorNotSupported when
+// this device cannot hold it (too few SMs beside the state CTAs, no
+// cooperative launch): the caller then runs the two kernels in turn.
+template <int DK>
+static cudaError_t launch_fused(const void* q, const void* k, const void* v, const float* g,
+                                const float* eta, float eps, const float* h0, void* o,
+                                float* hT, int B, int T, int H, uint8_t* ws, unsigned int* err,
+                                cudaStream_t st, float* hs) {
+  constexpr int DV = DK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  static int sms[64] = {};
+  static int fits[64] = {};  // 0 unknown, 1 yes, -1 no
+  constexpr size_t smem = fused_smem_bytes<DK>();
+  if (!fits[dev]) {
+    int coop = 0, nb = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(prefill_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, prefill_kernel<DK>, NTHREADS, smem);
+    if (e != cudaSuccess) return e;
+    fits[dev] = (coop && nb >= 1) ? 1 : -1;
+  }
+  const int n_chain = B * H * (DV / BV);
+  if (fits[dev] < 0 || n_chain + kMinUtCtas > sms[dev]) return cudaErrorNotSupported;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, DK, H, T, B) || !make_map(&mk, k, DK, H, T, B) ||
+      !make_map(&mv, v, DV, H, T, B))
+    return cudaErrorInvalidValue;
+  unsigned int* flags = reinterpret_cast<unsigned int*>(ws + ut_workspace_bytes(B, T, H));
+  cudaError_t e = cudaMemsetAsync(flags, 0, flag_bytes(B, T, H), st);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sms[dev]);
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<DK>, mq, mk, mv, g, eta, eps, h0,
+                            (__nv_bfloat16*)o, hT, hs, T, H, DV, ws, flags, n_chain, err);
+}
+
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                             const float* eta, float eps, const float* h0, void* o, float* hT,
                             int B, int T, int H, int dk, int dv, void* workspace,
                             size_t ws_bytes, unsigned int* err, cudaStream_t st, float* hs) {
   if (dk != dv || (dk != 64 && dk != 128)) return cudaErrorNotSupported;
+  if (fused_shape(B, T, H, dk, dv) &&
+      ws_bytes >= ut_workspace_bytes(B, T, H) + flag_bytes(B, T, H)) {
+    uint8_t* wsm = (uint8_t*)workspace;
+    const cudaError_t e =
+        dk == 128 ? launch_fused<128>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, wsm, err, st, hs)
+                  : launch_fused<64>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, wsm, err, st, hs);
+    if (e != cudaErrorNotSupported) return e;
+  }
   cudaError_t e = launch_chunk_ut(k, g, eta, eps, B, T, H, dk, workspace, err, st);
   if (e != cudaSuccess) return e;
   return launch_chunk_chain(q, k, v, g, h0, o, hT, B, T, H, dk, dv, workspace, ws_bytes, err,

@@ -12,7 +12,9 @@ namespace kla {
 
 // Device error word: one per device, owned by kla_api.cu, passed to kernels
 // as a pointer.  Bounded waits that give up set a bit instead of hanging.
-enum : unsigned int { KLA_DEVERR_TIMEOUT = 1u };
+// KLA_DEVERR_BOUND: a debug bound check of the UT factors found an entry
+// above its bound (kla_chunk_ut_bound_check).
+enum : unsigned int { KLA_DEVERR_TIMEOUT = 1u, KLA_DEVERR_BOUND = 2u };
 
 __device__ __forceinline__ void report_timeout(unsigned int* err) {
   atomicOr(err, KLA_DEVERR_TIMEOUT);
@@ -33,7 +35,7 @@ __device__ __forceinline__ float step_size(float eta, float knorm2, float eps) {
 cudaError_t launch_decode(const void* q, const void* k, const void* v,
                           const float* g, bool vector_gate, const float* eta, float eps,
                           float* S, void* o, int B, int H, int dk, int dv, int dtype,
-                          cudaStream_t st);
+                          unsigned int* err, cudaStream_t st);
 cudaError_t launch_recurrent(const void* q, const void* k, const void* v,
                              const float* g, bool vector_gate, const float* eta, float eps,
                              const float* h0, void* o, float* hT, int B, int T,

@@ -1,0 +1,504 @@
+// UT transform of every chunk (the device code, shared by the stand-alone UT
+// kernel and the single-launch prefill), in parallel over all chunks.
+//
+// For one chunk of C = 64 tokens ("Deep Dive into KDA", section 3; the
+// intermediates U and W named there are T diag(beta) V and T diag(beta e^G) K
+// in the reading this library takes, with the key-norm step size of
+// "Kaczmarz Linear Attention", Abstract):
+//
+//   beta_r = eta_r / (||k_r||^2 + eps),   G_r = sum_{j <= r} g_j (in chunk)
+//   A_rs   = beta_r (k_r . k_s) e^{G_r - G_s}   for s < r, else 0
+//   T      = (I + A)^{-1}                       (unit lower triangular)
+//   out:   T' = T diag(beta),  T'' = T diag(beta e^G), stored transposed
+//          (row c of each tile is column c of the factor), bf16
+//
+// The inverse is taken by blocks of 16.  With A_bj the 16 x 16 blocks of A
+// and D_b = (I + A_bb)^{-1}, block forward substitution gives T_bb = D_b and
+// T_bc = -D_b sum_{c <= j < b} A_bj T_jc (b > c).  It is evaluated on the
+// transposes, Y = T^T:
+//
+//   Y_cc = D_c^T,   Y_cb = -(sum_{c <= j < b} Y_cj A_bj^T) D_b^T   (b > c),
+//
+// so every block just formed is the left operand of the next product.
+//
+// A CTA of 128 threads takes two chunks (a "pair"):
+//   1. the Gram matrices of both chunks as one tcgen05 MMA, [K0; K1][K0; K1]^T
+//      (M = N = 128, bf16, fp32 in TMEM; the two 64 x 64 diagonal blocks are
+//      the chunks' Gram matrices); their diagonals give ||k||^2 and beta;
+//   2. thread t holds row t: it forms row r of A with the decay e^{G_r - G_s}
+//      as a running product of alpha_j = e^{g_j} over s < j <= r (every
+//      factor <= 1) and stores the blocks left of its diagonal block (bf16)
+//      and its part of the diagonal block (fp32);
+//   3. thread (chunk, b, c) solves column c of D_b by forward substitution
+//      (fp32) and writes the diagonal block of the outputs;
+//   4. warp (chunk, half) forms the off-diagonal row blocks Y_cb with
+//      warp-level bf16 products (mma.sync m16n8k16, fp32 sums): the fp32
+//      accumulators of one product are, packed to bf16, the left operand of
+//      the next one, so a row block never leaves its warp's registers.
+// Rounding the products' operands to bf16 moves the outputs no more than the
+// bf16 rounding of T' and T'' themselves (a CPU simulation of this exact
+// scheme on the stress and 0.4B-layer distributions gives the same error as
+// rounding the exact factors).  The next pair's keys are loaded as soon as
+// the Gram MMA has read them, so the load overlaps steps 2 to 4.
+//
+// The factors are written to global memory already in the 128-byte swizzled
+// bf16 layout the chain kernel's MMAs read (as MN-major A operands), so it
+// fetches them with one bulk copy per chunk.
+//
+// Debug bound check (CHECK): for eta in [0, 2] every factor
+// (I - beta_j k_j k_j^T) of the chunk's transition has norm <= 1, and then
+// |T_rs| ||k_r|| / ||k_s|| <= eta'_r e^{G_r - G_s} for r > s, with
+// eta'_r = beta_r ||k_r||^2.  The checked variant measures the largest ratio
+// of the two sides over every entry it forms (entries below 1e-30 skipped),
+// records it (atomicMax on the float's bits) and sets the device error word
+// when it exceeds kBoundSlack.
+#pragma once
+
+#include "kla_chunk.h"
+#include "kla_common.cuh"
+#include "kla_sync.cuh"
+#include "ptx_sm100.cuh"
+#include "tile_sw128.cuh"
+
+namespace kla {
+namespace utb {
+
+constexpr int C = 64;
+constexpr int NT = 128;
+constexpr uint32_t TILE = 128 * 64 * 2;  // one key panel of a pair: 128 rows x 64 bf16
+constexpr int AROW = 72;                 // bf16 per row of the A tile (64 + 8: 144 B rows)
+constexpr int DROW = 24;                 // bf16 per row of a D_b^T block (16 + 8: 48 B rows)
+constexpr float kBoundSlack = 1.25f;     // allowance for the factors' own rounding
+
+template <int DK>
+constexpr int ctas_per_sm() {
+  return DK == 128 ? 3 : 4;
+}
+
+template <int DK>
+struct alignas(1024) UtSmem {
+  static constexpr int NP = DK / 64;
+  uint8_t keys[NP * TILE];           // [K0; K1] per 64-column panel (TMA, 128-byte swizzle)
+  __nv_bfloat16 a[2][C][AROW];       // A left of the diagonal blocks, bf16, row-major
+  __nv_bfloat16 dt[2][4][16][DROW];  // D_b^T (row c = column c of D_b), bf16
+  float ad[2][4][16][17];            // diagonal blocks of A, fp32 ([row][column], padded)
+  float G[2][C], alpha[2][C], eta[2][C], n2[2][C];
+  float b1[2][C], b2[2][C];          // beta, beta e^G
+  uint64_t bar_tma, bar_mma;
+  uint32_t tmem_base;
+};
+
+// ---------------------------------------------------------------- warp MMA
+__device__ __forceinline__ void ldsm_x4(uint32_t* r, const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(ptx::smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t* r, const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(ptx::smem_u32(p)));
+}
+// d (16 x 8, fp32) += a (16 x 16, bf16, row-major fragment) . b (16 x 8)
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of element (row m, column n) in a 64 x 64 bf16 tile of 128-B
+// swizzled rows.
+__device__ __forceinline__ uint32_t tile_off(int m, int n) {
+  return (uint32_t)(m * 128 + ((((n >> 3) ^ (m & 7)) & 7) << 4) + (n & 7) * 2);
+}
+
+__device__ __forceinline__ void atomic_max_nonneg(float* p, float x) {
+  atomicMax(reinterpret_cast<unsigned int*>(p), __float_as_uint(x));
+}
+
+// Ratio of the P-UT bound for entry T_rs (r > s) of one chunk.
+template <int DK>
+__device__ __forceinline__ float bound_ratio(const UtSmem<DK>& s, int j, int r, int sc,
+                                             float t_rs) {
+  const float a = fabsf(t_rs);
+  if (!(a > 1e-30f)) return 0.f;
+  const float etap = s.b1[j][r] * s.n2[j][r];
+  const float den = etap * __expf(s.G[j][r] - s.G[j][sc]) * sqrtf(s.n2[j][sc]);
+  const float num = a * sqrtf(s.n2[j][r]);
+  if (!(den > 1e-30f)) return num > 1e-30f ? 3.0e38f : 0.f;
+  return num / den;
+}
+
+
+// Named barrier of one 128-thread lane, and its AND-reduction form.
+__device__ __forceinline__ void nbar_sync(int id) {
+  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ bool nbar_and(int id, bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return out != 0;
+}
+
+// One UT "lane": 128 threads (tid 0..127, TMEM lanes 0..127 of their own
+// 128-column allocation) that own the shared memory `s` and synchronise on
+// named barrier `bar_id` only.  It takes pairs first_pair, first_pair +
+// pair_stride, ... of the chunk order: chunk-major within each head when
+// `flags` is null (the stand-alone kernel), else chunk index n major over all
+// heads (n = 0 of every head first), publishing flags[head * nchunks + n] =
+// 1 once a chunk's factors are in memory (for state CTAs of the same launch
+// that wait on them).  `standalone`: the lane is the whole CTA (it may
+// relinquish the TMEM allocation permit).
+template <int DK, bool CHECK>
+__device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __restrict__ g,
+                                       const float* __restrict__ eta, float eps,
+                                       uint8_t* __restrict__ ws, int T, int H, int nchunks,
+                                       int total_chunks, unsigned int* err, float* ratio_max,
+                                       unsigned int* flags, UtSmem<DK>& s, const int tid,
+                                       const int bar_id, const int first_pair,
+                                       const int pair_stride, const bool standalone) {
+  constexpr int NP = UtSmem<DK>::NP;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int j = tid >> 6, r = tid & 63;  // chunk slot and its row
+  const int npairs = (total_chunks + 1) / 2;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const int BH = total_chunks / nchunks;
+  const bool nmajor = flags != nullptr;
+  // processing index -> (head, chunk)
+  auto chunk_of = [&](int p, int& hd, int& nn) {
+    if (nmajor) {
+      nn = p / BH;
+      hd = p - nn * BH;
+    } else {
+      hd = p / nchunks;
+      nn = p - hd * nchunks;
+    }
+  };
+
+  // keys of pair `pr` (two chunks stacked) -> s.keys, on bar_tma
+  auto load_keys = [&](int pr) {
+    const int c0 = 2 * pr, nv = min(2, total_chunks - c0);
+    ptx::mbar_arrive_expect_tx(&s.bar_tma, (uint32_t)(nv * NP * 8192));
+    for (int jj = 0; jj < nv; ++jj) {
+      int hd, nn;
+      chunk_of(c0 + jj, hd, nn);
+#pragma unroll
+      for (int p = 0; p < NP; ++p)
+        ptx::tma_load_4d(s.keys + p * TILE + jj * 8192, tm_k, &s.bar_tma, p * 64, hd % H,
+                         nn * C, hd / H);
+    }
+  };
+  // gate and relaxation of my token in pair `pr` (zero beyond the sequence:
+  // an identity step)
+  auto load_gates = [&](int pr, float& gv, float& ev) {
+    gv = 0.f;
+    ev = 0.f;
+    const int cj = 2 * pr + j;
+    if (pr < npairs && cj < total_chunks) {
+      int hd, nn;
+      chunk_of(cj, hd, nn);
+      const int tt = nn * C + r;
+      if (tt < T) {
+        const size_t tok = ((size_t)(hd / H) * T + tt) * H + hd % H;
+        gv = g[tok];
+        ev = eta[tok];
+      }
+    }
+  };
+
+  if (warp == 0) {
+    ptx::tmem_alloc(&s.tmem_base, 128);
+    if (standalone) ptx::tmem_relinquish();
+  }
+  if (tid == 0) {
+    ptx::prefetch_tensormap(tm_k);
+    ptx::mbar_init(&s.bar_tma, 1);
+    ptx::mbar_init(&s.bar_mma, 1);
+    ptx::mbar_init_fence();
+    if (first_pair < npairs) load_keys(first_pair);
+  }
+  float gr, er;
+  load_gates(first_pair, gr, er);
+  ptx::tc_fence_before();
+  nbar_sync(bar_id);
+  ptx::tc_fence_after();
+  const uint32_t tacc = s.tmem_base;  // the two Gram matrices (128 x 128 fp32)
+  bool ok = true;
+  uint32_t mma_phase = 0, tma_phase = 0;
+  bool keys_in_flight = tid == 0 && first_pair < npairs;
+  float worst = 0.f;  // CHECK: largest bound ratio this thread saw
+
+  // persistent: pairs first_pair, first_pair + pair_stride, ...  Every
+  // thread of the lane takes the same number of trips (the exit test is
+  // uniform over the lane).
+#pragma unroll 1
+  for (int pair = first_pair; pair < npairs; pair += pair_stride) {
+    if (!nbar_and(bar_id, ok)) break;  // also: the previous pair's readers are done
+    const bool valid = 2 * pair + j < total_chunks;
+    int hd_j = 0, nn_j = 0;
+    if (valid) chunk_of(2 * pair + j, hd_j, nn_j);
+    const int ci = hd_j * nchunks + nn_j;  // workspace index (head-major)
+    // chunk-local inclusive cumsum of g (warps 2j, 2j+1 hold chunk j)
+    float gs = gr;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, gs, off);
+      if (lane >= off) gs += y;
+    }
+    s.G[j][r] = gs;
+    s.alpha[j][r] = __expf(gr);
+    s.eta[j][r] = er;
+    nbar_sync(bar_id);
+    const float G31 = s.G[j][31];  // row 31 is not rewritten below
+    if (r >= 32) s.G[j][r] = gs + G31;
+    float gn, en;  // next pair's gate and relaxation
+    load_gates(pair + pair_stride, gn, en);
+
+    // ---- Gram matrices of both chunks: [K0; K1] [K0; K1]^T
+    if (tid == 0) {
+      ok = wait_bounded(&s.bar_tma, tma_phase);
+      tma_phase ^= 1u;
+      keys_in_flight = !ok;
+      if (ok) {
+        ptx::tc_fence_after();
+        constexpr uint32_t id = ptx::idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint32_t a = ptx::smem_u32(s.keys + (kk >> 2) * TILE) + (kk & 3) * 32;
+          ptx::mma_bf16(tacc, ptx::sdesc_sw128(a, 16, 1024), ptx::sdesc_sw128(a, 16, 1024),
+                        id, kk > 0);
+        }
+        ptx::mma_commit(&s.bar_mma);
+        ok = wait_bounded(&s.bar_mma, mma_phase);
+        // the MMA has read the keys: the next pair's may land now
+        if (ok && pair + pair_stride < npairs) {
+          load_keys(pair + pair_stride);
+          keys_in_flight = true;
+        }
+      }
+    }
+    mma_phase ^= 1u;
+    __syncwarp();
+    if (!nbar_and(bar_id, ok)) break;
+    ptx::tc_fence_after();
+
+    // ---- row r of the chunk's Gram matrix (its diagonal block), beta_r and
+    // row r of A
+    const int bb = r >> 4;  // my 16-row block
+    {
+      float v[64];
+      ptx::tmem_ld32(tacc + lane_base + 64 * j, v);
+      ptx::tmem_ld32(tacc + lane_base + 64 * j + 32, v + 32);
+      float nn2 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) nn2 = (c == r) ? v[c] : nn2;
+      const float beta = step_size(er, nn2, eps);
+      // A_rs = beta_r (k_r . k_s) e^{G_r - G_s}: per 16-column block, the
+      // decay at its last column s0 < r from one exponential (<= 1), then
+      // running products of alpha_i (each <= 1) down the block; the four
+      // blocks are independent chains
+      const float Gr = s.G[j][r];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int s0 = min(16 * q + 15, r - 1);
+        float d = s0 >= 16 * q ? __expf(Gr - s.G[j][s0]) : 0.f;
+#pragma unroll
+        for (int c = 16 * q + 15; c >= 16 * q; --c) {
+          const bool on = c < r;
+          d = (on && c < s0) ? d * s.alpha[j][c + 1] : d;
+          v[c] = on ? beta * v[c] * d : 0.f;
+        }
+      }
+      // diagonal block part (fp32) and the blocks left of it (bf16)
+      float* adr = &s.ad[j][bb][r & 15][0];
+#define KLA_UT_DIAG(B_)                                      \
+  if (bb == B_) {                                            \
+    _Pragma("unroll") for (int i = 0; i < 16; ++i) adr[i] = v[16 * B_ + i]; \
+  }
+      KLA_UT_DIAG(0) else KLA_UT_DIAG(1) else KLA_UT_DIAG(2) else KLA_UT_DIAG(3)
+#undef KLA_UT_DIAG
+      __nv_bfloat16* arow = &s.a[j][r][0];
+#pragma unroll
+      for (int q = 0; q < 6; ++q) {
+        if (q < 2 * bb) {
+          uint4 u;
+          u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+          u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+          u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+          u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+          *reinterpret_cast<uint4*>(arow + 8 * q) = u;
+        }
+      }
+      s.b1[j][r] = beta;
+      s.b2[j][r] = beta * __expf(s.G[j][r]);
+      s.n2[j][r] = nn2;
+    }
+    ptx::tc_fence_before();
+    nbar_sync(bar_id);
+
+    uint8_t* dst = ws + (size_t)ci * kUtTileBytes;  // T'^T, then T''^T
+    // ---- D_b = (I + A_bb)^{-1}: thread (j, b, c) solves column c; it is row
+    // m = 16 b + c of Y's diagonal block, written straight to the outputs
+    {
+      const int b = (tid >> 4) & 3, c = tid & 15, m = 16 * b + c;
+      // right-looking: once x_m is final, it is subtracted from every later
+      // row at once (16 dependent steps of independent updates)
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
+#pragma unroll
+      for (int mm = 0; mm < 15; ++mm) {
+#pragma unroll
+        for (int i = mm + 1; i < 16; ++i) x[i] = fmaf(-s.ad[j][b][i][mm], x[mm], x[i]);
+      }
+      uint4 lo, hi;
+      lo.x = pack_bf16x2(x[0], x[1]);   lo.y = pack_bf16x2(x[2], x[3]);
+      lo.z = pack_bf16x2(x[4], x[5]);   lo.w = pack_bf16x2(x[6], x[7]);
+      hi.x = pack_bf16x2(x[8], x[9]);   hi.y = pack_bf16x2(x[10], x[11]);
+      hi.z = pack_bf16x2(x[12], x[13]); hi.w = pack_bf16x2(x[14], x[15]);
+      *reinterpret_cast<uint4*>(&s.dt[j][b][c][0]) = lo;
+      *reinterpret_cast<uint4*>(&s.dt[j][b][c][8]) = hi;
+      if (valid) {
+        const float f1 = s.b1[j][m], f2 = s.b2[j][m];
+        const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int q = 0; q < 6; ++q) {
+          if (q < 2 * b) {
+            *reinterpret_cast<uint4*>(dst + m * 128 + (((q ^ (m & 7)) & 7) << 4)) = z;
+            *reinterpret_cast<uint4*>(dst + 8192 + m * 128 + (((q ^ (m & 7)) & 7) << 4)) = z;
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint4 u1, u2;
+          const float* xh = x + 8 * h;
+          u1.x = pack_bf16x2(f1 * xh[0], f1 * xh[1]); u1.y = pack_bf16x2(f1 * xh[2], f1 * xh[3]);
+          u1.z = pack_bf16x2(f1 * xh[4], f1 * xh[5]); u1.w = pack_bf16x2(f1 * xh[6], f1 * xh[7]);
+          u2.x = pack_bf16x2(f2 * xh[0], f2 * xh[1]); u2.y = pack_bf16x2(f2 * xh[2], f2 * xh[3]);
+          u2.z = pack_bf16x2(f2 * xh[4], f2 * xh[5]); u2.w = pack_bf16x2(f2 * xh[6], f2 * xh[7]);
+          const int q = 2 * b + h;
+          *reinterpret_cast<uint4*>(dst + m * 128 + (((q ^ (m & 7)) & 7) << 4)) = u1;
+          *reinterpret_cast<uint4*>(dst + 8192 + m * 128 + (((q ^ (m & 7)) & 7) << 4)) = u2;
+        }
+        if constexpr (CHECK) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (i > c) worst = fmaxf(worst, bound_ratio(s, j, 16 * b + i, m, x[i]));
+        }
+      }
+    }
+    nbar_sync(bar_id);
+
+    // ---- off-diagonal row blocks of Y = T^T: warp 2j takes row block 0,
+    // warp 2j + 1 row blocks 1 and 2 (row block 3 is D_3^T alone)
+    {
+      const int half = warp & 1;
+      const int g8 = lane >> 3, l8 = lane & 7;  // ldmatrix: matrix and row
+      const int fr = lane >> 2, fc = 2 * (lane & 3);  // fragment row / column pair
+      // c is a compile-time index in every unrolled copy (the register
+      // fragments y[] are indexed by it); the warp-uniform test picks the
+      // row blocks this warp owns
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        if (half ? c == 0 : c != 0) continue;
+        uint32_t y[4][4];  // A fragments of Y_cb, b = c .. 3 (bf16)
+        ldsm_x4(y[c], &s.dt[j][c][(g8 & 1) * 8 + l8][(g8 >> 1) * 8]);
+#pragma unroll
+        for (int b = 1; b < 4; ++b) {
+          if (b <= c) continue;
+          float acc[2][4] = {};
+#pragma unroll
+          for (int jj = 0; jj < 3; ++jj) {
+            if (jj < c || jj >= b) continue;
+            // A_{b,jj}^T as the B operand: rows 16 b + 8 h + (0..7) of A,
+            // columns 16 jj + (0..15)
+            uint32_t bf[4];
+            ldsm_x4(bf, &s.a[j][16 * b + (g8 >> 1) * 8 + l8][16 * jj + (g8 & 1) * 8]);
+            mma16816(acc[0], y[jj], bf[0], bf[1]);
+            mma16816(acc[1], y[jj], bf[2], bf[3]);
+          }
+          uint32_t sa[4] = {pack_bf16x2(acc[0][0], acc[0][1]), pack_bf16x2(acc[0][2], acc[0][3]),
+                            pack_bf16x2(acc[1][0], acc[1][1]), pack_bf16x2(acc[1][2], acc[1][3])};
+          // times D_b^T (stored row-major as D_b^T: transposed loads give the
+          // B fragments)
+          uint32_t db[4];
+          ldsm_x4_t(db, &s.dt[j][b][(g8 & 1) * 8 + l8][(g8 >> 1) * 8]);
+          float yb[2][4] = {};
+          mma16816(yb[0], sa, db[0], db[1]);
+          mma16816(yb[1], sa, db[2], db[3]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) yb[h][e] = -yb[h][e];
+          y[b][0] = pack_bf16x2(yb[0][0], yb[0][1]);
+          y[b][1] = pack_bf16x2(yb[0][2], yb[0][3]);
+          y[b][2] = pack_bf16x2(yb[1][0], yb[1][1]);
+          y[b][3] = pack_bf16x2(yb[1][2], yb[1][3]);
+          if (valid) {
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              const int m = 16 * c + fr + 8 * rr;
+              const float f1 = s.b1[j][m], f2 = s.b2[j][m];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int n = 16 * b + 8 * h + fc;
+                const float e0 = yb[h][2 * rr], e1 = yb[h][2 * rr + 1];
+                const uint32_t off = tile_off(m, n);
+                *reinterpret_cast<uint32_t*>(dst + off) = pack_bf16x2(f1 * e0, f1 * e1);
+                *reinterpret_cast<uint32_t*>(dst + 8192 + off) = pack_bf16x2(f2 * e0, f2 * e1);
+                if constexpr (CHECK) {
+                  worst = fmaxf(worst, bound_ratio(s, j, n, m, e0));
+                  worst = fmaxf(worst, bound_ratio(s, j, n + 1, m, e1));
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+    if (nmajor) {
+      // every thread's factor stores are visible (to the bulk copies of the
+      // state CTAs too) before the pair's flags are raised
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      nbar_sync(bar_id);
+      if (tid == 0) {
+        __threadfence();
+        for (int jj = 0; jj < 2; ++jj) {
+          int hd, nn;
+          if (2 * pair + jj < total_chunks) {
+            chunk_of(2 * pair + jj, hd, nn);
+            atomicExch(flags + (size_t)hd * nchunks + nn, 1u);
+          }
+        }
+      }
+    }
+    gr = gn;
+    er = en;
+  }  // pair loop
+  if (!ok) report_timeout(err);
+  if constexpr (CHECK) {
+    if (worst > 0.f) atomic_max_nonneg(ratio_max, worst);
+    if (worst > kBoundSlack) atomicOr(err, KLA_DEVERR_BOUND);
+  }
+  // a wait gave up: let this CTA's own key copy land before it exits
+  if (keys_in_flight) wait_bounded(&s.bar_tma, tma_phase);
+  ptx::tc_fence_before();
+  nbar_sync(bar_id);
+  if (warp == 0) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tacc, 128);
+  }
+}
+
+
+}  // namespace utb
+}  // namespace kla

@@ -50,7 +50,8 @@ typedef enum {
     KLA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, aliasing */
     KLA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not 64/128) */
     KLA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or launch failed   */
-    KLA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up            */
+    KLA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up            */
+    KLA_ERR_BOUND = 5         /* a debug bound check found a violation         */
 } kla_status;
 
 typedef enum { KLA_BF16 = 0, KLA_FP32 = 1 } kla_dtype;
@@ -76,11 +77,14 @@ typedef enum { KLA_BF16 = 0, KLA_FP32 = 1 } kla_dtype;
  *   workspace / ws_bytes: caller-owned device scratch of
  *     kla_chunk_fwd_workspace_size(...) bytes (NULL allowed when that is 0):
  *     the per-chunk factors (B * H * ceil(T / KLA_CHUNK) * 16384 bytes, the
- *     least accepted, else KLA_ERR_INVALID_ARG) followed, for few heads and
- *     long sequences, by the states of the sequence segments the state chain
- *     is cut into (run in parallel).  A workspace smaller than the full size
- *     but holding the factors runs the chain uncut.  It must not overlap any
- *     other argument.
+ *     least accepted, else KLA_ERR_INVALID_ARG) followed either, for few
+ *     heads and long sequences, by the states of the sequence segments the
+ *     state chain is cut into (run in parallel), or, where the whole prefill
+ *     runs as one launch (kla_chunk_fwd_single_launch), by one 4-byte ready
+ *     flag per chunk (rounded up to 256 bytes; cleared by the call itself).
+ *     A workspace smaller than the full size but holding the factors runs
+ *     the chain uncut, with the factors formed by a launch of their own.
+ *     It must not overlap any other argument.
  *
  * Supported: B, H >= 1; T >= 0 (T = 0 copies h0 to hT); dk = dv in {64, 128}.
  * A ragged tail (T not a multiple of the chunk) is processed as if padded
@@ -101,6 +105,20 @@ KLA_API size_t kla_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
  */
 KLA_API int kla_chunk_fwd_segments(int B, int T, int H, int dk, int dv, int dtype,
                                    size_t ws_bytes);
+
+/*
+ * 1 when the bf16 kla_chunk_fwd of this shape runs as a single kernel launch
+ * with a workspace of ws_bytes: the chain is uncut, the state CTAs (one per
+ * head and 64 state columns) leave at least 8 of a B200's 148 SMs for CTAs
+ * that form the per-chunk factors in the same launch (cooperative, every
+ * CTA resident; the state CTAs wait, bounded, on a per-chunk ready flag),
+ * and the workspace holds the flags after the factors (as sized by
+ * kla_chunk_fwd_workspace_size).  0 otherwise, when the factors are formed
+ * by a launch of their own first (also on a device where the single launch
+ * does not fit, which the call detects itself).  Host-only query.
+ */
+KLA_API int kla_chunk_fwd_single_launch(int B, int T, int H, int dk, int dv, int dtype,
+                                        size_t ws_bytes);
 
 KLA_API kla_status kla_chunk_fwd(const void *q, const void *k, const void *v,
                          const float *g, const float *eta, float eps,
@@ -156,6 +174,28 @@ KLA_API kla_status kla_chunk_state_fwd(const void *q, const void *k, const void 
                                const float *g, const float *h0, void *o, float *hT,
                                int B, int T, int H, int dk, int dv, int dtype,
                                void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * kla_chunk_ut_transform with a debug check of its factors (same arguments
+ * and workspace, plus `ratio_max`: one device float, 16-byte aligned,
+ * disjoint from the rest).  The bound follows from the recurrence: with
+ * k_s = ||k_s|| khat_s, T_rs (r > s) is -eta'_r (||k_s|| / ||k_r||)
+ * e^{G_r - G_s} khat_r^T P khat_s, P a product of erase factors
+ * (I - beta_j k_j k_j^T) that each have norm <= 1 when eta_j is in [0, 2]
+ * (the Kaczmarz step of the KLA Abstract, over-relaxed up to 2), and
+ * eta'_r = beta_r ||k_r||^2, so |T_rs| ||k_r|| / ||k_s|| <= eta'_r
+ * e^{G_r - G_s}.  The call writes the largest ratio of the left side to the
+ * right side over every entry the kernel forms (entries below 1e-30 are
+ * skipped) into *ratio_max, and when it exceeds 1.25 (the allowance for the
+ * factors' own bf16 rounding) it sets the device error word, so the next
+ * kla_check_device_error returns KLA_ERR_BOUND.  Nothing traps.  eta
+ * outside [0, 2] voids the bound (a ratio above 1 is then not an error of
+ * the kernel).
+ */
+KLA_API kla_status kla_chunk_ut_bound_check(const void *k, const float *g, const float *eta,
+                                            float eps, int B, int T, int H, int dk, int dtype,
+                                            void *workspace, size_t ws_bytes, float *ratio_max,
+                                            void *stream);
 
 /*
  * Token-serial prefill on CUDA cores: the recurrence evaluated one token at
@@ -414,9 +454,11 @@ KLA_API kla_status kla_chunk_fwd_host(const void *q, const void *k, const void *
  * KLA_BF16 or KLA_FP32) with a fixed scratch array compiled into libkla.so
  * instead of a workspace.  It allocates nothing itself.
  *
- *   Limit: B * H * ceil(T / KLA_CHUNK) <= KLA_NOALLOC_MAX_CHUNKS, else
- *          KLA_ERR_UNSUPPORTED (checked before any CUDA call).  The state
- *          chain is cut into segments only where their states also fit.
+ *   Limit (KLA_BF16 only; the KLA_FP32 path uses no scratch):
+ *          B * H * ceil(T / KLA_CHUNK) <= KLA_NOALLOC_MAX_CHUNKS, else
+ *          KLA_ERR_UNSUPPORTED (checked before any CUDA call, in 64-bit
+ *          arithmetic).  The state chain is cut into segments only where
+ *          their states also fit.
  *   Memory: every GPU that loads libkla.so holds KLA_NOALLOC_SCRATCH_BYTES
  *          for the life of the process.
  *   First call on a device looks up the array's device address
@@ -438,8 +480,10 @@ KLA_API kla_status kla_chunk_fwd_noalloc(const void *q, const void *k, const voi
 /*
  * Reads and clears the library's device error word for the current device
  * after synchronising `stream`.  Kernels set it instead of hanging when a
- * bounded wait on an mbarrier runs out (KLA_ERR_TIMEOUT).  Returns KLA_OK
- * when no kernel reported a problem.
+ * bounded wait on an mbarrier runs out (KLA_ERR_TIMEOUT), and the debug
+ * bound check sets it on a violation (KLA_ERR_BOUND; a timeout takes
+ * precedence when both happened).  Returns KLA_OK when no kernel reported a
+ * problem.
  */
 KLA_API kla_status kla_check_device_error(void *stream);
 
