@@ -9,10 +9,11 @@
 // this entry point uses a fixed scratch array that lives in this library's
 // device image instead.  Its cost: every GPU that loads the library holds
 // KLA_NOALLOC_SCRATCH_BYTES (16 MiB) for the rest of the process, and one
-// call handles at most KLA_NOALLOC_MAX_CHUNKS chunks of 64 tokens in total
-// (B * H * ceil(T / 64)).  The library's uses of a workspace are covered:
-// the per-chunk factors always fit, the segment states of a cut state chain
-// only when the chunk count leaves room.
+// bf16 call handles at most KLA_NOALLOC_MAX_CHUNKS chunks of 64 tokens in
+// total (B * H * ceil(T / 64)); fp32 calls use no scratch and have no limit.
+// The library's uses of a workspace are covered: the per-chunk factors
+// always fit, the segment states of a cut state chain only when the chunk
+// count leaves room.
 //
 // Nothing here allocates: no cudaMalloc, cudaFree, or allocating library call.
 // All calls share the single array and it keeps whatever the last call left
@@ -60,11 +61,15 @@ extern "C" KLA_API kla_status kla_chunk_fwd_noalloc(const void* q, const void* k
                                                     void* stream) {
   // Size limit first, before anything touches the GPU.
   if (B < 1 || H < 1 || T < 0) return KLA_ERR_INVALID_ARG;
-  const long long chunks = (long long)B * H * ((T + KLA_CHUNK - 1) / KLA_CHUNK);
+  // Only the bf16 chunk path uses scratch; the fp32 (token-serial) path needs
+  // none, so the chunk limit does not apply to it.  64-bit arithmetic: the
+  // count cannot wrap for any int-sized B, H, T.
+  const long long chunks =
+      (long long)B * H * (((long long)T + KLA_CHUNK - 1) / KLA_CHUNK);
   // (KLA_NOALLOC_MAX_CHUNKS tiles of UT factors fill the scratch exactly;
   // kla_chunk_fwd cuts the state chain into segments only if their states
   // fit in what is left)
-  if (chunks > KLA_NOALLOC_MAX_CHUNKS) return KLA_ERR_UNSUPPORTED;
+  if (dtype == KLA_BF16 && chunks > KLA_NOALLOC_MAX_CHUNKS) return KLA_ERR_UNSUPPORTED;
   void* scratch = scratch_address();
   if (!scratch) return KLA_ERR_CUDA;
   return kla_chunk_fwd(q, k, v, g, eta, eps, h0, o, hT, B, T, H, dk, dv, KLA_CHUNK, dtype,
