@@ -10,9 +10,12 @@ B=8 T=4096 H=8 d=128, bf16) through kla_chunk_fwd.  Each rank processes its
 own batch (independent sequences, no collective on the data path): weak
 scaling.  L2 is flushed (512 MiB written then read) before every timed step
 and each step is bracketed by CUDA events on the launching stream; the job
-time is the max over ranks.  The decode workload (B=64 H=16 d=128, 32K-token
-state, 1000 in-place steps, L2 flushed before each) is measured on every rank
-after the prefill and reported under "decode".
+time is the max over ranks.  The other halves of the prefill metric (65K
+context, the stress shape) are timed the same way and reported under
+"other_workloads".  The decode workload (B=64 H=16 d=128, 32K-token state)
+is timed as 1000 consecutive in-place steps with one event pair, on one
+state and on a rotating set of three states larger than L2, and reported
+under "decode".
 """
 from __future__ import annotations
 
@@ -62,12 +65,15 @@ def prefill_work(w):
 
 
 def stage_work(w):
-    """Algorithmic flops and bytes of each of the two kernels of one prefill.
+    """Algorithmic flops and bytes of each of the two kernels of one prefill
+    (minimum bytes: the inputs a kernel must read and the
+    outputs it must write; the per-chunk factors T', T'' that the first
+    kernel hands the second are an intermediate of this split, not
+    algorithmic bytes, and are reported separately).
 
-    UT transform: reads k, g, eta; writes the per-chunk factors T', T''
-    (2 x 64 x 64 bf16 per chunk); flops of K K^T.  State/output kernel:
-    reads q, k, v, g, h0 and the factors; writes o and h_T; flops of the
-    other seven products."""
+    UT transform: reads k, g, eta; flops of K K^T.  State/output kernel:
+    reads q, k, v, g (and h0); writes o and h_T; flops of the other seven
+    products."""
     C = 64
     d = w.dk
     es = 2
@@ -75,10 +81,12 @@ def stage_work(w):
     nchunk = w.B * w.H * ((w.T + C - 1) // C)
     fac = nchunk * 2 * C * C * 2
     state = w.B * w.H * w.dk * w.dv * 4
-    ut = {"flops": ntok * 2 * C * d, "bytes": ntok * w.dk * es + ntok * 8 + fac}
+    ut = {"flops": ntok * 2 * C * d, "bytes": ntok * w.dk * es + ntok * 8,
+          "intermediate_bytes": fac}
     chain = {"flops": ntok * (8 * C * d + 6 * d * d),
-             "bytes": ntok * (2 * w.dk + 2 * w.dv) * es + ntok * 4 + fac
-             + state * (2 if w.kind == "stress" else 1)}
+             "bytes": ntok * (2 * w.dk + 2 * w.dv) * es + ntok * 4
+             + state * (2 if w.kind == "stress" else 1),
+             "intermediate_bytes": fac}
     return ut, chain
 
 
@@ -202,20 +210,25 @@ def run_ours(args, rank, world, dev):
         nws = api.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype)
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
         fn = functools.partial(api.chunk_fwd, workspace=ws)
-        # UT kernel, then one chain launch, or three for a cut chain
-        # (segment transitions, start states, outputs)
         nseg = api.chunk_fwd_segments(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, nws)
-        launches_per_step = 1 + (3 if nseg > 1 else 1)
+        # one launch (UT lanes and state CTAs together), or the UT kernel
+        # then one chain launch, or three for a cut chain (segment
+        # transitions, start states, outputs)
+        single = api.chunk_fwd_single_launch(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, nws)
+        launches_per_step = 1 if single else 1 + (3 if nseg > 1 else 1)
     else:
         fn = api.recurrent_fwd
-        nseg, launches_per_step = 0, 1
+        nseg, launches_per_step, single = 0, 1, False
     stream = torch.cuda.current_stream()
     flush = L2Flush(dev)
 
     def step(mid=None):
-        # the chunk path as its two kernels (exactly what chunk_fwd launches),
-        # with an event between them when the split is being timed
-        if chunk:
+        # the single launch through chunk_fwd; otherwise the chunk path as
+        # its two kernels (exactly what chunk_fwd launches), with an event
+        # between them when the split is being timed
+        if single:
+            fn(xd["q"], xd["k"], xd["v"], xd["g"], xd["eta"], x["eps"], xd["h0"], o=o, hT=hT)
+        elif chunk:
             api.chunk_ut_transform(xd["k"], xd["g"], xd["eta"], x["eps"], workspace=ws)
             if mid is not None:
                 mid.record(stream)
@@ -253,20 +266,26 @@ def run_ours(args, rank, world, dev):
     api.check_device_error()
     ms = sum(a.elapsed_time(b) for a, _, b in evs) / args.steps
     ms_max = allreduce_max(ms, world, dev)
-    # per-kernel launch durations over the same timed steps
-    ms_ut = sum(a.elapsed_time(m) for a, m, _ in evs) / args.steps if chunk else 0.0
-    ms_chain = sum(m.elapsed_time(b) for _, m, b in evs) / args.steps if chunk else ms
+    # per-kernel launch durations over the same timed steps (two-kernel path)
+    two = chunk and not single
+    ms_ut = sum(a.elapsed_time(m) for a, m, _ in evs) / args.steps if two else 0.0
+    ms_chain = sum(m.elapsed_time(b) for _, m, b in evs) / args.steps if two else ms
 
     value = aggregate_throughput(w.B * w.T, world, ms_max)
     flops, byts = prefill_work(w)
     achieved_tf = flops / (ms / 1e3) / 1e12
     hbm_peak = float(peaks["hbm_gbs"])
     tc_peak = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
-    if chunk:
+    if two:
         ut_w, chain_w = stage_work(w)
     else:
-        ut_w, chain_w = None, {"flops": flops, "bytes": byts}
+        # one kernel does the whole step: its algorithmic bytes and flops are
+        # the step's (the per-chunk factors stay in L2 between its CTAs)
+        ut_w, chain_w = None, {"flops": flops, "bytes": byts, "intermediate_bytes": None}
     chain_gbs = chain_w["bytes"] / (ms_chain / 1e3) / 1e9
+    kernel_name = ("prefill_kernel" if single else "chain_kernel") if chunk else "recurrent_kernel"
+    traffic = (profiled_traffic("kla_chunk_tc.cu", "%s_prefill_4k.md" % kernel_name)
+               if chunk and w.name == "prefill_4k" else None)
 
     # end to end through the public API with host buffers (pinned)
     e2e = None if args.no_e2e else measure_e2e(args, w, x, fn, dev, stream, world)
@@ -291,30 +310,45 @@ def run_ours(args, rank, world, dev):
                    "l2": "flushed before every timed step (512 MiB write+read); inputs > L2"},
         # dominant kernel: the state/output (chain) kernel; its bytes at
         # the measured copy bandwidth take longer than its flops at the
-        # measured bf16 rate, so it is HBM-bound at the roofline
-        "roofline": {"kernel": "chain_kernel" if chunk else "recurrent_kernel",
-                     "bound": "hbm", "achieved": chain_gbs, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": chain_gbs / hbm_peak,
-                     "traffic": profiled_traffic("kla_chunk_tc.cu",
-                                                 "chain_kernel_prefill_4k.md")
-                     if chunk and w.name == "prefill_4k" else None,
-                     "algorithmic_bytes": chain_w["bytes"], "us_per_launch": ms_chain * 1e3,
-                     "tensor_tflops": chain_w["flops"] / (ms_chain / 1e3) / 1e12,
-                     "peak_source": peak_src + " (burst copy)"},
+        # measured bf16 rate, so it is HBM-bound at the roofline.  Its
+        # algorithmic bytes are the inputs it must read and the outputs it
+        # must write (q, k, v, g, h0, o, h_T); the per-chunk factors it also
+        # reads are an intermediate of the two-kernel split and show up in
+        # "traffic" (ncu DRAM bytes per launch) and "traffic_over_algorithmic"
+        "roofline": dict({"kernel": kernel_name,
+                          "bound": "hbm", "achieved": chain_gbs, "peak": hbm_peak,
+                          "unit": "GB/s", "frac": chain_gbs / hbm_peak,
+                          "traffic": traffic,
+                          "traffic_over_algorithmic": (None if traffic is None
+                                                       else traffic / chain_w["bytes"]),
+                          "algorithmic_bytes": chain_w["bytes"],
+                          "intermediate_bytes_read": chain_w.get("intermediate_bytes"),
+                          "us_per_launch": ms_chain * 1e3,
+                          "tensor_tflops": chain_w["flops"] / (ms_chain / 1e3) / 1e12,
+                          "peak_source": peak_src + " (burst copy)"}),
         # whole step against the dense bf16 tensor peak (tensor-pipe %)
         "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
                    "frac": achieved_tf / tc_peak, "algorithmic_flops": flops,
                    "algorithmic_bytes": byts,
                    "hbm_frac": byts / (ms / 1e3) / 1e9 / hbm_peak,
                    "peak_source": peak_src + " (burst cuBLAS bf16)"},
-        # our kernels per step: UT transform + chain (chunk path; three
-        # launches for a cut chain), one token-serial kernel otherwise; the
-        # L2 flush is torch's, not counted
+        # our kernels per step: one single-launch prefill, or UT transform +
+        # chain (three chain launches for a cut chain), one token-serial
+        # kernel otherwise; the L2 flush and the flag clear are not counted
         "gpu_launches": args.steps * launches_per_step,
         "wall_s": wall,
         "e2e": e2e,
     }
-    if chunk:
+    if single:
+        res["kernels"] = {
+            "prefill_kernel": {"us_per_launch": ms * 1e3, "algorithmic_bytes": byts,
+                               "gbs": byts / (ms / 1e3) / 1e9,
+                               "tflops": flops / (ms / 1e3) / 1e12,
+                               "launch": "cooperative, one CTA per SM: %d state CTAs and UT "
+                                         "lanes on the other SMs" % (w.B * w.H * w.dv // 64),
+                               "note": "event time of the step (the kernel and the clear of "
+                                       "its chunk flags)"}}
+    elif chunk:
         res["kernels"] = {
             "ut_kernel": {"us_per_launch": ms_ut * 1e3, "algorithmic_bytes": ut_w["bytes"],
                           "gbs": ut_w["bytes"] / (ms_ut / 1e3) / 1e9,
@@ -326,8 +360,14 @@ def run_ours(args, rank, world, dev):
             # the cut chain: its time spans its three launches
             res["kernels"]["chain_kernel"]["launches"] = (
                 "%d segments: transitions, start states, outputs" % nseg)
+    if chunk and not args.no_other and args.workload == "prefill_4k":
+        # the other halves of the prefill metric: 65K context and the
+        # stress shape, each its own workload through the same entry point
+        res["other_workloads"] = {
+            name: time_prefill(inputs.WORKLOADS[name], dev, stream, flush, peaks, rank)
+            for name in ("prefill_65k", "stress")}
     if not args.no_decode:
-        res["decode"] = run_decode(args, rank, dev, stream, flush, peaks, peak_src, fn, clk)
+        res["decode"] = run_decode(args, rank, dev, stream, peaks, peak_src, fn, clk)
     if not args.no_kda and w.dtype == "bf16":
         res["kda_prefill"] = run_kda_prefill(w, dev, stream, flush, peaks, peak_src)
     if not args.no_bwd:
@@ -338,6 +378,58 @@ def run_ours(args, rank, world, dev):
     res["clocks"]["window"] = "samples from 1 s of back-to-back warm-up steps and the timed steps"
     res["warmup_steps_run"] = i
     return res
+
+
+def time_prefill(w, dev, stream, flush, peaks, rank, steps=5, warmup=3):
+    """One more prefill workload through kla_chunk_fwd (workspace allocated
+    once, L2 flushed before every step, CUDA events per step): tokens/s and
+    its fractions of the measured tensor and HBM peaks on the algorithmic
+    flops and bytes."""
+    from delta_rule_linear_kla_b200 import api
+
+    w = rank_workload(w, rank)
+    x = inputs_to(dev, w)
+    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=w.torch_dtype, device=dev)
+    hT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    nws = api.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+    nseg = api.chunk_fwd_segments(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, nws)
+    run = lambda: api.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"],
+                                o=o, hT=hT, workspace=ws)
+    for _ in range(warmup):
+        flush()
+        run()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    torch.cuda.synchronize()
+    for e0, e1 in evs:
+        flush()
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    api.check_device_error()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    flops, byts = prefill_work(w)
+    tf = flops / (ms / 1e3) / 1e12
+    return {"metric": metric_name(w.name), "value": w.B * w.T / (ms / 1e3),
+            "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk,
+                       "dv": w.dv, "chain_segments": nseg},
+            "tensor": {"achieved": tf, "unit": "TFLOP/s",
+                       "frac": tf / float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])),
+                       "algorithmic_flops": flops},
+            "hbm": {"achieved": byts / (ms / 1e3) / 1e9, "unit": "GB/s",
+                    "frac": byts / (ms / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
+                    "algorithmic_bytes": byts},
+            "l2": "flushed before every timed step"}
+
+
+def inputs_to(dev, w):
+    from delta_rule_linear_kla_b200 import inputs
+
+    x = inputs.make_prefill(w)
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
 
 
 def measure_e2e(args, w, x, fn, dev, stream, world):
@@ -391,8 +483,30 @@ def measure_e2e(args, w, x, fn, dev, stream, world):
             "path": how}
 
 
-def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn, clk):
-    """Decode: state = our prefill over the trailing prefix; then in-place steps."""
+def _timed_steps(stream, nsteps, body):
+    """Times ``nsteps`` back-to-back calls ``body(i)`` with one CUDA event
+    pair on ``stream`` (no flush or sync between steps); ms per step."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(nsteps):
+        body(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / nsteps
+
+
+def run_decode(args, rank, dev, stream, peaks, peak_src, prefill_fn, clk):
+    """Decode: state = our prefill over the trailing prefix; then in-place
+    steps, 1000 consecutive ones timed with one event pair.
+
+    Two timings.  "value": every step updates the same 64 MiB state in
+    place, exactly the workload as stated; the state fits in the 126 MB L2,
+    so part of its traffic never reaches DRAM.  "roofline": the same steps
+    on a rotating set of three states (three batches of 64 sequences,
+    192 MiB > L2), step i on state i % 3, so every step's read and its
+    write-back of the previous steps' dirty lines go through HBM inside
+    the timed window; the HBM fraction is taken from this one."""
     from delta_rule_linear_kla_b200 import api, inputs
 
     w = inputs.DECODE.scaled(seed=inputs.DECODE.seed + 100 * rank)
@@ -402,62 +516,62 @@ def run_decode(args, rank, dev, stream, flush, peaks, peak_src, prefill_fn, clk)
     _, S = prefill_fn(p["q"], p["k"], p["v"], p["g"], p["eta"], d["eps"], None)
     st = {k: v.to(dev) for k, v in d["steps"].items()}
     o = torch.empty((w.B, w.H, w.dv), dtype=w.torch_dtype, device=dev)
-    for i in range(3):
-        api.decode_step(st["q"][i], st["k"][i], st["v"][i], st["g"][i], st["eta"][i], S,
+    states = [S] + [S.clone() for _ in range(2)]
+
+    def step(i, S_i):
+        api.decode_step(st["q"][i], st["k"][i], st["v"][i], st["g"][i], st["eta"][i], S_i,
                         d["eps"], o=o)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(nsteps)]
-    torch.cuda.synchronize()
+
+    for i in range(6):
+        step(i, states[i % 3])
     t0 = time.perf_counter()
-    for i, (e0, e1) in enumerate(evs):
-        flush()
-        e0.record(stream)
-        api.decode_step(st["q"][i], st["k"][i], st["v"][i], st["g"][i], st["eta"][i], S,
-                        d["eps"], o=o)
-        e1.record(stream)
-    torch.cuda.synchronize()
+    ms_one = _timed_steps(stream, nsteps, lambda i: step(i, states[0]))
+    ms_rot = _timed_steps(stream, nsteps, lambda i: step(i, states[i % 3]))
     t1 = time.perf_counter()
     api.check_device_error()
-    ms = sum(a.elapsed_time(b) for a, b in evs) / nsteps
     state_bytes = 2 * w.B * w.H * w.dk * w.dv * 4
     io_bytes = w.B * w.H * (2 * w.dk + 2 * w.dv) * 2 + w.B * w.H * 8
-    gbs = (state_bytes + io_bytes) / (ms / 1e3) / 1e9
+    gbs = (state_bytes + io_bytes) / (ms_rot / 1e3) / 1e9
+    gbs_one = (state_bytes + io_bytes) / (ms_one / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
 
     # the same steps with a per-channel gate (KDA form): 16 gate sets of
     # [B, H, dk] drawn once and cycled (the gate values do not change the
     # work); one more [B, H, dk] fp32 read per step than the scalar gate
     gv = inputs.channel_gates((16, w.B, w.H, w.dk), w.seed + 7).to(dev)
-    kevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(nsteps)]
-    for i in range(3):
-        api.kda_decode_step(st["q"][i], st["k"][i], st["v"][i], gv[i % 16], st["eta"][i], S,
+
+    def kstep(i, S_i):
+        api.kda_decode_step(st["q"][i], st["k"][i], st["v"][i], gv[i % 16], st["eta"][i], S_i,
                             d["eps"], o=o)
-    torch.cuda.synchronize()
-    for i, (e0, e1) in enumerate(kevs):
-        flush()
-        e0.record(stream)
-        api.kda_decode_step(st["q"][i], st["k"][i], st["v"][i], gv[i % 16], st["eta"][i], S,
-                            d["eps"], o=o)
-        e1.record(stream)
-    torch.cuda.synchronize()
+
+    for i in range(6):
+        kstep(i, states[i % 3])
+    kms = _timed_steps(stream, nsteps, lambda i: kstep(i, states[i % 3]))
     api.check_device_error()
-    kms = sum(a.elapsed_time(b) for a, b in kevs) / nsteps
     kbytes = state_bytes + io_bytes + w.B * w.H * (w.dk - 1) * 4
     kgbs = kbytes / (kms / 1e3) / 1e9
     return {"metric": "decode tokens/s (B=64 H=16 d=128, 32K-token state)",
-            "value": w.B / (ms / 1e3), "unit": "tokens/s", "us_per_step": ms * 1e3,
-            "steps": nsteps, "l2": "flushed before every step",
-            "clocks": clk.summary(t0, t1 + 0.15), "gpu_launches": nsteps,
+            "value": w.B / (ms_one / 1e3), "unit": "tokens/s", "us_per_step": ms_one * 1e3,
+            "steps": nsteps,
+            "timing": "%d consecutive in-place steps on one state, one event pair, no flush "
+                      "(the 64 MiB state stays partly in L2)" % nsteps,
+            "rotating_states": {
+                "value": w.B / (ms_rot / 1e3), "unit": "tokens/s", "us_per_step": ms_rot * 1e3,
+                "timing": "%d consecutive steps over 3 states of 64 MiB (192 MiB > L2), step "
+                          "i on state i %% 3, one event pair" % nsteps},
+            "clocks": clk.summary(t0, t1 + 0.15), "gpu_launches": 2 * nsteps,
             "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": gbs,
                          "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "timing": "rotating states (every step's bytes cross HBM)",
                          "traffic": profiled_traffic("kla_decode.cu",
                                                      "decode_kernel_decode_b64.md"),
                          "algorithmic_bytes": state_bytes + io_bytes,
+                         "one_state_gbs": gbs_one,
                          "peak_source": peak_src},
             "per_channel_gate": {
                 "value": w.B / (kms / 1e3), "unit": "tokens/s", "us_per_step": kms * 1e3,
                 "steps": nsteps, "gpu_launches": nsteps,
+                "timing": "rotating states, as the roofline above",
                 "roofline": {"kernel": "decode_kernel (per-channel gate)", "bound": "hbm",
                              "achieved": kgbs, "peak": peak, "unit": "GB/s",
                              "frac": kgbs / peak, "traffic": None,
@@ -690,6 +804,11 @@ def main():
                     help="skip the per-channel-gate (KDA form) prefill measurement")
     ap.add_argument("--no-bwd", action="store_true",
                     help="skip the backward (gradients) measurement")
+    ap.add_argument("--no-other", action="store_true",
+                    help="skip the 65K and stress prefill workloads")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode measurement (e.g. under a profiler) and print "
+                         "its JSON object")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
@@ -711,6 +830,16 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", device_id=dev,
                                              timeout=datetime.timedelta(seconds=120))
+    if args.decode_only:
+        from delta_rule_linear_kla_b200 import api
+        peaks, peak_src = load_peaks()
+        clk = ClockSampler(dev.index).__enter__()
+        res = run_decode(args, rank, dev, torch.cuda.current_stream(), peaks, peak_src,
+                         api.chunk_fwd, clk)
+        clk.__exit__()
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return 0
     try:
         res = run_ours(args, rank, world, dev)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

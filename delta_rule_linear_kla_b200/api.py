@@ -6,6 +6,7 @@ are allocated here with torch (the library itself never allocates).
 """
 from __future__ import annotations
 
+import contextlib
 from typing import Optional, Tuple
 
 import torch
@@ -35,11 +36,13 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
 
-def _need(t, name, dtype=None, shape=None):
+def _need(t, name, dtype=None, shape=None, dev=None):
     if t is None:
         return
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError("%s must be a CUDA tensor" % name)
+    if dev is not None and t.device != dev:
+        raise ValueError("%s is on %s, the call's other tensors on %s" % (name, t.device, dev))
     if not t.is_contiguous():
         raise ValueError("%s must be contiguous" % name)
     if dtype is not None and t.dtype != dtype:
@@ -48,9 +51,23 @@ def _need(t, name, dtype=None, shape=None):
         raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
 
 
-def _stream(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
-    return s.cuda_stream
+@contextlib.contextmanager
+def _on(ref, stream):
+    """Device and stream of one call: ``ref``'s device is made current (the
+    library sizes its TMA maps and error word for the current device) and
+    ``stream`` (default: that device's current stream) becomes torch's
+    current stream, so every temporary allocated inside (outputs,
+    workspaces) belongs to the stream the kernels run on.  The caching
+    allocator then only reuses a freed temporary for work ordered after
+    those kernels.  Yields the raw stream handle for the C call."""
+    _need(ref, "q")
+    dev = ref.device
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        if s.device != dev:
+            raise ValueError("stream is on %s, the tensors on %s" % (s.device, dev))
+        with torch.cuda.stream(s):
+            yield s.cuda_stream
 
 
 def chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
@@ -67,23 +84,36 @@ def chunk_fwd_segments(B: int, T: int, H: int, dk: int, dv: int,
     return int(_native.lib().kla_chunk_fwd_segments(B, T, H, dk, dv, _DT[dtype], ws_bytes))
 
 
+def chunk_fwd_single_launch(B: int, T: int, H: int, dk: int, dv: int,
+                            dtype: torch.dtype = torch.bfloat16,
+                            ws_bytes: Optional[int] = None) -> bool:
+    """Whether the bf16 prefill of this shape runs as one kernel launch
+    (kla_chunk_fwd_single_launch); ws_bytes defaults to the full workspace
+    size."""
+    if ws_bytes is None:
+        ws_bytes = chunk_fwd_workspace_size(B, T, H, dk, dv, dtype)
+    return bool(_native.lib().kla_chunk_fwd_single_launch(B, T, H, dk, dv, _DT[dtype],
+                                                          ws_bytes))
+
+
 def _prefill_args(q, k, v, g, eta, h0, o, hT, return_state):
     _need(q, "q")
     if q.dtype not in _DT:
         raise ValueError("q, k, v must be bfloat16 or float32")
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    _need(k, "k", q.dtype, (B, T, H, dk))
-    _need(v, "v", q.dtype, (B, T, H, dv))
-    _need(g, "g", torch.float32, (B, T, H))
-    _need(eta, "eta", torch.float32, (B, T, H))
-    _need(h0, "h0", torch.float32, (B, H, dk, dv))
+    d = q.device
+    _need(k, "k", q.dtype, (B, T, H, dk), d)
+    _need(v, "v", q.dtype, (B, T, H, dv), d)
+    _need(g, "g", torch.float32, (B, T, H), d)
+    _need(eta, "eta", torch.float32, (B, T, H), d)
+    _need(h0, "h0", torch.float32, (B, H, dk, dv), d)
     if o is None:
-        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
-    _need(o, "o", q.dtype, (B, T, H, dv))
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=d)
+    _need(o, "o", q.dtype, (B, T, H, dv), d)
     if hT is None and return_state:
-        hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
-    _need(hT, "hT", torch.float32, (B, H, dk, dv))
+        hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=d)
+    _need(hT, "hT", torch.float32, (B, H, dk, dv), d)
     return B, T, H, dk, dv, o, hT
 
 
@@ -91,15 +121,17 @@ def chunk_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
               return_state: bool = True, workspace=None,
               stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunkwise KLA prefill (kla_chunk_fwd).  Returns (o, hT)."""
-    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, eta, h0, o, hT, return_state)
-    need = chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = _native.lib().kla_chunk_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0),
-        _ptr(o), _ptr(hT), B, T, H, dk, dv, CHUNK, _DT[q.dtype], _ptr(workspace),
-        ws_bytes, _stream(stream))
+    with _on(q, stream) as s:
+        B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, eta, h0, o, hT, return_state)
+        need = chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _need(workspace, "workspace", torch.uint8, dev=q.device)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = _native.lib().kla_chunk_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0),
+            _ptr(o), _ptr(hT), B, T, H, dk, dv, CHUNK, _DT[q.dtype], _ptr(workspace),
+            ws_bytes, s)
     _check(st, "kla_chunk_fwd")
     return o, hT
 
@@ -109,18 +141,20 @@ def chunk_fwd_states(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, outputs: bo
     """bf16 chunk prefill that also returns the state at the start of every
     chunk (kla_chunk_fwd_states).  Returns (o, hT, hs) with hs
     [B, H, ceil(T / 64), dk, dv] fp32; o and hT are None if not outputs."""
-    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, eta, h0, None, None, outputs)
-    if not outputs:
-        o = None
-    hs = torch.empty((B, H, (T + CHUNK - 1) // CHUNK, dk, dv), dtype=torch.float32,
-                     device=q.device)
-    need = chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    ws_bytes = workspace.numel() * workspace.element_size()
-    st = _native.lib().kla_chunk_fwd_states(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0), _ptr(o), _ptr(hT),
-        _ptr(hs), B, T, H, dk, dv, _DT[q.dtype], _ptr(workspace), ws_bytes, _stream(stream))
+    with _on(q, stream) as s:
+        B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, eta, h0, None, None, outputs)
+        if not outputs:
+            o = None
+        hs = torch.empty((B, H, (T + CHUNK - 1) // CHUNK, dk, dv), dtype=torch.float32,
+                         device=q.device)
+        need = chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        _need(workspace, "workspace", torch.uint8, dev=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+        st = _native.lib().kla_chunk_fwd_states(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0), _ptr(o),
+            _ptr(hT), _ptr(hs), B, T, H, dk, dv, _DT[q.dtype], _ptr(workspace), ws_bytes, s)
     _check(st, "kla_chunk_fwd_states")
     return o, hT, hs
 
@@ -129,6 +163,7 @@ def _workspace(workspace, B, T, H, dk, dv, dtype, device):
     need = chunk_fwd_workspace_size(B, T, H, dk, dv, dtype)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    _need(workspace, "workspace", torch.uint8, dev=device)
     return workspace, workspace.numel() * workspace.element_size()
 
 
@@ -138,14 +173,36 @@ def chunk_ut_transform(k, g, eta, eps: float = 1e-6, *, workspace=None, stream=N
     which is returned."""
     _need(k, "k", torch.bfloat16)
     B, T, H, dk = k.shape
-    _need(g, "g", torch.float32, (B, T, H))
-    _need(eta, "eta", torch.float32, (B, T, H))
-    workspace, ws_bytes = _workspace(workspace, B, T, H, dk, dk, k.dtype, k.device)
-    st = _native.lib().kla_chunk_ut_transform(
-        _ptr(k), _ptr(g), _ptr(eta), float(eps), B, T, H, dk, KLA_BF16, _ptr(workspace),
-        ws_bytes, _stream(stream))
+    _need(g, "g", torch.float32, (B, T, H), k.device)
+    _need(eta, "eta", torch.float32, (B, T, H), k.device)
+    with _on(k, stream) as s:
+        workspace, ws_bytes = _workspace(workspace, B, T, H, dk, dk, k.dtype, k.device)
+        st = _native.lib().kla_chunk_ut_transform(
+            _ptr(k), _ptr(g), _ptr(eta), float(eps), B, T, H, dk, KLA_BF16, _ptr(workspace),
+            ws_bytes, s)
     _check(st, "kla_chunk_ut_transform")
     return workspace
+
+
+def chunk_ut_bound_check(k, g, eta, eps: float = 1e-6, *, workspace=None, stream=None):
+    """kla_chunk_ut_transform with the debug check of its factors
+    (kla_chunk_ut_bound_check).  Returns (workspace, ratio_max) with
+    ratio_max a one-element fp32 CUDA tensor: the largest ratio of
+    |T_rs| ||k_r|| / ||k_s|| to eta'_r e^{G_r - G_s} over the factors'
+    entries.  A ratio above 1.25 also sets the device error word
+    (check_device_error then raises KLAError with KLA_ERR_BOUND)."""
+    _need(k, "k", torch.bfloat16)
+    B, T, H, dk = k.shape
+    _need(g, "g", torch.float32, (B, T, H), k.device)
+    _need(eta, "eta", torch.float32, (B, T, H), k.device)
+    with _on(k, stream) as s:
+        workspace, ws_bytes = _workspace(workspace, B, T, H, dk, dk, k.dtype, k.device)
+        ratio = torch.empty(4, dtype=torch.float32, device=k.device)  # 16-byte aligned
+        st = _native.lib().kla_chunk_ut_bound_check(
+            _ptr(k), _ptr(g), _ptr(eta), float(eps), B, T, H, dk, KLA_BF16, _ptr(workspace),
+            ws_bytes, _ptr(ratio), s)
+    _check(st, "kla_chunk_ut_bound_check")
+    return workspace, ratio[:1]
 
 
 def chunk_state_fwd(q, k, v, g, workspace, h0=None, *, o=None, hT=None,
@@ -153,12 +210,15 @@ def chunk_state_fwd(q, k, v, g, workspace, h0=None, *, o=None, hT=None,
     """Second stage of the bf16 chunk prefill (kla_chunk_state_fwd): the
     state recurrence and outputs from a workspace made by chunk_ut_transform
     of the same k and g.  Returns (o, hT)."""
-    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, g, h0, o, hT, return_state)
-    _need(workspace, "workspace", torch.uint8)
-    ws_bytes = workspace.numel() * workspace.element_size()
-    st = _native.lib().kla_chunk_state_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(h0), _ptr(o), _ptr(hT), B, T, H, dk, dv,
-        _DT[q.dtype], _ptr(workspace), ws_bytes, _stream(stream))
+    with _on(q, stream) as s:
+        B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, g, h0, o, hT, return_state)
+        if workspace is None:
+            raise ValueError("workspace must be a CUDA tensor")
+        _need(workspace, "workspace", torch.uint8, dev=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+        st = _native.lib().kla_chunk_state_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(h0), _ptr(o), _ptr(hT), B, T, H, dk, dv,
+            _DT[q.dtype], _ptr(workspace), ws_bytes, s)
     _check(st, "kla_chunk_state_fwd")
     return o, hT
 
@@ -166,10 +226,11 @@ def chunk_state_fwd(q, k, v, g, workspace, h0=None, *, o=None, hT=None,
 def recurrent_fwd(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=None,
                   return_state: bool = True, stream=None):
     """Token-serial KLA prefill on CUDA cores (kla_recurrent_fwd)."""
-    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, eta, h0, o, hT, return_state)
-    st = _native.lib().kla_recurrent_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0),
-        _ptr(o), _ptr(hT), B, T, H, dk, dv, _DT[q.dtype], _stream(stream))
+    with _on(q, stream) as s:
+        B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, eta, h0, o, hT, return_state)
+        st = _native.lib().kla_recurrent_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0),
+            _ptr(o), _ptr(hT), B, T, H, dk, dv, _DT[q.dtype], s)
     _check(st, "kla_recurrent_fwd")
     return o, hT
 
@@ -194,14 +255,24 @@ def _bwd(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0, workspac
         raise ValueError("q, k, v must be bfloat16 or float32")
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    _need(k, "k", q.dtype, (B, T, H, dk))
-    _need(v, "v", q.dtype, (B, T, H, dv))
+    d = q.device
+    _need(k, "k", q.dtype, (B, T, H, dk), d)
+    _need(v, "v", q.dtype, (B, T, H, dv), d)
     gshape = (B, T, H, dk) if vector_gate else (B, T, H)
-    _need(g, "g", torch.float32, gshape)
-    _need(step, "eta/beta", torch.float32, (B, T, H))
-    _need(h0, "h0", torch.float32, (B, H, dk, dv))
-    _need(grad_o, "grad_o", q.dtype, (B, T, H, dv))
-    _need(grad_hT, "grad_hT", torch.float32, (B, H, dk, dv))
+    _need(g, "g", torch.float32, gshape, d)
+    _need(step, "eta/beta", torch.float32, (B, T, H), d)
+    _need(h0, "h0", torch.float32, (B, H, dk, dv), d)
+    _need(grad_o, "grad_o", q.dtype, (B, T, H, dv), d)
+    _need(grad_hT, "grad_hT", torch.float32, (B, H, dk, dv), d)
+    with _on(q, stream) as s:
+        return _bwd_launch(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0,
+                           workspace, s, gshape, vector_gate, chunked)
+
+
+def _bwd_launch(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0, workspace, s,
+                gshape, vector_gate, chunked):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
     f32 = dict(dtype=torch.float32, device=q.device)
     out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
                dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty(gshape, **f32),
@@ -214,13 +285,14 @@ def _bwd(fn, name, q, k, v, g, step, eps, h0, grad_o, grad_hT, need_h0, workspac
                 else recurrent_bwd_workspace_size)(B, T, H, dk, dv)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8, dev=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
     if eps is not None:
         args.append(float(eps))
     args += [_ptr(h0), _ptr(grad_o), _ptr(grad_hT), _ptr(out["dq"]), _ptr(out["dk"]),
              _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dstep"]), _ptr(out["dh0"]),
-             B, T, H, dk, dv, _DT[q.dtype], _ptr(workspace), ws_bytes, _stream(stream)]
+             B, T, H, dk, dv, _DT[q.dtype], _ptr(workspace), ws_bytes, s]
     _check(fn(*args), name)
     return out
 
@@ -294,17 +366,19 @@ def decode_step(q, k, v, g, eta, S, eps: float = 1e-6, *, o=None, stream=None):
         raise ValueError("q, k, v must be bfloat16 or float32")
     B, H, dk = q.shape
     dv = v.shape[-1]
-    _need(k, "k", q.dtype, (B, H, dk))
-    _need(v, "v", q.dtype, (B, H, dv))
-    _need(g, "g", torch.float32, (B, H))
-    _need(eta, "eta", torch.float32, (B, H))
-    _need(S, "S", torch.float32, (B, H, dk, dv))
-    if o is None:
-        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
-    _need(o, "o", q.dtype, (B, H, dv))
-    st = _native.lib().kla_decode_step(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(S), _ptr(o),
-        B, H, dk, dv, _DT[q.dtype], _stream(stream))
+    d = q.device
+    _need(k, "k", q.dtype, (B, H, dk), d)
+    _need(v, "v", q.dtype, (B, H, dv), d)
+    _need(g, "g", torch.float32, (B, H), d)
+    _need(eta, "eta", torch.float32, (B, H), d)
+    _need(S, "S", torch.float32, (B, H, dk, dv), d)
+    with _on(q, stream) as s:
+        if o is None:
+            o = torch.empty((B, H, dv), dtype=q.dtype, device=d)
+        _need(o, "o", q.dtype, (B, H, dv), d)
+        st = _native.lib().kla_decode_step(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(S), _ptr(o),
+            B, H, dk, dv, _DT[q.dtype], s)
     _check(st, "kla_decode_step")
     return o
 
@@ -313,14 +387,16 @@ def gdn_chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, hT=None, return_state: b
                   workspace=None, stream=None):
     """Gated DeltaNet prefill (kla_gdn_chunk_fwd): beta [B,T,H] fp32 is the
     step size itself.  Returns (o, hT)."""
-    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, beta, h0, o, hT, return_state)
-    need = chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = _native.lib().kla_gdn_chunk_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT),
-        B, T, H, dk, dv, CHUNK, _DT[q.dtype], _ptr(workspace), ws_bytes, _stream(stream))
+    with _on(q, stream) as s:
+        B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, g, beta, h0, o, hT, return_state)
+        need = chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _need(workspace, "workspace", torch.uint8, dev=q.device)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = _native.lib().kla_gdn_chunk_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT),
+            B, T, H, dk, dv, CHUNK, _DT[q.dtype], _ptr(workspace), ws_bytes, s)
     _check(st, "kla_gdn_chunk_fwd")
     return o, hT
 
@@ -333,17 +409,19 @@ def gdn_decode_step(q, k, v, g, beta, S, *, o=None, stream=None):
         raise ValueError("q, k, v must be bfloat16 or float32")
     B, H, dk = q.shape
     dv = v.shape[-1]
-    _need(k, "k", q.dtype, (B, H, dk))
-    _need(v, "v", q.dtype, (B, H, dv))
-    _need(g, "g", torch.float32, (B, H))
-    _need(beta, "beta", torch.float32, (B, H))
-    _need(S, "S", torch.float32, (B, H, dk, dv))
-    if o is None:
-        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
-    _need(o, "o", q.dtype, (B, H, dv))
-    st = _native.lib().kla_gdn_decode_step(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o), B, H, dk, dv,
-        _DT[q.dtype], _stream(stream))
+    d = q.device
+    _need(k, "k", q.dtype, (B, H, dk), d)
+    _need(v, "v", q.dtype, (B, H, dv), d)
+    _need(g, "g", torch.float32, (B, H), d)
+    _need(beta, "beta", torch.float32, (B, H), d)
+    _need(S, "S", torch.float32, (B, H, dk, dv), d)
+    with _on(q, stream) as s:
+        if o is None:
+            o = torch.empty((B, H, dv), dtype=q.dtype, device=d)
+        _need(o, "o", q.dtype, (B, H, dv), d)
+        st = _native.lib().kla_gdn_decode_step(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o), B, H, dk, dv,
+            _DT[q.dtype], s)
     _check(st, "kla_gdn_decode_step")
     return o
 
@@ -386,30 +464,39 @@ def chunk_fwd_host(q, k, v, g, eta, eps: float = 1e-6, h0=None, *, o=None, hT=No
     if hT is None and return_state:
         hT = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
     _need_host(hT, "hT", torch.float32, (B, H, dk, dv))
-    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    if device is None:
+        device = staging.device if staging is not None else (
+            stream.device if stream is not None else
+            torch.device("cuda", torch.cuda.current_device()))
+    dev = torch.device(device)
     need = chunk_fwd_host_staging_size(B, T, H, dk, dv, q.dtype)
-    if staging is None:
-        staging = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
-    _need(staging, "staging", torch.uint8)
-    st = _native.lib().kla_chunk_fwd_host(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0), _ptr(o),
-        _ptr(hT), B, T, H, dk, dv, _DT[q.dtype], _ptr(staging),
-        staging.numel() * staging.element_size(), _stream(stream))
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        if s.device != dev:
+            raise ValueError("stream is on %s, the staging buffer on %s" % (s.device, dev))
+        with torch.cuda.stream(s):
+            if staging is None:
+                staging = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+            _need(staging, "staging", torch.uint8, dev=dev)
+            st = _native.lib().kla_chunk_fwd_host(
+                _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(eta), float(eps), _ptr(h0), _ptr(o),
+                _ptr(hT), B, T, H, dk, dv, _DT[q.dtype], _ptr(staging),
+                staging.numel() * staging.element_size(), s.cuda_stream)
     _check(st, "kla_chunk_fwd_host")
     return o, hT
 
 
 def _kda_prefill(fn, name, q, k, v, g, step, eps, h0, o, hT, return_state, stream):
     # the per-token arguments as for chunk_fwd; g is checked on its own
-    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, None, step, h0, o, hT, return_state)
-    if g is None:
-        raise ValueError("g must be a CUDA tensor")
-    _need(g, "g", torch.float32, (B, T, H, dk))
-    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
-    if eps is not None:
-        args.append(float(eps))
-    st = fn(*args, _ptr(h0), _ptr(o), _ptr(hT), B, T, H, dk, dv, _DT[q.dtype],
-            _stream(stream))
+    with _on(q, stream) as s:
+        B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, None, step, h0, o, hT, return_state)
+        if g is None:
+            raise ValueError("g must be a CUDA tensor")
+        _need(g, "g", torch.float32, (B, T, H, dk), q.device)
+        args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
+        if eps is not None:
+            args.append(float(eps))
+        st = fn(*args, _ptr(h0), _ptr(o), _ptr(hT), B, T, H, dk, dv, _DT[q.dtype], s)
     _check(st, name)
     return o, hT
 
@@ -435,19 +522,21 @@ def kda_chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
 
 
 def _kda_chunk(fn, name, q, k, v, g, step, eps, h0, o, hT, return_state, workspace, stream):
-    B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, None, step, h0, o, hT, return_state)
-    if g is None:
-        raise ValueError("g must be a CUDA tensor")
-    _need(g, "g", torch.float32, (B, T, H, dk))
-    need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
-    if eps is not None:
-        args.append(float(eps))
-    st = fn(*args, _ptr(h0), _ptr(o), _ptr(hT), B, T, H, dk, dv, CHUNK, _DT[q.dtype],
-            _ptr(workspace), ws_bytes, _stream(stream))
+    with _on(q, stream) as s:
+        B, T, H, dk, dv, o, hT = _prefill_args(q, k, v, None, step, h0, o, hT, return_state)
+        if g is None:
+            raise ValueError("g must be a CUDA tensor")
+        _need(g, "g", torch.float32, (B, T, H, dk), q.device)
+        need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, q.dtype)
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _need(workspace, "workspace", torch.uint8, dev=q.device)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
+        if eps is not None:
+            args.append(float(eps))
+        st = fn(*args, _ptr(h0), _ptr(o), _ptr(hT), B, T, H, dk, dv, CHUNK, _DT[q.dtype],
+                _ptr(workspace), ws_bytes, s)
     _check(st, name)
     return o, hT
 
@@ -473,18 +562,21 @@ def _kda_decode(fn, name, q, k, v, g, step, eps, S, o, stream):
         raise ValueError("q, k, v must be bfloat16 or float32")
     B, H, dk = q.shape
     dv = v.shape[-1]
-    _need(k, "k", q.dtype, (B, H, dk))
-    _need(v, "v", q.dtype, (B, H, dv))
-    _need(g, "g", torch.float32, (B, H, dk))
-    _need(step, "eta" if eps is not None else "beta", torch.float32, (B, H))
-    _need(S, "S", torch.float32, (B, H, dk, dv))
-    if o is None:
-        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
-    _need(o, "o", q.dtype, (B, H, dv))
-    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
-    if eps is not None:
-        args.append(float(eps))
-    _check(fn(*args, _ptr(S), _ptr(o), B, H, dk, dv, _DT[q.dtype], _stream(stream)), name)
+    d = q.device
+    _need(k, "k", q.dtype, (B, H, dk), d)
+    _need(v, "v", q.dtype, (B, H, dv), d)
+    _need(g, "g", torch.float32, (B, H, dk), d)
+    _need(step, "eta" if eps is not None else "beta", torch.float32, (B, H), d)
+    _need(S, "S", torch.float32, (B, H, dk, dv), d)
+    with _on(q, stream) as s:
+        if o is None:
+            o = torch.empty((B, H, dv), dtype=q.dtype, device=d)
+        _need(o, "o", q.dtype, (B, H, dv), d)
+        args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(step)]
+        if eps is not None:
+            args.append(float(eps))
+        st = fn(*args, _ptr(S), _ptr(o), B, H, dk, dv, _DT[q.dtype], s)
+    _check(st, name)
     return o
 
 
@@ -502,5 +594,9 @@ def kda_decode_step_beta(q, k, v, g, beta, S, *, o=None, stream=None):
 
 
 def check_device_error(stream=None):
-    """Synchronise and raise KLAError if a kernel reported a timed-out wait."""
-    _check(_native.lib().kla_check_device_error(_stream(stream)), "kla_check_device_error")
+    """Synchronise and raise KLAError if a kernel reported a timed-out wait
+    (on the device of ``stream``; default: the current device's current
+    stream)."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    with torch.cuda.device(s.device):
+        _check(_native.lib().kla_check_device_error(s.cuda_stream), "kla_check_device_error")

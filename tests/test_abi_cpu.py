@@ -171,9 +171,29 @@ def test_selftest_rejects_bad_limits(lib):
     assert lib.kla_selftest_wait_timeout(10001, None) == INVALID
 
 
+def _flag_bytes(B, T, H):
+    """One ready flag (4 bytes) per chunk, rounded up to 256 bytes: the
+    single-launch prefill's chunk flags after the factors."""
+    return (B * H * ((T + 63) // 64) * 4 + 255) // 256 * 256
+
+
 def test_workspace_query(lib):
-    # enough heads to fill the GPU: the chain runs uncut, factors only
-    assert lib.kla_chunk_fwd_workspace_size(8, 4096, 8, 128, 128, 0) == _ut_bytes(8, 4096, 8)
+    # the 0.4B-scale layer: uncut chain in a single launch, the factors and
+    # one ready flag per chunk
+    assert lib.kla_chunk_fwd_workspace_size(8, 4096, 8, 128, 128, 0) == (
+        _ut_bytes(8, 4096, 8) + _flag_bytes(8, 4096, 8))
+    # more state CTAs than leave room for UT CTAs beside them: two launches,
+    # factors only
+    assert lib.kla_chunk_fwd_workspace_size(16, 4096, 8, 128, 128, 0) == _ut_bytes(16, 4096, 8)
+    # which shapes take the single launch (the full workspace; a workspace of
+    # the factors alone always runs two launches)
+    full = lambda *a: lib.kla_chunk_fwd_workspace_size(*a, 128, 128, 0)
+    assert lib.kla_chunk_fwd_single_launch(8, 4096, 8, 128, 128, 0, full(8, 4096, 8)) == 1
+    assert lib.kla_chunk_fwd_single_launch(8, 4096, 8, 128, 128, 0, _ut_bytes(8, 4096, 8)) == 0
+    assert lib.kla_chunk_fwd_single_launch(16, 4096, 8, 128, 128, 0, 1 << 40) == 0
+    assert lib.kla_chunk_fwd_single_launch(1, 65536, 16, 128, 128, 0, 1 << 40) == 0  # cut
+    assert lib.kla_chunk_fwd_single_launch(4, 8192, 32, 64, 64, 0, 1 << 40) == 1  # stress
+    assert lib.kla_chunk_fwd_single_launch(4, 8192, 32, 64, 64, 1, 1 << 40) == 0  # fp32 I/O
     # few heads and a long sequence: per-segment states (E, start state,
     # transition) follow the factors, for between 2 and 64 segments
     n = lib.kla_chunk_fwd_workspace_size(1, 65536, 16, 128, 128, 0)
@@ -186,7 +206,8 @@ def test_workspace_query(lib):
     assert lib.kla_chunk_fwd_segments(1, 65536, 16, 128, 128, 1, n) == 0  # fp32 I/O
     assert lib.kla_chunk_fwd_segments(1, 65536, 16, 96, 96, 0, n) == 0
     # short sequences are never cut (segments keep at least 8 chunks)
-    assert lib.kla_chunk_fwd_workspace_size(1, 64 * 15, 1, 64, 64, 0) == _ut_bytes(1, 960, 1)
+    assert lib.kla_chunk_fwd_workspace_size(1, 64 * 15, 1, 64, 64, 0) == (
+        _ut_bytes(1, 960, 1) + _flag_bytes(1, 960, 1))
     assert lib.kla_chunk_fwd_workspace_size(1, 65536, 16, 128, 128, 1) == 0  # fp32: none
 
 
@@ -289,7 +310,7 @@ def test_chunk_fwd_states_rejects_bad_arguments(lib):
     assert lib.kla_chunk_fwd_states(*bad) == INVALID
     bad = list(args); bad[15] = 1
     assert lib.kla_chunk_fwd_states(*bad) == UNSUPPORTED  # fp32 I/O
-    bad = list(args); bad[17] = ws - 1
+    bad = list(args); bad[17] = _ut_bytes(1, 128, 2) - 1  # the factors do not fit
     assert lib.kla_chunk_fwd_states(*bad) == INVALID
     bad = list(args); bad[11] = 0
     assert lib.kla_chunk_fwd_states(*bad) == INVALID  # T = 0

@@ -8,7 +8,7 @@ import torch
 import oracle
 from delta_rule_linear_kla_b200 import api, inputs
 
-from helpers import TOL, cuda, rel
+from helpers import TOL, assert_parity, assert_state_parity, cuda, rel
 
 pytestmark = pytest.mark.gpu
 
@@ -132,7 +132,8 @@ def test_kda_chunk_prefill(name, B, T, H, h0):
     o_ref, h_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["gv"], x["eta"], x["eps"],
                                       x["h0"])
     assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
-    assert rel(o.cpu(), o_ref) < TOL["bf16"] and rel(hT.cpu(), h_ref) < TOL["bf16"]
+    assert_parity(o.cpu(), o_ref, "bf16")
+    assert_state_parity(hT.cpu(), h_ref, "bf16")
 
 
 def test_kda_chunk_strong_and_zero_gates():
@@ -150,7 +151,8 @@ def test_kda_chunk_strong_and_zero_gates():
     api.check_device_error()
     o_ref, h_ref = oracle.kda_forward(x["q"], x["k"], x["v"], gv, x["eta"], x["eps"], x["h0"])
     assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
-    assert rel(o.cpu(), o_ref) < TOL["bf16"] and rel(hT.cpu(), h_ref) < TOL["bf16"]
+    assert_parity(o.cpu(), o_ref, "bf16")
+    assert_state_parity(hT.cpu(), h_ref, "bf16")
 
 
 def test_kda_chunk_beta_given_and_fp32():
@@ -185,7 +187,32 @@ def test_kda_chunk_segmented_chain():
     api.check_device_error()
     o_ref, h_ref = oracle.kda_forward(x["q"], x["k"], x["v"], x["gv"], x["eta"], x["eps"],
                                       x["h0"])
-    assert rel(o.cpu(), o_ref) < TOL["bf16"] and rel(hT.cpu(), h_ref) < TOL["bf16"]
+    assert_parity(o.cpu(), o_ref, "bf16")
+    assert_state_parity(hT.cpu(), h_ref, "bf16")
+
+
+@pytest.mark.parametrize("name,heads", [("prefill_4k", [(0, 0), (4, 3), (7, 7)]),
+                                        ("stress", [(0, 0), (2, 19), (3, 31)])])
+def test_kda_chunk_full_size_oracle_sampled(name, heads):
+    """The full-size per-channel-gate chunk prefill, in the launch
+    configuration the benchmark times (every chunk of every head through the
+    factor kernel and the chain), against the fp64 oracle on sampled heads:
+    each head is an independent recurrence the oracle can run alone."""
+    w = inputs.WORKLOADS[name]
+    x = inputs.make_prefill(w)
+    gv = inputs.channel_gates((w.B, w.T, w.H, w.dk), w.seed + 11)
+    xc = cuda(x)
+    o, hT = api.kda_chunk_fwd(xc["q"], xc["k"], xc["v"], cuda(gv), xc["eta"], x["eps"],
+                              xc["h0"])
+    api.check_device_error()
+    o, hT = o.cpu(), hT.cpu()
+    for (b, h) in heads:
+        sl = lambda t: t[b:b + 1, :, h:h + 1]
+        h0 = None if x["h0"] is None else x["h0"][b:b + 1, h:h + 1]
+        o_ref, h_ref = oracle.kda_forward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(gv),
+                                          sl(x["eta"]), x["eps"], h0)
+        assert_parity(sl(o), o_ref, "bf16")
+        assert_state_parity(hT[b:b + 1, h:h + 1], h_ref, "bf16")
 
 
 def test_kda_chunk_matches_token_serial_4k_sampled():
