@@ -242,7 +242,7 @@ def run_ours(args, rank, world, dev):
     # the clock samples that bracket the timed region are taken under load
     t_load = time.perf_counter()
     i = 0
-    while i < args.warmup or time.perf_counter() - t_load < 1.0:
+    while i < args.warmup or time.perf_counter() - t_load < args.min_warmup_s:
         flush()
         step()
         i += 1
@@ -579,10 +579,10 @@ def run_decode(args, rank, dev, stream, peaks, peak_src, prefill_fn, clk):
 
 
 def run_kda_prefill(w, dev, stream, flush, peaks, peak_src, steps=3):
-    """The per-channel-gate prefill (chunk path: per-chunk factor kernel,
-    then the tensor-core state kernel) on the same workload's q, k, v, eta
-    with per-channel gates: time per call and achieved GB/s of its
-    algorithmic bytes (q, k, v, o, the [B,T,H,dk] gates, eta, h_T)."""
+    """The per-channel-gate prefill through kla_kda_chunk_fwd on the same
+    workload's q, k, v, eta with per-channel gates: time per call and
+    achieved GB/s of its algorithmic bytes (q, k, v, o, the [B,T,H,dk]
+    gates, eta, h_T)."""
     from delta_rule_linear_kla_b200 import api, inputs
 
     x = inputs.make_prefill(w)
@@ -615,8 +615,9 @@ def run_kda_prefill(w, dev, stream, flush, peaks, peak_src, steps=3):
     return {"metric": "prefill tokens/s, per-channel gate (%s)" % w.name,
             "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
             "calls": steps,
-            "path": "kda_prep_kernel (per-chunk factors: fp32 CUDA cores and bf16 warp "
-                    "MMAs) + chain_kernel (KDA mode, tcgen05)",
+            "path": "kla_kda_chunk_fwd: the token-serial per-channel kernel (the chunk "
+                    "kernels of this form are not used: intermittent faults, cause not "
+                    "found)",
             "roofline": {"kernel": "whole call", "bound": "hbm",
                          "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "traffic": None, "algorithmic_bytes": byts,
@@ -804,6 +805,9 @@ def main():
                     help="skip the per-channel-gate (KDA form) prefill measurement")
     ap.add_argument("--no-bwd", action="store_true",
                     help="skip the backward (gradients) measurement")
+    ap.add_argument("--min-warmup-s", type=float, default=1.0,
+                    help="seconds of back-to-back warm-up steps before timing (clock "
+                         "samples under load); 0 for a profiler's short command")
     ap.add_argument("--no-other", action="store_true",
                     help="skip the 65K and stress prefill workloads")
     ap.add_argument("--decode-only", action="store_true",

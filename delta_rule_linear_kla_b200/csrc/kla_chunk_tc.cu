@@ -56,6 +56,8 @@
 // Every wait is bounded (about 2 s); on timeout the kernel raises the device
 // error word, stops all roles, drains its own TMA loads and MMAs and frees
 // TMEM.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -127,6 +129,14 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
       return false;
     }
   }
+}
+
+// The same wait taken by a whole warp that then runs warp-collective
+// instructions (elect.sync, tcgen05.ld, __syncwarp): every lane waits, and
+// if any lane gives up, all of them do, so the warp never splits.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag));
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -365,7 +375,7 @@ __device__ __forceinline__ void chain_body(
       __syncwarp();
     };
     bool ok = nchunks > 0;
-    if (ok) ok = wait_or_abort(&s.full[0], 0, abort_flag);
+    if (ok) ok = wait_warp(&s.full[0], 0, abort_flag);
     if (ok) {
       ptx::tc_fence_after();
       if constexpr (KDA) {
@@ -373,7 +383,7 @@ __device__ __forceinline__ void chain_body(
       } else {
         mma2(0);
         mma3(0);
-        ok = wait_or_abort(&s.w_done, 0, abort_flag);
+        ok = wait_warp(&s.w_done, 0, abort_flag);
         if (ok) {
           ptx::tc_fence_after();
           mma1(0);
@@ -386,8 +396,8 @@ __device__ __forceinline__ void chain_body(
       const uint32_t par = (uint32_t)(n & 1);
       const bool more = n + 1 < nchunks;
       // ---- MMA 4 (chunk n): needs W(n) and h_n (D_H of n-1 read)
-      if (!KDA && !wait_or_abort(&s.w_done, par, abort_flag)) break;
-      if (!wait_or_abort(&s.h_done, par, abort_flag)) break;
+      if (!KDA && !wait_warp(&s.w_done, par, abort_flag)) break;
+      if (!wait_warp(&s.h_done, par, abort_flag)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
@@ -400,13 +410,13 @@ __device__ __forceinline__ void chain_body(
       // ---- while V'(n) is formed: W of chunk n+1 (needed by its MMA 4);
       //      D_W was read before w_done(n)
       if (more) {
-        if (!wait_or_abort(&s.full[(n + 1) & 1], (uint32_t)(((n + 1) >> 1) & 1), abort_flag))
+        if (!wait_warp(&s.full[(n + 1) & 1], (uint32_t)(((n + 1) >> 1) & 1), abort_flag))
           break;
         ptx::tc_fence_after();
         if constexpr (!KDA) mma2(n + 1);
       }
       // ---- MMA 5 (state), committed on its own so the update starts at once
-      if (!wait_or_abort(&s.vpd_ready, par, abort_flag)) break;
+      if (!wait_warp(&s.vpd_ready, par, abort_flag)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
@@ -418,9 +428,9 @@ __device__ __forceinline__ void chain_body(
       __syncwarp();
       // ---- MMA 6 (chunk n): needs V'(n), P(n) and D_PV free (outputs of n-1
       //      read)
-      if (!wait_or_abort(&s.vp_ready, par, abort_flag)) break;
-      if (!KDA && !wait_or_abort(&s.p_done, par, abort_flag)) break;
-      if (n > 0 && !wait_or_abort(&s.pv_free, par ^ 1u, abort_flag)) break;
+      if (!wait_warp(&s.vp_ready, par, abort_flag)) break;
+      if (!KDA && !wait_warp(&s.p_done, par, abort_flag)) break;
+      if (n > 0 && !wait_warp(&s.pv_free, par ^ 1u, abort_flag)) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
@@ -434,14 +444,14 @@ __device__ __forceinline__ void chain_body(
         // ---- while the state is updated: U of chunk n+1 (D_U[(n+1)%2] was
         //      used by chunk n-1; MMA 4 of n+1 accumulates onto it) ...
         if (n >= 1 &&
-            !wait_or_abort(&s.u_free[(n + 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), abort_flag))
+            !wait_warp(&s.u_free[(n + 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), abort_flag))
           break;
         ptx::tc_fence_after();
         mma3(n + 1);
         if constexpr (!KDA) {
           // ... and Q K^T of chunk n+1: D_S was read by P(n) (waited above);
           // waiting for W(n+1) keeps its rows from changing under the read
-          if (!wait_or_abort(&s.w_done, par ^ 1u, abort_flag)) break;
+          if (!wait_warp(&s.w_done, par ^ 1u, abort_flag)) break;
           ptx::tc_fence_after();
           mma1(n + 1);
         }
@@ -456,7 +466,7 @@ __device__ __forceinline__ void chain_body(
     // W rows 0..63 (TMEM lanes 0..63) -> the stage's W slot (bf16)
     for (int n = 0; n < (KDA ? 0 : nchunks); ++n) {
       Stage<DK>& S = s.st[n & 1];
-      if (!wait_or_abort(&s.bW, (uint32_t)(n & 1), abort_flag)) break;
+      if (!wait_warp(&s.bW, (uint32_t)(n & 1), abort_flag)) break;
       ptx::tc_fence_after();
 #pragma unroll
       for (int p = 0; p < NP; ++p) {
@@ -484,7 +494,7 @@ __device__ __forceinline__ void chain_body(
       // the chunk decay e^{G_last} (one per key channel) arrives with the
       // stage; warp 2 publishes it through the g_ready ring
       for (int n = 0; n < (warp == 2 ? nchunks : 0); ++n) {
-        if (!wait_or_abort(&s.full[n & 1], (uint32_t)((n >> 1) & 1), abort_flag)) break;
+        if (!wait_warp(&s.full[n & 1], (uint32_t)((n >> 1) & 1), abort_flag)) break;
         const float* dsrc = reinterpret_cast<const float*>(s.st[n & 1].tp[TP2]);
         for (int i = lane; i < DK; i += 32) s.kdec[n % 3][i] = dsrc[i];
         __syncwarp();
@@ -521,7 +531,7 @@ __device__ __forceinline__ void chain_body(
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.g_ready[n % 3]);
       } else {
-        if (!wait_or_abort(&s.g_ready[n % 3], (uint32_t)((n / 3) & 1), abort_flag)) break;
+        if (!wait_warp(&s.g_ready[n % 3], (uint32_t)((n / 3) & 1), abort_flag)) break;
       }
       // ---- P row r, columns [32 hc, 32 hc + 32): e^{G_r - G_s} is the
       //      running product of alpha_j over s < j <= r, from the diagonal
@@ -536,7 +546,7 @@ __device__ __forceinline__ void chain_body(
         const float4 a4 = reinterpret_cast<const float4*>(&s.alpha[n % 3][32 * hc])[i];
         al[4 * i] = a4.x; al[4 * i + 1] = a4.y; al[4 * i + 2] = a4.z; al[4 * i + 3] = a4.w;
       }
-      if (!wait_or_abort(&s.bS, (uint32_t)(n & 1), abort_flag)) break;
+      if (!wait_warp(&s.bS, (uint32_t)(n & 1), abort_flag)) break;
       ptx::tc_fence_after();
       float srow[32];
       ptx::tmem_ld32(tb + lane_base + COL_S + 32 * hc, srow);
@@ -593,11 +603,11 @@ __device__ __forceinline__ void chain_body(
       const float* Gn = s.G[n % 3];
       const uint32_t par = (uint32_t)(n & 1);
       const uint32_t col_u = COL_U + 64 * (n & 1);
-      if (!wait_or_abort(&s.g_ready[n % 3], (uint32_t)((n / 3) & 1), abort_flag)) { ok = false; break; }
+      if (!wait_warp(&s.g_ready[n % 3], (uint32_t)((n / 3) & 1), abort_flag)) { ok = false; break; }
       const float gC = KDA ? 0.f : Gn[C - 1];
       if (v_rows && KDA) {
         // V' = U - W h (combined in TMEM); the keys of MMA 5 carry the decay
-        if (!wait_or_abort(&s.bX, par, abort_flag)) { ok = false; break; }
+        if (!wait_warp(&s.bX, par, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
         float u[32];
         ptx::tmem_ld32(tb + lane_base + col_u + cg, u);
@@ -614,7 +624,7 @@ __device__ __forceinline__ void chain_body(
         // V'_r = U_r - (W h)_r (already combined in TMEM) and its copy
         // decayed to the chunk end for MMA 5
         const float dec = __expf(gC - Gn[row]);
-        if (!wait_or_abort(&s.bX, par, abort_flag)) { ok = false; break; }
+        if (!wait_warp(&s.bX, par, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
         float u[32], ud[32];
         ptx::tmem_ld32(tb + lane_base + col_u + cg, u);
@@ -636,7 +646,7 @@ __device__ __forceinline__ void chain_body(
       }
       // every read of G(n) happens before this warp's last arrival of chunk n
       const float e_out = v_rows ? 0.f : (KDA ? -1.f : -__expf(Gn[row - 64]));
-      if (!wait_or_abort(&s.bH, par, abort_flag)) { ok = false; break; }
+      if (!wait_warp(&s.bH, par, abort_flag)) { ok = false; break; }
       ptx::tc_fence_after();
       if (has_h) {
         const float a = KDA ? s.kdec[n % 3][row] : __expf(gC);
@@ -655,7 +665,7 @@ __device__ __forceinline__ void chain_body(
         // -(Q h)_r in lanes 64..127 of D_U
         const int r = row - 64, t = (n0 + n) * C + r;
         const float e = e_out;
-        if (!wait_or_abort(&s.bHP, par, abort_flag)) { ok = false; break; }
+        if (!wait_warp(&s.bHP, par, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
         float x[32], pv[32];
         ptx::tmem_ld32(tb + lane_base + col_u + cg, x);
@@ -726,7 +736,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 // as the state CTA's shared memory holds.
 template <int DK>
 constexpr int fused_ut_lanes() {
-  return DK == 128 ? 3 : 4;
+  return 3;
 }
 template <int DK>
 constexpr size_t fused_smem_bytes() {
@@ -917,12 +927,26 @@ size_t segment_bytes(int B, int T, int H, int dk, int dv) {
 // the state CTAs.
 constexpr int kMinUtCtas = 8;
 
+// Measured costs on a B200 (in units of one chain step, ~1.9 us at the
+// 0.4B-scale layer): a UT lane takes ~5 chain steps per pair of chunks.
+constexpr long kPairCost = 5, kStepCost = 1;
+
 // Whether a shape runs as one launch: an uncut chain whose state CTAs leave
-// room for UT CTAs on the 148 SMs of a B200 (the launcher checks the actual
-// device again and otherwise runs the two kernels one after the other).
+// room for UT CTAs on the 148 SMs of a B200, and for which the UT lanes on
+// those SMs finish sooner than the UT kernel alone would on all of them plus
+// the chain after it (the launcher checks the actual device again and
+// otherwise runs the two kernels one after the other).
 bool fused_shape(int B, int T, int H, int dk, int dv) {
-  return chain_segments(B, T, H, dk, dv) == 1 &&
-         (long)B * H * (dv / BV) + kMinUtCtas <= kSmTarget;
+  if (chain_segments(B, T, H, dk, dv) != 1) return false;
+  const long n_chain = (long)B * H * (dv / BV);
+  if (n_chain + kMinUtCtas > kSmTarget) return false;
+  const long nchunks = (T + C - 1) / C, pairs = ((long)B * H * nchunks + 1) / 2;
+  const long lanes_alone = 3L * kSmTarget;
+  const long lanes_fused = 3L * (kSmTarget - n_chain);
+  const long chain = nchunks * kStepCost;
+  const long two = (pairs + lanes_alone - 1) / lanes_alone * kPairCost + chain;
+  const long one = std::max((pairs + lanes_fused - 1) / lanes_fused * kPairCost, chain);
+  return one < two;
 }
 
 // One ready flag per chunk after the factors (single launch only).
@@ -1107,24 +1131,20 @@ size_t kda_tiles_bytes(int B, int T, int H, int dk) {
 size_t kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
   if (dtype != KLA_BF16 || B < 1 || H < 1 || T < 1 || dk != dv || (dk != 64 && dk != 128))
     return 0;
-  return kda_tiles_bytes(B, T, H, dk) + segment_bytes(B, T, H, dk, dv);
+  return kda_tiles_bytes(B, T, H, dk);
 }
 
+// The per-channel-gate prefill always runs the uncut chain (its cut-chain
+// mode is not used: see the safety record of the design notes).
 cudaError_t launch_kda_chunk(const void* q, const void* k, const void* v, const float* g,
                              const float* eta, float eps, const float* h0, void* o, float* hT,
                              int B, int T, int H, int dk, int dv, void* workspace,
                              size_t ws_bytes, unsigned int* err, cudaStream_t st) {
+  (void)ws_bytes;
   if (dk != dv || (dk != 64 && dk != 128)) return cudaErrorNotSupported;
   cudaError_t e = launch_kda_prep(q, k, g, eta, eps, B, T, H, dk, workspace, st);
   if (e != cudaSuccess) return e;
-  const size_t tiles = kda_tiles_bytes(B, T, H, dk);
-  const int sg = chain_segments(B, T, H, dk, dv);
   uint8_t* ws = (uint8_t*)workspace;
-  if (sg > 1 && ws_bytes >= tiles + segment_bytes(B, T, H, dk, dv)) {
-    if (dk == 128)
-      return launch_segmented<128, true>(q, k, v, g, h0, o, hT, B, T, H, sg, ws, tiles, err, st);
-    return launch_segmented<64, true>(q, k, v, g, h0, o, hT, B, T, H, sg, ws, tiles, err, st);
-  }
   const int nchunks = (T + C - 1) / C;
   if (dk == 128)
     return launch_chain_dk<128, true>(q, k, v, g, h0, o, hT, nullptr, B, T, H, dv, 1, nchunks, 0,

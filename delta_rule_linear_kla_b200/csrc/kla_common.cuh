@@ -35,7 +35,7 @@ __device__ __forceinline__ float step_size(float eta, float knorm2, float eps) {
 cudaError_t launch_decode(const void* q, const void* k, const void* v,
                           const float* g, bool vector_gate, const float* eta, float eps,
                           float* S, void* o, int B, int H, int dk, int dv, int dtype,
-                          unsigned int* err, cudaStream_t st);
+                          cudaStream_t st);
 cudaError_t launch_recurrent(const void* q, const void* k, const void* v,
                              const float* g, bool vector_gate, const float* eta, float eps,
                              const float* h0, void* o, float* hT, int B, int T,

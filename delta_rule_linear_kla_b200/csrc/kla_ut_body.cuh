@@ -72,13 +72,17 @@ constexpr float kBoundSlack = 1.25f;     // allowance for the factors' own round
 
 template <int DK>
 constexpr int ctas_per_sm() {
-  return DK == 128 ? 3 : 4;
+  return 3;
 }
 
 template <int DK>
 struct alignas(1024) UtSmem {
   static constexpr int NP = DK / 64;
-  uint8_t keys[NP * TILE];           // [K0; K1] per 64-column panel (TMA, 128-byte swizzle)
+  // [K0; K1] per 64-column panel (TMA, 128-byte swizzle); once the Gram MMA
+  // has read them, the pair's two output tiles (16 KB each) are assembled
+  // here and leave with one bulk store per chunk
+  static constexpr int KEYS_BYTES = NP * TILE > 2 * 16384 ? NP * TILE : 2 * 16384;
+  uint8_t keys[KEYS_BYTES];
   __nv_bfloat16 a[2][C][AROW];       // A left of the diagonal blocks, bf16, row-major
   __nv_bfloat16 dt[2][4][16][DROW];  // D_b^T (row c = column c of D_b), bf16
   float ad[2][4][16][17];            // diagonal blocks of A, fp32 ([row][column], padded)
@@ -235,6 +239,18 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
   bool ok = true;
   uint32_t mma_phase = 0, tma_phase = 0;
   bool keys_in_flight = tid == 0 && first_pair < npairs;
+  int flag_pair = -1;  // pair whose factors were stored but not yet flagged
+  // raise the ready flags of both chunks of pair `pr` (after their stores
+  // completed and a fence)
+  auto publish = [&](int pr) {
+    for (int jj = 0; jj < 2; ++jj) {
+      if (2 * pr + jj < total_chunks) {
+        int hd, nn;
+        chunk_of(2 * pr + jj, hd, nn);
+        atomicExch(flags + (size_t)hd * nchunks + nn, 1u);
+      }
+    }
+  };
   float worst = 0.f;  // CHECK: largest bound ratio this thread saw
 
   // persistent: pairs first_pair, first_pair + pair_stride, ...  Every
@@ -244,9 +260,6 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
   for (int pair = first_pair; pair < npairs; pair += pair_stride) {
     if (!nbar_and(bar_id, ok)) break;  // also: the previous pair's readers are done
     const bool valid = 2 * pair + j < total_chunks;
-    int hd_j = 0, nn_j = 0;
-    if (valid) chunk_of(2 * pair + j, hd_j, nn_j);
-    const int ci = hd_j * nchunks + nn_j;  // workspace index (head-major)
     // chunk-local inclusive cumsum of g (warps 2j, 2j+1 hold chunk j)
     float gs = gr;
 #pragma unroll
@@ -279,10 +292,13 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
         }
         ptx::mma_commit(&s.bar_mma);
         ok = wait_bounded(&s.bar_mma, mma_phase);
-        // the MMA has read the keys: the next pair's may land now
-        if (ok && pair + pair_stride < npairs) {
-          load_keys(pair + pair_stride);
-          keys_in_flight = true;
+        // the previous pair's factors have landed by now: raise its flags
+        if (nmajor && flag_pair >= 0) {
+          ptx::bulk_wait_group_all();
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          __threadfence();
+          publish(flag_pair);
+          flag_pair = -1;
         }
       }
     }
@@ -295,47 +311,55 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
     // row r of A
     const int bb = r >> 4;  // my 16-row block
     {
-      float v[64];
-      ptx::tmem_ld32(tacc + lane_base + 64 * j, v);
-      ptx::tmem_ld32(tacc + lane_base + 64 * j + 32, v + 32);
+      // the row in two halves of 32 columns (registers), the half that
+      // holds the diagonal first: its ||k_r||^2 gives beta_r
+      const int hd = r >> 5;
+      float v[32];
+      ptx::tmem_ld32(tacc + lane_base + 64 * j + 32 * hd, v);
       float nn2 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) nn2 = (c == r) ? v[c] : nn2;
+      for (int c = 0; c < 32; ++c) nn2 = (c == (r & 31)) ? v[c] : nn2;
       const float beta = step_size(er, nn2, eps);
-      // A_rs = beta_r (k_r . k_s) e^{G_r - G_s}: per 16-column block, the
-      // decay at its last column s0 < r from one exponential (<= 1), then
-      // running products of alpha_i (each <= 1) down the block; the four
-      // blocks are independent chains
       const float Gr = s.G[j][r];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int s0 = min(16 * q + 15, r - 1);
-        float d = s0 >= 16 * q ? __expf(Gr - s.G[j][s0]) : 0.f;
-#pragma unroll
-        for (int c = 16 * q + 15; c >= 16 * q; --c) {
-          const bool on = c < r;
-          d = (on && c < s0) ? d * s.alpha[j][c + 1] : d;
-          v[c] = on ? beta * v[c] * d : 0.f;
-        }
-      }
-      // diagonal block part (fp32) and the blocks left of it (bf16)
       float* adr = &s.ad[j][bb][r & 15][0];
-#define KLA_UT_DIAG(B_)                                      \
-  if (bb == B_) {                                            \
-    _Pragma("unroll") for (int i = 0; i < 16; ++i) adr[i] = v[16 * B_ + i]; \
-  }
-      KLA_UT_DIAG(0) else KLA_UT_DIAG(1) else KLA_UT_DIAG(2) else KLA_UT_DIAG(3)
-#undef KLA_UT_DIAG
       __nv_bfloat16* arow = &s.a[j][r][0];
 #pragma unroll
-      for (int q = 0; q < 6; ++q) {
-        if (q < 2 * bb) {
-          uint4 u;
-          u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-          u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-          u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-          u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-          *reinterpret_cast<uint4*>(arow + 8 * q) = u;
+      for (int pass = 0; pass < 2; ++pass) {
+        const int h = pass == 0 ? hd : 1 - hd;
+        if (pass == 1) ptx::tmem_ld32(tacc + lane_base + 64 * j + 32 * h, v);
+        // A_rs = beta_r (k_r . k_s) e^{G_r - G_s}: per 16-column block, the
+        // decay at its last column s0 < r from one exponential (<= 1), then
+        // running products of alpha_i (each <= 1) down the block; the
+        // blocks are independent chains
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const int q = 2 * h + qq;
+          const int s0 = min(16 * q + 15, r - 1);
+          float d = s0 >= 16 * q ? __expf(Gr - s.G[j][s0]) : 0.f;
+#pragma unroll
+          for (int i = 15; i >= 0; --i) {
+            const int c = 16 * q + i;
+            const bool on = c < r;
+            d = (on && c < s0) ? d * s.alpha[j][c + 1] : d;
+            v[16 * qq + i] = on ? beta * v[16 * qq + i] * d : 0.f;
+          }
+          // my diagonal block (fp32) ...
+          if (q == bb) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) adr[i] = v[16 * qq + i];
+          }
+        }
+        // ... and the blocks left of it (bf16, 8 columns per store)
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          if (4 * h + q8 < 2 * bb) {
+            uint4 u;
+            u.x = pack_bf16x2(v[8 * q8 + 0], v[8 * q8 + 1]);
+            u.y = pack_bf16x2(v[8 * q8 + 2], v[8 * q8 + 3]);
+            u.z = pack_bf16x2(v[8 * q8 + 4], v[8 * q8 + 5]);
+            u.w = pack_bf16x2(v[8 * q8 + 6], v[8 * q8 + 7]);
+            *reinterpret_cast<uint4*>(arow + 8 * (4 * h + q8)) = u;
+          }
         }
       }
       s.b1[j][r] = beta;
@@ -345,7 +369,8 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
     ptx::tc_fence_before();
     nbar_sync(bar_id);
 
-    uint8_t* dst = ws + (size_t)ci * kUtTileBytes;  // T'^T, then T''^T
+    // this chunk's output tiles T'^T, then T''^T, assembled in shared memory
+    uint8_t* dst = s.keys + j * (int)kUtTileBytes;
     // ---- D_b = (I + A_bb)^{-1}: thread (j, b, c) solves column c; it is row
     // m = 16 b + c of Y's diagonal block, written straight to the outputs
     {
@@ -465,25 +490,38 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
         }
       }
     }
-    if (nmajor) {
-      // every thread's factor stores are visible (to the bulk copies of the
-      // state CTAs too) before the pair's flags are raised
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      nbar_sync(bar_id);
-      if (tid == 0) {
-        __threadfence();
-        for (int jj = 0; jj < 2; ++jj) {
+    // the assembled tiles leave with one bulk store per chunk; once the
+    // stores have read them, the next pair's keys may land in their place
+    ptx::fence_proxy_async_smem();
+    nbar_sync(bar_id);
+    if (tid == 0) {
+      for (int jj = 0; jj < 2; ++jj) {
+        if (2 * pair + jj < total_chunks) {
           int hd, nn;
-          if (2 * pair + jj < total_chunks) {
-            chunk_of(2 * pair + jj, hd, nn);
-            atomicExch(flags + (size_t)hd * nchunks + nn, 1u);
-          }
+          chunk_of(2 * pair + jj, hd, nn);
+          ptx::bulk_store(ws + ((size_t)hd * nchunks + nn) * kUtTileBytes,
+                          s.keys + jj * (int)kUtTileBytes, (uint32_t)kUtTileBytes);
         }
+      }
+      ptx::bulk_commit();
+      if (nmajor) flag_pair = pair;
+      ptx::bulk_wait_group_read<0>();
+      if (pair + pair_stride < npairs) {
+        load_keys(pair + pair_stride);
+        keys_in_flight = true;
       }
     }
     gr = gn;
     er = en;
   }  // pair loop
+  if (tid == 0) {
+    ptx::bulk_wait_group_all();  // every factor tile has landed
+    if (nmajor && flag_pair >= 0 && ok) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __threadfence();
+      publish(flag_pair);
+    }
+  }
   if (!ok) report_timeout(err);
   if constexpr (CHECK) {
     if (worst > 0.f) atomic_max_nonneg(ratio_max, worst);

@@ -266,14 +266,15 @@ KLA_API kla_status kla_gdn_decode_step(const void *q, const void *k, const void 
 /*
  * The per-channel-gate prefill as chunks (arguments as kla_kda_fwd plus
  * chunk = KLA_CHUNK and a workspace of kla_kda_chunk_fwd_workspace_size(...)
- * bytes, 16-byte aligned; as for kla_chunk_fwd, one holding only the
- * per-chunk factors, B * H * ceil(T / 64) * (16 KiB + 24 KiB * dk / 64 +
- * 1 KiB), is accepted and runs the state chain uncut).  bf16: a CUDA-core
- * kernel forms every chunk's factors in fp32 -- A and P summed channel by
- * channel with one e^{G_ri - G_si} <= 1 per term, T = (I + A)^{-1}, W,
- * Q o e^G, K o e^{G_last - G} -- and the tcgen05 chain kernel carries the
- * state; fp32: the token-serial kernel (no workspace needed).  The
- * workspace must not overlap any other argument.
+ * bytes, 16-byte aligned: the per-chunk factors, B * H * ceil(T / 64) *
+ * (16 KiB + 24 KiB * dk / 64 + 1 KiB), validated but at present not used).
+ * Both I/O types currently run the token-serial per-channel kernel (exact
+ * fp32 evaluation): the chunk kernels of this form -- a CUDA-core kernel
+ * forming every chunk's factors (A and P summed channel by channel with one
+ * e^{G_ri - G_si} <= 1 per term, T = (I + A)^{-1}, W, Q o e^G,
+ * K o e^{G_last - G}) and the tcgen05 chain kernel carrying the state --
+ * raised intermittent faults whose cause has not been found, and stay
+ * unused until it is.  The workspace must not overlap any other argument.
  */
 KLA_API size_t kla_kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int dtype);
 KLA_API kla_status kla_kda_chunk_fwd(const void *q, const void *k, const void *v,

@@ -178,22 +178,26 @@ def _flag_bytes(B, T, H):
 
 
 def test_workspace_query(lib):
-    # the 0.4B-scale layer: uncut chain in a single launch, the factors and
-    # one ready flag per chunk
-    assert lib.kla_chunk_fwd_workspace_size(8, 4096, 8, 128, 128, 0) == (
-        _ut_bytes(8, 4096, 8) + _flag_bytes(8, 4096, 8))
-    # more state CTAs than leave room for UT CTAs beside them: two launches,
-    # factors only
+    # a short batch: uncut chain in a single launch, the factors and one
+    # ready flag per chunk
+    assert lib.kla_chunk_fwd_workspace_size(2, 1000, 4, 128, 128, 0) == (
+        _ut_bytes(2, 1000, 4) + _flag_bytes(2, 1000, 4))
+    # the 0.4B-scale layer: its factors take the UT lanes of the 20 SMs the
+    # state CTAs leave longer than the UT kernel on all SMs plus the chain:
+    # two launches, factors only
+    assert lib.kla_chunk_fwd_workspace_size(8, 4096, 8, 128, 128, 0) == _ut_bytes(8, 4096, 8)
+    # more state CTAs than leave room for UT CTAs beside them: two launches
     assert lib.kla_chunk_fwd_workspace_size(16, 4096, 8, 128, 128, 0) == _ut_bytes(16, 4096, 8)
     # which shapes take the single launch (the full workspace; a workspace of
     # the factors alone always runs two launches)
     full = lambda *a: lib.kla_chunk_fwd_workspace_size(*a, 128, 128, 0)
-    assert lib.kla_chunk_fwd_single_launch(8, 4096, 8, 128, 128, 0, full(8, 4096, 8)) == 1
-    assert lib.kla_chunk_fwd_single_launch(8, 4096, 8, 128, 128, 0, _ut_bytes(8, 4096, 8)) == 0
+    assert lib.kla_chunk_fwd_single_launch(2, 1000, 4, 128, 128, 0, full(2, 1000, 4)) == 1
+    assert lib.kla_chunk_fwd_single_launch(2, 1000, 4, 128, 128, 0, _ut_bytes(2, 1000, 4)) == 0
+    assert lib.kla_chunk_fwd_single_launch(8, 4096, 8, 128, 128, 0, 1 << 40) == 0
     assert lib.kla_chunk_fwd_single_launch(16, 4096, 8, 128, 128, 0, 1 << 40) == 0
     assert lib.kla_chunk_fwd_single_launch(1, 65536, 16, 128, 128, 0, 1 << 40) == 0  # cut
-    assert lib.kla_chunk_fwd_single_launch(4, 8192, 32, 64, 64, 0, 1 << 40) == 1  # stress
-    assert lib.kla_chunk_fwd_single_launch(4, 8192, 32, 64, 64, 1, 1 << 40) == 0  # fp32 I/O
+    assert lib.kla_chunk_fwd_single_launch(2, 777, 8, 64, 64, 0, 1 << 40) == 1
+    assert lib.kla_chunk_fwd_single_launch(2, 777, 8, 64, 64, 1, 1 << 40) == 0  # fp32 I/O
     # few heads and a long sequence: per-segment states (E, start state,
     # transition) follow the factors, for between 2 and 64 segments
     n = lib.kla_chunk_fwd_workspace_size(1, 65536, 16, 128, 128, 0)

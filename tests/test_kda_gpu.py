@@ -177,10 +177,14 @@ def test_kda_chunk_beta_given_and_fp32():
     assert rel(o2.cpu(), o2_ref) < TOL["fp32"] and rel(h2.cpu(), h2_ref) < TOL["fp32"]
 
 
-def test_kda_chunk_segmented_chain():
-    """Few heads, long sequence: the cut state chain in the per-channel form."""
+def test_kda_chunk_few_heads_long_sequence():
+    """Few heads, long sequence (a shape the scalar-gate chain cuts into
+    segments): the per-channel form runs its chain uncut, and its workspace
+    holds the per-chunk tiles only."""
     w, x = _prefill_inputs("prefill_4k", 1, 4000, 2, "bf16", 99, with_h0=True)
     assert api.chunk_fwd_segments(1, 4000, 2, w.dk, w.dv) > 1
+    tiles = 1 * 2 * ((4000 + 63) // 64) * (16384 + 3 * 2 * 8192 + 1024)
+    assert api.kda_chunk_fwd_workspace_size(1, 4000, 2, w.dk, w.dv) == tiles
     xc = cuda(x)
     o, hT = api.kda_chunk_fwd(xc["q"], xc["k"], xc["v"], xc["gv"], xc["eta"], x["eps"],
                               xc["h0"])

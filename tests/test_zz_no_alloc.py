@@ -17,7 +17,7 @@ import torch
 
 import oracle
 from delta_rule_linear_kla_b200 import _native, api, inputs
-from helpers import assert_parity
+from helpers import assert_parity, assert_state_parity
 
 OK, UNSUPPORTED = 0, 2
 MAX_CHUNKS = 1024
@@ -51,8 +51,8 @@ def _run_twice(w_of_seed, expect_cut):
         assert torch.equal(o, o_ref) and torch.equal(hT, h_ref)
         o64, h64 = oracle.forward(xh["q"], xh["k"], xh["v"], xh["g"], xh["eta"], xh["eps"],
                                   xh["h0"])
-        assert_parity(o.cpu(), o64, "bf16", chunks=True)
-        assert_parity(hT.cpu(), h64, "bf16", per_head=False)
+        assert_parity(o.cpu(), o64, "bf16")
+        assert_state_parity(hT.cpu(), h64, "bf16")
 
 
 @pytest.mark.gpu
@@ -85,7 +85,7 @@ def test_noalloc_fp32_has_no_chunk_limit():
     o64, h64 = oracle.forward(xh["q"], xh["k"], xh["v"], xh["g"], xh["eta"], xh["eps"],
                               xh["h0"])
     assert_parity(o.cpu(), o64, "fp32")
-    assert_parity(hT.cpu(), h64, "fp32", per_head=False)
+    assert_state_parity(hT.cpu(), h64, "fp32")
 
 
 def test_noalloc_rejects_more_chunks_than_its_scratch():
