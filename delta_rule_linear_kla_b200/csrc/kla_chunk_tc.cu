@@ -57,6 +57,7 @@
 // error word, stops all roles, drains its own TMA loads and MMAs and frees
 // TMEM.
 #include <algorithm>
+#include <type_traits>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -131,12 +132,15 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
   }
 }
 
-// The same wait taken by a whole warp that then runs warp-collective
-// instructions (elect.sync, tcgen05.ld, __syncwarp): every lane waits, and
-// if any lane gives up, all of them do, so the warp never splits.
+// The same wait taken by every lane of a warp that then runs
+// warp-collective instructions (elect.sync, tcgen05.ld, __syncwarp).  The
+// lanes poll together and read the same barrier, abort flag and clock, so
+// they leave together; a vote on the result (to keep a warp whole even if
+// its lanes disagreed after a timeout) cost 5 % of the 4K prefill's state
+// kernel and is not taken.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag));
+  return wait_or_abort(bar, parity, abort_flag);
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -304,7 +308,19 @@ __device__ __forceinline__ void chain_body(
         issued = n + 1;
         if (n + 2 < nchunks) {  // warm L2 two chunks ahead of the loads
           const int m = n + 2;
-          if (!flags) ptx::bulk_prefetch_l2(ws_head + (size_t)m * TILE, TILE);
+          // the factors only once they exist (single launch: flagged
+          // already; a chunk not yet flagged is not waited for here)
+          bool made = !flags;
+          if (!made) {
+            unsigned int f;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];"
+                         : "=r"(f)
+                         : "l"(flags + head * (size_t)nchunks_all + n0 + m)
+                         : "memory");
+            made = f != 0u;
+            if (made) asm volatile("fence.proxy.async.global;" ::: "memory");
+          }
+          if (made) ptx::bulk_prefetch_l2(ws_head + (size_t)m * TILE, TILE);
           if constexpr (!KDA) {
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
@@ -771,17 +787,32 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     return;
   }
   constexpr int LANES = fused_ut_lanes<DK>();
+  static_assert(LANES == 3, "one call per lane below");
   const int lane_id = (int)threadIdx.x >> 7;
   if (lane_id >= LANES) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  auto& us = *reinterpret_cast<utb::UtSmem<DK>*>(base + lane_id * sizeof(utb::UtSmem<DK>));
-  const int total = (n_chain / (DV / BV)) * nchunks;  // chain CTAs cover every head once
+  const int BH = n_chain / (DV / BV);  // chain CTAs cover every head once
   const int nlanes = ((int)gridDim.x - n_chain) * LANES;
-  utb::ut_run<DK, false>(&tm_k, g, eta, eps, ws, T, H, nchunks, total, err, nullptr, flags, us,
-                         (int)threadIdx.x & 127, 1 + lane_id,
-                         ((int)blockIdx.x - n_chain) * LANES + lane_id, nlanes, false);
+  // every chunk of every head, n-major.  Each lane's shared memory sits at a
+  // compile-time offset (one inlined copy of the lane per lane index): with
+  // the offset taken at run time the lane code does not fit in the 128
+  // registers a thread of this launch has and spills.
+  auto run = [&](auto lane_c) {
+    constexpr int L = decltype(lane_c)::value;
+    auto& us = *reinterpret_cast<utb::UtSmem<DK>*>(base + L * sizeof(utb::UtSmem<DK>));
+    utb::ut_run<DK, false>(&tm_k, g, eta, eps, ws, T, H, nchunks, BH, 0, BH * nchunks, true,
+                           err, nullptr, flags, us,
+                           (int)threadIdx.x & 127, 1 + L,
+                           ((int)blockIdx.x - n_chain) * LANES + L, nlanes, false);
+  };
+  if (lane_id == 0)
+    run(std::integral_constant<int, 0>());
+  else if (lane_id == 1)
+    run(std::integral_constant<int, 1>());
+  else
+    run(std::integral_constant<int, 2>());
 }
 
 // ------------------------------------------------------------------ host

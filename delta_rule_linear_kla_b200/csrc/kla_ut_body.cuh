@@ -25,12 +25,17 @@
 //   1. the Gram matrices of both chunks as one tcgen05 MMA, [K0; K1][K0; K1]^T
 //      (M = N = 128, bf16, fp32 in TMEM; the two 64 x 64 diagonal blocks are
 //      the chunks' Gram matrices); their diagonals give ||k||^2 and beta;
-//   2. thread t holds row t: it forms row r of A with the decay e^{G_r - G_s}
-//      as a running product of alpha_j = e^{g_j} over s < j <= r (every
-//      factor <= 1) and stores the blocks left of its diagonal block (bf16)
-//      and its part of the diagonal block (fp32);
+//   2. thread t holds row t: it forms row r of A and stores the blocks left
+//      of its diagonal block (bf16) and its part of the diagonal block (fp32,
+//      transposed).  The decay e^{G_r - G_s} (s < r, so <= 1) is one
+//      exponential per entry in the 32 columns that hold the diagonal; in a
+//      16-column block q wholly left of row r it is the product of
+//      e^{G_r - G_{16q+15}} and E_s = e^{G_{16q+15} - G_s}, both <= 1, with
+//      E tabulated once per chunk.  A warp holds 32 rows of one chunk, so the
+//      half-row test is uniform over it: rows 0..31 touch columns 0..31 only;
 //   3. thread (chunk, b, c) solves column c of D_b by forward substitution
-//      (fp32) and writes the diagonal block of the outputs;
+//      (fp32, reading the transposed diagonal block four entries at a time)
+//      and writes the diagonal block of the outputs;
 //   4. warp (chunk, half) forms the off-diagonal row blocks Y_cb with
 //      warp-level bf16 products (mma.sync m16n8k16, fp32 sums): the fp32
 //      accumulators of one product are, packed to bf16, the left operand of
@@ -85,8 +90,10 @@ struct alignas(1024) UtSmem {
   uint8_t keys[KEYS_BYTES];
   __nv_bfloat16 a[2][C][AROW];       // A left of the diagonal blocks, bf16, row-major
   __nv_bfloat16 dt[2][4][16][DROW];  // D_b^T (row c = column c of D_b), bf16
-  float ad[2][4][16][17];            // diagonal blocks of A, fp32 ([row][column], padded)
-  float G[2][C], alpha[2][C], eta[2][C], n2[2][C];
+  // diagonal blocks of A, fp32, transposed: entry (row i, column m) of block
+  // b at [b][16 m + i]; 272-float block pitch (16 banks apart)
+  alignas(16) float adt[2][4][272];
+  float G[2][C], E[2][C], eta[2][C], n2[2][C];  // E_s = e^{G_{s | 15} - G_s}
   float b1[2][C], b2[2][C];          // beta, beta e^G
   uint64_t bar_tma, bar_mma;
   uint32_t tmem_base;
@@ -156,17 +163,19 @@ __device__ __forceinline__ bool nbar_and(int id, bool v) {
 // One UT "lane": 128 threads (tid 0..127, TMEM lanes 0..127 of their own
 // 128-column allocation) that own the shared memory `s` and synchronise on
 // named barrier `bar_id` only.  It takes pairs first_pair, first_pair +
-// pair_stride, ... of the chunk order: chunk-major within each head when
-// `flags` is null (the stand-alone kernel), else chunk index n major over all
-// heads (n = 0 of every head first), publishing flags[head * nchunks + n] =
-// 1 once a chunk's factors are in memory (for state CTAs of the same launch
-// that wait on them).  `standalone`: the lane is the whole CTA (it may
-// relinquish the TMEM allocation permit).
+// pair_stride, ... of the `count` chunks p0, p0 + 1, ... of a chunk order
+// over the BH heads: chunk-major within each head, or (nmajor) chunk index n
+// major over all heads (n = 0 of every head first).  With `flags` it raises
+// flags[head * nchunks + n] = 1 once a chunk's factors are in memory (for
+// state CTAs of the same launch that wait on them; needs nmajor).
+// `standalone`: the lane is the whole CTA (it may relinquish the TMEM
+// allocation permit).
 template <int DK, bool CHECK>
 __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __restrict__ g,
                                        const float* __restrict__ eta, float eps,
                                        uint8_t* __restrict__ ws, int T, int H, int nchunks,
-                                       int total_chunks, unsigned int* err, float* ratio_max,
+                                       int BH, int p0, int total_chunks, bool nmajor,
+                                       unsigned int* err, float* ratio_max,
                                        unsigned int* flags, UtSmem<DK>& s, const int tid,
                                        const int bar_id, const int first_pair,
                                        const int pair_stride, const bool standalone) {
@@ -175,10 +184,9 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
   const int j = tid >> 6, r = tid & 63;  // chunk slot and its row
   const int npairs = (total_chunks + 1) / 2;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const int BH = total_chunks / nchunks;
-  const bool nmajor = flags != nullptr;
-  // processing index -> (head, chunk)
+  // processing index (0 .. total_chunks - 1) -> (head, chunk)
   auto chunk_of = [&](int p, int& hd, int& nn) {
+    p += p0;
     if (nmajor) {
       nn = p / BH;
       hd = p - nn * BH;
@@ -268,7 +276,9 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       if (lane >= off) gs += y;
     }
     s.G[j][r] = gs;
-    s.alpha[j][r] = __expf(gr);
+    // s and s | 15 lie in the same warp: the difference of the warp's
+    // partial sums is G_{s | 15} - G_s (<= 0)
+    s.E[j][r] = __expf(__shfl_sync(0xffffffffu, gs, lane | 15) - gs);
     s.eta[j][r] = er;
     nbar_sync(bar_id);
     const float G31 = s.G[j][31];  // row 31 is not rewritten below
@@ -293,7 +303,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
         ptx::mma_commit(&s.bar_mma);
         ok = wait_bounded(&s.bar_mma, mma_phase);
         // the previous pair's factors have landed by now: raise its flags
-        if (nmajor && flag_pair >= 0) {
+        if (flags && flag_pair >= 0) {
           ptx::bulk_wait_group_all();
           asm volatile("fence.proxy.async.global;" ::: "memory");
           __threadfence();
@@ -311,9 +321,8 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
     // row r of A
     const int bb = r >> 4;  // my 16-row block
     {
-      // the row in two halves of 32 columns (registers), the half that
-      // holds the diagonal first: its ||k_r||^2 gives beta_r
-      const int hd = r >> 5;
+      // hd: the 32-column half that holds the diagonal (warp-uniform)
+      const int hd = warp & 1;
       float v[32];
       ptx::tmem_ld32(tacc + lane_base + 64 * j + 32 * hd, v);
       float nn2 = 0.f;
@@ -321,35 +330,25 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       for (int c = 0; c < 32; ++c) nn2 = (c == (r & 31)) ? v[c] : nn2;
       const float beta = step_size(er, nn2, eps);
       const float Gr = s.G[j][r];
-      float* adr = &s.ad[j][bb][r & 15][0];
       __nv_bfloat16* arow = &s.a[j][r][0];
+      // A_rs = beta_r (k_r . k_s) e^{G_r - G_s} for s < r: the diagonal half,
+      // one exponential per entry (its argument is <= 0 for s < r; the
+      // entries s >= r are discarded by the select)
 #pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        const int h = pass == 0 ? hd : 1 - hd;
-        if (pass == 1) ptx::tmem_ld32(tacc + lane_base + 64 * j + 32 * h, v);
-        // A_rs = beta_r (k_r . k_s) e^{G_r - G_s}: per 16-column block, the
-        // decay at its last column s0 < r from one exponential (<= 1), then
-        // running products of alpha_i (each <= 1) down the block; the
-        // blocks are independent chains
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = 2 * hd + qq;
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int q = 2 * h + qq;
-          const int s0 = min(16 * q + 15, r - 1);
-          float d = s0 >= 16 * q ? __expf(Gr - s.G[j][s0]) : 0.f;
-#pragma unroll
-          for (int i = 15; i >= 0; --i) {
-            const int c = 16 * q + i;
-            const bool on = c < r;
-            d = (on && c < s0) ? d * s.alpha[j][c + 1] : d;
-            v[16 * qq + i] = on ? beta * v[16 * qq + i] * d : 0.f;
-          }
-          // my diagonal block (fp32) ...
-          if (q == bb) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) adr[i] = v[16 * qq + i];
-          }
+        for (int i = 0; i < 16; ++i) {
+          const int c = 16 * q + i;
+          const float d = __expf(Gr - s.G[j][c]);
+          v[16 * qq + i] = c < r ? beta * v[16 * qq + i] * d : 0.f;
         }
-        // ... and the blocks left of it (bf16, 8 columns per store)
+        if (q == bb) {  // my row of the diagonal block, as a column of adt
+#pragma unroll
+          for (int i = 0; i < 16; ++i) s.adt[j][bb][16 * i + (r & 15)] = v[16 * qq + i];
+        }
+      }
+      auto store_bf16 = [&](int h) {  // the blocks of half h left of block bb
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           if (4 * h + q8 < 2 * bb) {
@@ -361,6 +360,19 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
             *reinterpret_cast<uint4*>(arow + 8 * (4 * h + q8)) = u;
           }
         }
+      };
+      store_bf16(hd);
+      if (hd == 1) {
+        // columns 0..31 lie wholly left of rows 32..63:
+        // e^{G_r - G_s} = e^{G_r - G_{16q+15}} E_s, both factors <= 1
+        ptx::tmem_ld32(tacc + lane_base + 64 * j, v);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float f = beta * __expf(Gr - s.G[j][16 * q + 15]);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[16 * q + i] *= f * s.E[j][16 * q + i];
+        }
+        store_bf16(0);
       }
       s.b1[j][r] = beta;
       s.b2[j][r] = beta * __expf(s.G[j][r]);
@@ -382,8 +394,15 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
 #pragma unroll
       for (int mm = 0; mm < 15; ++mm) {
+        const float* col = &s.adt[j][b][16 * mm];  // column mm of A_bb
 #pragma unroll
-        for (int i = mm + 1; i < 16; ++i) x[i] = fmaf(-s.ad[j][b][i][mm], x[mm], x[i]);
+        for (int i4 = (mm + 1) / 4; i4 < 4; ++i4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(col + 4 * i4);
+          const float ae[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (4 * i4 + e > mm) x[4 * i4 + e] = fmaf(-ae[e], x[mm], x[4 * i4 + e]);
+        }
       }
       uint4 lo, hi;
       lo.x = pack_bf16x2(x[0], x[1]);   lo.y = pack_bf16x2(x[2], x[3]);
@@ -504,7 +523,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
         }
       }
       ptx::bulk_commit();
-      if (nmajor) flag_pair = pair;
+      if (flags) flag_pair = pair;
       ptx::bulk_wait_group_read<0>();
       if (pair + pair_stride < npairs) {
         load_keys(pair + pair_stride);
@@ -516,7 +535,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
   }  // pair loop
   if (tid == 0) {
     ptx::bulk_wait_group_all();  // every factor tile has landed
-    if (nmajor && flag_pair >= 0 && ok) {
+    if (flags && flag_pair >= 0 && ok) {
       asm volatile("fence.proxy.async.global;" ::: "memory");
       __threadfence();
       publish(flag_pair);

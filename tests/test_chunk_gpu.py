@@ -272,3 +272,4 @@ def test_single_launch_equals_two_launches(name, B, T, H):
                                                      device="cuda"))
         api.check_device_error()
         assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
