@@ -43,12 +43,16 @@
 // Rounding the products' operands to bf16 moves the outputs no more than the
 // bf16 rounding of T' and T'' themselves (a CPU simulation of this exact
 // scheme on the stress and 0.4B-layer distributions gives the same error as
-// rounding the exact factors).  The next pair's keys are loaded as soon as
-// the Gram MMA has read them, so the load overlaps steps 2 to 4.
+// rounding the exact factors).  Once the Gram MMA has read the keys, their
+// shared memory holds A and its diagonal blocks (steps 2 to 4); the next
+// pair's keys are loaded when step 4 is done.  That keeps a lane at ~42 KB
+// of shared memory and 128 registers, so four lanes share an SM: the phases
+// are short dependent chains separated by barriers, and more lanes per SM
+// hide more of their latency.
 //
-// The factors are written to global memory already in the 128-byte swizzled
-// bf16 layout the chain kernel's MMAs read (as MN-major A operands), so it
-// fetches them with one bulk copy per chunk.
+// The factors are written to global memory (16- and 4-byte stores) already
+// in the 128-byte swizzled bf16 layout the chain kernel's MMAs read (as
+// MN-major A operands), so it fetches them with one bulk copy per chunk.
 //
 // Debug bound check (CHECK): for eta in [0, 2] every factor
 // (I - beta_j k_j k_j^T) of the chunk's transition has norm <= 1, and then
@@ -77,22 +81,24 @@ constexpr float kBoundSlack = 1.25f;     // allowance for the factors' own round
 
 template <int DK>
 constexpr int ctas_per_sm() {
-  return 3;
+  return 4;
 }
 
 template <int DK>
 struct alignas(1024) UtSmem {
   static constexpr int NP = DK / 64;
-  // [K0; K1] per 64-column panel (TMA, 128-byte swizzle); once the Gram MMA
-  // has read them, the pair's two output tiles (16 KB each) are assembled
-  // here and leave with one bulk store per chunk
-  static constexpr int KEYS_BYTES = NP * TILE > 2 * 16384 ? NP * TILE : 2 * 16384;
-  uint8_t keys[KEYS_BYTES];
-  __nv_bfloat16 a[2][C][AROW];       // A left of the diagonal blocks, bf16, row-major
+  // A of both chunks, in the keys' bytes once the Gram MMA has read them
+  struct Work {
+    __nv_bfloat16 a[2][C][AROW];  // A left of the diagonal blocks, bf16, row-major
+    // diagonal blocks of A, fp32, transposed: entry (row i, column m) of
+    // block b at [b][16 m + i]; 272-float block pitch (16 banks apart)
+    alignas(16) float adt[2][4][272];
+  };
+  union {
+    uint8_t keys[NP * TILE];  // [K0; K1] per 64-column panel (TMA, 128-byte swizzle)
+    Work w;
+  };
   __nv_bfloat16 dt[2][4][16][DROW];  // D_b^T (row c = column c of D_b), bf16
-  // diagonal blocks of A, fp32, transposed: entry (row i, column m) of block
-  // b at [b][16 m + i]; 272-float block pitch (16 banks apart)
-  alignas(16) float adt[2][4][272];
   float G[2][C], E[2][C], eta[2][C], n2[2][C];  // E_s = e^{G_{s | 15} - G_s}
   float b1[2][C], b2[2][C];          // beta, beta e^G
   uint64_t bar_tma, bar_mma;
@@ -247,9 +253,8 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
   bool ok = true;
   uint32_t mma_phase = 0, tma_phase = 0;
   bool keys_in_flight = tid == 0 && first_pair < npairs;
-  int flag_pair = -1;  // pair whose factors were stored but not yet flagged
-  // raise the ready flags of both chunks of pair `pr` (after their stores
-  // completed and a fence)
+  // raise the ready flags of both chunks of pair `pr` (after every thread's
+  // stores of its factors and a fence)
   auto publish = [&](int pr) {
     for (int jj = 0; jj < 2; ++jj) {
       if (2 * pr + jj < total_chunks) {
@@ -302,14 +307,6 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
         }
         ptx::mma_commit(&s.bar_mma);
         ok = wait_bounded(&s.bar_mma, mma_phase);
-        // the previous pair's factors have landed by now: raise its flags
-        if (flags && flag_pair >= 0) {
-          ptx::bulk_wait_group_all();
-          asm volatile("fence.proxy.async.global;" ::: "memory");
-          __threadfence();
-          publish(flag_pair);
-          flag_pair = -1;
-        }
       }
     }
     mma_phase ^= 1u;
@@ -330,7 +327,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       for (int c = 0; c < 32; ++c) nn2 = (c == (r & 31)) ? v[c] : nn2;
       const float beta = step_size(er, nn2, eps);
       const float Gr = s.G[j][r];
-      __nv_bfloat16* arow = &s.a[j][r][0];
+      __nv_bfloat16* arow = &s.w.a[j][r][0];
       // A_rs = beta_r (k_r . k_s) e^{G_r - G_s} for s < r: the diagonal half,
       // one exponential per entry (its argument is <= 0 for s < r; the
       // entries s >= r are discarded by the select)
@@ -345,7 +342,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
         }
         if (q == bb) {  // my row of the diagonal block, as a column of adt
 #pragma unroll
-          for (int i = 0; i < 16; ++i) s.adt[j][bb][16 * i + (r & 15)] = v[16 * qq + i];
+          for (int i = 0; i < 16; ++i) s.w.adt[j][bb][16 * i + (r & 15)] = v[16 * qq + i];
         }
       }
       auto store_bf16 = [&](int h) {  // the blocks of half h left of block bb
@@ -381,8 +378,13 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
     ptx::tc_fence_before();
     nbar_sync(bar_id);
 
-    // this chunk's output tiles T'^T, then T''^T, assembled in shared memory
-    uint8_t* dst = s.keys + j * (int)kUtTileBytes;
+    // this chunk's factor tile in the workspace: T'^T, then T''^T
+    uint8_t* dst = ws;
+    if (valid) {
+      int hd, nn;
+      chunk_of(2 * pair + j, hd, nn);
+      dst = ws + ((size_t)hd * nchunks + nn) * kUtTileBytes;
+    }
     // ---- D_b = (I + A_bb)^{-1}: thread (j, b, c) solves column c; it is row
     // m = 16 b + c of Y's diagonal block, written straight to the outputs
     {
@@ -394,7 +396,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
 #pragma unroll
       for (int mm = 0; mm < 15; ++mm) {
-        const float* col = &s.adt[j][b][16 * mm];  // column mm of A_bb
+        const float* col = &s.w.adt[j][b][16 * mm];  // column mm of A_bb
 #pragma unroll
         for (int i4 = (mm + 1) / 4; i4 < 4; ++i4) {
           const float4 a4 = *reinterpret_cast<const float4*>(col + 4 * i4);
@@ -466,7 +468,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
             // A_{b,jj}^T as the B operand: rows 16 b + 8 h + (0..7) of A,
             // columns 16 jj + (0..15)
             uint32_t bf[4];
-            ldsm_x4(bf, &s.a[j][16 * b + (g8 >> 1) * 8 + l8][16 * jj + (g8 & 1) * 8]);
+            ldsm_x4(bf, &s.w.a[j][16 * b + (g8 >> 1) * 8 + l8][16 * jj + (g8 & 1) * 8]);
             mma16816(acc[0], y[jj], bf[0], bf[1]);
             mma16816(acc[1], y[jj], bf[2], bf[3]);
           }
@@ -509,22 +511,17 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
         }
       }
     }
-    // the assembled tiles leave with one bulk store per chunk; once the
-    // stores have read them, the next pair's keys may land in their place
+    // every thread's factor stores are visible GPU-wide before the flags go
+    // up; A and its blocks have been read, so the next pair's keys may land
+    // in their place
+    if (flags) __threadfence();
     ptx::fence_proxy_async_smem();
     nbar_sync(bar_id);
     if (tid == 0) {
-      for (int jj = 0; jj < 2; ++jj) {
-        if (2 * pair + jj < total_chunks) {
-          int hd, nn;
-          chunk_of(2 * pair + jj, hd, nn);
-          ptx::bulk_store(ws + ((size_t)hd * nchunks + nn) * kUtTileBytes,
-                          s.keys + jj * (int)kUtTileBytes, (uint32_t)kUtTileBytes);
-        }
+      if (flags && ok) {
+        __threadfence();
+        publish(pair);
       }
-      ptx::bulk_commit();
-      if (flags) flag_pair = pair;
-      ptx::bulk_wait_group_read<0>();
       if (pair + pair_stride < npairs) {
         load_keys(pair + pair_stride);
         keys_in_flight = true;
@@ -533,14 +530,6 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
     gr = gn;
     er = en;
   }  // pair loop
-  if (tid == 0) {
-    ptx::bulk_wait_group_all();  // every factor tile has landed
-    if (flags && flag_pair >= 0 && ok) {
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      __threadfence();
-      publish(flag_pair);
-    }
-  }
   if (!ok) report_timeout(err);
   if constexpr (CHECK) {
     if (worst > 0.f) atomic_max_nonneg(ratio_max, worst);
