@@ -788,6 +788,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
   constexpr int LANES = fused_ut_lanes<DK>();
   static_assert(LANES == 4 && LANES * 128 == NTHREADS, "one call per lane below");
+  static_assert(1 + 3 * LANES <= 16, "named barriers: one per lane, two per chunk slot");
   const int lane_id = (int)threadIdx.x >> 7;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -803,7 +804,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     auto& us = *reinterpret_cast<utb::UtSmem<DK>*>(base + L * sizeof(utb::UtSmem<DK>));
     utb::ut_run<DK, false>(&tm_k, g, eta, eps, ws, T, H, nchunks, BH, 0, BH * nchunks, true,
                            err, nullptr, flags, us,
-                           (int)threadIdx.x & 127, 1 + L,
+                           (int)threadIdx.x & 127, 1 + L, 1 + LANES + 2 * L,
                            ((int)blockIdx.x - n_chain) * LANES + L, nlanes, false);
   };
   if (lane_id == 0)

@@ -16,7 +16,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ g,
   auto& s = *reinterpret_cast<utb::UtSmem<DK>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   utb::ut_run<DK, CHECK>(&tm_k, g, eta, eps, ws, T, H, nchunks, total_chunks / nchunks, 0,
-                         total_chunks, false, err, ratio_max, nullptr, s, threadIdx.x, 1,
+                         total_chunks, false, err, ratio_max, nullptr, s, threadIdx.x, 1, 2,
                          blockIdx.x, gridDim.x, true);
 }
 

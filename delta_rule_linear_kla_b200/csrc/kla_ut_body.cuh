@@ -149,9 +149,13 @@ __device__ __forceinline__ float bound_ratio(const UtSmem<DK>& s, int j, int r, 
 }
 
 
-// Named barrier of one 128-thread lane, and its AND-reduction form.
+// Named barrier of one 128-thread lane, of the 64 threads (two warps) of
+// one chunk slot, and the lane barrier's AND-reduction form.
 __device__ __forceinline__ void nbar_sync(int id) {
   asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ void nbar_sync64(int id) {
+  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
 }
 __device__ __forceinline__ bool nbar_and(int id, bool v) {
   uint32_t out;
@@ -168,7 +172,10 @@ __device__ __forceinline__ bool nbar_and(int id, bool v) {
 
 // One UT "lane": 128 threads (tid 0..127, TMEM lanes 0..127 of their own
 // 128-column allocation) that own the shared memory `s` and synchronise on
-// named barrier `bar_id` only.  It takes pairs first_pair, first_pair +
+// named barrier `bar_id`; between the Gram product and the end of a pair the
+// two warps of chunk slot j (threads 64 j .. 64 j + 63, which alone read and
+// write that chunk's rows, blocks and outputs) synchronise on their own
+// barrier chunk_bar + j, so one chunk's phases do not wait for the other's.  It takes pairs first_pair, first_pair +
 // pair_stride, ... of the `count` chunks p0, p0 + 1, ... of a chunk order
 // over the BH heads: chunk-major within each head, or (nmajor) chunk index n
 // major over all heads (n = 0 of every head first).  With `flags` it raises
@@ -183,7 +190,8 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
                                        int BH, int p0, int total_chunks, bool nmajor,
                                        unsigned int* err, float* ratio_max,
                                        unsigned int* flags, UtSmem<DK>& s, const int tid,
-                                       const int bar_id, const int first_pair,
+                                       const int bar_id, const int chunk_bar,
+                                       const int first_pair,
                                        const int pair_stride, const bool standalone) {
   constexpr int NP = UtSmem<DK>::NP;
   const int warp = tid >> 5, lane = tid & 31;
@@ -285,7 +293,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
     // partial sums is G_{s | 15} - G_s (<= 0)
     s.E[j][r] = __expf(__shfl_sync(0xffffffffu, gs, lane | 15) - gs);
     s.eta[j][r] = er;
-    nbar_sync(bar_id);
+    nbar_sync64(chunk_bar + j);
     const float G31 = s.G[j][31];  // row 31 is not rewritten below
     if (r >= 32) s.G[j][r] = gs + G31;
     float gn, en;  // next pair's gate and relaxation
@@ -376,7 +384,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       s.n2[j][r] = nn2;
     }
     ptx::tc_fence_before();
-    nbar_sync(bar_id);
+    nbar_sync64(chunk_bar + j);
 
     // this chunk's factor tile in the workspace: T'^T, then T''^T
     uint8_t* dst = ws;
@@ -442,7 +450,7 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
         }
       }
     }
-    nbar_sync(bar_id);
+    nbar_sync64(chunk_bar + j);
 
     // ---- off-diagonal row blocks of Y = T^T: warp 2j takes row block 0,
     // warp 2j + 1 row blocks 1 and 2 (row block 3 is D_3^T alone)
