@@ -28,8 +28,8 @@
 //   2. thread t holds row t: it forms row r of A and stores the blocks left
 //      of its diagonal block (bf16) and its part of the diagonal block (fp32,
 //      transposed).  The decay e^{G_r - G_s} (s < r, so <= 1) is one
-//      exponential per entry in the 32 columns that hold the diagonal; in a
-//      16-column block q wholly left of row r it is the product of
+//      exponential per entry inside the row's own 16-column diagonal block;
+//      in a block q wholly left of row r it is the product of
 //      e^{G_r - G_{16q+15}} and E_s = e^{G_{16q+15} - G_s}, both <= 1, with
 //      E tabulated once per chunk.  A warp holds 32 rows of one chunk, so the
 //      half-row test is uniform over it: rows 0..31 touch columns 0..31 only;
@@ -337,21 +337,31 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       const float Gr = s.G[j][r];
       __nv_bfloat16* arow = &s.w.a[j][r][0];
       // A_rs = beta_r (k_r . k_s) e^{G_r - G_s} for s < r: the diagonal half,
-      // one exponential per entry (its argument is <= 0 for s < r; the
-      // entries s >= r are discarded by the select)
+      // blocks 2 hd (v[0..15]) and 2 hd + 1 (v[16..31]); lanes 0..15 of the
+      // warp have their diagonal block first, lanes 16..31 second.  The
+      // decays inside my own block, one exponential per entry (argument
+      // <= 0; zero for s >= r); a first block left of my own one takes
+      // e^{G_r - G_{32 hd + 15}} E_s (both <= 1); a second block right of
+      // my own one is zero.  Every lane runs the same instructions: the
+      // two roles are selects.
+      const bool second = (bb & 1) != 0;
+      float ev[16];
 #pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {
-        const int q = 2 * hd + qq;
+      for (int i = 0; i < 16; ++i) {
+        const int c = 16 * bb + i;
+        ev[i] = c < r ? __expf(Gr - s.G[j][c]) : 0.f;
+      }
+      // meaningful in the second block only (the select below discards it
+      // in the first, where the argument is >= 0)
+      const float fl = beta * __expf(Gr - s.G[j][32 * hd + 15]);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = 16 * q + i;
-          const float d = __expf(Gr - s.G[j][c]);
-          v[16 * qq + i] = c < r ? beta * v[16 * qq + i] * d : 0.f;
-        }
-        if (q == bb) {  // my row of the diagonal block, as a column of adt
-#pragma unroll
-          for (int i = 0; i < 16; ++i) s.w.adt[j][bb][16 * i + (r & 15)] = v[16 * qq + i];
-        }
+      for (int i = 0; i < 16; ++i) {
+        const float own0 = beta * v[i] * ev[i], left = v[i] * (fl * s.E[j][32 * hd + i]);
+        const float own1 = beta * v[16 + i] * ev[i];
+        v[i] = second ? left : own0;
+        v[16 + i] = second ? own1 : 0.f;
+        // my row of the diagonal block, as a column of adt
+        s.w.adt[j][bb][16 * i + (r & 15)] = second ? own1 : own0;
       }
       auto store_bf16 = [&](int h) {  // the blocks of half h left of block bb
 #pragma unroll
