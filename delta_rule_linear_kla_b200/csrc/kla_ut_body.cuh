@@ -34,8 +34,11 @@
 //      E tabulated once per chunk.  A warp holds 32 rows of one chunk, so the
 //      half-row test is uniform over it: rows 0..31 touch columns 0..31 only;
 //   3. thread (chunk, b, c) solves column c of D_b by forward substitution
-//      (fp32, reading the transposed diagonal block four entries at a time)
-//      and writes the diagonal block of the outputs;
+//      (fp32, reading the transposed diagonal block four entries at a time);
+//      the outputs' diagonal blocks and the zeros left of them are then
+//      written row by row, eight threads to a 128-byte row (scattered
+//      16-byte stores of one row per thread had cost a third of the
+//      kernel's time);
 //   4. warp (chunk, half) forms the off-diagonal row blocks Y_cb with
 //      warp-level bf16 products (mma.sync m16n8k16, fp32 sums): the fp32
 //      accumulators of one product are, packed to bf16, the left operand of
@@ -404,7 +407,8 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       dst = ws + ((size_t)hd * nchunks + nn) * kUtTileBytes;
     }
     // ---- D_b = (I + A_bb)^{-1}: thread (j, b, c) solves column c; it is row
-    // m = 16 b + c of Y's diagonal block, written straight to the outputs
+    // m = 16 b + c of Y's diagonal block (kept for the products below as
+    // D_b^T, and for the outputs)
     {
       const int b = (tid >> 4) & 3, c = tid & 15, m = 16 * b + c;
       // right-looking: once x_m is final, it is subtracted from every later
@@ -431,36 +435,56 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       hi.z = pack_bf16x2(x[12], x[13]); hi.w = pack_bf16x2(x[14], x[15]);
       *reinterpret_cast<uint4*>(&s.dt[j][b][c][0]) = lo;
       *reinterpret_cast<uint4*>(&s.dt[j][b][c][8]) = hi;
-      if (valid) {
-        const float f1 = s.b1[j][m], f2 = s.b2[j][m];
-        const uint4 z = make_uint4(0, 0, 0, 0);
+      // row m of both outputs' diagonal block (16 columns each), bf16
+      const float f1 = s.b1[j][m], f2 = s.b2[j][m];
+      uint4 u1[2], u2[2];
 #pragma unroll
-        for (int q = 0; q < 6; ++q) {
-          if (q < 2 * b) {
-            *reinterpret_cast<uint4*>(dst + m * 128 + (((q ^ (m & 7)) & 7) << 4)) = z;
-            *reinterpret_cast<uint4*>(dst + 8192 + m * 128 + (((q ^ (m & 7)) & 7) << 4)) = z;
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint4 u1, u2;
-          const float* xh = x + 8 * h;
-          u1.x = pack_bf16x2(f1 * xh[0], f1 * xh[1]); u1.y = pack_bf16x2(f1 * xh[2], f1 * xh[3]);
-          u1.z = pack_bf16x2(f1 * xh[4], f1 * xh[5]); u1.w = pack_bf16x2(f1 * xh[6], f1 * xh[7]);
-          u2.x = pack_bf16x2(f2 * xh[0], f2 * xh[1]); u2.y = pack_bf16x2(f2 * xh[2], f2 * xh[3]);
-          u2.z = pack_bf16x2(f2 * xh[4], f2 * xh[5]); u2.w = pack_bf16x2(f2 * xh[6], f2 * xh[7]);
-          const int q = 2 * b + h;
-          *reinterpret_cast<uint4*>(dst + m * 128 + (((q ^ (m & 7)) & 7) << 4)) = u1;
-          *reinterpret_cast<uint4*>(dst + 8192 + m * 128 + (((q ^ (m & 7)) & 7) << 4)) = u2;
-        }
-        if constexpr (CHECK) {
+      for (int h = 0; h < 2; ++h) {
+        const float* xh = x + 8 * h;
+        u1[h].x = pack_bf16x2(f1 * xh[0], f1 * xh[1]); u1[h].y = pack_bf16x2(f1 * xh[2], f1 * xh[3]);
+        u1[h].z = pack_bf16x2(f1 * xh[4], f1 * xh[5]); u1[h].w = pack_bf16x2(f1 * xh[6], f1 * xh[7]);
+        u2[h].x = pack_bf16x2(f2 * xh[0], f2 * xh[1]); u2[h].y = pack_bf16x2(f2 * xh[2], f2 * xh[3]);
+        u2[h].z = pack_bf16x2(f2 * xh[4], f2 * xh[5]); u2[h].w = pack_bf16x2(f2 * xh[6], f2 * xh[7]);
+      }
+      if constexpr (CHECK) {
+        if (valid) {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             if (i > c) worst = fmaxf(worst, bound_ratio(s, j, 16 * b + i, m, x[i]));
         }
       }
+      // staged over the chunk's diagonal blocks of A once every thread of
+      // the chunk is done reading them: [output][row m][half]
+      uint4* stg = reinterpret_cast<uint4*>(&s.w.adt[j][0][0]);
+      nbar_sync64(chunk_bar + j);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        stg[m * 2 + h] = u1[h];
+        stg[(64 + m) * 2 + h] = u2[h];
+      }
     }
     nbar_sync64(chunk_bar + j);
+    // The 16-byte chunks of both output tiles that are known now (in row m
+    // of block b: the 2 b zero chunks left of the diagonal block and its 2
+    // chunks), written row by row: eight threads per 128-byte row, so a
+    // warp's store covers four whole rows (the off-diagonal chunks follow
+    // from the products below).
+    if (valid) {
+      const uint4* stg = reinterpret_cast<const uint4*>(&s.w.adt[j][0][0]);
+      const int u = tid & 63, p = u & 7;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int m = 8 * k + (u >> 3), q = p ^ (m & 7), bq = m >> 4;
+          if (q < 2 * bq + 2) {
+            const uint4 val = q < 2 * bq ? make_uint4(0, 0, 0, 0)
+                                         : stg[(64 * t + m) * 2 + (q - 2 * bq)];
+            *reinterpret_cast<uint4*>(dst + t * 8192 + m * 128 + p * 16) = val;
+          }
+        }
+      }
+    }
 
     // ---- off-diagonal row blocks of Y = T^T: warp 2j takes row block 0,
     // warp 2j + 1 row blocks 1 and 2 (row block 3 is D_3^T alone)
