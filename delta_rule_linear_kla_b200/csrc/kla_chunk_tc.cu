@@ -748,11 +748,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                       mode, ws, err, blockIdx.x, blockIdx.y, blockIdx.z, nullptr);
 }
 
-// UT lanes (128 threads each) per CTA of the single-launch prefill: all of
-// its 512 threads (the lanes' shared memory fits in the state CTA's).
+// UT lanes (128 threads each) per CTA of the single-launch prefill (the
+// lanes' shared memory fits in the state CTA's; the fourth group of 128
+// threads idles).
 template <int DK>
 constexpr int fused_ut_lanes() {
-  return 4;
+  return 3;
 }
 template <int DK>
 constexpr size_t fused_smem_bytes() {
@@ -787,9 +788,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     return;
   }
   constexpr int LANES = fused_ut_lanes<DK>();
-  static_assert(LANES == 4 && LANES * 128 == NTHREADS, "one call per lane below");
+  static_assert(LANES == 3 && LANES * 128 < NTHREADS, "one call per lane below");
   static_assert(1 + 3 * LANES <= 16, "named barriers: one per lane, two per chunk slot");
   const int lane_id = (int)threadIdx.x >> 7;
+  if (lane_id >= LANES) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -811,10 +813,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     run(std::integral_constant<int, 0>());
   else if (lane_id == 1)
     run(std::integral_constant<int, 1>());
-  else if (lane_id == 2)
-    run(std::integral_constant<int, 2>());
   else
-    run(std::integral_constant<int, 3>());
+    run(std::integral_constant<int, 2>());
 }
 
 // ------------------------------------------------------------------ host
@@ -975,7 +975,7 @@ bool fused_shape(int B, int T, int H, int dk, int dv) {
   if (n_chain + kMinUtCtas > kSmTarget) return false;
   const long nchunks = (T + C - 1) / C, pairs = ((long)B * H * nchunks + 1) / 2;
   const long lanes_alone = 4L * kSmTarget;
-  const long lanes_fused = 4L * (kSmTarget - n_chain);
+  const long lanes_fused = 3L * (kSmTarget - n_chain);
   const long chain = nchunks * kStepCost;
   const long two = (pairs + lanes_alone - 1) / lanes_alone * kPairCost + chain;
   const long one = std::max((pairs + lanes_fused - 1) / lanes_fused * kPairCost, chain);
