@@ -693,16 +693,27 @@ __device__ __forceinline__ void chain_body(
           mbar_arrive(&s.pv_free);
         }
         if (t < T && mode == 0 && o) {
-          uint4* dst = reinterpret_cast<uint4*>(o + (((size_t)b * T + t) * H + hh) * DV +
-                                                slab * BV + cg);
+          __nv_bfloat16* orow = o + (((size_t)b * T + t) * H + hh) * DV + slab * BV + cg;
+          uint32_t w[16];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint4 u4;
-            u4.x = pack_bf16x2(fmaf(e, x[8 * c + 0], pv[8 * c + 0]), fmaf(e, x[8 * c + 1], pv[8 * c + 1]));
-            u4.y = pack_bf16x2(fmaf(e, x[8 * c + 2], pv[8 * c + 2]), fmaf(e, x[8 * c + 3], pv[8 * c + 3]));
-            u4.z = pack_bf16x2(fmaf(e, x[8 * c + 4], pv[8 * c + 4]), fmaf(e, x[8 * c + 5], pv[8 * c + 5]));
-            u4.w = pack_bf16x2(fmaf(e, x[8 * c + 6], pv[8 * c + 6]), fmaf(e, x[8 * c + 7], pv[8 * c + 7]));
-            dst[c] = u4;
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(fmaf(e, x[2 * i], pv[2 * i]), fmaf(e, x[2 * i + 1], pv[2 * i + 1]));
+          // the row's 64 bytes as two 32-byte stores where o allows it (the
+          // offsets here are multiples of 64 bytes, so this is uniform over
+          // the launch), else four 16-byte ones
+          if ((reinterpret_cast<uintptr_t>(orow) & 31u) == 0u) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                               orow + 16 * c),
+                           "r"(w[8 * c]), "r"(w[8 * c + 1]), "r"(w[8 * c + 2]), "r"(w[8 * c + 3]),
+                           "r"(w[8 * c + 4]), "r"(w[8 * c + 5]), "r"(w[8 * c + 6]), "r"(w[8 * c + 7])
+                           : "memory");
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
           }
         }
       }
@@ -848,16 +859,20 @@ bool make_map(CUtensorMap* m, const void* base, int d, int H, int T, int B) {
 // Phi_s h(s) + E_s, for one head and 64-column slab per CTA, fp32 on CUDA
 // cores (nseg - 1 products of [DK][DK] by [DK][64]).  E and Phi hold the
 // nseg - 1 first segments ([B][nseg - 1][H]), hstart all nseg ([B][nseg][H]).
-// Thread t owns row t / 2 and 32 columns of the slab; the slab itself stays
-// in shared memory.
+// Thread t owns row t / 2 and 32 columns of the slab; the slab stays in
+// shared memory, and Phi passes through it 16 columns at a time in
+// coalesced loads (its rows read straight from global memory, one value per
+// step, left every step waiting on a load).
 template <int DK>
 __global__ void __launch_bounds__(2 * DK)
 segment_start_kernel(const float* __restrict__ h0, const float* __restrict__ E,
                      const float* __restrict__ Phi, float* __restrict__ hstart, int H, int DV,
                      int nseg) {
+  constexpr int KB = 16;  // columns of Phi per staged block
   __shared__ float hs[DK][BV];
+  __shared__ float phs[DK][KB + 1];
   const int slab = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
-  const int i = threadIdx.x >> 1, c0 = 32 * (threadIdx.x & 1);
+  const int tid = threadIdx.x, i = tid >> 1, c0 = 32 * (tid & 1);
   const size_t head = (size_t)b * H + hh;
   float acc[32];
 #pragma unroll
@@ -867,15 +882,27 @@ segment_start_kernel(const float* __restrict__ h0, const float* __restrict__ E,
     const size_t sidx = ((size_t)b * nseg + sg) * H + hh;
     if (sg > 0) {
       const size_t pidx = ((size_t)b * (nseg - 1) + sg - 1) * H + hh;  // segment sg - 1
-      const float* ph = Phi + (pidx * DK + i) * DK;
+      const float* ph = Phi + pidx * DK * DK;
       const float* e = E + (pidx * DK + i) * DV + slab * BV + c0;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) acc[c] = e[c];
-#pragma unroll 4
-      for (int kq = 0; kq < DK; ++kq) {
-        const float a = ph[kq];
+      for (int c = 0; c < 32; c += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(e + c);
+        acc[c] = x.x; acc[c + 1] = x.y; acc[c + 2] = x.z; acc[c + 3] = x.w;
+      }
+#pragma unroll 1
+      for (int kq0 = 0; kq0 < DK; kq0 += KB) {
+        __syncthreads();  // the previous block of Phi has been read
+        for (int idx = tid; idx < DK * KB; idx += 2 * DK) {
+          const int r = idx / KB, c = idx % KB;
+          phs[r][c] = ph[(size_t)r * DK + kq0 + c];
+        }
+        __syncthreads();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) acc[c] = fmaf(a, hs[kq][c0 + c], acc[c]);
+        for (int kk = 0; kk < KB; ++kk) {
+          const float a = phs[i][kk];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) acc[c] = fmaf(a, hs[kq0 + kk][c0 + c], acc[c]);
+        }
       }
       __syncthreads();  // everyone has read h(sg - 1)
     }
@@ -883,7 +910,8 @@ segment_start_kernel(const float* __restrict__ h0, const float* __restrict__ E,
     for (int c = 0; c < 32; ++c) hs[i][c0 + c] = acc[c];
     float* dst = hstart + (sidx * DK + i) * DV + slab * BV + c0;
 #pragma unroll
-    for (int c = 0; c < 32; ++c) dst[c] = acc[c];
+    for (int c = 0; c < 32; c += 4)
+      *reinterpret_cast<float4*>(dst + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
     __syncthreads();
   }
 }
