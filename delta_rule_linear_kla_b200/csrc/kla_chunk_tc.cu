@@ -684,8 +684,7 @@ __device__ __forceinline__ void chain_body(
         if (!wait_warp(&s.bHP, par, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
         float x[32], pv[32];
-        ptx::tmem_ld32(tb + lane_base + col_u + cg, x);
-        ptx::tmem_ld32(tb + lane_base + COL_PV + cg, pv);
+        ptx::tmem_ld32x2(tb + lane_base + col_u + cg, tb + lane_base + COL_PV + cg, x, pv);
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) {

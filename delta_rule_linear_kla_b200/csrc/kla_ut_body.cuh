@@ -331,8 +331,11 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
     {
       // hd: the 32-column half that holds the diagonal (warp-uniform)
       const int hd = warp & 1;
-      float v[32];
-      ptx::tmem_ld32(tacc + lane_base + 64 * j + 32 * hd, v);
+      float v[32], vl[32];  // the half that holds the diagonal; (hd = 1) the left half
+      if (hd == 1)
+        ptx::tmem_ld32x2(tacc + lane_base + 64 * j + 32, tacc + lane_base + 64 * j, v, vl);
+      else
+        ptx::tmem_ld32(tacc + lane_base + 64 * j, v);
       float nn2 = 0.f;
 #pragma unroll
       for (int c = 0; c < 32; ++c) nn2 = (c == (r & 31)) ? v[c] : nn2;
@@ -383,12 +386,11 @@ __device__ __forceinline__ void ut_run(const CUtensorMap* tm_k, const float* __r
       if (hd == 1) {
         // columns 0..31 lie wholly left of rows 32..63:
         // e^{G_r - G_s} = e^{G_r - G_{16q+15}} E_s, both factors <= 1
-        ptx::tmem_ld32(tacc + lane_base + 64 * j, v);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const float f = beta * __expf(Gr - s.G[j][16 * q + 15]);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[16 * q + i] *= f * s.E[j][16 * q + i];
+          for (int i = 0; i < 16; ++i) v[16 * q + i] = vl[16 * q + i] * (f * s.E[j][16 * q + i]);
         }
         store_bf16(0);
       }
