@@ -486,12 +486,11 @@ __device__ __forceinline__ void chain_body(
       ptx::tc_fence_after();
 #pragma unroll
       for (int p = 0; p < NP; ++p) {
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float w[32];
-          ptx::tmem_ld32(tb + lane_base + COL_W + p * 64 + 32 * hf, w);
-          sw128_store_row32(S.panel[p][SW], row, hf, w);
-        }
+        float w0[32], w1[32];  // the panel's two 32-column halves, one wait
+        ptx::tmem_ld32x2(tb + lane_base + COL_W + p * 64, tb + lane_base + COL_W + p * 64 + 32,
+                         w0, w1);
+        sw128_store_row32(S.panel[p][SW], row, 0, w0);
+        sw128_store_row32(S.panel[p][SW], row, 1, w1);
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
