@@ -86,4 +86,10 @@ cudaError_t launch_ut(const CUtensorMap& tm_k, const float* g, const float* eta,
                       uint8_t* ws, int B, int T, int H, int dk, unsigned int* err,
                       cudaStream_t st, float* ratio_max = nullptr);
 
+// The same kernel for the chunks n < n_first of every head only (chunk index
+// major): the factors the first pass of a cut chain reads.
+cudaError_t launch_ut_first(const CUtensorMap& tm_k, const float* g, const float* eta,
+                            float eps, uint8_t* ws, int B, int T, int H, int dk, int n_first,
+                            unsigned int* err, cudaStream_t st);
+
 }  // namespace kla

@@ -826,6 +826,53 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     run(std::integral_constant<int, 2>());
 }
 
+// Pass 1 of a cut chain (the transitions E, Phi of segments 0 .. S-2: CTAs
+// 0 .. n_chain - 1, the mode-1 chain grid flattened, slab fastest, then
+// head, then batch x segment) and, on the SMs those CTAs leave, UT lanes that
+// make the factors of the chunks n >= n_split of every head (the last
+// segment, which only pass 2 reads).  The two roles share no data and wait
+// on nothing from each other, so this is a plain launch.
+template <int DK>
+__global__ void __launch_bounds__(NTHREADS, 1)
+pass1_ut_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+                const float* __restrict__ eta, float eps, float* __restrict__ E,
+                float* __restrict__ phi, int T, int H, int DV, int nseg1, int seg_chunks,
+                uint8_t* __restrict__ ws, int n_chain, int BH, int n_split, unsigned int* err) {
+  const int nchunks = (T + C - 1) / C;
+  if ((int)blockIdx.x < n_chain) {
+    const int nx = (DV + DK) / BV;
+    const int bx = (int)blockIdx.x % nx, by = ((int)blockIdx.x / nx) % H,
+              bz = (int)blockIdx.x / (nx * H);
+    chain_body<DK, false>(&tm_q, &tm_k, &tm_v, g, nullptr, nullptr, E, phi, nullptr, T, H, DV,
+                          nseg1, seg_chunks, 1, ws, err, bx, by, bz, nullptr);
+    return;
+  }
+  constexpr int LANES = fused_ut_lanes<DK>();
+  static_assert(LANES == 3 && LANES * 128 < NTHREADS, "one call per lane below");
+  const int lane_id = (int)threadIdx.x >> 7;
+  if (lane_id >= LANES) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int nlanes = ((int)gridDim.x - n_chain) * LANES;
+  // each lane's shared memory at a compile-time offset (see prefill_kernel)
+  auto run = [&](auto lane_c) {
+    constexpr int L = decltype(lane_c)::value;
+    auto& us = *reinterpret_cast<utb::UtSmem<DK>*>(base + L * sizeof(utb::UtSmem<DK>));
+    utb::ut_run<DK, false>(&tm_k, g, eta, eps, ws, T, H, nchunks, BH, BH * n_split,
+                           BH * (nchunks - n_split), true, err, nullptr, nullptr, us,
+                           (int)threadIdx.x & 127, 1 + L, 1 + LANES + 2 * L,
+                           ((int)blockIdx.x - n_chain) * LANES + L, nlanes, false);
+  };
+  if (lane_id == 0)
+    run(std::integral_constant<int, 0>());
+  else if (lane_id == 1)
+    run(std::integral_constant<int, 1>());
+  else
+    run(std::integral_constant<int, 2>());
+}
+
 // ------------------------------------------------------------------ host
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1112,6 +1159,65 @@ static cudaError_t launch_segmented(const void* q, const void* k, const void* v,
                                   ws, err, st, hs);
 }
 
+// The cut chain with the UT work overlapped: the UT kernel for the chunks of
+// segments 0 .. S-2 only, then pass 1 with UT lanes for the last segment on
+// the SMs its CTAs leave, the start states and pass 2.  cudaErrorNotSupported
+// (nothing launched) where those lanes would not finish within pass 1 by the
+// cost model, or pass 1 leaves fewer than kMinUtCtas SMs.
+template <int DK>
+static cudaError_t launch_segmented_overlap(const void* q, const void* k, const void* v,
+                                            const float* g, const float* eta, float eps,
+                                            const float* h0, void* o, float* hT, int B, int T,
+                                            int H, int sg, uint8_t* ws, size_t tiles,
+                                            unsigned int* err, cudaStream_t st, float* hs) {
+  constexpr int DV = DK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  static int sms[64] = {};
+  static bool attr[64] = {};
+  constexpr size_t smem = fused_smem_bytes<DK>();
+  if (!sms[dev]) {
+    cudaError_t e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  const int nchunks = (T + C - 1) / C;
+  const int len = (nchunks + sg - 1) / sg;
+  const int n_split = (sg - 1) * len;
+  const long BH = (long)B * H;
+  const long n_chain = BH * ((DV + DK) / BV) * (sg - 1);
+  const long ut_ctas = sms[dev] - n_chain;
+  if (ut_ctas < kMinUtCtas) return cudaErrorNotSupported;
+  const long lanes = (long)fused_ut_lanes<DK>() * ut_ctas;
+  const long pairs = (BH * (nchunks - n_split) + 1) / 2;
+  if ((pairs + lanes - 1) / lanes * kPairCost > (long)len * kStepCost) return cudaErrorNotSupported;
+  if (!attr[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(pass1_ut_kernel<DK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr[dev] = true;
+  }
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, DK, H, T, B) || !make_map(&mk, k, DK, H, T, B) ||
+      !make_map(&mv, v, DV, H, T, B))
+    return cudaErrorInvalidValue;
+  const size_t n = (size_t)B * sg * H;
+  float* E = reinterpret_cast<float*>(ws + tiles);
+  float* hstart = E + n * DK * DV;
+  float* Phi = hstart + n * DK * DV;
+  cudaError_t e = launch_ut_first(mk, g, eta, eps, ws, B, T, H, DK, n_split, err, st);
+  if (e != cudaSuccess) return e;
+  pass1_ut_kernel<DK><<<(unsigned)(n_chain + ut_ctas), NTHREADS, smem, st>>>(
+      mq, mk, mv, g, eta, eps, E, Phi, T, H, DV, sg - 1, len, ws, (int)n_chain, (int)BH, n_split,
+      err);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  segment_start_kernel<DK><<<dim3(DV / BV, H, B), 2 * DK, 0, st>>>(h0, E, Phi, hstart, H, DV, sg);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_chain_dk<DK, false>(q, k, v, g, hstart, o, hT, nullptr, B, T, H, DV, sg, len, 0,
+                                    ws, err, st, hs);
+}
+
 // The single-launch prefill (see prefill_kernel).  cudaErrorNotSupported when
 // this device cannot hold it (too few SMs beside the state CTAs, no
 // cooperative launch): the caller then runs the two kernels in turn.
@@ -1172,6 +1278,17 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
     const cudaError_t e =
         dk == 128 ? launch_fused<128>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, wsm, err, st, hs)
                   : launch_fused<64>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, wsm, err, st, hs);
+    if (e != cudaErrorNotSupported) return e;
+  }
+  const int sg = chunk_chain_segments(B, T, H, dk, dv, ws_bytes);
+  if (sg > 1) {
+    uint8_t* wsm = (uint8_t*)workspace;
+    const size_t tiles = ut_workspace_bytes(B, T, H);
+    const cudaError_t e =
+        dk == 128 ? launch_segmented_overlap<128>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, sg,
+                                                  wsm, tiles, err, st, hs)
+                  : launch_segmented_overlap<64>(q, k, v, g, eta, eps, h0, o, hT, B, T, H, sg,
+                                                 wsm, tiles, err, st, hs);
     if (e != cudaErrorNotSupported) return e;
   }
   cudaError_t e = launch_chunk_ut(k, g, eta, eps, B, T, H, dk, workspace, err, st);

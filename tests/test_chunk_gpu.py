@@ -273,3 +273,24 @@ def test_single_launch_equals_two_launches(name, B, T, H):
         api.check_device_error()
         assert torch.equal(o1, o2) and torch.equal(h1, h2)
 
+
+
+@pytest.mark.parametrize("name,B,T,H,h0", SEGMENTED)
+def test_cut_chain_overlapped_ut_equals_staged(name, B, T, H, h0):
+    """The cut chain as kla_chunk_fwd runs it (the UT kernel for the chunks
+    of the first segments, then pass 1 beside UT lanes that make the last
+    segment's factors) equals the staged calls (kla_chunk_ut_transform for
+    every chunk, then kla_chunk_state_fwd on the same workspace) bit for bit:
+    the factors do not depend on which kernel makes them."""
+    w = W[name].scaled(B=B, T=T, H=H, seed=19)
+    x = cuda(inputs.make_prefill(w, with_h0=h0))
+    nws = api.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv)
+    assert api.chunk_fwd_segments(w.B, w.T, w.H, w.dk, w.dv, ws_bytes=nws) > 1
+    ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+    o1, h1 = api.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"],
+                           workspace=ws)
+    ws2 = torch.empty(nws, dtype=torch.uint8, device="cuda")
+    api.chunk_ut_transform(x["k"], x["g"], x["eta"], x["eps"], workspace=ws2)
+    o2, h2 = api.chunk_state_fwd(x["q"], x["k"], x["v"], x["g"], ws2, x["h0"])
+    api.check_device_error()
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
