@@ -900,65 +900,72 @@ bool make_map(CUtensorMap* m, const void* base, int d, int H, int T, int B) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Start state of every segment: h(0) = h0 (NULL = zeros), h(s + 1) =
-// Phi_s h(s) + E_s, for one head and 64-column slab per CTA, fp32 on CUDA
-// cores (nseg - 1 products of [DK][DK] by [DK][64]).  E and Phi hold the
-// nseg - 1 first segments ([B][nseg - 1][H]), hstart all nseg ([B][nseg][H]).
-// Thread t owns row t / 2 and 32 columns of the slab; the slab stays in
-// shared memory, and Phi passes through it 16 columns at a time in
-// coalesced loads (its rows read straight from global memory, one value per
-// step, left every step waiting on a load).
+// One step of the segment start states: hstart(s + 1) = Phi_s h(s) + E_s,
+// with h(0) = h0 (NULL = zeros), which step 0 also copies to hstart(0); fp32
+// on CUDA cores, one launch per step.  A CTA takes 16 rows of one head's
+// 64-column slab (h(s)'s slab and Phi_s's 16 rows staged in shared memory);
+// thread t owns row t / 16 and 4 columns.  E and Phi hold the nseg - 1 first
+// segments ([B][nseg - 1][H]), hstart all nseg ([B][nseg][H]).  (One CTA per
+// head and slab walking every step, Phi's rows read one value per step from
+// global memory, took ~80 µs of the 65K step; staging Phi in that form,
+// ~60 µs.)
+constexpr int kStartRows = 16;
 template <int DK>
-__global__ void __launch_bounds__(2 * DK)
-segment_start_kernel(const float* __restrict__ h0, const float* __restrict__ E,
-                     const float* __restrict__ Phi, float* __restrict__ hstart, int H, int DV,
-                     int nseg) {
-  constexpr int KB = 16;  // columns of Phi per staged block
-  __shared__ float hs[DK][BV];
-  __shared__ float phs[DK][KB + 1];
-  const int slab = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, i = tid >> 1, c0 = 32 * (tid & 1);
+__global__ void __launch_bounds__(256)
+segment_step_kernel(const float* __restrict__ h0, const float* __restrict__ E,
+                    const float* __restrict__ Phi, float* __restrict__ hstart, int H, int DV,
+                    int nseg, int step) {
+  constexpr int RB = kStartRows;
+  __shared__ __align__(16) float hsrc[DK][BV];
+  __shared__ float ph[RB][DK + 1];
+  const int slab = blockIdx.x, hh = blockIdx.y;
+  const int b = blockIdx.z / (DK / RB), rb = blockIdx.z % (DK / RB);
+  const int tid = threadIdx.x;
   const size_t head = (size_t)b * H + hh;
-  float acc[32];
-#pragma unroll
-  for (int c = 0; c < 32; ++c)
-    acc[c] = h0 ? h0[(head * DK + i) * DV + slab * BV + c0 + c] : 0.f;
-  for (int sg = 0; sg < nseg; ++sg) {
-    const size_t sidx = ((size_t)b * nseg + sg) * H + hh;
-    if (sg > 0) {
-      const size_t pidx = ((size_t)b * (nseg - 1) + sg - 1) * H + hh;  // segment sg - 1
-      const float* ph = Phi + pidx * DK * DK;
-      const float* e = E + (pidx * DK + i) * DV + slab * BV + c0;
-#pragma unroll
-      for (int c = 0; c < 32; c += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(e + c);
-        acc[c] = x.x; acc[c + 1] = x.y; acc[c + 2] = x.z; acc[c + 3] = x.w;
-      }
-#pragma unroll 1
-      for (int kq0 = 0; kq0 < DK; kq0 += KB) {
-        __syncthreads();  // the previous block of Phi has been read
-        for (int idx = tid; idx < DK * KB; idx += 2 * DK) {
-          const int r = idx / KB, c = idx % KB;
-          phs[r][c] = ph[(size_t)r * DK + kq0 + c];
-        }
-        __syncthreads();
-#pragma unroll
-        for (int kk = 0; kk < KB; ++kk) {
-          const float a = phs[i][kk];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) acc[c] = fmaf(a, hs[kq0 + kk][c0 + c], acc[c]);
-        }
-      }
-      __syncthreads();  // everyone has read h(sg - 1)
-    }
-#pragma unroll
-    for (int c = 0; c < 32; ++c) hs[i][c0 + c] = acc[c];
-    float* dst = hstart + (sidx * DK + i) * DV + slab * BV + c0;
-#pragma unroll
-    for (int c = 0; c < 32; c += 4)
-      *reinterpret_cast<float4*>(dst + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-    __syncthreads();
+  const float* src = step > 0 ? hstart + (((size_t)b * nseg + step) * H + hh) * DK * DV
+                     : h0     ? h0 + head * DK * DV
+                              : nullptr;
+  float* dst0 = hstart + ((size_t)b * nseg * H + hh) * DK * DV;  // hstart(0) of this head
+  for (int idx = tid; idx < DK * BV / 4; idx += 256) {
+    const int r = idx / (BV / 4), c = 4 * (idx % (BV / 4));
+    const float4 x = src ? *reinterpret_cast<const float4*>(src + (size_t)r * DV + slab * BV + c)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(&hsrc[r][c]) = x;
+    if (step == 0 && r / RB == rb)
+      *reinterpret_cast<float4*>(dst0 + (size_t)r * DV + slab * BV + c) = x;
   }
+  const size_t pidx = ((size_t)b * (nseg - 1) + step) * H + hh;
+  for (int idx = tid; idx < RB * DK; idx += 256) {
+    const int r = idx / DK, k = idx % DK;
+    ph[r][k] = Phi[(pidx * DK + rb * RB + r) * DK + k];
+  }
+  __syncthreads();
+  const int r = tid >> 4, c = 4 * (tid & 15), row = rb * RB + r;
+  float4 acc = *reinterpret_cast<const float4*>(E + (pidx * DK + row) * DV + slab * BV + c);
+#pragma unroll 8
+  for (int k = 0; k < DK; ++k) {
+    const float a = ph[r][k];
+    const float4 hv = *reinterpret_cast<const float4*>(&hsrc[k][c]);
+    acc.x = fmaf(a, hv.x, acc.x);
+    acc.y = fmaf(a, hv.y, acc.y);
+    acc.z = fmaf(a, hv.z, acc.z);
+    acc.w = fmaf(a, hv.w, acc.w);
+  }
+  *reinterpret_cast<float4*>(
+      hstart + ((((size_t)b * nseg + step + 1) * H + hh) * DK + row) * DV + slab * BV + c) = acc;
+}
+
+template <int DK>
+static cudaError_t launch_segment_starts(const float* h0, const float* E, const float* Phi,
+                                         float* hstart, int B, int H, int DV, int nseg,
+                                         cudaStream_t st) {
+  for (int step = 0; step + 1 < nseg; ++step) {
+    segment_step_kernel<DK><<<dim3(DV / BV, H, B * (DK / kStartRows)), 256, 0, st>>>(
+        h0, E, Phi, hstart, H, DV, nseg, step);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template <int DK, bool KDA>
@@ -1152,8 +1159,7 @@ static cudaError_t launch_segmented(const void* q, const void* k, const void* v,
   cudaError_t e = launch_chain_dk<DK, KDA>(q, k, v, g, nullptr, nullptr, E, Phi, B, T, H, DV,
                                            sg - 1, len, 1, ws, err, st);
   if (e != cudaSuccess) return e;
-  segment_start_kernel<DK><<<dim3(DV / BV, H, B), 2 * DK, 0, st>>>(h0, E, Phi, hstart, H, DV, sg);
-  e = cudaGetLastError();
+  e = launch_segment_starts<DK>(h0, E, Phi, hstart, B, H, DV, sg, st);
   if (e != cudaSuccess) return e;
   return launch_chain_dk<DK, KDA>(q, k, v, g, hstart, o, hT, nullptr, B, T, H, DV, sg, len, 0,
                                   ws, err, st, hs);
@@ -1211,8 +1217,7 @@ static cudaError_t launch_segmented_overlap(const void* q, const void* k, const 
       err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  segment_start_kernel<DK><<<dim3(DV / BV, H, B), 2 * DK, 0, st>>>(h0, E, Phi, hstart, H, DV, sg);
-  e = cudaGetLastError();
+  e = launch_segment_starts<DK>(h0, E, Phi, hstart, B, H, DV, sg, st);
   if (e != cudaSuccess) return e;
   return launch_chain_dk<DK, false>(q, k, v, g, hstart, o, hT, nullptr, B, T, H, DV, sg, len, 0,
                                     ws, err, st, hs);
