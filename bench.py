@@ -212,10 +212,11 @@ def run_ours(args, rank, world, dev):
         fn = functools.partial(api.chunk_fwd, workspace=ws)
         nseg = api.chunk_fwd_segments(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, nws)
         # one launch (UT lanes and state CTAs together), or the UT kernel
-        # then one chain launch, or three for a cut chain (segment
-        # transitions, start states, outputs)
+        # then one chain launch, or for a cut chain of S segments S + 1
+        # launches after the UT kernel (segment transitions, one start-state
+        # launch per segment boundary, outputs)
         single = api.chunk_fwd_single_launch(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, nws)
-        launches_per_step = 1 if single else 1 + (3 if nseg > 1 else 1)
+        launches_per_step = 1 if single else 1 + (nseg + 1 if nseg > 1 else 1)
     else:
         fn = api.recurrent_fwd
         nseg, launches_per_step, single = 0, 1, False
@@ -333,7 +334,7 @@ def run_ours(args, rank, world, dev):
                    "hbm_frac": byts / (ms / 1e3) / 1e9 / hbm_peak,
                    "peak_source": peak_src + " (burst cuBLAS bf16)"},
         # our kernels per step: one single-launch prefill, or UT transform +
-        # chain (three chain launches for a cut chain), one token-serial
+        # chain (S + 1 launches for a chain cut into S segments), one token-serial
         # kernel otherwise; the L2 flush and the flag clear are not counted
         "gpu_launches": args.steps * launches_per_step,
         "wall_s": wall,
