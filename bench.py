@@ -358,7 +358,7 @@ def run_ours(args, rank, world, dev):
                              "algorithmic_bytes": chain_w["bytes"], "gbs": chain_gbs,
                              "tflops": chain_w["flops"] / (ms_chain / 1e3) / 1e12}}
         if nseg > 1:
-            # the cut chain: its time spans its three launches
+            # the cut chain: its time spans its S + 1 launches
             res["kernels"]["chain_kernel"]["launches"] = (
                 "%d segments: transitions, start states, outputs" % nseg)
     if chunk and not args.no_other and args.workload == "prefill_4k":
