@@ -130,7 +130,9 @@ decode_kernel(const T* __restrict__ q, const T* __restrict__ k,
     x.z = fmaf(kk, u4.z, alpha * x.z); x.w = fmaf(kk, u4.w, alpha * x.w);
     *reinterpret_cast<float4*>(Sh + (size_t)(row0 + m * RPP) * DV + col) = x;
   }
-  __syncthreads();  // the next tile reuses the reduction buffers
+  // no barrier here: every read of red_r, red_s and kq_sh for this tile came
+  // before the barrier above, and the next tile writes u_sh only after its
+  // first barrier, which every thread reaches after this update
   }
 }
 
