@@ -1049,7 +1049,15 @@ constexpr long kPairCost = 5, kStepCost = 1;
 // those SMs finish sooner than the UT kernel alone would on all of them plus
 // the chain after it (the launcher checks the actual device again and
 // otherwise runs the two kernels one after the other).
+//
+// The single launch is built but not taken: twice, a full run of the GPU
+// tests stopped on an "unspecified launch failure" in the chunkwise backward
+// of a short sequence whose forward ran it (once with four UT lanes per CTA,
+// once with three), and reading the code has not found the cause.  Every
+// shape runs the two kernels in turn until it is found.
+constexpr bool kSingleLaunchTaken = false;
 bool fused_shape(int B, int T, int H, int dk, int dv) {
+  if (!kSingleLaunchTaken) return false;
   if (chain_segments(B, T, H, dk, dv) != 1) return false;
   const long n_chain = (long)B * H * (dv / BV);
   if (n_chain + kMinUtCtas > kSmTarget) return false;

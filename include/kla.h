@@ -79,11 +79,9 @@ typedef enum { KLA_BF16 = 0, KLA_FP32 = 1 } kla_dtype;
  *     the per-chunk factors (B * H * ceil(T / KLA_CHUNK) * 16384 bytes, the
  *     least accepted, else KLA_ERR_INVALID_ARG) followed either, for few
  *     heads and long sequences, by the states of the sequence segments the
- *     state chain is cut into (run in parallel), or, where the whole prefill
- *     runs as one launch (kla_chunk_fwd_single_launch), by one 4-byte ready
- *     flag per chunk (rounded up to 256 bytes; cleared by the call itself).
- *     A workspace smaller than the full size but holding the factors runs
- *     the chain uncut, with the factors formed by a launch of their own.
+ *     state chain is cut into (run in parallel).  A workspace smaller than
+ *     the full size but holding the factors runs the chain uncut.  The
+ *     factors are formed by a launch of their own before the chain.
  *     It must not overlap any other argument.
  *
  * Supported: B, H >= 1; T >= 0 (T = 0 copies h0 to hT); dk = dv in {64, 128}.
@@ -107,15 +105,12 @@ KLA_API int kla_chunk_fwd_segments(int B, int T, int H, int dk, int dv, int dtyp
                                    size_t ws_bytes);
 
 /*
- * 1 when the bf16 kla_chunk_fwd of this shape runs as a single kernel launch
- * with a workspace of ws_bytes: the chain is uncut, the state CTAs (one per
- * head and 64 state columns) leave at least 8 of a B200's 148 SMs for CTAs
- * that form the per-chunk factors in the same launch (cooperative, every
- * CTA resident; the state CTAs wait, bounded, on a per-chunk ready flag),
- * and the workspace holds the flags after the factors (as sized by
- * kla_chunk_fwd_workspace_size).  0 otherwise, when the factors are formed
- * by a launch of their own first (also on a device where the single launch
- * does not fit, which the call detects itself).  Host-only query.
+ * 1 when the bf16 kla_chunk_fwd of this shape would run as a single kernel
+ * launch with a workspace of ws_bytes (the per-chunk factors formed beside
+ * the state CTAs in one cooperative launch).  At present 0 for every shape:
+ * that launch is built but not taken, after an intermittent launch failure
+ * whose cause has not been found, so the factors are always formed by a
+ * launch of their own first.  Host-only query.
  */
 KLA_API int kla_chunk_fwd_single_launch(int B, int T, int H, int dk, int dv, int dtype,
                                         size_t ws_bytes);

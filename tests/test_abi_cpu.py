@@ -171,33 +171,20 @@ def test_selftest_rejects_bad_limits(lib):
     assert lib.kla_selftest_wait_timeout(10001, None) == INVALID
 
 
-def _flag_bytes(B, T, H):
-    """One ready flag (4 bytes) per chunk, rounded up to 256 bytes: the
-    single-launch prefill's chunk flags after the factors."""
-    return (B * H * ((T + 63) // 64) * 4 + 255) // 256 * 256
-
-
 def test_workspace_query(lib):
-    # a short batch: uncut chain in a single launch, the factors and one
-    # ready flag per chunk
-    assert lib.kla_chunk_fwd_workspace_size(2, 1000, 4, 128, 128, 0) == (
-        _ut_bytes(2, 1000, 4) + _flag_bytes(2, 1000, 4))
-    # the 0.4B-scale layer: its factors take the UT lanes of the 20 SMs the
-    # state CTAs leave longer than the UT kernel on all SMs plus the chain:
-    # two launches, factors only
+    # an uncut chain: the per-chunk factors alone (a short batch, the
+    # 0.4B-scale layer, more state CTAs than SMs)
+    assert lib.kla_chunk_fwd_workspace_size(2, 1000, 4, 128, 128, 0) == _ut_bytes(2, 1000, 4)
     assert lib.kla_chunk_fwd_workspace_size(8, 4096, 8, 128, 128, 0) == _ut_bytes(8, 4096, 8)
-    # more state CTAs than leave room for UT CTAs beside them: two launches
     assert lib.kla_chunk_fwd_workspace_size(16, 4096, 8, 128, 128, 0) == _ut_bytes(16, 4096, 8)
-    # which shapes take the single launch (the full workspace; a workspace of
-    # the factors alone always runs two launches)
+    # the single launch is not taken for any shape: its factors are always
+    # formed by a launch of their own
     full = lambda *a: lib.kla_chunk_fwd_workspace_size(*a, 128, 128, 0)
-    assert lib.kla_chunk_fwd_single_launch(2, 1000, 4, 128, 128, 0, full(2, 1000, 4)) == 1
-    assert lib.kla_chunk_fwd_single_launch(2, 1000, 4, 128, 128, 0, _ut_bytes(2, 1000, 4)) == 0
-    assert lib.kla_chunk_fwd_single_launch(8, 4096, 8, 128, 128, 0, 1 << 40) == 0
-    assert lib.kla_chunk_fwd_single_launch(16, 4096, 8, 128, 128, 0, 1 << 40) == 0
-    assert lib.kla_chunk_fwd_single_launch(1, 65536, 16, 128, 128, 0, 1 << 40) == 0  # cut
-    assert lib.kla_chunk_fwd_single_launch(2, 777, 8, 64, 64, 0, 1 << 40) == 1
-    assert lib.kla_chunk_fwd_single_launch(2, 777, 8, 64, 64, 1, 1 << 40) == 0  # fp32 I/O
+    for B, T, H, d in ((2, 1000, 4, 128), (8, 4096, 8, 128), (16, 4096, 8, 128),
+                       (1, 65536, 16, 128), (2, 777, 8, 64), (1, 64, 1, 128)):
+        for dt in (0, 1):
+            assert lib.kla_chunk_fwd_single_launch(B, T, H, d, d, dt, 1 << 40) == 0
+    assert lib.kla_chunk_fwd_single_launch(2, 1000, 4, 128, 128, 0, full(2, 1000, 4)) == 0
     # few heads and a long sequence: per-segment states (E, start state,
     # transition) follow the factors, for between 2 and 64 segments
     n = lib.kla_chunk_fwd_workspace_size(1, 65536, 16, 128, 128, 0)
@@ -210,8 +197,7 @@ def test_workspace_query(lib):
     assert lib.kla_chunk_fwd_segments(1, 65536, 16, 128, 128, 1, n) == 0  # fp32 I/O
     assert lib.kla_chunk_fwd_segments(1, 65536, 16, 96, 96, 0, n) == 0
     # short sequences are never cut (segments keep at least 8 chunks)
-    assert lib.kla_chunk_fwd_workspace_size(1, 64 * 15, 1, 64, 64, 0) == (
-        _ut_bytes(1, 960, 1) + _flag_bytes(1, 960, 1))
+    assert lib.kla_chunk_fwd_workspace_size(1, 64 * 15, 1, 64, 64, 0) == _ut_bytes(1, 960, 1)
     assert lib.kla_chunk_fwd_workspace_size(1, 65536, 16, 128, 128, 1) == 0  # fp32: none
 
 

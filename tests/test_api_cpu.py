@@ -58,9 +58,9 @@ def test_host_tensors_are_refused(name):
 
 def test_workspace_queries_need_no_gpu():
     d = dict(B=2, T=300, H=3, dk=128, dv=128)
-    # the factors (16 KiB per chunk) and one ready flag per chunk (4 bytes,
-    # rounded up to 256) for the single-launch prefill
-    assert api.chunk_fwd_workspace_size(**d) == 2 * 3 * 5 * 16384 + 256
+    # the factors (16 KiB per chunk); the chain is uncut at this length
+    assert api.chunk_fwd_workspace_size(**d) == 2 * 3 * 5 * 16384
+    assert not api.chunk_fwd_single_launch(**d)
     assert api.chunk_bwd_workspace_size(**d) > api.chunk_fwd_workspace_size(**d)
     assert api.recurrent_bwd_workspace_size(**d) > 0
     assert api.kda_chunk_fwd_workspace_size(**d) > 0

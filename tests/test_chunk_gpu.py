@@ -251,30 +251,6 @@ def test_side_stream_matches_current_stream():
     del junk
 
 
-@pytest.mark.parametrize("name,B,T,H", [("prefill_4k", 2, 1000, 4), ("stress", 2, 777, 8),
-                                        ("prefill_4k", 1, 64, 1)])
-def test_single_launch_equals_two_launches(name, B, T, H):
-    """The one-launch prefill (UT lanes and state CTAs in one cooperative
-    kernel, the state CTAs waiting on per-chunk flags) and the two launches
-    (UT kernel, then the state kernel; a workspace holding only the factors)
-    run the same arithmetic: identical outputs, twice in a row on the same
-    workspace (the flags are cleared by every call)."""
-    w = W[name].scaled(B=B, T=T, H=H, seed=73)
-    x = cuda(inputs.make_prefill(w, with_h0=True))
-    assert api.chunk_fwd_single_launch(B, T, H, w.dk, w.dv)
-    ws = torch.empty(api.chunk_fwd_workspace_size(B, T, H, w.dk, w.dv), dtype=torch.uint8,
-                     device="cuda")
-    for _ in range(2):
-        o1, h1 = api.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"],
-                               workspace=ws)
-        o2, h2 = api.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["eta"], x["eps"], x["h0"],
-                               workspace=torch.empty(_ut_bytes(w), dtype=torch.uint8,
-                                                     device="cuda"))
-        api.check_device_error()
-        assert torch.equal(o1, o2) and torch.equal(h1, h2)
-
-
-
 @pytest.mark.parametrize("name,B,T,H,h0", SEGMENTED)
 def test_cut_chain_overlapped_ut_equals_staged(name, B, T, H, h0):
     """The cut chain as kla_chunk_fwd runs it (the UT kernel for the chunks
