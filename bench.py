@@ -225,8 +225,12 @@ def run_ours(args, rank, world, dev):
 
     def step(mid=None):
         # the single launch through chunk_fwd; otherwise the chunk path as
-        # its two kernels (exactly what chunk_fwd launches), with an event
-        # between them when the split is being timed
+        # its two stages, with an event between them when the split is being
+        # timed.  For an uncut chain that is exactly what chunk_fwd launches.
+        # For a cut chain chunk_fwd makes the last segment's factors beside
+        # the first chain pass instead of before it, so this step (factors of
+        # every chunk, then the cut chain) is the staged form; the 65K entry
+        # of "other_workloads" times chunk_fwd itself
         if single:
             fn(xd["q"], xd["k"], xd["v"], xd["g"], xd["eta"], x["eps"], xd["h0"], o=o, hT=hT)
         elif chunk:
