@@ -192,6 +192,11 @@ def test_workspace_query(lib):
     extra = n - _ut_bytes(1, 65536, 16)
     assert extra > 0 and extra % per_seg == 0 and 2 <= extra // per_seg <= 64
     assert lib.kla_chunk_fwd_segments(1, 65536, 16, 128, 128, 0, n) == extra // per_seg
+    # the cost model's choices at the benchmark shapes: three segments at 65K
+    # (on a B200 the fastest of 1..16 segments: 1.29 ms against 1.84 ms for
+    # two and 1.50 ms for four), the 4K layer and the stress shape uncut
+    assert extra // per_seg == 3
+    assert lib.kla_chunk_fwd_segments(4, 8192, 32, 64, 64, 0, 1 << 40) == 1
     assert lib.kla_chunk_fwd_segments(1, 65536, 16, 128, 128, 0, n - 16) == 1  # no room: uncut
     assert lib.kla_chunk_fwd_segments(8, 4096, 8, 128, 128, 0, 1 << 40) == 1
     assert lib.kla_chunk_fwd_segments(1, 65536, 16, 128, 128, 1, n) == 0  # fp32 I/O
