@@ -13,7 +13,8 @@ completion.  It fails on:
   * reuse hazards of TMEM accumulators and shared-memory slots: a buffer
     overwritten before its previous reader of the same data has finished.
 
-The sequences below must be kept identical to the kernel's program order.
+The sequences below must be kept identical to the kernel's program order,
+in both of its modes: the scalar gate and the per-channel gate (KDA).
 """
 import random
 
@@ -36,7 +37,7 @@ class Hazard(AssertionError):
     pass
 
 
-def build(N):
+def build(N, kda=False):
     bars = {}
 
     def B(name, count):
@@ -65,6 +66,8 @@ def build(N):
         prod.append(("tma", n))
     roles["producer"] = prod
 
+    if kda:
+        return bars, build_kda_roles(N, W, A, I, Cm, Do, prod)
     m = [W(("full", 0), 0), I("mma2", 0), Cm("bW"), I("mma3", 0),
          W("w_done", 0), I("mma1", 0), Cm("bS")]
     for n in range(N):
@@ -111,9 +114,53 @@ def build(N):
     return bars, roles
 
 
-def run(N, seed):
+def build_kda_roles(N, W, A, I, Cm, Do, prod):
+    """The per-channel-gate mode: the stage brings W, P, Q o e^G, the decayed
+    keys and the per-channel chunk decay, so there are no Q K^T or W
+    products and no P or W epilogues; warp 2 copies the decay of chunk n from
+    the stage into slot n % 3 of a ring (g_ready); V' is written once (no
+    decayed copy) and feeds both MMA 5 and MMA 6; the state update reads the
+    decay from the ring."""
+    roles = {"producer": prod}
+    m = [W(("full", 0), 0), I("mma3", 0)]
+    for n in range(N):
+        more = n + 1 < N
+        m += [W("h_done", n), I("mma4", n), Cm("bX")]
+        if more:
+            m.append(W(("full", (n + 1) & 1), (n + 1) >> 1))
+        m += [W("vpd_ready", n), I("mma5", n), Cm("bH"), W("vp_ready", n)]
+        if n > 0:
+            m.append(W("pv_free", n - 1))
+        m += [I("mma6", n), Cm("bHP"), Cm(("empty", n & 1))]
+        if more:
+            if n >= 1:
+                m.append(W(("u_free", (n + 1) & 1), (n - 1) >> 1))
+            m.append(I("mma3", n + 1))
+    roles["mma"] = m
+    seq = []
+    for n in range(N):
+        seq += [W(("full", n & 1), n >> 1), Do("D", n), A(("g_ready", n % 3))]
+    roles["p2"] = seq
+    for w in range(6, 14):
+        v_rows = (w & 3) < 2
+        seq = [A("h_done")]
+        for n in range(N):
+            seq.append(W(("g_ready", n % 3), n // 3))
+            if v_rows:
+                seq += [W("bX", n), Do("Vp", n), A("vpd_ready"), A(("u_free", n & 1)),
+                        A("vp_ready")]
+            seq += [W("bH", n), Do("h", n), A("h_done")]
+            if not v_rows:
+                seq += [W("bHP", n), Do("o", n), A(("u_free", n & 1)), A("pv_free")]
+        roles[f"c{w}"] = seq
+    return roles
+
+
+def run(N, seed, kda=False, mutate=None):
     rng = random.Random(seed)
-    bars, roles = build(N)
+    bars, roles = build(N, kda)
+    if mutate is not None:
+        mutate(roles)
     # per-run speeds: some roles (and the pipe / TMA) run far ahead of others,
     # which is where ordering bugs show up
     speed = {r: rng.choice([0.05, 1.0, 20.0]) for r in list(roles) + ["pipe", "tma"]}
@@ -126,11 +173,50 @@ def run(N, seed):
     G_written = {}       # slot -> chunk
     G_readers = {}       # chunk -> readers done
     tma_done = {}
+    D_written = {}       # per-channel mode: decay ring slot -> chunk
+    D_readers = {}       # chunk -> state-update warps that read its decay
 
     def finished(tag, n, count):
         return did.get((tag, n), 0) >= count
 
+    def check_issue_kda(tag, n):
+        if tag in ("mma3", "mma4", "mma5", "mma6") and not tma_done.get(n):
+            raise Hazard(f"{tag} of {n} before the stage of chunk {n} landed")
+        if tag == "mma3" and n >= 2 and not (finished("Vp", n - 2, 4) and finished("o", n - 2, 4)):
+            raise Hazard(f"D_U[{n % 2}] overwritten by chunk {n} while chunk {n - 2} uses it")
+        if tag == "mma4" and n >= 1 and not finished("h", n - 1, 8):
+            raise Hazard(f"MMA 4 of {n} before h_{n} is written")
+        if tag == "mma5":
+            if not finished("Vp", n, 4):
+                raise Hazard(f"MMA 5 of {n} before V'({n})")
+            if n >= 1 and not finished("h", n - 1, 8):
+                raise Hazard(f"D_H of {n} overwritten before chunk {n - 1} read it")
+        if tag == "mma6":
+            if not finished("Vp", n, 4):
+                raise Hazard(f"MMA 6 of {n} before V'({n})")
+            if n >= 1 and not finished("o", n - 1, 4):
+                raise Hazard(f"D_PV of {n} overwritten before chunk {n - 1} read it")
+
+    def check_do_kda(tag, n):
+        if tag == "Vp" and n >= 1 and not {("mma5", n - 1), ("mma6", n - 1)} <= done_mma:
+            raise Hazard(f"V'({n}) overwrites vp while MMA 5 / 6 of {n - 1} may read it")
+        if tag == "h":
+            if not {("mma4", n), ("mma5", n)} <= done_mma:
+                raise Hazard(f"h_{n + 1} written while MMA 4 / 5 of {n} may read h_{n}")
+            if D_written.get(n % 3) != n:
+                raise Hazard(f"decay of chunk {n} read from slot {n % 3} before it was written")
+            D_readers[n] = D_readers.get(n, 0) + 1
+        if tag == "D":
+            if not tma_done.get(n):
+                raise Hazard(f"decay of chunk {n} copied before its stage landed")
+            old = D_written.get(n % 3)
+            if old is not None and D_readers.get(old, 0) < 8:
+                raise Hazard(f"decay of {n} overwrites slot {n % 3} still read for chunk {old}")
+            D_written[n % 3] = n
+
     def check_issue(tag, n):
+        if kda:
+            return check_issue_kda(tag, n)
         # TMEM / smem reuse before the previous user is done
         if tag == "mma1":
             if n >= 1 and not finished("P", n - 1, 4):
@@ -158,6 +244,8 @@ def run(N, seed):
                 raise Hazard(f"D_PV of {n} overwritten before chunk {n - 1} read it")
 
     def check_do(tag, n):
+        if kda:
+            return check_do_kda(tag, n)
         if tag == "Vpd" and n >= 1 and ("mma5", n - 1) not in done_mma:
             raise Hazard(f"V'({n}) overwrites vpd while MMA 5 of {n - 1} may read it")
         if tag == "Vp" and n >= 1 and ("mma6", n - 1) not in done_mma:
@@ -233,6 +321,8 @@ def run(N, seed):
             n = st[1]
             if n >= 2 and not {("mma5", n - 2), ("mma6", n - 2)} <= done_mma:
                 raise Hazard(f"stage of chunk {n} reloaded while chunk {n - 2} uses it")
+            if kda and n >= 2 and not finished("D", n - 2, 1):
+                raise Hazard(f"stage of chunk {n} reloaded before the decay of {n - 2} was copied")
             tma_done.pop(n - 2, None)
             tma.append(n)
         elif st[0] == "do":
@@ -247,6 +337,28 @@ def run(N, seed):
 def test_chain_protocol_random_interleavings(N):
     for seed in range(300):
         run(N, seed)
+
+
+@pytest.mark.parametrize("N", [1, 2, 3, 4, 7, 12])
+def test_chain_protocol_per_channel_mode(N):
+    """The per-channel-gate mode's own issue order and roles: no deadlock,
+    no skipped phase, no stage, decay-ring, V' or accumulator reuse hazard."""
+    for seed in range(300):
+        run(N, seed, kda=True)
+
+
+def test_model_catches_a_decay_published_before_it_is_copied():
+    """Planted in the model, not the kernel: warp 2 raising the ring's ready
+    barrier before copying the chunk's decay must be reported."""
+    def swap(roles):
+        seq = roles["p2"]
+        for i in range(len(seq) - 1):
+            if seq[i][0] == "do" and seq[i][1] == "D":
+                seq[i], seq[i + 1] = seq[i + 1], seq[i]
+
+    with pytest.raises(AssertionError, match="decay"):
+        for seed in range(300):
+            run(3, seed, kda=True, mutate=swap)
 
 
 def test_model_catches_a_skipped_phase():
