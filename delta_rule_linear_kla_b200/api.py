@@ -89,7 +89,8 @@ def chunk_fwd_single_launch(B: int, T: int, H: int, dk: int, dv: int,
                             ws_bytes: Optional[int] = None) -> bool:
     """Whether the bf16 prefill of this shape runs as one kernel launch
     (kla_chunk_fwd_single_launch); ws_bytes defaults to the full workspace
-    size."""
+    size.  False for every shape at present: the single launch is built but
+    not taken."""
     if ws_bytes is None:
         ws_bytes = chunk_fwd_workspace_size(B, T, H, dk, dv, dtype)
     return bool(_native.lib().kla_chunk_fwd_single_launch(B, T, H, dk, dv, _DT[dtype],

@@ -778,7 +778,8 @@ constexpr size_t fused_smem_bytes() {
 // factors in chunk order n = 0, 1, ... over all heads and raise one flag per
 // chunk, which the state CTAs wait for before they fetch that chunk's
 // factors.  The launch is cooperative (all CTAs resident at once, one per
-// SM), so those waits always end; they are bounded all the same.
+// SM), so those waits always end; they are bounded all the same.  Not taken
+// at present (see fused_shape): every shape runs the two kernels in turn.
 template <int DK>
 __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
